@@ -1,0 +1,515 @@
+/*
+ * STEPQuant CPU oracle -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Only tests/, __graft_entry__.smoke() and the cpu_baseline leg of bench.py
+ * may load this file's library.  The product path (libstepq.so) shares no
+ * code with it: both sides implement the arithmetic and the packed format
+ * from the written definition, each on its own.
+ *
+ * Source: "STEPQuant: When and Where Errors Matter in Delta-Rule Recurrent
+ * State Quantization" (paper digest page, vibe-research), sections
+ * "背景与动机" (the state S_t in R^{dk x dv}, update with key/value/gate,
+ * readout with the query; error recursion E_t = A_t E_{t-1} + eps_t),
+ * "方法-3 Key-Row-Aware Dual-Axis Fitting" (X_hat = r_i c_j z_ij) and
+ * "方法-4 每个 decode step 的执行路径" (reconstruct -> retention + delta +
+ * readout -> refit r, c -> pack).  The update formula, the quantizer formulas
+ * and the numeric precision are not printed on the pages; the readings used
+ * here are stated beside each function and listed in the design doc.
+ *
+ * Build: gcc -O2 -ffp-contract=off -fno-fast-math -shared -fPIC
+ * (no contraction: every fp32 operation below rounds exactly where written).
+ *
+ * Parity status of each function is stated in its comment.  Functions not
+ * marked otherwise are pinned by tests/test_oracle_*.py.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define SQ_PIVOT_BITS 16
+
+/* ------------------------------------------------------------------------ */
+/* IEEE 754 binary16 <-> binary32, written from the format definition       */
+/* (1 sign bit, 5 exponent bits with bias 15, 10 fraction bits).             */
+/* Pivot units are stored in FP16 ("方法-1": FP16 pivots).                    */
+/* ------------------------------------------------------------------------ */
+
+float sq_f16_to_f32(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int f = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);                 /* subnormal: f * 2^-24 */
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + f), e - 25);     /* (1 + f/1024) * 2^(e-15) */
+    return (float)(sign ? -v : v);
+}
+
+/* Round-to-nearest-even conversion; overflow goes to +-inf. */
+uint16_t sq_f32_to_f16(float x)
+{
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs((double)x);
+    if (isnan(x)) return 0x7e00;
+    if (a == 0.0) return sign;
+    /* quantum of the binade that holds a (subnormal range uses 2^-24) */
+    int ex;
+    frexp(a, &ex);                 /* a = m * 2^ex, m in [0.5, 1) */
+    int e = ex - 1;                /* a in [2^e, 2^(e+1)) */
+    if (e < -14) e = -14;          /* subnormal quantum */
+    double q = ldexp(1.0, e - 10);
+    double n = a / q;              /* exact: power-of-two scaling */
+    double fl = floor(n);
+    double rem = n - fl;
+    if (rem > 0.5 || (rem == 0.5 && fmod(fl, 2.0) != 0.0)) fl += 1.0;
+    double r = fl * q;
+    if (r >= 65520.0 || r > 65504.0) return sign | 0x7c00;
+    /* encode r */
+    if (r < ldexp(1.0, -14)) {
+        int f = (int)(r / ldexp(1.0, -24));
+        return sign | (uint16_t)f;
+    }
+    frexp(r, &ex);
+    e = ex - 1;
+    int f = (int)(r / ldexp(1.0, e - 10)) - 1024;
+    return sign | (uint16_t)(((e + 15) << 10) | f);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Packed format (our own; the pages fix only that the layout is decided     */
+/* offline, "方法-4": 离线分配固定 packed layout).                             */
+/*                                                                          */
+/* Codes are offset-binary: the stored field of a b-bit code z is          */
+/* u = z + 2^(b-1), in [1, 2^b - 1] for |z| <= qmax = 2^(b-1) - 1.            */
+/*                                                                          */
+/* Uniform-width unit (a head whose rows all share width b):                */
+/*   RT = D/8 rows per band, NT = 2D threads.  Element (i,j) belongs to     */
+/*   thread t = (i/RT)*(D/4) + j/4 at stream position p = (i%RT)*4 + j%4.    */
+/*   Its field occupies stream bits [p*b, p*b+b) (LSB-first bytes).  Stream  */
+/*   byte B of thread t lives at block byte ((B/RT)*NT + t)*RT + B%RT.        */
+/* Row-major unit (rows of mixed width): row i starts at the sum of the     */
+/*   byte sizes D*b/8 of the rows before it; code j occupies row bits         */
+/*   [b*j, b*j+b).  A 16-bit row holds binary16 values, 2 bytes per column.  */
+/* ------------------------------------------------------------------------ */
+
+static int get_bit(const uint8_t *blk, long bit) { return (blk[bit >> 3] >> (bit & 7)) & 1; }
+static void set_bit(uint8_t *blk, long bit, int v)
+{
+    if (v) blk[bit >> 3] |= (uint8_t)(1u << (bit & 7));
+    else   blk[bit >> 3] &= (uint8_t)~(1u << (bit & 7));
+}
+
+/* Block bit address of stream bit s of thread t (uniform layout). */
+static long uniform_bit_addr(int D, int t, long s)
+{
+    int RT = D / 8, NT = 2 * D;
+    long B = s >> 3;
+    long byte = ((B / RT) * NT + t) * RT + (B % RT);
+    return byte * 8 + (s & 7);
+}
+
+long sq_codes_bytes_uniform(int D, int b) { return (long)D * D * b / 8; }
+
+void sq_pack_uniform(int D, int b, const int32_t *z, uint8_t *blk)
+{
+    int RT = D / 8;
+    memset(blk, 0, (size_t)sq_codes_bytes_uniform(D, b));
+    for (int i = 0; i < D; i++)
+        for (int j = 0; j < D; j++) {
+            int t = (i / RT) * (D / 4) + j / 4;
+            int p = (i % RT) * 4 + j % 4;
+            unsigned u = (unsigned)(z[i * D + j] + (1 << (b - 1)));
+            for (int k = 0; k < b; k++)
+                set_bit(blk, uniform_bit_addr(D, t, (long)p * b + k), (u >> k) & 1);
+        }
+}
+
+void sq_unpack_uniform(int D, int b, const uint8_t *blk, int32_t *z)
+{
+    int RT = D / 8;
+    for (int i = 0; i < D; i++)
+        for (int j = 0; j < D; j++) {
+            int t = (i / RT) * (D / 4) + j / 4;
+            int p = (i % RT) * 4 + j % 4;
+            unsigned u = 0;
+            for (int k = 0; k < b; k++)
+                u |= (unsigned)get_bit(blk, uniform_bit_addr(D, t, (long)p * b + k)) << k;
+            z[i * D + j] = (int32_t)u - (1 << (b - 1));
+        }
+}
+
+long sq_row_bytes(int D, int b) { return (long)D * b / 8; }
+
+long sq_codes_bytes_rows(int D, const int *widths)
+{
+    long n = 0;
+    for (int i = 0; i < D; i++) n += sq_row_bytes(D, widths[i]);
+    return n;
+}
+
+/* Row-major pack.  z holds codes for quantized rows; h holds binary16
+ * patterns for 16-bit rows (entries of other rows are ignored). */
+void sq_pack_rows(int D, const int *widths, const int32_t *z, const uint16_t *h, uint8_t *blk)
+{
+    long off = 0;
+    memset(blk, 0, (size_t)sq_codes_bytes_rows(D, widths));
+    for (int i = 0; i < D; i++) {
+        int b = widths[i];
+        uint8_t *row = blk + off;
+        for (int j = 0; j < D; j++) {
+            if (b == SQ_PIVOT_BITS) {
+                row[2 * j] = (uint8_t)(h[i * D + j] & 0xff);
+                row[2 * j + 1] = (uint8_t)(h[i * D + j] >> 8);
+            } else {
+                unsigned u = (unsigned)(z[i * D + j] + (1 << (b - 1)));
+                for (int k = 0; k < b; k++) set_bit(row, (long)b * j + k, (u >> k) & 1);
+            }
+        }
+        off += sq_row_bytes(D, b);
+    }
+}
+
+void sq_unpack_rows(int D, const int *widths, const uint8_t *blk, int32_t *z, uint16_t *h)
+{
+    long off = 0;
+    for (int i = 0; i < D; i++) {
+        int b = widths[i];
+        const uint8_t *row = blk + off;
+        for (int j = 0; j < D; j++) {
+            if (b == SQ_PIVOT_BITS) {
+                h[i * D + j] = (uint16_t)(row[2 * j] | (row[2 * j + 1] << 8));
+                z[i * D + j] = 0;
+            } else {
+                unsigned u = 0;
+                for (int k = 0; k < b; k++) u |= (unsigned)get_bit(row, (long)b * j + k) << k;
+                z[i * D + j] = (int32_t)u - (1 << (b - 1));
+                h[i * D + j] = 0;
+            }
+        }
+        off += sq_row_bytes(D, b);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Reductions.                                                               */
+/* ------------------------------------------------------------------------ */
+
+/* fp32 pairwise sum of n = 2^m terms: sum(x[0:n]) = sum(x[0:n/2]) +
+ * sum(x[n/2:n]), each addition rounded to fp32.  This is the summation order
+ * the quantizer's row and column sums are defined with. */
+float sq_pairwise_sum(const float *x, int n)
+{
+    if (n == 1) return x[0];
+    float a = sq_pairwise_sum(x, n / 2);
+    float b = sq_pairwise_sum(x + n / 2, n / 2);
+    return a + b;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Quantizer (section 方法-3): X_hat_ij = r_i * c_j * z_ij.                   */
+/*   rho_i   = (omega_i / mean omega)^(-1/4)          (from the plan)         */
+/*   r_i     = max(mean_j |S_ij|, 1e-12) * rho_i                              */
+/*   c0_j    = max_i |S_ij / r_i| / qmax_i                                    */
+/*   z0      = rhe(S / (r c0))                                                */
+/*   c_j     = sum_i w_i r_i z0_ij S_ij / sum_i w_i r_i^2 z0_ij^2  (w = omega) */
+/*   z       = clamp(rhe(S / (r c)), -qmax, qmax)                             */
+/* Readings (the pages print none of these formulas):                        */
+/*   - the row mean is the fp32 pairwise sum of |S_ij| over j, times 1/D;     */
+/*   - S/(r c) is taken as y = fl(S * fl(1/r)) and then the exact product    */
+/*     y * fl(1/c) is rounded to the nearest integer, ties to even;          */
+/*   - c0_j = max_i fl(|y_ij| / qmax_i); an all-zero column gets c0 = 1;      */
+/*   - the refinement sums are fp32 pairwise sums over i of                   */
+/*     fl(b_i * fl(z0*y)) and fl(b_i * fl(z0*z0)), b_i = fl(wbar_i*fl(r_i r_i)),*/
+/*     which equal w r z0 S and w r^2 z0^2 up to the common factor 1/r;       */
+/*     rows of 16-bit (pivot) width contribute 0; a zero denominator keeps c0; */
+/*   - c_j is rounded to fp32 before the final codes are taken.               */
+/* 16-bit rows are stored as binary16 (RNE) and carry no row factor (r = 0).  */
+/* tie_out (optional, D*D): bit0 = final code within 1e-6 relative of a .5   */
+/* boundary; bit1 = its column had such a tie in z0 (column tie-affected).   */
+/* z0_out (optional, D*D): the initial codes z0 (exposed for the LS pin).     */
+/* ------------------------------------------------------------------------ */
+
+static int qmax_of(int b) { return (1 << (b - 1)) - 1; }
+
+static int near_half(double x)
+{
+    double ax = fabs(x);
+    double f = floor(ax);
+    return fabs(ax - (f + 0.5)) <= 1e-6 * ax;
+}
+
+void sq_quantize(int D, const int *widths, const float *rho, const float *wbar,
+                 const float *S, int32_t *z, uint16_t *h, float *r, float *c,
+                 uint8_t *tie_out, int32_t *z0_out)
+{
+    float *absrow = (float *)malloc(sizeof(float) * D);
+    float *y = (float *)malloc(sizeof(float) * D * D);
+    float *bw = (float *)malloc(sizeof(float) * D);
+    float *tn = (float *)malloc(sizeof(float) * D);
+    float *td = (float *)malloc(sizeof(float) * D);
+    int32_t *z0 = (int32_t *)malloc(sizeof(int32_t) * D * D);
+    uint8_t *coltie = (uint8_t *)calloc(D, 1);
+
+    /* row factors */
+    for (int i = 0; i < D; i++) {
+        if (widths[i] == SQ_PIVOT_BITS) {
+            r[i] = 0.0f;
+            bw[i] = 0.0f;
+            for (int j = 0; j < D; j++) {
+                h[i * D + j] = sq_f32_to_f16(S[i * D + j]);
+                z[i * D + j] = 0;
+                y[i * D + j] = 0.0f;
+            }
+            continue;
+        }
+        for (int j = 0; j < D; j++) absrow[j] = fabsf(S[i * D + j]);
+        float m = sq_pairwise_sum(absrow, D) * (1.0f / (float)D);
+        if (!(m > 1e-12f)) m = 1e-12f;
+        r[i] = m * rho[i];
+        float inv_r = 1.0f / r[i];
+        for (int j = 0; j < D; j++) {
+            y[i * D + j] = S[i * D + j] * inv_r;
+            h[i * D + j] = 0;
+        }
+        float rr = r[i] * r[i];
+        bw[i] = wbar[i] * rr;
+    }
+
+    for (int j = 0; j < D; j++) {
+        /* initial column factor */
+        float c0 = 0.0f;
+        for (int i = 0; i < D; i++) {
+            if (widths[i] == SQ_PIVOT_BITS) continue;
+            float v = fabsf(y[i * D + j]) / (float)qmax_of(widths[i]);
+            if (v > c0) c0 = v;
+        }
+        if (c0 == 0.0f) c0 = 1.0f;
+        float inv_c0 = 1.0f / c0;
+        /* initial codes and weighted least-squares refinement */
+        for (int i = 0; i < D; i++) {
+            if (widths[i] == SQ_PIVOT_BITS) { tn[i] = 0.0f; td[i] = 0.0f; continue; }
+            double x0 = (double)y[i * D + j] * (double)inv_c0;
+            z0[i * D + j] = (int32_t)rint(x0);
+            if (near_half(x0)) coltie[j] = 1;
+            float zf = (float)z0[i * D + j];
+            float pn = zf * y[i * D + j];
+            float pd = zf * zf;
+            tn[i] = bw[i] * pn;
+            td[i] = bw[i] * pd;
+        }
+        float num = sq_pairwise_sum(tn, D);
+        float den = sq_pairwise_sum(td, D);
+        float cj = (den > 0.0f) ? num / den : c0;
+        c[j] = cj;
+        float inv_c = 1.0f / cj;
+        for (int i = 0; i < D; i++) {
+            if (widths[i] == SQ_PIVOT_BITS) continue;
+            int q = qmax_of(widths[i]);
+            double x = (double)y[i * D + j] * (double)inv_c;
+            double zr = rint(x);
+            if (zr > q) zr = q;
+            if (zr < -q) zr = -q;
+            z[i * D + j] = (int32_t)zr;
+            if (tie_out)
+                tie_out[i * D + j] = (uint8_t)((near_half(x) ? 1 : 0) | (coltie[j] ? 2 : 0));
+        }
+    }
+    if (tie_out)
+        for (int i = 0; i < D; i++)
+            if (widths[i] == SQ_PIVOT_BITS)
+                for (int j = 0; j < D; j++) tie_out[i * D + j] = 0;
+    if (z0_out)
+        for (int i = 0; i < D; i++)
+            for (int j = 0; j < D; j++)
+                z0_out[i * D + j] = (widths[i] == SQ_PIVOT_BITS) ? 0 : z0[i * D + j];
+
+    free(absrow); free(y); free(bw); free(tn); free(td); free(z0); free(coltie);
+}
+
+/* Reconstruction X_hat_ij = fl(fl(r_i * c_j) * z_ij); 16-bit rows decode the
+ * stored binary16 value. */
+void sq_reconstruct(int D, const int *widths, const int32_t *z, const uint16_t *h,
+                    const float *r, const float *c, float *S_hat)
+{
+    for (int i = 0; i < D; i++)
+        for (int j = 0; j < D; j++) {
+            if (widths[i] == SQ_PIVOT_BITS)
+                S_hat[i * D + j] = sq_f16_to_f32(h[i * D + j]);
+            else {
+                float rc = r[i] * c[j];
+                S_hat[i * D + j] = rc * (float)z[i * D + j];
+            }
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* One decode step of a packed head (sections 背景与动机 and 方法-4).           */
+/*                                                                          */
+/* Recurrence (gated delta rule; KDA reading with Diag(alpha) applied first): */
+/*   S_t = (I - beta k k^T) Diag(alpha) S_{t-1} + beta k v^T,  o_t = S_t^T q  */
+/* Readings:                                                                 */
+/*   - retention is folded into the row factor: a_i = fl(alpha_i r_i) and      */
+/*     S'_ij = fl(fl(a_i c_j) z_ij); 16-bit rows: S'_ij = fl(alpha_i h_ij);   */
+/*   - u_j = sum_i k_i R_ij with R_ij = a_i c_j z_ij (or alpha_i h_ij) the    */
+/*     exact retained reconstruction, evaluated in fp64 and rounded once;     */
+/*   - w_j = fl(beta * fl(v_j - u_j));  S_ij = fma(k_i, w_j, S'_ij);           */
+/*   - o_j = sum_i q_i (R_ij + k_i w_j) in fp64, rounded once: the readout of */
+/*     the updated state, taken before requantization.                        */
+/* alpha has D entries (GDN: all equal).  S_out receives the fp32 S_t that    */
+/* the requantizer consumes.                                                 */
+/* ------------------------------------------------------------------------ */
+
+void sq_step_from_codes(int D, const int *widths, const int32_t *z, const uint16_t *h,
+                        const float *r, const float *c,
+                        const float *q, const float *k, const float *v,
+                        const float *alpha, float beta,
+                        float *S_out, float *o_out, float *u_out, float *w_out)
+{
+    double *R = (double *)malloc(sizeof(double) * D * D);
+    float *w = (float *)malloc(sizeof(float) * D);
+    for (int i = 0; i < D; i++) {
+        if (widths[i] == SQ_PIVOT_BITS) {
+            for (int j = 0; j < D; j++) {
+                float hv = sq_f16_to_f32(h[i * D + j]);
+                S_out[i * D + j] = alpha[i] * hv;
+                R[i * D + j] = (double)alpha[i] * (double)hv;
+            }
+        } else {
+            float a = alpha[i] * r[i];
+            for (int j = 0; j < D; j++) {
+                float A = a * c[j];
+                S_out[i * D + j] = A * (float)z[i * D + j];
+                R[i * D + j] = (double)a * (double)c[j] * (double)z[i * D + j];
+            }
+        }
+    }
+    for (int j = 0; j < D; j++) {
+        double acc = 0.0;
+        for (int i = 0; i < D; i++) acc += (double)k[i] * R[i * D + j];
+        float u = (float)acc;
+        float d = v[j] - u;
+        w[j] = beta * d;
+        if (u_out) u_out[j] = u;
+        if (w_out) w_out[j] = w[j];
+    }
+    for (int j = 0; j < D; j++) {
+        double acc = 0.0;
+        for (int i = 0; i < D; i++)
+            acc += (double)q[i] * (R[i * D + j] + (double)k[i] * (double)w[j]);
+        o_out[j] = (float)acc;
+    }
+    for (int i = 0; i < D; i++)
+        for (int j = 0; j < D; j++)
+            S_out[i * D + j] = fmaf(k[i], w[j], S_out[i * D + j]);
+    free(R);
+    free(w);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Plain FP32-state recurrence (the unquantized reference the pages compare  */
+/* against, "FP32-state").  Same update; u and o summed in fp64, rounded once.*/
+/* ------------------------------------------------------------------------ */
+
+void sq_step_fp32(int D, float *S, const float *q, const float *k, const float *v,
+                  const float *alpha, float beta, float *o_out)
+{
+    float *w = (float *)malloc(sizeof(float) * D);
+    for (int i = 0; i < D; i++)
+        for (int j = 0; j < D; j++) S[i * D + j] = alpha[i] * S[i * D + j];
+    for (int j = 0; j < D; j++) {
+        double acc = 0.0;
+        for (int i = 0; i < D; i++) acc += (double)k[i] * (double)S[i * D + j];
+        float u = (float)acc;
+        float d = v[j] - u;
+        w[j] = beta * d;
+    }
+    for (int i = 0; i < D; i++)
+        for (int j = 0; j < D; j++) S[i * D + j] = fmaf(k[i], w[j], S[i * D + j]);
+    for (int j = 0; j < D; j++) {
+        double acc = 0.0;
+        for (int i = 0; i < D; i++) acc += (double)q[i] * (double)S[i * D + j];
+        o_out[j] = (float)acc;
+    }
+    free(w);
+}
+
+/* The same recurrence in fp64 (used for the invariants and the drift study). */
+void sq_step_fp64(int D, double *S, const double *q, const double *k, const double *v,
+                  const double *alpha, double beta, double *o_out)
+{
+    double *w = (double *)malloc(sizeof(double) * D);
+    for (int i = 0; i < D; i++)
+        for (int j = 0; j < D; j++) S[i * D + j] = alpha[i] * S[i * D + j];
+    for (int j = 0; j < D; j++) {
+        double u = 0.0;
+        for (int i = 0; i < D; i++) u += k[i] * S[i * D + j];
+        w[j] = beta * (v[j] - u);
+    }
+    for (int i = 0; i < D; i++)
+        for (int j = 0; j < D; j++) S[i * D + j] = S[i * D + j] + k[i] * w[j];
+    for (int j = 0; j < D; j++) {
+        double o = 0.0;
+        for (int i = 0; i < D; i++) o += q[i] * S[i * D + j];
+        o_out[j] = o;
+    }
+    free(w);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Calibration statistics (sections 方法-1 and 方法-2).                        */
+/*   g_t = A_t^T q_t with A_t = (I - beta k k^T) Diag(alpha):                 */
+/*   g = alpha (.) (q - beta k (k^T q)); omega_i accumulates g_i^2.           */
+/*   lsum accumulates log(alpha_i) (mean log retention gate).                 */
+/* ------------------------------------------------------------------------ */
+
+void sq_calib_accumulate(int D, const float *q, const float *k, const float *alpha,
+                         float beta, double *omega_acc, double *lsum_acc)
+{
+    double kq = 0.0;
+    for (int i = 0; i < D; i++) kq += (double)k[i] * (double)q[i];
+    for (int i = 0; i < D; i++) {
+        double g = (double)alpha[i] * ((double)q[i] - (double)beta * (double)k[i] * kq);
+        omega_acc[i] += g * g;
+        lsum_acc[i] += log((double)alpha[i]);
+    }
+}
+
+/* Squared Frobenius reconstruction error of each row when the whole head is
+ * quantized at uniform width b (distortion d_u(b), section 方法-1).  rho and
+ * wbar are the plan's row weights.  err_rows receives D values. */
+void sq_distortion_rows(int D, int b, const float *rho, const float *wbar,
+                        const float *S, double *err_rows)
+{
+    int *widths = (int *)malloc(sizeof(int) * D);
+    int32_t *z = (int32_t *)malloc(sizeof(int32_t) * D * D);
+    uint16_t *h = (uint16_t *)malloc(sizeof(uint16_t) * D * D);
+    float *r = (float *)malloc(sizeof(float) * D);
+    float *c = (float *)malloc(sizeof(float) * D);
+    float *Sh = (float *)malloc(sizeof(float) * D * D);
+    for (int i = 0; i < D; i++) widths[i] = b;
+    sq_quantize(D, widths, rho, wbar, S, z, h, r, c, NULL, NULL);
+    sq_reconstruct(D, widths, z, h, r, c, Sh);
+    for (int i = 0; i < D; i++) {
+        double e = 0.0;
+        for (int j = 0; j < D; j++) {
+            double d = (double)Sh[i * D + j] - (double)S[i * D + j];
+            e += d * d;
+        }
+        err_rows[i] = e;
+    }
+    free(widths); free(z); free(h); free(r); free(c); free(Sh);
+}
+
+/* Lifetime weight L_u = sum_{j=0}^{H-1} exp(2 j l_u) (section 方法-1),
+ * summed term by term. */
+double sq_lifetime_weight(double l, long H)
+{
+    double s = 0.0;
+    for (long j = 0; j < H; j++) s += exp(2.0 * (double)j * l);
+    return s;
+}

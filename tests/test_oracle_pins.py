@@ -1,0 +1,486 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a closed
+form, an invariant of the recurrence, a library routine for a special case,
+brute-force enumeration, or a hand-derived byte image.  Sources: STEPQuant
+paper digest page, sections 背景与动机 (update / readout / error recursion),
+方法-1 (lifetime weight, allocation, pivots, bit/value), 方法-3 (dual-axis fit).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import allocator, core, model, plan_io
+from quantized_recurrent_state_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(12345)
+
+
+# --------------------------------------------------------------------------
+# binary16 conversion == numpy's IEEE half conversion (a library routine)
+# --------------------------------------------------------------------------
+
+def test_f16_matches_numpy():
+    xs = np.concatenate([
+        rng.standard_normal(4000).astype(np.float32) * 10.0 ** rng.integers(-9, 6, 4000),
+        np.array([0.0, -0.0, 65504.0, 65519.99, 65520.0, 1e-8, 5.96e-8, 2.98e-8, 2.99e-8,
+                  6.1e-5, 1.0 + 2 ** -11, 1.0 + 3 * 2 ** -11, -2.5e-7, 1e6], dtype=np.float32),
+    ])
+    for x in xs:
+        with np.errstate(over="ignore"):
+            ref = int(np.array([x], np.float32).astype(np.float16).view(np.uint16)[0])
+        assert core.f32_to_f16(x) == ref, x
+        back = core.f16_to_f32(ref)
+        refb = float(np.array([ref], np.uint16).view(np.float16).astype(np.float32)[0])
+        assert back == refb or (math.isnan(back) and math.isnan(refb))
+
+
+# --------------------------------------------------------------------------
+# packed format
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("D", [16, 128])
+@pytest.mark.parametrize("b", [2, 4, 6, 8])
+def test_uniform_pack_roundtrip(D, b):
+    q = (1 << (b - 1)) - 1
+    z = rng.integers(-q, q + 1, size=(D, D)).astype(np.int32)
+    blk = core.pack_uniform(D, b, z)
+    assert blk.size == D * D * b // 8
+    assert np.array_equal(core.unpack_uniform(D, b, blk), z)
+
+
+def test_rows_pack_roundtrip():
+    D = 128
+    widths = rng.choice([4, 6, 8, 16], size=D).astype(np.int32)
+    z = np.zeros((D, D), np.int32)
+    h = np.zeros((D, D), np.uint16)
+    for i, b in enumerate(widths):
+        if b == 16:
+            h[i] = rng.integers(0, 1 << 16, size=D).astype(np.uint16)
+        else:
+            q = (1 << (b - 1)) - 1
+            z[i] = rng.integers(-q, q + 1, size=D)
+    blk = core.pack_rows(D, widths, z, h)
+    assert blk.size == sum(D * int(b) // 8 for b in widths)
+    z2, h2 = core.unpack_rows(D, widths, blk)
+    assert np.array_equal(z2, z) and np.array_equal(h2, h)
+
+
+def _golden_layout():
+    cases = {}
+    with open(os.path.join(GOLDEN, "layout_d16.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            cases.setdefault(parts[0], {})[parts[1]] = parts[2:]
+    return cases
+
+
+def test_uniform_layout_hand_bytes():
+    cases = _golden_layout()
+    # b = 4 case
+    z = np.zeros((16, 16), np.int32)
+    for item in cases["b4"]["set"]:
+        i, j, val = (int(x) for x in item.split(","))
+        z[i, j] = val
+    blk = core.pack_uniform(16, 4, z)
+    exp = np.full(128, 0x88, np.uint8)
+    for item in cases["b4"]["expect"]:
+        if item.startswith("default="):
+            continue
+        k, val = item.split("=")
+        exp[int(k)] = int(val, 16)
+    assert np.array_equal(blk, exp)
+    # b = 6 case, all zero codes
+    blk = core.pack_uniform(16, 6, np.zeros((16, 16), np.int32))
+    exp = np.zeros(192, np.uint8)
+    for item in cases["b6"]["expect"][1:]:
+        rng_s, pat = item.split("=")
+        a, b_ = (int(x) for x in rng_s.split(":"))
+        p = [int(x, 16) for x in pat.split(",")]
+        exp[a:b_] = np.tile(np.array(p, np.uint8), (b_ - a) // 2)
+    assert np.array_equal(blk, exp)
+
+
+def test_rows_layout_lsb_first():
+    # row-major: code j of a b-bit row occupies row bits [b*j, b*j+b)
+    D = 16
+    widths = np.array([4] * 8 + [2] * 8, np.int32)
+    z = np.zeros((D, D), np.int32)
+    z[0, 1] = 7            # u = 15 -> bits 4..7 of byte 0 (low nibble: code 0 = u 8)
+    z[8, 3] = -1           # 2-bit row 8 (offset 8 rows * 8 bytes = 64), u = 1, bits 6..7
+    blk = core.pack_rows(D, widths, z, np.zeros((D, D), np.uint16))
+    assert blk[0] == 0xF8
+    assert blk[64] == (0b10 | 0b10 << 2 | 0b10 << 4 | 0b01 << 6)
+
+
+# --------------------------------------------------------------------------
+# reductions
+# --------------------------------------------------------------------------
+
+def test_pairwise_sum_order_and_accuracy():
+    # tree order: (1 + 0) + (2^-24 + 2^-24) = 1 + 2^-23, sequential would give 1
+    assert core.pairwise_sum(np.array([1, 0, 2 ** -24, 2 ** -24], np.float32)) == np.float32(1 + 2 ** -23)
+    for n in (16, 128):
+        x = np.abs(rng.standard_normal(n)).astype(np.float32)
+        s = float(core.pairwise_sum(x))
+        exact = math.fsum(float(v) for v in x)
+        assert abs(s - exact) <= math.log2(n) * 2.0 ** -24 * exact * 1.0001
+
+
+# --------------------------------------------------------------------------
+# recurrence invariants (背景与动机: S_t updated by key, value, gate; readout S^T q)
+# --------------------------------------------------------------------------
+
+def _rand_inputs(D, kda=False):
+    q = rng.standard_normal(D).astype(np.float32)
+    n = rng.standard_normal(D)
+    k = (n / np.linalg.norm(n)).astype(np.float32)
+    v = rng.standard_normal(D).astype(np.float32)
+    alpha = (rng.uniform(0.5, 1.0, D) if kda else np.full(D, rng.uniform(0.5, 1.0))).astype(np.float32)
+    beta = np.float32(rng.uniform(0, 1))
+    return q, k, v, alpha, beta
+
+
+def test_fixed_point_alpha1_beta0_fp32():
+    D = 128
+    S = rng.standard_normal((D, D)).astype(np.float32)
+    S0 = S.copy()
+    q, k, v, _, _ = _rand_inputs(D)
+    o = core.step_fp32(S, q, k, v, 1.0, 0.0)
+    assert np.array_equal(S, S0)
+    exact = (S0.astype(np.float64).T @ q.astype(np.float64))
+    assert np.allclose(o, exact, rtol=1e-6, atol=1e-6)
+
+
+def test_fixed_point_alpha1_beta0_from_codes():
+    D = 128
+    rw = np.full(D, 6, np.int32)
+    S = rng.standard_normal((D, D)).astype(np.float32)
+    z, h, r, c, _ = core.quantize(D, rw, np.ones(D, np.float32), np.ones(D, np.float32), S)
+    q, k, v, _, _ = _rand_inputs(D)
+    St, o, u, w = core.step_from_codes(D, rw, z, h, r, c, q, k, v, 1.0, 0.0)
+    assert np.array_equal(St, core.reconstruct(D, rw, z, h, r, c))
+    assert np.all(w == 0)
+
+
+@pytest.mark.parametrize("kda", [False, True])
+def test_retrieval_beta1_unit_key_fp64(kda):
+    # beta = 1, ||k|| = 1: the written association is recalled exactly, S_t^T k = v,
+    # for any retention (reading: Diag(alpha) acts before (I - beta k k^T)).
+    D = 128
+    S = rng.standard_normal((D, D))
+    q, k, v, alpha, _ = _rand_inputs(D, kda)
+    k64 = k.astype(np.float64)
+    k64 /= np.linalg.norm(k64)
+    core.step_fp64(S, q, k64, v, alpha, 1.0)
+    assert np.max(np.abs(S.T @ k64 - v)) < 1e-12 * max(1.0, np.abs(v).max())
+
+
+def test_pure_decay_beta0_fp64():
+    D = 64
+    S0 = rng.standard_normal((D, D))
+    S = S0.copy()
+    a = 0.97
+    for t in range(50):
+        q, k, v, _, _ = _rand_inputs(D)
+        core.step_fp64(S, q, k, v, a, 0.0)
+    assert np.allclose(S, a ** 50 * S0, rtol=1e-13, atol=0)
+
+
+def test_fp32_tracks_fp64_over_256_steps():
+    D = 128
+    S32 = (rng.standard_normal((D, D))).astype(np.float32)
+    S64 = S32.astype(np.float64)
+    a = np.float32(0.995)
+    worst = 0.0
+    for t in range(256):
+        q, k, v, _, beta = _rand_inputs(D)
+        o32 = core.step_fp32(S32, q, k, v, a, beta)
+        o64 = core.step_fp64(S64, q, k, v, np.float64(a), np.float64(beta))
+        worst = max(worst, np.max(np.abs(o32 - o64)) / np.abs(o64).max())
+    assert worst < 1e-5
+    assert np.max(np.abs(S32 - S64)) < 1e-4 * max(1.0, np.abs(S64).max())
+
+
+@pytest.mark.parametrize("kda", [False, True])
+def test_step_from_codes_matches_fp64_update(kda):
+    # the packed step equals the fp64 recurrence applied to the retained
+    # reconstruction, up to the fp32 roundings of the state elements
+    D = 128
+    rw = np.where(rng.uniform(size=D) < 0.1, 16, 6).astype(np.int32) if kda else np.full(D, 6, np.int32)
+    S = rng.standard_normal((D, D)).astype(np.float32)
+    z, h, r, c, _ = core.quantize(D, rw, np.ones(D, np.float32), np.ones(D, np.float32), S)
+    Shat = core.reconstruct(D, rw, z, h, r, c).astype(np.float64)
+    q, k, v, alpha, beta = _rand_inputs(D, kda)
+    St, o, u, w = core.step_from_codes(D, rw, z, h, r, c, q, k, v, alpha, beta)
+    ref = Shat.copy()
+    o_ref = core.step_fp64(ref, q, k, v, alpha.astype(np.float64), np.float64(beta))
+    scale = np.abs(ref).max()
+    assert np.max(np.abs(St - ref)) < 4e-6 * scale
+    assert np.allclose(o, o_ref, rtol=2e-5, atol=2e-5 * scale)
+
+
+def test_error_recursion_and_output_error_fp64():
+    # E_t = A_t E_{t-1} + eps_t and output error = E_{t-1}^T A_t^T q_t
+    # (背景与动机).  Quantized trajectory: exact update of the reconstructed
+    # state, then requantization (eps_t = S_hat_t - S_tilde_t).
+    D = 128
+    rw = np.full(D, 4, np.int32)
+    ones = np.ones(D, np.float32)
+    S_fp = rng.standard_normal((D, D))
+    S_hat = S_fp.copy()
+    E = S_hat - S_fp
+    for t in range(24):
+        q, k, v, alpha, beta = _rand_inputs(D, kda=True)
+        a64, b64 = alpha.astype(np.float64), np.float64(beta)
+        o_fp = core.step_fp64(S_fp, q, k, v, a64, b64)
+        S_tilde = S_hat.copy()
+        o_q = core.step_fp64(S_tilde, q, k, v, a64, b64)
+        AE = E.copy()
+        o_err = core.step_fp64(AE, q, k, np.zeros(D), a64, b64)   # A_t E_{t-1}, (A_t E)^T q
+        z, h, r, c, _ = core.quantize(D, rw, ones, ones, S_tilde.astype(np.float32))
+        S_new = r.astype(np.float64)[:, None] * c.astype(np.float64)[None, :] * z
+        eps = S_new - S_tilde
+        S_hat = S_new
+        E_new = S_hat - S_fp
+        scale = np.abs(E_new).max()
+        assert np.max(np.abs(E_new - (AE + eps))) <= 1e-12 * max(scale, np.abs(S_fp).max())
+        assert np.max(np.abs((o_q - o_fp) - o_err)) <= 1e-11 * np.abs(o_fp).max()
+        E = E_new
+
+
+# --------------------------------------------------------------------------
+# lifetime weight (方法-1)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("h", [2.0, 50.0, 1000.0, 20000.0])
+def test_lifetime_closed_form(h):
+    l = -math.log(2.0) / h
+    H = 4096
+    assert math.isclose(core.lifetime_weight(l, H), allocator.lifetime_weight_closed_form(l, H), rel_tol=1e-12)
+    assert core.lifetime_weight(0.0, 100) == 100.0
+
+
+# --------------------------------------------------------------------------
+# quantizer (方法-3)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("b", [2, 4, 6, 8])
+def test_quantizer_constant_magnitude(b):
+    D = 128
+    s = np.float32(0.25)
+    S = (s * np.where(rng.uniform(size=(D, D)) < 0.5, -1, 1)).astype(np.float32)
+    rw = np.full(D, b, np.int32)
+    ones = np.ones(D, np.float32)
+    z, h, r, c, tie = core.quantize(D, rw, ones, ones, S)
+    q = (1 << (b - 1)) - 1
+    assert np.array_equal(np.abs(z), np.full((D, D), q))
+    assert np.array_equal(np.sign(z), np.sign(S).astype(np.int32))
+    Sh = core.reconstruct(D, rw, z, h, r, c)
+    assert np.max(np.abs(Sh - S)) <= 2 * np.spacing(s)
+
+
+@pytest.mark.parametrize("b", [2, 4, 6, 8])
+def test_quantizer_half_step_bound(b):
+    D = 128
+    S = (rng.standard_normal((D, D)) * rng.uniform(0.1, 10, (D, 1)) * rng.uniform(0.1, 19, (1, D))).astype(np.float32)
+    rw = np.full(D, b, np.int32)
+    wbar = rng.uniform(0.2, 5.0, D).astype(np.float32)
+    rho = (1.0 / np.sqrt(np.sqrt(wbar.astype(np.float64)))).astype(np.float32)
+    z, h, r, c, tie = core.quantize(D, rw, rho, wbar, S)
+    q = (1 << (b - 1)) - 1
+    assert np.abs(z).max() <= q
+    Sh = core.reconstruct(D, rw, z, h, r, c).astype(np.float64)
+    step = r.astype(np.float64)[:, None] * c.astype(np.float64)[None, :]
+    unclamped = np.abs(z) < q
+    err = np.abs(Sh - S)
+    bound = 0.5 * step * (1 + 1e-5) + 2 * np.spacing(np.abs(S.astype(np.float32)))
+    assert np.all(err[unclamped] <= bound[unclamped])
+
+
+def test_quantizer_refinement_is_weighted_ls():
+    # for the initial codes z0, c_j minimises sum_i w_i (S_ij - r_i c z0_ij)^2
+    D = 128
+    b = 4
+    S = (rng.standard_normal((D, D)) * rng.uniform(0.5, 3, (D, 1))).astype(np.float32)
+    rw = np.full(D, b, np.int32)
+    wbar = rng.uniform(0.2, 5.0, D).astype(np.float32)
+    rho = (1.0 / np.sqrt(np.sqrt(wbar.astype(np.float64)))).astype(np.float32)
+    z, h, r, c, tie, z0 = core.quantize(D, rw, rho, wbar, S, return_z0=True)
+    S64, r64, w64 = S.astype(np.float64), r.astype(np.float64), wbar.astype(np.float64)
+    invphi = (math.sqrt(5) - 1) / 2
+    for j in range(0, D, 7):
+        f = lambda cc: float(np.sum(w64 * (S64[:, j] - r64 * cc * z0[:, j]) ** 2))
+        lo, hi = 0.2 * c[j], 5.0 * c[j]
+        x1, x2 = hi - invphi * (hi - lo), lo + invphi * (hi - lo)
+        f1, f2 = f(x1), f(x2)
+        for _ in range(120):
+            if f1 < f2:
+                hi, x2, f2 = x2, x1, f1
+                x1 = hi - invphi * (hi - lo)
+                f1 = f(x1)
+            else:
+                lo, x1, f1 = x1, x2, f2
+                x2 = lo + invphi * (hi - lo)
+                f2 = f(x2)
+        assert math.isclose(c[j], 0.5 * (lo + hi), rel_tol=1e-5)
+
+
+def test_quantizer_scale_invariance():
+    # S -> 2^k S scales the row factors by 2^k and leaves c and z unchanged
+    D = 128
+    S = rng.standard_normal((D, D)).astype(np.float32)
+    rw = np.full(D, 6, np.int32)
+    wbar = rng.uniform(0.2, 5.0, D).astype(np.float32)
+    rho = (1.0 / np.sqrt(np.sqrt(wbar.astype(np.float64)))).astype(np.float32)
+    z1, _, r1, c1, _ = core.quantize(D, rw, rho, wbar, S)
+    z2, _, r2, c2, _ = core.quantize(D, rw, rho, wbar, (S * np.float32(8.0)).astype(np.float32))
+    assert np.array_equal(z1, z2) and np.array_equal(c1, c2) and np.array_equal(r2, r1 * 8)
+
+
+def test_quantizer_degenerate():
+    D = 16
+    rw = np.full(D, 4, np.int32)
+    ones = np.ones(D, np.float32)
+    S = np.zeros((D, D), np.float32)
+    z, h, r, c, _ = core.quantize(D, rw, ones, ones, S)
+    assert np.all(z == 0) and np.all(c == 1.0) and np.all(r == np.float32(1e-12))
+    S = rng.standard_normal((D, D)).astype(np.float32)
+    S[:, 3] = 0
+    z, h, r, c, _ = core.quantize(D, rw, ones, ones, S)
+    assert c[3] == 1.0 and np.all(z[:, 3] == 0)
+
+
+def test_quantizer_pivot_rows_fp16():
+    D = 16
+    rw = np.array([4] * 12 + [16] * 4, np.int32)
+    ones = np.ones(D, np.float32)
+    S = rng.standard_normal((D, D)).astype(np.float32)
+    z, h, r, c, _ = core.quantize(D, rw, ones, ones, S)
+    assert np.array_equal(h[12:], S[12:].astype(np.float16).view(np.uint16))
+    assert np.all(r[12:] == 0)
+    # the pivot rows take no part in the column fit: same c as without them
+    z2, _, _, c2, _ = core.quantize(D, rw[:12].tolist() + [16] * 4, ones, ones,
+                                    np.concatenate([S[:12], np.zeros((4, D), np.float32)]))
+    assert np.array_equal(c, c2)
+
+
+def test_tie_flag():
+    # a value placed on a .5 boundary is flagged
+    D = 16
+    rw = np.full(D, 2, np.int32)
+    ones = np.ones(D, np.float32)
+    S = np.ones((D, D), np.float32)
+    S[0, 0] = 0.5       # with r = mean|S| ~ 1, c = 1: x = 0.5 / r ... near .5 boundary
+    z, h, r, c, tie = core.quantize(D, rw, ones, ones, S)
+    y = (S * (np.float32(1) / r)[:, None]).astype(np.float32)
+    x = y.astype(np.float64) * (np.float32(1) / c).astype(np.float64)[None, :]
+    frac = np.abs(np.abs(x) - (np.floor(np.abs(x)) + 0.5))
+    assert np.array_equal(tie & 1, (frac <= 1e-6 * np.abs(x)).astype(np.uint8))
+
+
+# --------------------------------------------------------------------------
+# allocator (方法-1)
+# --------------------------------------------------------------------------
+
+def _convex_costs(N, widths):
+    # d(b) decreasing and convex in b, times a lifetime weight
+    out = np.zeros((N, len(widths)))
+    for u in range(N):
+        base = rng.uniform(0.5, 2.0)
+        rate = rng.uniform(0.3, 0.7)
+        Lw = rng.uniform(1.0, 100.0)
+        out[u] = Lw * base * np.exp(-rate * np.asarray(widths, float))
+    return out
+
+
+@pytest.mark.parametrize("widths", [(4, 6, 8), (2, 4, 6, 8)])
+@pytest.mark.parametrize("N", [3, 5, 7])
+def test_dp_equals_brute_force(widths, N):
+    for trial in range(6):
+        cost = rng.uniform(0, 10, (N, len(widths)))   # arbitrary (non-convex too)
+        for nominal in (widths[0] + 0.5, (widths[0] + widths[-1]) / 2, widths[-1] - 1.0):
+            cap = allocator.budget_cap(nominal, N)
+            a = allocator.dp_allocate_budget(cost, widths, cap)
+            bf = allocator.brute_force(cost, widths, cap)
+            assert np.array_equal(a, bf)
+            assert a.sum() <= cap
+
+
+@pytest.mark.parametrize("widths", [(4, 6, 8), (2, 4, 6, 8)])
+@pytest.mark.parametrize("N", [4, 6, 8])
+def test_lagrangian_equals_brute_force_convex(widths, N):
+    for trial in range(6):
+        cost = _convex_costs(N, widths)
+        for nominal in (widths[0] + 0.7, (widths[0] + widths[-1]) / 2, widths[-1] - 0.6):
+            cap = allocator.budget_cap(nominal, N)
+            a = allocator.lagrangian_allocate(cost, widths, cap)
+            bf = allocator.brute_force(cost, widths, cap)
+            assert a.sum() <= cap
+            assert math.isclose(allocator.total_cost(cost, widths, a),
+                                allocator.total_cost(cost, widths, bf), rel_tol=1e-12)
+
+
+def test_lagrangian_nonconvex_gap_reported():
+    widths = (4, 6, 8)
+    gaps = []
+    for trial in range(20):
+        cost = rng.uniform(0, 10, (6, 3))
+        cap = allocator.budget_cap(6.0, 6)
+        a = allocator.lagrangian_allocate(cost, widths, cap)
+        bf = allocator.brute_force(cost, widths, cap)
+        assert a.sum() <= cap
+        ca, cb = allocator.total_cost(cost, widths, a), allocator.total_cost(cost, widths, bf)
+        assert ca >= cb - 1e-12
+        gaps.append(ca / cb - 1)
+    print("non-convex Lagrangian gap: max %.3g mean %.3g" % (max(gaps), float(np.mean(gaps))))
+
+
+def test_pivots_top_scores_ties_lower_index():
+    L = np.array([1.0, 2.0, 2.0, 0.5, 3.0])
+    d = np.array([1.0, 1.0, 1.0, 1.0, 1.0])
+    assert list(allocator.select_pivots(L, d, 2)) == [1, 4]
+    assert list(allocator.select_pivots(L, d, 3)) == [1, 2, 4]
+
+
+def test_bits_per_value_hand_count():
+    # mode 0, D = 16, two heads at widths 4 and 16 (pivot):
+    # codes 4*256 + 16*256 = 5120; scales of head 0: (16 + 16) * 32 = 1024 -> 6144 / 512
+    assert allocator.bits_per_value(0, 1, 2, 16, [4, 16]) == 12.0
+    # mode 1, D = 16, one head: 15 rows at 4 bits and 1 FP16 row:
+    # codes 15*16*4 + 16*16 = 1216; r 15*32 = 480; c 16*32 = 512 -> 2208 / 256
+    assert allocator.bits_per_value(1, 1, 1, 16, [4] * 15 + [16]) == 2208 / 256
+    # 16-bit scale accounting of the same head
+    assert allocator.bits_per_value(1, 1, 1, 16, [4] * 15 + [16], scale_bits=16) == (1216 + 15 * 16 + 256) / 256
+
+
+def test_real_distortion_curves_are_convex():
+    # the quantizer's distortion falls convexly with the width on this data,
+    # which is what makes the Lagrangian + repair exact
+    D = 128
+    S = (rng.standard_normal((D, D)) * rng.uniform(0.5, 3, (D, 1))).astype(np.float32)
+    ones = np.ones(D, np.float32)
+    d = [core.distortion_rows(D, b, ones, ones, S).sum() for b in (2, 4, 6, 8)]
+    drops = -np.diff(d)
+    assert np.all(drops > 0) and np.all(np.diff(drops) < 0)
+
+
+def test_plan_roundtrip(tmp_path):
+    wl = synth.workloads()["tiny_gdn"]
+    D = wl.d
+    plan = dict(mode=0, n_layers=1, n_heads=4, d=D, n_pivots=1, bitset=[2, 4, 6], nominal_bits=4.0,
+                horizon=65536, widths=np.array([2, 6, 16, 4], np.uint8),
+                wbar=np.ones(4 * D, np.float32), rho=np.ones(4 * D, np.float32),
+                lgate=np.zeros(4), lifetime=np.ones(4))
+    data = plan_io.write_plan(str(tmp_path / "p.bin"), plan)
+    back = plan_io.read_plan(data)
+    assert np.array_equal(back["widths"], plan["widths"]) and back["mode"] == 0
+    offs, slot = plan_io.pool_layout(back)
+    # records: b=2: 64+128 -> 256; b=6: 192+128 -> 384; pivot 512; b=4: 128+128 = 256
+    assert list(offs) == [0, 256, 640, 1152] and slot == 1408
