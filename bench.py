@@ -1,0 +1,618 @@
+#!/usr/bin/env python
+"""Packed-state decode benchmark on B200.
+
+Workload: the 2,304-head GDN state pool (48 layers x 48 heads, d_k = d_v =
+128) at 70 concurrent requests, nominal 6-bit plan over {4,6,8} with 32 FP16
+pivot heads, synthetic seeded inputs.  A step is one decode step of every
+(request, layer, head) state: reconstruct -> retention + delta update ->
+readout -> refit r, c -> pack -> write back.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+                    [--variant two_stream|fused] [--batch B] [--plan 6|4] [--sweep]
+
+Prints one JSON line (rank 0).  N > 1: launched by torch.distributed.run, one
+independent pool per GPU (no collective on the data path), barrier + max of
+the per-rank device times.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "packed-state decode head-steps/s and HBM GB/s (% of peak), 2304 heads, bs=70"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["stepq_step.cu", "stepq_dev.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="stepq", choices=["stepq", "reference"])
+    ap.add_argument("--variant", default="fused", choices=["fused", "two_stream"])
+    ap.add_argument("--batch", type=int, default=70)
+    ap.add_argument("--plan", type=int, default=6, choices=[4, 6])
+    ap.add_argument("--sweep", action="store_true", help="also time batch 1/16/70/128/256")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_init():
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# measurement helpers
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "quantized_recurrent_state_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(variant: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    f = os.path.join(ROOT, "profiles", f"{variant}_kernel_traffic.txt")
+    try:
+        kv = dict(line.split(":", 1) for line in open(f) if ":" in line and not line.startswith("#"))
+    except OSError:
+        return None
+    if kv.get("kernel_hash", "").strip() != kernel_hash():
+        return None
+    try:
+        return float(kv["dram_bytes_per_full_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------
+# product path
+# ---------------------------------------------------------------------------
+
+def product_plan(stepq, synth, wl, device):
+    """Calibrate on the GPU (FP32-state recurrence + omega / log-gate /
+    distortion kernels) and build the plan with the library's planner."""
+    import torch
+    L, H, D = wl.n_layers, wl.n_heads, wl.d
+    bits = list(wl.bits)
+    # a uniform 8-bit plan only to host the calibration kernels' context
+    units = L * H
+    dummy = stepq.Plan.build(0, L, H, D, bits, float(max(bits)), 0, wl.horizon, np.zeros(units),
+                             np.tile(np.linspace(1.0, 0.25, len(bits)), (units, 1)), np.ones(L * H * D, np.float32))
+    n = wl.calib_req
+    ctx = stepq.Context(dummy, n)
+    alpha = synth.gates(wl, wl.calib_seed)
+    om = torch.zeros((L, H, D), dtype=torch.float64, device=device)
+    ls = torch.zeros_like(om)
+    S = torch.cat([synth.initial_states_torch(wl, wl.calib_seed, n, l, device) for l in range(L)], dim=1)
+    slots = torch.arange(n, dtype=torch.int32, device=device)
+    steps = [synth.step_inputs_torch(wl, wl.calib_seed, n, t, alpha, device) for t in range(wl.calib_steps)]
+    for st in steps:
+        ctx.calib_accumulate(n, 0, L, st["q"], st["k"], st["alpha"], st["beta"], om, ls)
+    ctx.sync()
+    omega = om.cpu().numpy() / (wl.calib_steps * n)
+    lmean = ls.cpu().numpy() / (wl.calib_steps * n)
+    wbar = np.maximum(omega / omega.mean(axis=2, keepdims=True), 1e-12).astype(np.float32)
+    wbar_d = torch.from_numpy(wbar).to(device)
+    dist = torch.zeros((L, H, D, len(bits)), dtype=torch.float64, device=device)
+    o = torch.zeros((n, L, H, D), dtype=torch.float32, device=device)
+    n_snap = 0
+    for t, st in enumerate(steps):
+        ctx.fp32_decode_step(S, slots, n, 0, L, st["q"], st["k"], st["v"], st["alpha"], st["beta"], o)
+        if (t + 1) % 8 == 0:
+            ctx.calib_distortion(n, 0, L, S, wbar_d, bits, dist)
+            n_snap += 1
+    ctx.sync()
+    d = dist.cpu().numpy() / (n_snap * n)
+    ctx.close()
+    import tempfile
+    fd, path = tempfile.mkstemp(suffix=".plan")
+    os.close(fd)
+    plan = stepq.Plan.build(0, L, H, D, bits, wl.nominal_bits, wl.n_pivots, wl.horizon,
+                            lmean.mean(axis=2).reshape(-1), d.sum(axis=2).reshape(-1, len(bits)),
+                            wbar.reshape(-1), path=path)
+    data = open(path, "rb").read()
+    os.unlink(path)
+    return plan, data
+
+
+def step_bytes(plan, n_req):
+    """Algorithmic bytes of one single-pass step: every record read and
+    written once, q, k, v read, o written, alpha and beta read."""
+    L, H, D = plan.n_layers, plan.n_heads, plan.d
+    rec = 0
+    for l in range(L):
+        for h in range(H):
+            rec += plan.record(l, h)[1]
+    per_slot = 2 * rec + L * H * (3 * 4 * D + 8 + 4 * D)
+    return per_slot * n_req
+
+
+def kernel_bytes(plan, n_req, kind):
+    """Algorithmic bytes per launch of the per-kernel roofline: decode reads
+    records, q, k, v, alpha, beta and writes o, w; fit-pack reads records, k,
+    w, alpha, beta and writes records."""
+    L, H, D = plan.n_layers, plan.n_heads, plan.d
+    rec = sum(plan.record(l, h)[1] for l in range(L) for h in range(H))
+    if kind == "fused":
+        return step_bytes(plan, n_req)
+    if kind == "decode":
+        return n_req * (rec + L * H * (3 * 4 * D + 8 + 2 * 4 * D))
+    return n_req * (2 * rec + L * H * (2 * 4 * D + 8))
+
+
+def run_step(ctx, variant, pool, slots, n, L, inp, o, ws):
+    if variant == "fused":
+        ctx.decode_step_fused(pool, slots, n, 0, L, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o)
+    else:
+        ctx.decode_step(pool, slots, n, 0, L, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o, ws)
+
+
+def time_steps(torch, ctx, variant, pool, slots, n, L, sets, o, ws, warmup, steps, ws_ranks, clocks=None):
+    """Device time of `steps` steps (CUDA events on the main stream, which
+    waits for the side stream at the end); returns (seconds, kernel stats)."""
+    main, side = ctx.main, ctx.side
+    for i in range(warmup):
+        run_step(ctx, variant, pool, slots, n, L, sets[i % len(sets)], o, ws)
+    ctx.sync()
+    ctx.kernel_stats()
+    torch.cuda.synchronize()
+    barrier(ws_ranks)
+    torch.cuda.synchronize()
+    ctx.set_timing(True)
+    launches0 = ctx.launches
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    join = torch.cuda.Event()
+    if clocks:
+        clocks.__enter__()
+    e0.record(main)
+    for i in range(steps):
+        run_step(ctx, variant, pool, slots, n, L, sets[i % len(sets)], o, ws)
+    join.record(side)
+    main.wait_event(join)
+    e1.record(main)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.__exit__(None, None, None)
+    ctx.sync()
+    barrier(ws_ranks)
+    torch.cuda.synchronize()
+    ctx.set_timing(False)
+    launches = ctx.launches - launches0
+    stats = ctx.kernel_stats()
+    return e0.elapsed_time(e1) / 1e3, stats, launches
+
+
+def run_product(args):
+    import torch
+    from quantized_recurrent_state_b200 import build as qbuild
+    ws, rank, local = dist_init()
+    if rank == 0:
+        qbuild.build()
+    barrier(ws)
+    from quantized_recurrent_state_b200 import stepq, synth
+    device = torch.device("cuda", local)
+    wl = synth.workloads()["qwen_pool6" if args.plan == 6 else "qwen_pool4"]
+    n = args.batch
+    plan, plan_bytes = product_plan(stepq, synth, wl, device)
+    L, H, D = wl.n_layers, wl.n_heads, wl.d
+    ctx = stepq.Context(plan, n)
+    pool = torch.zeros(n * plan.slot_bytes, dtype=torch.uint8, device=device)
+    slots = torch.arange(n, dtype=torch.int32, device=device)
+    for l in range(L):
+        ctx.requant_pack(pool, slots, n, l, l + 1, synth.initial_states_torch(wl, wl.seed, n, l, device))
+    ctx.sync()
+    alpha = synth.gates(wl, wl.seed)
+    sets = [synth.step_inputs_torch(wl, wl.seed, n, t, alpha, device) for t in range(4)]
+    o = torch.zeros((n, L, H, D), dtype=torch.float32, device=device)
+    wsp = torch.empty(ctx.workspace_bytes(n, L) // 4, dtype=torch.float32, device=device)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    secs, stats, launches = time_steps(torch, ctx, args.variant, pool, slots, n, L, sets, o, wsp,
+                                       args.warmup, args.steps, ws, clocks)
+    secs = max_over_ranks(secs, ws)
+    head_steps = n * L * H * args.steps
+    value = sum_over_ranks(head_steps, ws) / secs
+    sb = step_bytes(plan, n)
+    gbs = sb * args.steps / secs / 1e9
+    peak, peak_kind = measured_peaks()
+
+    # dominant kernel of the variant: its own algorithmic bytes over its mean launch time
+    kind = "fused" if args.variant == "fused" else max(("decode", "fitpack"), key=lambda k: stats[k][0])
+    k_ms, k_n = stats[kind]
+    k_bytes = kernel_bytes(plan, n, kind)
+    achieved = k_bytes / (k_ms / k_n / 1e3) / 1e9 if k_n else None
+    traffic = profiled_traffic(args.variant)
+
+    extra = {}
+    # FP32-state reference kernel: same workload, fp32 state pool
+    if rank == 0:
+        S32 = torch.empty((n, L, H, D, D), dtype=torch.float32, device=device)
+        for l in range(L):
+            S32[:, l:l + 1] = synth.initial_states_torch(wl, wl.seed, n, l, device)
+        for i in range(2):
+            ctx.fp32_decode_step(S32, slots, n, 0, L, sets[i]["q"], sets[i]["k"], sets[i]["v"], sets[i]["alpha"],
+                                 sets[i]["beta"], o)
+        torch.cuda.synchronize()
+        reps = 4
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(ctx.main)
+        for i in range(reps):
+            ctx.fp32_decode_step(S32, slots, n, 0, L, sets[i % 4]["q"], sets[i % 4]["k"], sets[i % 4]["v"],
+                                 sets[i % 4]["alpha"], sets[i % 4]["beta"], o)
+        e1.record(ctx.main)
+        torch.cuda.synchronize()
+        t32 = e0.elapsed_time(e1) / 1e3 / reps
+        b32 = n * L * H * (2 * 4 * D * D + 3 * 4 * D + 8 + 4 * D)
+        extra["fp32_state_kernel"] = {"head_steps_per_s": n * L * H / t32, "ms_per_step": t32 * 1e3,
+                                      "gbs": b32 / t32 / 1e9, "frac": b32 / t32 / 1e9 / peak}
+        del S32
+        torch.cuda.empty_cache()
+        # in-run stream-copy peak
+        nb = 4 << 30
+        a = torch.empty(nb, dtype=torch.uint8, device=device)
+        b = torch.empty_like(a)
+        stream = torch.cuda.current_stream()
+        stepq.copy_probe(b, a, nb, stream)
+        best = 0.0
+        for _ in range(10):
+            c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            c0.record(stream)
+            stepq.copy_probe(b, a, nb, stream)
+            c1.record(stream)
+            torch.cuda.synchronize()
+            best = max(best, 2 * nb / (c0.elapsed_time(c1) / 1e3) / 1e9)
+        extra["copy_probe_gbs"] = best
+        del a, b
+        torch.cuda.empty_cache()
+
+    # end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {k: v.cpu().pin_memory() for k, v in sets[0].items()}
+        dev_in = {k: torch.empty_like(v) for k, v in sets[0].items()}
+        o_host = torch.empty(o.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(v.numel() * 4 for v in host.values())
+        d2h = o_host.numel() * 4
+        k_e2e = min(args.steps, 16)
+        torch.cuda.synchronize()
+        barrier(ws)
+        t0 = time.perf_counter()
+        with torch.cuda.stream(ctx.main):
+            for i in range(k_e2e):
+                for kk in host:
+                    dev_in[kk].copy_(host[kk], non_blocking=True)
+                run_step(ctx, args.variant, pool, slots, n, L, dev_in, o, wsp)
+                ctx.main.wait_stream(ctx.side)
+                o_host.copy_(o, non_blocking=True)
+        ctx.sync()
+        torch.cuda.synchronize()
+        t_e2e = max_over_ranks(time.perf_counter() - t0, ws)
+        e2e = {"value": sum_over_ranks(n * L * H * k_e2e, ws) / t_e2e, "unit": "head-steps/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e}
+
+    sweep = None
+    if args.sweep and rank == 0:
+        sweep = []
+        for bs in (1, 16, 70, 128, 256):
+            c2 = stepq.Context(plan, bs)
+            p2 = torch.zeros(bs * plan.slot_bytes, dtype=torch.uint8, device=device)
+            s2 = torch.arange(bs, dtype=torch.int32, device=device)
+            for l in range(L):
+                c2.requant_pack(p2, s2, bs, l, l + 1, synth.initial_states_torch(wl, wl.seed, bs, l, device))
+            st2 = [synth.step_inputs_torch(wl, wl.seed, bs, t, alpha, device) for t in range(2)]
+            o2 = torch.zeros((bs, L, H, D), dtype=torch.float32, device=device)
+            w2 = torch.empty(c2.workspace_bytes(bs, L) // 4, dtype=torch.float32, device=device)
+            sec2, _, _ = time_steps(torch, c2, args.variant, p2, s2, bs, L, st2, o2, w2, 3, 16, 1)
+            sweep.append({"batch": bs, "head_steps_per_s": bs * L * H * 16 / sec2,
+                          "tokens_per_s": bs * 16 / sec2, "gbs": step_bytes(plan, bs) * 16 / sec2 / 1e9,
+                          "ms_per_step": sec2 / 16 * 1e3})
+            c2.close()
+            del p2, st2, o2, w2
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu:
+        cpu = cpu_baseline(plan_bytes, wl, budget_s=12.0)
+
+    if rank == 0:
+        csum = clocks.summary()
+        out = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "head-steps/s",
+            "n_gpus": ws,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic",
+            "config": {
+                "workload": f"GDN state pool, {L} layers x {H} heads = {L * H} heads, d_k=d_v={D}, batch {n}, "
+                            f"nominal {wl.nominal_bits:g}-bit plan over {set(wl.bits)}, {wl.n_pivots} FP16 pivot heads",
+                "batch": n, "heads": L * H, "d": D, "variant": args.variant,
+                "bits_per_value": plan.info.bits_per_value, "bits_per_value_s16": plan.info.bits_per_value_s16,
+                "pool_bytes": n * plan.slot_bytes, "l2": "inputs larger than L2 (pool and q/k/v far above 126 MB)",
+                "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+            },
+            "hbm_gbs": gbs,
+            "hbm_frac": gbs / peak,
+            "tokens_per_s": sum_over_ranks(n * args.steps, ws) / secs,
+            "roofline": {"bound": "hbm", "kernel": kind, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak if achieved else None, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": k_bytes, "launch_ms": k_ms / k_n if k_n else None,
+                         "peak_source": peak_kind},
+            "kernel_ms": {k: v[0] for k, v in stats.items() if v[1]},
+            "kernel_launches": {k: v[1] for k, v in stats.items() if v[1]},
+            "gpu_launches": launches,
+            "clocks": {"sm_mhz": csum["sm_mhz"], "sm_max_mhz": csum["sm_max_mhz"], "reasons": csum["reasons"]},
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            **extra,
+        }
+        if sweep:
+            out["sweep"] = sweep
+        print(json.dumps(out), flush=True)
+    ctx.close()
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+
+def _oracle_sample(payload):
+    """One decode step of a set of (layer, head) states of request 0 with the
+    oracle.  Packing S_0 and drawing inputs are not timed; returns the seconds
+    spent stepping."""
+    import numpy as np
+    from oracle import model, plan_io
+    from quantized_recurrent_state_b200 import synth
+    plan_bytes, wname, heads, t = payload
+    plan = plan_io.read_plan(plan_bytes)
+    pv = model.PlanView(plan)
+    wl = synth.workloads()[wname]
+    alpha = synth.gates(wl, wl.seed)
+    layers = sorted({l for l, _ in heads})
+    inp = synth.step_inputs(wl, wl.seed, 1, t, alpha=alpha, layers=layers)
+    slot = np.zeros(pv.slot_bytes, np.uint8)
+    for li, l in enumerate(layers):
+        S0 = synth.initial_states(wl, wl.seed, 1, layers=[l])
+        for (l2, h) in heads:
+            if l2 == l:
+                pv.quantize_into(slot, l, h, S0[0, 0, h])
+    t0 = time.perf_counter()
+    for (l, h) in heads:
+        li = layers.index(l)
+        pv.step(slot, l, h, inp["q"][0, li, h], inp["k"][0, li, h], inp["v"][0, li, h],
+                inp["alpha"][0, li, h], inp["beta"][0, li, h])
+    return time.perf_counter() - t0
+
+
+def _oracle_calib_layer(payload):
+    """Oracle calibration statistics of one layer (all its heads)."""
+    from oracle import model
+    from quantized_recurrent_state_b200 import synth
+    wname, l = payload
+    wl = synth.workloads()[wname]
+    S0 = synth.initial_states(wl, wl.calib_seed, wl.calib_req, layers=[l])
+    alpha = synth.gates(wl, wl.calib_seed)
+    steps = [synth.step_inputs(wl, wl.calib_seed, wl.calib_req, t, alpha=alpha, layers=[l])
+             for t in range(wl.calib_steps)]
+    return model.calibrate(wl.mode, wl.d, 1, wl.n_heads, S0, steps, wl.bits)
+
+
+def _n_cores():
+    return max(1, min(os.cpu_count() or 1, 32))
+
+
+def cpu_sample_rate(plan_bytes, wl, heads_per_step, t, pool, cores):
+    """Head-steps/s of the oracle over one sample: heads split across the
+    worker processes; the step time is the slowest worker's stepping time."""
+    heads = [(l, h) for l in range(wl.n_layers) for h in range(wl.n_heads)][:heads_per_step]
+    chunks = [heads[i::cores] for i in range(cores)]
+    secs = pool.map(_oracle_sample, [(plan_bytes, wl.name, c, t) for c in chunks if c])
+    return len(heads), max(secs)
+
+
+def cpu_baseline(plan_bytes, wl, budget_s=12.0):
+    """The oracle, as it stands, on the host cores: a bounded sample of the
+    same workload (request 0's heads in layer order, one decode step each)
+    sized to about budget_s seconds of CPU work in total."""
+    import multiprocessing as mp
+    cores = _n_cores()
+    per_head = _oracle_sample((plan_bytes, wl.name, [(0, 0)], 0))
+    heads = int(min(wl.n_layers * wl.n_heads, max(cores, budget_s / max(per_head, 1e-4))))
+    with mp.get_context("spawn").Pool(cores) as pool:
+        nh, sec = cpu_sample_rate(plan_bytes, wl, heads, 0, pool, cores)
+    return {"value": nh / sec, "unit": "head-steps/s", "cores": cores, "kind": "oracle",
+            "sample": f"{nh} (layer, head) states of request 0, one decode step each, split over {cores} "
+                      f"spawned processes; time = slowest process's stepping time"}
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: same metric and workload, each
+    step a bounded sample of (layer, head) states of one request."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import multiprocessing as mp
+    from oracle import model, plan_io
+    from quantized_recurrent_state_b200 import synth
+    wl = synth.workloads()["qwen_pool6" if args.plan == 6 else "qwen_pool4"]
+    cores = _n_cores()
+    with mp.get_context("spawn").Pool(cores) as pool:
+        layer_stats = pool.map(_oracle_calib_layer, [(wl.name, l) for l in range(wl.n_layers)])
+        stats = {k: np.concatenate([np.asarray(s[k]).reshape((1,) + np.asarray(s[k]).shape[1:])
+                                    if k in ("wbar", "rho") else np.asarray(s[k]) for s in layer_stats])
+                 for k in ("wbar", "rho", "lgate", "dist")}
+        plan = model.build_plan(wl.mode, wl.d, wl.n_layers, wl.n_heads, stats, wl.bits, wl.nominal_bits,
+                                wl.n_pivots, wl.horizon)
+        plan_bytes = plan_io.write_plan(None, plan)
+        heads_per_step = 4 * cores
+        for i in range(args.warmup):
+            cpu_sample_rate(plan_bytes, wl, heads_per_step, i, pool, cores)
+        tot_h, tot_s = 0, 0.0
+        for i in range(args.steps):
+            nh, sec = cpu_sample_rate(plan_bytes, wl, heads_per_step, i, pool, cores)
+            tot_h += nh
+            tot_s += sec
+    value = tot_h / tot_s
+    sample = (f"each step: {heads_per_step} (layer, head) states of one request stepped once, split over "
+              f"{cores} spawned processes (time = slowest process)")
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "head-steps/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+           "data": "synthetic",
+           "config": {"workload": f"GDN state pool, {wl.n_layers} layers x {wl.n_heads} heads, d={wl.d}, "
+                                  f"nominal {wl.nominal_bits:g}-bit plan, {wl.n_pivots} FP16 pivot heads (CPU oracle sample)",
+                      "batch": args.batch, "heads": wl.n_layers * wl.n_heads, "d": wl.d},
+           "cpu_baseline": {"value": value, "unit": "head-steps/s", "cores": cores, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": "head-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_product(args)
+
+
+if __name__ == "__main__":
+    main()

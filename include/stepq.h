@@ -1,0 +1,236 @@
+/*
+ * stepq.h -- C ABI of libstepq.so, the B200 (sm_100a) packed recurrent-state
+ * decode step of STEPQuant.
+ *
+ * Source of the method: "STEPQuant: When and Where Errors Matter in
+ * Delta-Rule Recurrent State Quantization", paper digest page
+ * (vibe-research):
+ *   - 背景与动机: one state S_t in R^{dk x dv} per (request, head), updated
+ *     each decode step with the key, value and retention gate and read out
+ *     with the query; E_t = A_t E_{t-1} + eps_t;
+ *   - 方法-1 Lifetime-aware Bit Allocation: per-unit widths {2,4,6,8} from an
+ *     offline precision map, FP16 pivot units, a fixed average-bit budget;
+ *   - 方法-2 Row-impact: omega_i = E[g_{t,i}^2], g_t = A_t^T q_t;
+ *   - 方法-3 Key-Row-Aware Dual-Axis Fitting: X_hat_ij = r_i c_j z_ij;
+ *   - 方法-4 per-step path: reconstruct the tile from codes, scales and FP16
+ *     pivots -> retention + delta update + readout in floating point -> the
+ *     readout goes on at once -> refit r and c -> pack -> asynchronous
+ *     writeback before the next read, scale fitting on a separate stream.
+ *
+ * Arithmetic (the pages print no formulas for it; this library and its CPU
+ * checker implement the same definitions independently):
+ *   recurrence  S_t = (I - beta k k^T) Diag(alpha) S_{t-1} + beta k v^T,
+ *               o_t = S_t^T q_t  (GDN: alpha scalar per head; KDA: per key row)
+ *   decode      a_i = fl(alpha_i r_i);  S'_ij = fl(fl(a_i c_j) z_ij)
+ *               (16-bit rows: S'_ij = fl(alpha_i h_ij))
+ *               u_j = fl32(sum_i k_i a_i c_j z_ij)   exact sum, rounded once
+ *               w_j = fl(beta fl(v_j - u_j));  S_t,ij = fma(k_i, w_j, S'_ij)
+ *               o_j = fl32(sum_i q_i (a_i c_j z_ij + k_i w_j))  exact, rounded once
+ *   requantize  r_i = fl(max(pairwise_j |S_ij| / D, 1e-12) rho_i)
+ *               y = fl(S fl(1/r));  c0_j = max_i fl(|y_ij| / qmax_i) (0 -> 1)
+ *               z0 = rint(y * fl(1/c0))   (exact product, ties to even)
+ *               c_j = fl(pairwise_i fl(b_i fl(z0 y)) / pairwise_i fl(b_i fl(z0 z0))),
+ *                     b_i = fl(wbar_i fl(r_i r_i)); a zero denominator keeps c0
+ *               z = clamp(rint(y * fl(1/c)), -qmax, qmax); 16-bit rows: fp16 RNE
+ *   qmax(b) = 2^(b-1) - 1.  pairwise = fp32 sum in balanced binary-tree order.
+ *
+ * Packed format (decided offline, 方法-4 "fixed packed layout").  Codes are
+ * stored offset-binary, u = z + 2^(b-1).
+ *   per-head units (mode 0), width b in {2,4,6,8}: thread-major layout with
+ *     RT = D/8, NT = 2D: element (i,j) -> thread t = (i/RT)(D/4) + j/4,
+ *     position p = (i%RT)*4 + j%4, stream bits [p b, p b + b) LSB first;
+ *     stream byte B of thread t at block byte ((B/RT) NT + t) RT + B%RT.
+ *   per-row units (mode 1): rows in order, row i = D*b_i/8 bytes, code j at
+ *     row bits [b_i j, b_i j + b_i); a 16-bit row holds binary16 values.
+ *   record = codes | f32 r[D] | f32 c[D], zero-padded to 128 bytes; a mode-0
+ *     pivot head's record is its binary16 tile, row-major, D*D*2 bytes.
+ *   pool   = n_slots slots of slot_bytes each; inside a slot the records of
+ *     (layer, head) follow layer-major (offsets: stepq_plan_record).
+ *
+ * Plan file: see the byte table in the implementation's plan parser
+ * (magic "STEPQPL1", version 1, CRC-32 trailer); fields are listed with
+ * stepq_plan_info.
+ *
+ * Conventions for every call:
+ *   - Device pointers are plain CUDA device addresses on the context's
+ *     device, owned by the caller; the library never frees them.  The
+ *     library allocates only its plan tables, events and a 4-byte error
+ *     word per context.
+ *   - Alignment: pool 128 bytes; all other arrays 16 bytes.
+ *   - q, k, v, o, workspace: [n_req][n_layers_launched][n_heads][D] fp32.
+ *     alpha: mode 0 [n_req][nL][n_heads], mode 1 [n_req][nL][n_heads][D].
+ *     beta: [n_req][nL][n_heads].  S (fp32 states): [n_req][nL][n_heads][D][D].
+ *     slots: device int32[n_req], each in [0, n_slots).
+ *   - Calls are asynchronous on the context's streams, except stepq_sync,
+ *     the plan functions and stepq_last_error.
+ *   - Return 0 (STEPQ_OK) or a negative STEPQ_E* code; stepq_last_error()
+ *     gives a thread-local message.  No C++ exception crosses the ABI.
+ *   - No CPU fallback: without a usable sm_100 device, calls that launch
+ *     work return STEPQ_ECUDA.
+ */
+#ifndef STEPQ_H
+#define STEPQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define STEPQ_OK 0
+#define STEPQ_EINVAL (-1)    /* bad argument: null/misaligned pointer, range, dims */
+#define STEPQ_EFORMAT (-2)   /* plan file malformed: magic, version, CRC, budget ... */
+#define STEPQ_ECUDA (-3)     /* CUDA runtime error (message has the CUDA string) */
+#define STEPQ_ETIMEDOUT (-4) /* stepq_sync gave up waiting */
+#define STEPQ_EDEVICE (-5)   /* a kernel flagged a bad slot or a stalled copy */
+#define STEPQ_ENOMEM (-6)    /* host allocation failed */
+
+#define STEPQ_PIVOT_BITS 16
+
+typedef struct stepq_plan stepq_plan; /* opaque, host-side plan */
+typedef struct stepq_ctx stepq_ctx;   /* opaque, per device: tables, streams, events */
+
+typedef struct stepq_plan_info {
+    int mode;            /* 0 per-head units (GDN), 1 per-key-row units (KDA) */
+    int n_layers;
+    int n_heads;
+    int d;               /* d_k == d_v: 16, 32, 64 or 128 */
+    int n_units;         /* mode 0: n_layers*n_heads; mode 1: times d */
+    int n_pivots;        /* units stored as FP16 */
+    uint32_t bitset;     /* bit b set: width b allowed */
+    float nominal_bits;  /* average-bit budget of the non-pivot units */
+    uint64_t horizon;    /* H of the lifetime weight */
+    uint64_t slot_bytes; /* bytes of one request's packed state */
+    double bits_per_value;       /* codes + FP16 pivots + fp32 scales */
+    double bits_per_value_s16;   /* the same with 16-bit scale accounting */
+    int units_by_width[17];      /* histogram of unit widths (index = bits) */
+} stepq_plan_info;
+
+/* ---- plan (方法-1 offline precision map) -------------------------------- */
+
+/* Parse and validate a plan file.  Checks magic, version, CRC-32, dims, that
+ * every width is allowed by the bitset or is 16, that the number of 16-bit
+ * units equals n_pivots, that the non-pivot widths sum to at most
+ * floor(nominal * N), and that wbar and rho are finite and positive.
+ * Errors: STEPQ_EINVAL (null args, unreadable file), STEPQ_EFORMAT. */
+int stepq_plan_load(const char *path, stepq_plan **out);
+/* Same from a memory image of the file. */
+int stepq_plan_load_mem(const void *data, size_t bytes, stepq_plan **out);
+void stepq_plan_free(stepq_plan *plan);
+int stepq_plan_get_info(const stepq_plan *plan, stepq_plan_info *out);
+/* Copy the unit widths (n_units bytes: 2,4,6,8 or 16). */
+int stepq_plan_widths(const stepq_plan *plan, uint8_t *out);
+/* Byte offset inside a slot and size of the record of (layer, head). */
+int stepq_plan_record(const stepq_plan *plan, int layer, int head, uint64_t *offset, uint64_t *bytes);
+
+/* Build a plan from calibration statistics (方法-1): pivots are the top
+ * n_pivots units by L_u * d_u(b_max) (ties to the lower index); the rest get
+ * widths from `bits` (ascending, spaced by 2) minimising sum L_u d_u(b_u)
+ * with sum b_u <= floor(nominal * N): multiple-choice DP for mode 0, the
+ * Lagrangian with discrete repair for mode 1 (ties: smaller cost, then fewer
+ * bits, then the lexicographically smaller width vector; Lagrangian ties to
+ * the smaller width and the lower index).  L_u = sum_{j<H} exp(2 j l_u),
+ * evaluated in closed form.
+ *   lgate[n_units]            mean log retention gate l_u
+ *   dist[n_units][n_bits]     distortion d_u(b) per allowed width
+ *   wbar[n_layers*n_heads*d]  normalised row impact omega_i / mean omega
+ * rho_i = fl32(1/sqrt(sqrt(wbar_i))) is derived.  Host pointers.  Writes the
+ * plan file to `path` (NULL: none) and returns the parsed plan in *out. */
+int stepq_plan_build(int mode, int n_layers, int n_heads, int d, const int *bits, int n_bits,
+                     float nominal_bits, int n_pivots, uint64_t horizon, const double *lgate,
+                     const double *dist, const float *wbar, const char *path, stepq_plan **out);
+
+/* ---- context ------------------------------------------------------------ */
+
+/* Bind a plan to the current CUDA device.  main/side are cudaStream_t (NULL
+ * for the legacy default stream is rejected: pass real streams).  n_slots is
+ * the capacity of every pool used with this context.  chunk_layers groups
+ * layers per launch pair in stepq_decode_step (<= 0: 4). */
+int stepq_ctx_create(const stepq_plan *plan, void *main_stream, void *side_stream, int n_slots,
+                     int chunk_layers, stepq_ctx **out);
+void stepq_ctx_free(stepq_ctx *ctx);
+/* Bytes of fp32 workspace stepq_decode_step needs for a launch of n_req
+ * requests over nL layers (= n_req*nL*n_heads*d*4). */
+size_t stepq_workspace_bytes(const stepq_ctx *ctx, int n_req, int n_layers_launched);
+
+/* ---- the decode step (方法-4) --------------------------------------------- */
+
+/* Pack fp32 states S into the pool records of (slots, layers [lb, le)):
+ * the requantizer of the header comment (used for S_0).  Enqueued on main. */
+int stepq_requant_pack(stepq_ctx *ctx, void *pool, const int32_t *slots, int n_req, int lb, int le,
+                       const float *S);
+
+/* One decode step over (slots, layers [lb, le), all heads), two streams:
+ * per layer chunk, the decode kernel (reconstruct -> retention + delta ->
+ * readout o, and w for the fit) runs on `main`, and the fit-and-pack kernel
+ * (recompute S_t from the same record and w, refit r and c, pack, write the
+ * record in place) runs on `side` after it.  Before reading a chunk, `main`
+ * waits for the previous call's side work on the same layers.  o is valid on
+ * `main` when the call returns (enqueue order); the pool is valid after
+ * stepq_sync.  workspace: stepq_workspace_bytes() bytes. */
+int stepq_decode_step(stepq_ctx *ctx, void *pool, const int32_t *slots, int n_req, int lb, int le,
+                      const float *q, const float *k, const float *v, const float *alpha,
+                      const float *beta, float *o, void *workspace);
+
+/* The same step in one fused pass per record on `main` (no re-read of the
+ * record, no workspace).  Results are bit-identical to stepq_decode_step. */
+int stepq_decode_step_fused(stepq_ctx *ctx, void *pool, const int32_t *slots, int n_req, int lb,
+                            int le, const float *q, const float *k, const float *v,
+                            const float *alpha, const float *beta, float *o);
+
+/* Wait for all work of the context (both streams) with a host-side timeout
+ * (<= 0: wait without limit), then return the device error word:
+ * STEPQ_OK, STEPQ_ETIMEDOUT, STEPQ_EDEVICE (the word is cleared) or ECUDA. */
+int stepq_sync(stepq_ctx *ctx, int timeout_ms);
+
+/* Reconstruct X_hat = r c z (16-bit rows: their value) into S. */
+int stepq_unpack(stepq_ctx *ctx, const void *pool, const int32_t *slots, int n_req, int lb, int le,
+                 float *S);
+
+/* FP32-state reference step (the unquantized baseline) on an fp32 pool of
+ * [n_slots][n_layers][n_heads][D][D]: S'_ij = fl(alpha_i S_ij), u and o
+ * summed exactly and rounded once, S_ij = fma(k_i, w_j, S'_ij).  On main. */
+int stepq_fp32_decode_step(stepq_ctx *ctx, float *S_pool, const int32_t *slots, int n_req, int lb,
+                           int le, const float *q, const float *k, const float *v,
+                           const float *alpha, const float *beta, float *o);
+
+/* ---- calibration statistics on the device (方法-1, 方法-2) ---------------- */
+
+/* Accumulate, for one calibration step, omega_acc[l][h][i] += g_i^2 with
+ * g = alpha (.) (q - beta k (k^T q)) and lsum_acc[l][h][i] += log alpha_i,
+ * over n_req requests and layers [lb, le).  Accumulators: device fp64
+ * [n_layers][n_heads][d]. */
+int stepq_calib_accumulate(stepq_ctx *ctx, int n_req, int lb, int le, const float *q,
+                           const float *k, const float *alpha, const float *beta,
+                           double *omega_acc, double *lsum_acc);
+/* Accumulate dist_acc[l][h][i][m] += squared reconstruction error of row i
+ * when head (l, h) of each fp32 state in S ([n_req][nL][H][D][D]) is
+ * quantized at uniform width bits[m] with the row weights wbar (device fp32
+ * [n_layers][n_heads][d]). */
+int stepq_calib_distortion(stepq_ctx *ctx, int n_req, int lb, int le, const float *S,
+                           const float *wbar, const int *bits, int n_bits, double *dist_acc);
+
+/* ---- measurement -------------------------------------------------------- */
+
+/* Plain device copy of `bytes` (multiple of 16, 16-byte aligned) on `stream`
+ * (a cudaStream_t): the in-run HBM bandwidth probe. */
+int stepq_copy_probe(void *dst, const void *src, size_t bytes, void *stream);
+
+/* Number of kernel launches this context has issued so far. */
+uint64_t stepq_launch_count(const stepq_ctx *ctx);
+
+/* Kernel timing.  While enabled, every launch of the context is bracketed by
+ * two CUDA events on the stream it runs on.  stepq_kernel_stats waits for
+ * them, adds up the device time per kernel kind (0 decode, 1 fit-pack,
+ * 2 fused, 3 pack/unpack/fp32/calibration), writes ms[4] and launches[4]
+ * (host arrays) and forgets the recorded launches. */
+int stepq_ctx_set_timing(stepq_ctx *ctx, int enable);
+int stepq_kernel_stats(stepq_ctx *ctx, double *ms, uint64_t *launches);
+
+const char *stepq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* STEPQ_H */

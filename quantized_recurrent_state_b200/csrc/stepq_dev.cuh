@@ -1,0 +1,175 @@
+// Device-side helpers of libstepq: launch arguments, the bulk-copy pipeline
+// (cp.async.bulk into shared memory, mbarrier completion, bounded waits),
+// packed-code field extraction and packing, and pairwise reductions.
+//
+// Method: STEPQuant paper digest (vibe-research), 方法-3 (X_hat = r c z) and
+// 方法-4 (fused read -> update -> readout; refit and packed writeback).  The
+// arithmetic definitions are stated in include/stepq.h.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace stepq {
+
+constexpr int kPivotBits = 16;
+constexpr int kErrBadSlot = 1;
+constexpr int kErrWait = 2;
+constexpr int kErrArgs = 4;
+
+// Device copy of the plan tables.
+struct Tables {
+    const uint64_t *rec_off;     // [L*H] record offset inside a slot
+    const uint32_t *rec_bytes;   // [L*H]
+    const uint32_t *codes_bytes; // [L*H] bytes of the codes block
+    const uint8_t *width;        // [L*H] mode 0 unit width (16 = pivot head)
+    const uint8_t *row_width;    // [L*H*D] mode 1 row widths (else null)
+    const uint32_t *row_off;     // [L*H*D] mode 1 row byte offsets (else null)
+    const float *wbar;           // [L*H*D]
+    const float *rho;            // [L*H*D]
+};
+
+struct Args {
+    uint8_t *pool;
+    uint64_t slot_bytes;
+    const int32_t *slots;
+    int n_slots;
+    int n_req;
+    int lb;   // first layer of the launch (absolute)
+    int nL;   // layers in the launch
+    int nL_in;  // layers in the layout of the input/output arrays
+    int l_in0;  // index of layer lb inside that layout
+    int H;
+    int mode;
+    int n_items;             // n_req * nL * H
+    const float *q, *k, *v, *alpha, *beta;
+    float *o;
+    float *w;                // workspace (decode writes, fit-pack reads)
+    const float *S_in;       // requant_pack input
+    float *S_out;            // unpack output
+    Tables t;
+    int *err;
+    uint32_t stage_bytes;    // bytes of one pipeline stage
+    uint32_t rec_stage_bytes;// bytes reserved for the record in a stage
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers: mbarrier + 1-D bulk copy (no multicast).
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// global -> shared bulk copy; dst, src 16-byte aligned, bytes a multiple of 16
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(phase)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: gives up after `limit` polls (each poll may suspend the
+// thread for a hardware-chosen interval), so a lost copy cannot hang the GPU.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t phase, uint32_t limit = (1u << 22)) {
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, phase)) return true;
+    return false;
+}
+
+// ---------------------------------------------------------------------------
+// Packed fields.  A b-bit code z is stored as u = z + 2^(b-1).  The value
+//   X = 0x4B000000 | (u << 12)
+// is at once the fp32 number 2^23 + u 2^12 (so z 2^12 = X - (2^23 + off 2^12)
+// exactly) and, as the high word of an fp64 with a zero low word, the number
+// 2^177 + 2^169 u (so sum_i kap_i 2^-169 X_i = sum_i kap_i (256 + u_i)).
+// ---------------------------------------------------------------------------
+
+template <int B>
+__device__ __forceinline__ uint32_t field_x(const uint32_t *W, int p) {
+    const int bit = p * B;
+    const int w = bit >> 5;
+    const int s = bit & 31;
+    uint32_t x;
+    if (s + B <= 32) {
+        x = (s >= 12) ? (W[w] >> (s - 12)) : (W[w] << (12 - s));
+    } else {
+        x = __funnelshift_r(W[w], W[w + 1], s - 12);
+    }
+    return (x & (((1u << B) - 1u) << 12)) | 0x4B000000u;
+}
+
+__device__ __forceinline__ double x_as_f64(uint32_t X) { return __hiloint2double((int)X, 0); }
+
+template <int B>
+__device__ __forceinline__ float x_as_zscaled(uint32_t X) {
+    // z * 2^12, exact
+    return __fsub_rn(__uint_as_float(X), 8388608.0f + (float)(1 << (B - 1)) * 4096.0f);
+}
+
+// OR a B-bit field into stream position p of W (W zero-initialised).
+template <int B>
+__device__ __forceinline__ void field_put(uint32_t *W, int p, uint32_t u) {
+    const int bit = p * B;
+    const int w = bit >> 5;
+    const int s = bit & 31;
+    W[w] |= u << s;
+    if (s + B > 32) W[w + 1] |= u >> (32 - s);
+}
+
+// ---------------------------------------------------------------------------
+// Reductions: butterfly over `lanes` consecutive lanes.  Adding the partner's
+// value in xor order reproduces the balanced pairwise tree over lane order,
+// and a + b == b + a makes every lane hold the identical root.
+// ---------------------------------------------------------------------------
+
+template <int LANES>
+__device__ __forceinline__ float lane_pairwise_sum(float v) {
+#pragma unroll
+    for (int m = 1; m < LANES; m <<= 1) v = v + __shfl_xor_sync(0xffffffffu, v, m);
+    return v;
+}
+
+template <int LANES>
+__device__ __forceinline__ double lane_sum_f64(double v) {
+#pragma unroll
+    for (int m = 1; m < LANES; m <<= 1) v = v + __shfl_xor_sync(0xffffffffu, v, m);
+    return v;
+}
+
+__device__ __forceinline__ void flag_error(int *err, int code) { atomicOr(err, code); }
+
+}  // namespace stepq

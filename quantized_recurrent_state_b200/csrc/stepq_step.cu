@@ -1,0 +1,913 @@
+// Packed-state decode step kernels for per-head units (GDN, mode 0).
+//
+// STEPQuant paper digest (vibe-research), 方法-4: reconstruct the state tile
+// from integer codes, row/column scales and FP16 pivots; retention, delta
+// update and readout on the floating-point tile; the readout goes on at once;
+// refit the row/column factors; pack codes and scales; write back before the
+// next read.  Arithmetic definitions: include/stepq.h.
+//
+// One CTA of NT = 2D threads handles one (request, layer, head) record at a
+// time.  Thread t owns rows [g RT, g RT + RT) x columns [4l, 4l + 4) with
+// RT = D/8, g = t / (D/4), l = t % (D/4); the packed layout stores thread t's
+// codes as its own bit stream, so its chunks come straight out of a 16-byte
+// shared-memory load.  Persistent CTAs stream records through a ring of
+// shared-memory stages filled by 1-D bulk copies (cp.async.bulk, completion
+// on an mbarrier).  Kernels:
+//   kDecode   reconstruct -> u, w -> o (readout) ; writes o and w
+//   kFitPack  reconstruct -> S_t = S' + k w^T -> refit r, c -> pack, in place
+//   kFused    both in one pass over the record
+#include "stepq_dev.cuh"
+
+namespace stepq {
+
+enum Kind { kDecode = 0, kFitPack = 1, kFused = 2 };
+
+constexpr int kStages = 3;
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: fl(x + kMagic) - kMagic = rint(x), |x| < 2^22
+constexpr double kTwoM169 = 1.0 / 748288838313422294120286634350736906063837462003712.0;  // 2^-169
+
+template <int D>
+struct Geo {
+    static constexpr int NT = 2 * D;       // threads per CTA
+    static constexpr int RT = D / 8;       // rows per thread
+    static constexpr int LANES = D / 4;    // threads across a row band
+    static constexpr int BANDS = 8;
+};
+
+template <int D, int B>
+struct Stream {
+    static constexpr int RT = D / 8;
+    static constexpr int WORDS = (RT * B + 7) / 8;  // 32-bit words of a thread stream (4 RT B bits)
+    static constexpr int NW = WORDS + 1;                                // + guard word
+    static constexpr int NCH = B / 2;                                   // chunks of RT bytes
+};
+
+// Shared memory besides the stages.
+template <int D>
+struct Scratch {
+    double pU[8][D];
+    double pO[8][D];
+    float pf0[8][D];
+    float pf1[8][D];
+    float a[D];       // a_i = fl(alpha_i r_i)  (pivot: alpha_i)
+    float kf[D];      // k_i
+    double kap[D];    // k_i a_i 2^-169   (pivot: k_i alpha_i)
+    double qt[D];     // q_i a_i 2^-169   (pivot: q_i alpha_i)
+    float rho[D];
+    float wbar[D];
+    float cpr[D];     // c_j 2^-12
+    float cold[D];    // c_j
+    float wv[D];      // w_j
+    float ic0[D];
+    float c0[D];
+    float ic[D];
+    double cst[3];    // Kc, Qc, q.k
+    double red[3][8];
+    int meta[kStages][4];  // slot, width, valid, unused
+};
+
+template <int D>
+__device__ __forceinline__ void item_coords(const Args &a, int it, int &n, int &ll, int &h, int &gl, int &row) {
+    const int per_req = a.nL * a.H;
+    n = it / per_req;
+    const int rem = it - n * per_req;
+    ll = rem / a.H;
+    h = rem - ll * a.H;
+    gl = (a.lb + ll) * a.H + h;
+    row = (n * a.nL_in + a.l_in0 + ll) * a.H + h;  // index of the (request, layer, head) input row
+}
+
+// Thread 0: stage item `it` into stage s (record + input rows), or mark it invalid.
+template <int D, int KIND>
+__device__ void issue_item(const Args &a, int it, uint8_t *stage, uint64_t *bar, int *meta) {
+    int n, ll, h, gl, row;
+    item_coords<D>(a, it, n, ll, h, gl, row);
+    const int slot = a.slots[n];
+    const bool ok = slot >= 0 && slot < a.n_slots;
+    const int width = a.t.width[gl];
+    meta[0] = slot;
+    meta[1] = width;
+    meta[2] = ok ? 1 : 0;
+    if (!ok) {
+        flag_error(a.err, kErrBadSlot);
+        mbar_arrive(bar);
+        return;
+    }
+    fence_proxy_async();
+    const uint8_t *rec = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[gl];
+    const uint32_t rec_bytes = (width == kPivotBits) ? 0u : a.t.rec_bytes[gl];
+    float *qs = reinterpret_cast<float *>(stage + a.rec_stage_bytes);
+    float *ks = qs + D;
+    float *vs = ks + D;
+    float *xs = vs + D;
+    constexpr uint32_t RB = D * 4;
+    uint32_t total = rec_bytes;
+    if (KIND != kFitPack) total += 3 * RB;
+    else total += 2 * RB;
+    mbar_arrive_expect(bar, total);
+    if (rec_bytes) bulk_g2s(stage, rec, rec_bytes, bar);
+    const size_t off = (size_t)row * D;
+    if (KIND != kFitPack) {
+        bulk_g2s(qs, a.q + off, RB, bar);
+        bulk_g2s(ks, a.k + off, RB, bar);
+        bulk_g2s(vs, a.v + off, RB, bar);
+    } else {
+        bulk_g2s(ks, a.k + off, RB, bar);
+        bulk_g2s(xs, a.w + off, RB, bar);
+    }
+}
+
+// Load thread t's code stream (NCH chunks of RT bytes) from the codes block.
+template <int D, int B>
+__device__ __forceinline__ void load_stream(const uint8_t *blk, int t, uint32_t (&W)[Stream<D, B>::NW]) {
+    constexpr int RT = D / 8, NT = 2 * D, NCH = B / 2;
+#pragma unroll
+    for (int i = 0; i < Stream<D, B>::NW; ++i) W[i] = 0u;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        const uint8_t *p = blk + (size_t)(c * NT + t) * RT;
+        if constexpr (RT == 16) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(p);
+            W[4 * c] = v.x; W[4 * c + 1] = v.y; W[4 * c + 2] = v.z; W[4 * c + 3] = v.w;
+        } else if constexpr (RT == 8) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(p);
+            W[2 * c] = v.x; W[2 * c + 1] = v.y;
+        } else if constexpr (RT == 4) {
+            W[c] = *reinterpret_cast<const uint32_t *>(p);
+        } else {
+            const uint32_t v = *reinterpret_cast<const uint16_t *>(p);
+            W[c >> 1] |= v << (16 * (c & 1));
+        }
+    }
+}
+
+template <int D, int B>
+__device__ __forceinline__ void store_stream(uint8_t *blk, int t, const uint32_t (&W)[Stream<D, B>::NW]) {
+    constexpr int RT = D / 8, NT = 2 * D, NCH = B / 2;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        uint8_t *p = blk + (size_t)(c * NT + t) * RT;
+        if constexpr (RT == 16) {
+            *reinterpret_cast<uint4 *>(p) = make_uint4(W[4 * c], W[4 * c + 1], W[4 * c + 2], W[4 * c + 3]);
+        } else if constexpr (RT == 8) {
+            *reinterpret_cast<uint2 *>(p) = make_uint2(W[2 * c], W[2 * c + 1]);
+        } else if constexpr (RT == 4) {
+            *reinterpret_cast<uint32_t *>(p) = W[c];
+        } else {
+            *reinterpret_cast<uint16_t *>(p) = (uint16_t)(W[c >> 1] >> (16 * (c & 1)));
+        }
+    }
+}
+
+// Pairwise (balanced tree) sum of N float2 values, in index order.
+template <int N>
+__device__ __forceinline__ float2 tree_sum2(float2 (&x)[N]) {
+#pragma unroll
+    for (int s = 1; s < N; s <<= 1)
+#pragma unroll
+        for (int i = 0; i + s < N; i += 2 * s) x[i] = __fadd2_rn(x[i], x[i + s]);
+    return x[0];
+}
+
+template <int N>
+__device__ __forceinline__ float tree_sum1(float (&x)[N]) {
+#pragma unroll
+    for (int s = 1; s < N; s <<= 1)
+#pragma unroll
+        for (int i = 0; i + s < N; i += 2 * s) x[i] = x[i] + x[i + s];
+    return x[0];
+}
+
+// ---------------------------------------------------------------------------
+// Refit of the fp32 tile S held in registers (all rows at width B).  On
+// return S holds y = fl(S * fl(1/r)), rr[] the row factors of the thread's
+// rows, sc.ic[j] = fl(1/c_j) and sc.cold[j] = c_j.  Requires rho and wbar of
+// the head in sc.rho / sc.wbar.
+// ---------------------------------------------------------------------------
+template <int D, int B>
+__device__ void fit_scales(float (&S)[D / 8][4], float (&rr)[D / 8], Scratch<D> &sc, int tid) {
+    using G = Geo<D>;
+    constexpr int RT = G::RT, LANES = G::LANES;
+    constexpr int Q = (1 << (B - 1)) - 1;
+    const int g = tid / LANES, l = tid % LANES;
+    const int j0 = 4 * l;
+
+    // 1. row factors: r_i = fl(max(pairwise_j |S_ij| / D, 1e-12) rho_i)
+    float inv_r[RT], bw[RT];
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+        const int i = g * RT + r;
+        float s = (fabsf(S[r][0]) + fabsf(S[r][1])) + (fabsf(S[r][2]) + fabsf(S[r][3]));
+        s = lane_pairwise_sum<LANES>(s);
+        float m = __fmul_rn(s, 1.0f / (float)D);
+        m = fmaxf(m, 1e-12f);
+        const float ri = __fmul_rn(m, sc.rho[i]);
+        rr[r] = ri;
+        inv_r[r] = __frcp_rn(ri);
+        bw[r] = __fmul_rn(sc.wbar[i], __fmul_rn(ri, ri));
+    }
+    // 2. y = fl(S * (1/r)) in place
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+        const float2 ir = make_float2(inv_r[r], inv_r[r]);
+        const float2 a01 = __fmul2_rn(make_float2(S[r][0], S[r][1]), ir);
+        const float2 a23 = __fmul2_rn(make_float2(S[r][2], S[r][3]), ir);
+        S[r][0] = a01.x; S[r][1] = a01.y; S[r][2] = a23.x; S[r][3] = a23.y;
+    }
+    // 3. column absmax -> c0
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+        float m = 0.0f;
+#pragma unroll
+        for (int r = 0; r < RT; ++r) m = fmaxf(m, fabsf(S[r][jj]));
+        sc.pf0[g][j0 + jj] = m;
+    }
+    __syncthreads();
+    if (tid < D) {
+        float m = 0.0f;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) m = fmaxf(m, sc.pf0[b][tid]);
+        const float c0 = (m == 0.0f) ? 1.0f : __fdiv_rn(m, (float)Q);
+        sc.c0[tid] = c0;
+        sc.ic0[tid] = __frcp_rn(c0);
+    }
+    __syncthreads();
+    // 4. z0 and the weighted least-squares sums (pairwise over rows)
+    {
+        const float2 mg = make_float2(kMagic, kMagic);
+        const float2 nmg = make_float2(-kMagic, -kMagic);
+#pragma unroll
+        for (int hp = 0; hp < 2; ++hp) {
+            const int jA = j0 + 2 * hp;
+            const float2 ic = make_float2(sc.ic0[jA], sc.ic0[jA + 1]);
+            float2 tn[RT], td[RT];
+#pragma unroll
+            for (int r = 0; r < RT; ++r) {
+                const float2 y = make_float2(S[r][2 * hp], S[r][2 * hp + 1]);
+                const float2 t = __ffma2_rn(y, ic, mg);
+                const float2 z0 = __fadd2_rn(t, nmg);
+                const float2 b2 = make_float2(bw[r], bw[r]);
+                tn[r] = __fmul2_rn(b2, __fmul2_rn(z0, y));
+                td[r] = __fmul2_rn(b2, __fmul2_rn(z0, z0));
+            }
+            const float2 sn = tree_sum2<RT>(tn);
+            const float2 sd = tree_sum2<RT>(td);
+            sc.pf0[g][jA] = sn.x; sc.pf0[g][jA + 1] = sn.y;
+            sc.pf1[g][jA] = sd.x; sc.pf1[g][jA + 1] = sd.y;
+        }
+    }
+    __syncthreads();
+    if (tid < D) {
+        float xn[8], xd[8];
+#pragma unroll
+        for (int b = 0; b < 8; ++b) { xn[b] = sc.pf0[b][tid]; xd[b] = sc.pf1[b][tid]; }
+        const float num = tree_sum1<8>(xn);
+        const float den = tree_sum1<8>(xd);
+        const float c = (den > 0.0f) ? __fdiv_rn(num, den) : sc.c0[tid];
+        sc.ic[tid] = __frcp_rn(c);
+        sc.cold[tid] = c;
+    }
+    __syncthreads();
+}
+
+// Final code of y with 1/c: the fp32 bits of kMagic + 2^(B-1) + z, z clamped
+// to [-qmax, qmax]; the low B bits are the stored field z + 2^(B-1).
+template <int B>
+__device__ __forceinline__ int2 final_codes(float2 y, float2 ic) {
+    constexpr int Q = (1 << (B - 1)) - 1;
+    constexpr int OFF = 1 << (B - 1);
+    constexpr float MG2 = kMagic + (float)OFF;
+    constexpr int LO = 0x4B400000 + OFF - Q;
+    constexpr int HI = 0x4B400000 + OFF + Q;
+    const float2 t = __ffma2_rn(y, ic, make_float2(MG2, MG2));
+    int T0 = __float_as_int(t.x), T1 = __float_as_int(t.y);
+    T0 = min(max(T0, LO), HI);
+    T1 = min(max(T1, LO), HI);
+    return make_int2(T0, T1);
+}
+
+// Refit and pack into the record at `rec` (global): codes, r, c.
+template <int D, int B>
+__device__ void fit_pack(float (&S)[D / 8][4], uint8_t *rec, Scratch<D> &sc, int tid) {
+    using G = Geo<D>;
+    constexpr int RT = G::RT, LANES = G::LANES;
+    const int g = tid / LANES, l = tid % LANES;
+    const int j0 = 4 * l;
+    const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
+    float *rec_r = reinterpret_cast<float *>(rec + codes_bytes);
+    float *rec_c = rec_r + D;
+    float rr[RT];
+    fit_scales<D, B>(S, rr, sc, tid);
+#pragma unroll
+    for (int r = 0; r < RT; ++r)
+        if (l == (r % LANES)) rec_r[g * RT + r] = rr[r];
+    if (tid < D) rec_c[tid] = sc.cold[tid];
+    uint32_t W[Stream<D, B>::NW];
+#pragma unroll
+    for (int i = 0; i < Stream<D, B>::NW; ++i) W[i] = 0u;
+#pragma unroll
+    for (int hp = 0; hp < 2; ++hp) {
+        const int jA = j0 + 2 * hp;
+        const float2 ic = make_float2(sc.ic[jA], sc.ic[jA + 1]);
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            const int2 T = final_codes<B>(make_float2(S[r][2 * hp], S[r][2 * hp + 1]), ic);
+            field_put<B>(W, 4 * r + 2 * hp, (uint32_t)T.x & ((1u << B) - 1u));
+            field_put<B>(W, 4 * r + 2 * hp + 1, (uint32_t)T.y & ((1u << B) - 1u));
+        }
+    }
+    store_stream<D, B>(rec, tid, W);
+}
+
+// Pivot head (binary16 tile): S_t -> fp16 RNE, written in place.
+template <int D>
+__device__ __forceinline__ void store_pivot(float (&S)[D / 8][4], uint8_t *rec, int tid) {
+    using G = Geo<D>;
+    const int g = tid / G::LANES, l = tid % G::LANES;
+#pragma unroll
+    for (int r = 0; r < G::RT; ++r) {
+        const int i = g * G::RT + r;
+        const __half2 h01 = __floats2half2_rn(S[r][0], S[r][1]);
+        const __half2 h23 = __floats2half2_rn(S[r][2], S[r][3]);
+        uint2 v;
+        v.x = *reinterpret_cast<const uint32_t *>(&h01);
+        v.y = *reinterpret_cast<const uint32_t *>(&h23);
+        *reinterpret_cast<uint2 *>(rec + ((size_t)i * D + 4 * l) * 2) = v;
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void load_pivot(const uint8_t *rec, int tid, float (&h)[D / 8][4]) {
+    using G = Geo<D>;
+    const int g = tid / G::LANES, l = tid % G::LANES;
+#pragma unroll
+    for (int r = 0; r < G::RT; ++r) {
+        const int i = g * G::RT + r;
+        const uint2 v = *reinterpret_cast<const uint2 *>(rec + ((size_t)i * D + 4 * l) * 2);
+        const __half2 h01 = *reinterpret_cast<const __half2 *>(&v.x);
+        const __half2 h23 = *reinterpret_cast<const __half2 *>(&v.y);
+        const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+        h[r][0] = f01.x; h[r][1] = f01.y; h[r][2] = f23.x; h[r][3] = f23.y;
+    }
+}
+
+// Block-wide fp64 sums of three values (every thread passes its share, 0 if none).
+template <int D>
+__device__ __forceinline__ void block_sum3(Scratch<D> &sc, int tid, double x0, double x1, double x2) {
+    constexpr int NWP = (2 * D) / 32;
+    x0 = lane_sum_f64<32>(x0);
+    x1 = lane_sum_f64<32>(x1);
+    x2 = lane_sum_f64<32>(x2);
+    if ((tid & 31) == 0) {
+        sc.red[0][tid >> 5] = x0;
+        sc.red[1][tid >> 5] = x1;
+        sc.red[2][tid >> 5] = x2;
+    }
+    __syncthreads();
+    if (tid < 3) {
+        double s = 0.0;
+        for (int w = 0; w < NWP; ++w) s += sc.red[tid][w];
+        sc.cst[tid] = s;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// One quantized head of width B: decode / fit-pack / fused.
+// ---------------------------------------------------------------------------
+template <int D, int B, int KIND>
+__device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int row, int gl,
+                             Scratch<D> &sc, int tid) {
+    using G = Geo<D>;
+    constexpr int RT = G::RT, LANES = G::LANES;
+    constexpr int OFF = 1 << (B - 1);
+    const int g = tid / LANES, l = tid % LANES;
+    const int j0 = 4 * l;
+    const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
+    const float *st_r = reinterpret_cast<const float *>(stage + codes_bytes);
+    const float *st_c = st_r + D;
+    const float *qs = reinterpret_cast<const float *>(stage + a.rec_stage_bytes);
+    const float *ks = qs + D;
+    const float *vs = ks + D;
+    const float *xs = vs + D;
+    const float alpha = a.alpha[row];
+    const float beta = a.beta[row];
+
+    // per-row and per-column parameters
+    if (tid < D) {
+        const int i = tid;
+        const float ai = __fmul_rn(alpha, st_r[i]);
+        sc.a[i] = ai;
+        sc.kf[i] = ks[i];
+        sc.cpr[i] = __fmul_rn(st_c[i], 1.0f / 4096.0f);
+        sc.cold[i] = st_c[i];
+        if (KIND != kDecode) {
+            sc.rho[i] = a.t.rho[(size_t)gl * D + i];
+            sc.wbar[i] = a.t.wbar[(size_t)gl * D + i];
+        }
+        if (KIND == kFitPack) sc.wv[i] = xs[i];
+    }
+    if (KIND != kFitPack) {
+        double kc = 0.0, qc = 0.0, qk = 0.0;
+        if (tid < D) {
+            const int i = tid;
+            const double ka = (double)ks[i] * (double)sc.a[i];
+            const double qa = (double)qs[i] * (double)sc.a[i];
+            sc.kap[i] = ka * kTwoM169;
+            sc.qt[i] = qa * kTwoM169;
+            kc = ka * (double)(256 + OFF);
+            qc = qa * (double)(256 + OFF);
+            qk = (double)qs[i] * (double)ks[i];
+        }
+        block_sum3<D>(sc, tid, kc, qc, qk);
+    }
+    __syncthreads();
+
+    uint32_t W[Stream<D, B>::NW];
+    load_stream<D, B>(stage, tid, W);
+
+    float S[RT][4];
+    double accU[4] = {0.0, 0.0, 0.0, 0.0}, accO[4] = {0.0, 0.0, 0.0, 0.0};
+    float2 cp01, cp23;
+    if (KIND != kDecode) {
+        cp01 = make_float2(sc.cpr[j0], sc.cpr[j0 + 1]);
+        cp23 = make_float2(sc.cpr[j0 + 2], sc.cpr[j0 + 3]);
+    }
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+        const int i = g * RT + r;
+        uint32_t X[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) X[jj] = field_x<B>(W, 4 * r + jj);
+        if (KIND != kFitPack) {
+            const double kap = sc.kap[i], qt = sc.qt[i];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const double d = x_as_f64(X[jj]);
+                accU[jj] = fma(kap, d, accU[jj]);
+                accO[jj] = fma(qt, d, accO[jj]);
+            }
+        }
+        if (KIND != kDecode) {
+            const float ai = sc.a[i];
+            const float2 a2 = make_float2(ai, ai);
+            const float2 A01 = __fmul2_rn(a2, cp01);
+            const float2 A23 = __fmul2_rn(a2, cp23);
+            const float2 z01 = make_float2(x_as_zscaled<B>(X[0]), x_as_zscaled<B>(X[1]));
+            const float2 z23 = make_float2(x_as_zscaled<B>(X[2]), x_as_zscaled<B>(X[3]));
+            const float2 s01 = __fmul2_rn(A01, z01);
+            const float2 s23 = __fmul2_rn(A23, z23);
+            S[r][0] = s01.x; S[r][1] = s01.y; S[r][2] = s23.x; S[r][3] = s23.y;
+        }
+    }
+
+    if (KIND != kFitPack) {
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            sc.pU[g][j0 + jj] = accU[jj];
+            sc.pO[g][j0 + jj] = accO[jj];
+        }
+        __syncthreads();
+        if (tid < D) {
+            const int j = tid;
+            double su = 0.0, so = 0.0;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) { su += sc.pU[b][j]; so += sc.pO[b][j]; }
+            const double cj = (double)sc.cold[j];
+            const float u = __double2float_rn(cj * (su - sc.cst[0]));
+            const float w = __fmul_rn(beta, __fsub_rn(vs[j], u));
+            const float o = __double2float_rn(cj * (so - sc.cst[1]) + sc.cst[2] * (double)w);
+            a.o[(size_t)row * D + j] = o;
+            if (KIND == kDecode) a.w[(size_t)row * D + j] = w;
+            else sc.wv[j] = w;
+        }
+        if (KIND == kFused) __syncthreads();
+    }
+
+    if (KIND != kDecode) {
+        const float2 w01 = make_float2(sc.wv[j0], sc.wv[j0 + 1]);
+        const float2 w23 = make_float2(sc.wv[j0 + 2], sc.wv[j0 + 3]);
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            const float ki = sc.kf[g * RT + r];
+            const float2 k2 = make_float2(ki, ki);
+            const float2 s01 = __ffma2_rn(k2, w01, make_float2(S[r][0], S[r][1]));
+            const float2 s23 = __ffma2_rn(k2, w23, make_float2(S[r][2], S[r][3]));
+            S[r][0] = s01.x; S[r][1] = s01.y; S[r][2] = s23.x; S[r][3] = s23.y;
+        }
+        fit_pack<D, B>(S, rec_g, sc, tid);
+    }
+}
+
+// One FP16 pivot head.
+template <int D, int KIND>
+__device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int row, Scratch<D> &sc, int tid) {
+    using G = Geo<D>;
+    constexpr int RT = G::RT, LANES = G::LANES;
+    const int g = tid / LANES, l = tid % LANES;
+    const int j0 = 4 * l;
+    const float *qs = reinterpret_cast<const float *>(stage + a.rec_stage_bytes);
+    const float *ks = qs + D;
+    const float *vs = ks + D;
+    const float *xs = vs + D;
+    const float alpha = a.alpha[row];
+    const float beta = a.beta[row];
+    if (tid < D) {
+        sc.kf[tid] = ks[tid];
+        if (KIND == kFitPack) sc.wv[tid] = xs[tid];
+    }
+    if (KIND != kFitPack) {
+        double qk = 0.0;
+        if (tid < D) {
+            sc.kap[tid] = (double)ks[tid] * (double)alpha;
+            sc.qt[tid] = (double)qs[tid] * (double)alpha;
+            qk = (double)qs[tid] * (double)ks[tid];
+        }
+        block_sum3<D>(sc, tid, 0.0, 0.0, qk);
+    }
+    __syncthreads();
+    float S[RT][4];
+    load_pivot<D>(rec_g, tid, S);
+    if (KIND != kFitPack) {
+        double accU[4] = {0.0, 0.0, 0.0, 0.0}, accO[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            const int i = g * RT + r;
+            const double kap = sc.kap[i], qt = sc.qt[i];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const double d = (double)S[r][jj];
+                accU[jj] = fma(kap, d, accU[jj]);
+                accO[jj] = fma(qt, d, accO[jj]);
+            }
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            sc.pU[g][j0 + jj] = accU[jj];
+            sc.pO[g][j0 + jj] = accO[jj];
+        }
+        __syncthreads();
+        if (tid < D) {
+            const int j = tid;
+            double su = 0.0, so = 0.0;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) { su += sc.pU[b][j]; so += sc.pO[b][j]; }
+            const float u = __double2float_rn(su);
+            const float w = __fmul_rn(beta, __fsub_rn(vs[j], u));
+            const float o = __double2float_rn(so + sc.cst[2] * (double)w);
+            a.o[(size_t)row * D + j] = o;
+            if (KIND == kDecode) a.w[(size_t)row * D + j] = w;
+            else sc.wv[j] = w;
+        }
+        if (KIND == kFused) __syncthreads();
+    }
+    if (KIND != kDecode) {
+        const float2 al = make_float2(alpha, alpha);
+        const float2 w01 = make_float2(sc.wv[j0], sc.wv[j0 + 1]);
+        const float2 w23 = make_float2(sc.wv[j0 + 2], sc.wv[j0 + 3]);
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            const float ki = sc.kf[g * RT + r];
+            const float2 k2 = make_float2(ki, ki);
+            const float2 p01 = __fmul2_rn(al, make_float2(S[r][0], S[r][1]));
+            const float2 p23 = __fmul2_rn(al, make_float2(S[r][2], S[r][3]));
+            const float2 s01 = __ffma2_rn(k2, w01, p01);
+            const float2 s23 = __ffma2_rn(k2, w23, p23);
+            S[r][0] = s01.x; S[r][1] = s01.y; S[r][2] = s23.x; S[r][3] = s23.y;
+        }
+        store_pivot<D>(S, rec_g, tid);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Persistent pipeline kernel.
+// ---------------------------------------------------------------------------
+template <int D, int KIND>
+__global__ void __launch_bounds__(2 * D) k_step(Args a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x;
+    uint8_t *stages = smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * a.stage_bytes);
+    Scratch<D> &sc = *reinterpret_cast<Scratch<D> *>(smem + kStages * a.stage_bytes + 64);
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            const int it = blockIdx.x + s * gridDim.x;
+            if (it < a.n_items) issue_item<D, KIND>(a, it, stages + s * a.stage_bytes, &bars[s], sc.meta[s]);
+        }
+    }
+    int s = 0;
+    uint32_t phase = 0;
+    for (int it = blockIdx.x; it < a.n_items; it += gridDim.x) {
+        const bool ok = mbar_wait_bounded(&bars[s], phase);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                flag_error(a.err, kErrWait);
+                // let every copy still in flight land before shared memory goes away
+                for (int k = 0; k < kStages; ++k) mbar_wait_bounded(&bars[k], phase ^ (k < s ? 1u : 0u), 1u << 20);
+            }
+            return;
+        }
+        uint8_t *stage = stages + s * a.stage_bytes;
+        const int slot = sc.meta[s][0];
+        const int width = sc.meta[s][1];
+        const int valid = sc.meta[s][2];
+        if (valid) {
+            int n, ll, h, gl, row;
+            item_coords<D>(a, it, n, ll, h, gl, row);
+            uint8_t *rec_g = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[gl];
+            switch (width) {
+                case 2: item_uniform<D, 2, KIND>(a, stage, rec_g, row, gl, sc, tid); break;
+                case 4: item_uniform<D, 4, KIND>(a, stage, rec_g, row, gl, sc, tid); break;
+                case 6: item_uniform<D, 6, KIND>(a, stage, rec_g, row, gl, sc, tid); break;
+                case 8: item_uniform<D, 8, KIND>(a, stage, rec_g, row, gl, sc, tid); break;
+                case kPivotBits: item_pivot<D, KIND>(a, stage, rec_g, row, sc, tid); break;
+                default: if (tid == 0) flag_error(a.err, kErrArgs); break;
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {
+            const int nx = it + kStages * gridDim.x;
+            if (nx < a.n_items) issue_item<D, KIND>(a, nx, stage, &bars[s], sc.meta[s]);
+        }
+        if (++s == kStages) { s = 0; phase ^= 1u; }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Pack fp32 states (S_0) and unpack records: one CTA per head, no pipeline.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(2 * D) k_requant_pack(Args a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    Scratch<D> &sc = *reinterpret_cast<Scratch<D> *>(smem);
+    using G = Geo<D>;
+    const int tid = threadIdx.x;
+    const int g = tid / G::LANES, l = tid % G::LANES;
+    const int it = blockIdx.x;
+    int n, ll, h, gl, row;
+    item_coords<D>(a, it, n, ll, h, gl, row);
+    const int slot = a.slots[n];
+    if (slot < 0 || slot >= a.n_slots) {
+        if (tid == 0) flag_error(a.err, kErrBadSlot);
+        return;
+    }
+    uint8_t *rec = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[gl];
+    const float *Sg = a.S_in + (size_t)row * D * D;
+    float S[G::RT][4];
+#pragma unroll
+    for (int r = 0; r < G::RT; ++r) {
+        const float4 v = *reinterpret_cast<const float4 *>(Sg + (size_t)(g * G::RT + r) * D + 4 * l);
+        S[r][0] = v.x; S[r][1] = v.y; S[r][2] = v.z; S[r][3] = v.w;
+    }
+    const int width = a.t.width[gl];
+    if (width == kPivotBits) {
+        store_pivot<D>(S, rec, tid);
+        return;
+    }
+    if (tid < D) {
+        sc.rho[tid] = a.t.rho[(size_t)gl * D + tid];
+        sc.wbar[tid] = a.t.wbar[(size_t)gl * D + tid];
+    }
+    __syncthreads();
+    switch (width) {
+        case 2: fit_pack<D, 2>(S, rec, sc, tid); break;
+        case 4: fit_pack<D, 4>(S, rec, sc, tid); break;
+        case 6: fit_pack<D, 6>(S, rec, sc, tid); break;
+        case 8: fit_pack<D, 8>(S, rec, sc, tid); break;
+        default: if (tid == 0) flag_error(a.err, kErrArgs); break;
+    }
+}
+
+template <int D, int B>
+__device__ void unpack_uniform(const uint8_t *rec, float *out, int tid) {
+    using G = Geo<D>;
+    const int g = tid / G::LANES, l = tid % G::LANES;
+    const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
+    const float *rr = reinterpret_cast<const float *>(rec + codes_bytes);
+    const float *cc = rr + D;
+    uint32_t W[Stream<D, B>::NW];
+    load_stream<D, B>(rec, tid, W);
+    const float2 c01 = make_float2(__fmul_rn(cc[4 * l], 1.0f / 4096.0f), __fmul_rn(cc[4 * l + 1], 1.0f / 4096.0f));
+    const float2 c23 = make_float2(__fmul_rn(cc[4 * l + 2], 1.0f / 4096.0f), __fmul_rn(cc[4 * l + 3], 1.0f / 4096.0f));
+#pragma unroll
+    for (int r = 0; r < G::RT; ++r) {
+        const int i = g * G::RT + r;
+        const float ri = rr[i];
+        const float2 r2 = make_float2(ri, ri);
+        const float2 A01 = __fmul2_rn(r2, c01), A23 = __fmul2_rn(r2, c23);
+        const float2 z01 = make_float2(x_as_zscaled<B>(field_x<B>(W, 4 * r)), x_as_zscaled<B>(field_x<B>(W, 4 * r + 1)));
+        const float2 z23 = make_float2(x_as_zscaled<B>(field_x<B>(W, 4 * r + 2)), x_as_zscaled<B>(field_x<B>(W, 4 * r + 3)));
+        const float2 s01 = __fmul2_rn(A01, z01), s23 = __fmul2_rn(A23, z23);
+        *reinterpret_cast<float4 *>(out + (size_t)i * D + 4 * l) = make_float4(s01.x, s01.y, s23.x, s23.y);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(2 * D) k_unpack(Args a) {
+    using G = Geo<D>;
+    const int tid = threadIdx.x;
+    const int it = blockIdx.x;
+    int n, ll, h, gl, row;
+    item_coords<D>(a, it, n, ll, h, gl, row);
+    const int slot = a.slots[n];
+    if (slot < 0 || slot >= a.n_slots) {
+        if (tid == 0) flag_error(a.err, kErrBadSlot);
+        return;
+    }
+    const uint8_t *rec = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[gl];
+    float *out = a.S_out + (size_t)row * D * D;
+    switch (a.t.width[gl]) {
+        case 2: unpack_uniform<D, 2>(rec, out, tid); break;
+        case 4: unpack_uniform<D, 4>(rec, out, tid); break;
+        case 6: unpack_uniform<D, 6>(rec, out, tid); break;
+        case 8: unpack_uniform<D, 8>(rec, out, tid); break;
+        case kPivotBits: {
+            float S[G::RT][4];
+            load_pivot<D>(rec, tid, S);
+            const int g = tid / G::LANES, l = tid % G::LANES;
+#pragma unroll
+            for (int r = 0; r < G::RT; ++r)
+                *reinterpret_cast<float4 *>(out + (size_t)(g * G::RT + r) * D + 4 * l) =
+                    make_float4(S[r][0], S[r][1], S[r][2], S[r][3]);
+            break;
+        }
+        default: if (tid == 0) flag_error(a.err, kErrArgs); break;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Calibration distortion d_u(b) (方法-1): squared reconstruction error per key
+// row when the whole head is quantized at uniform width B, accumulated into
+// dist_acc[(gl*D + i)*n_bits + m].  Row weights: wbar from the calibration,
+// rho_i = fl32(1/sqrt(sqrt(wbar_i))) (fp64).  One CTA per (item, width).
+// ---------------------------------------------------------------------------
+struct BitList {
+    int b[4];
+    int n;
+};
+
+template <int D, int B>
+__device__ void dist_uniform(const float *Sg, int gl, int m, int n_bits, double *dist_acc, Scratch<D> &sc, int tid) {
+    using G = Geo<D>;
+    constexpr int RT = G::RT, LANES = G::LANES;
+    constexpr int OFF = 1 << (B - 1);
+    const int g = tid / LANES, l = tid % LANES;
+    const int j0 = 4 * l;
+    float S[RT][4];
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+        const float4 v = *reinterpret_cast<const float4 *>(Sg + (size_t)(g * RT + r) * D + j0);
+        S[r][0] = v.x; S[r][1] = v.y; S[r][2] = v.z; S[r][3] = v.w;
+    }
+    float rr[RT];
+    fit_scales<D, B>(S, rr, sc, tid);
+    const float c0 = sc.cold[j0], c1 = sc.cold[j0 + 1], c2 = sc.cold[j0 + 2], c3 = sc.cold[j0 + 3];
+    const float2 ic01 = make_float2(sc.ic[j0], sc.ic[j0 + 1]);
+    const float2 ic23 = make_float2(sc.ic[j0 + 2], sc.ic[j0 + 3]);
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+        const int i = g * RT + r;
+        const int2 T01 = final_codes<B>(make_float2(S[r][0], S[r][1]), ic01);
+        const int2 T23 = final_codes<B>(make_float2(S[r][2], S[r][3]), ic23);
+        const int zb = 0x4B400000 + OFF;
+        const float z[4] = {(float)(T01.x - zb), (float)(T01.y - zb), (float)(T23.x - zb), (float)(T23.y - zb)};
+        const float cc[4] = {c0, c1, c2, c3};
+        const float4 orig = *reinterpret_cast<const float4 *>(Sg + (size_t)i * D + j0);
+        const float o4[4] = {orig.x, orig.y, orig.z, orig.w};
+        double e = 0.0;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const float sh = __fmul_rn(__fmul_rn(rr[r], cc[jj]), z[jj]);
+            const double d = (double)sh - (double)o4[jj];
+            e = fma(d, d, e);
+        }
+        e = lane_sum_f64<LANES>(e);
+        if (l == (r % LANES)) atomicAdd(&dist_acc[((size_t)gl * D + i) * n_bits + m], e);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(2 * D) k_calib_dist(Args a, BitList bl, double *dist_acc) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    Scratch<D> &sc = *reinterpret_cast<Scratch<D> *>(smem);
+    const int tid = threadIdx.x;
+    const int it = blockIdx.x;
+    const int m = blockIdx.y;
+    int n, ll, h, gl, row;
+    item_coords<D>(a, it, n, ll, h, gl, row);
+    if (tid < D) {
+        const float wb = a.t.wbar[(size_t)gl * D + tid];
+        sc.wbar[tid] = wb;
+        sc.rho[tid] = (float)(1.0 / sqrt(sqrt((double)wb)));
+    }
+    __syncthreads();
+    const float *Sg = a.S_in + (size_t)row * D * D;
+    switch (bl.b[m]) {
+        case 2: dist_uniform<D, 2>(Sg, gl, m, bl.n, dist_acc, sc, tid); break;
+        case 4: dist_uniform<D, 4>(Sg, gl, m, bl.n, dist_acc, sc, tid); break;
+        case 6: dist_uniform<D, 6>(Sg, gl, m, bl.n, dist_acc, sc, tid); break;
+        case 8: dist_uniform<D, 8>(Sg, gl, m, bl.n, dist_acc, sc, tid); break;
+        default: if (tid == 0) flag_error(a.err, kErrArgs); break;
+    }
+}
+
+template <int D>
+static cudaError_t launch_dist_d(const Args &a, const BitList &bl, double *acc, cudaStream_t st) {
+    if (a.n_items <= 0) return cudaSuccess;
+    const size_t smem = sizeof(Scratch<D>);
+    cudaError_t e = cudaFuncSetAttribute(k_calib_dist<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k_calib_dist<D><<<dim3(a.n_items, bl.n), 2 * D, smem, st>>>(a, bl, acc);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_calib_dist(int D, const Args &a, const int *bits, int n_bits, double *acc, cudaStream_t st) {
+    BitList bl{};
+    if (n_bits < 1 || n_bits > 4) return cudaErrorInvalidValue;
+    for (int i = 0; i < n_bits; ++i) bl.b[i] = bits[i];
+    bl.n = n_bits;
+    switch (D) {
+        case 16: return launch_dist_d<16>(a, bl, acc, st);
+        case 32: return launch_dist_d<32>(a, bl, acc, st);
+        case 64: return launch_dist_d<64>(a, bl, acc, st);
+        case 128: return launch_dist_d<128>(a, bl, acc, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (called by the C ABI in stepq_api.cpp).
+// ---------------------------------------------------------------------------
+template <int D>
+static size_t step_smem(uint32_t stage_bytes) {
+    return (size_t)kStages * stage_bytes + 64 + sizeof(Scratch<D>);
+}
+
+template <int D, int KIND>
+static cudaError_t launch_step_d(Args a, int n_sms, cudaStream_t st, int *grid_out) {
+    const size_t smem = step_smem<D>(a.stage_bytes);
+    auto kern = k_step<D, KIND>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 2 * D, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    int grid = n_sms * per_sm;
+    if (grid > a.n_items) grid = a.n_items;
+    if (grid_out) *grid_out = grid;
+    if (grid <= 0) return cudaSuccess;
+    kern<<<grid, 2 * D, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <int KIND>
+static cudaError_t launch_step_kind(int D, Args a, int n_sms, cudaStream_t st, int *grid) {
+    switch (D) {
+        case 16: return launch_step_d<16, KIND>(a, n_sms, st, grid);
+        case 32: return launch_step_d<32, KIND>(a, n_sms, st, grid);
+        case 64: return launch_step_d<64, KIND>(a, n_sms, st, grid);
+        case 128: return launch_step_d<128, KIND>(a, n_sms, st, grid);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_step(int kind, int D, const Args &a, int n_sms, cudaStream_t st, int *grid) {
+    switch (kind) {
+        case kDecode: return launch_step_kind<kDecode>(D, a, n_sms, st, grid);
+        case kFitPack: return launch_step_kind<kFitPack>(D, a, n_sms, st, grid);
+        case kFused: return launch_step_kind<kFused>(D, a, n_sms, st, grid);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int D>
+static cudaError_t launch_pack_d(const Args &a, bool unpack, cudaStream_t st) {
+    if (a.n_items <= 0) return cudaSuccess;
+    if (unpack) {
+        k_unpack<D><<<a.n_items, 2 * D, 0, st>>>(a);
+    } else {
+        const size_t smem = sizeof(Scratch<D>);
+        cudaError_t e = cudaFuncSetAttribute(k_requant_pack<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        k_requant_pack<D><<<a.n_items, 2 * D, smem, st>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack(int D, const Args &a, bool unpack, cudaStream_t st) {
+    switch (D) {
+        case 16: return launch_pack_d<16>(a, unpack, st);
+        case 32: return launch_pack_d<32>(a, unpack, st);
+        case 64: return launch_pack_d<64>(a, unpack, st);
+        case 128: return launch_pack_d<128>(a, unpack, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace stepq

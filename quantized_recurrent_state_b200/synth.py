@@ -113,6 +113,48 @@ def normal_torch(key: int, shape, device, start: int = 0):
     return out[:n].reshape(shape)
 
 
+def uniform_torch(key: int, shape, device):
+    """Same stream as uniform_np, on a device."""
+    import torch
+    n = int(np.prod(shape))
+    idx = torch.arange(1, n + 1, dtype=torch.int64, device=device)
+
+    def srl(x, s):
+        return (x >> s) & ((1 << (64 - s)) - 1)
+
+    z = _to_i64(key) + idx * _to_i64(GOLDEN)
+    z = (z ^ srl(z, 30)) * _to_i64(M1)
+    z = (z ^ srl(z, 27)) * _to_i64(M2)
+    z = z ^ srl(z, 31)
+    return (srl(z, 11).to(torch.float64) * 2.0 ** -53).reshape(shape)
+
+
+def initial_states_torch(wl: "Workload", seed: int, n_req: int, layer: int, device):
+    """S_0 of one layer, [n_req, 1, H, D, D] float32, on a device (same recipe)."""
+    import torch
+    gam = torch.from_numpy(column_scales(wl, seed)[layer]).to(device)
+    rsc = torch.from_numpy(row_scales(wl, seed)[layer]).to(device)
+    G = normal_torch(stream_key(seed, S_G, layer), (n_req, wl.n_heads, wl.d, wl.d), device)
+    S = G * rsc[None, :, :, None].double() * gam[None, :, None, :].double()
+    return S.float().unsqueeze(1).contiguous()
+
+
+def step_inputs_torch(wl: "Workload", seed: int, n_req: int, t: int, alpha: np.ndarray, device) -> dict:
+    """step_inputs for all layers, generated on a device (same recipe and streams)."""
+    import torch
+    shape = (n_req, wl.n_layers, wl.n_heads, wl.d)
+    q = normal_torch(stream_key(seed, S_Q, t), shape, device)
+    n = normal_torch(stream_key(seed, S_K, t), shape, device)
+    k = n / torch.sqrt((n * n).sum(dim=-1, keepdim=True))
+    gam = torch.from_numpy(column_scales(wl, seed)).to(device).double()
+    v = normal_torch(stream_key(seed, S_V, t), shape, device) * gam[None]
+    beta = uniform_torch(stream_key(seed, S_BETA, t), (n_req, wl.n_layers, wl.n_heads), device)
+    al = torch.from_numpy(np.ascontiguousarray(alpha)).to(device)
+    al = al.unsqueeze(0).expand((n_req,) + tuple(al.shape)).contiguous()
+    return dict(q=q.float().contiguous(), k=k.float().contiguous(), v=v.float().contiguous(),
+                alpha=al.float().contiguous(), beta=beta.float().contiguous())
+
+
 # ---- workloads -------------------------------------------------------------
 
 @dataclass

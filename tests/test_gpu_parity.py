@@ -1,0 +1,314 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Lockstep protocol: at every step the oracle starts from the records the GPU
+holds, so one excused rounding tie cannot propagate.  Packed codes must be
+bit-exact except codes whose oracle pre-rounding value lies within 1e-6
+relative of a .5 boundary (or whose column's initial codes had such a tie);
+those are counted and must stay <= 1e-5 of all codes.  Readouts must satisfy
+|o_gpu - o_ref| <= 1e-5 + 1e-4 |o_ref|.
+"""
+import numpy as np
+import pytest
+
+from oracle import core, model
+from quantized_recurrent_state_b200 import synth
+from tests._workloads import compare_records, oracle_plan
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+RTOL, ATOL = 1e-4, 1e-5
+
+
+@pytest.fixture(scope="module")
+def stepq():
+    from quantized_recurrent_state_b200 import build as qbuild
+    qbuild.build()
+    from quantized_recurrent_state_b200 import stepq as s
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return s
+
+
+def _close(g, r):
+    return np.abs(g - r) <= ATOL + RTOL * np.abs(r)
+
+
+def _inputs_to_dev(inp):
+    return {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in inp.items()}
+
+
+class Run:
+    """A GPU pool for a workload plus an oracle view of the same plan."""
+
+    def __init__(self, stepq, name, n_req, n_layers=None, n_pivots=None, extra_slots=3, chunk=2):
+        self.plan, data, self.wl, _ = oracle_plan(name, n_layers, n_pivots)
+        self.pv = model.PlanView(self.plan)
+        self.P = stepq.Plan.from_bytes(data)
+        self.n_req = n_req
+        self.n_slots = n_req + extra_slots
+        rng = np.random.default_rng(7)
+        self.slots = rng.permutation(self.n_slots)[:n_req].astype(np.int32)
+        self.slots_t = torch.from_numpy(self.slots).cuda()
+        self.ctx = stepq.Context(self.P, self.n_slots, chunk_layers=chunk)
+        self.pool = torch.zeros(self.n_slots * self.P.slot_bytes, dtype=torch.uint8, device="cuda")
+        self.L = self.wl.n_layers
+        self.alpha = synth.gates(self.wl, self.wl.seed)
+
+    def slot_bytes_host(self, n):
+        sb = self.P.slot_bytes
+        s = int(self.slots[n])
+        return self.pool[s * sb:(s + 1) * sb].cpu().numpy()
+
+    def pack_initial(self):
+        S0 = synth.initial_states(self.wl, self.wl.seed, self.n_req)
+        self.ctx.requant_pack(self.pool, self.slots_t, self.n_req, 0, self.L, torch.from_numpy(S0).cuda())
+        self.ctx.sync()
+        return S0
+
+    def step(self, t, fused=False, ws=None):
+        inp = synth.step_inputs(self.wl, self.wl.seed, self.n_req, t, alpha=self.alpha)
+        d = _inputs_to_dev(inp)
+        o = torch.zeros_like(d["q"])
+        if fused:
+            self.ctx.decode_step_fused(self.pool, self.slots_t, self.n_req, 0, self.L, d["q"], d["k"], d["v"],
+                                       d["alpha"], d["beta"], o)
+        else:
+            if ws is None:
+                ws = torch.empty(self.ctx.workspace_bytes(self.n_req, self.L) // 4, dtype=torch.float32,
+                                 device="cuda")
+            self.ctx.decode_step(self.pool, self.slots_t, self.n_req, 0, self.L, d["q"], d["k"], d["v"],
+                                 d["alpha"], d["beta"], o, ws)
+        self.ctx.sync()
+        return inp, o.cpu().numpy()
+
+
+def _lockstep(stepq, name, n_req, steps, check, n_layers=None, n_pivots=None, fused=False, heads=None):
+    run = Run(stepq, name, n_req, n_layers, n_pivots)
+    S0 = run.pack_initial()
+    pv = run.pv
+    tot_codes = tot_exc = tot_bad = 0
+    # packing of S_0
+    for n in check:
+        g = run.slot_bytes_host(n)
+        ora = np.zeros_like(g)
+        ties = {}
+        for l in range(pv.L):
+            for h in range(pv.H):
+                if heads is not None and h not in heads:
+                    continue
+                ties[(l, h)] = pv.quantize_into(ora, l, h, S0[n, l, h])
+        c, e, b, _ = compare_records(pv, g, ora, ties)
+        tot_codes += c; tot_exc += e; tot_bad += b
+    assert tot_bad == 0
+    worst_o = 0.0
+    for t in range(steps):
+        prev = {n: run.slot_bytes_host(n) for n in check}
+        inp, o = run.step(t, fused=fused)
+        for n in check:
+            g = run.slot_bytes_host(n)
+            ora = prev[n].copy()
+            ties = {}
+            for l in range(pv.L):
+                for h in range(pv.H):
+                    if heads is not None and h not in heads:
+                        continue
+                    o_ref, tie, S, w = pv.step(ora, l, h, inp["q"][n, l, h], inp["k"][n, l, h], inp["v"][n, l, h],
+                                               inp["alpha"][n, l, h], inp["beta"][n, l, h])
+                    ties[(l, h)] = tie
+                    ok = _close(o[n, l, h], o_ref)
+                    assert ok.all(), (t, n, l, h, np.max(np.abs(o[n, l, h] - o_ref)))
+                    worst_o = max(worst_o, float(np.max(np.abs(o[n, l, h] - o_ref) / (ATOL + RTOL * np.abs(o_ref)))))
+            c, e, b, _ = compare_records(pv, g, ora, ties)
+            tot_codes += c; tot_exc += e; tot_bad += b
+            assert b == 0, (t, n, b)
+    print(f"{name}: codes {tot_codes}, tie-excused {tot_exc}, bad {tot_bad}, worst o/tol {worst_o:.3g}")
+    assert tot_exc <= 1e-5 * tot_codes
+    return run
+
+
+def test_tiny_gdn_pack_and_unpack(stepq):
+    run = Run(stepq, "tiny_gdn", 1)
+    S0 = run.pack_initial()
+    pv = run.pv
+    g = run.slot_bytes_host(0)
+    ora = np.zeros_like(g)
+    for h in range(pv.H):
+        pv.quantize_into(ora, 0, h, S0[0, 0, h])
+    assert np.array_equal(g, ora)
+    Sh = torch.zeros((1, 1, pv.H, pv.D, pv.D), dtype=torch.float32, device="cuda")
+    run.ctx.unpack(run.pool, run.slots_t, 1, 0, 1, Sh)
+    run.ctx.sync()
+    Sh = Sh.cpu().numpy()
+    for h in range(pv.H):
+        assert np.array_equal(Sh[0, 0, h], pv.reconstruct(ora, 0, h))
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_tiny_gdn_lockstep_32_steps(stepq, fused):
+    _lockstep(stepq, "tiny_gdn", 1, 32, check=[0], fused=fused)
+
+
+def test_qwen_layer_lockstep_256_steps(stepq):
+    # 64 requests x 48 heads, d = 128, nominal 6 bits over {4,6,8}, 1 pivot head;
+    # the oracle follows two of the requests (96 heads) at every step.
+    _lockstep(stepq, "qwen_layer", 64, 256, check=[0, 37])
+
+
+@pytest.mark.parametrize("name", ["qwen_pool6", "qwen_pool4"])
+def test_pool_slice_lockstep(stepq, name):
+    # a 2-layer slice of the 2,304-head pool at batch 70 (2 pivot heads), 8 steps
+    _lockstep(stepq, name, 70, 8, check=[0, 69], n_layers=2, n_pivots=2)
+
+
+def test_fused_bit_identical_to_two_stream(stepq):
+    a = Run(stepq, "qwen_layer", 9)
+    b = Run(stepq, "qwen_layer", 9)
+    a.pack_initial()
+    b.pack_initial()
+    for t in range(6):
+        _, oa = a.step(t, fused=False)
+        _, ob = b.step(t, fused=True)
+        assert np.array_equal(oa, ob)
+        assert torch.equal(a.pool, b.pool)
+
+
+def test_ragged_and_empty(stepq):
+    run = Run(stepq, "qwen_layer", 5, extra_slots=11)
+    run.pack_initial()
+    before = run.pool.clone()
+    d = _inputs_to_dev(synth.step_inputs(run.wl, run.wl.seed, 5, 0, alpha=run.alpha))
+    o = torch.zeros_like(d["q"])
+    ws = torch.empty(run.ctx.workspace_bytes(5, 1) // 4, dtype=torch.float32, device="cuda")
+    run.ctx.decode_step(run.pool, run.slots_t, 0, 0, 1, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o, ws)
+    run.ctx.sync()
+    assert torch.equal(run.pool, before) and float(o.abs().sum()) == 0.0
+    # slots not named by the call stay untouched
+    sb = run.P.slot_bytes
+    untouched = sorted(set(range(run.n_slots)) - set(run.slots.tolist()))
+    run.step(0)
+    for s in untouched:
+        assert torch.equal(run.pool[s * sb:(s + 1) * sb], before[s * sb:(s + 1) * sb])
+
+
+def test_bad_slot_reports_device_error(stepq):
+    run = Run(stepq, "tiny_gdn", 2)
+    run.pack_initial()
+    bad = torch.tensor([0, run.n_slots + 5], dtype=torch.int32, device="cuda")
+    d = _inputs_to_dev(synth.step_inputs(run.wl, run.wl.seed, 2, 0, alpha=run.alpha))
+    o = torch.zeros_like(d["q"])
+    run.ctx.decode_step_fused(run.pool, bad, 2, 0, 1, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)
+    with pytest.raises(stepq.StepqError) as ei:
+        run.ctx.sync()
+    assert ei.value.code == stepq.EDEVICE
+    run.ctx.sync()  # the word was cleared
+    with pytest.raises(stepq.StepqError) as ei:
+        run.ctx.decode_step_fused(run.pool[1:], run.slots_t, 2, 0, 1, d["q"], d["k"], d["v"], d["alpha"],
+                                  d["beta"], o)
+    assert ei.value.code == stepq.EINVAL
+    with pytest.raises(stepq.StepqError) as ei:
+        run.ctx.decode_step_fused(run.pool, run.slots_t, 2, 0, 2, d["q"], d["k"], d["v"], d["alpha"],
+                                  d["beta"], o)
+    assert ei.value.code == stepq.EINVAL
+
+
+def test_fp32_reference_kernel(stepq):
+    plan, data, wl, _ = oracle_plan("qwen_layer")
+    P = stepq.Plan.from_bytes(data)
+    n = 3
+    ctx = stepq.Context(P, n)
+    S0 = synth.initial_states(wl, wl.seed, n)
+    Sd = torch.from_numpy(S0).cuda().contiguous()
+    slots = torch.arange(n, dtype=torch.int32, device="cuda")
+    alpha = synth.gates(wl, wl.seed)
+    S_ref = S0.copy()
+    for t in range(16):
+        inp = synth.step_inputs(wl, wl.seed, n, t, alpha=alpha)
+        d = _inputs_to_dev(inp)
+        o = torch.zeros_like(d["q"])
+        ctx.fp32_decode_step(Sd, slots, n, 0, 1, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)
+        ctx.sync()
+        og = o.cpu().numpy()
+        for r in range(n):
+            for h in range(0, wl.n_heads, 5):
+                o_ref = core.step_fp32(S_ref[r, 0, h], inp["q"][r, 0, h], inp["k"][r, 0, h], inp["v"][r, 0, h],
+                                       inp["alpha"][r, 0, h], inp["beta"][r, 0, h])
+                assert _close(og[r, 0, h], o_ref).all()
+    Sg = Sd.cpu().numpy()
+    for r in range(n):
+        for h in range(0, wl.n_heads, 5):
+            assert _close(Sg[r, 0, h], S_ref[r, 0, h]).all()
+
+
+def test_calibration_kernels_match_oracle(stepq):
+    plan, data, wl, stats = oracle_plan("tiny_gdn")
+    P = stepq.Plan.from_bytes(data)
+    D, H = wl.d, wl.n_heads
+    ctx = stepq.Context(P, 1)
+    alpha = synth.gates(wl, wl.calib_seed)
+    om = torch.zeros((1, H, D), dtype=torch.float64, device="cuda")
+    ls = torch.zeros_like(om)
+    om_ref = np.zeros((1, H, D))
+    ls_ref = np.zeros((1, H, D))
+    for t in range(8):
+        inp = synth.step_inputs(wl, wl.calib_seed, 1, t, alpha=alpha)
+        d = _inputs_to_dev(inp)
+        ctx.calib_accumulate(1, 0, 1, d["q"], d["k"], d["alpha"], d["beta"], om, ls)
+        for h in range(H):
+            core.calib_accumulate(inp["q"][0, 0, h], inp["k"][0, 0, h], inp["alpha"][0, 0, h], inp["beta"][0, 0, h],
+                                  om_ref[0, h], ls_ref[0, h])
+    ctx.sync()
+    assert np.allclose(om.cpu().numpy(), om_ref, rtol=1e-12, atol=0)
+    assert np.allclose(ls.cpu().numpy(), ls_ref, rtol=1e-12, atol=1e-300)
+    S = synth.initial_states(wl, wl.seed, 1)
+    wbar = stats["wbar"].reshape(1, H, D)
+    dist = torch.zeros((1, H, D, 3), dtype=torch.float64, device="cuda")
+    ctx.calib_distortion(1, 0, 1, torch.from_numpy(S).cuda(), torch.from_numpy(wbar).cuda(), [2, 4, 6], dist)
+    ctx.sync()
+    dg = dist.cpu().numpy()
+    for h in range(H):
+        for m, b in enumerate((2, 4, 6)):
+            ref = core.distortion_rows(D, b, stats["rho"][0, h], stats["wbar"][0, h], S[0, 0, h])
+            assert np.allclose(dg[0, h, :, m], ref, rtol=1e-12, atol=0)
+
+
+def test_full_pool_sampled_heads(stepq):
+    """The 2,304-head pool at batch 70 (nominal 6 bits, 32 pivots), in the
+    launch configuration the benchmark times: one fused step, then sampled
+    (request, layer, head) records checked against the oracle."""
+    plan, data, wl, _ = oracle_plan("qwen_pool6")
+    pv = model.PlanView(plan)
+    P = stepq.Plan.from_bytes(data)
+    n = 70
+    ctx = stepq.Context(P, n)
+    pool = torch.zeros(n * P.slot_bytes, dtype=torch.uint8, device="cuda")
+    slots = torch.arange(n, dtype=torch.int32, device="cuda")
+    rng = np.random.default_rng(11)
+    for l in range(wl.n_layers):       # pack S_0 layer by layer to bound host memory
+        S0 = synth.initial_states(wl, wl.seed, n, layers=[l])
+        ctx.requant_pack(pool, slots, n, l, l + 1, torch.from_numpy(S0).cuda())
+    ctx.sync()
+    alpha = synth.gates(wl, wl.seed)
+    inp = synth.step_inputs(wl, wl.seed, n, 0, alpha=alpha)
+    d = _inputs_to_dev(inp)
+    sb = P.slot_bytes
+    prev = pool.clone()
+    o = torch.zeros_like(d["q"])
+    ctx.decode_step_fused(pool, slots, n, 0, wl.n_layers, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)
+    ctx.sync()
+    og = o.cpu().numpy()
+    widths = P.widths()
+    samples = [(int(rng.integers(n)), int(rng.integers(wl.n_layers)), int(rng.integers(wl.n_heads))) for _ in range(24)]
+    samples += [(5, int(u) // wl.n_heads, int(u) % wl.n_heads) for u in np.nonzero(widths == 16)[0][:3]]
+    for (r, l, h) in samples:
+        off, nb = P.record(l, h)
+        rec_prev = prev[r * sb + off:r * sb + off + nb].cpu().numpy()
+        rec_new = pool[r * sb + off:r * sb + off + nb].cpu().numpy()
+        new_rec, o_ref, tie, S, w = model.step_head(pv.mode, pv.D, pv.rw(l, h), pv.rho[l, h], pv.wbar[l, h],
+                                                    rec_prev, inp["q"][r, l, h], inp["k"][r, l, h],
+                                                    inp["v"][r, l, h], inp["alpha"][r, l, h], inp["beta"][r, l, h])
+        assert _close(og[r, l, h], o_ref).all(), (r, l, h)
+        if not np.array_equal(rec_new, new_rec):
+            zg, hg, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), rec_new)
+            zo, ho, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), new_rec)
+            mism = (zg != zo) | (hg != ho)
+            assert not (mism & (tie == 0)).any(), (r, l, h)

@@ -1,0 +1,150 @@
+"""Host-side checks of libstepq.so that need no GPU: the library loads, exports
+every entry point its header declares, parses and validates plan files
+written by the oracle's independent writer, and its offline planner picks
+the same widths and pivots as the oracle's allocator on the same statistics.
+"""
+import os
+import re
+import struct
+import zlib
+
+import numpy as np
+import pytest
+
+from oracle import allocator, model, plan_io
+from quantized_recurrent_state_b200 import build as qbuild
+from quantized_recurrent_state_b200 import stepq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    qbuild.build()
+
+
+def test_exports_every_declared_symbol():
+    hdr = open(os.path.join(ROOT, "include", "stepq.h")).read()
+    declared = set(re.findall(r"^\s*(?:const char \*|int|void|size_t|uint64_t)\s*\*?\s*(stepq_\w+)\s*\(", hdr, re.M))
+    assert len(declared) >= 20
+    l = stepq.lib()
+    for name in declared:
+        assert hasattr(l, name), name
+    assert declared == set(stepq.EXPORTED)
+
+
+def _tiny_plan_dict(mode=0):
+    D = 16
+    if mode == 0:
+        widths = np.array([2, 6, 16, 4], np.uint8)
+        units = 4
+    else:
+        rng = np.random.default_rng(3)
+        widths = rng.choice([4, 6, 8], size=4 * D).astype(np.uint8)
+        widths[[3, 40]] = 16
+        # keep inside the budget
+        while widths[widths != 16].astype(int).sum() > 6 * (widths != 16).sum():
+            widths[np.argmax(widths * (widths != 16))] -= 2
+        units = 4 * D
+    return dict(mode=mode, n_layers=2, n_heads=2, d=D, n_pivots=int((widths == 16).sum()),
+                bitset=[2, 4, 6] if mode == 0 else [4, 6, 8], nominal_bits=4.0 if mode == 0 else 6.0,
+                horizon=65536, widths=widths, wbar=np.linspace(0.5, 2.0, 4 * D).astype(np.float32),
+                rho=np.linspace(0.8, 1.2, 4 * D).astype(np.float32), lgate=-np.linspace(0.01, 0.1, units),
+                lifetime=np.linspace(1, 10, units))
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_plan_parse_matches_oracle_layout(mode):
+    pd = _tiny_plan_dict(mode)
+    data = plan_io.write_plan(None, pd)
+    p = stepq.Plan.from_bytes(data)
+    assert (p.mode, p.n_layers, p.n_heads, p.d) == (mode, 2, 2, 16)
+    assert np.array_equal(p.widths(), pd["widths"])
+    offs, slot = plan_io.pool_layout(pd)
+    assert p.slot_bytes == slot
+    for l in range(2):
+        for h in range(2):
+            off, nb = p.record(l, h)
+            assert off == offs[l * 2 + h]
+            assert nb == plan_io.record_bytes(mode, 16, plan_io.head_row_widths(pd, l, h))
+    assert p.info.bits_per_value == pytest.approx(allocator.bits_per_value(mode, 2, 2, 16, pd["widths"]), rel=1e-15)
+    assert p.info.bits_per_value_s16 == pytest.approx(
+        allocator.bits_per_value(mode, 2, 2, 16, pd["widths"], scale_bits=16), rel=1e-15)
+    assert p.info.n_pivots == pd["n_pivots"]
+
+
+def _expect_format_error(data):
+    with pytest.raises(stepq.StepqError) as ei:
+        stepq.Plan.from_bytes(data)
+    assert ei.value.code == stepq.EFORMAT, str(ei.value)
+
+
+def _recrc(b: bytearray) -> bytes:
+    b[-4:] = struct.pack("<I", zlib.crc32(bytes(b[:-4])) & 0xFFFFFFFF)
+    return bytes(b)
+
+
+def test_plan_validation_errors():
+    pd = _tiny_plan_dict(0)
+    good = bytearray(plan_io.write_plan(None, pd))
+    bad = bytearray(good); bad[0] = ord("X"); _expect_format_error(_recrc(bad))                 # magic
+    bad = bytearray(good); bad[70] ^= 1; _expect_format_error(bytes(bad))                        # CRC
+    bad = bytearray(good); bad[8] = 2; _expect_format_error(_recrc(bad))                         # version
+    _expect_format_error(bytes(good[:-8]))                                                       # truncated
+    bad = bytearray(good); bad[36] = 2; _expect_format_error(_recrc(bad))                        # pivot count
+    bad = bytearray(good); bad[64 + 0] = 8; _expect_format_error(_recrc(bad))                    # width not in bitset
+    pd2 = dict(pd); pd2["widths"] = np.array([6, 6, 16, 4], np.uint8)                            # 16 bits > floor(4*3)
+    _expect_format_error(plan_io.write_plan(None, pd2))
+    pd3 = dict(pd); pd3["wbar"] = pd["wbar"].copy(); pd3["wbar"][5] = 0.0                       # non-positive weight
+    _expect_format_error(plan_io.write_plan(None, pd3))
+    with pytest.raises(stepq.StepqError) as ei:
+        stepq.Plan.load("/nonexistent/plan.bin")
+    assert ei.value.code == stepq.EINVAL
+
+
+def _random_stats(mode, L, H, D, bits, seed):
+    rng = np.random.default_rng(seed)
+    units = L * H if mode == 0 else L * H * D
+    lgate = -np.log(2) / np.exp(rng.uniform(np.log(4), np.log(20000), units))
+    # decreasing distortion in the width
+    base = rng.uniform(0.5, 2.0, units)[:, None]
+    rate = rng.uniform(0.4, 0.8, units)[:, None]
+    dist = base * np.exp(-rate * np.asarray(bits, float)[None, :])
+    wbar = rng.uniform(0.2, 5.0, L * H * D).astype(np.float32)
+    return dict(lgate=lgate, dist=dist, wbar=wbar,
+                rho=(1.0 / np.sqrt(np.sqrt(wbar.astype(np.float64)))).astype(np.float32))
+
+
+@pytest.mark.parametrize("mode,bits,nominal,pivots", [(0, (4, 6, 8), 6.0, 5), (0, (2, 4, 6, 8), 4.0, 3),
+                                                       (1, (4, 6, 8), 6.0, 40), (1, (2, 4, 6, 8), 4.0, 7)])
+def test_product_planner_equals_oracle_allocator(mode, bits, nominal, pivots):
+    L, H, D = 3, 8, 16
+    for seed in range(3):
+        st = _random_stats(mode, L, H, D, bits, seed)
+        ora = model.build_plan(mode, D, L, H, st, bits, nominal, pivots, 65536)
+        p = stepq.Plan.build(mode, L, H, D, bits, nominal, pivots, 65536, st["lgate"], st["dist"], st["wbar"])
+        assert np.array_equal(p.widths(), ora["widths"]), (mode, seed)
+        # rho derived identically
+        data = plan_io.write_plan(None, ora)
+        assert plan_io.read_plan(data)["rho"].tobytes() == ora["rho"].tobytes()
+
+
+def test_product_planner_writes_file(tmp_path):
+    st = _random_stats(0, 2, 4, 16, (4, 6, 8), 9)
+    path = str(tmp_path / "p.plan")
+    p = stepq.Plan.build(0, 2, 4, 16, (4, 6, 8), 6.0, 1, 4096, st["lgate"], st["dist"], st["wbar"], path=path)
+    back = plan_io.read_plan(open(path, "rb").read())
+    assert np.array_equal(back["widths"], p.widths())
+    assert np.array_equal(back["rho"], st["rho"])
+
+
+def test_calls_without_device_fail_cleanly():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    pd = _tiny_plan_dict(0)
+    p = stepq.Plan.from_bytes(plan_io.write_plan(None, pd))
+    import ctypes
+    h = ctypes.c_void_p()
+    rc = stepq.lib().stepq_ctx_create(p._h, ctypes.c_void_p(1), ctypes.c_void_p(2), 4, 1, ctypes.byref(h))
+    assert rc == stepq.ECUDA
