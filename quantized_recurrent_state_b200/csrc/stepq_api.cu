@@ -558,6 +558,7 @@ stepq::Args base_args(stepq_ctx *c, void *pool, const int32_t *slots, int n_req,
     a.n_items = n_req * (le - lb) * c->plan->H;
     a.t = c->t;
     a.err = c->err;
+    a.neg_zero = -0.0f;
     return a;
 }
 

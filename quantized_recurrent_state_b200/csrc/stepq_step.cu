@@ -64,6 +64,7 @@ struct Scratch {
     double cst[3];    // Kc, Qc, q.k
     double red[3][8];
     int meta[kStages][4];  // slot, width, valid, unused
+    float nz;              // -0.0f, read at run time (see fit_scales)
 };
 
 template <int D>
@@ -165,7 +166,7 @@ __device__ __forceinline__ float2 tree_sum2(float2 (&x)[N]) {
 #pragma unroll
     for (int s = 1; s < N; s <<= 1)
 #pragma unroll
-        for (int i = 0; i + s < N; i += 2 * s) x[i] = __fadd2_rn(x[i], x[i + s]);
+        for (int i = 0; i + s < N; i += 2 * s) x[i] = add2(x[i], x[i + s]);
     return x[0];
 }
 
@@ -210,8 +211,8 @@ __device__ void fit_scales(float (&S)[D / 8][4], float (&rr)[D / 8], Scratch<D> 
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
         const float2 ir = make_float2(inv_r[r], inv_r[r]);
-        const float2 a01 = __fmul2_rn(make_float2(S[r][0], S[r][1]), ir);
-        const float2 a23 = __fmul2_rn(make_float2(S[r][2], S[r][3]), ir);
+        const float2 a01 = mul2(make_float2(S[r][0], S[r][1]), ir);
+        const float2 a23 = mul2(make_float2(S[r][2], S[r][3]), ir);
         S[r][0] = a01.x; S[r][1] = a01.y; S[r][2] = a23.x; S[r][3] = a23.y;
     }
     // 3. column absmax -> c0
@@ -236,6 +237,7 @@ __device__ void fit_scales(float (&S)[D / 8][4], float (&rr)[D / 8], Scratch<D> 
     {
         const float2 mg = make_float2(kMagic, kMagic);
         const float2 nmg = make_float2(-kMagic, -kMagic);
+        const float2 nz2 = make_float2(sc.nz, sc.nz);
 #pragma unroll
         for (int hp = 0; hp < 2; ++hp) {
             const int jA = j0 + 2 * hp;
@@ -244,11 +246,14 @@ __device__ void fit_scales(float (&S)[D / 8][4], float (&rr)[D / 8], Scratch<D> 
 #pragma unroll
             for (int r = 0; r < RT; ++r) {
                 const float2 y = make_float2(S[r][2 * hp], S[r][2 * hp + 1]);
-                const float2 t = __ffma2_rn(y, ic, mg);
-                const float2 z0 = __fadd2_rn(t, nmg);
+                const float2 t = fma2(y, ic, mg);
+                const float2 z0 = add2(t, nmg);
                 const float2 b2 = make_float2(bw[r], bw[r]);
-                tn[r] = __fmul2_rn(b2, __fmul2_rn(z0, y));
-                td[r] = __fmul2_rn(b2, __fmul2_rn(z0, z0));
+                // fl(b * p) written as fma(b, p, -0) with a run-time -0: the
+                // product is rounded once and cannot be contracted into the
+                // pairwise additions that follow
+                tn[r] = fma2(b2, mul2(z0, y), nz2);
+                td[r] = fma2(b2, mul2(z0, z0), nz2);
             }
             const float2 sn = tree_sum2<RT>(tn);
             const float2 sd = tree_sum2<RT>(td);
@@ -279,7 +284,7 @@ __device__ __forceinline__ int2 final_codes(float2 y, float2 ic) {
     constexpr float MG2 = kMagic + (float)OFF;
     constexpr int LO = 0x4B400000 + OFF - Q;
     constexpr int HI = 0x4B400000 + OFF + Q;
-    const float2 t = __ffma2_rn(y, ic, make_float2(MG2, MG2));
+    const float2 t = fma2(y, ic, make_float2(MG2, MG2));
     int T0 = __float_as_int(t.x), T1 = __float_as_int(t.y);
     T0 = min(max(T0, LO), HI);
     T1 = min(max(T1, LO), HI);
@@ -450,12 +455,12 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
         if (KIND != kDecode) {
             const float ai = sc.a[i];
             const float2 a2 = make_float2(ai, ai);
-            const float2 A01 = __fmul2_rn(a2, cp01);
-            const float2 A23 = __fmul2_rn(a2, cp23);
+            const float2 A01 = mul2(a2, cp01);
+            const float2 A23 = mul2(a2, cp23);
             const float2 z01 = make_float2(x_as_zscaled<B>(X[0]), x_as_zscaled<B>(X[1]));
             const float2 z23 = make_float2(x_as_zscaled<B>(X[2]), x_as_zscaled<B>(X[3]));
-            const float2 s01 = __fmul2_rn(A01, z01);
-            const float2 s23 = __fmul2_rn(A23, z23);
+            const float2 s01 = mul2(A01, z01);
+            const float2 s23 = mul2(A23, z23);
             S[r][0] = s01.x; S[r][1] = s01.y; S[r][2] = s23.x; S[r][3] = s23.y;
         }
     }
@@ -490,8 +495,8 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
         for (int r = 0; r < RT; ++r) {
             const float ki = sc.kf[g * RT + r];
             const float2 k2 = make_float2(ki, ki);
-            const float2 s01 = __ffma2_rn(k2, w01, make_float2(S[r][0], S[r][1]));
-            const float2 s23 = __ffma2_rn(k2, w23, make_float2(S[r][2], S[r][3]));
+            const float2 s01 = fma2(k2, w01, make_float2(S[r][0], S[r][1]));
+            const float2 s23 = fma2(k2, w23, make_float2(S[r][2], S[r][3]));
             S[r][0] = s01.x; S[r][1] = s01.y; S[r][2] = s23.x; S[r][3] = s23.y;
         }
         fit_pack<D, B>(S, rec_g, sc, tid);
@@ -568,10 +573,10 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
         for (int r = 0; r < RT; ++r) {
             const float ki = sc.kf[g * RT + r];
             const float2 k2 = make_float2(ki, ki);
-            const float2 p01 = __fmul2_rn(al, make_float2(S[r][0], S[r][1]));
-            const float2 p23 = __fmul2_rn(al, make_float2(S[r][2], S[r][3]));
-            const float2 s01 = __ffma2_rn(k2, w01, p01);
-            const float2 s23 = __ffma2_rn(k2, w23, p23);
+            const float2 p01 = mul2(al, make_float2(S[r][0], S[r][1]));
+            const float2 p23 = mul2(al, make_float2(S[r][2], S[r][3]));
+            const float2 s01 = fma2(k2, w01, p01);
+            const float2 s23 = fma2(k2, w23, p23);
             S[r][0] = s01.x; S[r][1] = s01.y; S[r][2] = s23.x; S[r][3] = s23.y;
         }
         store_pivot<D>(S, rec_g, tid);
@@ -592,6 +597,7 @@ __global__ void __launch_bounds__(2 * D) k_step(Args a) {
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
+        sc.nz = a.neg_zero;
     }
     __syncthreads();
     if (tid == 0) {
@@ -673,6 +679,7 @@ __global__ void __launch_bounds__(2 * D) k_requant_pack(Args a) {
         sc.rho[tid] = a.t.rho[(size_t)gl * D + tid];
         sc.wbar[tid] = a.t.wbar[(size_t)gl * D + tid];
     }
+    if (tid == 0) sc.nz = a.neg_zero;
     __syncthreads();
     switch (width) {
         case 2: fit_pack<D, 2>(S, rec, sc, tid); break;
@@ -699,10 +706,10 @@ __device__ void unpack_uniform(const uint8_t *rec, float *out, int tid) {
         const int i = g * G::RT + r;
         const float ri = rr[i];
         const float2 r2 = make_float2(ri, ri);
-        const float2 A01 = __fmul2_rn(r2, c01), A23 = __fmul2_rn(r2, c23);
+        const float2 A01 = mul2(r2, c01), A23 = mul2(r2, c23);
         const float2 z01 = make_float2(x_as_zscaled<B>(field_x<B>(W, 4 * r)), x_as_zscaled<B>(field_x<B>(W, 4 * r + 1)));
         const float2 z23 = make_float2(x_as_zscaled<B>(field_x<B>(W, 4 * r + 2)), x_as_zscaled<B>(field_x<B>(W, 4 * r + 3)));
-        const float2 s01 = __fmul2_rn(A01, z01), s23 = __fmul2_rn(A23, z23);
+        const float2 s01 = mul2(A01, z01), s23 = mul2(A23, z23);
         *reinterpret_cast<float4 *>(out + (size_t)i * D + 4 * l) = make_float4(s01.x, s01.y, s23.x, s23.y);
     }
 }
@@ -805,6 +812,7 @@ __global__ void __launch_bounds__(2 * D) k_calib_dist(Args a, BitList bl, double
         sc.wbar[tid] = wb;
         sc.rho[tid] = (float)(1.0 / sqrt(sqrt((double)wb)));
     }
+    if (tid == 0) sc.nz = a.neg_zero;
     __syncthreads();
     const float *Sg = a.S_in + (size_t)row * D * D;
     switch (bl.b[m]) {
