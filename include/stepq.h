@@ -179,6 +179,32 @@ int stepq_decode_step_fused(stepq_ctx *ctx, void *pool, const int32_t *slots, in
                             int le, const float *q, const float *k, const float *v,
                             const float *alpha, const float *beta, float *o);
 
+/* Allocation-free variant of stepq_decode_step (the paper has no
+ * counterpart; it exists for callers that cannot allocate device memory,
+ * such as plugins whose host framework owns every allocation, or latency-
+ * critical loops where an allocator call is not allowed).  The caller passes
+ * the same inputs and outputs but no workspace: the w values the decode
+ * kernel hands to the fit-and-pack kernel live in a fixed array of
+ * STEPQ_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.  The call allocates nothing.
+ *   - Limit: n_req * (le - lb) * n_heads * d * 4 bytes must not exceed
+ *     STEPQ_NOALLOC_SCRATCH_BYTES; larger calls return STEPQ_EINVAL (split
+ *     them, e.g. one layer range at a time).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents (nothing in it needs to start at zero: every value is written
+ *     before it is read).  Before launching, the call makes `main` wait for
+ *     all earlier side-stream work of this context; calls from different
+ *     contexts, threads or processes' streams that overlap on the GPU race
+ *     on the array.
+ * Results are bit-identical to stepq_decode_step. */
+#define STEPQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+int stepq_decode_step_noalloc(stepq_ctx *ctx, void *pool, const int32_t *slots, int n_req, int lb, int le,
+                              const float *q, const float *k, const float *v, const float *alpha,
+                              const float *beta, float *o);
+
 /* Wait for all work of the context (both streams) with a host-side timeout
  * (<= 0: wait without limit), then return the device error word:
  * STEPQ_OK, STEPQ_ETIMEDOUT, STEPQ_EDEVICE (the word is cleared) or ECUDA. */

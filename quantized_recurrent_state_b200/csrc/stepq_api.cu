@@ -15,6 +15,7 @@
 #include <cstdio>
 #include <cstring>
 #include <limits>
+#include <mutex>
 #include <new>
 #include <string>
 #include <thread>
@@ -936,3 +937,53 @@ extern "C" int stepq_kernel_stats(stepq_ctx *c, double *ms, uint64_t *launches) 
 }
 
 extern "C" const char *stepq_last_error(void) { return g_err.c_str(); }
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the two-stream step: the decode -> fit-pack
+// hand-off values w live in a fixed device array owned by the library, for
+// callers that cannot allocate device memory themselves.
+// ---------------------------------------------------------------------------
+
+static __device__ __align__(256) float g_noalloc_w[STEPQ_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+namespace {
+std::mutex g_noalloc_mu;
+constexpr int kMaxDevices = 128;
+float *g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_w on the current device `dev` (looked up once
+// per device; in host code the symbol itself is only a host-side stand-in).
+int noalloc_scratch(int dev, float **out) {
+    if (dev < 0 || dev >= kMaxDevices) return fail(STEPQ_EINVAL, "decode_step_noalloc: device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_w);
+        if (e != cudaSuccess) return cuda_fail(e, "decode_step_noalloc: cudaGetSymbolAddress");
+        g_noalloc_addr[dev] = static_cast<float *>(p);
+    }
+    *out = g_noalloc_addr[dev];
+    return STEPQ_OK;
+}
+}  // namespace
+
+extern "C" int stepq_decode_step_noalloc(stepq_ctx *c, void *pool, const int32_t *slots, int n_req, int lb, int le,
+                                         const float *q, const float *k, const float *v, const float *alpha,
+                                         const float *beta, float *o) {
+    int rc = check_range(c, n_req, lb, le);
+    if (rc) return rc;
+    if ((rc = check_step_io(c, pool, slots, q, k, v, alpha, beta, o))) return rc;
+    const size_t need = stepq_workspace_bytes(c, n_req, le - lb);
+    if (need > STEPQ_NOALLOC_SCRATCH_BYTES)
+        return fail(STEPQ_EINVAL,
+                    "decode_step_noalloc: this call needs %zu bytes of scratch, more than the built-in %u bytes; "
+                    "split it into calls over fewer requests or layers",
+                    need, (unsigned)STEPQ_NOALLOC_SCRATCH_BYTES);
+    if ((rc = set_device(c))) return rc;
+    if (n_req == 0) return STEPQ_OK;
+    float *scratch = nullptr;
+    if ((rc = noalloc_scratch(c->device, &scratch))) return rc;
+    // every earlier fit-pack of this context may still read the shared array
+    if ((rc = wait_side(c, 0, c->plan->L))) return rc;
+    return stepq_decode_step(c, pool, slots, n_req, lb, le, q, k, v, alpha, beta, o, scratch);
+}

@@ -25,7 +25,9 @@ EXPORTED = [
     "stepq_decode_step_fused", "stepq_sync", "stepq_unpack", "stepq_fp32_decode_step",
     "stepq_calib_accumulate", "stepq_calib_distortion", "stepq_copy_probe",
     "stepq_launch_count", "stepq_last_error", "stepq_ctx_set_timing", "stepq_kernel_stats",
+    "stepq_decode_step_noalloc",
 ]
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class StepqError(RuntimeError):
@@ -85,6 +87,7 @@ def lib():
         l.stepq_launch_count.restype = ctypes.c_uint64
         l.stepq_ctx_set_timing.argtypes = [P, I]
         l.stepq_kernel_stats.argtypes = [P, P, P]
+        l.stepq_decode_step_noalloc.argtypes = [P, P, P, I, I, I, P, P, P, P, P, P]
         _lib = l
     return _lib
 
@@ -185,6 +188,14 @@ class Context:
         return _check(lib().stepq_decode_step_fused(self._h, _ptr(pool), _ptr(slots), n_req, lb, le,
                                                     _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                                     _ptr(o)))
+
+    def decode_step_noalloc(self, pool, slots, n_req, lb, le, q, k, v, alpha, beta, o):
+        """The two-stream step without a workspace argument: for callers that
+        cannot allocate device memory.  The hand-off values live in a fixed
+        8 MiB array inside the library (shared by all calls on the device)."""
+        return _check(lib().stepq_decode_step_noalloc(self._h, _ptr(pool), _ptr(slots), n_req, lb, le,
+                                                      _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                                      _ptr(o)))
 
     def sync(self, timeout_ms: int = 60000):
         return _check(lib().stepq_sync(self._h, timeout_ms))
