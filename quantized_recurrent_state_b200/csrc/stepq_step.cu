@@ -44,25 +44,36 @@ struct Stream {
 
 // Shared memory besides the stages.
 template <int D>
-struct Scratch {
-    double pU[8][D];
-    double pO[8][D];
+struct __align__(16) Scratch {
+    static constexpr int RT = D / 8, LANES = D / 4, RS = D / 4 + 4;  // RS: padded row of the transpose
+    union {
+        struct {
+            double pU[8][D];  // per-band column partials of u and o
+            double pO[8][D];
+        } col;
+        float rsum[8][RT][RS];  // per-thread row partials, transposed for the row reduction
+    } u;
     float pf0[8][D];
     float pf1[8][D];
-    float a[D];       // a_i = fl(alpha_i r_i)  (pivot: alpha_i)
+    float a[D];       // a_i = fl(alpha_i r_i)
     float kf[D];      // k_i
     double kap[D];    // k_i a_i 2^-169   (pivot: k_i alpha_i)
     double qt[D];     // q_i a_i 2^-169   (pivot: q_i alpha_i)
     float rho[D];
     float wbar[D];
+    float2 rowfit[D]; // (fl(1/r_i), b_i) of the refit
+    float rowr[D];    // r_i of the refit
     float cpr[D];     // c_j 2^-12
-    float cold[D];    // c_j
+    float cold[D];    // c_j (old on entry, refitted after fit_scales)
     float wv[D];      // w_j
     float ic0[D];
     float c0[D];
     float ic[D];
-    double cst[3];    // Kc, Qc, q.k
-    double red[3][8];
+    float colmax[D];
+    double bandK[8];  // per band: sum_i k_i a_i (256 + off), sum_i q_i a_i (256 + off), sum_i q_i k_i
+    double bandQ[8];
+    double bandQK[8];
+    int need_clamp;
     int meta[kStages][4];  // slot, width, valid, unused
     float nz;              // -0.0f, read at run time (see fit_scales)
 };
@@ -160,16 +171,6 @@ __device__ __forceinline__ void store_stream(uint8_t *blk, int t, const uint32_t
     }
 }
 
-// Pairwise (balanced tree) sum of N float2 values, in index order.
-template <int N>
-__device__ __forceinline__ float2 tree_sum2(float2 (&x)[N]) {
-#pragma unroll
-    for (int s = 1; s < N; s <<= 1)
-#pragma unroll
-        for (int i = 0; i + s < N; i += 2 * s) x[i] = add2(x[i], x[i + s]);
-    return x[0];
-}
-
 template <int N>
 __device__ __forceinline__ float tree_sum1(float (&x)[N]) {
 #pragma unroll
@@ -179,49 +180,121 @@ __device__ __forceinline__ float tree_sum1(float (&x)[N]) {
     return x[0];
 }
 
+// Balanced pairwise tree over terms pushed in index order, holding only
+// log2(N) + 1 partial sums (push(r, v) with r = 0, 1, ..., N-1 unrolled).
+template <int N>
+struct PairTree {
+    static constexpr int LV = (N >= 16) ? 5 : (N >= 8) ? 4 : (N >= 4) ? 3 : (N >= 2) ? 2 : 1;
+    float2 s[LV];
+    __device__ __forceinline__ void push(int r, float2 v) {
+        int lvl = 0;
+#pragma unroll
+        for (int b = 0; b < LV - 1; ++b) {
+            if (r & (1 << b)) {
+                v = add2(s[lvl], v);
+                ++lvl;
+            } else {
+                break;
+            }
+        }
+        s[lvl] = v;
+    }
+    __device__ __forceinline__ float2 total() const { return s[LV - 1]; }
+};
+
+// Word-level packing: the final-code bits T = 0x4B400000 + 2^(B-1) + z are
+// added into the stream at their bit offsets, and the constant high parts are
+// removed per word at the end.
+template <int D, int B>
+__host__ __device__ constexpr uint32_t pack_correction(int w) {
+    uint32_t c = 0;
+    for (int p = 0; p < 4 * (D / 8); ++p) {
+        const int bit = p * B;
+        if ((bit >> 5) == w) c += 0x4B400000u << (bit & 31);
+    }
+    return c;
+}
+
+template <int B>
+__device__ __forceinline__ void field_acc(uint32_t *W, int p, uint32_t T) {
+    const int bit = p * B;
+    const int w = bit >> 5;
+    const int s = bit & 31;
+    W[w] += T << s;
+    if (s + B > 32) W[w + 1] += (T & ((1u << B) - 1u)) >> (32 - s);
+}
+
 // ---------------------------------------------------------------------------
 // Refit of the fp32 tile S held in registers (all rows at width B).  On
-// return S holds y = fl(S * fl(1/r)), rr[] the row factors of the thread's
-// rows, sc.ic[j] = fl(1/c_j) and sc.cold[j] = c_j.  Requires rho and wbar of
-// the head in sc.rho / sc.wbar.
+// return S holds y = fl(S * fl(1/r)); sc.rowr[i] = r_i, sc.cold[j] = c_j,
+// sc.ic[j] = fl(1/c_j), sc.colmax[j] = max_i |y_ij|, sc.need_clamp != 0 iff
+// some final code needs the clamp.  rec_r (global, may be null) receives r.
+// Requires rho and wbar of the head in sc.rho / sc.wbar.
 // ---------------------------------------------------------------------------
 template <int D, int B>
-__device__ void fit_scales(float (&S)[D / 8][4], float (&rr)[D / 8], Scratch<D> &sc, int tid) {
+__device__ void fit_scales(float (&S)[D / 8][4], Scratch<D> &sc, int tid, float *rec_r) {
     using G = Geo<D>;
-    constexpr int RT = G::RT, LANES = G::LANES;
+    constexpr int RT = G::RT, LANES = G::LANES, RS = Scratch<D>::RS, HALF = LANES / 2;
     constexpr int Q = (1 << (B - 1)) - 1;
     const int g = tid / LANES, l = tid % LANES;
     const int j0 = 4 * l;
 
-    // 1. row factors: r_i = fl(max(pairwise_j |S_ij| / D, 1e-12) rho_i)
-    float inv_r[RT], bw[RT];
+    // 1. row sums: thread partial over its 4 columns, then the other lanes'
+    //    partials of the row through shared memory (pairwise in lane order)
+    float *rs = &sc.u.rsum[g][0][0];
 #pragma unroll
-    for (int r = 0; r < RT; ++r) {
-        const int i = g * RT + r;
-        float s = (fabsf(S[r][0]) + fabsf(S[r][1])) + (fabsf(S[r][2]) + fabsf(S[r][3]));
-        s = lane_pairwise_sum<LANES>(s);
+    for (int r = 0; r < RT; ++r)
+        rs[r * RS + l] = (fabsf(S[r][0]) + fabsf(S[r][1])) + (fabsf(S[r][2]) + fabsf(S[r][3]));
+    __syncwarp();
+    {
+        const int rr = l >> 1, hh = l & 1;
+        const float *src = rs + rr * RS + hh * HALF;
+        float v[HALF];
+        if constexpr (HALF % 4 == 0) {
+#pragma unroll
+            for (int k = 0; k < HALF / 4; ++k) {
+                const float4 x = *reinterpret_cast<const float4 *>(src + 4 * k);
+                v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < HALF; ++k) v[k] = src[k];
+        }
+        float s = tree_sum1<HALF>(v);
+        s = s + __shfl_xor_sync(0xffffffffu, s, 1);
+        const int i = g * RT + rr;
         float m = __fmul_rn(s, 1.0f / (float)D);
         m = fmaxf(m, 1e-12f);
         const float ri = __fmul_rn(m, sc.rho[i]);
-        rr[r] = ri;
-        inv_r[r] = __frcp_rn(ri);
-        bw[r] = __fmul_rn(sc.wbar[i], __fmul_rn(ri, ri));
+        const float inv = __frcp_rn(ri);
+        const float bw = __fmul_rn(sc.wbar[i], __fmul_rn(ri, ri));
+        if (hh == 0) {
+            sc.rowfit[i] = make_float2(inv, bw);
+            sc.rowr[i] = ri;
+            if (rec_r) rec_r[i] = ri;
+        }
     }
+    __syncwarp();
     // 2. y = fl(S * (1/r)) in place
 #pragma unroll
-    for (int r = 0; r < RT; ++r) {
-        const float2 ir = make_float2(inv_r[r], inv_r[r]);
-        const float2 a01 = mul2(make_float2(S[r][0], S[r][1]), ir);
-        const float2 a23 = mul2(make_float2(S[r][2], S[r][3]), ir);
+    for (int r = 0; r < RT; r += 2) {
+        const float4 f = *reinterpret_cast<const float4 *>(&sc.rowfit[g * RT + r]);
+        const float2 i0 = make_float2(f.x, f.x), i1 = make_float2(f.z, f.z);
+        const float2 a01 = mul2(make_float2(S[r][0], S[r][1]), i0);
+        const float2 a23 = mul2(make_float2(S[r][2], S[r][3]), i0);
+        const float2 b01 = mul2(make_float2(S[r + 1][0], S[r + 1][1]), i1);
+        const float2 b23 = mul2(make_float2(S[r + 1][2], S[r + 1][3]), i1);
         S[r][0] = a01.x; S[r][1] = a01.y; S[r][2] = a23.x; S[r][3] = a23.y;
+        S[r + 1][0] = b01.x; S[r + 1][1] = b01.y; S[r + 1][2] = b23.x; S[r + 1][3] = b23.y;
     }
     // 3. column absmax -> c0
+    {
+        float m[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-        float m = 0.0f;
+        for (int r = 0; r < RT; ++r)
 #pragma unroll
-        for (int r = 0; r < RT; ++r) m = fmaxf(m, fabsf(S[r][jj]));
-        sc.pf0[g][j0 + jj] = m;
+            for (int jj = 0; jj < 4; ++jj) m[jj] = fmaxf(m[jj], fabsf(S[r][jj]));
+        *reinterpret_cast<float4 *>(&sc.pf0[g][j0]) = make_float4(m[0], m[1], m[2], m[3]);
     }
     __syncthreads();
     if (tid < D) {
@@ -231,6 +304,8 @@ __device__ void fit_scales(float (&S)[D / 8][4], float (&rr)[D / 8], Scratch<D> 
         const float c0 = (m == 0.0f) ? 1.0f : __fdiv_rn(m, (float)Q);
         sc.c0[tid] = c0;
         sc.ic0[tid] = __frcp_rn(c0);
+        sc.colmax[tid] = m;
+        if (tid == 0) sc.need_clamp = 0;
     }
     __syncthreads();
     // 4. z0 and the weighted least-squares sums (pairwise over rows)
@@ -238,27 +313,29 @@ __device__ void fit_scales(float (&S)[D / 8][4], float (&rr)[D / 8], Scratch<D> 
         const float2 mg = make_float2(kMagic, kMagic);
         const float2 nmg = make_float2(-kMagic, -kMagic);
         const float2 nz2 = make_float2(sc.nz, sc.nz);
+        const float4 ic4 = *reinterpret_cast<const float4 *>(&sc.ic0[j0]);
 #pragma unroll
         for (int hp = 0; hp < 2; ++hp) {
             const int jA = j0 + 2 * hp;
-            const float2 ic = make_float2(sc.ic0[jA], sc.ic0[jA + 1]);
-            float2 tn[RT], td[RT];
+            const float2 ic = hp ? make_float2(ic4.z, ic4.w) : make_float2(ic4.x, ic4.y);
+            PairTree<RT> tn, td;
+            float4 f;
 #pragma unroll
             for (int r = 0; r < RT; ++r) {
+                if ((r & 1) == 0) f = *reinterpret_cast<const float4 *>(&sc.rowfit[g * RT + r]);
+                const float bwr = (r & 1) ? f.w : f.y;
                 const float2 y = make_float2(S[r][2 * hp], S[r][2 * hp + 1]);
                 const float2 t = fma2(y, ic, mg);
                 const float2 z0 = add2(t, nmg);
-                const float2 b2 = make_float2(bw[r], bw[r]);
+                const float2 b2 = make_float2(bwr, bwr);
                 // fl(b * p) written as fma(b, p, -0) with a run-time -0: the
                 // product is rounded once and cannot be contracted into the
                 // pairwise additions that follow
-                tn[r] = fma2(b2, mul2(z0, y), nz2);
-                td[r] = fma2(b2, mul2(z0, z0), nz2);
+                tn.push(r, fma2(b2, mul2(z0, y), nz2));
+                td.push(r, fma2(b2, mul2(z0, z0), nz2));
             }
-            const float2 sn = tree_sum2<RT>(tn);
-            const float2 sd = tree_sum2<RT>(td);
-            sc.pf0[g][jA] = sn.x; sc.pf0[g][jA + 1] = sn.y;
-            sc.pf1[g][jA] = sd.x; sc.pf1[g][jA + 1] = sd.y;
+            *reinterpret_cast<float2 *>(&sc.pf0[g][jA]) = tn.total();
+            *reinterpret_cast<float2 *>(&sc.pf1[g][jA]) = td.total();
         }
     }
     __syncthreads();
@@ -269,26 +346,14 @@ __device__ void fit_scales(float (&S)[D / 8][4], float (&rr)[D / 8], Scratch<D> 
         const float num = tree_sum1<8>(xn);
         const float den = tree_sum1<8>(xd);
         const float c = (den > 0.0f) ? __fdiv_rn(num, den) : sc.c0[tid];
-        sc.ic[tid] = __frcp_rn(c);
+        const float ic = __frcp_rn(c);
+        sc.ic[tid] = ic;
         sc.cold[tid] = c;
+        // the largest code of the column is rint(max|y| * fl(1/c)): clamp needed
+        // only if that exceeds qmax (exact product in fp64)
+        if ((double)sc.colmax[tid] * (double)ic >= (double)Q + 0.5) sc.need_clamp = 1;
     }
     __syncthreads();
-}
-
-// Final code of y with 1/c: the fp32 bits of kMagic + 2^(B-1) + z, z clamped
-// to [-qmax, qmax]; the low B bits are the stored field z + 2^(B-1).
-template <int B>
-__device__ __forceinline__ int2 final_codes(float2 y, float2 ic) {
-    constexpr int Q = (1 << (B - 1)) - 1;
-    constexpr int OFF = 1 << (B - 1);
-    constexpr float MG2 = kMagic + (float)OFF;
-    constexpr int LO = 0x4B400000 + OFF - Q;
-    constexpr int HI = 0x4B400000 + OFF + Q;
-    const float2 t = fma2(y, ic, make_float2(MG2, MG2));
-    int T0 = __float_as_int(t.x), T1 = __float_as_int(t.y);
-    T0 = min(max(T0, LO), HI);
-    T1 = min(max(T1, LO), HI);
-    return make_int2(T0, T1);
 }
 
 // Refit and pack into the record at `rec` (global): codes, r, c.
@@ -296,31 +361,41 @@ template <int D, int B>
 __device__ void fit_pack(float (&S)[D / 8][4], uint8_t *rec, Scratch<D> &sc, int tid) {
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES;
-    const int g = tid / LANES, l = tid % LANES;
+    constexpr int Q = (1 << (B - 1)) - 1;
+    constexpr int OFF = 1 << (B - 1);
+    constexpr float MG2 = kMagic + (float)OFF;
+    constexpr int LO = 0x4B400000 + OFF - Q;
+    constexpr int HI = 0x4B400000 + OFF + Q;
+    const int l = tid % LANES;
     const int j0 = 4 * l;
     const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
     float *rec_r = reinterpret_cast<float *>(rec + codes_bytes);
     float *rec_c = rec_r + D;
-    float rr[RT];
-    fit_scales<D, B>(S, rr, sc, tid);
-#pragma unroll
-    for (int r = 0; r < RT; ++r)
-        if (l == (r % LANES)) rec_r[g * RT + r] = rr[r];
+    fit_scales<D, B>(S, sc, tid, rec_r);
     if (tid < D) rec_c[tid] = sc.cold[tid];
+    const bool clampit = sc.need_clamp != 0;
     uint32_t W[Stream<D, B>::NW];
 #pragma unroll
     for (int i = 0; i < Stream<D, B>::NW; ++i) W[i] = 0u;
+    const float4 ic4 = *reinterpret_cast<const float4 *>(&sc.ic[j0]);
+    const float2 mg2 = make_float2(MG2, MG2);
 #pragma unroll
     for (int hp = 0; hp < 2; ++hp) {
-        const int jA = j0 + 2 * hp;
-        const float2 ic = make_float2(sc.ic[jA], sc.ic[jA + 1]);
+        const float2 ic = hp ? make_float2(ic4.z, ic4.w) : make_float2(ic4.x, ic4.y);
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
-            const int2 T = final_codes<B>(make_float2(S[r][2 * hp], S[r][2 * hp + 1]), ic);
-            field_put<B>(W, 4 * r + 2 * hp, (uint32_t)T.x & ((1u << B) - 1u));
-            field_put<B>(W, 4 * r + 2 * hp + 1, (uint32_t)T.y & ((1u << B) - 1u));
+            const float2 t = fma2(make_float2(S[r][2 * hp], S[r][2 * hp + 1]), ic, mg2);
+            int T0 = __float_as_int(t.x), T1 = __float_as_int(t.y);
+            if (clampit) {
+                T0 = min(max(T0, LO), HI);
+                T1 = min(max(T1, LO), HI);
+            }
+            field_acc<B>(W, 4 * r + 2 * hp, (uint32_t)T0);
+            field_acc<B>(W, 4 * r + 2 * hp + 1, (uint32_t)T1);
         }
     }
+#pragma unroll
+    for (int w = 0; w < Stream<D, B>::WORDS; ++w) W[w] -= pack_correction<D, B>(w);
     store_stream<D, B>(rec, tid, W);
 }
 
@@ -356,23 +431,21 @@ __device__ __forceinline__ void load_pivot(const uint8_t *rec, int tid, float (&
     }
 }
 
-// Block-wide fp64 sums of three values (every thread passes its share, 0 if none).
+// Per-band fp64 sums of three per-row values: thread tid holds row tid (0 for
+// tid >= D); rows of band g are tid in [g RT, g RT + RT).  All threads call it.
 template <int D>
-__device__ __forceinline__ void block_sum3(Scratch<D> &sc, int tid, double x0, double x1, double x2) {
-    constexpr int NWP = (2 * D) / 32;
-    x0 = lane_sum_f64<32>(x0);
-    x1 = lane_sum_f64<32>(x1);
-    x2 = lane_sum_f64<32>(x2);
-    if ((tid & 31) == 0) {
-        sc.red[0][tid >> 5] = x0;
-        sc.red[1][tid >> 5] = x1;
-        sc.red[2][tid >> 5] = x2;
+__device__ __forceinline__ void band_sums(Scratch<D> &sc, int tid, double x0, double x1, double x2) {
+    constexpr int RT = D / 8;
+#pragma unroll
+    for (int m = 1; m < RT; m <<= 1) {
+        x0 += __shfl_xor_sync(0xffffffffu, x0, m);
+        x1 += __shfl_xor_sync(0xffffffffu, x1, m);
+        x2 += __shfl_xor_sync(0xffffffffu, x2, m);
     }
-    __syncthreads();
-    if (tid < 3) {
-        double s = 0.0;
-        for (int w = 0; w < NWP; ++w) s += sc.red[tid][w];
-        sc.cst[tid] = s;
+    if (tid < D && (tid % RT) == 0) {
+        sc.bandK[tid / RT] = x0;
+        sc.bandQ[tid / RT] = x1;
+        sc.bandQK[tid / RT] = x2;
     }
 }
 
@@ -398,6 +471,7 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
     const float beta = a.beta[row];
 
     // per-row and per-column parameters
+    double bk = 0.0, bq = 0.0, bqk = 0.0;
     if (tid < D) {
         const int i = tid;
         const float ai = __fmul_rn(alpha, st_r[i]);
@@ -410,21 +484,17 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
             sc.wbar[i] = a.t.wbar[(size_t)gl * D + i];
         }
         if (KIND == kFitPack) sc.wv[i] = xs[i];
-    }
-    if (KIND != kFitPack) {
-        double kc = 0.0, qc = 0.0, qk = 0.0;
-        if (tid < D) {
-            const int i = tid;
-            const double ka = (double)ks[i] * (double)sc.a[i];
-            const double qa = (double)qs[i] * (double)sc.a[i];
+        if (KIND != kFitPack) {
+            const double ka = (double)ks[i] * (double)ai;
+            const double qa = (double)qs[i] * (double)ai;
             sc.kap[i] = ka * kTwoM169;
             sc.qt[i] = qa * kTwoM169;
-            kc = ka * (double)(256 + OFF);
-            qc = qa * (double)(256 + OFF);
-            qk = (double)qs[i] * (double)ks[i];
+            bk = ka * (double)(256 + OFF);
+            bq = qa * (double)(256 + OFF);
+            bqk = (double)qs[i] * (double)ks[i];
         }
-        block_sum3<D>(sc, tid, kc, qc, qk);
     }
+    if (KIND != kFitPack) band_sums<D>(sc, tid, bk, bq, bqk);
     __syncthreads();
 
     uint32_t W[Stream<D, B>::NW];
@@ -434,53 +504,71 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
     double accU[4] = {0.0, 0.0, 0.0, 0.0}, accO[4] = {0.0, 0.0, 0.0, 0.0};
     float2 cp01, cp23;
     if (KIND != kDecode) {
-        cp01 = make_float2(sc.cpr[j0], sc.cpr[j0 + 1]);
-        cp23 = make_float2(sc.cpr[j0 + 2], sc.cpr[j0 + 3]);
+        const float4 c4 = *reinterpret_cast<const float4 *>(&sc.cpr[j0]);
+        cp01 = make_float2(c4.x, c4.y);
+        cp23 = make_float2(c4.z, c4.w);
     }
+    constexpr float ZB = 8388608.0f + (float)OFF * 4096.0f;
+    const float2 nzb = make_float2(-ZB, -ZB);
 #pragma unroll
-    for (int r = 0; r < RT; ++r) {
+    for (int r = 0; r < RT; r += 2) {
         const int i = g * RT + r;
-        uint32_t X[4];
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) X[jj] = field_x<B>(W, 4 * r + jj);
+        double2 kap2, qt2;
         if (KIND != kFitPack) {
-            const double kap = sc.kap[i], qt = sc.qt[i];
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const double d = x_as_f64(X[jj]);
-                accU[jj] = fma(kap, d, accU[jj]);
-                accO[jj] = fma(qt, d, accO[jj]);
-            }
+            kap2 = *reinterpret_cast<const double2 *>(&sc.kap[i]);
+            qt2 = *reinterpret_cast<const double2 *>(&sc.qt[i]);
         }
-        if (KIND != kDecode) {
-            const float ai = sc.a[i];
-            const float2 a2 = make_float2(ai, ai);
-            const float2 A01 = mul2(a2, cp01);
-            const float2 A23 = mul2(a2, cp23);
-            const float2 z01 = make_float2(x_as_zscaled<B>(X[0]), x_as_zscaled<B>(X[1]));
-            const float2 z23 = make_float2(x_as_zscaled<B>(X[2]), x_as_zscaled<B>(X[3]));
-            const float2 s01 = mul2(A01, z01);
-            const float2 s23 = mul2(A23, z23);
-            S[r][0] = s01.x; S[r][1] = s01.y; S[r][2] = s23.x; S[r][3] = s23.y;
+        float2 a2r;
+        if (KIND != kDecode) a2r = *reinterpret_cast<const float2 *>(&sc.a[i]);
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            uint32_t X[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) X[jj] = field_x<B>(W, 4 * (r + rr) + jj);
+            if (KIND != kFitPack) {
+                const double kap = rr ? kap2.y : kap2.x, qt = rr ? qt2.y : qt2.x;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const double d = x_as_f64(X[jj]);
+                    accU[jj] = fma(kap, d, accU[jj]);
+                    accO[jj] = fma(qt, d, accO[jj]);
+                }
+            }
+            if (KIND != kDecode) {
+                const float ai = rr ? a2r.y : a2r.x;
+                const float2 a2 = make_float2(ai, ai);
+                const float2 A01 = mul2(a2, cp01);
+                const float2 A23 = mul2(a2, cp23);
+                const float2 z01 = add2(make_float2(__uint_as_float(X[0]), __uint_as_float(X[1])), nzb);
+                const float2 z23 = add2(make_float2(__uint_as_float(X[2]), __uint_as_float(X[3])), nzb);
+                const float2 s01 = mul2(A01, z01);
+                const float2 s23 = mul2(A23, z23);
+                S[r + rr][0] = s01.x; S[r + rr][1] = s01.y; S[r + rr][2] = s23.x; S[r + rr][3] = s23.y;
+            }
         }
     }
 
     if (KIND != kFitPack) {
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            sc.pU[g][j0 + jj] = accU[jj];
-            sc.pO[g][j0 + jj] = accO[jj];
-        }
+        *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0]) = make_double2(accU[0], accU[1]);
+        *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0 + 2]) = make_double2(accU[2], accU[3]);
+        *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0]) = make_double2(accO[0], accO[1]);
+        *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0 + 2]) = make_double2(accO[2], accO[3]);
         __syncthreads();
         if (tid < D) {
             const int j = tid;
-            double su = 0.0, so = 0.0;
+            double su = 0.0, so = 0.0, kc = 0.0, qc = 0.0, qk = 0.0;
 #pragma unroll
-            for (int b = 0; b < 8; ++b) { su += sc.pU[b][j]; so += sc.pO[b][j]; }
+            for (int b = 0; b < 8; ++b) {
+                su += sc.u.col.pU[b][j];
+                so += sc.u.col.pO[b][j];
+                kc += sc.bandK[b];
+                qc += sc.bandQ[b];
+                qk += sc.bandQK[b];
+            }
             const double cj = (double)sc.cold[j];
-            const float u = __double2float_rn(cj * (su - sc.cst[0]));
+            const float u = __double2float_rn(cj * (su - kc));
             const float w = __fmul_rn(beta, __fsub_rn(vs[j], u));
-            const float o = __double2float_rn(cj * (so - sc.cst[1]) + sc.cst[2] * (double)w);
+            const float o = __double2float_rn(cj * (so - qc) + qk * (double)w);
             a.o[(size_t)row * D + j] = o;
             if (KIND == kDecode) a.w[(size_t)row * D + j] = w;
             else sc.wv[j] = w;
@@ -489,15 +577,20 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
     }
 
     if (KIND != kDecode) {
-        const float2 w01 = make_float2(sc.wv[j0], sc.wv[j0 + 1]);
-        const float2 w23 = make_float2(sc.wv[j0 + 2], sc.wv[j0 + 3]);
+        const float4 w4 = *reinterpret_cast<const float4 *>(&sc.wv[j0]);
+        const float2 w01 = make_float2(w4.x, w4.y);
+        const float2 w23 = make_float2(w4.z, w4.w);
 #pragma unroll
-        for (int r = 0; r < RT; ++r) {
-            const float ki = sc.kf[g * RT + r];
-            const float2 k2 = make_float2(ki, ki);
-            const float2 s01 = fma2(k2, w01, make_float2(S[r][0], S[r][1]));
-            const float2 s23 = fma2(k2, w23, make_float2(S[r][2], S[r][3]));
-            S[r][0] = s01.x; S[r][1] = s01.y; S[r][2] = s23.x; S[r][3] = s23.y;
+        for (int r = 0; r < RT; r += 2) {
+            const float2 k2r = *reinterpret_cast<const float2 *>(&sc.kf[g * RT + r]);
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const float ki = rr ? k2r.y : k2r.x;
+                const float2 k2 = make_float2(ki, ki);
+                const float2 s01 = fma2(k2, w01, make_float2(S[r + rr][0], S[r + rr][1]));
+                const float2 s23 = fma2(k2, w23, make_float2(S[r + rr][2], S[r + rr][3]));
+                S[r + rr][0] = s01.x; S[r + rr][1] = s01.y; S[r + rr][2] = s23.x; S[r + rr][3] = s23.y;
+            }
         }
         fit_pack<D, B>(S, rec_g, sc, tid);
     }
@@ -516,19 +609,17 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
     const float *xs = vs + D;
     const float alpha = a.alpha[row];
     const float beta = a.beta[row];
+    double bqk = 0.0;
     if (tid < D) {
         sc.kf[tid] = ks[tid];
         if (KIND == kFitPack) sc.wv[tid] = xs[tid];
-    }
-    if (KIND != kFitPack) {
-        double qk = 0.0;
-        if (tid < D) {
+        if (KIND != kFitPack) {
             sc.kap[tid] = (double)ks[tid] * (double)alpha;
             sc.qt[tid] = (double)qs[tid] * (double)alpha;
-            qk = (double)qs[tid] * (double)ks[tid];
+            bqk = (double)qs[tid] * (double)ks[tid];
         }
-        block_sum3<D>(sc, tid, 0.0, 0.0, qk);
     }
+    if (KIND != kFitPack) band_sums<D>(sc, tid, 0.0, 0.0, bqk);
     __syncthreads();
     float S[RT][4];
     load_pivot<D>(rec_g, tid, S);
@@ -547,18 +638,18 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
         }
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-            sc.pU[g][j0 + jj] = accU[jj];
-            sc.pO[g][j0 + jj] = accO[jj];
+            sc.u.col.pU[g][j0 + jj] = accU[jj];
+            sc.u.col.pO[g][j0 + jj] = accO[jj];
         }
         __syncthreads();
         if (tid < D) {
             const int j = tid;
-            double su = 0.0, so = 0.0;
+            double su = 0.0, so = 0.0, qk = 0.0;
 #pragma unroll
-            for (int b = 0; b < 8; ++b) { su += sc.pU[b][j]; so += sc.pO[b][j]; }
+            for (int b = 0; b < 8; ++b) { su += sc.u.col.pU[b][j]; so += sc.u.col.pO[b][j]; qk += sc.bandQK[b]; }
             const float u = __double2float_rn(su);
             const float w = __fmul_rn(beta, __fsub_rn(vs[j], u));
-            const float o = __double2float_rn(so + sc.cst[2] * (double)w);
+            const float o = __double2float_rn(so + qk * (double)w);
             a.o[(size_t)row * D + j] = o;
             if (KIND == kDecode) a.w[(size_t)row * D + j] = w;
             else sc.wv[j] = w;
@@ -587,7 +678,7 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
 // Persistent pipeline kernel.
 // ---------------------------------------------------------------------------
 template <int D, int KIND>
-__global__ void __launch_bounds__(2 * D) k_step(Args a) {
+__global__ void __launch_bounds__(2 * D, 2) k_step(Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x;
     uint8_t *stages = smem;
@@ -763,6 +854,10 @@ __device__ void dist_uniform(const float *Sg, int gl, int m, int n_bits, double 
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES;
     constexpr int OFF = 1 << (B - 1);
+    constexpr int Q = (1 << (B - 1)) - 1;
+    constexpr float MG2 = kMagic + (float)OFF;
+    constexpr int LO = 0x4B400000 + OFF - Q;
+    constexpr int HI = 0x4B400000 + OFF + Q;
     const int g = tid / LANES, l = tid % LANES;
     const int j0 = 4 * l;
     float S[RT][4];
@@ -771,25 +866,23 @@ __device__ void dist_uniform(const float *Sg, int gl, int m, int n_bits, double 
         const float4 v = *reinterpret_cast<const float4 *>(Sg + (size_t)(g * RT + r) * D + j0);
         S[r][0] = v.x; S[r][1] = v.y; S[r][2] = v.z; S[r][3] = v.w;
     }
-    float rr[RT];
-    fit_scales<D, B>(S, rr, sc, tid);
-    const float c0 = sc.cold[j0], c1 = sc.cold[j0 + 1], c2 = sc.cold[j0 + 2], c3 = sc.cold[j0 + 3];
-    const float2 ic01 = make_float2(sc.ic[j0], sc.ic[j0 + 1]);
-    const float2 ic23 = make_float2(sc.ic[j0 + 2], sc.ic[j0 + 3]);
+    fit_scales<D, B>(S, sc, tid, nullptr);
+    float cc[4], icc[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) { cc[jj] = sc.cold[j0 + jj]; icc[jj] = sc.ic[j0 + jj]; }
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
         const int i = g * RT + r;
-        const int2 T01 = final_codes<B>(make_float2(S[r][0], S[r][1]), ic01);
-        const int2 T23 = final_codes<B>(make_float2(S[r][2], S[r][3]), ic23);
-        const int zb = 0x4B400000 + OFF;
-        const float z[4] = {(float)(T01.x - zb), (float)(T01.y - zb), (float)(T23.x - zb), (float)(T23.y - zb)};
-        const float cc[4] = {c0, c1, c2, c3};
+        const float ri = sc.rowr[i];
         const float4 orig = *reinterpret_cast<const float4 *>(Sg + (size_t)i * D + j0);
         const float o4[4] = {orig.x, orig.y, orig.z, orig.w};
         double e = 0.0;
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-            const float sh = __fmul_rn(__fmul_rn(rr[r], cc[jj]), z[jj]);
+            const float t = __fmaf_rn(S[r][jj], icc[jj], MG2);
+            const int T = min(max(__float_as_int(t), LO), HI);
+            const float z = (float)(T - (0x4B400000 + OFF));
+            const float sh = __fmul_rn(__fmul_rn(ri, cc[jj]), z);
             const double d = (double)sh - (double)o4[jj];
             e = fma(d, d, e);
         }

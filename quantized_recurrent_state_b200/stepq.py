@@ -173,18 +173,30 @@ class Context:
         self._h = h
         self.n_slots = n_slots
 
+    def _after_caller(self):
+        """Order the context's main stream after the caller's current torch
+        stream, so that tensors produced there are complete before the
+        library's kernels read or write them."""
+        import torch
+        cur = torch.cuda.current_stream()
+        if cur.cuda_stream != self.main.cuda_stream:
+            self.main.wait_stream(cur)
+
     def workspace_bytes(self, n_req: int, n_layers: int) -> int:
         return int(lib().stepq_workspace_bytes(self._h, n_req, n_layers))
 
     def requant_pack(self, pool, slots, n_req, lb, le, S):
+        self._after_caller()
         return _check(lib().stepq_requant_pack(self._h, _ptr(pool), _ptr(slots), n_req, lb, le, _ptr(S)))
 
     def decode_step(self, pool, slots, n_req, lb, le, q, k, v, alpha, beta, o, workspace):
+        self._after_caller()
         return _check(lib().stepq_decode_step(self._h, _ptr(pool), _ptr(slots), n_req, lb, le, _ptr(q),
                                               _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o),
                                               _ptr(workspace)))
 
     def decode_step_fused(self, pool, slots, n_req, lb, le, q, k, v, alpha, beta, o):
+        self._after_caller()
         return _check(lib().stepq_decode_step_fused(self._h, _ptr(pool), _ptr(slots), n_req, lb, le,
                                                     _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                                     _ptr(o)))
@@ -193,6 +205,7 @@ class Context:
         """The two-stream step without a workspace argument: for callers that
         cannot allocate device memory.  The hand-off values live in a fixed
         8 MiB array inside the library (shared by all calls on the device)."""
+        self._after_caller()
         return _check(lib().stepq_decode_step_noalloc(self._h, _ptr(pool), _ptr(slots), n_req, lb, le,
                                                       _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                                       _ptr(o)))
@@ -201,18 +214,22 @@ class Context:
         return _check(lib().stepq_sync(self._h, timeout_ms))
 
     def unpack(self, pool, slots, n_req, lb, le, S):
+        self._after_caller()
         return _check(lib().stepq_unpack(self._h, _ptr(pool), _ptr(slots), n_req, lb, le, _ptr(S)))
 
     def fp32_decode_step(self, S_pool, slots, n_req, lb, le, q, k, v, alpha, beta, o):
+        self._after_caller()
         return _check(lib().stepq_fp32_decode_step(self._h, _ptr(S_pool), _ptr(slots), n_req, lb, le,
                                                    _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                                    _ptr(o)))
 
     def calib_accumulate(self, n_req, lb, le, q, k, alpha, beta, omega_acc, lsum_acc):
+        self._after_caller()
         return _check(lib().stepq_calib_accumulate(self._h, n_req, lb, le, _ptr(q), _ptr(k), _ptr(alpha),
                                                    _ptr(beta), _ptr(omega_acc), _ptr(lsum_acc)))
 
     def calib_distortion(self, n_req, lb, le, S, wbar, bits, dist_acc):
+        self._after_caller()
         b = (ctypes.c_int * len(bits))(*[int(x) for x in bits])
         return _check(lib().stepq_calib_distortion(self._h, n_req, lb, le, _ptr(S), _ptr(wbar), b,
                                                    len(bits), _ptr(dist_acc)))
