@@ -153,6 +153,26 @@ __device__ __forceinline__ void load_stream(const uint8_t *blk, int t, uint32_t 
     }
 }
 
+// Load chunk c of thread t's code stream into W (RT bytes per chunk).
+template <int D, int B>
+__device__ __forceinline__ void load_chunk(const uint8_t *blk, int t, int c, uint32_t (&W)[Stream<D, B>::NW]) {
+    constexpr int RT = D / 8, NT = 2 * D;
+    const uint8_t *p = blk + (size_t)(c * NT + t) * RT;
+    if constexpr (RT == 16) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(p);
+        W[4 * c] = v.x; W[4 * c + 1] = v.y; W[4 * c + 2] = v.z; W[4 * c + 3] = v.w;
+    } else if constexpr (RT == 8) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(p);
+        W[2 * c] = v.x; W[2 * c + 1] = v.y;
+    } else if constexpr (RT == 4) {
+        W[c] = *reinterpret_cast<const uint32_t *>(p);
+    } else {
+        const uint32_t v = *reinterpret_cast<const uint16_t *>(p);
+        if (c & 1) W[c >> 1] |= v << 16;
+        else W[c >> 1] = v;
+    }
+}
+
 template <int D, int B>
 __device__ __forceinline__ void store_stream(uint8_t *blk, int t, const uint32_t (&W)[Stream<D, B>::NW]) {
     constexpr int RT = D / 8, NT = 2 * D, NCH = B / 2;
@@ -202,37 +222,66 @@ struct PairTree {
     __device__ __forceinline__ float2 total() const { return s[LV - 1]; }
 };
 
-// Word-level packing: the final-code bits T = 0x4B400000 + 2^(B-1) + z are
-// added into the stream at their bit offsets, and the constant high parts are
-// removed per word at the end.
+// Packing of e = z + qmax in [0, 2 qmax] (the stored field is e + 1): e is
+// added into the stream at its bit offset, the +1 of every field is a
+// per-word constant folded in at the end.
 template <int D, int B>
-__host__ __device__ constexpr uint32_t pack_correction(int w) {
+__host__ __device__ constexpr uint32_t pack_ones(int w) {
     uint32_t c = 0;
     for (int p = 0; p < 4 * (D / 8); ++p) {
         const int bit = p * B;
-        if ((bit >> 5) == w) c += 0x4B400000u << (bit & 31);
+        if ((bit >> 5) == w && (bit & 31) + B <= 32) c += 1u << (bit & 31);
     }
     return c;
 }
 
+template <int D, int B, int W>
+struct PackOnes {
+    static constexpr uint32_t value = pack_ones<D, B>(W);
+};
+
+template <int D, int B, int W = 0>
+__device__ __forceinline__ void add_pack_ones(uint32_t *w) {
+    if constexpr (W < Stream<D, B>::WORDS) {
+        w[W] += PackOnes<D, B, W>::value;
+        add_pack_ones<D, B, W + 1>(w);
+    }
+}
+
 template <int B>
-__device__ __forceinline__ void field_acc(uint32_t *W, int p, uint32_t T) {
+__device__ __forceinline__ void field_acc(uint32_t *W, int p, uint32_t e) {
     const int bit = p * B;
     const int w = bit >> 5;
     const int s = bit & 31;
-    W[w] += T << s;
-    if (s + B > 32) W[w + 1] += (T & ((1u << B) - 1u)) >> (32 - s);
+    if (s + B <= 32) {
+        W[w] += e << s;
+    } else {  // a field split across two words carries its own +1
+        const uint32_t v = e + 1u;
+        W[w] += v << s;
+        W[w + 1] += v >> (32 - s);
+    }
+}
+
+// Final code as e = z + qmax, clamped to [0, 2 qmax], from t = fma(y, 1/c,
+// kMagic + 2^(B-1)): bits(t) = 0x4B400000 + 2^(B-1) + rint(y/c), and
+// |y/c| <= 2 qmax because the refit c is at least c0/2, so the difference
+// below cannot overflow.
+template <int B>
+__device__ __forceinline__ uint32_t final_e(float t) {
+    constexpr int Q = (1 << (B - 1)) - 1;
+    constexpr int LO = 0x4B400000 + (1 << (B - 1)) - Q;
+    return (uint32_t)__viaddmin_s32_relu(__float_as_int(t), -LO, 2 * Q);
 }
 
 // ---------------------------------------------------------------------------
-// Refit of the fp32 tile S held in registers (all rows at width B).  On
-// return S holds y = fl(S * fl(1/r)); sc.rowr[i] = r_i, sc.cold[j] = c_j,
-// sc.ic[j] = fl(1/c_j), sc.colmax[j] = max_i |y_ij|, sc.need_clamp != 0 iff
-// some final code needs the clamp.  rec_r (global, may be null) receives r.
-// Requires rho and wbar of the head in sc.rho / sc.wbar.
+// Refit of the fp32 tile S held in registers as column pairs (all rows at
+// width B).  On return S holds y = fl(S * fl(1/r)); sc.rowr[i] = r_i,
+// sc.cold[j] = c_j, sc.ic[j] = fl(1/c_j).  rec_r / rec_c (global, may be
+// null) receive r and c.  Requires rho and wbar of the head in sc.rho /
+// sc.wbar.
 // ---------------------------------------------------------------------------
 template <int D, int B>
-__device__ void fit_scales(float (&S)[D / 8][4], Scratch<D> &sc, int tid, float *rec_r) {
+__device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, float *rec_r, float *rec_c) {
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES, RS = Scratch<D>::RS, HALF = LANES / 2;
     constexpr int Q = (1 << (B - 1)) - 1;
@@ -244,7 +293,7 @@ __device__ void fit_scales(float (&S)[D / 8][4], Scratch<D> &sc, int tid, float 
     float *rs = &sc.u.rsum[g][0][0];
 #pragma unroll
     for (int r = 0; r < RT; ++r)
-        rs[r * RS + l] = (fabsf(S[r][0]) + fabsf(S[r][1])) + (fabsf(S[r][2]) + fabsf(S[r][3]));
+        rs[r * RS + l] = (fabsf(S[r][0].x) + fabsf(S[r][0].y)) + (fabsf(S[r][1].x) + fabsf(S[r][1].y));
     __syncwarp();
     {
         const int rr = l >> 1, hh = l & 1;
@@ -275,26 +324,23 @@ __device__ void fit_scales(float (&S)[D / 8][4], Scratch<D> &sc, int tid, float 
         }
     }
     __syncwarp();
-    // 2. y = fl(S * (1/r)) in place
-#pragma unroll
-    for (int r = 0; r < RT; r += 2) {
-        const float4 f = *reinterpret_cast<const float4 *>(&sc.rowfit[g * RT + r]);
-        const float2 i0 = make_float2(f.x, f.x), i1 = make_float2(f.z, f.z);
-        const float2 a01 = mul2(make_float2(S[r][0], S[r][1]), i0);
-        const float2 a23 = mul2(make_float2(S[r][2], S[r][3]), i0);
-        const float2 b01 = mul2(make_float2(S[r + 1][0], S[r + 1][1]), i1);
-        const float2 b23 = mul2(make_float2(S[r + 1][2], S[r + 1][3]), i1);
-        S[r][0] = a01.x; S[r][1] = a01.y; S[r][2] = a23.x; S[r][3] = a23.y;
-        S[r + 1][0] = b01.x; S[r + 1][1] = b01.y; S[r + 1][2] = b23.x; S[r + 1][3] = b23.y;
-    }
-    // 3. column absmax -> c0
+    // 2. y = fl(S * (1/r)) in place; 3. column absmax partials
     {
-        float m[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        float2 m01 = make_float2(0.0f, 0.0f), m23 = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int r = 0; r < RT; ++r)
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) m[jj] = fmaxf(m[jj], fabsf(S[r][jj]));
-        *reinterpret_cast<float4 *>(&sc.pf0[g][j0]) = make_float4(m[0], m[1], m[2], m[3]);
+        for (int r = 0; r < RT; r += 2) {
+            const float4 f = *reinterpret_cast<const float4 *>(&sc.rowfit[g * RT + r]);
+            const float2 i0 = make_float2(f.x, f.x), i1 = make_float2(f.z, f.z);
+            S[r][0] = mul2(S[r][0], i0);
+            S[r][1] = mul2(S[r][1], i0);
+            S[r + 1][0] = mul2(S[r + 1][0], i1);
+            S[r + 1][1] = mul2(S[r + 1][1], i1);
+            m01.x = fmaxf(m01.x, fmaxf(fabsf(S[r][0].x), fabsf(S[r + 1][0].x)));
+            m01.y = fmaxf(m01.y, fmaxf(fabsf(S[r][0].y), fabsf(S[r + 1][0].y)));
+            m23.x = fmaxf(m23.x, fmaxf(fabsf(S[r][1].x), fabsf(S[r + 1][1].x)));
+            m23.y = fmaxf(m23.y, fmaxf(fabsf(S[r][1].y), fabsf(S[r + 1][1].y)));
+        }
+        *reinterpret_cast<float4 *>(&sc.pf0[g][j0]) = make_float4(m01.x, m01.y, m23.x, m23.y);
     }
     __syncthreads();
     if (tid < D) {
@@ -304,8 +350,6 @@ __device__ void fit_scales(float (&S)[D / 8][4], Scratch<D> &sc, int tid, float 
         const float c0 = (m == 0.0f) ? 1.0f : __fdiv_rn(m, (float)Q);
         sc.c0[tid] = c0;
         sc.ic0[tid] = __frcp_rn(c0);
-        sc.colmax[tid] = m;
-        if (tid == 0) sc.need_clamp = 0;
     }
     __syncthreads();
     // 4. z0 and the weighted least-squares sums (pairwise over rows)
@@ -324,9 +368,8 @@ __device__ void fit_scales(float (&S)[D / 8][4], Scratch<D> &sc, int tid, float 
             for (int r = 0; r < RT; ++r) {
                 if ((r & 1) == 0) f = *reinterpret_cast<const float4 *>(&sc.rowfit[g * RT + r]);
                 const float bwr = (r & 1) ? f.w : f.y;
-                const float2 y = make_float2(S[r][2 * hp], S[r][2 * hp + 1]);
-                const float2 t = fma2(y, ic, mg);
-                const float2 z0 = add2(t, nmg);
+                const float2 y = S[r][hp];
+                const float2 z0 = add2(fma2(y, ic, mg), nmg);
                 const float2 b2 = make_float2(bwr, bwr);
                 // fl(b * p) written as fma(b, p, -0) with a run-time -0: the
                 // product is rounded once and cannot be contracted into the
@@ -346,34 +389,26 @@ __device__ void fit_scales(float (&S)[D / 8][4], Scratch<D> &sc, int tid, float 
         const float num = tree_sum1<8>(xn);
         const float den = tree_sum1<8>(xd);
         const float c = (den > 0.0f) ? __fdiv_rn(num, den) : sc.c0[tid];
-        const float ic = __frcp_rn(c);
-        sc.ic[tid] = ic;
+        sc.ic[tid] = __frcp_rn(c);
         sc.cold[tid] = c;
-        // the largest code of the column is rint(max|y| * fl(1/c)): clamp needed
-        // only if that exceeds qmax (exact product in fp64)
-        if ((double)sc.colmax[tid] * (double)ic >= (double)Q + 0.5) sc.need_clamp = 1;
+        if (rec_c) rec_c[tid] = c;
     }
     __syncthreads();
 }
 
 // Refit and pack into the record at `rec` (global): codes, r, c.
 template <int D, int B>
-__device__ void fit_pack(float (&S)[D / 8][4], uint8_t *rec, Scratch<D> &sc, int tid) {
+__device__ void fit_pack(float2 (&S)[D / 8][2], uint8_t *rec, Scratch<D> &sc, int tid) {
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES;
-    constexpr int Q = (1 << (B - 1)) - 1;
     constexpr int OFF = 1 << (B - 1);
     constexpr float MG2 = kMagic + (float)OFF;
-    constexpr int LO = 0x4B400000 + OFF - Q;
-    constexpr int HI = 0x4B400000 + OFF + Q;
     const int l = tid % LANES;
     const int j0 = 4 * l;
     const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
     float *rec_r = reinterpret_cast<float *>(rec + codes_bytes);
     float *rec_c = rec_r + D;
-    fit_scales<D, B>(S, sc, tid, rec_r);
-    if (tid < D) rec_c[tid] = sc.cold[tid];
-    const bool clampit = sc.need_clamp != 0;
+    fit_scales<D, B>(S, sc, tid, rec_r, rec_c);
     uint32_t W[Stream<D, B>::NW];
 #pragma unroll
     for (int i = 0; i < Stream<D, B>::NW; ++i) W[i] = 0u;
@@ -384,31 +419,25 @@ __device__ void fit_pack(float (&S)[D / 8][4], uint8_t *rec, Scratch<D> &sc, int
         const float2 ic = hp ? make_float2(ic4.z, ic4.w) : make_float2(ic4.x, ic4.y);
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
-            const float2 t = fma2(make_float2(S[r][2 * hp], S[r][2 * hp + 1]), ic, mg2);
-            int T0 = __float_as_int(t.x), T1 = __float_as_int(t.y);
-            if (clampit) {
-                T0 = min(max(T0, LO), HI);
-                T1 = min(max(T1, LO), HI);
-            }
-            field_acc<B>(W, 4 * r + 2 * hp, (uint32_t)T0);
-            field_acc<B>(W, 4 * r + 2 * hp + 1, (uint32_t)T1);
+            const float2 t = fma2(S[r][hp], ic, mg2);
+            field_acc<B>(W, 4 * r + 2 * hp, final_e<B>(t.x));
+            field_acc<B>(W, 4 * r + 2 * hp + 1, final_e<B>(t.y));
         }
     }
-#pragma unroll
-    for (int w = 0; w < Stream<D, B>::WORDS; ++w) W[w] -= pack_correction<D, B>(w);
+    add_pack_ones<D, B>(W);
     store_stream<D, B>(rec, tid, W);
 }
 
 // Pivot head (binary16 tile): S_t -> fp16 RNE, written in place.
 template <int D>
-__device__ __forceinline__ void store_pivot(float (&S)[D / 8][4], uint8_t *rec, int tid) {
+__device__ __forceinline__ void store_pivot(float2 (&S)[D / 8][2], uint8_t *rec, int tid) {
     using G = Geo<D>;
     const int g = tid / G::LANES, l = tid % G::LANES;
 #pragma unroll
     for (int r = 0; r < G::RT; ++r) {
         const int i = g * G::RT + r;
-        const __half2 h01 = __floats2half2_rn(S[r][0], S[r][1]);
-        const __half2 h23 = __floats2half2_rn(S[r][2], S[r][3]);
+        const __half2 h01 = __float22half2_rn(S[r][0]);
+        const __half2 h23 = __float22half2_rn(S[r][1]);
         uint2 v;
         v.x = *reinterpret_cast<const uint32_t *>(&h01);
         v.y = *reinterpret_cast<const uint32_t *>(&h23);
@@ -417,25 +446,25 @@ __device__ __forceinline__ void store_pivot(float (&S)[D / 8][4], uint8_t *rec, 
 }
 
 template <int D>
-__device__ __forceinline__ void load_pivot(const uint8_t *rec, int tid, float (&h)[D / 8][4]) {
+__device__ __forceinline__ void load_pivot(const uint8_t *rec, int tid, float2 (&h)[D / 8][2]) {
     using G = Geo<D>;
     const int g = tid / G::LANES, l = tid % G::LANES;
 #pragma unroll
     for (int r = 0; r < G::RT; ++r) {
         const int i = g * G::RT + r;
         const uint2 v = *reinterpret_cast<const uint2 *>(rec + ((size_t)i * D + 4 * l) * 2);
-        const __half2 h01 = *reinterpret_cast<const __half2 *>(&v.x);
-        const __half2 h23 = *reinterpret_cast<const __half2 *>(&v.y);
-        const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-        h[r][0] = f01.x; h[r][1] = f01.y; h[r][2] = f23.x; h[r][3] = f23.y;
+        h[r][0] = __half22float2(*reinterpret_cast<const __half2 *>(&v.x));
+        h[r][1] = __half22float2(*reinterpret_cast<const __half2 *>(&v.y));
     }
 }
 
 // Per-band fp64 sums of three per-row values: thread tid holds row tid (0 for
-// tid >= D); rows of band g are tid in [g RT, g RT + RT).  All threads call it.
+// tid >= D); rows of band g are tid in [g RT, g RT + RT).  For D >= 32 only
+// the warps holding rows take part; below that the whole warp does.
 template <int D>
 __device__ __forceinline__ void band_sums(Scratch<D> &sc, int tid, double x0, double x1, double x2) {
     constexpr int RT = D / 8;
+    if (D >= 32 && tid >= D) return;
 #pragma unroll
     for (int m = 1; m < RT; m <<= 1) {
         x0 += __shfl_xor_sync(0xffffffffu, x0, m);
@@ -446,6 +475,29 @@ __device__ __forceinline__ void band_sums(Scratch<D> &sc, int tid, double x0, do
         sc.bandK[tid / RT] = x0;
         sc.bandQ[tid / RT] = x1;
         sc.bandQK[tid / RT] = x2;
+    }
+}
+
+// Column phase of the decode: u, w, o of column j from the band partials
+// (already relative to the offset-binary bias), two threads per column.
+template <int D, int KIND>
+__device__ __forceinline__ void finish_columns(const Args &a, Scratch<D> &sc, int tid, int row, float beta,
+                                               const float *vs, bool scaled) {
+    const int j = tid >> 1, h = tid & 1, b0 = 4 * h;
+    double su = (sc.u.col.pU[b0][j] + sc.u.col.pU[b0 + 1][j]) + (sc.u.col.pU[b0 + 2][j] + sc.u.col.pU[b0 + 3][j]);
+    double so = (sc.u.col.pO[b0][j] + sc.u.col.pO[b0 + 1][j]) + (sc.u.col.pO[b0 + 2][j] + sc.u.col.pO[b0 + 3][j]);
+    double qk = (sc.bandQK[b0] + sc.bandQK[b0 + 1]) + (sc.bandQK[b0 + 2] + sc.bandQK[b0 + 3]);
+    su += __shfl_xor_sync(0xffffffffu, su, 1);
+    so += __shfl_xor_sync(0xffffffffu, so, 1);
+    qk += __shfl_xor_sync(0xffffffffu, qk, 1);
+    const double cj = scaled ? (double)sc.cold[j] : 1.0;
+    const float u = __double2float_rn(cj * su);
+    const float w = __fmul_rn(beta, __fsub_rn(vs[j], u));
+    const float o = __double2float_rn(cj * so + qk * (double)w);
+    if (h == 0) {
+        a.o[(size_t)row * D + j] = o;
+        if (KIND == kDecode) a.w[(size_t)row * D + j] = w;
+        else sc.wv[j] = w;
     }
 }
 
@@ -498,9 +550,10 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
     __syncthreads();
 
     uint32_t W[Stream<D, B>::NW];
-    load_stream<D, B>(stage, tid, W);
+    W[Stream<D, B>::NW - 1] = 0u;
+    int loaded = -1;  // chunks are loaded as the rows reach them (fewer live registers)
 
-    float S[RT][4];
+    float2 S[RT][2];
     double accU[4] = {0.0, 0.0, 0.0, 0.0}, accO[4] = {0.0, 0.0, 0.0, 0.0};
     float2 cp01, cp23;
     if (KIND != kDecode) {
@@ -522,6 +575,14 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
         if (KIND != kDecode) a2r = *reinterpret_cast<const float2 *>(&sc.a[i]);
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
+            {
+                constexpr int CB = D / 8;  // chunk bytes
+                const int last = ((4 * (r + rr + 1) * B - 1) / 8) / CB;
+#pragma unroll
+                for (int c = 0; c < B / 2; ++c)
+                    if (c > loaded && c <= last) load_chunk<D, B>(stage, tid, c, W);
+                if (last > loaded) loaded = last;
+            }
             uint32_t X[4];
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) X[jj] = field_x<B>(W, 4 * (r + rr) + jj);
@@ -537,42 +598,23 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
             if (KIND != kDecode) {
                 const float ai = rr ? a2r.y : a2r.x;
                 const float2 a2 = make_float2(ai, ai);
-                const float2 A01 = mul2(a2, cp01);
-                const float2 A23 = mul2(a2, cp23);
                 const float2 z01 = add2(make_float2(__uint_as_float(X[0]), __uint_as_float(X[1])), nzb);
                 const float2 z23 = add2(make_float2(__uint_as_float(X[2]), __uint_as_float(X[3])), nzb);
-                const float2 s01 = mul2(A01, z01);
-                const float2 s23 = mul2(A23, z23);
-                S[r + rr][0] = s01.x; S[r + rr][1] = s01.y; S[r + rr][2] = s23.x; S[r + rr][3] = s23.y;
+                S[r + rr][0] = mul2(mul2(a2, cp01), z01);
+                S[r + rr][1] = mul2(mul2(a2, cp23), z23);
             }
         }
     }
 
     if (KIND != kFitPack) {
-        *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0]) = make_double2(accU[0], accU[1]);
-        *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0 + 2]) = make_double2(accU[2], accU[3]);
-        *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0]) = make_double2(accO[0], accO[1]);
-        *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0 + 2]) = make_double2(accO[2], accO[3]);
+        // remove this band's offset-binary bias, then hand the partials over
+        const double bK = sc.bandK[g], bQ = sc.bandQ[g];
+        *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0]) = make_double2(accU[0] - bK, accU[1] - bK);
+        *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0 + 2]) = make_double2(accU[2] - bK, accU[3] - bK);
+        *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0]) = make_double2(accO[0] - bQ, accO[1] - bQ);
+        *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0 + 2]) = make_double2(accO[2] - bQ, accO[3] - bQ);
         __syncthreads();
-        if (tid < D) {
-            const int j = tid;
-            double su = 0.0, so = 0.0, kc = 0.0, qc = 0.0, qk = 0.0;
-#pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                su += sc.u.col.pU[b][j];
-                so += sc.u.col.pO[b][j];
-                kc += sc.bandK[b];
-                qc += sc.bandQ[b];
-                qk += sc.bandQK[b];
-            }
-            const double cj = (double)sc.cold[j];
-            const float u = __double2float_rn(cj * (su - kc));
-            const float w = __fmul_rn(beta, __fsub_rn(vs[j], u));
-            const float o = __double2float_rn(cj * (so - qc) + qk * (double)w);
-            a.o[(size_t)row * D + j] = o;
-            if (KIND == kDecode) a.w[(size_t)row * D + j] = w;
-            else sc.wv[j] = w;
-        }
+        finish_columns<D, KIND>(a, sc, tid, row, beta, vs, true);
         if (KIND == kFused) __syncthreads();
     }
 
@@ -587,9 +629,8 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
             for (int rr = 0; rr < 2; ++rr) {
                 const float ki = rr ? k2r.y : k2r.x;
                 const float2 k2 = make_float2(ki, ki);
-                const float2 s01 = fma2(k2, w01, make_float2(S[r + rr][0], S[r + rr][1]));
-                const float2 s23 = fma2(k2, w23, make_float2(S[r + rr][2], S[r + rr][3]));
-                S[r + rr][0] = s01.x; S[r + rr][1] = s01.y; S[r + rr][2] = s23.x; S[r + rr][3] = s23.y;
+                S[r + rr][0] = fma2(k2, w01, S[r + rr][0]);
+                S[r + rr][1] = fma2(k2, w23, S[r + rr][1]);
             }
         }
         fit_pack<D, B>(S, rec_g, sc, tid);
@@ -621,7 +662,7 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
     }
     if (KIND != kFitPack) band_sums<D>(sc, tid, 0.0, 0.0, bqk);
     __syncthreads();
-    float S[RT][4];
+    float2 S[RT][2];
     load_pivot<D>(rec_g, tid, S);
     if (KIND != kFitPack) {
         double accU[4] = {0.0, 0.0, 0.0, 0.0}, accO[4] = {0.0, 0.0, 0.0, 0.0};
@@ -629,11 +670,11 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
         for (int r = 0; r < RT; ++r) {
             const int i = g * RT + r;
             const double kap = sc.kap[i], qt = sc.qt[i];
+            const double d[4] = {(double)S[r][0].x, (double)S[r][0].y, (double)S[r][1].x, (double)S[r][1].y};
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
-                const double d = (double)S[r][jj];
-                accU[jj] = fma(kap, d, accU[jj]);
-                accO[jj] = fma(qt, d, accO[jj]);
+                accU[jj] = fma(kap, d[jj], accU[jj]);
+                accO[jj] = fma(qt, d[jj], accO[jj]);
             }
         }
 #pragma unroll
@@ -642,18 +683,7 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
             sc.u.col.pO[g][j0 + jj] = accO[jj];
         }
         __syncthreads();
-        if (tid < D) {
-            const int j = tid;
-            double su = 0.0, so = 0.0, qk = 0.0;
-#pragma unroll
-            for (int b = 0; b < 8; ++b) { su += sc.u.col.pU[b][j]; so += sc.u.col.pO[b][j]; qk += sc.bandQK[b]; }
-            const float u = __double2float_rn(su);
-            const float w = __fmul_rn(beta, __fsub_rn(vs[j], u));
-            const float o = __double2float_rn(so + qk * (double)w);
-            a.o[(size_t)row * D + j] = o;
-            if (KIND == kDecode) a.w[(size_t)row * D + j] = w;
-            else sc.wv[j] = w;
-        }
+        finish_columns<D, KIND>(a, sc, tid, row, beta, vs, false);
         if (KIND == kFused) __syncthreads();
     }
     if (KIND != kDecode) {
@@ -664,11 +694,8 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
         for (int r = 0; r < RT; ++r) {
             const float ki = sc.kf[g * RT + r];
             const float2 k2 = make_float2(ki, ki);
-            const float2 p01 = mul2(al, make_float2(S[r][0], S[r][1]));
-            const float2 p23 = mul2(al, make_float2(S[r][2], S[r][3]));
-            const float2 s01 = fma2(k2, w01, p01);
-            const float2 s23 = fma2(k2, w23, p23);
-            S[r][0] = s01.x; S[r][1] = s01.y; S[r][2] = s23.x; S[r][3] = s23.y;
+            S[r][0] = fma2(k2, w01, mul2(al, S[r][0]));
+            S[r][1] = fma2(k2, w23, mul2(al, S[r][1]));
         }
         store_pivot<D>(S, rec_g, tid);
     }
@@ -755,11 +782,12 @@ __global__ void __launch_bounds__(2 * D) k_requant_pack(Args a) {
     }
     uint8_t *rec = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[gl];
     const float *Sg = a.S_in + (size_t)row * D * D;
-    float S[G::RT][4];
+    float2 S[G::RT][2];
 #pragma unroll
     for (int r = 0; r < G::RT; ++r) {
         const float4 v = *reinterpret_cast<const float4 *>(Sg + (size_t)(g * G::RT + r) * D + 4 * l);
-        S[r][0] = v.x; S[r][1] = v.y; S[r][2] = v.z; S[r][3] = v.w;
+        S[r][0] = make_float2(v.x, v.y);
+        S[r][1] = make_float2(v.z, v.w);
     }
     const int width = a.t.width[gl];
     if (width == kPivotBits) {
@@ -825,13 +853,13 @@ __global__ void __launch_bounds__(2 * D) k_unpack(Args a) {
         case 6: unpack_uniform<D, 6>(rec, out, tid); break;
         case 8: unpack_uniform<D, 8>(rec, out, tid); break;
         case kPivotBits: {
-            float S[G::RT][4];
+            float2 S[G::RT][2];
             load_pivot<D>(rec, tid, S);
             const int g = tid / G::LANES, l = tid % G::LANES;
 #pragma unroll
             for (int r = 0; r < G::RT; ++r)
                 *reinterpret_cast<float4 *>(out + (size_t)(g * G::RT + r) * D + 4 * l) =
-                    make_float4(S[r][0], S[r][1], S[r][2], S[r][3]);
+                    make_float4(S[r][0].x, S[r][0].y, S[r][1].x, S[r][1].y);
             break;
         }
         default: if (tid == 0) flag_error(a.err, kErrArgs); break;
@@ -856,17 +884,16 @@ __device__ void dist_uniform(const float *Sg, int gl, int m, int n_bits, double 
     constexpr int OFF = 1 << (B - 1);
     constexpr int Q = (1 << (B - 1)) - 1;
     constexpr float MG2 = kMagic + (float)OFF;
-    constexpr int LO = 0x4B400000 + OFF - Q;
-    constexpr int HI = 0x4B400000 + OFF + Q;
     const int g = tid / LANES, l = tid % LANES;
     const int j0 = 4 * l;
-    float S[RT][4];
+    float2 S[RT][2];
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
         const float4 v = *reinterpret_cast<const float4 *>(Sg + (size_t)(g * RT + r) * D + j0);
-        S[r][0] = v.x; S[r][1] = v.y; S[r][2] = v.z; S[r][3] = v.w;
+        S[r][0] = make_float2(v.x, v.y);
+        S[r][1] = make_float2(v.z, v.w);
     }
-    fit_scales<D, B>(S, sc, tid, nullptr);
+    fit_scales<D, B>(S, sc, tid, nullptr, nullptr);
     float cc[4], icc[4];
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) { cc[jj] = sc.cold[j0 + jj]; icc[jj] = sc.ic[j0 + jj]; }
@@ -876,12 +903,12 @@ __device__ void dist_uniform(const float *Sg, int gl, int m, int n_bits, double 
         const float ri = sc.rowr[i];
         const float4 orig = *reinterpret_cast<const float4 *>(Sg + (size_t)i * D + j0);
         const float o4[4] = {orig.x, orig.y, orig.z, orig.w};
+        const float y4[4] = {S[r][0].x, S[r][0].y, S[r][1].x, S[r][1].y};
         double e = 0.0;
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-            const float t = __fmaf_rn(S[r][jj], icc[jj], MG2);
-            const int T = min(max(__float_as_int(t), LO), HI);
-            const float z = (float)(T - (0x4B400000 + OFF));
+            const float t = __fmaf_rn(y4[jj], icc[jj], MG2);
+            const float z = (float)((int)final_e<B>(t) - Q);
             const float sh = __fmul_rn(__fmul_rn(ri, cc[jj]), z);
             const double d = (double)sh - (double)o4[jj];
             e = fma(d, d, e);
