@@ -348,7 +348,8 @@ def run_product(args):
     # dominant kernel of the variant: its own algorithmic bytes over its mean launch time
     kind = "fused" if args.variant == "fused" else max(("decode", "fitpack"), key=lambda k: stats[k][0])
     k_ms, k_n = stats[kind]
-    k_bytes = kernel_bytes(plan, n, kind)
+    # algorithmic bytes of one launch: the kernel's bytes per step over its launches per step
+    k_bytes = kernel_bytes(plan, n, kind) / (k_n / args.steps) if k_n else None
     achieved = k_bytes / (k_ms / k_n / 1e3) / 1e9 if k_n else None
     traffic = profiled_traffic(args.variant)
 
