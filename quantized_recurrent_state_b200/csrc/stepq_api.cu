@@ -716,7 +716,6 @@ extern "C" int stepq_requant_pack(stepq_ctx *c, void *pool, const int32_t *slots
     int rc = check_range(c, n_req, lb, le);
     if (rc) return rc;
     if ((rc = check_ptr(pool, 128, "pool")) || (rc = check_ptr(slots, 4, "slots")) || (rc = check_ptr(S, 16, "S"))) return rc;
-    if (c->plan->mode != 0) return fail(STEPQ_EINVAL, "requant_pack: per-row (mode 1) records are not supported by this build");
     if ((rc = set_device(c))) return rc;
     if (n_req == 0) return STEPQ_OK;
     if ((rc = wait_side(c, lb, le))) return rc;
@@ -733,7 +732,6 @@ extern "C" int stepq_unpack(stepq_ctx *c, const void *pool, const int32_t *slots
     int rc = check_range(c, n_req, lb, le);
     if (rc) return rc;
     if ((rc = check_ptr(pool, 128, "pool")) || (rc = check_ptr(slots, 4, "slots")) || (rc = check_ptr(S, 16, "S"))) return rc;
-    if (c->plan->mode != 0) return fail(STEPQ_EINVAL, "unpack: per-row (mode 1) records are not supported by this build");
     if ((rc = set_device(c))) return rc;
     if (n_req == 0) return STEPQ_OK;
     if ((rc = wait_side(c, lb, le))) return rc;
@@ -753,7 +751,6 @@ static int check_step_io(stepq_ctx *c, void *pool, const int32_t *slots, const f
         (rc = check_ptr(k, 16, "k")) || (rc = check_ptr(v, 16, "v")) || (rc = check_ptr(alpha, 4, "alpha")) ||
         (rc = check_ptr(beta, 4, "beta")) || (rc = check_ptr(o, 16, "o")))
         return rc;
-    if (c->plan->mode != 0) return fail(STEPQ_EINVAL, "decode_step: per-row (mode 1) records are not supported by this build");
     return STEPQ_OK;
 }
 

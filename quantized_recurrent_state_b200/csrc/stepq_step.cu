@@ -51,8 +51,9 @@ struct __align__(16) Scratch {
             double pU[8][D];  // per-band column partials of u and o
             double pO[8][D];
         } col;
-        float rsum[8][RT][RS];  // per-thread row partials, transposed for the row reduction
+        float pmax[4][8][D];  // per-row records: column absmax per width class and band
     } u;
+    float rsum[8][RT][RS];  // per-thread row partials, transposed for the row reduction
     float pf0[8][D];
     float pf1[8][D];
     float a[D];       // a_i = fl(alpha_i r_i)
@@ -73,7 +74,8 @@ struct __align__(16) Scratch {
     double bandK[8];  // per band: sum_i k_i a_i (256 + off), sum_i q_i a_i (256 + off), sum_i q_i k_i
     double bandQ[8];
     double bandQK[8];
-    int need_clamp;
+    int rw[D];          // per-row records: row width (16 = FP16 row)
+    uint32_t roff[D];   // per-row records: row byte offset in the codes block
     int meta[kStages][4];  // slot, width, valid, unused
     float nz;              // -0.0f, read at run time (see fit_scales)
 };
@@ -290,7 +292,7 @@ __device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, float
 
     // 1. row sums: thread partial over its 4 columns, then the other lanes'
     //    partials of the row through shared memory (pairwise in lane order)
-    float *rs = &sc.u.rsum[g][0][0];
+    float *rs = &sc.rsum[g][0][0];
 #pragma unroll
     for (int r = 0; r < RT; ++r)
         rs[r * RS + l] = (fabsf(S[r][0].x) + fabsf(S[r][0].y)) + (fabsf(S[r][1].x) + fabsf(S[r][1].y));
@@ -702,9 +704,358 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
 }
 
 // ---------------------------------------------------------------------------
+// Per-key-row units (KDA, mode 1): every key row has its own width b_i
+// (2, 4, 6, 8, or 16 for an FP16 pivot row) and its own retention gate.
+// Row-major codes: lane l's four codes of a row are row bits [4 b l, 4 b l + 4 b).
+// The width of a row is the same for all lanes of a band, so the per-row
+// branches below are uniform across a warp.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t row_field(const uint8_t *row, int b, int l) {
+    const int bit = 4 * b * l;
+    const uint32_t *wp = reinterpret_cast<const uint32_t *>(row);  // rows start 16-byte aligned
+    const int w = bit >> 5, sh = bit & 31;
+    const uint32_t lo = wp[w];
+    const uint32_t hi = (sh + 4 * b > 32) ? wp[w + 1] : 0u;
+    return __funnelshift_r(lo, hi, sh);
+}
+
+// Store lane l's 4b-bit field of a row (row bits [4 b l, 4 b l + 4 b)).
+__device__ __forceinline__ void row_field_store(uint8_t *row, int b, int l, uint32_t f) {
+    if (b == 8) {
+        reinterpret_cast<uint32_t *>(row)[l] = f;
+    } else if (b == 4) {
+        reinterpret_cast<uint16_t *>(row)[l] = (uint16_t)f;
+    } else if (b == 2) {
+        row[l] = (uint8_t)f;
+    } else {  // b == 6: three bytes at byte 3l
+        uint8_t *p = row + 3 * l;
+        p[0] = (uint8_t)f;
+        p[1] = (uint8_t)(f >> 8);
+        p[2] = (uint8_t)(f >> 16);
+    }
+}
+
+// Final code e = z + qmax in [0, 2 qmax] of a row of width b (see final_e).
+__device__ __forceinline__ uint32_t final_e_rt(float y, float ic, int b) {
+    const int off = 1 << (b - 1);
+    const float t = __fmaf_rn(y, ic, kMagic + (float)off);
+    return (uint32_t)__viaddmin_s32_relu(__float_as_int(t), -(0x4B400000 + 1), 2 * (off - 1));
+}
+
+// Refit of a tile of per-row units held in registers; writes r and c to
+// rec_r / rec_c (global, may be null) and the packed rows into `codes`
+// (shared memory holding the codes block; it is copied out by the caller).
+// FP16 rows keep S_t and are stored as binary16; they take no part in the
+// column fit and carry r = 0.
+template <int D>
+__device__ void fit_rows(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, uint8_t *codes, float *rec_r,
+                         float *rec_c) {
+    using G = Geo<D>;
+    constexpr int RT = G::RT, LANES = G::LANES, RS = Scratch<D>::RS, HALF = LANES / 2;
+    const int g = tid / LANES, l = tid % LANES;
+    const int j0 = 4 * l;
+
+    // 1. row sums and row factors
+    float *rs = &sc.rsum[g][0][0];
+#pragma unroll
+    for (int r = 0; r < RT; ++r)
+        rs[r * RS + l] = (fabsf(S[r][0].x) + fabsf(S[r][0].y)) + (fabsf(S[r][1].x) + fabsf(S[r][1].y));
+    __syncwarp();
+    {
+        const int rr = l >> 1, hh = l & 1;
+        const float *src = rs + rr * RS + hh * HALF;
+        float v[HALF];
+#pragma unroll
+        for (int k = 0; k < HALF; ++k) v[k] = src[k];
+        float s = tree_sum1<HALF>(v);
+        s = s + __shfl_xor_sync(0xffffffffu, s, 1);
+        const int i = g * RT + rr;
+        float ri = 0.0f, inv = 0.0f, bw = 0.0f;
+        if (sc.rw[i] != kPivotBits) {
+            float m = __fmul_rn(s, 1.0f / (float)D);
+            m = fmaxf(m, 1e-12f);
+            ri = __fmul_rn(m, sc.rho[i]);
+            inv = __frcp_rn(ri);
+            bw = __fmul_rn(sc.wbar[i], __fmul_rn(ri, ri));
+        }
+        if (hh == 0) {
+            sc.rowfit[i] = make_float2(inv, bw);
+            sc.rowr[i] = ri;
+            if (rec_r) rec_r[i] = ri;
+        }
+    }
+    __syncwarp();
+    // 2. y = fl(S * (1/r)) on quantized rows; 3. column absmax per width class
+    {
+        float m[4][4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) m[c][jj] = 0.0f;
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            const int i = g * RT + r;
+            const int b = sc.rw[i];
+            if (b == kPivotBits) continue;
+            const float inv = sc.rowfit[i].x;
+            const float2 i2 = make_float2(inv, inv);
+            S[r][0] = mul2(S[r][0], i2);
+            S[r][1] = mul2(S[r][1], i2);
+            const float a0 = fabsf(S[r][0].x), a1 = fabsf(S[r][0].y), a2 = fabsf(S[r][1].x), a3 = fabsf(S[r][1].y);
+            switch (b) {
+                case 2: m[0][0] = fmaxf(m[0][0], a0); m[0][1] = fmaxf(m[0][1], a1); m[0][2] = fmaxf(m[0][2], a2); m[0][3] = fmaxf(m[0][3], a3); break;
+                case 4: m[1][0] = fmaxf(m[1][0], a0); m[1][1] = fmaxf(m[1][1], a1); m[1][2] = fmaxf(m[1][2], a2); m[1][3] = fmaxf(m[1][3], a3); break;
+                case 6: m[2][0] = fmaxf(m[2][0], a0); m[2][1] = fmaxf(m[2][1], a1); m[2][2] = fmaxf(m[2][2], a2); m[2][3] = fmaxf(m[2][3], a3); break;
+                default: m[3][0] = fmaxf(m[3][0], a0); m[3][1] = fmaxf(m[3][1], a1); m[3][2] = fmaxf(m[3][2], a2); m[3][3] = fmaxf(m[3][3], a3); break;
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<float4 *>(&sc.u.pmax[c][g][j0]) = make_float4(m[c][0], m[c][1], m[c][2], m[c][3]);
+    }
+    __syncthreads();
+    if (tid < D) {
+        float c0 = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float mm = 0.0f;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) mm = fmaxf(mm, sc.u.pmax[c][b][tid]);
+            const int q = (1 << (2 * c + 1)) - 1;  // widths 2, 4, 6, 8
+            if (mm > 0.0f) c0 = fmaxf(c0, __fdiv_rn(mm, (float)q));
+        }
+        if (c0 == 0.0f) c0 = 1.0f;
+        sc.c0[tid] = c0;
+        sc.ic0[tid] = __frcp_rn(c0);
+    }
+    __syncthreads();
+    // 4. z0 and the weighted least-squares sums over the quantized rows
+    {
+        const float2 mg = make_float2(kMagic, kMagic);
+        const float2 nmg = make_float2(-kMagic, -kMagic);
+        const float2 nz2 = make_float2(sc.nz, sc.nz);
+        const float4 ic4 = *reinterpret_cast<const float4 *>(&sc.ic0[j0]);
+#pragma unroll
+        for (int hp = 0; hp < 2; ++hp) {
+            const int jA = j0 + 2 * hp;
+            const float2 ic = hp ? make_float2(ic4.z, ic4.w) : make_float2(ic4.x, ic4.y);
+            PairTree<RT> tn, td;
+#pragma unroll
+            for (int r = 0; r < RT; ++r) {
+                const int i = g * RT + r;
+                float2 vn = make_float2(0.0f, 0.0f), vd = make_float2(0.0f, 0.0f);
+                if (sc.rw[i] != kPivotBits) {
+                    const float bwr = sc.rowfit[i].y;
+                    const float2 y = S[r][hp];
+                    const float2 z0 = add2(fma2(y, ic, mg), nmg);
+                    const float2 b2 = make_float2(bwr, bwr);
+                    vn = fma2(b2, mul2(z0, y), nz2);
+                    vd = fma2(b2, mul2(z0, z0), nz2);
+                }
+                tn.push(r, vn);
+                td.push(r, vd);
+            }
+            *reinterpret_cast<float2 *>(&sc.pf0[g][jA]) = tn.total();
+            *reinterpret_cast<float2 *>(&sc.pf1[g][jA]) = td.total();
+        }
+    }
+    __syncthreads();
+    if (tid < D) {
+        float xn[8], xd[8];
+#pragma unroll
+        for (int b = 0; b < 8; ++b) { xn[b] = sc.pf0[b][tid]; xd[b] = sc.pf1[b][tid]; }
+        const float num = tree_sum1<8>(xn);
+        const float den = tree_sum1<8>(xd);
+        const float c = (den > 0.0f) ? __fdiv_rn(num, den) : sc.c0[tid];
+        sc.ic[tid] = __frcp_rn(c);
+        sc.cold[tid] = c;
+        if (rec_c) rec_c[tid] = c;
+    }
+    __syncthreads();
+    // 5. final codes (or binary16) of every row into the shared codes block
+    {
+        const float4 ic4 = *reinterpret_cast<const float4 *>(&sc.ic[j0]);
+        const float icj[4] = {ic4.x, ic4.y, ic4.z, ic4.w};
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            const int i = g * RT + r;
+            const int b = sc.rw[i];
+            uint8_t *row = codes + sc.roff[i];
+            if (b == kPivotBits) {
+                const __half2 h01 = __float22half2_rn(S[r][0]);
+                const __half2 h23 = __float22half2_rn(S[r][1]);
+                uint2 v;
+                v.x = *reinterpret_cast<const uint32_t *>(&h01);
+                v.y = *reinterpret_cast<const uint32_t *>(&h23);
+                *reinterpret_cast<uint2 *>(row + 8 * l) = v;
+            } else {
+                const float y4[4] = {S[r][0].x, S[r][0].y, S[r][1].x, S[r][1].y};
+                uint32_t f = 0u;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) f |= (final_e_rt(y4[jj], icj[jj], b) + 1u) << (b * jj);
+                row_field_store(row, b, l, f);
+            }
+        }
+    }
+    __syncthreads();
+}
+
+// Copy `bytes` (a multiple of 16) from shared to global memory, all threads.
+template <int D>
+__device__ __forceinline__ void copy_out(uint8_t *dst, const uint8_t *src, uint32_t bytes, int tid) {
+    for (uint32_t o = 16u * tid; o < bytes; o += 16u * (2 * D))
+        *reinterpret_cast<uint4 *>(dst + o) = *reinterpret_cast<const uint4 *>(src + o);
+}
+
+template <int D>
+__device__ __forceinline__ void rows_prologue_tables(const Args &a, Scratch<D> &sc, int tid, int gl) {
+    if (tid < D) {
+        sc.rw[tid] = a.t.row_width[(size_t)gl * D + tid];
+        sc.roff[tid] = a.t.row_off[(size_t)gl * D + tid];
+        sc.rho[tid] = a.t.rho[(size_t)gl * D + tid];
+        sc.wbar[tid] = a.t.wbar[(size_t)gl * D + tid];
+    }
+}
+
+// One head of per-row units: decode / fit-pack / fused.
+template <int D, int KIND>
+__device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row, int gl, Scratch<D> &sc,
+                          int tid) {
+    using G = Geo<D>;
+    constexpr int RT = G::RT, LANES = G::LANES;
+    const int g = tid / LANES, l = tid % LANES;
+    const int j0 = 4 * l;
+    const uint32_t codes_bytes = a.t.codes_bytes[gl];
+    const float *st_r = reinterpret_cast<const float *>(stage + codes_bytes);
+    const float *st_c = st_r + D;
+    const float *qs = reinterpret_cast<const float *>(stage + a.rec_stage_bytes);
+    const float *ks = qs + D;
+    const float *vs = ks + D;
+    const float *xs = vs + D;
+    const float beta = a.beta[row];
+
+    double bk = 0.0, bq = 0.0, bqk = 0.0;
+    rows_prologue_tables<D>(a, sc, tid, gl);
+    if (tid < D) {
+        const int i = tid;
+        const int b = sc.rw[i];
+        const float al = a.alpha[(size_t)row * D + i];
+        const float ai = (b == kPivotBits) ? al : __fmul_rn(al, st_r[i]);
+        sc.a[i] = ai;
+        sc.kf[i] = ks[i];
+        sc.cpr[i] = __fmul_rn(st_c[i], 1.0f / 4096.0f);
+        sc.cold[i] = st_c[i];
+        if (KIND == kFitPack) sc.wv[i] = xs[i];
+        if (KIND != kFitPack) {
+            const double ka = (double)ks[i] * (double)ai;
+            const double qa = (double)qs[i] * (double)ai;
+            if (b == kPivotBits) {
+                sc.kap[i] = ka;
+                sc.qt[i] = qa;
+            } else {
+                sc.kap[i] = ka * kTwoM169;
+                sc.qt[i] = qa * kTwoM169;
+                bk = ka * (double)(256 + (1 << (b - 1)));
+                bq = qa * (double)(256 + (1 << (b - 1)));
+            }
+            bqk = (double)qs[i] * (double)ks[i];
+        }
+    }
+    if (KIND != kFitPack) band_sums<D>(sc, tid, bk, bq, bqk);
+    __syncthreads();
+
+    float2 S[RT][2];
+    double accU[4] = {0.0, 0.0, 0.0, 0.0}, accO[4] = {0.0, 0.0, 0.0, 0.0};
+    double accUp[4] = {0.0, 0.0, 0.0, 0.0}, accOp[4] = {0.0, 0.0, 0.0, 0.0};
+    const float4 c4 = *reinterpret_cast<const float4 *>(&sc.cpr[j0]);
+    const float2 cp01 = make_float2(c4.x, c4.y), cp23 = make_float2(c4.z, c4.w);
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+        const int i = g * RT + r;
+        const int b = sc.rw[i];
+        const float ai = sc.a[i];
+        const float2 a2 = make_float2(ai, ai);
+        if (b == kPivotBits) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(stage + sc.roff[i] + 8 * l);
+            const float2 h01 = __half22float2(*reinterpret_cast<const __half2 *>(&v.x));
+            const float2 h23 = __half22float2(*reinterpret_cast<const __half2 *>(&v.y));
+            if (KIND != kFitPack) {
+                const double kap = sc.kap[i], qt = sc.qt[i];
+                const double d[4] = {(double)h01.x, (double)h01.y, (double)h23.x, (double)h23.y};
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    accUp[jj] = fma(kap, d[jj], accUp[jj]);
+                    accOp[jj] = fma(qt, d[jj], accOp[jj]);
+                }
+            }
+            S[r][0] = mul2(a2, h01);
+            S[r][1] = mul2(a2, h23);
+        } else {
+            const uint32_t f = row_field(stage + sc.roff[i], b, l);
+            const uint32_t mask = (1u << b) - 1u;
+            const float zb = 8388608.0f + (float)(1 << (b - 1)) * 4096.0f;
+            uint32_t X[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) X[jj] = (((f >> (b * jj)) & mask) << 12) | 0x4B000000u;
+            if (KIND != kFitPack) {
+                const double kap = sc.kap[i], qt = sc.qt[i];
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const double d = x_as_f64(X[jj]);
+                    accU[jj] = fma(kap, d, accU[jj]);
+                    accO[jj] = fma(qt, d, accO[jj]);
+                }
+            }
+            const float2 nzb = make_float2(-zb, -zb);
+            const float2 z01 = add2(make_float2(__uint_as_float(X[0]), __uint_as_float(X[1])), nzb);
+            const float2 z23 = add2(make_float2(__uint_as_float(X[2]), __uint_as_float(X[3])), nzb);
+            S[r][0] = mul2(mul2(a2, cp01), z01);
+            S[r][1] = mul2(mul2(a2, cp23), z23);
+        }
+    }
+
+    if (KIND != kFitPack) {
+        // quantized rows carry c_j; FP16 rows do not: scale the band partial here
+        const double bK = sc.bandK[g], bQ = sc.bandQ[g];
+        double pu[4], po[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const double cj = (double)sc.cold[j0 + jj];
+            pu[jj] = cj * (accU[jj] - bK) + accUp[jj];
+            po[jj] = cj * (accO[jj] - bQ) + accOp[jj];
+        }
+        *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0]) = make_double2(pu[0], pu[1]);
+        *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0 + 2]) = make_double2(pu[2], pu[3]);
+        *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0]) = make_double2(po[0], po[1]);
+        *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0 + 2]) = make_double2(po[2], po[3]);
+        __syncthreads();
+        finish_columns<D, KIND>(a, sc, tid, row, beta, vs, false);
+        if (KIND == kFused) __syncthreads();
+    }
+
+    if (KIND != kDecode) {
+        const float4 w4 = *reinterpret_cast<const float4 *>(&sc.wv[j0]);
+        const float2 w01 = make_float2(w4.x, w4.y);
+        const float2 w23 = make_float2(w4.z, w4.w);
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            const float ki = sc.kf[g * RT + r];
+            const float2 k2 = make_float2(ki, ki);
+            S[r][0] = fma2(k2, w01, S[r][0]);
+            S[r][1] = fma2(k2, w23, S[r][1]);
+        }
+        // the staged codes are no longer read: assemble the new rows there
+        float *rec_r = reinterpret_cast<float *>(rec_g + codes_bytes);
+        fit_rows<D>(S, sc, tid, stage, rec_r, rec_r + D);
+        copy_out<D>(rec_g, stage, codes_bytes, tid);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Persistent pipeline kernel.
 // ---------------------------------------------------------------------------
-template <int D, int KIND>
+template <int D, int KIND, int MODE>
 __global__ void __launch_bounds__(2 * D, 2) k_step(Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x;
@@ -740,7 +1091,12 @@ __global__ void __launch_bounds__(2 * D, 2) k_step(Args a) {
         const int slot = sc.meta[s][0];
         const int width = sc.meta[s][1];
         const int valid = sc.meta[s][2];
-        if (valid) {
+        if (valid && MODE == 1) {
+            int n, ll, h, gl, row;
+            item_coords<D>(a, it, n, ll, h, gl, row);
+            uint8_t *rec_g = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[gl];
+            item_rows<D, KIND>(a, stage, rec_g, row, gl, sc, tid);
+        } else if (valid) {
             int n, ll, h, gl, row;
             item_coords<D>(a, it, n, ll, h, gl, row);
             uint8_t *rec_g = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[gl];
@@ -769,6 +1125,7 @@ template <int D>
 __global__ void __launch_bounds__(2 * D) k_requant_pack(Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     Scratch<D> &sc = *reinterpret_cast<Scratch<D> *>(smem);
+    uint8_t *codes = smem + ((sizeof(Scratch<D>) + 127) / 128) * 128;  // per-row records: D*D*2 bytes
     using G = Geo<D>;
     const int tid = threadIdx.x;
     const int g = tid / G::LANES, l = tid % G::LANES;
@@ -788,6 +1145,16 @@ __global__ void __launch_bounds__(2 * D) k_requant_pack(Args a) {
         const float4 v = *reinterpret_cast<const float4 *>(Sg + (size_t)(g * G::RT + r) * D + 4 * l);
         S[r][0] = make_float2(v.x, v.y);
         S[r][1] = make_float2(v.z, v.w);
+    }
+    if (a.mode == 1) {
+        rows_prologue_tables<D>(a, sc, tid, gl);
+        if (tid == 0) sc.nz = a.neg_zero;
+        __syncthreads();
+        const uint32_t codes_bytes = a.t.codes_bytes[gl];
+        float *rec_r = reinterpret_cast<float *>(rec + codes_bytes);
+        fit_rows<D>(S, sc, tid, codes, rec_r, rec_r + D);
+        copy_out<D>(rec, codes, codes_bytes, tid);
+        return;
     }
     const int width = a.t.width[gl];
     if (width == kPivotBits) {
@@ -834,6 +1201,41 @@ __device__ void unpack_uniform(const uint8_t *rec, float *out, int tid) {
 }
 
 template <int D>
+__device__ void unpack_rows(const Args &a, const uint8_t *rec, float *out, int gl, int tid) {
+    using G = Geo<D>;
+    const int g = tid / G::LANES, l = tid % G::LANES;
+    const uint32_t codes_bytes = a.t.codes_bytes[gl];
+    const float *rr = reinterpret_cast<const float *>(rec + codes_bytes);
+    const float *cc = rr + D;
+    const float2 c01 = make_float2(__fmul_rn(cc[4 * l], 1.0f / 4096.0f), __fmul_rn(cc[4 * l + 1], 1.0f / 4096.0f));
+    const float2 c23 = make_float2(__fmul_rn(cc[4 * l + 2], 1.0f / 4096.0f), __fmul_rn(cc[4 * l + 3], 1.0f / 4096.0f));
+#pragma unroll
+    for (int r = 0; r < G::RT; ++r) {
+        const int i = g * G::RT + r;
+        const int b = a.t.row_width[(size_t)gl * D + i];
+        const uint8_t *row = rec + a.t.row_off[(size_t)gl * D + i];
+        float2 s01, s23;
+        if (b == kPivotBits) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(row + 8 * l);
+            s01 = __half22float2(*reinterpret_cast<const __half2 *>(&v.x));
+            s23 = __half22float2(*reinterpret_cast<const __half2 *>(&v.y));
+        } else {
+            const uint32_t f = row_field(row, b, l);
+            const uint32_t mask = (1u << b) - 1u;
+            const float zb = 8388608.0f + (float)(1 << (b - 1)) * 4096.0f;
+            float z[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+                z[jj] = __fsub_rn(__uint_as_float((((f >> (b * jj)) & mask) << 12) | 0x4B000000u), zb);
+            const float2 r2 = make_float2(rr[i], rr[i]);
+            s01 = mul2(mul2(r2, c01), make_float2(z[0], z[1]));
+            s23 = mul2(mul2(r2, c23), make_float2(z[2], z[3]));
+        }
+        *reinterpret_cast<float4 *>(out + (size_t)i * D + 4 * l) = make_float4(s01.x, s01.y, s23.x, s23.y);
+    }
+}
+
+template <int D>
 __global__ void __launch_bounds__(2 * D) k_unpack(Args a) {
     using G = Geo<D>;
     const int tid = threadIdx.x;
@@ -847,6 +1249,10 @@ __global__ void __launch_bounds__(2 * D) k_unpack(Args a) {
     }
     const uint8_t *rec = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[gl];
     float *out = a.S_out + (size_t)row * D * D;
+    if (a.mode == 1) {
+        unpack_rows<D>(a, rec, out, gl, tid);
+        return;
+    }
     switch (a.t.width[gl]) {
         case 2: unpack_uniform<D, 2>(rec, out, tid); break;
         case 4: unpack_uniform<D, 4>(rec, out, tid); break;
@@ -979,7 +1385,7 @@ static size_t step_smem(uint32_t stage_bytes) {
 template <int D, int KIND>
 static cudaError_t launch_step_d(Args a, int n_sms, cudaStream_t st, int *grid_out) {
     const size_t smem = step_smem<D>(a.stage_bytes);
-    auto kern = k_step<D, KIND>;
+    auto kern = a.mode == 1 ? k_step<D, KIND, 1> : k_step<D, KIND, 0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
@@ -1020,7 +1426,7 @@ static cudaError_t launch_pack_d(const Args &a, bool unpack, cudaStream_t st) {
     if (unpack) {
         k_unpack<D><<<a.n_items, 2 * D, 0, st>>>(a);
     } else {
-        const size_t smem = sizeof(Scratch<D>);
+        const size_t smem = ((sizeof(Scratch<D>) + 127) / 128) * 128 + (a.mode == 1 ? (size_t)D * D * 2 : 0);
         cudaError_t e = cudaFuncSetAttribute(k_requant_pack<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         k_requant_pack<D><<<a.n_items, 2 * D, smem, st>>>(a);

@@ -312,3 +312,82 @@ def test_full_pool_sampled_heads(stepq):
             zo, ho, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), new_rec)
             mism = (zg != zo) | (hg != ho)
             assert not (mism & (tie == 0)).any(), (r, l, h)
+
+
+# ---------------------------------------------------------------------------
+# per-key-row units (KDA): mixed row widths, FP16 pivot rows, per-row gates
+# ---------------------------------------------------------------------------
+
+def test_kda_slice_lockstep(stepq):
+    # 2 layers x 32 heads x 128 key rows of the KDA pool, Lagrangian nominal
+    # 6-bit plan over {4,6,8} with 16 FP16 rows, batch 8, 8 steps
+    _lockstep(stepq, "kda_rows", 8, 8, check=[0, 7], n_layers=2, n_pivots=16)
+
+
+def test_kda_two_stream_equals_fused(stepq):
+    a = Run(stepq, "kda_rows", 5, n_layers=2, n_pivots=16)
+    b = Run(stepq, "kda_rows", 5, n_layers=2, n_pivots=16)
+    a.pack_initial()
+    b.pack_initial()
+    for t in range(4):
+        _, oa = a.step(t, fused=False)
+        _, ob = b.step(t, fused=True)
+        assert np.array_equal(oa, ob)
+        assert torch.equal(a.pool, b.pool)
+
+
+def test_kda_unpack(stepq):
+    run = Run(stepq, "kda_rows", 2, n_layers=2, n_pivots=16)
+    run.pack_initial()
+    pv = run.pv
+    Sh = torch.zeros((2, pv.L, pv.H, pv.D, pv.D), dtype=torch.float32, device="cuda")
+    run.ctx.unpack(run.pool, run.slots_t, 2, 0, pv.L, Sh)
+    run.ctx.sync()
+    Sh = Sh.cpu().numpy()
+    for n in range(2):
+        g = run.slot_bytes_host(n)
+        for (l, h) in [(0, 0), (1, 31), (0, 17)]:
+            assert np.array_equal(Sh[n, l, h], pv.reconstruct(g, l, h))
+
+
+def test_kda_full_sampled_heads(stepq):
+    """81,920 key rows (20 layers x 32 heads x 128), 512 FP16 rows, batch 128:
+    one fused step, sampled heads checked against the oracle."""
+    plan, data, wl, _ = oracle_plan("kda_rows")
+    pv = model.PlanView(plan)
+    P = stepq.Plan.from_bytes(data)
+    n = 128
+    ctx = stepq.Context(P, n)
+    pool = torch.zeros(n * P.slot_bytes, dtype=torch.uint8, device="cuda")
+    slots = torch.arange(n, dtype=torch.int32, device="cuda")
+    for l in range(wl.n_layers):
+        S0 = synth.initial_states(wl, wl.seed, n, layers=[l])
+        ctx.requant_pack(pool, slots, n, l, l + 1, torch.from_numpy(S0).cuda())
+    ctx.sync()
+    alpha = synth.gates(wl, wl.seed)
+    inp = synth.step_inputs(wl, wl.seed, n, 0, alpha=alpha)
+    d = _inputs_to_dev(inp)
+    prev = pool.clone()
+    o = torch.zeros_like(d["q"])
+    ctx.decode_step_fused(pool, slots, n, 0, wl.n_layers, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)
+    ctx.sync()
+    og = o.cpu().numpy()
+    sb = P.slot_bytes
+    rng = np.random.default_rng(5)
+    widths = P.widths().reshape(wl.n_layers * wl.n_heads, wl.d)
+    piv_heads = np.nonzero((widths == 16).any(axis=1))[0]
+    samples = [(int(rng.integers(n)), int(rng.integers(wl.n_layers)), int(rng.integers(wl.n_heads))) for _ in range(16)]
+    samples += [(3, int(u) // wl.n_heads, int(u) % wl.n_heads) for u in piv_heads[:4]]
+    for (r, l, h) in samples:
+        off, nb = P.record(l, h)
+        rec_prev = prev[r * sb + off:r * sb + off + nb].cpu().numpy()
+        rec_new = pool[r * sb + off:r * sb + off + nb].cpu().numpy()
+        new_rec, o_ref, tie, S, w = model.step_head(pv.mode, pv.D, pv.rw(l, h), pv.rho[l, h], pv.wbar[l, h],
+                                                    rec_prev, inp["q"][r, l, h], inp["k"][r, l, h],
+                                                    inp["v"][r, l, h], inp["alpha"][r, l, h], inp["beta"][r, l, h])
+        assert _close(og[r, l, h], o_ref).all(), (r, l, h)
+        if not np.array_equal(rec_new, new_rec):
+            zg, hg, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), rec_new)
+            zo, ho, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), new_rec)
+            mism = (zg != zo) | (hg != ho)
+            assert not (mism & (tie == 0)).any(), (r, l, h)
