@@ -45,8 +45,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="stepq", choices=["stepq", "reference"])
     ap.add_argument("--variant", default="fused", choices=["fused", "two_stream"])
-    ap.add_argument("--batch", type=int, default=70)
-    ap.add_argument("--plan", type=int, default=6, choices=[4, 6])
+    ap.add_argument("--batch", type=int, default=None, help="requests (default: 70 GDN pool, 128 KDA)")
+    ap.add_argument("--plan", type=int, default=6, choices=[4, 6], help="nominal bits of the GDN pool plan")
+    ap.add_argument("--workload", default="gdn", choices=["gdn", "kda"],
+                    help="gdn: 2,304-head pool; kda: 81,920 key rows (20 x 32 x 128)")
     ap.add_argument("--sweep", action="store_true", help="also time batch 1/16/70/128/256")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
     ap.add_argument("--no-e2e", action="store_true")
@@ -79,24 +81,34 @@ def barrier(ws):
         dist.barrier()
 
 
+def _reduce(x: float, ws: int, op):
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=op)
+    return float(t.item())
+
+
 def max_over_ranks(x: float, ws: int) -> float:
     if ws == 1:
         return x
-    import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return _reduce(x, ws, dist.ReduceOp.MAX)
 
 
 def sum_over_ranks(x: float, ws: int) -> float:
     if ws == 1:
         return x
-    import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce(x, ws, dist.ReduceOp.SUM)
+
+
+def replica_throughput(units_local: float, secs_local: float, ws: int):
+    """Whole-job throughput of independent replicas: all ranks' units over the
+    slowest rank's device time.  Returns (units/s, max seconds)."""
+    secs = max_over_ranks(secs_local, ws)
+    return sum_over_ranks(units_local, ws) / secs, secs
 
 
 # ---------------------------------------------------------------------------
@@ -202,9 +214,9 @@ def product_plan(stepq, synth, wl, device):
     import torch
     L, H, D = wl.n_layers, wl.n_heads, wl.d
     bits = list(wl.bits)
-    # a uniform 8-bit plan only to host the calibration kernels' context
-    units = L * H
-    dummy = stepq.Plan.build(0, L, H, D, bits, float(max(bits)), 0, wl.horizon, np.zeros(units),
+    # a uniform plan at the largest width only to host the calibration kernels' context
+    units = L * H if wl.mode == 0 else L * H * D
+    dummy = stepq.Plan.build(wl.mode, L, H, D, bits, float(max(bits)), 0, wl.horizon, np.zeros(units),
                              np.tile(np.linspace(1.0, 0.25, len(bits)), (units, 1)), np.ones(L * H * D, np.float32))
     n = wl.calib_req
     ctx = stepq.Context(dummy, n)
@@ -235,12 +247,20 @@ def product_plan(stepq, synth, wl, device):
     import tempfile
     fd, path = tempfile.mkstemp(suffix=".plan")
     os.close(fd)
-    plan = stepq.Plan.build(0, L, H, D, bits, wl.nominal_bits, wl.n_pivots, wl.horizon,
-                            lmean.mean(axis=2).reshape(-1), d.sum(axis=2).reshape(-1, len(bits)),
-                            wbar.reshape(-1), path=path)
+    if wl.mode == 0:
+        lgate, dist = lmean.mean(axis=2).reshape(-1), d.sum(axis=2).reshape(-1, len(bits))
+    else:
+        lgate, dist = lmean.reshape(-1), d.reshape(-1, len(bits))
+    plan = stepq.Plan.build(wl.mode, L, H, D, bits, wl.nominal_bits, wl.n_pivots, wl.horizon,
+                            lgate, dist, wbar.reshape(-1), path=path)
     data = open(path, "rb").read()
     os.unlink(path)
     return plan, data
+
+
+def gate_bytes(plan):
+    """alpha + beta bytes of one head-step: scalar alpha (GDN) or one per key row (KDA)."""
+    return (4 if plan.mode == 0 else 4 * plan.d) + 4
 
 
 def step_bytes(plan, n_req):
@@ -251,7 +271,7 @@ def step_bytes(plan, n_req):
     for l in range(L):
         for h in range(H):
             rec += plan.record(l, h)[1]
-    per_slot = 2 * rec + L * H * (3 * 4 * D + 8 + 4 * D)
+    per_slot = 2 * rec + L * H * (3 * 4 * D + gate_bytes(plan) + 4 * D)
     return per_slot * n_req
 
 
@@ -264,8 +284,8 @@ def kernel_bytes(plan, n_req, kind):
     if kind == "fused":
         return step_bytes(plan, n_req)
     if kind == "decode":
-        return n_req * (rec + L * H * (3 * 4 * D + 8 + 2 * 4 * D))
-    return n_req * (2 * rec + L * H * (2 * 4 * D + 8))
+        return n_req * (rec + L * H * (3 * 4 * D + gate_bytes(plan) + 2 * 4 * D))
+    return n_req * (2 * rec + L * H * (2 * 4 * D + gate_bytes(plan)))
 
 
 def run_step(ctx, variant, pool, slots, n, L, inp, o, ws):
@@ -310,6 +330,16 @@ def time_steps(torch, ctx, variant, pool, slots, n, L, sets, o, ws, warmup, step
     return e0.elapsed_time(e1) / 1e3, stats, launches
 
 
+def workload_of(args, synth):
+    if args.workload == "kda":
+        wl = synth.workloads()["kda_rows"]
+    else:
+        wl = synth.workloads()["qwen_pool6" if args.plan == 6 else "qwen_pool4"]
+    if args.batch is None:
+        args.batch = 128 if args.workload == "kda" else 70
+    return wl
+
+
 def run_product(args):
     import torch
     from quantized_recurrent_state_b200 import build as qbuild
@@ -319,7 +349,7 @@ def run_product(args):
     barrier(ws)
     from quantized_recurrent_state_b200 import stepq, synth
     device = torch.device("cuda", local)
-    wl = synth.workloads()["qwen_pool6" if args.plan == 6 else "qwen_pool4"]
+    wl = workload_of(args, synth)
     n = args.batch
     plan, plan_bytes = product_plan(stepq, synth, wl, device)
     L, H, D = wl.n_layers, wl.n_heads, wl.d
@@ -338,9 +368,8 @@ def run_product(args):
     clocks = ClockSampler(local)
     secs, stats, launches = time_steps(torch, ctx, args.variant, pool, slots, n, L, sets, o, wsp,
                                        args.warmup, args.steps, ws, clocks)
-    secs = max_over_ranks(secs, ws)
     head_steps = n * L * H * args.steps
-    value = sum_over_ranks(head_steps, ws) / secs
+    value, secs = replica_throughput(head_steps, secs, ws)
     sb = step_bytes(plan, n)
     gbs = sb * args.steps / secs / 1e9
     peak, peak_kind = measured_peaks()
@@ -372,7 +401,7 @@ def run_product(args):
         e1.record(ctx.main)
         torch.cuda.synchronize()
         t32 = e0.elapsed_time(e1) / 1e3 / reps
-        b32 = n * L * H * (2 * 4 * D * D + 3 * 4 * D + 8 + 4 * D)
+        b32 = n * L * H * (2 * 4 * D * D + 3 * 4 * D + gate_bytes(plan) + 4 * D)
         extra["fp32_state_kernel"] = {"head_steps_per_s": n * L * H / t32, "ms_per_step": t32 * 1e3,
                                       "gbs": b32 / t32 / 1e9, "frac": b32 / t32 / 1e9 / peak}
         del S32
@@ -460,8 +489,12 @@ def run_product(args):
             "dtype": "f32",
             "data": "synthetic",
             "config": {
-                "workload": f"GDN state pool, {L} layers x {H} heads = {L * H} heads, d_k=d_v={D}, batch {n}, "
-                            f"nominal {wl.nominal_bits:g}-bit plan over {set(wl.bits)}, {wl.n_pivots} FP16 pivot heads",
+                "workload": (f"GDN state pool, {L} layers x {H} heads = {L * H} heads, d_k=d_v={D}, batch {n}, "
+                             f"nominal {wl.nominal_bits:g}-bit plan over {sorted(wl.bits)}, {wl.n_pivots} FP16 pivot heads")
+                if wl.mode == 0 else
+                            (f"KDA per-key-row units, {L} layers x {H} heads x {D} rows = {L * H * D} rows, d_v={D}, "
+                             f"batch {n}, Lagrangian nominal {wl.nominal_bits:g}-bit plan over {sorted(wl.bits)}, "
+                             f"{wl.n_pivots} FP16 pivot rows, per-row gates"),
                 "batch": n, "heads": L * H, "d": D, "variant": args.variant,
                 "bits_per_value": plan.info.bits_per_value, "bits_per_value_s16": plan.info.bits_per_value_s16,
                 "pool_bytes": n * plan.slot_bytes, "l2": "inputs larger than L2 (pool and q/k/v far above 126 MB)",
@@ -573,7 +606,7 @@ def run_reference(args):
     import multiprocessing as mp
     from oracle import model, plan_io
     from quantized_recurrent_state_b200 import synth
-    wl = synth.workloads()["qwen_pool6" if args.plan == 6 else "qwen_pool4"]
+    wl = workload_of(args, synth)
     cores = _n_cores()
     with mp.get_context("spawn").Pool(cores) as pool:
         layer_stats = pool.map(_oracle_calib_layer, [(wl.name, l) for l in range(wl.n_layers)])

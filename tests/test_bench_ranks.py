@@ -1,0 +1,46 @@
+"""Multi-rank plumbing of bench.py on CPU (gloo, world size 2).
+
+The decode path shards into independent replicas (every (request, head)
+state is independent, no exchange step), so the only cross-rank work is the
+timing aggregation: the whole-job value is all ranks' units over the slowest
+rank's time.  This test runs that aggregation in two gloo processes.
+"""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, ws, port, out):
+    import datetime
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws, timeout=datetime.timedelta(seconds=60))
+    import bench
+    units = 1000.0 * (rank + 1)
+    secs = 0.5 + rank          # rank 1 is the slow one
+    value, smax = bench.replica_throughput(units, secs, ws)
+    bench.barrier(ws)
+    out[rank] = (value, smax)
+    dist.destroy_process_group()
+
+
+def test_replica_throughput_two_ranks():
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_worker, args=(2, port, out), nprocs=2, join=True, start_method="spawn")
+    assert out[0] == out[1] == (3000.0 / 1.5, 1.5)
