@@ -567,7 +567,7 @@ void set_stages(stepq_ctx *c, stepq::Args &a, int lb, int le) {
     uint32_t m = 128;
     for (int l = lb; l < le; ++l) m = std::max(m, c->layer_max_rec[l]);
     a.rec_stage_bytes = (uint32_t)align_up(m, 128);
-    a.stage_bytes = a.rec_stage_bytes + 4u * 4u * (uint32_t)c->plan->D;
+    a.stage_bytes = a.rec_stage_bytes + (uint32_t)align_up(stepq::stage_tail_bytes(c->plan->D), 128);
 }
 
 cudaEvent_t take_event(stepq_ctx *c) {
@@ -639,7 +639,8 @@ extern "C" int stepq_ctx_create(const stepq_plan *plan, void *main_stream, void 
     const size_t heads = (size_t)p->L * p->H, nrow = heads * p->D;
     const size_t sz_off = 8 * heads, sz_u32 = 4 * heads, sz_hw = align_up(heads, 16), sz_rw = align_up(p->mode == 1 ? nrow : 16, 16),
                  sz_ro = 4 * (p->mode == 1 ? nrow : 4), sz_f = 4 * nrow;
-    const size_t total = sz_off + 2 * sz_u32 + sz_hw + sz_rw + sz_ro + 2 * sz_f + 64 * 8;
+    const size_t sz_desc = 16 * heads;
+    const size_t total = sz_desc + sz_off + 2 * sz_u32 + sz_hw + sz_rw + sz_ro + 2 * sz_f + 64 * 9;
     e = cudaMalloc(&c->tables_mem, total);
     if (e != cudaSuccess) { delete c; return cuda_fail(e, "cudaMalloc(tables)"); }
     uint8_t *m = static_cast<uint8_t *>(c->tables_mem);
@@ -650,6 +651,16 @@ extern "C" int stepq_ctx_create(const stepq_plan *plan, void *main_stream, void 
         o += align_up(reserve, 64);
         return dst;
     };
+    // per-head descriptor for the step kernels' copy issue: one 16-byte read
+    std::vector<uint32_t> desc(4 * heads);
+    for (size_t hd = 0; hd < heads; ++hd) {
+        const bool staged = !(p->mode == 0 && p->head_width[hd] == STEPQ_PIVOT_BITS);
+        desc[4 * hd] = (uint32_t)p->rec_off[hd];
+        desc[4 * hd + 1] = (uint32_t)(p->rec_off[hd] >> 32);
+        desc[4 * hd + 2] = staged ? p->rec_bytes[hd] : 0u;
+        desc[4 * hd + 3] = (uint32_t)(p->mode == 0 ? p->head_width[hd] : 0) | (p->codes_bytes[hd] << 8);
+    }
+    c->t.desc = (const uint4 *)put(desc.data(), sz_desc, sz_desc);
     c->t.rec_off = (const uint64_t *)put(p->rec_off.data(), sz_off, sz_off);
     c->t.rec_bytes = (const uint32_t *)put(p->rec_bytes.data(), sz_u32, sz_u32);
     c->t.codes_bytes = (const uint32_t *)put(p->codes_bytes.data(), sz_u32, sz_u32);
@@ -748,7 +759,8 @@ static int check_step_io(stepq_ctx *c, void *pool, const int32_t *slots, const f
                          const float *v, const float *alpha, const float *beta, float *o) {
     int rc;
     if ((rc = check_ptr(pool, 128, "pool")) || (rc = check_ptr(slots, 4, "slots")) || (rc = check_ptr(q, 16, "q")) ||
-        (rc = check_ptr(k, 16, "k")) || (rc = check_ptr(v, 16, "v")) || (rc = check_ptr(alpha, 4, "alpha")) ||
+        (rc = check_ptr(k, 16, "k")) || (rc = check_ptr(v, 16, "v")) ||
+        (rc = check_ptr(alpha, c->plan->mode == 1 ? 16 : 4, "alpha")) ||  // per-row alpha rows are bulk-copied
         (rc = check_ptr(beta, 4, "beta")) || (rc = check_ptr(o, 16, "o")))
         return rc;
     return STEPQ_OK;

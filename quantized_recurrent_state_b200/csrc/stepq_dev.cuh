@@ -20,6 +20,8 @@ constexpr int kErrArgs = 4;
 
 // Device copy of the plan tables.
 struct Tables {
+    const uint4 *desc;           // [L*H] {record offset lo, hi, staged record bytes (0 for an FP16
+                                 //  head), head width | codes-block bytes << 8}: one 16-byte read
     const uint64_t *rec_off;     // [L*H] record offset inside a slot
     const uint32_t *rec_bytes;   // [L*H]
     const uint32_t *codes_bytes; // [L*H] bytes of the codes block
@@ -54,6 +56,14 @@ struct Args {
     uint32_t stage_bytes;    // bytes of one pipeline stage
     uint32_t rec_stage_bytes;// bytes reserved for the record in a stage
 };
+
+// Tail of a pipeline stage (after the staged record), in 4-byte words of D:
+// q, k, v, x (the w workspace), rho, wbar, the per-row alpha (per-row
+// records), row byte offsets (per-row records), then D bytes of row widths
+// and a 16-byte block {alpha (per-head records), beta}.
+enum StageTail { kTailQ = 0, kTailK, kTailV, kTailX, kTailRho, kTailWbar, kTailAlpha, kTailRoff, kTailRw };
+
+__host__ __device__ constexpr uint32_t stage_tail_bytes(int D) { return 4u * kTailRw * D + D + 16u; }
 
 // ---------------------------------------------------------------------------
 // PTX wrappers: mbarrier + 1-D bulk copy (no multicast).
@@ -92,6 +102,26 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+
+// 4- and 16-byte asynchronous copies global -> shared (non-bulk).  Their
+// completion is handed to an mbarrier (cp_async_mbar_arrive: an arrival
+// that lands once every earlier cp.async of this thread has) or to a group
+// (cp_async_commit / cp_async_wait_all).
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
     uint32_t ok;

@@ -16,13 +16,15 @@
 //   kDecode   reconstruct -> u, w -> o (readout) ; writes o and w
 //   kFitPack  reconstruct -> S_t = S' + k w^T -> refit r, c -> pack, in place
 //   kFused    both in one pass over the record
+#include <cstddef>
+
 #include "stepq_dev.cuh"
 
 namespace stepq {
 
 enum Kind { kDecode = 0, kFitPack = 1, kFused = 2 };
 
-constexpr int kStages = 3;
+constexpr int kStages = 2;  // one item in flight while the other is worked on
 constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: fl(x + kMagic) - kMagic = rint(x), |x| < 2^22
 constexpr double kTwoM169 = 1.0 / 748288838313422294120286634350736906063837462003712.0;  // 2^-169
 
@@ -42,7 +44,9 @@ struct Stream {
     static constexpr int NCH = B / 2;                                   // chunks of RT bytes
 };
 
-// Shared memory besides the stages.
+// Shared memory besides the stages.  Per-row factors that multiply a pair
+// of columns are kept duplicated ((x_i, x_i) pairs), so a 16-byte load gives
+// two rows' packed operands without register moves.
 template <int D>
 struct __align__(16) Scratch {
     static constexpr int RT = D / 8, LANES = D / 4, RS = D / 4 + 4;  // RS: padded row of the transpose
@@ -56,13 +60,14 @@ struct __align__(16) Scratch {
     float rsum[8][RT][RS];  // per-thread row partials, transposed for the row reduction
     float pf0[8][D];
     float pf1[8][D];
-    float a[D];       // a_i = fl(alpha_i r_i)
-    float kf[D];      // k_i
+    float2 a2[D];     // (a_i, a_i), a_i = fl(alpha_i r_i)
+    float2 k2[D];     // (k_i, k_i)
     double kap[D];    // k_i a_i 2^-169   (pivot: k_i alpha_i)
     double qt[D];     // q_i a_i 2^-169   (pivot: q_i alpha_i)
-    float rho[D];
+    float rho[D];     // (requant and calibration kernels; the step reads them from the stage)
     float wbar[D];
-    float2 rowfit[D]; // (fl(1/r_i), b_i) of the refit
+    float2 rinv2[D];  // (fl(1/r_i), fl(1/r_i)) of the refit
+    float2 bw2[D];    // (b_i, b_i) of the refit
     float rowr[D];    // r_i of the refit
     float cpr[D];     // c_j 2^-12
     float cold[D];    // c_j (old on entry, refitted after fit_scales)
@@ -74,11 +79,28 @@ struct __align__(16) Scratch {
     double bandK[8];  // per band: sum_i k_i a_i (256 + off), sum_i q_i a_i (256 + off), sum_i q_i k_i
     double bandQ[8];
     double bandQK[8];
-    int rw[D];          // per-row records: row width (16 = FP16 row)
-    uint32_t roff[D];   // per-row records: row byte offset in the codes block
-    int meta[kStages][4];  // slot, width, valid, unused
-    float nz;              // -0.0f, read at run time (see fit_scales)
+    uint4 dring[2];    // prefetched item descriptors (thread 0)
+    int dslot[2];
+    int meta[kStages][8];  // slot, width, valid, codes bytes, record address lo, hi
+    uint32_t roff[D];  // per-row records (requant kernel): row byte offset in the codes block
+    uint8_t rw[D];     // per-row records (requant kernel): row width (16 = FP16 row)
+    float nz;          // -0.0f, read at run time (see fit_scales)
 };
+
+// Every array read or written with 8- or 16-byte vector accesses starts on a
+// 16-byte boundary of the (16-byte aligned) scratch block.
+template <int D>
+constexpr bool scratch_aligned() {
+    using S = Scratch<D>;
+    return offsetof(S, u) % 16 == 0 && offsetof(S, rsum) % 16 == 0 && offsetof(S, pf0) % 16 == 0 &&
+           offsetof(S, pf1) % 16 == 0 && offsetof(S, a2) % 16 == 0 && offsetof(S, k2) % 16 == 0 &&
+           offsetof(S, kap) % 16 == 0 && offsetof(S, qt) % 16 == 0 && offsetof(S, rinv2) % 16 == 0 &&
+           offsetof(S, bw2) % 16 == 0 && offsetof(S, cpr) % 16 == 0 && offsetof(S, cold) % 16 == 0 &&
+           offsetof(S, wv) % 16 == 0 && offsetof(S, ic0) % 16 == 0 && offsetof(S, ic) % 16 == 0 &&
+           offsetof(S, dring) % 16 == 0 && (sizeof(float) * Scratch<D>::RS) % 16 == 0;
+}
+static_assert(scratch_aligned<16>() && scratch_aligned<32>() && scratch_aligned<64>() && scratch_aligned<128>(),
+              "scratch arrays must stay 16-byte aligned");
 
 template <int D>
 __device__ __forceinline__ void item_coords(const Args &a, int it, int &n, int &ll, int &h, int &gl, int &row) {
@@ -91,43 +113,68 @@ __device__ __forceinline__ void item_coords(const Args &a, int it, int &n, int &
     row = (n * a.nL_in + a.l_in0 + ll) * a.H + h;  // index of the (request, layer, head) input row
 }
 
-// Thread 0: stage item `it` into stage s (record + input rows), or mark it invalid.
-template <int D, int KIND>
-__device__ void issue_item(const Args &a, int it, uint8_t *stage, uint64_t *bar, int *meta) {
+// Thread 0: start the 16-byte descriptor and the slot of item `it` on their
+// way into the descriptor ring entry e (cp.async, completion by group).
+template <int D>
+__device__ __forceinline__ void prefetch_desc(const Args &a, int it, Scratch<D> &sc, int e) {
     int n, ll, h, gl, row;
     item_coords<D>(a, it, n, ll, h, gl, row);
-    const int slot = a.slots[n];
+    cp_async16(&sc.dring[e], &a.t.desc[gl]);
+    cp_async4(&sc.dslot[e], &a.slots[n]);
+    cp_async_commit();
+}
+
+// Thread 0: stage item `it` (descriptor dsc, slot) into `stage`: the record,
+// the input rows and the head's tables by bulk copies, the per-item scalars
+// by cp.async, all completing on `bar`; or mark the item invalid.
+template <int D, int KIND, int MODE>
+__device__ void issue_item(const Args &a, int it, uint4 dsc, int slot, uint8_t *stage, uint64_t *bar, int *meta) {
+    int n, ll, h, gl, row;
+    item_coords<D>(a, it, n, ll, h, gl, row);
     const bool ok = slot >= 0 && slot < a.n_slots;
-    const int width = a.t.width[gl];
+    const uint8_t *rec = a.pool + (uint64_t)slot * a.slot_bytes + ((uint64_t)dsc.y << 32 | dsc.x);
     meta[0] = slot;
-    meta[1] = width;
+    meta[1] = (int)(dsc.w & 0xffu);
     meta[2] = ok ? 1 : 0;
+    meta[3] = (int)(dsc.w >> 8);
+    meta[4] = (int)(uint32_t)(uintptr_t)rec;
+    meta[5] = (int)(uint32_t)((uintptr_t)rec >> 32);
     if (!ok) {
         flag_error(a.err, kErrBadSlot);
         mbar_arrive(bar);
         return;
     }
+    uint8_t *tail = stage + a.rec_stage_bytes;
+    float *ab = reinterpret_cast<float *>(tail + 4 * kTailRw * D + D);
+    if (MODE == 0) cp_async4(ab, a.alpha + row);
+    if (KIND != kFitPack) cp_async4(ab + 1, a.beta + row);
+    cp_async_mbar_arrive(bar);  // before the expect-tx arrival, so the phase waits for them
     fence_proxy_async();
-    const uint8_t *rec = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[gl];
-    const uint32_t rec_bytes = (width == kPivotBits) ? 0u : a.t.rec_bytes[gl];
-    float *qs = reinterpret_cast<float *>(stage + a.rec_stage_bytes);
-    float *ks = qs + D;
-    float *vs = ks + D;
-    float *xs = vs + D;
     constexpr uint32_t RB = D * 4;
-    uint32_t total = rec_bytes;
-    if (KIND != kFitPack) total += 3 * RB;
-    else total += 2 * RB;
+    const uint32_t rec_bytes = dsc.z;
+    uint32_t total = rec_bytes + (KIND != kFitPack ? 3 * RB : 2 * RB);
+    if (KIND != kDecode) total += 2 * RB;
+    if (MODE == 1) total += 2 * RB + D;
     mbar_arrive_expect(bar, total);
     if (rec_bytes) bulk_g2s(stage, rec, rec_bytes, bar);
     const size_t off = (size_t)row * D;
+    const size_t goff = (size_t)gl * D;
+    float *tf = reinterpret_cast<float *>(tail);
     if (KIND != kFitPack) {
-        bulk_g2s(qs, a.q + off, RB, bar);
-        bulk_g2s(ks, a.k + off, RB, bar);
-        bulk_g2s(vs, a.v + off, RB, bar);
+        bulk_g2s(tf + kTailQ * D, a.q + off, RB, bar);
+        bulk_g2s(tf + kTailV * D, a.v + off, RB, bar);
     } else {
-        bulk_g2s(ks, a.k + off, RB, bar);
-        bulk_g2s(xs, a.w + off, RB, bar);
+        bulk_g2s(tf + kTailX * D, a.w + off, RB, bar);
+    }
+    bulk_g2s(tf + kTailK * D, a.k + off, RB, bar);
+    if (KIND != kDecode) {
+        bulk_g2s(tf + kTailRho * D, a.t.rho + goff, RB, bar);
+        bulk_g2s(tf + kTailWbar * D, a.t.wbar + goff, RB, bar);
+    }
+    if (MODE == 1) {
+        bulk_g2s(tf + kTailAlpha * D, a.alpha + off, RB, bar);
+        bulk_g2s(tail + 4 * kTailRw * D, a.t.row_width + goff, D, bar);
+        bulk_g2s(tf + kTailRoff * D, a.t.row_off + goff, RB, bar);
     }
 }
 
@@ -279,11 +326,12 @@ __device__ __forceinline__ uint32_t final_e(float t) {
 // Refit of the fp32 tile S held in registers as column pairs (all rows at
 // width B).  On return S holds y = fl(S * fl(1/r)); sc.rowr[i] = r_i,
 // sc.cold[j] = c_j, sc.ic[j] = fl(1/c_j).  rec_r / rec_c (global, may be
-// null) receive r and c.  Requires rho and wbar of the head in sc.rho /
-// sc.wbar.
+// null) receive r and c.  rho / wbar: the head's rho_i and wbar_i (shared
+// memory).
 // ---------------------------------------------------------------------------
 template <int D, int B>
-__device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, float *rec_r, float *rec_c) {
+__device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const float *rho, const float *wbar,
+                           float *rec_r, float *rec_c) {
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES, RS = Scratch<D>::RS, HALF = LANES / 2;
     constexpr int Q = (1 << (B - 1)) - 1;
@@ -316,11 +364,12 @@ __device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, float
         const int i = g * RT + rr;
         float m = __fmul_rn(s, 1.0f / (float)D);
         m = fmaxf(m, 1e-12f);
-        const float ri = __fmul_rn(m, sc.rho[i]);
+        const float ri = __fmul_rn(m, rho[i]);
         const float inv = __frcp_rn(ri);
-        const float bw = __fmul_rn(sc.wbar[i], __fmul_rn(ri, ri));
+        const float bw = __fmul_rn(wbar[i], __fmul_rn(ri, ri));
         if (hh == 0) {
-            sc.rowfit[i] = make_float2(inv, bw);
+            sc.rinv2[i] = make_float2(inv, inv);
+            sc.bw2[i] = make_float2(bw, bw);
             sc.rowr[i] = ri;
             if (rec_r) rec_r[i] = ri;
         }
@@ -331,8 +380,8 @@ __device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, float
         float2 m01 = make_float2(0.0f, 0.0f), m23 = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int r = 0; r < RT; r += 2) {
-            const float4 f = *reinterpret_cast<const float4 *>(&sc.rowfit[g * RT + r]);
-            const float2 i0 = make_float2(f.x, f.x), i1 = make_float2(f.z, f.z);
+            const float4 f = *reinterpret_cast<const float4 *>(&sc.rinv2[g * RT + r]);
+            const float2 i0 = make_float2(f.x, f.y), i1 = make_float2(f.z, f.w);
             S[r][0] = mul2(S[r][0], i0);
             S[r][1] = mul2(S[r][1], i0);
             S[r + 1][0] = mul2(S[r + 1][0], i1);
@@ -368,11 +417,10 @@ __device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, float
             float4 f;
 #pragma unroll
             for (int r = 0; r < RT; ++r) {
-                if ((r & 1) == 0) f = *reinterpret_cast<const float4 *>(&sc.rowfit[g * RT + r]);
-                const float bwr = (r & 1) ? f.w : f.y;
+                if ((r & 1) == 0) f = *reinterpret_cast<const float4 *>(&sc.bw2[g * RT + r]);
+                const float2 b2 = (r & 1) ? make_float2(f.z, f.w) : make_float2(f.x, f.y);
                 const float2 y = S[r][hp];
                 const float2 z0 = add2(fma2(y, ic, mg), nmg);
-                const float2 b2 = make_float2(bwr, bwr);
                 // fl(b * p) written as fma(b, p, -0) with a run-time -0: the
                 // product is rounded once and cannot be contracted into the
                 // pairwise additions that follow
@@ -400,7 +448,8 @@ __device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, float
 
 // Refit and pack into the record at `rec` (global): codes, r, c.
 template <int D, int B>
-__device__ void fit_pack(float2 (&S)[D / 8][2], uint8_t *rec, Scratch<D> &sc, int tid) {
+__device__ void fit_pack(float2 (&S)[D / 8][2], uint8_t *rec, Scratch<D> &sc, int tid, const float *rho,
+                         const float *wbar) {
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES;
     constexpr int OFF = 1 << (B - 1);
@@ -410,7 +459,7 @@ __device__ void fit_pack(float2 (&S)[D / 8][2], uint8_t *rec, Scratch<D> &sc, in
     const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
     float *rec_r = reinterpret_cast<float *>(rec + codes_bytes);
     float *rec_c = rec_r + D;
-    fit_scales<D, B>(S, sc, tid, rec_r, rec_c);
+    fit_scales<D, B>(S, sc, tid, rho, wbar, rec_r, rec_c);
     uint32_t W[Stream<D, B>::NW];
 #pragma unroll
     for (int i = 0; i < Stream<D, B>::NW; ++i) W[i] = 0u;
@@ -507,8 +556,7 @@ __device__ __forceinline__ void finish_columns(const Args &a, Scratch<D> &sc, in
 // One quantized head of width B: decode / fit-pack / fused.
 // ---------------------------------------------------------------------------
 template <int D, int B, int KIND>
-__device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int row, int gl,
-                             Scratch<D> &sc, int tid) {
+__device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int row, Scratch<D> &sc, int tid) {
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES;
     constexpr int OFF = 1 << (B - 1);
@@ -517,26 +565,25 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
     const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
     const float *st_r = reinterpret_cast<const float *>(stage + codes_bytes);
     const float *st_c = st_r + D;
-    const float *qs = reinterpret_cast<const float *>(stage + a.rec_stage_bytes);
-    const float *ks = qs + D;
-    const float *vs = ks + D;
-    const float *xs = vs + D;
-    const float alpha = a.alpha[row];
-    const float beta = a.beta[row];
+    const float *tf = reinterpret_cast<const float *>(stage + a.rec_stage_bytes);
+    const float *qs = tf + kTailQ * D;
+    const float *ks = tf + kTailK * D;
+    const float *vs = tf + kTailV * D;
+    const float *xs = tf + kTailX * D;
+    const float *ab = tf + kTailRw * D + D / 4;
+    const float alpha = ab[0];
+    const float beta = ab[1];
 
     // per-row and per-column parameters
     double bk = 0.0, bq = 0.0, bqk = 0.0;
     if (tid < D) {
         const int i = tid;
         const float ai = __fmul_rn(alpha, st_r[i]);
-        sc.a[i] = ai;
-        sc.kf[i] = ks[i];
+        const float ki = ks[i];
+        sc.a2[i] = make_float2(ai, ai);
+        sc.k2[i] = make_float2(ki, ki);
         sc.cpr[i] = __fmul_rn(st_c[i], 1.0f / 4096.0f);
         sc.cold[i] = st_c[i];
-        if (KIND != kDecode) {
-            sc.rho[i] = a.t.rho[(size_t)gl * D + i];
-            sc.wbar[i] = a.t.wbar[(size_t)gl * D + i];
-        }
         if (KIND == kFitPack) sc.wv[i] = xs[i];
         if (KIND != kFitPack) {
             const double ka = (double)ks[i] * (double)ai;
@@ -573,8 +620,8 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
             kap2 = *reinterpret_cast<const double2 *>(&sc.kap[i]);
             qt2 = *reinterpret_cast<const double2 *>(&sc.qt[i]);
         }
-        float2 a2r;
-        if (KIND != kDecode) a2r = *reinterpret_cast<const float2 *>(&sc.a[i]);
+        float4 a4;
+        if (KIND != kDecode) a4 = *reinterpret_cast<const float4 *>(&sc.a2[i]);
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
             {
@@ -598,8 +645,7 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
                 }
             }
             if (KIND != kDecode) {
-                const float ai = rr ? a2r.y : a2r.x;
-                const float2 a2 = make_float2(ai, ai);
+                const float2 a2 = rr ? make_float2(a4.z, a4.w) : make_float2(a4.x, a4.y);
                 const float2 z01 = add2(make_float2(__uint_as_float(X[0]), __uint_as_float(X[1])), nzb);
                 const float2 z23 = add2(make_float2(__uint_as_float(X[2]), __uint_as_float(X[3])), nzb);
                 S[r + rr][0] = mul2(mul2(a2, cp01), z01);
@@ -626,16 +672,15 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
         const float2 w23 = make_float2(w4.z, w4.w);
 #pragma unroll
         for (int r = 0; r < RT; r += 2) {
-            const float2 k2r = *reinterpret_cast<const float2 *>(&sc.kf[g * RT + r]);
+            const float4 k4 = *reinterpret_cast<const float4 *>(&sc.k2[g * RT + r]);
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
-                const float ki = rr ? k2r.y : k2r.x;
-                const float2 k2 = make_float2(ki, ki);
+                const float2 k2 = rr ? make_float2(k4.z, k4.w) : make_float2(k4.x, k4.y);
                 S[r + rr][0] = fma2(k2, w01, S[r + rr][0]);
                 S[r + rr][1] = fma2(k2, w23, S[r + rr][1]);
             }
         }
-        fit_pack<D, B>(S, rec_g, sc, tid);
+        fit_pack<D, B>(S, rec_g, sc, tid, tf + kTailRho * D, tf + kTailWbar * D);
     }
 }
 
@@ -646,15 +691,17 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
     constexpr int RT = G::RT, LANES = G::LANES;
     const int g = tid / LANES, l = tid % LANES;
     const int j0 = 4 * l;
-    const float *qs = reinterpret_cast<const float *>(stage + a.rec_stage_bytes);
-    const float *ks = qs + D;
-    const float *vs = ks + D;
-    const float *xs = vs + D;
-    const float alpha = a.alpha[row];
-    const float beta = a.beta[row];
+    const float *tf = reinterpret_cast<const float *>(stage + a.rec_stage_bytes);
+    const float *qs = tf + kTailQ * D;
+    const float *ks = tf + kTailK * D;
+    const float *vs = tf + kTailV * D;
+    const float *xs = tf + kTailX * D;
+    const float *ab = tf + kTailRw * D + D / 4;
+    const float alpha = ab[0];
+    const float beta = ab[1];
     double bqk = 0.0;
     if (tid < D) {
-        sc.kf[tid] = ks[tid];
+        sc.k2[tid] = make_float2(ks[tid], ks[tid]);
         if (KIND == kFitPack) sc.wv[tid] = xs[tid];
         if (KIND != kFitPack) {
             sc.kap[tid] = (double)ks[tid] * (double)alpha;
@@ -694,8 +741,7 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
         const float2 w23 = make_float2(sc.wv[j0 + 2], sc.wv[j0 + 3]);
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
-            const float ki = sc.kf[g * RT + r];
-            const float2 k2 = make_float2(ki, ki);
+            const float2 k2 = sc.k2[g * RT + r];
             S[r][0] = fma2(k2, w01, mul2(al, S[r][0]));
             S[r][1] = fma2(k2, w23, mul2(al, S[r][1]));
         }
@@ -749,8 +795,8 @@ __device__ __forceinline__ uint32_t final_e_rt(float y, float ic, int b) {
 // FP16 rows keep S_t and are stored as binary16; they take no part in the
 // column fit and carry r = 0.
 template <int D>
-__device__ void fit_rows(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, uint8_t *codes, float *rec_r,
-                         float *rec_c) {
+__device__ void fit_rows(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const uint8_t *rw, const uint32_t *roff,
+                         const float *rho, const float *wbar, uint8_t *codes, float *rec_r, float *rec_c) {
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES, RS = Scratch<D>::RS, HALF = LANES / 2;
     const int g = tid / LANES, l = tid % LANES;
@@ -772,15 +818,16 @@ __device__ void fit_rows(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, uint8_t
         s = s + __shfl_xor_sync(0xffffffffu, s, 1);
         const int i = g * RT + rr;
         float ri = 0.0f, inv = 0.0f, bw = 0.0f;
-        if (sc.rw[i] != kPivotBits) {
+        if (rw[i] != kPivotBits) {
             float m = __fmul_rn(s, 1.0f / (float)D);
             m = fmaxf(m, 1e-12f);
-            ri = __fmul_rn(m, sc.rho[i]);
+            ri = __fmul_rn(m, rho[i]);
             inv = __frcp_rn(ri);
-            bw = __fmul_rn(sc.wbar[i], __fmul_rn(ri, ri));
+            bw = __fmul_rn(wbar[i], __fmul_rn(ri, ri));
         }
         if (hh == 0) {
-            sc.rowfit[i] = make_float2(inv, bw);
+            sc.rinv2[i] = make_float2(inv, inv);
+            sc.bw2[i] = make_float2(bw, bw);
             sc.rowr[i] = ri;
             if (rec_r) rec_r[i] = ri;
         }
@@ -796,10 +843,9 @@ __device__ void fit_rows(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, uint8_t
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
             const int i = g * RT + r;
-            const int b = sc.rw[i];
+            const int b = rw[i];
             if (b == kPivotBits) continue;
-            const float inv = sc.rowfit[i].x;
-            const float2 i2 = make_float2(inv, inv);
+            const float2 i2 = sc.rinv2[i];
             S[r][0] = mul2(S[r][0], i2);
             S[r][1] = mul2(S[r][1], i2);
             const float a0 = fabsf(S[r][0].x), a1 = fabsf(S[r][0].y), a2 = fabsf(S[r][1].x), a3 = fabsf(S[r][1].y);
@@ -845,11 +891,10 @@ __device__ void fit_rows(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, uint8_t
             for (int r = 0; r < RT; ++r) {
                 const int i = g * RT + r;
                 float2 vn = make_float2(0.0f, 0.0f), vd = make_float2(0.0f, 0.0f);
-                if (sc.rw[i] != kPivotBits) {
-                    const float bwr = sc.rowfit[i].y;
+                if (rw[i] != kPivotBits) {
+                    const float2 b2 = sc.bw2[i];
                     const float2 y = S[r][hp];
                     const float2 z0 = add2(fma2(y, ic, mg), nmg);
-                    const float2 b2 = make_float2(bwr, bwr);
                     vn = fma2(b2, mul2(z0, y), nz2);
                     vd = fma2(b2, mul2(z0, z0), nz2);
                 }
@@ -880,8 +925,8 @@ __device__ void fit_rows(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, uint8_t
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
             const int i = g * RT + r;
-            const int b = sc.rw[i];
-            uint8_t *row = codes + sc.roff[i];
+            const int b = rw[i];
+            uint8_t *row = codes + roff[i];
             if (b == kPivotBits) {
                 const __half2 h01 = __float22half2_rn(S[r][0]);
                 const __half2 h23 = __float22half2_rn(S[r][1]);
@@ -920,30 +965,32 @@ __device__ __forceinline__ void rows_prologue_tables(const Args &a, Scratch<D> &
 
 // One head of per-row units: decode / fit-pack / fused.
 template <int D, int KIND>
-__device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row, int gl, Scratch<D> &sc,
-                          int tid) {
+__device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row, uint32_t codes_bytes,
+                          Scratch<D> &sc, int tid) {
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES;
     const int g = tid / LANES, l = tid % LANES;
     const int j0 = 4 * l;
-    const uint32_t codes_bytes = a.t.codes_bytes[gl];
     const float *st_r = reinterpret_cast<const float *>(stage + codes_bytes);
     const float *st_c = st_r + D;
-    const float *qs = reinterpret_cast<const float *>(stage + a.rec_stage_bytes);
-    const float *ks = qs + D;
-    const float *vs = ks + D;
-    const float *xs = vs + D;
-    const float beta = a.beta[row];
+    const float *tf = reinterpret_cast<const float *>(stage + a.rec_stage_bytes);
+    const float *qs = tf + kTailQ * D;
+    const float *ks = tf + kTailK * D;
+    const float *vs = tf + kTailV * D;
+    const float *xs = tf + kTailX * D;
+    const float *als = tf + kTailAlpha * D;
+    const uint32_t *roff = reinterpret_cast<const uint32_t *>(tf + kTailRoff * D);
+    const uint8_t *rw = reinterpret_cast<const uint8_t *>(tf + kTailRw * D);
+    const float beta = (tf + kTailRw * D + D / 4)[1];
 
     double bk = 0.0, bq = 0.0, bqk = 0.0;
-    rows_prologue_tables<D>(a, sc, tid, gl);
     if (tid < D) {
         const int i = tid;
-        const int b = sc.rw[i];
-        const float al = a.alpha[(size_t)row * D + i];
+        const int b = rw[i];
+        const float al = als[i];
         const float ai = (b == kPivotBits) ? al : __fmul_rn(al, st_r[i]);
-        sc.a[i] = ai;
-        sc.kf[i] = ks[i];
+        sc.a2[i] = make_float2(ai, ai);
+        sc.k2[i] = make_float2(ks[i], ks[i]);
         sc.cpr[i] = __fmul_rn(st_c[i], 1.0f / 4096.0f);
         sc.cold[i] = st_c[i];
         if (KIND == kFitPack) sc.wv[i] = xs[i];
@@ -973,11 +1020,10 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
         const int i = g * RT + r;
-        const int b = sc.rw[i];
-        const float ai = sc.a[i];
-        const float2 a2 = make_float2(ai, ai);
+        const int b = rw[i];
+        const float2 a2 = sc.a2[i];
         if (b == kPivotBits) {
-            const uint2 v = *reinterpret_cast<const uint2 *>(stage + sc.roff[i] + 8 * l);
+            const uint2 v = *reinterpret_cast<const uint2 *>(stage + roff[i] + 8 * l);
             const float2 h01 = __half22float2(*reinterpret_cast<const __half2 *>(&v.x));
             const float2 h23 = __half22float2(*reinterpret_cast<const __half2 *>(&v.y));
             if (KIND != kFitPack) {
@@ -992,7 +1038,7 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
             S[r][0] = mul2(a2, h01);
             S[r][1] = mul2(a2, h23);
         } else {
-            const uint32_t f = row_field(stage + sc.roff[i], b, l);
+            const uint32_t f = row_field(stage + roff[i], b, l);
             const uint32_t mask = (1u << b) - 1u;
             const float zb = 8388608.0f + (float)(1 << (b - 1)) * 4096.0f;
             uint32_t X[4];
@@ -1040,14 +1086,13 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
         const float2 w23 = make_float2(w4.z, w4.w);
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
-            const float ki = sc.kf[g * RT + r];
-            const float2 k2 = make_float2(ki, ki);
+            const float2 k2 = sc.k2[g * RT + r];
             S[r][0] = fma2(k2, w01, S[r][0]);
             S[r][1] = fma2(k2, w23, S[r][1]);
         }
         // the staged codes are no longer read: assemble the new rows there
         float *rec_r = reinterpret_cast<float *>(rec_g + codes_bytes);
-        fit_rows<D>(S, sc, tid, stage, rec_r, rec_r + D);
+        fit_rows<D>(S, sc, tid, rw, roff, tf + kTailRho * D, tf + kTailWbar * D, stage, rec_r, rec_r + D);
         copy_out<D>(rec_g, stage, codes_bytes, tid);
     }
 }
@@ -1059,60 +1104,77 @@ template <int D, int KIND, int MODE>
 __global__ void __launch_bounds__(2 * D, 2) k_step(Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x;
+    const int G = gridDim.x;
     uint8_t *stages = smem;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * a.stage_bytes);
     Scratch<D> &sc = *reinterpret_cast<Scratch<D> *>(smem + kStages * a.stage_bytes + 64);
 
+    // Thread 0 keeps the ring full: the first kStages items here, then the
+    // item kStages - 1 ahead right after the barrier that opens each item
+    // (every thread is past the previous item, so its stage is free).  The
+    // descriptor of the item after that is fetched one item ahead by
+    // cp.async, so thread 0 never waits on a global load on this path.
+    int dsel = 0;
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
         sc.nz = a.neg_zero;
+        for (int s = 0; s < kStages; ++s) {
+            const int it = blockIdx.x + s * G;
+            if (it >= a.n_items) break;
+            int n, ll, h, gl, row;
+            item_coords<D>(a, it, n, ll, h, gl, row);
+            issue_item<D, KIND, MODE>(a, it, a.t.desc[gl], a.slots[n], stages + s * a.stage_bytes, &bars[s],
+                                      sc.meta[s]);
+        }
+        const int nx = blockIdx.x + kStages * G;
+        if (nx < a.n_items) prefetch_desc<D>(a, nx, sc, 0);
     }
     __syncthreads();
-    if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            const int it = blockIdx.x + s * gridDim.x;
-            if (it < a.n_items) issue_item<D, KIND>(a, it, stages + s * a.stage_bytes, &bars[s], sc.meta[s]);
-        }
-    }
     int s = 0;
     uint32_t phase = 0;
-    for (int it = blockIdx.x; it < a.n_items; it += gridDim.x) {
+    for (int it = blockIdx.x; it < a.n_items; it += G) {
         const bool ok = mbar_wait_bounded(&bars[s], phase);
         if (__syncthreads_or(!ok)) {
             if (tid == 0) {
                 flag_error(a.err, kErrWait);
                 // let every copy still in flight land before shared memory goes away
+                cp_async_wait_all();
                 for (int k = 0; k < kStages; ++k) mbar_wait_bounded(&bars[k], phase ^ (k < s ? 1u : 0u), 1u << 20);
             }
             return;
         }
-        uint8_t *stage = stages + s * a.stage_bytes;
-        const int slot = sc.meta[s][0];
-        const int width = sc.meta[s][1];
-        const int valid = sc.meta[s][2];
-        if (valid && MODE == 1) {
-            int n, ll, h, gl, row;
-            item_coords<D>(a, it, n, ll, h, gl, row);
-            uint8_t *rec_g = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[gl];
-            item_rows<D, KIND>(a, stage, rec_g, row, gl, sc, tid);
-        } else if (valid) {
-            int n, ll, h, gl, row;
-            item_coords<D>(a, it, n, ll, h, gl, row);
-            uint8_t *rec_g = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[gl];
-            switch (width) {
-                case 2: item_uniform<D, 2, KIND>(a, stage, rec_g, row, gl, sc, tid); break;
-                case 4: item_uniform<D, 4, KIND>(a, stage, rec_g, row, gl, sc, tid); break;
-                case 6: item_uniform<D, 6, KIND>(a, stage, rec_g, row, gl, sc, tid); break;
-                case 8: item_uniform<D, 8, KIND>(a, stage, rec_g, row, gl, sc, tid); break;
-                case kPivotBits: item_pivot<D, KIND>(a, stage, rec_g, row, sc, tid); break;
-                default: if (tid == 0) flag_error(a.err, kErrArgs); break;
+        if (tid == 0 && it != (int)blockIdx.x) {
+            const int ps = (s + kStages - 1) % kStages;
+            const int nx = it + (kStages - 1) * G;
+            if (nx < a.n_items) {
+                cp_async_wait_all();
+                issue_item<D, KIND, MODE>(a, nx, sc.dring[dsel], sc.dslot[dsel], stages + ps * a.stage_bytes,
+                                          &bars[ps], sc.meta[ps]);
+                dsel ^= 1;
+                if (nx + G < a.n_items) prefetch_desc<D>(a, nx + G, sc, dsel);
             }
         }
-        __syncthreads();
-        if (tid == 0) {
-            const int nx = it + kStages * gridDim.x;
-            if (nx < a.n_items) issue_item<D, KIND>(a, nx, stage, &bars[s], sc.meta[s]);
+        uint8_t *stage = stages + s * a.stage_bytes;
+        const int width = sc.meta[s][1];
+        const int valid = sc.meta[s][2];
+        uint8_t *rec_g = reinterpret_cast<uint8_t *>((uintptr_t)(uint32_t)sc.meta[s][4] |
+                                                     ((uintptr_t)(uint32_t)sc.meta[s][5] << 32));
+        if (valid) {
+            int n, ll, h, gl, row;
+            item_coords<D>(a, it, n, ll, h, gl, row);
+            if (MODE == 1) {
+                item_rows<D, KIND>(a, stage, rec_g, row, (uint32_t)sc.meta[s][3], sc, tid);
+            } else {
+                switch (width) {
+                    case 2: item_uniform<D, 2, KIND>(a, stage, rec_g, row, sc, tid); break;
+                    case 4: item_uniform<D, 4, KIND>(a, stage, rec_g, row, sc, tid); break;
+                    case 6: item_uniform<D, 6, KIND>(a, stage, rec_g, row, sc, tid); break;
+                    case 8: item_uniform<D, 8, KIND>(a, stage, rec_g, row, sc, tid); break;
+                    case kPivotBits: item_pivot<D, KIND>(a, stage, rec_g, row, sc, tid); break;
+                    default: if (tid == 0) flag_error(a.err, kErrArgs); break;
+                }
+            }
         }
         if (++s == kStages) { s = 0; phase ^= 1u; }
     }
@@ -1152,7 +1214,7 @@ __global__ void __launch_bounds__(2 * D) k_requant_pack(Args a) {
         __syncthreads();
         const uint32_t codes_bytes = a.t.codes_bytes[gl];
         float *rec_r = reinterpret_cast<float *>(rec + codes_bytes);
-        fit_rows<D>(S, sc, tid, codes, rec_r, rec_r + D);
+        fit_rows<D>(S, sc, tid, sc.rw, sc.roff, sc.rho, sc.wbar, codes, rec_r, rec_r + D);
         copy_out<D>(rec, codes, codes_bytes, tid);
         return;
     }
@@ -1168,10 +1230,10 @@ __global__ void __launch_bounds__(2 * D) k_requant_pack(Args a) {
     if (tid == 0) sc.nz = a.neg_zero;
     __syncthreads();
     switch (width) {
-        case 2: fit_pack<D, 2>(S, rec, sc, tid); break;
-        case 4: fit_pack<D, 4>(S, rec, sc, tid); break;
-        case 6: fit_pack<D, 6>(S, rec, sc, tid); break;
-        case 8: fit_pack<D, 8>(S, rec, sc, tid); break;
+        case 2: fit_pack<D, 2>(S, rec, sc, tid, sc.rho, sc.wbar); break;
+        case 4: fit_pack<D, 4>(S, rec, sc, tid, sc.rho, sc.wbar); break;
+        case 6: fit_pack<D, 6>(S, rec, sc, tid, sc.rho, sc.wbar); break;
+        case 8: fit_pack<D, 8>(S, rec, sc, tid, sc.rho, sc.wbar); break;
         default: if (tid == 0) flag_error(a.err, kErrArgs); break;
     }
 }
@@ -1299,7 +1361,7 @@ __device__ void dist_uniform(const float *Sg, int gl, int m, int n_bits, double 
         S[r][0] = make_float2(v.x, v.y);
         S[r][1] = make_float2(v.z, v.w);
     }
-    fit_scales<D, B>(S, sc, tid, nullptr, nullptr);
+    fit_scales<D, B>(S, sc, tid, sc.rho, sc.wbar, nullptr, nullptr);
     float cc[4], icc[4];
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) { cc[jj] = sc.cold[j0 + jj]; icc[jj] = sc.ic[j0 + jj]; }
