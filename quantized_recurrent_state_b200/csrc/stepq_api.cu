@@ -651,14 +651,28 @@ extern "C" int stepq_ctx_create(const stepq_plan *plan, void *main_stream, void 
         o += align_up(reserve, 64);
         return dst;
     };
-    // per-head descriptor for the step kernels' copy issue: one 16-byte read
+    // Step-kernel descriptors, one 16-byte read per item: per layer, the
+    // heads in width order (per-head units; per-row units keep head order),
+    // so concurrently running items mostly share one width's code path.
+    // Entry: record offset low word, (offset bits 32..47) | head << 16,
+    // staged record bytes (0 for an FP16 head), width | codes bytes << 8.
+    if (p->slot_bytes >> 48) { cudaFree(c->tables_mem); delete c; return fail(STEPQ_EFORMAT, "ctx_create: slot above 2^48 bytes"); }
     std::vector<uint32_t> desc(4 * heads);
-    for (size_t hd = 0; hd < heads; ++hd) {
-        const bool staged = !(p->mode == 0 && p->head_width[hd] == STEPQ_PIVOT_BITS);
-        desc[4 * hd] = (uint32_t)p->rec_off[hd];
-        desc[4 * hd + 1] = (uint32_t)(p->rec_off[hd] >> 32);
-        desc[4 * hd + 2] = staged ? p->rec_bytes[hd] : 0u;
-        desc[4 * hd + 3] = (uint32_t)(p->mode == 0 ? p->head_width[hd] : 0) | (p->codes_bytes[hd] << 8);
+    for (int l = 0; l < p->L; ++l) {
+        std::vector<int> order(p->H);
+        for (int h = 0; h < p->H; ++h) order[h] = h;
+        if (p->mode == 0)
+            std::stable_sort(order.begin(), order.end(), [&](int x, int y) {
+                return p->head_width[(size_t)l * p->H + x] < p->head_width[(size_t)l * p->H + y];
+            });
+        for (int k = 0; k < p->H; ++k) {
+            const size_t hd = (size_t)l * p->H + order[k], e = 4 * ((size_t)l * p->H + k);
+            const bool staged = !(p->mode == 0 && p->head_width[hd] == STEPQ_PIVOT_BITS);
+            desc[e] = (uint32_t)p->rec_off[hd];
+            desc[e + 1] = (uint32_t)((p->rec_off[hd] >> 32) & 0xffffu) | ((uint32_t)order[k] << 16);
+            desc[e + 2] = staged ? p->rec_bytes[hd] : 0u;
+            desc[e + 3] = (uint32_t)(p->mode == 0 ? p->head_width[hd] : 0) | (p->codes_bytes[hd] << 8);
+        }
     }
     c->t.desc = (const uint4 *)put(desc.data(), sz_desc, sz_desc);
     c->t.rec_off = (const uint64_t *)put(p->rec_off.data(), sz_off, sz_off);

@@ -69,7 +69,6 @@ struct __align__(16) Scratch {
     float2 rinv2[D];  // (fl(1/r_i), fl(1/r_i)) of the refit
     float2 bw2[D];    // (b_i, b_i) of the refit
     float rowr[D];    // r_i of the refit
-    float cpr[D];     // c_j 2^-12
     float cold[D];    // c_j (old on entry, refitted after fit_scales)
     float wv[D];      // w_j
     float ic0[D];
@@ -95,7 +94,7 @@ constexpr bool scratch_aligned() {
     return offsetof(S, u) % 16 == 0 && offsetof(S, rsum) % 16 == 0 && offsetof(S, pf0) % 16 == 0 &&
            offsetof(S, pf1) % 16 == 0 && offsetof(S, a2) % 16 == 0 && offsetof(S, k2) % 16 == 0 &&
            offsetof(S, kap) % 16 == 0 && offsetof(S, qt) % 16 == 0 && offsetof(S, rinv2) % 16 == 0 &&
-           offsetof(S, bw2) % 16 == 0 && offsetof(S, cpr) % 16 == 0 && offsetof(S, cold) % 16 == 0 &&
+           offsetof(S, bw2) % 16 == 0 && offsetof(S, cold) % 16 == 0 &&
            offsetof(S, wv) % 16 == 0 && offsetof(S, ic0) % 16 == 0 && offsetof(S, ic) % 16 == 0 &&
            offsetof(S, dring) % 16 == 0 && (sizeof(float) * Scratch<D>::RS) % 16 == 0;
 }
@@ -113,13 +112,25 @@ __device__ __forceinline__ void item_coords(const Args &a, int it, int &n, int &
     row = (n * a.nL_in + a.l_in0 + ll) * a.H + h;  // index of the (request, layer, head) input row
 }
 
+// Item order of the step kernels: requests fastest, then the layer's heads
+// in the order of its descriptor table (sorted by width on the host, so the
+// CTAs of an SM run one width's code at a time), then layers.  Returns the
+// request n, the layer ll inside the launch and the descriptor index.
+template <int D>
+__device__ __forceinline__ void step_coords(const Args &a, int it, int &n, int &ll, int &di) {
+    n = it % a.n_req;
+    const int k = it / a.n_req;
+    ll = k / a.H;
+    di = (a.lb + ll) * a.H + (k - ll * a.H);
+}
+
 // Thread 0: start the 16-byte descriptor and the slot of item `it` on their
 // way into the descriptor ring entry e (cp.async, completion by group).
 template <int D>
 __device__ __forceinline__ void prefetch_desc(const Args &a, int it, Scratch<D> &sc, int e) {
-    int n, ll, h, gl, row;
-    item_coords<D>(a, it, n, ll, h, gl, row);
-    cp_async16(&sc.dring[e], &a.t.desc[gl]);
+    int n, ll, di;
+    step_coords<D>(a, it, n, ll, di);
+    cp_async16(&sc.dring[e], &a.t.desc[di]);
     cp_async4(&sc.dslot[e], &a.slots[n]);
     cp_async_commit();
 }
@@ -129,16 +140,20 @@ __device__ __forceinline__ void prefetch_desc(const Args &a, int it, Scratch<D> 
 // by cp.async, all completing on `bar`; or mark the item invalid.
 template <int D, int KIND, int MODE>
 __device__ void issue_item(const Args &a, int it, uint4 dsc, int slot, uint8_t *stage, uint64_t *bar, int *meta) {
-    int n, ll, h, gl, row;
-    item_coords<D>(a, it, n, ll, h, gl, row);
+    int n, ll, di;
+    step_coords<D>(a, it, n, ll, di);
+    const int h = (int)(dsc.y >> 16);
+    const int gl = (a.lb + ll) * a.H + h;
+    const int row = (n * a.nL_in + a.l_in0 + ll) * a.H + h;  // the (request, layer, head) input row
     const bool ok = slot >= 0 && slot < a.n_slots;
-    const uint8_t *rec = a.pool + (uint64_t)slot * a.slot_bytes + ((uint64_t)dsc.y << 32 | dsc.x);
+    const uint8_t *rec = a.pool + (uint64_t)slot * a.slot_bytes + ((uint64_t)(dsc.y & 0xffffu) << 32 | dsc.x);
     meta[0] = slot;
     meta[1] = (int)(dsc.w & 0xffu);
     meta[2] = ok ? 1 : 0;
     meta[3] = (int)(dsc.w >> 8);
     meta[4] = (int)(uint32_t)(uintptr_t)rec;
     meta[5] = (int)(uint32_t)((uintptr_t)rec >> 32);
+    meta[6] = row;
     if (!ok) {
         flag_error(a.err, kErrBadSlot);
         mbar_arrive(bar);
@@ -322,6 +337,26 @@ __device__ __forceinline__ uint32_t final_e(float t) {
     return (uint32_t)__viaddmin_s32_relu(__float_as_int(t), -LO, 2 * Q);
 }
 
+// Column refit from the per-band least-squares partials in pf0 (numerator)
+// and pf1 (denominator): c_j = num / den (c0_j when den = 0), two threads
+// per column; each sums four bands pairwise and the pair adds the halves,
+// which is the balanced tree over the eight bands.
+template <int D>
+__device__ __forceinline__ void column_ls_fit(Scratch<D> &sc, int tid, float *rec_c) {
+    const int j = tid >> 1, h = tid & 1, b0 = 4 * h;
+    float num = (sc.pf0[b0][j] + sc.pf0[b0 + 1][j]) + (sc.pf0[b0 + 2][j] + sc.pf0[b0 + 3][j]);
+    float den = (sc.pf1[b0][j] + sc.pf1[b0 + 1][j]) + (sc.pf1[b0 + 2][j] + sc.pf1[b0 + 3][j]);
+    num = num + __shfl_xor_sync(0xffffffffu, num, 1);
+    den = den + __shfl_xor_sync(0xffffffffu, den, 1);
+    if (h == 0) {
+        const float c = (den > 0.0f) ? __fdiv_rn(num, den) : sc.c0[j];
+        sc.ic[j] = __frcp_rn(c);
+        sc.cold[j] = c;
+        if (rec_c) rec_c[j] = c;
+    }
+    __syncthreads();
+}
+
 // ---------------------------------------------------------------------------
 // Refit of the fp32 tile S held in registers as column pairs (all rows at
 // width B).  On return S holds y = fl(S * fl(1/r)); sc.rowr[i] = r_i,
@@ -375,9 +410,10 @@ __device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const
         }
     }
     __syncwarp();
-    // 2. y = fl(S * (1/r)) in place; 3. column absmax partials
+    // 2. y = fl(S * (1/r)) in place; 3. column absmax partials, as
+    //    max(max_i y_ij, -min_i y_ij) (no absolute values needed)
     {
-        float2 m01 = make_float2(0.0f, 0.0f), m23 = make_float2(0.0f, 0.0f);
+        float mx[4] = {0.0f, 0.0f, 0.0f, 0.0f}, mn[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
         for (int r = 0; r < RT; r += 2) {
             const float4 f = *reinterpret_cast<const float4 *>(&sc.rinv2[g * RT + r]);
@@ -386,21 +422,27 @@ __device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const
             S[r][1] = mul2(S[r][1], i0);
             S[r + 1][0] = mul2(S[r + 1][0], i1);
             S[r + 1][1] = mul2(S[r + 1][1], i1);
-            m01.x = fmaxf(m01.x, fmaxf(fabsf(S[r][0].x), fabsf(S[r + 1][0].x)));
-            m01.y = fmaxf(m01.y, fmaxf(fabsf(S[r][0].y), fabsf(S[r + 1][0].y)));
-            m23.x = fmaxf(m23.x, fmaxf(fabsf(S[r][1].x), fabsf(S[r + 1][1].x)));
-            m23.y = fmaxf(m23.y, fmaxf(fabsf(S[r][1].y), fabsf(S[r + 1][1].y)));
+            const float ya[4] = {S[r][0].x, S[r][0].y, S[r][1].x, S[r][1].y};
+            const float yb[4] = {S[r + 1][0].x, S[r + 1][0].y, S[r + 1][1].x, S[r + 1][1].y};
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                mx[jj] = fmaxf(mx[jj], fmaxf(ya[jj], yb[jj]));
+                mn[jj] = fminf(mn[jj], fminf(ya[jj], yb[jj]));
+            }
         }
-        *reinterpret_cast<float4 *>(&sc.pf0[g][j0]) = make_float4(m01.x, m01.y, m23.x, m23.y);
+        *reinterpret_cast<float4 *>(&sc.pf0[g][j0]) =
+            make_float4(fmaxf(mx[0], -mn[0]), fmaxf(mx[1], -mn[1]), fmaxf(mx[2], -mn[2]), fmaxf(mx[3], -mn[3]));
     }
     __syncthreads();
-    if (tid < D) {
-        float m = 0.0f;
-#pragma unroll
-        for (int b = 0; b < 8; ++b) m = fmaxf(m, sc.pf0[b][tid]);
-        const float c0 = (m == 0.0f) ? 1.0f : __fdiv_rn(m, (float)Q);
-        sc.c0[tid] = c0;
-        sc.ic0[tid] = __frcp_rn(c0);
+    {  // two threads per column, four bands each
+        const int j = tid >> 1, h = tid & 1;
+        float m = fmaxf(fmaxf(sc.pf0[4 * h][j], sc.pf0[4 * h + 1][j]), fmaxf(sc.pf0[4 * h + 2][j], sc.pf0[4 * h + 3][j]));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        if (h == 0) {
+            const float c0 = (m == 0.0f) ? 1.0f : __fdiv_rn(m, (float)Q);
+            sc.c0[j] = c0;
+            sc.ic0[j] = __frcp_rn(c0);
+        }
     }
     __syncthreads();
     // 4. z0 and the weighted least-squares sums (pairwise over rows)
@@ -432,18 +474,7 @@ __device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const
         }
     }
     __syncthreads();
-    if (tid < D) {
-        float xn[8], xd[8];
-#pragma unroll
-        for (int b = 0; b < 8; ++b) { xn[b] = sc.pf0[b][tid]; xd[b] = sc.pf1[b][tid]; }
-        const float num = tree_sum1<8>(xn);
-        const float den = tree_sum1<8>(xd);
-        const float c = (den > 0.0f) ? __fdiv_rn(num, den) : sc.c0[tid];
-        sc.ic[tid] = __frcp_rn(c);
-        sc.cold[tid] = c;
-        if (rec_c) rec_c[tid] = c;
-    }
-    __syncthreads();
+    column_ls_fit<D>(sc, tid, rec_c);
 }
 
 // Refit and pack into the record at `rec` (global): codes, r, c.
@@ -509,23 +540,24 @@ __device__ __forceinline__ void load_pivot(const uint8_t *rec, int tid, float2 (
     }
 }
 
-// Per-band fp64 sums of three per-row values: thread tid holds row tid (0 for
-// tid >= D); rows of band g are tid in [g RT, g RT + RT).  For D >= 32 only
-// the warps holding rows take part; below that the whole warp does.
+// Per-band fp64 sums of three per-row values.  Warp w holds rows
+// [16 w, 16 w + 16): lane L < 16 carries row 16 w + L (lanes 16..31 carry
+// zeros); a band is RT consecutive rows, so the butterfly over RT lanes
+// stays inside the warp.
 template <int D>
 __device__ __forceinline__ void band_sums(Scratch<D> &sc, int tid, double x0, double x1, double x2) {
     constexpr int RT = D / 8;
-    if (D >= 32 && tid >= D) return;
 #pragma unroll
     for (int m = 1; m < RT; m <<= 1) {
         x0 += __shfl_xor_sync(0xffffffffu, x0, m);
         x1 += __shfl_xor_sync(0xffffffffu, x1, m);
         x2 += __shfl_xor_sync(0xffffffffu, x2, m);
     }
-    if (tid < D && (tid % RT) == 0) {
-        sc.bandK[tid / RT] = x0;
-        sc.bandQ[tid / RT] = x1;
-        sc.bandQK[tid / RT] = x2;
+    const int lane = tid & 31, i = 16 * (tid >> 5) + lane;
+    if (lane < 16 && (lane % RT) == 0) {
+        sc.bandK[i / RT] = x0;
+        sc.bandQ[i / RT] = x1;
+        sc.bandQK[i / RT] = x2;
     }
 }
 
@@ -533,7 +565,7 @@ __device__ __forceinline__ void band_sums(Scratch<D> &sc, int tid, double x0, do
 // (already relative to the offset-binary bias), two threads per column.
 template <int D, int KIND>
 __device__ __forceinline__ void finish_columns(const Args &a, Scratch<D> &sc, int tid, int row, float beta,
-                                               const float *vs, bool scaled) {
+                                               const float *vs, const float *cs) {
     const int j = tid >> 1, h = tid & 1, b0 = 4 * h;
     double su = (sc.u.col.pU[b0][j] + sc.u.col.pU[b0 + 1][j]) + (sc.u.col.pU[b0 + 2][j] + sc.u.col.pU[b0 + 3][j]);
     double so = (sc.u.col.pO[b0][j] + sc.u.col.pO[b0 + 1][j]) + (sc.u.col.pO[b0 + 2][j] + sc.u.col.pO[b0 + 3][j]);
@@ -541,7 +573,7 @@ __device__ __forceinline__ void finish_columns(const Args &a, Scratch<D> &sc, in
     su += __shfl_xor_sync(0xffffffffu, su, 1);
     so += __shfl_xor_sync(0xffffffffu, so, 1);
     qk += __shfl_xor_sync(0xffffffffu, qk, 1);
-    const double cj = scaled ? (double)sc.cold[j] : 1.0;
+    const double cj = cs ? (double)cs[j] : 1.0;
     const float u = __double2float_rn(cj * su);
     const float w = __fmul_rn(beta, __fsub_rn(vs[j], u));
     const float o = __double2float_rn(cj * so + qk * (double)w);
@@ -574,17 +606,14 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
     const float alpha = ab[0];
     const float beta = ab[1];
 
-    // per-row and per-column parameters
+    // per-row parameters of this warp's 16 rows (only this warp reads them)
     double bk = 0.0, bq = 0.0, bqk = 0.0;
-    if (tid < D) {
-        const int i = tid;
+    if ((tid & 31) < 16) {
+        const int i = 16 * (tid >> 5) + (tid & 31);
         const float ai = __fmul_rn(alpha, st_r[i]);
         const float ki = ks[i];
         sc.a2[i] = make_float2(ai, ai);
         sc.k2[i] = make_float2(ki, ki);
-        sc.cpr[i] = __fmul_rn(st_c[i], 1.0f / 4096.0f);
-        sc.cold[i] = st_c[i];
-        if (KIND == kFitPack) sc.wv[i] = xs[i];
         if (KIND != kFitPack) {
             const double ka = (double)ks[i] * (double)ai;
             const double qa = (double)qs[i] * (double)ai;
@@ -596,7 +625,7 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
         }
     }
     if (KIND != kFitPack) band_sums<D>(sc, tid, bk, bq, bqk);
-    __syncthreads();
+    __syncwarp();
 
     uint32_t W[Stream<D, B>::NW];
     W[Stream<D, B>::NW - 1] = 0u;
@@ -605,10 +634,11 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
     float2 S[RT][2];
     double accU[4] = {0.0, 0.0, 0.0, 0.0}, accO[4] = {0.0, 0.0, 0.0, 0.0};
     float2 cp01, cp23;
-    if (KIND != kDecode) {
-        const float4 c4 = *reinterpret_cast<const float4 *>(&sc.cpr[j0]);
-        cp01 = make_float2(c4.x, c4.y);
-        cp23 = make_float2(c4.z, c4.w);
+    if (KIND != kDecode) {  // c_j 2^-12 of this thread's columns (exact scaling)
+        const float4 c4 = *reinterpret_cast<const float4 *>(&st_c[j0]);
+        const float2 s12 = make_float2(1.0f / 4096.0f, 1.0f / 4096.0f);
+        cp01 = mul2(make_float2(c4.x, c4.y), s12);
+        cp23 = mul2(make_float2(c4.z, c4.w), s12);
     }
     constexpr float ZB = 8388608.0f + (float)OFF * 4096.0f;
     const float2 nzb = make_float2(-ZB, -ZB);
@@ -662,12 +692,12 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
         *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0]) = make_double2(accO[0] - bQ, accO[1] - bQ);
         *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0 + 2]) = make_double2(accO[2] - bQ, accO[3] - bQ);
         __syncthreads();
-        finish_columns<D, KIND>(a, sc, tid, row, beta, vs, true);
+        finish_columns<D, KIND>(a, sc, tid, row, beta, vs, st_c);
         if (KIND == kFused) __syncthreads();
     }
 
     if (KIND != kDecode) {
-        const float4 w4 = *reinterpret_cast<const float4 *>(&sc.wv[j0]);
+        const float4 w4 = *reinterpret_cast<const float4 *>(KIND == kFitPack ? &xs[j0] : &sc.wv[j0]);
         const float2 w01 = make_float2(w4.x, w4.y);
         const float2 w23 = make_float2(w4.z, w4.w);
 #pragma unroll
@@ -700,17 +730,17 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
     const float alpha = ab[0];
     const float beta = ab[1];
     double bqk = 0.0;
-    if (tid < D) {
-        sc.k2[tid] = make_float2(ks[tid], ks[tid]);
-        if (KIND == kFitPack) sc.wv[tid] = xs[tid];
+    if ((tid & 31) < 16) {  // this warp's 16 rows
+        const int i = 16 * (tid >> 5) + (tid & 31);
+        sc.k2[i] = make_float2(ks[i], ks[i]);
         if (KIND != kFitPack) {
-            sc.kap[tid] = (double)ks[tid] * (double)alpha;
-            sc.qt[tid] = (double)qs[tid] * (double)alpha;
-            bqk = (double)qs[tid] * (double)ks[tid];
+            sc.kap[i] = (double)ks[i] * (double)alpha;
+            sc.qt[i] = (double)qs[i] * (double)alpha;
+            bqk = (double)qs[i] * (double)ks[i];
         }
     }
     if (KIND != kFitPack) band_sums<D>(sc, tid, 0.0, 0.0, bqk);
-    __syncthreads();
+    __syncwarp();
     float2 S[RT][2];
     load_pivot<D>(rec_g, tid, S);
     if (KIND != kFitPack) {
@@ -732,13 +762,14 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
             sc.u.col.pO[g][j0 + jj] = accO[jj];
         }
         __syncthreads();
-        finish_columns<D, KIND>(a, sc, tid, row, beta, vs, false);
+        finish_columns<D, KIND>(a, sc, tid, row, beta, vs, nullptr);
         if (KIND == kFused) __syncthreads();
     }
     if (KIND != kDecode) {
         const float2 al = make_float2(alpha, alpha);
-        const float2 w01 = make_float2(sc.wv[j0], sc.wv[j0 + 1]);
-        const float2 w23 = make_float2(sc.wv[j0 + 2], sc.wv[j0 + 3]);
+        const float4 w4 = *reinterpret_cast<const float4 *>(KIND == kFitPack ? &xs[j0] : &sc.wv[j0]);
+        const float2 w01 = make_float2(w4.x, w4.y);
+        const float2 w23 = make_float2(w4.z, w4.w);
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
             const float2 k2 = sc.k2[g * RT + r];
@@ -861,19 +892,26 @@ __device__ void fit_rows(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const u
             *reinterpret_cast<float4 *>(&sc.u.pmax[c][g][j0]) = make_float4(m[c][0], m[c][1], m[c][2], m[c][3]);
     }
     __syncthreads();
-    if (tid < D) {
-        float c0 = 0.0f;
+    {  // two threads per column, four bands each
+        const int j = tid >> 1, h = tid & 1, b0 = 4 * h;
+        float mm[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            float mm = 0.0f;
-#pragma unroll
-            for (int b = 0; b < 8; ++b) mm = fmaxf(mm, sc.u.pmax[c][b][tid]);
-            const int q = (1 << (2 * c + 1)) - 1;  // widths 2, 4, 6, 8
-            if (mm > 0.0f) c0 = fmaxf(c0, __fdiv_rn(mm, (float)q));
+            mm[c] = fmaxf(fmaxf(sc.u.pmax[c][b0][j], sc.u.pmax[c][b0 + 1][j]),
+                          fmaxf(sc.u.pmax[c][b0 + 2][j], sc.u.pmax[c][b0 + 3][j]));
+            mm[c] = fmaxf(mm[c], __shfl_xor_sync(0xffffffffu, mm[c], 1));
         }
-        if (c0 == 0.0f) c0 = 1.0f;
-        sc.c0[tid] = c0;
-        sc.ic0[tid] = __frcp_rn(c0);
+        if (h == 0) {
+            float c0 = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int q = (1 << (2 * c + 1)) - 1;  // widths 2, 4, 6, 8
+                if (mm[c] > 0.0f) c0 = fmaxf(c0, __fdiv_rn(mm[c], (float)q));
+            }
+            if (c0 == 0.0f) c0 = 1.0f;
+            sc.c0[j] = c0;
+            sc.ic0[j] = __frcp_rn(c0);
+        }
     }
     __syncthreads();
     // 4. z0 and the weighted least-squares sums over the quantized rows
@@ -906,18 +944,7 @@ __device__ void fit_rows(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const u
         }
     }
     __syncthreads();
-    if (tid < D) {
-        float xn[8], xd[8];
-#pragma unroll
-        for (int b = 0; b < 8; ++b) { xn[b] = sc.pf0[b][tid]; xd[b] = sc.pf1[b][tid]; }
-        const float num = tree_sum1<8>(xn);
-        const float den = tree_sum1<8>(xd);
-        const float c = (den > 0.0f) ? __fdiv_rn(num, den) : sc.c0[tid];
-        sc.ic[tid] = __frcp_rn(c);
-        sc.cold[tid] = c;
-        if (rec_c) rec_c[tid] = c;
-    }
-    __syncthreads();
+    column_ls_fit<D>(sc, tid, rec_c);
     // 5. final codes (or binary16) of every row into the shared codes block
     {
         const float4 ic4 = *reinterpret_cast<const float4 *>(&sc.ic[j0]);
@@ -984,16 +1011,13 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
     const float beta = (tf + kTailRw * D + D / 4)[1];
 
     double bk = 0.0, bq = 0.0, bqk = 0.0;
-    if (tid < D) {
-        const int i = tid;
+    if ((tid & 31) < 16) {  // this warp's 16 rows
+        const int i = 16 * (tid >> 5) + (tid & 31);
         const int b = rw[i];
         const float al = als[i];
         const float ai = (b == kPivotBits) ? al : __fmul_rn(al, st_r[i]);
         sc.a2[i] = make_float2(ai, ai);
         sc.k2[i] = make_float2(ks[i], ks[i]);
-        sc.cpr[i] = __fmul_rn(st_c[i], 1.0f / 4096.0f);
-        sc.cold[i] = st_c[i];
-        if (KIND == kFitPack) sc.wv[i] = xs[i];
         if (KIND != kFitPack) {
             const double ka = (double)ks[i] * (double)ai;
             const double qa = (double)qs[i] * (double)ai;
@@ -1010,13 +1034,14 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
         }
     }
     if (KIND != kFitPack) band_sums<D>(sc, tid, bk, bq, bqk);
-    __syncthreads();
+    __syncwarp();
 
     float2 S[RT][2];
     double accU[4] = {0.0, 0.0, 0.0, 0.0}, accO[4] = {0.0, 0.0, 0.0, 0.0};
     double accUp[4] = {0.0, 0.0, 0.0, 0.0}, accOp[4] = {0.0, 0.0, 0.0, 0.0};
-    const float4 c4 = *reinterpret_cast<const float4 *>(&sc.cpr[j0]);
-    const float2 cp01 = make_float2(c4.x, c4.y), cp23 = make_float2(c4.z, c4.w);
+    const float4 c4 = *reinterpret_cast<const float4 *>(&st_c[j0]);
+    const float2 s12 = make_float2(1.0f / 4096.0f, 1.0f / 4096.0f);
+    const float2 cp01 = mul2(make_float2(c4.x, c4.y), s12), cp23 = mul2(make_float2(c4.z, c4.w), s12);
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
         const int i = g * RT + r;
@@ -1067,7 +1092,7 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
         double pu[4], po[4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-            const double cj = (double)sc.cold[j0 + jj];
+            const double cj = (double)st_c[j0 + jj];
             pu[jj] = cj * (accU[jj] - bK) + accUp[jj];
             po[jj] = cj * (accO[jj] - bQ) + accOp[jj];
         }
@@ -1076,12 +1101,12 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
         *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0]) = make_double2(po[0], po[1]);
         *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0 + 2]) = make_double2(po[2], po[3]);
         __syncthreads();
-        finish_columns<D, KIND>(a, sc, tid, row, beta, vs, false);
+        finish_columns<D, KIND>(a, sc, tid, row, beta, vs, nullptr);
         if (KIND == kFused) __syncthreads();
     }
 
     if (KIND != kDecode) {
-        const float4 w4 = *reinterpret_cast<const float4 *>(&sc.wv[j0]);
+        const float4 w4 = *reinterpret_cast<const float4 *>(KIND == kFitPack ? &xs[j0] : &sc.wv[j0]);
         const float2 w01 = make_float2(w4.x, w4.y);
         const float2 w23 = make_float2(w4.z, w4.w);
 #pragma unroll
@@ -1122,9 +1147,9 @@ __global__ void __launch_bounds__(2 * D, 2) k_step(Args a) {
         for (int s = 0; s < kStages; ++s) {
             const int it = blockIdx.x + s * G;
             if (it >= a.n_items) break;
-            int n, ll, h, gl, row;
-            item_coords<D>(a, it, n, ll, h, gl, row);
-            issue_item<D, KIND, MODE>(a, it, a.t.desc[gl], a.slots[n], stages + s * a.stage_bytes, &bars[s],
+            int n, ll, di;
+            step_coords<D>(a, it, n, ll, di);
+            issue_item<D, KIND, MODE>(a, it, a.t.desc[di], a.slots[n], stages + s * a.stage_bytes, &bars[s],
                                       sc.meta[s]);
         }
         const int nx = blockIdx.x + kStages * G;
@@ -1161,8 +1186,7 @@ __global__ void __launch_bounds__(2 * D, 2) k_step(Args a) {
         uint8_t *rec_g = reinterpret_cast<uint8_t *>((uintptr_t)(uint32_t)sc.meta[s][4] |
                                                      ((uintptr_t)(uint32_t)sc.meta[s][5] << 32));
         if (valid) {
-            int n, ll, h, gl, row;
-            item_coords<D>(a, it, n, ll, h, gl, row);
+            const int row = sc.meta[s][6];
             if (MODE == 1) {
                 item_rows<D, KIND>(a, stage, rec_g, row, (uint32_t)sc.meta[s][3], sc, tid);
             } else {
