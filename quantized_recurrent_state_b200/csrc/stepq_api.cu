@@ -560,6 +560,7 @@ stepq::Args base_args(stepq_ctx *c, void *pool, const int32_t *slots, int n_req,
     a.t = c->t;
     a.err = c->err;
     a.neg_zero = -0.0f;
+    a.x_bits = 0x4B000000u;
     return a;
 }
 

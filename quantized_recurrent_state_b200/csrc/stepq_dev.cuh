@@ -53,6 +53,7 @@ struct Args {
     Tables t;
     int *err;
     float neg_zero;          // -0.0f (a run-time value the compiler cannot fold)
+    uint32_t x_bits;         // 0x4B000000, the exponent word of the X encoding, held in a register
     uint32_t stage_bytes;    // bytes of one pipeline stage
     uint32_t rec_stage_bytes;// bytes reserved for the record in a stage
 };
@@ -183,7 +184,7 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 // ---------------------------------------------------------------------------
 
 template <int B>
-__device__ __forceinline__ uint32_t field_x(const uint32_t *W, int p) {
+__device__ __forceinline__ uint32_t field_x(const uint32_t *W, int p, uint32_t xbits = 0x4B000000u) {
     const int bit = p * B;
     const int w = bit >> 5;
     const int s = bit & 31;
@@ -193,7 +194,7 @@ __device__ __forceinline__ uint32_t field_x(const uint32_t *W, int p) {
     } else {
         x = __funnelshift_r(W[w], W[w + 1], s - 12);
     }
-    return (x & (((1u << B) - 1u) << 12)) | 0x4B000000u;
+    return (x & (((1u << B) - 1u) << 12)) | xbits;
 }
 
 __device__ __forceinline__ double x_as_f64(uint32_t X) { return __hiloint2double((int)X, 0); }

@@ -410,10 +410,9 @@ __device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const
         }
     }
     __syncwarp();
-    // 2. y = fl(S * (1/r)) in place; 3. column absmax partials, as
-    //    max(max_i y_ij, -min_i y_ij) (no absolute values needed)
+    // 2. y = fl(S * (1/r)) in place; 3. column absmax partials
     {
-        float mx[4] = {0.0f, 0.0f, 0.0f, 0.0f}, mn[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        float2 m01 = make_float2(0.0f, 0.0f), m23 = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int r = 0; r < RT; r += 2) {
             const float4 f = *reinterpret_cast<const float4 *>(&sc.rinv2[g * RT + r]);
@@ -422,16 +421,12 @@ __device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const
             S[r][1] = mul2(S[r][1], i0);
             S[r + 1][0] = mul2(S[r + 1][0], i1);
             S[r + 1][1] = mul2(S[r + 1][1], i1);
-            const float ya[4] = {S[r][0].x, S[r][0].y, S[r][1].x, S[r][1].y};
-            const float yb[4] = {S[r + 1][0].x, S[r + 1][0].y, S[r + 1][1].x, S[r + 1][1].y};
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                mx[jj] = fmaxf(mx[jj], fmaxf(ya[jj], yb[jj]));
-                mn[jj] = fminf(mn[jj], fminf(ya[jj], yb[jj]));
-            }
+            m01.x = fmaxf(m01.x, fmaxf(fabsf(S[r][0].x), fabsf(S[r + 1][0].x)));
+            m01.y = fmaxf(m01.y, fmaxf(fabsf(S[r][0].y), fabsf(S[r + 1][0].y)));
+            m23.x = fmaxf(m23.x, fmaxf(fabsf(S[r][1].x), fabsf(S[r + 1][1].x)));
+            m23.y = fmaxf(m23.y, fmaxf(fabsf(S[r][1].y), fabsf(S[r + 1][1].y)));
         }
-        *reinterpret_cast<float4 *>(&sc.pf0[g][j0]) =
-            make_float4(fmaxf(mx[0], -mn[0]), fmaxf(mx[1], -mn[1]), fmaxf(mx[2], -mn[2]), fmaxf(mx[3], -mn[3]));
+        *reinterpret_cast<float4 *>(&sc.pf0[g][j0]) = make_float4(m01.x, m01.y, m23.x, m23.y);
     }
     __syncthreads();
     {  // two threads per column, four bands each
@@ -629,6 +624,7 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
 
     uint32_t W[Stream<D, B>::NW];
     W[Stream<D, B>::NW - 1] = 0u;
+    const uint32_t xb = a.x_bits;
     int loaded = -1;  // chunks are loaded as the rows reach them (fewer live registers)
 
     float2 S[RT][2];
@@ -664,7 +660,7 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
             }
             uint32_t X[4];
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) X[jj] = field_x<B>(W, 4 * (r + rr) + jj);
+            for (int jj = 0; jj < 4; ++jj) X[jj] = field_x<B>(W, 4 * (r + rr) + jj, xb);
             if (KIND != kFitPack) {
                 const double kap = rr ? kap2.y : kap2.x, qt = rr ? qt2.y : qt2.x;
 #pragma unroll
