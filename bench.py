@@ -340,6 +340,21 @@ def workload_of(args, synth):
     return wl
 
 
+def workload_config(wl, n, ws):
+    """The `config` keys both arms print for the same workload."""
+    L, H, D = wl.n_layers, wl.n_heads, wl.d
+    if wl.mode == 0:
+        name = (f"GDN state pool, {L} layers x {H} heads = {L * H} heads, d_k=d_v={D}, batch {n}, "
+                f"nominal {wl.nominal_bits:g}-bit plan over {sorted(wl.bits)}, {wl.n_pivots} FP16 pivot heads")
+    else:
+        name = (f"KDA per-key-row units, {L} layers x {H} heads x {D} rows = {L * H * D} rows, d_v={D}, "
+                f"batch {n}, Lagrangian nominal {wl.nominal_bits:g}-bit plan over {sorted(wl.bits)}, "
+                f"{wl.n_pivots} FP16 pivot rows, per-row gates")
+    return {"workload": name, "batch": n, "heads": L * H, "d": D,
+            "l2": "inputs larger than L2 (pool and q/k/v far above 126 MB)",
+            "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"}
+
+
 def run_product(args):
     import torch
     from quantized_recurrent_state_b200 import build as qbuild
@@ -489,16 +504,10 @@ def run_product(args):
             "dtype": "f32",
             "data": "synthetic",
             "config": {
-                "workload": (f"GDN state pool, {L} layers x {H} heads = {L * H} heads, d_k=d_v={D}, batch {n}, "
-                             f"nominal {wl.nominal_bits:g}-bit plan over {sorted(wl.bits)}, {wl.n_pivots} FP16 pivot heads")
-                if wl.mode == 0 else
-                            (f"KDA per-key-row units, {L} layers x {H} heads x {D} rows = {L * H * D} rows, d_v={D}, "
-                             f"batch {n}, Lagrangian nominal {wl.nominal_bits:g}-bit plan over {sorted(wl.bits)}, "
-                             f"{wl.n_pivots} FP16 pivot rows, per-row gates"),
-                "batch": n, "heads": L * H, "d": D, "variant": args.variant,
+                **workload_config(wl, n, ws),
+                "variant": args.variant,
                 "bits_per_value": plan.info.bits_per_value, "bits_per_value_s16": plan.info.bits_per_value_s16,
-                "pool_bytes": n * plan.slot_bytes, "l2": "inputs larger than L2 (pool and q/k/v far above 126 MB)",
-                "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                "pool_bytes": n * plan.slot_bytes,
             },
             "hbm_gbs": gbs,
             "hbm_frac": gbs / peak,
@@ -631,9 +640,7 @@ def run_reference(args):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
            "data": "synthetic",
-           "config": {"workload": f"GDN state pool, {wl.n_layers} layers x {wl.n_heads} heads, d={wl.d}, "
-                                  f"nominal {wl.nominal_bits:g}-bit plan, {wl.n_pivots} FP16 pivot heads (CPU oracle sample)",
-                      "batch": args.batch, "heads": wl.n_layers * wl.n_heads, "d": wl.d},
+           "config": {**workload_config(wl, args.batch, args.gpus), "variant": "oracle (CPU)"},
            "cpu_baseline": {"value": value, "unit": "head-steps/s", "cores": cores, "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": value, "unit": "head-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
