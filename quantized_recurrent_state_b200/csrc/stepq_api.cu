@@ -557,6 +557,8 @@ stepq::Args base_args(stepq_ctx *c, void *pool, const int32_t *slots, int n_req,
     a.H = c->plan->H;
     a.mode = c->plan->mode;
     a.n_items = n_req * (le - lb) * c->plan->H;
+    a.div_nreq = stepq::div_magic((uint32_t)n_req);
+    a.div_h = stepq::div_magic((uint32_t)c->plan->H);
     a.t = c->t;
     a.err = c->err;
     a.neg_zero = -0.0f;

@@ -45,6 +45,8 @@ struct Args {
     int H;
     int mode;
     int n_items;             // n_req * nL * H
+    uint64_t div_nreq;       // floor(2^64 / n_req) + 1 (0 when n_req == 1): n / n_req = umul64hi(n, div_nreq)
+    uint64_t div_h;          // the same for H
     const float *q, *k, *v, *alpha, *beta;
     float *o;
     float *w;                // workspace (decode writes, fit-pack reads)
@@ -236,5 +238,16 @@ __device__ __forceinline__ double lane_sum_f64(double v) {
 }
 
 __device__ __forceinline__ void flag_error(int *err, int code) { atomicOr(err, code); }
+
+// n / d for n < 2^32 with m = div_magic(d): floor(n m / 2^64) differs from
+// n / d by less than n / 2^64 < 1 / d, which cannot cross an integer.
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, uint64_t m) {
+    return m ? (uint32_t)__umul64hi((unsigned long long)n, (unsigned long long)m) : n;
+}
+
+__host__ __forceinline__ uint64_t div_magic(uint32_t d) {
+    if (d <= 1) return 0;
+    return (uint64_t)(((unsigned __int128)1 << 64) / d) + 1;
+}
 
 }  // namespace stepq

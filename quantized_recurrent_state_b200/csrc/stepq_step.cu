@@ -118,9 +118,9 @@ __device__ __forceinline__ void item_coords(const Args &a, int it, int &n, int &
 // request n, the layer ll inside the launch and the descriptor index.
 template <int D>
 __device__ __forceinline__ void step_coords(const Args &a, int it, int &n, int &ll, int &di) {
-    n = it % a.n_req;
-    const int k = it / a.n_req;
-    ll = k / a.H;
+    const int k = (int)fast_div((uint32_t)it, a.div_nreq);
+    n = it - k * a.n_req;
+    ll = (int)fast_div((uint32_t)k, a.div_h);
     di = (a.lb + ll) * a.H + (k - ll * a.H);
 }
 
