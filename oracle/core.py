@@ -71,6 +71,7 @@ def _declare(l):
     l.sq_pairwise_sum.argtypes = [P, I]
     l.sq_pairwise_sum.restype = F
     l.sq_quantize.argtypes = [I, P, P, P, P, P, P, P, P, P, P]
+    l.sq_quantize_absmax.argtypes = [I, P, P, P, P, P, P, P]
     l.sq_reconstruct.argtypes = [I, P, P, P, P, P, P]
     l.sq_step_from_codes.argtypes = [I, P, P, P, P, P, P, P, P, P, F, P, P, P, P]
     l.sq_step_fp32.argtypes = [I, P, P, P, P, P, F, P]
@@ -175,6 +176,20 @@ def quantize(D: int, widths, rho, wbar, S, return_z0: bool = False):
     lib().sq_quantize(D, _p(w), _p(rho), _p(wbar), _p(S), _p(z), _p(h), _p(r), _p(c), _p(tie), _p(z0))
     if return_z0:
         return z, h, r, c, tie, z0
+    return z, h, r, c, tie
+
+
+def quantize_absmax(D: int, widths, S):
+    """Return (z, h, r, c, tie) for one head under the per-row absmax
+    quantizer (see sq_quantize_absmax)."""
+    w = _i32(widths)
+    S = _f32(S).reshape(D, D)
+    z = np.zeros((D, D), dtype=np.int32)
+    h = np.zeros((D, D), dtype=np.uint16)
+    r = np.zeros(D, dtype=np.float32)
+    c = np.zeros(D, dtype=np.float32)
+    tie = np.zeros((D, D), dtype=np.uint8)
+    lib().sq_quantize_absmax(D, _p(w), _p(S), _p(z), _p(h), _p(r), _p(c), _p(tie))
     return z, h, r, c, tie
 
 

@@ -56,8 +56,15 @@ def unpack_head(mode: int, D: int, rw, rec: np.ndarray):
     return z, h, r, c
 
 
-def quantize_head(mode, D, rw, rho, wbar, S):
-    z, h, r, c, tie = core.quantize(D, rw, rho, wbar, S)
+QUANT_DUAL_AXIS = 0  # STEPQuant row/column fit (方法-3)
+QUANT_ABSMAX = 1     # ordinary per-row absmax baseline (实验)
+
+
+def quantize_head(mode, D, rw, rho, wbar, S, quantizer: int = QUANT_DUAL_AXIS):
+    if quantizer == QUANT_ABSMAX:
+        z, h, r, c, tie = core.quantize_absmax(D, rw, S)
+    else:
+        z, h, r, c, tie = core.quantize(D, rw, rho, wbar, S)
     return pack_head(mode, D, rw, z, h, r, c), tie
 
 
@@ -66,11 +73,11 @@ def reconstruct_head(mode, D, rw, rec):
     return core.reconstruct(D, rw, z, h, r, c)
 
 
-def step_head(mode, D, rw, rho, wbar, rec, q, k, v, alpha, beta):
+def step_head(mode, D, rw, rho, wbar, rec, q, k, v, alpha, beta, quantizer: int = QUANT_DUAL_AXIS):
     """Decode step of one packed head.  Returns (new record, o, tie, S_t, w)."""
     z, h, r, c = unpack_head(mode, D, rw, rec)
     S, o, u, w = core.step_from_codes(D, rw, z, h, r, c, q, k, v, alpha, beta)
-    new_rec, tie = quantize_head(mode, D, rw, rho, wbar, S)
+    new_rec, tie = quantize_head(mode, D, rw, rho, wbar, S, quantizer)
     return new_rec, o, tie, S, w
 
 
@@ -90,6 +97,7 @@ class PlanView:
         self.offsets, self.slot_bytes = plan_io.pool_layout(plan)
         self.rho = np.asarray(plan["rho"], np.float32).reshape(self.L, self.H, self.D)
         self.wbar = np.asarray(plan["wbar"], np.float32).reshape(self.L, self.H, self.D)
+        self.quantizer = int(plan.get("quantizer", QUANT_DUAL_AXIS))
 
     def rw(self, l, h):
         return plan_io.head_row_widths(self.plan, l, h)
@@ -102,7 +110,8 @@ class PlanView:
         return pool_slot[o:o + self.rec_bytes(l, h)]
 
     def quantize_into(self, pool_slot: np.ndarray, l, h, S):
-        rec, tie = quantize_head(self.mode, self.D, self.rw(l, h), self.rho[l, h], self.wbar[l, h], S)
+        rec, tie = quantize_head(self.mode, self.D, self.rw(l, h), self.rho[l, h], self.wbar[l, h], S,
+                                 self.quantizer)
         o = int(self.offsets[l * self.H + h])
         pool_slot[o:o + rec.size] = rec
         return tie
@@ -111,7 +120,7 @@ class PlanView:
         """Step one (slot, layer, head) in place; returns (o, tie, S_t, w)."""
         rec = self.record(pool_slot, l, h).copy()
         new_rec, o, tie, S, w = step_head(self.mode, self.D, self.rw(l, h), self.rho[l, h],
-                                          self.wbar[l, h], rec, q, k, v, alpha, beta)
+                                          self.wbar[l, h], rec, q, k, v, alpha, beta, self.quantizer)
         off = int(self.offsets[l * self.H + h])
         pool_slot[off:off + new_rec.size] = new_rec
         return o, tie, S, w
@@ -218,6 +227,20 @@ def build_plan(mode: int, D: int, n_layers: int, n_heads: int, stats: dict, bits
                 wbar=np.asarray(stats["wbar"], np.float32).reshape(-1),
                 rho=np.asarray(stats["rho"], np.float32).reshape(-1),
                 lgate=lgate, lifetime=np.asarray(lifetime, np.float64))
+
+
+def uniform_plan(mode: int, D: int, n_layers: int, n_heads: int, bits: int, quantizer: int,
+                 horizon: int, wbar=None) -> dict:
+    """A baseline plan: every unit at `bits`, no pivots (实验: uniform INT-b).
+    wbar defaults to ones (rho = 1); lgate is 0, so L_u = horizon."""
+    n_units = n_layers * n_heads * (D if mode == 1 else 1)
+    nrow = n_layers * n_heads * D
+    wbar = np.ones(nrow, np.float32) if wbar is None else np.asarray(wbar, np.float32).reshape(-1)
+    rho = np.array([1.0 / math.sqrt(math.sqrt(float(x))) for x in wbar], dtype=np.float32)
+    return dict(mode=mode, n_layers=n_layers, n_heads=n_heads, d=D, n_pivots=0, bitset=[int(bits)],
+                nominal_bits=float(bits), horizon=horizon, widths=np.full(n_units, int(bits), np.uint8),
+                wbar=wbar, rho=rho, lgate=np.zeros(n_units), lifetime=np.full(n_units, float(horizon)),
+                quantizer=int(quantizer))
 
 
 def lifetime_l_from_halflife(h: float) -> float:

@@ -13,7 +13,9 @@ Plan file, little-endian:
   32  4  u32 n_units (mode 0: n_layers*n_heads, mode 1: that times d_k)
   36  4  u32 n_pivots        40  4  u32 bitset (bit b set: width b allowed)
   44  4  f32 nominal bits    48  8  u64 horizon H
-  56  8  zero
+  56  4  u32 quantizer: 0 = STEPQuant dual-axis fit, 1 = per-row absmax
+         (mode 0 only; every record keeps the codes | r | c layout, c = 1)
+  60  4  u32 zero
   64     u8  width[n_units]  (2, 4, 6, 8, or 16 for an FP16 pivot)
          zero padding to a multiple of 4 bytes
          f32 wbar[n_layers*n_heads*d_k]   row impact omega_i / mean omega
@@ -39,7 +41,7 @@ import numpy as np
 
 MAGIC = b"STEPQPL1"
 VERSION = 1
-HEADER = struct.Struct("<8sIIIIIIIIIfQQ")
+HEADER = struct.Struct("<8sIIIIIIIIIfQII")
 PIVOT_BITS = 16
 
 
@@ -57,7 +59,8 @@ def write_plan(path: str, plan: dict) -> bytes:
     for b in plan["bitset"]:
         bitset |= 1 << int(b)
     head = HEADER.pack(MAGIC, VERSION, mode, L, H, D, D, n_units, int(plan["n_pivots"]),
-                       bitset, float(plan["nominal_bits"]), int(plan["horizon"]), 0)
+                       bitset, float(plan["nominal_bits"]), int(plan["horizon"]),
+                       int(plan.get("quantizer", 0)), 0)
     body = bytearray(head)
     body += widths.tobytes()
     body += b"\0" * (_align(len(body), 4) - len(body))
@@ -75,7 +78,7 @@ def write_plan(path: str, plan: dict) -> bytes:
 
 def read_plan(data: bytes) -> dict:
     (magic, ver, mode, L, H, dk, dv, n_units, n_piv, bitset, nominal, horizon,
-     _z) = HEADER.unpack_from(data, 0)
+     quantizer, _z) = HEADER.unpack_from(data, 0)
     assert magic == MAGIC and ver == VERSION
     off = HEADER.size
     widths = np.frombuffer(data, dtype=np.uint8, count=n_units, offset=off).copy()
@@ -89,7 +92,8 @@ def read_plan(data: bytes) -> dict:
     assert crc == zlib.crc32(data[:off]) & 0xFFFFFFFF
     return dict(mode=mode, n_layers=L, n_heads=H, d=dk, n_pivots=n_piv,
                 bitset=[b for b in range(32) if bitset >> b & 1], nominal_bits=nominal,
-                horizon=horizon, widths=widths, wbar=wbar, rho=rho, lgate=lgate, lifetime=life)
+                horizon=horizon, widths=widths, wbar=wbar, rho=rho, lgate=lgate, lifetime=life,
+                quantizer=quantizer)
 
 
 # --------------------------------------------------------------------------

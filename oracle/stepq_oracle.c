@@ -331,6 +331,53 @@ void sq_quantize(int D, const int *widths, const float *rho, const float *wbar,
     free(absrow); free(y); free(bw); free(tn); free(td); free(z0); free(coltie);
 }
 
+/* ------------------------------------------------------------------------ */
+/* Per-row absmax quantizer: the ordinary baseline the pages set against     */
+/* STEPQuant (实验: uniform INT4 / INT6 / INT8 and the remark that plain      */
+/* per-row absmax stays unstable even at 8 bits).  Reading, per row i of     */
+/* width b (qmax = 2^(b-1) - 1):                                             */
+/*   m_i = max_j |S_ij|;  r_i = fl(m_i / qmax), or 1 when m_i = 0;           */
+/*   z_ij = clamp(nearest integer, ties to even, to the exact product        */
+/*          S_ij * fl(1/r_i), -qmax, +qmax);  c_j = 1 for every column.      */
+/* The record keeps the r | c layout, so X_hat = fl(fl(r_i c_j) z_ij) =      */
+/* fl(r_i z_ij) decodes it unchanged.  16-bit rows as in sq_quantize.        */
+/* tie_out (optional): bit0 = code within 1e-6 relative of a .5 boundary.    */
+/* ------------------------------------------------------------------------ */
+
+void sq_quantize_absmax(int D, const int *widths, const float *S, int32_t *z, uint16_t *h,
+                        float *r, float *c, uint8_t *tie_out)
+{
+    for (int j = 0; j < D; j++) c[j] = 1.0f;
+    for (int i = 0; i < D; i++) {
+        if (widths[i] == SQ_PIVOT_BITS) {
+            r[i] = 0.0f;
+            for (int j = 0; j < D; j++) {
+                h[i * D + j] = sq_f32_to_f16(S[i * D + j]);
+                z[i * D + j] = 0;
+                if (tie_out) tie_out[i * D + j] = 0;
+            }
+            continue;
+        }
+        int q = qmax_of(widths[i]);
+        float m = 0.0f;
+        for (int j = 0; j < D; j++) {
+            float a = fabsf(S[i * D + j]);
+            if (a > m) m = a;
+        }
+        r[i] = (m > 0.0f) ? m / (float)q : 1.0f;
+        float inv_r = 1.0f / r[i];
+        for (int j = 0; j < D; j++) {
+            double x = (double)S[i * D + j] * (double)inv_r; /* exact: 24 x 24 bits */
+            double zr = rint(x);
+            if (zr > q) zr = q;
+            if (zr < -q) zr = -q;
+            z[i * D + j] = (int32_t)zr;
+            h[i * D + j] = 0;
+            if (tie_out) tie_out[i * D + j] = (uint8_t)(near_half(x) ? 1 : 0);
+        }
+    }
+}
+
 /* Reconstruction X_hat_ij = fl(fl(r_i * c_j) * z_ij); 16-bit rows decode the
  * stored binary16 value. */
 void sq_reconstruct(int D, const int *widths, const int32_t *z, const uint16_t *h,

@@ -400,6 +400,88 @@ def _convex_costs(N, widths):
     return out
 
 
+# --------------------------------------------------------------------------
+# per-row absmax baseline quantizer (实验: uniform INT-b, ordinary per-row
+# absmax): nearest code by enumeration, the row maximum at +-qmax, the
+# half-step bound, c = 1, degenerate rows, scale invariance
+# --------------------------------------------------------------------------
+
+def _outlier_state(D, seed):
+    g = np.random.default_rng(seed)
+    S = g.standard_normal((D, D)).astype(np.float32)
+    S[g.integers(D)] *= 10.0
+    S[:, g.integers(D)] *= 19.0
+    return S
+
+
+@pytest.mark.parametrize("b", [2, 4, 6, 8])
+def test_absmax_codes_are_nearest_by_enumeration(b):
+    D, q = 16, (1 << (b - 1)) - 1
+    S = _outlier_state(D, 100 + b)
+    z, h, r, c, tie = core.quantize_absmax(D, np.full(D, b), S)
+    assert np.all(c == 1.0)
+    cand = np.arange(-q, q + 1, dtype=np.float64)
+    for i in range(D):
+        m = float(np.max(np.abs(S[i])))
+        assert abs(float(r[i]) * q - m) <= 2.0 ** -23 * m  # r_i is m_i / qmax rounded once
+        inv = np.float32(1.0) / r[i]
+        for j in range(D):
+            x = float(S[i, j]) * float(inv)
+            d = np.abs(cand - x)
+            best = cand[d == d.min()]
+            pick = best[0] if best.size == 1 else best[np.argmin(np.abs(best) % 2)]  # ties to even
+            assert z[i, j] == int(pick), (i, j, x)
+
+
+@pytest.mark.parametrize("b", [2, 4, 6, 8])
+def test_absmax_row_max_at_qmax_and_half_step(b):
+    D, q = 128, (1 << (b - 1)) - 1
+    S = _outlier_state(D, 200 + b)
+    z, h, r, c, tie = core.quantize_absmax(D, np.full(D, b), S)
+    jmax = np.argmax(np.abs(S), axis=1)
+    assert np.all(np.abs(z[np.arange(D), jmax]) == q)
+    assert np.all(np.sign(z[np.arange(D), jmax]) == np.sign(S[np.arange(D), jmax]))
+    err = np.abs(S.astype(np.float64) - r[:, None].astype(np.float64) * z)
+    assert np.all(err <= 0.5 * r[:, None] * (1 + 1e-5))
+
+
+def test_absmax_degenerate_and_scale_invariance():
+    D, b = 16, 6
+    S = _outlier_state(D, 300)
+    S[3] = 0.0
+    z, h, r, c, tie = core.quantize_absmax(D, np.full(D, b), S)
+    assert r[3] == 1.0 and np.all(z[3] == 0)
+    z2, h2, r2, c2, tie2 = core.quantize_absmax(D, np.full(D, b), S * np.float32(2.0 ** 7))
+    assert np.array_equal(z2, z)
+    nz = np.arange(D) != 3
+    assert np.array_equal(r2[nz], r[nz] * np.float32(2.0 ** 7))
+
+
+def test_absmax_pivot_rows_fp16_and_plan_field(tmp_path):
+    D = 16
+    S = _outlier_state(D, 400)
+    widths = np.full(D, 6)
+    widths[[2, 9]] = model.PIVOT_BITS
+    z, h, r, c, tie = core.quantize_absmax(D, widths, S)
+    for i in (2, 9):
+        assert r[i] == 0.0 and np.all(z[i] == 0)
+        assert np.array_equal(h[i], S[i].astype(np.float16).view(np.uint16))
+    plan = model.uniform_plan(0, D, 2, 3, 4, model.QUANT_ABSMAX, 65536)
+    back = plan_io.read_plan(plan_io.write_plan(str(tmp_path / "p.bin"), plan))
+    assert back["quantizer"] == model.QUANT_ABSMAX and np.all(back["widths"] == 4)
+    # a decode step through the plan view keeps c = 1 in the record
+    pv = model.PlanView(back)
+    slot = np.zeros(pv.slot_bytes, np.uint8)
+    pv.quantize_into(slot, 1, 2, S)
+    g = np.random.default_rng(5)
+    k = g.standard_normal(D).astype(np.float32)
+    k /= np.linalg.norm(k)
+    pv.step(slot, 1, 2, g.standard_normal(D).astype(np.float32), k, g.standard_normal(D).astype(np.float32),
+            np.full(D, 0.9, np.float32), np.float32(0.5))
+    zz, hh, rr, cc = pv.unpack(slot, 1, 2)
+    assert np.all(cc == 1.0) and np.all(np.abs(zz) <= 7)
+
+
 @pytest.mark.parametrize("widths", [(4, 6, 8), (2, 4, 6, 8)])
 @pytest.mark.parametrize("N", [3, 5, 7])
 def test_dp_equals_brute_force(widths, N):
