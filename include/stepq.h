@@ -88,6 +88,16 @@ extern "C" {
 
 #define STEPQ_PIVOT_BITS 16
 
+/* Requantizer of a plan (plan header word at byte 56).
+ * STEPQ_QUANT_DUAL_AXIS: the STEPQuant row/column fit above (方法-3).
+ * STEPQ_QUANT_ABSMAX: the ordinary per-row absmax baseline the pages compare
+ *   against (实验: uniform INT4/INT6/INT8), per-head units only:
+ *   r_i = fl(max_j |S_ij| / qmax) (1 for a zero row), z_ij = clamp(nearest
+ *   integer, ties to even, to the exact S_ij * fl(1/r_i), +-qmax), c_j = 1;
+ *   the record keeps the codes | r | c layout and decodes unchanged. */
+#define STEPQ_QUANT_DUAL_AXIS 0
+#define STEPQ_QUANT_ABSMAX 1
+
 typedef struct stepq_plan stepq_plan; /* opaque, host-side plan */
 typedef struct stepq_ctx stepq_ctx;   /* opaque, per device: tables, streams, events */
 
@@ -105,6 +115,7 @@ typedef struct stepq_plan_info {
     double bits_per_value;       /* codes + FP16 pivots + fp32 scales */
     double bits_per_value_s16;   /* the same with 16-bit scale accounting */
     int units_by_width[17];      /* histogram of unit widths (index = bits) */
+    int quantizer;               /* STEPQ_QUANT_DUAL_AXIS or STEPQ_QUANT_ABSMAX */
 } stepq_plan_info;
 
 /* ---- plan (方法-1 offline precision map) -------------------------------- */
@@ -140,6 +151,14 @@ int stepq_plan_record(const stepq_plan *plan, int layer, int head, uint64_t *off
 int stepq_plan_build(int mode, int n_layers, int n_heads, int d, const int *bits, int n_bits,
                      float nominal_bits, int n_pivots, uint64_t horizon, const double *lgate,
                      const double *dist, const float *wbar, const char *path, stepq_plan **out);
+
+/* A baseline plan (实验: uniform INT-b): every unit at width `bits` (2, 4, 6
+ * or 8), no pivots, the given quantizer (STEPQ_QUANT_ABSMAX needs mode 0).
+ * wbar[n_layers*n_heads*d] (host, NULL: all ones) feeds rho for the
+ * dual-axis fit; lgate is 0 for every unit.  Writes the plan file to `path`
+ * (NULL: none) and returns the parsed plan.  Errors: STEPQ_EINVAL. */
+int stepq_plan_build_uniform(int mode, int n_layers, int n_heads, int d, int bits, int quantizer,
+                             uint64_t horizon, const float *wbar, const char *path, stepq_plan **out);
 
 /* ---- context ------------------------------------------------------------ */
 

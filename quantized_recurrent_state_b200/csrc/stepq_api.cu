@@ -85,6 +85,7 @@ T rd(const uint8_t *p) {
 
 struct stepq_plan {
     int mode = 0, L = 0, H = 0, D = 0, n_units = 0, n_pivots = 0;
+    int quantizer = 0;                // 0 dual-axis fit, 1 per-row absmax (mode 0)
     uint32_t bitset = 0;
     float nominal = 0.f;
     uint64_t horizon = 0;
@@ -105,7 +106,8 @@ struct stepq_plan {
  * Plan file, little-endian:
  *   0  8 magic "STEPQPL1" | 8 u32 version=1 | 12 u32 mode | 16 u32 n_layers
  *   20 u32 n_heads | 24 u32 d_k | 28 u32 d_v | 32 u32 n_units | 36 u32 n_pivots
- *   40 u32 bitset | 44 f32 nominal bits | 48 u64 horizon | 56 u64 zero
+ *   40 u32 bitset | 44 f32 nominal bits | 48 u64 horizon | 56 u32 quantizer
+ *   (0 dual-axis fit, 1 per-row absmax; mode 0 only) | 60 u32 zero
  *   64 u8 width[n_units], zero pad to 4 | f32 wbar[L*H*d] | f32 rho[L*H*d]
  *   f64 lgate[n_units] | f64 lifetime[n_units] | u32 CRC-32 of all before it
  */
@@ -124,7 +126,11 @@ static int plan_parse(const uint8_t *d, size_t n, stepq_plan *p) {
     p->bitset = rd<uint32_t>(d + 40);
     p->nominal = rd<float>(d + 44);
     p->horizon = rd<uint64_t>(d + 48);
+    p->quantizer = (int)rd<uint32_t>(d + 56);
     if (p->mode != 0 && p->mode != 1) return fail(STEPQ_EFORMAT, "plan: mode %d", p->mode);
+    if (p->quantizer != 0 && !(p->quantizer == 1 && p->mode == 0))
+        return fail(STEPQ_EFORMAT, "plan: quantizer %d with mode %d", p->quantizer, p->mode);
+    if (rd<uint32_t>(d + 60) != 0) return fail(STEPQ_EFORMAT, "plan: reserved header word is not zero");
     if (dk != dv) return fail(STEPQ_EFORMAT, "plan: d_k %u != d_v %u", dk, dv);
     if (dk != 16 && dk != 32 && dk != 64 && dk != 128) return fail(STEPQ_EFORMAT, "plan: d = %u unsupported", dk);
     p->D = (int)dk;
@@ -257,6 +263,7 @@ extern "C" int stepq_plan_get_info(const stepq_plan *p, stepq_plan_info *o) {
     o->slot_bytes = p->slot_bytes;
     o->bits_per_value = p->bpv;
     o->bits_per_value_s16 = p->bpv16;
+    o->quantizer = p->quantizer;
     for (int w : p->width) o->units_by_width[w <= 16 ? w : 0]++;
     return STEPQ_OK;
 }
@@ -415,6 +422,56 @@ bool lagrangian_allocate(const std::vector<double> &cost, int N, const std::vect
 void put_u32(std::vector<uint8_t> &v, uint32_t x) { v.insert(v.end(), (uint8_t *)&x, (uint8_t *)&x + 4); }
 void put_u64(std::vector<uint8_t> &v, uint64_t x) { v.insert(v.end(), (uint8_t *)&x, (uint8_t *)&x + 8); }
 
+// The plan file image (format above); rho_i = fl32(1/sqrt(sqrt(wbar_i))).
+std::vector<uint8_t> serialize_plan(int mode, int n_layers, int n_heads, int d, int n_pivots, uint32_t bitset,
+                                    float nominal_bits, uint64_t horizon, int quantizer,
+                                    const std::vector<uint8_t> &width, const float *wbar, const double *lgate,
+                                    const std::vector<double> &life) {
+    const size_t heads = (size_t)n_layers * n_heads, nrow = heads * d, units = width.size();
+    std::vector<uint8_t> f;
+    f.insert(f.end(), (const uint8_t *)"STEPQPL1", (const uint8_t *)"STEPQPL1" + 8);
+    put_u32(f, 1);
+    put_u32(f, (uint32_t)mode);
+    put_u32(f, (uint32_t)n_layers);
+    put_u32(f, (uint32_t)n_heads);
+    put_u32(f, (uint32_t)d);
+    put_u32(f, (uint32_t)d);
+    put_u32(f, (uint32_t)units);
+    put_u32(f, (uint32_t)n_pivots);
+    put_u32(f, bitset);
+    uint32_t nb;
+    std::memcpy(&nb, &nominal_bits, 4);
+    put_u32(f, nb);
+    put_u64(f, horizon);
+    put_u32(f, (uint32_t)quantizer);
+    put_u32(f, 0);
+    f.insert(f.end(), width.begin(), width.end());
+    while (f.size() % 4) f.push_back(0);
+    const size_t off_wb = f.size();
+    f.resize(off_wb + 8 * nrow);
+    std::memcpy(&f[off_wb], wbar, 4 * nrow);
+    for (size_t i = 0; i < nrow; ++i) {
+        const float r = (float)(1.0 / std::sqrt(std::sqrt((double)wbar[i])));
+        std::memcpy(&f[off_wb + 4 * nrow + 4 * i], &r, 4);
+    }
+    const size_t off_l = f.size();
+    f.resize(off_l + 16 * units);
+    std::memcpy(&f[off_l], lgate, 8 * units);
+    std::memcpy(&f[off_l + 8 * units], life.data(), 8 * units);
+    put_u32(f, crc32(f.data(), f.size()));
+    return f;
+}
+
+int write_plan_file(const char *path, const std::vector<uint8_t> &f, const char *who) {
+    if (!path) return STEPQ_OK;
+    FILE *fp = std::fopen(path, "wb");
+    if (!fp) return fail(STEPQ_EINVAL, "%s: cannot write %s", who, path);
+    const size_t wr = std::fwrite(f.data(), 1, f.size(), fp);
+    std::fclose(fp);
+    if (wr != f.size()) return fail(STEPQ_EINVAL, "%s: short write to %s", who, path);
+    return STEPQ_OK;
+}
+
 }  // namespace
 
 extern "C" int stepq_plan_build(int mode, int n_layers, int n_heads, int d, const int *bits, int n_bits,
@@ -459,45 +516,33 @@ extern "C" int stepq_plan_build(int mode, int n_layers, int n_heads, int d, cons
     const bool ok = mode == 0 ? dp_allocate(cost, N, w, cap, alloc) : lagrangian_allocate(cost, N, w, cap, alloc);
     if (!ok) return fail(STEPQ_EINVAL, "plan_build: budget %lld below the smallest width", cap);
     for (int k = 0; k < N; ++k) width[keep[k]] = (uint8_t)alloc[k];
-    // serialise
-    const size_t nrow = (size_t)heads * d;
-    std::vector<uint8_t> f;
-    f.insert(f.end(), (const uint8_t *)"STEPQPL1", (const uint8_t *)"STEPQPL1" + 8);
-    put_u32(f, 1);
-    put_u32(f, (uint32_t)mode);
-    put_u32(f, (uint32_t)n_layers);
-    put_u32(f, (uint32_t)n_heads);
-    put_u32(f, (uint32_t)d);
-    put_u32(f, (uint32_t)d);
-    put_u32(f, (uint32_t)units);
-    put_u32(f, (uint32_t)n_pivots);
-    put_u32(f, bitset);
-    uint32_t nb;
-    std::memcpy(&nb, &nominal_bits, 4);
-    put_u32(f, nb);
-    put_u64(f, horizon);
-    put_u64(f, 0);
-    f.insert(f.end(), width.begin(), width.end());
-    while (f.size() % 4) f.push_back(0);
-    const size_t off_wb = f.size();
-    f.resize(off_wb + 8 * nrow);
-    std::memcpy(&f[off_wb], wbar, 4 * nrow);
-    for (size_t i = 0; i < nrow; ++i) {
-        const float r = (float)(1.0 / std::sqrt(std::sqrt((double)wbar[i])));
-        std::memcpy(&f[off_wb + 4 * nrow + 4 * i], &r, 4);
+    const std::vector<uint8_t> f = serialize_plan(mode, n_layers, n_heads, d, n_pivots, bitset, nominal_bits, horizon,
+                                                  0, width, wbar, lgate, life);
+    if (int rc = write_plan_file(path, f, "plan_build")) return rc;
+    return stepq_plan_load_mem(f.data(), f.size(), out);
+}
+
+extern "C" int stepq_plan_build_uniform(int mode, int n_layers, int n_heads, int d, int bits, int quantizer,
+                                        uint64_t horizon, const float *wbar, const char *path, stepq_plan **out) {
+    if (!out) return fail(STEPQ_EINVAL, "plan_build_uniform: null argument");
+    if (mode != 0 && mode != 1) return fail(STEPQ_EINVAL, "plan_build_uniform: mode %d", mode);
+    if (n_layers <= 0 || n_heads <= 0 || (d != 16 && d != 32 && d != 64 && d != 128))
+        return fail(STEPQ_EINVAL, "plan_build_uniform: bad dims");
+    if (bits != 2 && bits != 4 && bits != 6 && bits != 8) return fail(STEPQ_EINVAL, "plan_build_uniform: width %d", bits);
+    if (quantizer != 0 && !(quantizer == 1 && mode == 0))
+        return fail(STEPQ_EINVAL, "plan_build_uniform: quantizer %d with mode %d", quantizer, mode);
+    const size_t heads = (size_t)n_layers * n_heads, nrow = heads * d, units = mode == 0 ? heads : nrow;
+    std::vector<float> ones;
+    if (!wbar) {
+        ones.assign(nrow, 1.0f);
+        wbar = ones.data();
     }
-    const size_t off_l = f.size();
-    f.resize(off_l + 16 * (size_t)units);
-    std::memcpy(&f[off_l], lgate, 8 * (size_t)units);
-    std::memcpy(&f[off_l + 8 * (size_t)units], life.data(), 8 * (size_t)units);
-    put_u32(f, crc32(f.data(), f.size()));
-    if (path) {
-        FILE *fp = std::fopen(path, "wb");
-        if (!fp) return fail(STEPQ_EINVAL, "plan_build: cannot write %s", path);
-        const size_t wr = std::fwrite(f.data(), 1, f.size(), fp);
-        std::fclose(fp);
-        if (wr != f.size()) return fail(STEPQ_EINVAL, "plan_build: short write to %s", path);
-    }
+    const std::vector<uint8_t> width(units, (uint8_t)bits);
+    const std::vector<double> lgate(units, 0.0);
+    const std::vector<double> life(units, lifetime_weight(0.0, horizon));
+    const std::vector<uint8_t> f = serialize_plan(mode, n_layers, n_heads, d, 0, 1u << bits, (float)bits, horizon,
+                                                  quantizer, width, wbar, lgate.data(), life);
+    if (int rc = write_plan_file(path, f, "plan_build_uniform")) return rc;
     return stepq_plan_load_mem(f.data(), f.size(), out);
 }
 
@@ -556,6 +601,7 @@ stepq::Args base_args(stepq_ctx *c, void *pool, const int32_t *slots, int n_req,
     a.l_in0 = 0;
     a.H = c->plan->H;
     a.mode = c->plan->mode;
+    a.quantizer = c->plan->quantizer;
     a.n_items = n_req * (le - lb) * c->plan->H;
     a.div_nreq = stepq::div_magic((uint32_t)n_req);
     a.div_h = stepq::div_magic((uint32_t)c->plan->H);

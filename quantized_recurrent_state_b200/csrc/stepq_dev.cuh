@@ -14,6 +14,8 @@
 namespace stepq {
 
 constexpr int kPivotBits = 16;
+constexpr int kQuantDualAxis = 0;  // plan quantizer: STEPQuant row/column fit
+constexpr int kQuantAbsmax = 1;    // plan quantizer: per-row absmax, c = 1
 constexpr int kErrBadSlot = 1;
 constexpr int kErrWait = 2;
 constexpr int kErrArgs = 4;
@@ -44,6 +46,7 @@ struct Args {
     int l_in0;  // index of layer lb inside that layout
     int H;
     int mode;
+    int quantizer;           // kQuantDualAxis or kQuantAbsmax (per-head units)
     int n_items;             // n_req * nL * H
     uint64_t div_nreq;       // floor(2^64 / n_req) + 1 (0 when n_req == 1): n / n_req = umul64hi(n, div_nreq)
     uint64_t div_h;          // the same for H

@@ -505,6 +505,67 @@ __device__ void fit_pack(float2 (&S)[D / 8][2], uint8_t *rec, Scratch<D> &sc, in
     store_stream<D, B>(rec, tid, W);
 }
 
+// Per-row absmax requantization (the baseline quantizer of the plan's
+// quantizer field): r_i = fl(max_j |S_ij| / qmax) (1 for a zero row), codes
+// = clamp(rne(S_ij * fl(1/r_i))), c = 1.  Rows live inside one warp, so the
+// whole fit needs no block barrier.  Writes codes, r and c to `rec`.
+template <int D, int B>
+__device__ void fit_pack_absmax(float2 (&S)[D / 8][2], uint8_t *rec, Scratch<D> &sc, int tid) {
+    using G = Geo<D>;
+    constexpr int RT = G::RT, LANES = G::LANES, RS = Scratch<D>::RS, HALF = LANES / 2;
+    constexpr int Q = (1 << (B - 1)) - 1;
+    constexpr float MG2 = kMagic + (float)(1 << (B - 1));
+    const int g = tid / LANES, l = tid % LANES;
+    const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
+    float *rec_r = reinterpret_cast<float *>(rec + codes_bytes);
+    float *rec_c = rec_r + D;
+    // 1. row maxima: this thread's 4 columns, then the row's lanes (transpose)
+    float *rs = &sc.rsum[g][0][0];
+#pragma unroll
+    for (int r = 0; r < RT; ++r)
+        rs[r * RS + l] = fmaxf(fmaxf(fabsf(S[r][0].x), fabsf(S[r][0].y)), fmaxf(fabsf(S[r][1].x), fabsf(S[r][1].y)));
+    __syncwarp();
+    {
+        const int rr = l >> 1, hh = l & 1;
+        const float *src = rs + rr * RS + hh * HALF;
+        float m = 0.0f;
+#pragma unroll
+        for (int k = 0; k < HALF; ++k) m = fmaxf(m, src[k]);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        const int i = g * RT + rr;
+        const float ri = (m > 0.0f) ? __fdiv_rn(m, (float)Q) : 1.0f;
+        const float inv = __frcp_rn(ri);
+        if (hh == 0) {
+            sc.rinv2[i] = make_float2(inv, inv);
+            rec_r[i] = ri;
+        }
+    }
+    __syncwarp();
+    if (tid < D) rec_c[tid] = 1.0f;
+    // 2. codes e = rne(S * fl(1/r)) + qmax, clamped, packed into the stream
+    uint32_t W[Stream<D, B>::NW];
+#pragma unroll
+    for (int i = 0; i < Stream<D, B>::NW; ++i) W[i] = 0u;
+    const float2 mg2 = make_float2(MG2, MG2);
+#pragma unroll
+    for (int r = 0; r < RT; r += 2) {
+        const float4 f = *reinterpret_cast<const float4 *>(&sc.rinv2[g * RT + r]);
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            const float2 inv2 = rr ? make_float2(f.z, f.w) : make_float2(f.x, f.y);
+#pragma unroll
+            for (int hp = 0; hp < 2; ++hp) {
+                const float2 t = fma2(S[r + rr][hp], inv2, mg2);
+                field_acc<B>(W, 4 * (r + rr) + 2 * hp, final_e<B>(t.x));
+                field_acc<B>(W, 4 * (r + rr) + 2 * hp + 1, final_e<B>(t.y));
+            }
+        }
+    }
+    add_pack_ones<D, B>(W);
+    store_stream<D, B>(rec, tid, W);
+    (void)Q;
+}
+
 // Pivot head (binary16 tile): S_t -> fp16 RNE, written in place.
 template <int D>
 __device__ __forceinline__ void store_pivot(float2 (&S)[D / 8][2], uint8_t *rec, int tid) {
@@ -706,7 +767,8 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
                 S[r + rr][1] = fma2(k2, w23, S[r + rr][1]);
             }
         }
-        fit_pack<D, B>(S, rec_g, sc, tid, tf + kTailRho * D, tf + kTailWbar * D);
+        if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, B>(S, rec_g, sc, tid);
+        else fit_pack<D, B>(S, rec_g, sc, tid, tf + kTailRho * D, tf + kTailWbar * D);
     }
 }
 
@@ -1250,10 +1312,22 @@ __global__ void __launch_bounds__(2 * D) k_requant_pack(Args a) {
     if (tid == 0) sc.nz = a.neg_zero;
     __syncthreads();
     switch (width) {
-        case 2: fit_pack<D, 2>(S, rec, sc, tid, sc.rho, sc.wbar); break;
-        case 4: fit_pack<D, 4>(S, rec, sc, tid, sc.rho, sc.wbar); break;
-        case 6: fit_pack<D, 6>(S, rec, sc, tid, sc.rho, sc.wbar); break;
-        case 8: fit_pack<D, 8>(S, rec, sc, tid, sc.rho, sc.wbar); break;
+        case 2:
+            if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 2>(S, rec, sc, tid);
+            else fit_pack<D, 2>(S, rec, sc, tid, sc.rho, sc.wbar);
+            break;
+        case 4:
+            if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 4>(S, rec, sc, tid);
+            else fit_pack<D, 4>(S, rec, sc, tid, sc.rho, sc.wbar);
+            break;
+        case 6:
+            if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 6>(S, rec, sc, tid);
+            else fit_pack<D, 6>(S, rec, sc, tid, sc.rho, sc.wbar);
+            break;
+        case 8:
+            if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 8>(S, rec, sc, tid);
+            else fit_pack<D, 8>(S, rec, sc, tid, sc.rho, sc.wbar);
+            break;
         default: if (tid == 0) flag_error(a.err, kErrArgs); break;
     }
 }

@@ -25,8 +25,10 @@ EXPORTED = [
     "stepq_decode_step_fused", "stepq_sync", "stepq_unpack", "stepq_fp32_decode_step",
     "stepq_calib_accumulate", "stepq_calib_distortion", "stepq_copy_probe",
     "stepq_launch_count", "stepq_last_error", "stepq_ctx_set_timing", "stepq_kernel_stats",
-    "stepq_decode_step_noalloc",
+    "stepq_decode_step_noalloc", "stepq_plan_build_uniform",
 ]
+QUANT_DUAL_AXIS = 0  # plan requantizer: STEPQuant row/column fit
+QUANT_ABSMAX = 1     # plan requantizer: per-row absmax baseline, c = 1
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -43,6 +45,7 @@ class PlanInfo(ctypes.Structure):
         ("bitset", ctypes.c_uint32), ("nominal_bits", ctypes.c_float), ("horizon", ctypes.c_uint64),
         ("slot_bytes", ctypes.c_uint64), ("bits_per_value", ctypes.c_double),
         ("bits_per_value_s16", ctypes.c_double), ("units_by_width", ctypes.c_int * 17),
+        ("quantizer", ctypes.c_int),
     ]
 
 
@@ -69,6 +72,8 @@ def lib():
         l.stepq_plan_record.argtypes = [P, I, I, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)]
         l.stepq_plan_build.argtypes = [I, I, I, I, P, I, ctypes.c_float, I, ctypes.c_uint64, P, P, P,
                                        ctypes.c_char_p, ctypes.POINTER(P)]
+        l.stepq_plan_build_uniform.argtypes = [I, I, I, I, I, I, ctypes.c_uint64, P, ctypes.c_char_p,
+                                               ctypes.POINTER(P)]
         l.stepq_ctx_create.argtypes = [P, P, P, I, I, ctypes.POINTER(P)]
         l.stepq_ctx_free.argtypes = [P]
         l.stepq_ctx_free.restype = None
@@ -140,6 +145,16 @@ class Plan:
                                       float(nominal_bits), n_pivots, int(horizon), lg.ctypes.data,
                                       di.ctypes.data, wb.ctypes.data,
                                       path.encode() if path else None, ctypes.byref(h)))
+        return cls(h)
+
+    @classmethod
+    def build_uniform(cls, mode, n_layers, n_heads, d, bits, quantizer=QUANT_DUAL_AXIS, horizon=65536,
+                      wbar=None, path=None) -> "Plan":
+        wb = None if wbar is None else np.ascontiguousarray(wbar, dtype=np.float32)
+        h = P()
+        _check(lib().stepq_plan_build_uniform(mode, n_layers, n_heads, d, int(bits), int(quantizer), int(horizon),
+                                              None if wb is None else wb.ctypes.data,
+                                              path.encode() if path else None, ctypes.byref(h)))
         return cls(h)
 
     def widths(self) -> np.ndarray:

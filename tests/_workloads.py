@@ -33,6 +33,16 @@ def oracle_plan(name: str, n_layers: int = None, n_pivots: int = None, d: int = 
     return plan, data, wl, stats
 
 
+@functools.lru_cache(maxsize=None)
+def uniform_plan(name: str, bits: int, quantizer: int, n_layers: int = None):
+    """(plan dict, plan bytes, Workload) of a baseline plan (every unit at
+    `bits`, no pivots) over a workload's shape."""
+    wl = synth.workloads()[name]
+    wl = synth.Workload(**{**wl.__dict__, "n_layers": n_layers or wl.n_layers, "n_pivots": 0})
+    plan = model.uniform_plan(wl.mode, wl.d, wl.n_layers, wl.n_heads, bits, quantizer, wl.horizon)
+    return plan, plan_io.write_plan(None, plan), wl, None
+
+
 def compare_records(pv: model.PlanView, gpu_slot: np.ndarray, ora_slot: np.ndarray, ties: dict):
     """Compare every record of one slot.  ties[(l, h)] = the oracle's tie map
     for that head (None: expect exact).  Returns (n_codes, n_excused, n_bad,

@@ -12,7 +12,7 @@ import pytest
 
 from oracle import core, model
 from quantized_recurrent_state_b200 import synth
-from tests._workloads import compare_records, oracle_plan
+from tests._workloads import compare_records, oracle_plan, uniform_plan
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -40,8 +40,11 @@ def _inputs_to_dev(inp):
 class Run:
     """A GPU pool for a workload plus an oracle view of the same plan."""
 
-    def __init__(self, stepq, name, n_req, n_layers=None, n_pivots=None, extra_slots=3, chunk=2):
-        self.plan, data, self.wl, _ = oracle_plan(name, n_layers, n_pivots)
+    def __init__(self, stepq, name, n_req, n_layers=None, n_pivots=None, extra_slots=3, chunk=2, uniform=None):
+        if uniform is None:
+            self.plan, data, self.wl, _ = oracle_plan(name, n_layers, n_pivots)
+        else:  # (bits, quantizer): a baseline plan over the workload's shape
+            self.plan, data, self.wl, _ = uniform_plan(name, uniform[0], uniform[1], n_layers)
         self.pv = model.PlanView(self.plan)
         self.P = stepq.Plan.from_bytes(data)
         self.n_req = n_req
@@ -82,8 +85,9 @@ class Run:
         return inp, o.cpu().numpy()
 
 
-def _lockstep(stepq, name, n_req, steps, check, n_layers=None, n_pivots=None, fused=False, heads=None):
-    run = Run(stepq, name, n_req, n_layers, n_pivots)
+def _lockstep(stepq, name, n_req, steps, check, n_layers=None, n_pivots=None, fused=False, heads=None,
+              uniform=None):
+    run = Run(stepq, name, n_req, n_layers, n_pivots, uniform=uniform)
     S0 = run.pack_initial()
     pv = run.pv
     tot_codes = tot_exc = tot_bad = 0
@@ -158,6 +162,20 @@ def test_qwen_layer_lockstep_256_steps(stepq):
 def test_pool_slice_lockstep(stepq, name):
     # a 2-layer slice of the 2,304-head pool at batch 70 (2 pivot heads), 8 steps
     _lockstep(stepq, name, 70, 8, check=[0, 69], n_layers=2, n_pivots=2)
+
+
+@pytest.mark.parametrize("bits", [4, 6, 8])
+@pytest.mark.parametrize("fused", [False, True])
+def test_absmax_baseline_lockstep(stepq, bits, fused):
+    # uniform INT-b plans with the per-row absmax requantizer over a 2-layer
+    # slice of the pool, batch 70, 6 steps; both step variants
+    _lockstep(stepq, "qwen_pool6", 70, 6, check=[0, 69], n_layers=2, fused=fused,
+              uniform=(bits, model.QUANT_ABSMAX))
+
+
+def test_uniform_dual_axis_lockstep(stepq):
+    # uniform INT8 with the STEPQuant fit (no pivots), fused
+    _lockstep(stepq, "qwen_pool6", 70, 6, check=[0, 69], n_layers=2, fused=True, uniform=(8, model.QUANT_DUAL_AXIS))
 
 
 def test_fused_bit_identical_to_two_stream(stepq):

@@ -148,3 +148,27 @@ def test_calls_without_device_fail_cleanly():
     h = ctypes.c_void_p()
     rc = stepq.lib().stepq_ctx_create(p._h, ctypes.c_void_p(1), ctypes.c_void_p(2), 4, 1, ctypes.byref(h))
     assert rc == stepq.ECUDA
+
+
+@pytest.mark.parametrize("mode,quant", [(0, stepq.QUANT_ABSMAX), (0, stepq.QUANT_DUAL_AXIS), (1, stepq.QUANT_DUAL_AXIS)])
+def test_uniform_plan_file_matches_oracle(tmp_path, mode, quant):
+    L, H, D = 2, 3, 16
+    wbar = np.linspace(0.5, 2.0, L * H * D).astype(np.float32)
+    path = str(tmp_path / "u.plan")
+    p = stepq.Plan.build_uniform(mode, L, H, D, 6, quant, 4096, wbar, path=path)
+    ora = model.uniform_plan(mode, D, L, H, 6, quant, 4096, wbar)
+    assert open(path, "rb").read() == plan_io.write_plan(None, ora)
+    assert p.info.quantizer == quant and p.info.n_pivots == 0
+    assert p.info.units_by_width[6] == p.info.n_units
+
+
+def test_quantizer_field_validation():
+    good = bytearray(plan_io.write_plan(None, model.uniform_plan(0, 16, 2, 2, 4, model.QUANT_ABSMAX, 4096)))
+    assert stepq.Plan.from_bytes(bytes(good)).info.quantizer == stepq.QUANT_ABSMAX
+    bad = bytearray(good); bad[56] = 2; _expect_format_error(_recrc(bad))                        # unknown quantizer
+    bad = bytearray(good); bad[60] = 1; _expect_format_error(_recrc(bad))                        # reserved word
+    kda = bytearray(plan_io.write_plan(None, model.uniform_plan(1, 16, 2, 2, 4, 0, 4096)))
+    kda[56] = 1; _expect_format_error(_recrc(kda))                                               # absmax needs mode 0
+    with pytest.raises(stepq.StepqError) as ei:
+        stepq.Plan.build_uniform(1, 2, 2, 16, 4, stepq.QUANT_ABSMAX)
+    assert ei.value.code == stepq.EINVAL
