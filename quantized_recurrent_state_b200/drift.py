@@ -7,9 +7,10 @@ written back every step and propagates as E_t = A_t E_{t-1} + eps_t, so a
 long-lived state can carry it for many steps.  This study runs, on the GPU,
 the packed path (fused kernel) and the FP32-state kernel side by side from
 the same S_0 on the drift workload (4 requests x 8 GDN heads, d = 128,
-half-lives 1,000-20,000 steps) for three plans: nominal 4-bit over
-{2,4,6,8}, nominal 6-bit over {4,6,8} and uniform INT8 (no pivots, 8 bits
-everywhere).  It reports the relative readout error every step and the
+half-lives 1,000-20,000 steps) for the plans: nominal 4-bit over {2,4,6,8} and nominal 6-bit over {4,6,8}
+(calibrated, with pivots), uniform INT8 with the STEPQuant fit, and the
+pages' baselines, uniform INT8 / INT6 / INT4 with the ordinary per-row
+absmax quantizer (实验).  It reports the relative readout error every step and the
 relative state error every `every` steps, and at a few steps checks the
 recorded error recursion: with S~_t the fp32 update of the reconstructed
 state, eps_t = S^_t - S~_t and A_t E_{t-1} the update of E_{t-1} with v = 0,
@@ -27,18 +28,20 @@ import math
 import numpy as np
 
 
+KINDS = ("nominal4", "nominal6", "int8", "absmax8", "absmax6", "absmax4")
+
+
 def plan_for(stepq, synth, wl, kind, device):
-    """GPU calibration + the library planner (uniform INT8: a fixed plan)."""
+    """GPU calibration + the library planner; the uniform baselines are
+    fixed plans from the library's uniform-plan builder."""
     import torch
     L, H, D = wl.n_layers, wl.n_heads, wl.d
     if kind == "int8":
-        units = L * H
-        return stepq.Plan.build(0, L, H, D, [8], 8.0, 0, wl.horizon, np.zeros(units), np.ones((units, 1)),
-                                np.ones(L * H * D, np.float32))
+        return stepq.Plan.build_uniform(0, L, H, D, 8, stepq.QUANT_DUAL_AXIS, wl.horizon)
+    if kind.startswith("absmax"):
+        return stepq.Plan.build_uniform(0, L, H, D, int(kind[6:]), stepq.QUANT_ABSMAX, wl.horizon)
     bits, nominal = ((2, 4, 6, 8), 4.0) if kind == "nominal4" else ((4, 6, 8), 6.0)
-    units = L * H
-    host = stepq.Plan.build(0, L, H, D, [8], 8.0, 0, wl.horizon, np.zeros(units), np.ones((units, 1)),
-                            np.ones(L * H * D, np.float32))
+    host = stepq.Plan.build_uniform(0, L, H, D, 8, stepq.QUANT_DUAL_AXIS, wl.horizon)
     n = wl.calib_req
     ctx = stepq.Context(host, n)
     alpha = synth.gates(wl, wl.calib_seed)
@@ -68,7 +71,7 @@ def plan_for(stepq, synth, wl, kind, device):
                             lmean.mean(axis=2).reshape(-1), d.sum(axis=2).reshape(-1, len(bits)), wbar.reshape(-1))
 
 
-def run(steps: int = 8192, every: int = 256, checks: int = 4, device: str = "cuda"):
+def run(steps: int = 8192, every: int = 256, checks: int = 4, device: str = "cuda", kinds=KINDS):
     import torch
 
     from quantized_recurrent_state_b200 import build as qbuild
@@ -81,7 +84,7 @@ def run(steps: int = 8192, every: int = 256, checks: int = 4, device: str = "cud
     out = {"workload": f"{n} requests x {H} GDN heads, d={D}, half-lives {wl.halflife[0]:g}-{wl.halflife[1]:g}",
            "steps": steps, "plans": {}}
     check_at = set(int(x) for x in np.linspace(every, steps, checks))
-    for kind in ("nominal4", "nominal6", "int8"):
+    for kind in kinds:
         plan = plan_for(stepq, synth, wl, kind, device)
         ctx = stepq.Context(plan, n)
         slots = torch.arange(n, dtype=torch.int32, device=device)

@@ -4,7 +4,8 @@ On the drift workload every half-life is 1,000-20,000 steps, so the
 quantization error written back each step barely decays (背景与动机).  The
 test checks that the recorded error follows E_t = A_t E_{t-1} + eps_t to
 fp32 rounding, that the errors are finite, and that they order with the
-bit budget (uniform INT8 < nominal 6-bit < nominal 4-bit).
+bit budget (uniform INT8 < nominal 6-bit < nominal 4-bit; absmax INT8 <
+absmax INT6 < absmax INT4).
 """
 import math
 
@@ -26,3 +27,5 @@ def test_drift_short():
             assert res < 1e-4, (kind, res)
     p = out["plans"]
     assert p["int8"]["readout_rel_err_mean"] < p["nominal6"]["readout_rel_err_mean"] < p["nominal4"]["readout_rel_err_mean"]
+    assert (p["absmax8"]["readout_rel_err_mean"] < p["absmax6"]["readout_rel_err_mean"]
+            < p["absmax4"]["readout_rel_err_mean"])
