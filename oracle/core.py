@@ -72,6 +72,12 @@ def _declare(l):
     l.sq_pairwise_sum.restype = F
     l.sq_quantize.argtypes = [I, P, P, P, P, P, P, P, P, P, P]
     l.sq_quantize_absmax.argtypes = [I, P, P, P, P, P, P, P]
+    l.sq_quantize_s.argtypes = [I, P, P, P, P, P, P, P, P, P, P, I]
+    l.sq_quantize_absmax_s.argtypes = [I, P, P, P, P, P, P, P, I]
+    l.sq_f32_to_bf16.argtypes = [F]
+    l.sq_f32_to_bf16.restype = ctypes.c_uint16
+    l.sq_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    l.sq_bf16_to_f32.restype = F
     l.sq_reconstruct.argtypes = [I, P, P, P, P, P, P]
     l.sq_step_from_codes.argtypes = [I, P, P, P, P, P, P, P, P, P, F, P, P, P, P]
     l.sq_step_fp32.argtypes = [I, P, P, P, P, P, F, P]
@@ -161,8 +167,16 @@ def pairwise_sum(x: np.ndarray) -> np.float32:
     return np.float32(lib().sq_pairwise_sum(_p(x), x.size))
 
 
-def quantize(D: int, widths, rho, wbar, S, return_z0: bool = False):
-    """Return (z, h, r, c, tie[, z0]) for one head (see sq_quantize)."""
+def f32_to_bf16(x: float) -> int:
+    return int(lib().sq_f32_to_bf16(float(x)))
+
+
+def bf16_to_f32(bits: int) -> float:
+    return float(lib().sq_bf16_to_f32(int(bits)))
+
+
+def quantize(D: int, widths, rho, wbar, S, return_z0: bool = False, scale_bits: int = 32):
+    """Return (z, h, r, c, tie[, z0]) for one head (see sq_quantize_s)."""
     w = _i32(widths)
     rho = _f32(rho)
     wbar = _f32(wbar)
@@ -173,13 +187,14 @@ def quantize(D: int, widths, rho, wbar, S, return_z0: bool = False):
     c = np.zeros(D, dtype=np.float32)
     tie = np.zeros((D, D), dtype=np.uint8)
     z0 = np.zeros((D, D), dtype=np.int32)
-    lib().sq_quantize(D, _p(w), _p(rho), _p(wbar), _p(S), _p(z), _p(h), _p(r), _p(c), _p(tie), _p(z0))
+    lib().sq_quantize_s(D, _p(w), _p(rho), _p(wbar), _p(S), _p(z), _p(h), _p(r), _p(c), _p(tie), _p(z0),
+                        int(scale_bits))
     if return_z0:
         return z, h, r, c, tie, z0
     return z, h, r, c, tie
 
 
-def quantize_absmax(D: int, widths, S):
+def quantize_absmax(D: int, widths, S, scale_bits: int = 32):
     """Return (z, h, r, c, tie) for one head under the per-row absmax
     quantizer (see sq_quantize_absmax)."""
     w = _i32(widths)
@@ -189,7 +204,7 @@ def quantize_absmax(D: int, widths, S):
     r = np.zeros(D, dtype=np.float32)
     c = np.zeros(D, dtype=np.float32)
     tie = np.zeros((D, D), dtype=np.uint8)
-    lib().sq_quantize_absmax(D, _p(w), _p(S), _p(z), _p(h), _p(r), _p(c), _p(tie))
+    lib().sq_quantize_absmax_s(D, _p(w), _p(S), _p(z), _p(h), _p(r), _p(c), _p(tie), int(scale_bits))
     return z, h, r, c, tie
 
 

@@ -22,9 +22,22 @@ PIVOT_BITS = 16
 # one head
 # --------------------------------------------------------------------------
 
-def pack_head(mode: int, D: int, rw, z, h, r, c) -> np.ndarray:
+def _scales_to_bytes(x, scale_bits):
+    x = np.asarray(x, dtype=np.float32)
+    if scale_bits == 16:
+        return np.array([core.f32_to_bf16(float(v)) for v in x], dtype="<u2").view(np.uint8)
+    return x.astype("<f4").view(np.uint8)
+
+
+def _scales_from_bytes(b, D, scale_bits):
+    if scale_bits == 16:
+        return np.array([core.bf16_to_f32(int(v)) for v in b[:2 * D].view("<u2")], dtype=np.float32)
+    return b[:4 * D].view("<f4").astype(np.float32)
+
+
+def pack_head(mode: int, D: int, rw, z, h, r, c, scale_bits: int = 32) -> np.ndarray:
     rw = np.asarray(rw, dtype=np.int32)
-    rec = np.zeros(plan_io.record_bytes(mode, D, rw), dtype=np.uint8)
+    rec = np.zeros(plan_io.record_bytes(mode, D, rw, scale_bits), dtype=np.uint8)
     if mode == 0 and rw[0] == PIVOT_BITS:
         blk = core.pack_rows(D, rw, np.zeros((D, D), np.int32), h)
         rec[:blk.size] = blk
@@ -34,12 +47,13 @@ def pack_head(mode: int, D: int, rw, z, h, r, c) -> np.ndarray:
     else:
         blk = core.pack_rows(D, rw, z, h)
     rec[:blk.size] = blk
-    rec[blk.size:blk.size + 4 * D] = np.asarray(r, dtype="<f4").view(np.uint8)
-    rec[blk.size + 4 * D:blk.size + 8 * D] = np.asarray(c, dtype="<f4").view(np.uint8)
+    e = scale_bits // 8
+    rec[blk.size:blk.size + e * D] = _scales_to_bytes(r, scale_bits)
+    rec[blk.size + e * D:blk.size + 2 * e * D] = _scales_to_bytes(c, scale_bits)
     return rec
 
 
-def unpack_head(mode: int, D: int, rw, rec: np.ndarray):
+def unpack_head(mode: int, D: int, rw, rec: np.ndarray, scale_bits: int = 32):
     rw = np.asarray(rw, dtype=np.int32)
     rec = np.ascontiguousarray(rec, dtype=np.uint8)
     nb = plan_io.codes_block_bytes(mode, D, rw)
@@ -51,8 +65,9 @@ def unpack_head(mode: int, D: int, rw, rec: np.ndarray):
         h = np.zeros((D, D), np.uint16)
     else:
         z, h = core.unpack_rows(D, rw, rec[:nb])
-    r = rec[nb:nb + 4 * D].view("<f4").astype(np.float32)
-    c = rec[nb + 4 * D:nb + 8 * D].view("<f4").astype(np.float32)
+    e = scale_bits // 8
+    r = _scales_from_bytes(rec[nb:nb + e * D], D, scale_bits)
+    c = _scales_from_bytes(rec[nb + e * D:nb + 2 * e * D], D, scale_bits)
     return z, h, r, c
 
 
@@ -60,24 +75,25 @@ QUANT_DUAL_AXIS = 0  # STEPQuant row/column fit (方法-3)
 QUANT_ABSMAX = 1     # ordinary per-row absmax baseline (实验)
 
 
-def quantize_head(mode, D, rw, rho, wbar, S, quantizer: int = QUANT_DUAL_AXIS):
+def quantize_head(mode, D, rw, rho, wbar, S, quantizer: int = QUANT_DUAL_AXIS, scale_bits: int = 32):
     if quantizer == QUANT_ABSMAX:
-        z, h, r, c, tie = core.quantize_absmax(D, rw, S)
+        z, h, r, c, tie = core.quantize_absmax(D, rw, S, scale_bits=scale_bits)
     else:
-        z, h, r, c, tie = core.quantize(D, rw, rho, wbar, S)
-    return pack_head(mode, D, rw, z, h, r, c), tie
+        z, h, r, c, tie = core.quantize(D, rw, rho, wbar, S, scale_bits=scale_bits)
+    return pack_head(mode, D, rw, z, h, r, c, scale_bits), tie
 
 
-def reconstruct_head(mode, D, rw, rec):
-    z, h, r, c = unpack_head(mode, D, rw, rec)
+def reconstruct_head(mode, D, rw, rec, scale_bits: int = 32):
+    z, h, r, c = unpack_head(mode, D, rw, rec, scale_bits)
     return core.reconstruct(D, rw, z, h, r, c)
 
 
-def step_head(mode, D, rw, rho, wbar, rec, q, k, v, alpha, beta, quantizer: int = QUANT_DUAL_AXIS):
+def step_head(mode, D, rw, rho, wbar, rec, q, k, v, alpha, beta, quantizer: int = QUANT_DUAL_AXIS,
+              scale_bits: int = 32):
     """Decode step of one packed head.  Returns (new record, o, tie, S_t, w)."""
-    z, h, r, c = unpack_head(mode, D, rw, rec)
+    z, h, r, c = unpack_head(mode, D, rw, rec, scale_bits)
     S, o, u, w = core.step_from_codes(D, rw, z, h, r, c, q, k, v, alpha, beta)
-    new_rec, tie = quantize_head(mode, D, rw, rho, wbar, S, quantizer)
+    new_rec, tie = quantize_head(mode, D, rw, rho, wbar, S, quantizer, scale_bits)
     return new_rec, o, tie, S, w
 
 
@@ -98,12 +114,13 @@ class PlanView:
         self.rho = np.asarray(plan["rho"], np.float32).reshape(self.L, self.H, self.D)
         self.wbar = np.asarray(plan["wbar"], np.float32).reshape(self.L, self.H, self.D)
         self.quantizer = int(plan.get("quantizer", QUANT_DUAL_AXIS))
+        self.scale_bits = int(plan.get("scale_bits", 32))
 
     def rw(self, l, h):
         return plan_io.head_row_widths(self.plan, l, h)
 
     def rec_bytes(self, l, h):
-        return plan_io.record_bytes(self.mode, self.D, self.rw(l, h))
+        return plan_io.record_bytes(self.mode, self.D, self.rw(l, h), self.scale_bits)
 
     def record(self, pool_slot: np.ndarray, l, h):
         o = int(self.offsets[l * self.H + h])
@@ -111,7 +128,7 @@ class PlanView:
 
     def quantize_into(self, pool_slot: np.ndarray, l, h, S):
         rec, tie = quantize_head(self.mode, self.D, self.rw(l, h), self.rho[l, h], self.wbar[l, h], S,
-                                 self.quantizer)
+                                 self.quantizer, self.scale_bits)
         o = int(self.offsets[l * self.H + h])
         pool_slot[o:o + rec.size] = rec
         return tie
@@ -120,16 +137,17 @@ class PlanView:
         """Step one (slot, layer, head) in place; returns (o, tie, S_t, w)."""
         rec = self.record(pool_slot, l, h).copy()
         new_rec, o, tie, S, w = step_head(self.mode, self.D, self.rw(l, h), self.rho[l, h],
-                                          self.wbar[l, h], rec, q, k, v, alpha, beta, self.quantizer)
+                                          self.wbar[l, h], rec, q, k, v, alpha, beta, self.quantizer,
+                                          self.scale_bits)
         off = int(self.offsets[l * self.H + h])
         pool_slot[off:off + new_rec.size] = new_rec
         return o, tie, S, w
 
     def unpack(self, pool_slot, l, h):
-        return unpack_head(self.mode, self.D, self.rw(l, h), self.record(pool_slot, l, h))
+        return unpack_head(self.mode, self.D, self.rw(l, h), self.record(pool_slot, l, h), self.scale_bits)
 
     def reconstruct(self, pool_slot, l, h):
-        return reconstruct_head(self.mode, self.D, self.rw(l, h), self.record(pool_slot, l, h))
+        return reconstruct_head(self.mode, self.D, self.rw(l, h), self.record(pool_slot, l, h), self.scale_bits)
 
 
 # --------------------------------------------------------------------------
@@ -204,7 +222,7 @@ def _alpha_rows(a, D):
 
 
 def build_plan(mode: int, D: int, n_layers: int, n_heads: int, stats: dict, bits,
-               nominal_bits: float, n_pivots: int, horizon: int, lifetime=None) -> dict:
+               nominal_bits: float, n_pivots: int, horizon: int, lifetime=None, scale_bits: int = 32) -> dict:
     """Pivots, then DP (mode 0) or Lagrangian + repair (mode 1) allocation."""
     lgate = np.asarray(stats["lgate"], dtype=np.float64)
     if lifetime is None:
@@ -226,11 +244,11 @@ def build_plan(mode: int, D: int, n_layers: int, n_heads: int, stats: dict, bits
                 bitset=bits, nominal_bits=nominal_bits, horizon=horizon, widths=widths,
                 wbar=np.asarray(stats["wbar"], np.float32).reshape(-1),
                 rho=np.asarray(stats["rho"], np.float32).reshape(-1),
-                lgate=lgate, lifetime=np.asarray(lifetime, np.float64))
+                lgate=lgate, lifetime=np.asarray(lifetime, np.float64), scale_bits=int(scale_bits))
 
 
 def uniform_plan(mode: int, D: int, n_layers: int, n_heads: int, bits: int, quantizer: int,
-                 horizon: int, wbar=None) -> dict:
+                 horizon: int, wbar=None, scale_bits: int = 32) -> dict:
     """A baseline plan: every unit at `bits`, no pivots (实验: uniform INT-b).
     wbar defaults to ones (rho = 1); lgate is 0, so L_u = horizon."""
     n_units = n_layers * n_heads * (D if mode == 1 else 1)
@@ -240,7 +258,7 @@ def uniform_plan(mode: int, D: int, n_layers: int, n_heads: int, bits: int, quan
     return dict(mode=mode, n_layers=n_layers, n_heads=n_heads, d=D, n_pivots=0, bitset=[int(bits)],
                 nominal_bits=float(bits), horizon=horizon, widths=np.full(n_units, int(bits), np.uint8),
                 wbar=wbar, rho=rho, lgate=np.zeros(n_units), lifetime=np.full(n_units, float(horizon)),
-                quantizer=int(quantizer))
+                quantizer=int(quantizer), scale_bits=int(scale_bits))
 
 
 def lifetime_l_from_halflife(h: float) -> float:

@@ -15,7 +15,7 @@ Plan file, little-endian:
   44  4  f32 nominal bits    48  8  u64 horizon H
   56  4  u32 quantizer: 0 = STEPQuant dual-axis fit, 1 = per-row absmax
          (mode 0 only; every record keeps the codes | r | c layout, c = 1)
-  60  4  u32 zero
+  60  4  u32 scale storage: 0 = fp32 r and c, 16 = bfloat16 r and c
   64     u8  width[n_units]  (2, 4, 6, 8, or 16 for an FP16 pivot)
          zero padding to a multiple of 4 bytes
          f32 wbar[n_layers*n_heads*d_k]   row impact omega_i / mean omega
@@ -28,8 +28,9 @@ Pool layout: slot-major.  Slot s starts at s * slot_bytes; inside a slot the
 records of the (layer, head) pairs follow in order layer-major.  Record of a
 head:
   mode 0, pivot head : binary16 tile, row-major, D*D*2 bytes
-  mode 0, width b    : codes (uniform layout, D*D*b/8 bytes) | f32 r[D] | f32 c[D]
-  mode 1             : codes (row-major layout) | f32 r[D] | f32 c[D]
+  mode 0, width b    : codes (uniform layout, D*D*b/8 bytes) | r[D] | c[D]
+  mode 1             : codes (row-major layout) | r[D] | c[D]
+r and c are f32, or bf16 in plans with 16-bit scales;
 each padded with zeros to a multiple of 128 bytes.
 """
 from __future__ import annotations
@@ -60,7 +61,7 @@ def write_plan(path: str, plan: dict) -> bytes:
         bitset |= 1 << int(b)
     head = HEADER.pack(MAGIC, VERSION, mode, L, H, D, D, n_units, int(plan["n_pivots"]),
                        bitset, float(plan["nominal_bits"]), int(plan["horizon"]),
-                       int(plan.get("quantizer", 0)), 0)
+                       int(plan.get("quantizer", 0)), 16 if int(plan.get("scale_bits", 32)) == 16 else 0)
     body = bytearray(head)
     body += widths.tobytes()
     body += b"\0" * (_align(len(body), 4) - len(body))
@@ -78,7 +79,7 @@ def write_plan(path: str, plan: dict) -> bytes:
 
 def read_plan(data: bytes) -> dict:
     (magic, ver, mode, L, H, dk, dv, n_units, n_piv, bitset, nominal, horizon,
-     quantizer, _z) = HEADER.unpack_from(data, 0)
+     quantizer, sbits) = HEADER.unpack_from(data, 0)
     assert magic == MAGIC and ver == VERSION
     off = HEADER.size
     widths = np.frombuffer(data, dtype=np.uint8, count=n_units, offset=off).copy()
@@ -93,7 +94,7 @@ def read_plan(data: bytes) -> dict:
     return dict(mode=mode, n_layers=L, n_heads=H, d=dk, n_pivots=n_piv,
                 bitset=[b for b in range(32) if bitset >> b & 1], nominal_bits=nominal,
                 horizon=horizon, widths=widths, wbar=wbar, rho=rho, lgate=lgate, lifetime=life,
-                quantizer=quantizer)
+                quantizer=quantizer, scale_bits=16 if sbits == 16 else 32)
 
 
 # --------------------------------------------------------------------------
@@ -108,15 +109,16 @@ def head_row_widths(plan: dict, layer: int, head: int) -> np.ndarray:
     return np.asarray(plan["widths"][hidx * D:(hidx + 1) * D], dtype=np.int32)
 
 
-def record_bytes(mode: int, D: int, row_widths) -> int:
+def record_bytes(mode: int, D: int, row_widths, scale_bits: int = 32) -> int:
     rw = np.asarray(row_widths)
+    sb = 2 * D * (scale_bits // 8)  # r[D] and c[D]
     if mode == 0:
         b = int(rw[0])
         if b == PIVOT_BITS:
             return _align(D * D * 2, 128)
-        return _align(D * D * b // 8 + 8 * D, 128)
+        return _align(D * D * b // 8 + sb, 128)
     codes = int(sum(D * int(b) // 8 for b in rw))
-    return _align(codes + 8 * D, 128)
+    return _align(codes + sb, 128)
 
 
 def codes_block_bytes(mode: int, D: int, row_widths) -> int:
@@ -134,5 +136,5 @@ def pool_layout(plan: dict):
     for l in range(plan["n_layers"]):
         for h in range(plan["n_heads"]):
             offs.append(o)
-            o += record_bytes(plan["mode"], plan["d"], head_row_widths(plan, l, h))
+            o += record_bytes(plan["mode"], plan["d"], head_row_widths(plan, l, h), int(plan.get("scale_bits", 32)))
     return np.array(offs, dtype=np.int64), o

@@ -81,6 +81,35 @@ uint16_t sq_f32_to_f16(float x)
 }
 
 /* ------------------------------------------------------------------------ */
+/* bfloat16 (the top 16 bits of a binary32: 1 sign, 8 exponent, 7 fraction) */
+/* with round to nearest, ties to even, written from the format definition. */
+/* Storage of the r and c scales in plans with 16-bit scales.               */
+/* ------------------------------------------------------------------------ */
+
+uint16_t sq_f32_to_bf16(float x)
+{
+    uint32_t u;
+    memcpy(&u, &x, 4);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return (uint16_t)((u >> 16) | 0x0040u); /* NaN */
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7FFFu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+float sq_bf16_to_f32(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float x;
+    memcpy(&x, &u, 4);
+    return x;
+}
+
+static float round_scale(float x, int scale_bits)
+{
+    return scale_bits == 16 ? sq_bf16_to_f32(sq_f32_to_bf16(x)) : x;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Packed format (our own; the pages fix only that the layout is decided     */
 /* offline, "方法-4": 离线分配固定 packed layout).                             */
 /*                                                                          */
@@ -228,6 +257,10 @@ float sq_pairwise_sum(const float *x, int n)
 /*     which equal w r z0 S and w r^2 z0^2 up to the common factor 1/r;       */
 /*     rows of 16-bit (pivot) width contribute 0; a zero denominator keeps c0; */
 /*   - c_j is rounded to fp32 before the final codes are taken.               */
+/*   - 16-bit scale storage (scale_bits = 16, survey row f1): r_i is rounded  */
+/*     to bfloat16 (RNE) as soon as it is formed and that value is used      */
+/*     everywhere after (1/r, b_i, the record); c_j likewise after the        */
+/*     refinement, before the final codes.  sq_quantize = scale_bits 32.      */
 /* 16-bit rows are stored as binary16 (RNE) and carry no row factor (r = 0).  */
 /* tie_out (optional, D*D): bit0 = final code within 1e-6 relative of a .5   */
 /* boundary; bit1 = its column had such a tie in z0 (column tie-affected).   */
@@ -243,9 +276,9 @@ static int near_half(double x)
     return fabs(ax - (f + 0.5)) <= 1e-6 * ax;
 }
 
-void sq_quantize(int D, const int *widths, const float *rho, const float *wbar,
-                 const float *S, int32_t *z, uint16_t *h, float *r, float *c,
-                 uint8_t *tie_out, int32_t *z0_out)
+void sq_quantize_s(int D, const int *widths, const float *rho, const float *wbar,
+                   const float *S, int32_t *z, uint16_t *h, float *r, float *c,
+                   uint8_t *tie_out, int32_t *z0_out, int scale_bits)
 {
     float *absrow = (float *)malloc(sizeof(float) * D);
     float *y = (float *)malloc(sizeof(float) * D * D);
@@ -270,7 +303,7 @@ void sq_quantize(int D, const int *widths, const float *rho, const float *wbar,
         for (int j = 0; j < D; j++) absrow[j] = fabsf(S[i * D + j]);
         float m = sq_pairwise_sum(absrow, D) * (1.0f / (float)D);
         if (!(m > 1e-12f)) m = 1e-12f;
-        r[i] = m * rho[i];
+        r[i] = round_scale(m * rho[i], scale_bits);
         float inv_r = 1.0f / r[i];
         for (int j = 0; j < D; j++) {
             y[i * D + j] = S[i * D + j] * inv_r;
@@ -304,7 +337,7 @@ void sq_quantize(int D, const int *widths, const float *rho, const float *wbar,
         }
         float num = sq_pairwise_sum(tn, D);
         float den = sq_pairwise_sum(td, D);
-        float cj = (den > 0.0f) ? num / den : c0;
+        float cj = round_scale((den > 0.0f) ? num / den : c0, scale_bits);
         c[j] = cj;
         float inv_c = 1.0f / cj;
         for (int i = 0; i < D; i++) {
@@ -331,6 +364,13 @@ void sq_quantize(int D, const int *widths, const float *rho, const float *wbar,
     free(absrow); free(y); free(bw); free(tn); free(td); free(z0); free(coltie);
 }
 
+void sq_quantize(int D, const int *widths, const float *rho, const float *wbar,
+                 const float *S, int32_t *z, uint16_t *h, float *r, float *c,
+                 uint8_t *tie_out, int32_t *z0_out)
+{
+    sq_quantize_s(D, widths, rho, wbar, S, z, h, r, c, tie_out, z0_out, 32);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Per-row absmax quantizer: the ordinary baseline the pages set against     */
 /* STEPQuant (实验: uniform INT4 / INT6 / INT8 and the remark that plain      */
@@ -344,8 +384,8 @@ void sq_quantize(int D, const int *widths, const float *rho, const float *wbar,
 /* tie_out (optional): bit0 = code within 1e-6 relative of a .5 boundary.    */
 /* ------------------------------------------------------------------------ */
 
-void sq_quantize_absmax(int D, const int *widths, const float *S, int32_t *z, uint16_t *h,
-                        float *r, float *c, uint8_t *tie_out)
+void sq_quantize_absmax_s(int D, const int *widths, const float *S, int32_t *z, uint16_t *h,
+                          float *r, float *c, uint8_t *tie_out, int scale_bits)
 {
     for (int j = 0; j < D; j++) c[j] = 1.0f;
     for (int i = 0; i < D; i++) {
@@ -364,7 +404,7 @@ void sq_quantize_absmax(int D, const int *widths, const float *S, int32_t *z, ui
             float a = fabsf(S[i * D + j]);
             if (a > m) m = a;
         }
-        r[i] = (m > 0.0f) ? m / (float)q : 1.0f;
+        r[i] = round_scale((m > 0.0f) ? m / (float)q : 1.0f, scale_bits);
         float inv_r = 1.0f / r[i];
         for (int j = 0; j < D; j++) {
             double x = (double)S[i * D + j] * (double)inv_r; /* exact: 24 x 24 bits */
@@ -376,6 +416,12 @@ void sq_quantize_absmax(int D, const int *widths, const float *S, int32_t *z, ui
             if (tie_out) tie_out[i * D + j] = (uint8_t)(near_half(x) ? 1 : 0);
         }
     }
+}
+
+void sq_quantize_absmax(int D, const int *widths, const float *S, int32_t *z, uint16_t *h,
+                        float *r, float *c, uint8_t *tie_out)
+{
+    sq_quantize_absmax_s(D, widths, S, z, h, r, c, tie_out, 32);
 }
 
 /* Reconstruction X_hat_ij = fl(fl(r_i * c_j) * z_ij); 16-bit rows decode the

@@ -414,6 +414,70 @@ def _outlier_state(D, seed):
     return S
 
 
+# --------------------------------------------------------------------------
+# 16-bit (bfloat16) scale storage: the conversion against torch's bfloat16,
+# r = bf16(r of the fp32 fit), codes nearest to y * fl(1/c) with the stored
+# scales, the half-step bound with the stored scales, record bytes
+# --------------------------------------------------------------------------
+
+def test_bf16_matches_torch():
+    torch = pytest.importorskip("torch")
+    xs = np.concatenate([
+        rng.standard_normal(5000).astype(np.float32) * 10.0 ** rng.integers(-30, 30, 5000),
+        np.array([0.0, -0.0, 1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9, 3e38, 1e-40, -2.5], np.float32),
+    ]).astype(np.float32)
+    ref = torch.from_numpy(xs).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    for x, rb in zip(xs, ref):
+        assert core.f32_to_bf16(x) == int(rb), x
+        assert core.bf16_to_f32(int(rb)) == float(torch.tensor([int(rb)], dtype=torch.int32).to(torch.int16)
+                                                   .view(torch.bfloat16).float()[0])
+
+
+@pytest.mark.parametrize("b", [4, 6, 8])
+def test_scale16_rows_are_rounded_fp32_rows_and_codes_nearest(b):
+    torch = pytest.importorskip("torch")
+    D, q = 16, (1 << (b - 1)) - 1
+    S = _outlier_state(D, 500 + b)
+    widths = np.full(D, b)
+    rho = np.linspace(0.7, 1.3, D).astype(np.float32)
+    wbar = (1.0 / rho.astype(np.float64) ** 4).astype(np.float32)
+    z32, _, r32, c32, _ = core.quantize(D, widths, rho, wbar, S)
+    z16, _, r16, c16, _ = core.quantize(D, widths, rho, wbar, S, scale_bits=16)
+    bf = torch.from_numpy(r32).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(r16, bf)
+    for x in np.concatenate([r16, c16]):  # representable in bfloat16
+        assert np.float32(x).view(np.uint32) & 0xFFFF == 0
+    cand = np.arange(-q, q + 1, dtype=np.float64)
+    for i in range(D):
+        inv_r = np.float32(1.0) / r16[i]
+        for j in range(D):
+            y = np.float32(S[i, j] * inv_r)
+            x = float(y) * float(np.float32(1.0) / c16[j])
+            dd = np.abs(cand - x)
+            best = cand[dd == dd.min()]
+            pick = best[0] if best.size == 1 else best[np.argmin(np.abs(best) % 2)]
+            assert z16[i, j] == int(pick), (i, j)
+            if abs(x) <= q:
+                assert abs(float(S[i, j]) - float(r16[i]) * float(c16[j]) * z16[i, j]) <= \
+                    0.5 * float(r16[i]) * float(c16[j]) * (1 + 1e-5) + 1e-6 * abs(float(S[i, j]))
+
+
+def test_scale16_record_layout_and_plan_field(tmp_path):
+    D = 16
+    plan = model.uniform_plan(0, D, 2, 2, 6, model.QUANT_DUAL_AXIS, 4096, scale_bits=16)
+    back = plan_io.read_plan(plan_io.write_plan(str(tmp_path / "p.bin"), plan))
+    assert back["scale_bits"] == 16
+    assert plan_io.record_bytes(0, D, np.full(D, 6), 16) == 256  # 192 code bytes + 64 scale bytes
+    assert plan_io.record_bytes(0, 128, np.full(128, 6), 16) == 12288 + 512
+    pv = model.PlanView(back)
+    slot = np.zeros(pv.slot_bytes, np.uint8)
+    S = _outlier_state(D, 600)
+    pv.quantize_into(slot, 1, 1, S)
+    z, h, r, c = pv.unpack(slot, 1, 1)
+    z2, _, r2, c2, _ = core.quantize(D, np.full(D, 6), pv.rho[1, 1], pv.wbar[1, 1], S, scale_bits=16)
+    assert np.array_equal(z, z2) and np.array_equal(r, r2) and np.array_equal(c, c2)
+
+
 @pytest.mark.parametrize("b", [2, 4, 6, 8])
 def test_absmax_codes_are_nearest_by_enumeration(b):
     D, q = 16, (1 << (b - 1)) - 1
