@@ -42,8 +42,12 @@
  *     stream byte B of thread t at block byte ((B/RT) NT + t) RT + B%RT.
  *   per-row units (mode 1): rows in order, row i = D*b_i/8 bytes, code j at
  *     row bits [b_i j, b_i j + b_i); a 16-bit row holds binary16 values.
- *   record = codes | f32 r[D] | f32 c[D], zero-padded to 128 bytes; a mode-0
- *     pivot head's record is its binary16 tile, row-major, D*D*2 bytes.
+ *   record = codes | r[D] | c[D], zero-padded to 128 bytes, r and c fp32, or
+ *     bfloat16 in plans with 16-bit scales (header word at byte 60 = 16: r_i
+ *     is rounded to bfloat16, RNE, as soon as it is formed and used rounded
+ *     from then on; c_j likewise after the refinement); a mode-0 pivot head's
+ *     record is its binary16 tile, row-major, D*D*2 bytes.  Per-row units
+ *     (mode 1) run on the device at D = 128 only (stepq_ctx_create).
  *   pool   = n_slots slots of slot_bytes each; inside a slot the records of
  *     (layer, head) follow layer-major (offsets: stepq_plan_record).
  *
@@ -116,6 +120,7 @@ typedef struct stepq_plan_info {
     double bits_per_value_s16;   /* the same with 16-bit scale accounting */
     int units_by_width[17];      /* histogram of unit widths (index = bits) */
     int quantizer;               /* STEPQ_QUANT_DUAL_AXIS or STEPQ_QUANT_ABSMAX */
+    int scale_bits;              /* storage of r and c: 32 (fp32) or 16 (bfloat16) */
 } stepq_plan_info;
 
 /* ---- plan (方法-1 offline precision map) -------------------------------- */
@@ -146,19 +151,23 @@ int stepq_plan_record(const stepq_plan *plan, int layer, int head, uint64_t *off
  *   lgate[n_units]            mean log retention gate l_u
  *   dist[n_units][n_bits]     distortion d_u(b) per allowed width
  *   wbar[n_layers*n_heads*d]  normalised row impact omega_i / mean omega
- * rho_i = fl32(1/sqrt(sqrt(wbar_i))) is derived.  Host pointers.  Writes the
- * plan file to `path` (NULL: none) and returns the parsed plan in *out. */
+ * rho_i = fl32(1/sqrt(sqrt(wbar_i))) is derived.  scale_bits: 32 (fp32 r, c)
+ * or 16 (bfloat16 r, c).  Host pointers.  Writes the plan file to `path`
+ * (NULL: none) and returns the parsed plan in *out. */
 int stepq_plan_build(int mode, int n_layers, int n_heads, int d, const int *bits, int n_bits,
                      float nominal_bits, int n_pivots, uint64_t horizon, const double *lgate,
-                     const double *dist, const float *wbar, const char *path, stepq_plan **out);
+                     const double *dist, const float *wbar, int scale_bits, const char *path,
+                     stepq_plan **out);
 
 /* A baseline plan (实验: uniform INT-b): every unit at width `bits` (2, 4, 6
  * or 8), no pivots, the given quantizer (STEPQ_QUANT_ABSMAX needs mode 0).
  * wbar[n_layers*n_heads*d] (host, NULL: all ones) feeds rho for the
- * dual-axis fit; lgate is 0 for every unit.  Writes the plan file to `path`
+ * dual-axis fit; lgate is 0 for every unit; scale_bits 32 or 16 as for
+ * stepq_plan_build.  Writes the plan file to `path`
  * (NULL: none) and returns the parsed plan.  Errors: STEPQ_EINVAL. */
 int stepq_plan_build_uniform(int mode, int n_layers, int n_heads, int d, int bits, int quantizer,
-                             uint64_t horizon, const float *wbar, const char *path, stepq_plan **out);
+                             uint64_t horizon, const float *wbar, int scale_bits, const char *path,
+                             stepq_plan **out);
 
 /* ---- context ------------------------------------------------------------ */
 

@@ -86,6 +86,7 @@ T rd(const uint8_t *p) {
 struct stepq_plan {
     int mode = 0, L = 0, H = 0, D = 0, n_units = 0, n_pivots = 0;
     int quantizer = 0;                // 0 dual-axis fit, 1 per-row absmax (mode 0)
+    int scale_bits = 32;              // storage of r and c: 32 (fp32) or 16 (bfloat16)
     uint32_t bitset = 0;
     float nominal = 0.f;
     uint64_t horizon = 0;
@@ -107,7 +108,8 @@ struct stepq_plan {
  *   0  8 magic "STEPQPL1" | 8 u32 version=1 | 12 u32 mode | 16 u32 n_layers
  *   20 u32 n_heads | 24 u32 d_k | 28 u32 d_v | 32 u32 n_units | 36 u32 n_pivots
  *   40 u32 bitset | 44 f32 nominal bits | 48 u64 horizon | 56 u32 quantizer
- *   (0 dual-axis fit, 1 per-row absmax; mode 0 only) | 60 u32 zero
+ *   (0 dual-axis fit, 1 per-row absmax; mode 0 only) | 60 u32 scale storage
+ *   (0: fp32 r and c, 16: bfloat16 r and c)
  *   64 u8 width[n_units], zero pad to 4 | f32 wbar[L*H*d] | f32 rho[L*H*d]
  *   f64 lgate[n_units] | f64 lifetime[n_units] | u32 CRC-32 of all before it
  */
@@ -130,7 +132,9 @@ static int plan_parse(const uint8_t *d, size_t n, stepq_plan *p) {
     if (p->mode != 0 && p->mode != 1) return fail(STEPQ_EFORMAT, "plan: mode %d", p->mode);
     if (p->quantizer != 0 && !(p->quantizer == 1 && p->mode == 0))
         return fail(STEPQ_EFORMAT, "plan: quantizer %d with mode %d", p->quantizer, p->mode);
-    if (rd<uint32_t>(d + 60) != 0) return fail(STEPQ_EFORMAT, "plan: reserved header word is not zero");
+    const uint32_t sw = rd<uint32_t>(d + 60);
+    if (sw != 0 && sw != 16) return fail(STEPQ_EFORMAT, "plan: scale storage word %u (0 or 16)", sw);
+    p->scale_bits = sw == 16 ? 16 : 32;
     if (dk != dv) return fail(STEPQ_EFORMAT, "plan: d_k %u != d_v %u", dk, dv);
     if (dk != 16 && dk != 32 && dk != 64 && dk != 128) return fail(STEPQ_EFORMAT, "plan: d = %u unsupported", dk);
     p->D = (int)dk;
@@ -188,14 +192,14 @@ static int plan_parse(const uint8_t *d, size_t n, stepq_plan *p) {
             const int w = p->width[hd];
             p->head_width[hd] = (uint8_t)w;
             codes = (uint64_t)D * D * w / 8;
-            rec = (w == STEPQ_PIVOT_BITS) ? align_up(codes, 128) : align_up(codes + 8ull * D, 128);
+            rec = (w == STEPQ_PIVOT_BITS) ? align_up(codes, 128) : align_up(codes + 2ull * (p->scale_bits / 8) * D, 128);
         } else {
             codes = 0;
             for (int i = 0; i < D; ++i) {
                 p->row_off[hd * D + i] = (uint32_t)codes;
                 codes += (uint64_t)D * p->width[hd * D + i] / 8;
             }
-            rec = align_up(codes + 8ull * D, 128);
+            rec = align_up(codes + 2ull * (p->scale_bits / 8) * D, 128);
         }
         p->rec_off[hd] = off;
         p->codes_bytes[hd] = (uint32_t)codes;
@@ -264,6 +268,7 @@ extern "C" int stepq_plan_get_info(const stepq_plan *p, stepq_plan_info *o) {
     o->bits_per_value = p->bpv;
     o->bits_per_value_s16 = p->bpv16;
     o->quantizer = p->quantizer;
+    o->scale_bits = p->scale_bits;
     for (int w : p->width) o->units_by_width[w <= 16 ? w : 0]++;
     return STEPQ_OK;
 }
@@ -424,7 +429,7 @@ void put_u64(std::vector<uint8_t> &v, uint64_t x) { v.insert(v.end(), (uint8_t *
 
 // The plan file image (format above); rho_i = fl32(1/sqrt(sqrt(wbar_i))).
 std::vector<uint8_t> serialize_plan(int mode, int n_layers, int n_heads, int d, int n_pivots, uint32_t bitset,
-                                    float nominal_bits, uint64_t horizon, int quantizer,
+                                    float nominal_bits, uint64_t horizon, int quantizer, int scale_bits,
                                     const std::vector<uint8_t> &width, const float *wbar, const double *lgate,
                                     const std::vector<double> &life) {
     const size_t heads = (size_t)n_layers * n_heads, nrow = heads * d, units = width.size();
@@ -444,7 +449,7 @@ std::vector<uint8_t> serialize_plan(int mode, int n_layers, int n_heads, int d, 
     put_u32(f, nb);
     put_u64(f, horizon);
     put_u32(f, (uint32_t)quantizer);
-    put_u32(f, 0);
+    put_u32(f, scale_bits == 16 ? 16u : 0u);
     f.insert(f.end(), width.begin(), width.end());
     while (f.size() % 4) f.push_back(0);
     const size_t off_wb = f.size();
@@ -476,8 +481,10 @@ int write_plan_file(const char *path, const std::vector<uint8_t> &f, const char 
 
 extern "C" int stepq_plan_build(int mode, int n_layers, int n_heads, int d, const int *bits, int n_bits,
                                 float nominal_bits, int n_pivots, uint64_t horizon, const double *lgate,
-                                const double *dist, const float *wbar, const char *path, stepq_plan **out) {
+                                const double *dist, const float *wbar, int scale_bits, const char *path,
+                                stepq_plan **out) {
     if (!bits || !lgate || !dist || !wbar || !out) return fail(STEPQ_EINVAL, "plan_build: null argument");
+    if (scale_bits != 16 && scale_bits != 32) return fail(STEPQ_EINVAL, "plan_build: scale_bits %d", scale_bits);
     if (mode != 0 && mode != 1) return fail(STEPQ_EINVAL, "plan_build: mode %d", mode);
     if (n_layers <= 0 || n_heads <= 0 || (d != 16 && d != 32 && d != 64 && d != 128))
         return fail(STEPQ_EINVAL, "plan_build: bad dims");
@@ -517,14 +524,16 @@ extern "C" int stepq_plan_build(int mode, int n_layers, int n_heads, int d, cons
     if (!ok) return fail(STEPQ_EINVAL, "plan_build: budget %lld below the smallest width", cap);
     for (int k = 0; k < N; ++k) width[keep[k]] = (uint8_t)alloc[k];
     const std::vector<uint8_t> f = serialize_plan(mode, n_layers, n_heads, d, n_pivots, bitset, nominal_bits, horizon,
-                                                  0, width, wbar, lgate, life);
+                                                  0, scale_bits, width, wbar, lgate, life);
     if (int rc = write_plan_file(path, f, "plan_build")) return rc;
     return stepq_plan_load_mem(f.data(), f.size(), out);
 }
 
 extern "C" int stepq_plan_build_uniform(int mode, int n_layers, int n_heads, int d, int bits, int quantizer,
-                                        uint64_t horizon, const float *wbar, const char *path, stepq_plan **out) {
+                                        uint64_t horizon, const float *wbar, int scale_bits, const char *path,
+                                        stepq_plan **out) {
     if (!out) return fail(STEPQ_EINVAL, "plan_build_uniform: null argument");
+    if (scale_bits != 16 && scale_bits != 32) return fail(STEPQ_EINVAL, "plan_build_uniform: scale_bits %d", scale_bits);
     if (mode != 0 && mode != 1) return fail(STEPQ_EINVAL, "plan_build_uniform: mode %d", mode);
     if (n_layers <= 0 || n_heads <= 0 || (d != 16 && d != 32 && d != 64 && d != 128))
         return fail(STEPQ_EINVAL, "plan_build_uniform: bad dims");
@@ -541,7 +550,7 @@ extern "C" int stepq_plan_build_uniform(int mode, int n_layers, int n_heads, int
     const std::vector<double> lgate(units, 0.0);
     const std::vector<double> life(units, lifetime_weight(0.0, horizon));
     const std::vector<uint8_t> f = serialize_plan(mode, n_layers, n_heads, d, 0, 1u << bits, (float)bits, horizon,
-                                                  quantizer, width, wbar, lgate.data(), life);
+                                                  quantizer, scale_bits, width, wbar, lgate.data(), life);
     if (int rc = write_plan_file(path, f, "plan_build_uniform")) return rc;
     return stepq_plan_load_mem(f.data(), f.size(), out);
 }
@@ -602,6 +611,7 @@ stepq::Args base_args(stepq_ctx *c, void *pool, const int32_t *slots, int n_req,
     a.H = c->plan->H;
     a.mode = c->plan->mode;
     a.quantizer = c->plan->quantizer;
+    a.scale16 = c->plan->scale_bits == 16 ? 1 : 0;
     a.n_items = n_req * (le - lb) * c->plan->H;
     a.div_nreq = stepq::div_magic((uint32_t)n_req);
     a.div_h = stepq::div_magic((uint32_t)c->plan->H);
@@ -675,6 +685,8 @@ extern "C" int stepq_ctx_create(const stepq_plan *plan, void *main_stream, void 
     e = cudaGetDeviceProperties(&prop, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
     if (prop.major < 10) return fail(STEPQ_ECUDA, "ctx_create: device %d is sm_%d%d; this library is built for sm_100a", dev, prop.major, prop.minor);
+    if (plan->mode == 1 && plan->D != 128)
+        return fail(STEPQ_EINVAL, "ctx_create: per-key-row plans run on the device at d = 128 only (d = %d)", plan->D);
     stepq_ctx *c = new (std::nothrow) stepq_ctx;
     if (!c) return fail(STEPQ_ENOMEM, "ctx_create: out of memory");
     c->plan = plan;

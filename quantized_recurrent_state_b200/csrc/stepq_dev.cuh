@@ -7,6 +7,7 @@
 // arithmetic definitions are stated in include/stepq.h.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -47,6 +48,7 @@ struct Args {
     int H;
     int mode;
     int quantizer;           // kQuantDualAxis or kQuantAbsmax (per-head units)
+    int scale16;             // 1: r and c stored as bfloat16 (else fp32)
     int n_items;             // n_req * nL * H
     uint64_t div_nreq;       // floor(2^64 / n_req) + 1 (0 when n_req == 1): n / n_req = umul64hi(n, div_nreq)
     uint64_t div_h;          // the same for H
@@ -241,6 +243,33 @@ __device__ __forceinline__ double lane_sum_f64(double v) {
 }
 
 __device__ __forceinline__ void flag_error(int *err, int code) { atomicOr(err, code); }
+
+// Scale storage: fp32, or bfloat16 (the top half of an fp32, RNE).
+__device__ __forceinline__ float scale_at(const uint8_t *base, int i, int s16) {
+    return s16 ? __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(base)[i] << 16)
+               : reinterpret_cast<const float *>(base)[i];
+}
+
+// Four consecutive scales from index j0 (a multiple of 4; base 8-byte aligned).
+__device__ __forceinline__ float4 scale4_at(const uint8_t *base, int j0, int s16) {
+    if (s16) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(base + 2 * j0);
+        return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                           __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+    }
+    return *reinterpret_cast<const float4 *>(base + 4 * j0);
+}
+
+// x rounded to the stored scale precision.
+__device__ __forceinline__ float scale_round(float x, int s16) {
+    return s16 ? __uint_as_float((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x)) << 16) : x;
+}
+
+// Store a scale already rounded by scale_round.
+__device__ __forceinline__ void scale_put(uint8_t *base, int i, float x, int s16) {
+    if (s16) reinterpret_cast<uint16_t *>(base)[i] = (uint16_t)(__float_as_uint(x) >> 16);
+    else reinterpret_cast<float *>(base)[i] = x;
+}
 
 // n / d for n < 2^32 with m = div_magic(d): floor(n m / 2^64) differs from
 // n / d by less than n / 2^64 < 1 / d, which cannot cross an integer.

@@ -341,18 +341,18 @@ __device__ __forceinline__ uint32_t final_e(float t) {
 // and pf1 (denominator): c_j = num / den (c0_j when den = 0), two threads
 // per column; each sums four bands pairwise and the pair adds the halves,
 // which is the balanced tree over the eight bands.
-template <int D>
-__device__ __forceinline__ void column_ls_fit(Scratch<D> &sc, int tid, float *rec_c) {
+template <int D, int s16>
+__device__ __forceinline__ void column_ls_fit(Scratch<D> &sc, int tid, uint8_t *rec_c) {
     const int j = tid >> 1, h = tid & 1, b0 = 4 * h;
     float num = (sc.pf0[b0][j] + sc.pf0[b0 + 1][j]) + (sc.pf0[b0 + 2][j] + sc.pf0[b0 + 3][j]);
     float den = (sc.pf1[b0][j] + sc.pf1[b0 + 1][j]) + (sc.pf1[b0 + 2][j] + sc.pf1[b0 + 3][j]);
     num = num + __shfl_xor_sync(0xffffffffu, num, 1);
     den = den + __shfl_xor_sync(0xffffffffu, den, 1);
     if (h == 0) {
-        const float c = (den > 0.0f) ? __fdiv_rn(num, den) : sc.c0[j];
+        const float c = scale_round((den > 0.0f) ? __fdiv_rn(num, den) : sc.c0[j], s16);
         sc.ic[j] = __frcp_rn(c);
         sc.cold[j] = c;
-        if (rec_c) rec_c[j] = c;
+        if (rec_c) scale_put(rec_c, j, c, s16);
     }
     __syncthreads();
 }
@@ -360,13 +360,14 @@ __device__ __forceinline__ void column_ls_fit(Scratch<D> &sc, int tid, float *re
 // ---------------------------------------------------------------------------
 // Refit of the fp32 tile S held in registers as column pairs (all rows at
 // width B).  On return S holds y = fl(S * fl(1/r)); sc.rowr[i] = r_i,
-// sc.cold[j] = c_j, sc.ic[j] = fl(1/c_j).  rec_r / rec_c (global, may be
+// sc.cold[j] = c_j, sc.ic[j] = fl(1/c_j) (r and c rounded to the stored
+// precision first when s16).  rec_r / rec_c (global scale arrays, may be
 // null) receive r and c.  rho / wbar: the head's rho_i and wbar_i (shared
 // memory).
 // ---------------------------------------------------------------------------
-template <int D, int B>
+template <int D, int B, int s16>
 __device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const float *rho, const float *wbar,
-                           float *rec_r, float *rec_c) {
+                           uint8_t *rec_r, uint8_t *rec_c) {
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES, RS = Scratch<D>::RS, HALF = LANES / 2;
     constexpr int Q = (1 << (B - 1)) - 1;
@@ -399,14 +400,14 @@ __device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const
         const int i = g * RT + rr;
         float m = __fmul_rn(s, 1.0f / (float)D);
         m = fmaxf(m, 1e-12f);
-        const float ri = __fmul_rn(m, rho[i]);
+        const float ri = scale_round(__fmul_rn(m, rho[i]), s16);
         const float inv = __frcp_rn(ri);
         const float bw = __fmul_rn(wbar[i], __fmul_rn(ri, ri));
         if (hh == 0) {
             sc.rinv2[i] = make_float2(inv, inv);
             sc.bw2[i] = make_float2(bw, bw);
             sc.rowr[i] = ri;
-            if (rec_r) rec_r[i] = ri;
+            if (rec_r) scale_put(rec_r, i, ri, s16);
         }
     }
     __syncwarp();
@@ -469,11 +470,11 @@ __device__ void fit_scales(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const
         }
     }
     __syncthreads();
-    column_ls_fit<D>(sc, tid, rec_c);
+    column_ls_fit<D, s16>(sc, tid, rec_c);
 }
 
 // Refit and pack into the record at `rec` (global): codes, r, c.
-template <int D, int B>
+template <int D, int B, int s16>
 __device__ void fit_pack(float2 (&S)[D / 8][2], uint8_t *rec, Scratch<D> &sc, int tid, const float *rho,
                          const float *wbar) {
     using G = Geo<D>;
@@ -483,9 +484,9 @@ __device__ void fit_pack(float2 (&S)[D / 8][2], uint8_t *rec, Scratch<D> &sc, in
     const int l = tid % LANES;
     const int j0 = 4 * l;
     const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
-    float *rec_r = reinterpret_cast<float *>(rec + codes_bytes);
-    float *rec_c = rec_r + D;
-    fit_scales<D, B>(S, sc, tid, rho, wbar, rec_r, rec_c);
+    uint8_t *rec_r = rec + codes_bytes;
+    uint8_t *rec_c = rec_r + D * (s16 ? 2 : 4);
+    fit_scales<D, B, s16>(S, sc, tid, rho, wbar, rec_r, rec_c);
     uint32_t W[Stream<D, B>::NW];
 #pragma unroll
     for (int i = 0; i < Stream<D, B>::NW; ++i) W[i] = 0u;
@@ -509,7 +510,7 @@ __device__ void fit_pack(float2 (&S)[D / 8][2], uint8_t *rec, Scratch<D> &sc, in
 // quantizer field): r_i = fl(max_j |S_ij| / qmax) (1 for a zero row), codes
 // = clamp(rne(S_ij * fl(1/r_i))), c = 1.  Rows live inside one warp, so the
 // whole fit needs no block barrier.  Writes codes, r and c to `rec`.
-template <int D, int B>
+template <int D, int B, int s16>
 __device__ void fit_pack_absmax(float2 (&S)[D / 8][2], uint8_t *rec, Scratch<D> &sc, int tid) {
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES, RS = Scratch<D>::RS, HALF = LANES / 2;
@@ -517,8 +518,8 @@ __device__ void fit_pack_absmax(float2 (&S)[D / 8][2], uint8_t *rec, Scratch<D> 
     constexpr float MG2 = kMagic + (float)(1 << (B - 1));
     const int g = tid / LANES, l = tid % LANES;
     const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
-    float *rec_r = reinterpret_cast<float *>(rec + codes_bytes);
-    float *rec_c = rec_r + D;
+    uint8_t *rec_r = rec + codes_bytes;
+    uint8_t *rec_c = rec_r + D * (s16 ? 2 : 4);
     // 1. row maxima: this thread's 4 columns, then the row's lanes (transpose)
     float *rs = &sc.rsum[g][0][0];
 #pragma unroll
@@ -533,15 +534,15 @@ __device__ void fit_pack_absmax(float2 (&S)[D / 8][2], uint8_t *rec, Scratch<D> 
         for (int k = 0; k < HALF; ++k) m = fmaxf(m, src[k]);
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
         const int i = g * RT + rr;
-        const float ri = (m > 0.0f) ? __fdiv_rn(m, (float)Q) : 1.0f;
+        const float ri = scale_round((m > 0.0f) ? __fdiv_rn(m, (float)Q) : 1.0f, s16);
         const float inv = __frcp_rn(ri);
         if (hh == 0) {
             sc.rinv2[i] = make_float2(inv, inv);
-            rec_r[i] = ri;
+            scale_put(rec_r, i, ri, s16);
         }
     }
     __syncwarp();
-    if (tid < D) rec_c[tid] = 1.0f;
+    if (tid < D) scale_put(rec_c, tid, 1.0f, s16);
     // 2. codes e = rne(S * fl(1/r)) + qmax, clamped, packed into the stream
     uint32_t W[Stream<D, B>::NW];
 #pragma unroll
@@ -619,9 +620,9 @@ __device__ __forceinline__ void band_sums(Scratch<D> &sc, int tid, double x0, do
 
 // Column phase of the decode: u, w, o of column j from the band partials
 // (already relative to the offset-binary bias), two threads per column.
-template <int D, int KIND>
+template <int D, int KIND, int s16 = 0>
 __device__ __forceinline__ void finish_columns(const Args &a, Scratch<D> &sc, int tid, int row, float beta,
-                                               const float *vs, const float *cs) {
+                                               const float *vs, const uint8_t *cs) {
     const int j = tid >> 1, h = tid & 1, b0 = 4 * h;
     double su = (sc.u.col.pU[b0][j] + sc.u.col.pU[b0 + 1][j]) + (sc.u.col.pU[b0 + 2][j] + sc.u.col.pU[b0 + 3][j]);
     double so = (sc.u.col.pO[b0][j] + sc.u.col.pO[b0 + 1][j]) + (sc.u.col.pO[b0 + 2][j] + sc.u.col.pO[b0 + 3][j]);
@@ -629,7 +630,7 @@ __device__ __forceinline__ void finish_columns(const Args &a, Scratch<D> &sc, in
     su += __shfl_xor_sync(0xffffffffu, su, 1);
     so += __shfl_xor_sync(0xffffffffu, so, 1);
     qk += __shfl_xor_sync(0xffffffffu, qk, 1);
-    const double cj = cs ? (double)cs[j] : 1.0;
+    const double cj = cs ? (double)scale_at(cs, j, s16) : 1.0;
     const float u = __double2float_rn(cj * su);
     const float w = __fmul_rn(beta, __fsub_rn(vs[j], u));
     const float o = __double2float_rn(cj * so + qk * (double)w);
@@ -643,7 +644,7 @@ __device__ __forceinline__ void finish_columns(const Args &a, Scratch<D> &sc, in
 // ---------------------------------------------------------------------------
 // One quantized head of width B: decode / fit-pack / fused.
 // ---------------------------------------------------------------------------
-template <int D, int B, int KIND>
+template <int D, int B, int KIND, int s16>
 __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int row, Scratch<D> &sc, int tid) {
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES;
@@ -651,8 +652,8 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
     const int g = tid / LANES, l = tid % LANES;
     const int j0 = 4 * l;
     const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
-    const float *st_r = reinterpret_cast<const float *>(stage + codes_bytes);
-    const float *st_c = st_r + D;
+    const uint8_t *st_r = stage + codes_bytes;              // staged r[D] and c[D]
+    const uint8_t *st_c = st_r + D * (s16 ? 2 : 4);
     const float *tf = reinterpret_cast<const float *>(stage + a.rec_stage_bytes);
     const float *qs = tf + kTailQ * D;
     const float *ks = tf + kTailK * D;
@@ -666,7 +667,7 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
     double bk = 0.0, bq = 0.0, bqk = 0.0;
     if ((tid & 31) < 16) {
         const int i = 16 * (tid >> 5) + (tid & 31);
-        const float ai = __fmul_rn(alpha, st_r[i]);
+        const float ai = __fmul_rn(alpha, scale_at(st_r, i, s16));
         const float ki = ks[i];
         sc.a2[i] = make_float2(ai, ai);
         sc.k2[i] = make_float2(ki, ki);
@@ -692,7 +693,7 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
     double accU[4] = {0.0, 0.0, 0.0, 0.0}, accO[4] = {0.0, 0.0, 0.0, 0.0};
     float2 cp01, cp23;
     if (KIND != kDecode) {  // c_j 2^-12 of this thread's columns (exact scaling)
-        const float4 c4 = *reinterpret_cast<const float4 *>(&st_c[j0]);
+        const float4 c4 = scale4_at(st_c, j0, s16);
         const float2 s12 = make_float2(1.0f / 4096.0f, 1.0f / 4096.0f);
         cp01 = mul2(make_float2(c4.x, c4.y), s12);
         cp23 = mul2(make_float2(c4.z, c4.w), s12);
@@ -749,7 +750,7 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
         *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0]) = make_double2(accO[0] - bQ, accO[1] - bQ);
         *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0 + 2]) = make_double2(accO[2] - bQ, accO[3] - bQ);
         __syncthreads();
-        finish_columns<D, KIND>(a, sc, tid, row, beta, vs, st_c);
+        finish_columns<D, KIND, s16>(a, sc, tid, row, beta, vs, st_c);
         if (KIND == kFused) __syncthreads();
     }
 
@@ -767,8 +768,8 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
                 S[r + rr][1] = fma2(k2, w23, S[r + rr][1]);
             }
         }
-        if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, B>(S, rec_g, sc, tid);
-        else fit_pack<D, B>(S, rec_g, sc, tid, tf + kTailRho * D, tf + kTailWbar * D);
+        if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, B, s16>(S, rec_g, sc, tid);
+        else fit_pack<D, B, s16>(S, rec_g, sc, tid, tf + kTailRho * D, tf + kTailWbar * D);
     }
 }
 
@@ -883,9 +884,9 @@ __device__ __forceinline__ uint32_t final_e_rt(float y, float ic, int b) {
 // (shared memory holding the codes block; it is copied out by the caller).
 // FP16 rows keep S_t and are stored as binary16; they take no part in the
 // column fit and carry r = 0.
-template <int D>
+template <int D, int s16>
 __device__ void fit_rows(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const uint8_t *rw, const uint32_t *roff,
-                         const float *rho, const float *wbar, uint8_t *codes, float *rec_r, float *rec_c) {
+                         const float *rho, const float *wbar, uint8_t *codes, uint8_t *rec_r, uint8_t *rec_c) {
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES, RS = Scratch<D>::RS, HALF = LANES / 2;
     const int g = tid / LANES, l = tid % LANES;
@@ -910,7 +911,7 @@ __device__ void fit_rows(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const u
         if (rw[i] != kPivotBits) {
             float m = __fmul_rn(s, 1.0f / (float)D);
             m = fmaxf(m, 1e-12f);
-            ri = __fmul_rn(m, rho[i]);
+            ri = scale_round(__fmul_rn(m, rho[i]), s16);
             inv = __frcp_rn(ri);
             bw = __fmul_rn(wbar[i], __fmul_rn(ri, ri));
         }
@@ -918,7 +919,7 @@ __device__ void fit_rows(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const u
             sc.rinv2[i] = make_float2(inv, inv);
             sc.bw2[i] = make_float2(bw, bw);
             sc.rowr[i] = ri;
-            if (rec_r) rec_r[i] = ri;
+            if (rec_r) scale_put(rec_r, i, ri, s16);
         }
     }
     __syncwarp();
@@ -1002,7 +1003,7 @@ __device__ void fit_rows(float2 (&S)[D / 8][2], Scratch<D> &sc, int tid, const u
         }
     }
     __syncthreads();
-    column_ls_fit<D>(sc, tid, rec_c);
+    column_ls_fit<D, s16>(sc, tid, rec_c);
     // 5. final codes (or binary16) of every row into the shared codes block
     {
         const float4 ic4 = *reinterpret_cast<const float4 *>(&sc.ic[j0]);
@@ -1049,15 +1050,15 @@ __device__ __forceinline__ void rows_prologue_tables(const Args &a, Scratch<D> &
 }
 
 // One head of per-row units: decode / fit-pack / fused.
-template <int D, int KIND>
+template <int D, int KIND, int s16>
 __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row, uint32_t codes_bytes,
                           Scratch<D> &sc, int tid) {
     using G = Geo<D>;
     constexpr int RT = G::RT, LANES = G::LANES;
     const int g = tid / LANES, l = tid % LANES;
     const int j0 = 4 * l;
-    const float *st_r = reinterpret_cast<const float *>(stage + codes_bytes);
-    const float *st_c = st_r + D;
+    const uint8_t *st_r = stage + codes_bytes;              // staged r[D] and c[D]
+    const uint8_t *st_c = st_r + D * (s16 ? 2 : 4);
     const float *tf = reinterpret_cast<const float *>(stage + a.rec_stage_bytes);
     const float *qs = tf + kTailQ * D;
     const float *ks = tf + kTailK * D;
@@ -1073,7 +1074,7 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
         const int i = 16 * (tid >> 5) + (tid & 31);
         const int b = rw[i];
         const float al = als[i];
-        const float ai = (b == kPivotBits) ? al : __fmul_rn(al, st_r[i]);
+        const float ai = (b == kPivotBits) ? al : __fmul_rn(al, scale_at(st_r, i, s16));
         sc.a2[i] = make_float2(ai, ai);
         sc.k2[i] = make_float2(ks[i], ks[i]);
         if (KIND != kFitPack) {
@@ -1097,7 +1098,7 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
     float2 S[RT][2];
     double accU[4] = {0.0, 0.0, 0.0, 0.0}, accO[4] = {0.0, 0.0, 0.0, 0.0};
     double accUp[4] = {0.0, 0.0, 0.0, 0.0}, accOp[4] = {0.0, 0.0, 0.0, 0.0};
-    const float4 c4 = *reinterpret_cast<const float4 *>(&st_c[j0]);
+    const float4 c4 = scale4_at(st_c, j0, s16);
     const float2 s12 = make_float2(1.0f / 4096.0f, 1.0f / 4096.0f);
     const float2 cp01 = mul2(make_float2(c4.x, c4.y), s12), cp23 = mul2(make_float2(c4.z, c4.w), s12);
 #pragma unroll
@@ -1150,7 +1151,7 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
         double pu[4], po[4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-            const double cj = (double)st_c[j0 + jj];
+            const double cj = (double)scale_at(st_c, j0 + jj, s16);
             pu[jj] = cj * (accU[jj] - bK) + accUp[jj];
             po[jj] = cj * (accO[jj] - bQ) + accOp[jj];
         }
@@ -1174,8 +1175,9 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
             S[r][1] = fma2(k2, w23, S[r][1]);
         }
         // the staged codes are no longer read: assemble the new rows there
-        float *rec_r = reinterpret_cast<float *>(rec_g + codes_bytes);
-        fit_rows<D>(S, sc, tid, rw, roff, tf + kTailRho * D, tf + kTailWbar * D, stage, rec_r, rec_r + D);
+        uint8_t *rec_r = rec_g + codes_bytes;
+        fit_rows<D, s16>(S, sc, tid, rw, roff, tf + kTailRho * D, tf + kTailWbar * D, stage, rec_r,
+                         rec_r + D * (s16 ? 2 : 4));
         copy_out<D>(rec_g, stage, codes_bytes, tid);
     }
 }
@@ -1183,7 +1185,7 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
 // ---------------------------------------------------------------------------
 // Persistent pipeline kernel.
 // ---------------------------------------------------------------------------
-template <int D, int KIND, int MODE>
+template <int D, int KIND, int MODE, int S16>
 __global__ void __launch_bounds__(2 * D, 2) k_step(Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x;
@@ -1246,13 +1248,13 @@ __global__ void __launch_bounds__(2 * D, 2) k_step(Args a) {
         if (valid) {
             const int row = sc.meta[s][6];
             if (MODE == 1) {
-                item_rows<D, KIND>(a, stage, rec_g, row, (uint32_t)sc.meta[s][3], sc, tid);
+                item_rows<D, KIND, S16>(a, stage, rec_g, row, (uint32_t)sc.meta[s][3], sc, tid);
             } else {
                 switch (width) {
-                    case 2: item_uniform<D, 2, KIND>(a, stage, rec_g, row, sc, tid); break;
-                    case 4: item_uniform<D, 4, KIND>(a, stage, rec_g, row, sc, tid); break;
-                    case 6: item_uniform<D, 6, KIND>(a, stage, rec_g, row, sc, tid); break;
-                    case 8: item_uniform<D, 8, KIND>(a, stage, rec_g, row, sc, tid); break;
+                    case 2: item_uniform<D, 2, KIND, S16>(a, stage, rec_g, row, sc, tid); break;
+                    case 4: item_uniform<D, 4, KIND, S16>(a, stage, rec_g, row, sc, tid); break;
+                    case 6: item_uniform<D, 6, KIND, S16>(a, stage, rec_g, row, sc, tid); break;
+                    case 8: item_uniform<D, 8, KIND, S16>(a, stage, rec_g, row, sc, tid); break;
                     case kPivotBits: item_pivot<D, KIND>(a, stage, rec_g, row, sc, tid); break;
                     default: if (tid == 0) flag_error(a.err, kErrArgs); break;
                 }
@@ -1295,8 +1297,9 @@ __global__ void __launch_bounds__(2 * D) k_requant_pack(Args a) {
         if (tid == 0) sc.nz = a.neg_zero;
         __syncthreads();
         const uint32_t codes_bytes = a.t.codes_bytes[gl];
-        float *rec_r = reinterpret_cast<float *>(rec + codes_bytes);
-        fit_rows<D>(S, sc, tid, sc.rw, sc.roff, sc.rho, sc.wbar, codes, rec_r, rec_r + D);
+        uint8_t *rec_r = rec + codes_bytes;
+        if (a.scale16) fit_rows<D, 1>(S, sc, tid, sc.rw, sc.roff, sc.rho, sc.wbar, codes, rec_r, rec_r + 2 * D);
+        else fit_rows<D, 0>(S, sc, tid, sc.rw, sc.roff, sc.rho, sc.wbar, codes, rec_r, rec_r + 4 * D);
         copy_out<D>(rec, codes, codes_bytes, tid);
         return;
     }
@@ -1313,40 +1316,61 @@ __global__ void __launch_bounds__(2 * D) k_requant_pack(Args a) {
     __syncthreads();
     switch (width) {
         case 2:
-            if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 2>(S, rec, sc, tid);
-            else fit_pack<D, 2>(S, rec, sc, tid, sc.rho, sc.wbar);
+            if (a.scale16) {
+                if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 2, 1>(S, rec, sc, tid);
+                else fit_pack<D, 2, 1>(S, rec, sc, tid, sc.rho, sc.wbar);
+            } else {
+                if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 2, 0>(S, rec, sc, tid);
+                else fit_pack<D, 2, 0>(S, rec, sc, tid, sc.rho, sc.wbar);
+            }
             break;
         case 4:
-            if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 4>(S, rec, sc, tid);
-            else fit_pack<D, 4>(S, rec, sc, tid, sc.rho, sc.wbar);
+            if (a.scale16) {
+                if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 4, 1>(S, rec, sc, tid);
+                else fit_pack<D, 4, 1>(S, rec, sc, tid, sc.rho, sc.wbar);
+            } else {
+                if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 4, 0>(S, rec, sc, tid);
+                else fit_pack<D, 4, 0>(S, rec, sc, tid, sc.rho, sc.wbar);
+            }
             break;
         case 6:
-            if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 6>(S, rec, sc, tid);
-            else fit_pack<D, 6>(S, rec, sc, tid, sc.rho, sc.wbar);
+            if (a.scale16) {
+                if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 6, 1>(S, rec, sc, tid);
+                else fit_pack<D, 6, 1>(S, rec, sc, tid, sc.rho, sc.wbar);
+            } else {
+                if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 6, 0>(S, rec, sc, tid);
+                else fit_pack<D, 6, 0>(S, rec, sc, tid, sc.rho, sc.wbar);
+            }
             break;
         case 8:
-            if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 8>(S, rec, sc, tid);
-            else fit_pack<D, 8>(S, rec, sc, tid, sc.rho, sc.wbar);
+            if (a.scale16) {
+                if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 8, 1>(S, rec, sc, tid);
+                else fit_pack<D, 8, 1>(S, rec, sc, tid, sc.rho, sc.wbar);
+            } else {
+                if (a.quantizer == kQuantAbsmax) fit_pack_absmax<D, 8, 0>(S, rec, sc, tid);
+                else fit_pack<D, 8, 0>(S, rec, sc, tid, sc.rho, sc.wbar);
+            }
             break;
         default: if (tid == 0) flag_error(a.err, kErrArgs); break;
     }
 }
 
 template <int D, int B>
-__device__ void unpack_uniform(const uint8_t *rec, float *out, int tid) {
+__device__ void unpack_uniform(const uint8_t *rec, float *out, int tid, int s16) {
     using G = Geo<D>;
     const int g = tid / G::LANES, l = tid % G::LANES;
     const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
-    const float *rr = reinterpret_cast<const float *>(rec + codes_bytes);
-    const float *cc = rr + D;
+    const uint8_t *rr = rec + codes_bytes;
+    const uint8_t *cc = rr + D * (s16 ? 2 : 4);
     uint32_t W[Stream<D, B>::NW];
     load_stream<D, B>(rec, tid, W);
-    const float2 c01 = make_float2(__fmul_rn(cc[4 * l], 1.0f / 4096.0f), __fmul_rn(cc[4 * l + 1], 1.0f / 4096.0f));
-    const float2 c23 = make_float2(__fmul_rn(cc[4 * l + 2], 1.0f / 4096.0f), __fmul_rn(cc[4 * l + 3], 1.0f / 4096.0f));
+    const float4 c4 = scale4_at(cc, 4 * l, s16);
+    const float2 c01 = make_float2(__fmul_rn(c4.x, 1.0f / 4096.0f), __fmul_rn(c4.y, 1.0f / 4096.0f));
+    const float2 c23 = make_float2(__fmul_rn(c4.z, 1.0f / 4096.0f), __fmul_rn(c4.w, 1.0f / 4096.0f));
 #pragma unroll
     for (int r = 0; r < G::RT; ++r) {
         const int i = g * G::RT + r;
-        const float ri = rr[i];
+        const float ri = scale_at(rr, i, s16);
         const float2 r2 = make_float2(ri, ri);
         const float2 A01 = mul2(r2, c01), A23 = mul2(r2, c23);
         const float2 z01 = make_float2(x_as_zscaled<B>(field_x<B>(W, 4 * r)), x_as_zscaled<B>(field_x<B>(W, 4 * r + 1)));
@@ -1361,10 +1385,12 @@ __device__ void unpack_rows(const Args &a, const uint8_t *rec, float *out, int g
     using G = Geo<D>;
     const int g = tid / G::LANES, l = tid % G::LANES;
     const uint32_t codes_bytes = a.t.codes_bytes[gl];
-    const float *rr = reinterpret_cast<const float *>(rec + codes_bytes);
-    const float *cc = rr + D;
-    const float2 c01 = make_float2(__fmul_rn(cc[4 * l], 1.0f / 4096.0f), __fmul_rn(cc[4 * l + 1], 1.0f / 4096.0f));
-    const float2 c23 = make_float2(__fmul_rn(cc[4 * l + 2], 1.0f / 4096.0f), __fmul_rn(cc[4 * l + 3], 1.0f / 4096.0f));
+    const int s16 = a.scale16;
+    const uint8_t *rr = rec + codes_bytes;
+    const uint8_t *cc = rr + D * (s16 ? 2 : 4);
+    const float4 c4 = scale4_at(cc, 4 * l, s16);
+    const float2 c01 = make_float2(__fmul_rn(c4.x, 1.0f / 4096.0f), __fmul_rn(c4.y, 1.0f / 4096.0f));
+    const float2 c23 = make_float2(__fmul_rn(c4.z, 1.0f / 4096.0f), __fmul_rn(c4.w, 1.0f / 4096.0f));
 #pragma unroll
     for (int r = 0; r < G::RT; ++r) {
         const int i = g * G::RT + r;
@@ -1383,7 +1409,8 @@ __device__ void unpack_rows(const Args &a, const uint8_t *rec, float *out, int g
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj)
                 z[jj] = __fsub_rn(__uint_as_float((((f >> (b * jj)) & mask) << 12) | 0x4B000000u), zb);
-            const float2 r2 = make_float2(rr[i], rr[i]);
+            const float ri = scale_at(rr, i, s16);
+            const float2 r2 = make_float2(ri, ri);
             s01 = mul2(mul2(r2, c01), make_float2(z[0], z[1]));
             s23 = mul2(mul2(r2, c23), make_float2(z[2], z[3]));
         }
@@ -1410,10 +1437,10 @@ __global__ void __launch_bounds__(2 * D) k_unpack(Args a) {
         return;
     }
     switch (a.t.width[gl]) {
-        case 2: unpack_uniform<D, 2>(rec, out, tid); break;
-        case 4: unpack_uniform<D, 4>(rec, out, tid); break;
-        case 6: unpack_uniform<D, 6>(rec, out, tid); break;
-        case 8: unpack_uniform<D, 8>(rec, out, tid); break;
+        case 2: unpack_uniform<D, 2>(rec, out, tid, a.scale16); break;
+        case 4: unpack_uniform<D, 4>(rec, out, tid, a.scale16); break;
+        case 6: unpack_uniform<D, 6>(rec, out, tid, a.scale16); break;
+        case 8: unpack_uniform<D, 8>(rec, out, tid, a.scale16); break;
         case kPivotBits: {
             float2 S[G::RT][2];
             load_pivot<D>(rec, tid, S);
@@ -1455,7 +1482,7 @@ __device__ void dist_uniform(const float *Sg, int gl, int m, int n_bits, double 
         S[r][0] = make_float2(v.x, v.y);
         S[r][1] = make_float2(v.z, v.w);
     }
-    fit_scales<D, B>(S, sc, tid, sc.rho, sc.wbar, nullptr, nullptr);
+    fit_scales<D, B, 0>(S, sc, tid, sc.rho, sc.wbar, nullptr, nullptr);
     float cc[4], icc[4];
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) { cc[jj] = sc.cold[j0 + jj]; icc[jj] = sc.ic[j0 + jj]; }
@@ -1541,7 +1568,8 @@ static size_t step_smem(uint32_t stage_bytes) {
 template <int D, int KIND>
 static cudaError_t launch_step_d(Args a, int n_sms, cudaStream_t st, int *grid_out) {
     const size_t smem = step_smem<D>(a.stage_bytes);
-    auto kern = a.mode == 1 ? k_step<D, KIND, 1> : k_step<D, KIND, 0>;
+    auto kern = a.mode == 1 ? (a.scale16 ? k_step<D, KIND, 1, 1> : k_step<D, KIND, 1, 0>)
+                            : (a.scale16 ? k_step<D, KIND, 0, 1> : k_step<D, KIND, 0, 0>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;

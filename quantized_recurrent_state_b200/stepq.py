@@ -45,7 +45,7 @@ class PlanInfo(ctypes.Structure):
         ("bitset", ctypes.c_uint32), ("nominal_bits", ctypes.c_float), ("horizon", ctypes.c_uint64),
         ("slot_bytes", ctypes.c_uint64), ("bits_per_value", ctypes.c_double),
         ("bits_per_value_s16", ctypes.c_double), ("units_by_width", ctypes.c_int * 17),
-        ("quantizer", ctypes.c_int),
+        ("quantizer", ctypes.c_int), ("scale_bits", ctypes.c_int),
     ]
 
 
@@ -70,9 +70,9 @@ def lib():
         l.stepq_plan_get_info.argtypes = [P, ctypes.POINTER(PlanInfo)]
         l.stepq_plan_widths.argtypes = [P, P]
         l.stepq_plan_record.argtypes = [P, I, I, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)]
-        l.stepq_plan_build.argtypes = [I, I, I, I, P, I, ctypes.c_float, I, ctypes.c_uint64, P, P, P,
+        l.stepq_plan_build.argtypes = [I, I, I, I, P, I, ctypes.c_float, I, ctypes.c_uint64, P, P, P, I,
                                        ctypes.c_char_p, ctypes.POINTER(P)]
-        l.stepq_plan_build_uniform.argtypes = [I, I, I, I, I, I, ctypes.c_uint64, P, ctypes.c_char_p,
+        l.stepq_plan_build_uniform.argtypes = [I, I, I, I, I, I, ctypes.c_uint64, P, I, ctypes.c_char_p,
                                                ctypes.POINTER(P)]
         l.stepq_ctx_create.argtypes = [P, P, P, I, I, ctypes.POINTER(P)]
         l.stepq_ctx_free.argtypes = [P]
@@ -135,7 +135,7 @@ class Plan:
 
     @classmethod
     def build(cls, mode, n_layers, n_heads, d, bits, nominal_bits, n_pivots, horizon,
-              lgate, dist, wbar, path=None) -> "Plan":
+              lgate, dist, wbar, path=None, scale_bits=32) -> "Plan":
         bits_a = np.ascontiguousarray(bits, dtype=np.int32)
         lg = np.ascontiguousarray(lgate, dtype=np.float64)
         di = np.ascontiguousarray(dist, dtype=np.float64)
@@ -143,17 +143,17 @@ class Plan:
         h = P()
         _check(lib().stepq_plan_build(mode, n_layers, n_heads, d, bits_a.ctypes.data, len(bits_a),
                                       float(nominal_bits), n_pivots, int(horizon), lg.ctypes.data,
-                                      di.ctypes.data, wb.ctypes.data,
+                                      di.ctypes.data, wb.ctypes.data, int(scale_bits),
                                       path.encode() if path else None, ctypes.byref(h)))
         return cls(h)
 
     @classmethod
     def build_uniform(cls, mode, n_layers, n_heads, d, bits, quantizer=QUANT_DUAL_AXIS, horizon=65536,
-                      wbar=None, path=None) -> "Plan":
+                      wbar=None, path=None, scale_bits=32) -> "Plan":
         wb = None if wbar is None else np.ascontiguousarray(wbar, dtype=np.float32)
         h = P()
         _check(lib().stepq_plan_build_uniform(mode, n_layers, n_heads, d, int(bits), int(quantizer), int(horizon),
-                                              None if wb is None else wb.ctypes.data,
+                                              None if wb is None else wb.ctypes.data, int(scale_bits),
                                               path.encode() if path else None, ctypes.byref(h)))
         return cls(h)
 

@@ -16,7 +16,7 @@ from quantized_recurrent_state_b200 import synth
 
 
 @functools.lru_cache(maxsize=None)
-def oracle_plan(name: str, n_layers: int = None, n_pivots: int = None, d: int = None):
+def oracle_plan(name: str, n_layers: int = None, n_pivots: int = None, d: int = None, scale_bits: int = 32):
     """(plan dict, plan bytes, Workload) for a workload, optionally sliced."""
     wl = synth.workloads()[name]
     if n_layers is not None or n_pivots is not None:
@@ -28,18 +28,19 @@ def oracle_plan(name: str, n_layers: int = None, n_pivots: int = None, d: int = 
     steps = [synth.step_inputs(wl, wl.calib_seed, wl.calib_req, t, alpha=alpha) for t in range(wl.calib_steps)]
     stats = model.calibrate(wl.mode, wl.d, L, wl.n_heads, S0, steps, wl.bits)
     plan = model.build_plan(wl.mode, wl.d, L, wl.n_heads, stats, wl.bits, wl.nominal_bits, wl.n_pivots,
-                            wl.horizon)
+                            wl.horizon, scale_bits=scale_bits)
     data = plan_io.write_plan(None, plan)
     return plan, data, wl, stats
 
 
 @functools.lru_cache(maxsize=None)
-def uniform_plan(name: str, bits: int, quantizer: int, n_layers: int = None):
+def uniform_plan(name: str, bits: int, quantizer: int, n_layers: int = None, scale_bits: int = 32):
     """(plan dict, plan bytes, Workload) of a baseline plan (every unit at
     `bits`, no pivots) over a workload's shape."""
     wl = synth.workloads()[name]
     wl = synth.Workload(**{**wl.__dict__, "n_layers": n_layers or wl.n_layers, "n_pivots": 0})
-    plan = model.uniform_plan(wl.mode, wl.d, wl.n_layers, wl.n_heads, bits, quantizer, wl.horizon)
+    plan = model.uniform_plan(wl.mode, wl.d, wl.n_layers, wl.n_heads, bits, quantizer, wl.horizon,
+                              scale_bits=scale_bits)
     return plan, plan_io.write_plan(None, plan), wl, None
 
 

@@ -40,11 +40,12 @@ def _inputs_to_dev(inp):
 class Run:
     """A GPU pool for a workload plus an oracle view of the same plan."""
 
-    def __init__(self, stepq, name, n_req, n_layers=None, n_pivots=None, extra_slots=3, chunk=2, uniform=None):
+    def __init__(self, stepq, name, n_req, n_layers=None, n_pivots=None, extra_slots=3, chunk=2, uniform=None,
+                 scale_bits=32):
         if uniform is None:
-            self.plan, data, self.wl, _ = oracle_plan(name, n_layers, n_pivots)
+            self.plan, data, self.wl, _ = oracle_plan(name, n_layers, n_pivots, scale_bits=scale_bits)
         else:  # (bits, quantizer): a baseline plan over the workload's shape
-            self.plan, data, self.wl, _ = uniform_plan(name, uniform[0], uniform[1], n_layers)
+            self.plan, data, self.wl, _ = uniform_plan(name, uniform[0], uniform[1], n_layers, scale_bits=scale_bits)
         self.pv = model.PlanView(self.plan)
         self.P = stepq.Plan.from_bytes(data)
         self.n_req = n_req
@@ -86,8 +87,8 @@ class Run:
 
 
 def _lockstep(stepq, name, n_req, steps, check, n_layers=None, n_pivots=None, fused=False, heads=None,
-              uniform=None):
-    run = Run(stepq, name, n_req, n_layers, n_pivots, uniform=uniform)
+              uniform=None, scale_bits=32):
+    run = Run(stepq, name, n_req, n_layers, n_pivots, uniform=uniform, scale_bits=scale_bits)
     S0 = run.pack_initial()
     pv = run.pv
     tot_codes = tot_exc = tot_bad = 0
@@ -176,6 +177,17 @@ def test_absmax_baseline_lockstep(stepq, bits, fused):
 def test_uniform_dual_axis_lockstep(stepq):
     # uniform INT8 with the STEPQuant fit (no pivots), fused
     _lockstep(stepq, "qwen_pool6", 70, 6, check=[0, 69], n_layers=2, fused=True, uniform=(8, model.QUANT_DUAL_AXIS))
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_scale16_lockstep(stepq, fused):
+    # calibrated nominal-6 plan with bfloat16 scale storage, 2-layer pool slice
+    _lockstep(stepq, "qwen_pool6", 70, 6, check=[0, 69], n_layers=2, n_pivots=2, fused=fused, scale_bits=16)
+
+
+def test_scale16_absmax_lockstep(stepq):
+    _lockstep(stepq, "qwen_pool6", 70, 4, check=[0, 69], n_layers=2, fused=True,
+              uniform=(6, model.QUANT_ABSMAX), scale_bits=16)
 
 
 def test_fused_bit_identical_to_two_stream(stepq):
@@ -340,6 +352,10 @@ def test_kda_slice_lockstep(stepq):
     # 2 layers x 32 heads x 128 key rows of the KDA pool, Lagrangian nominal
     # 6-bit plan over {4,6,8} with 16 FP16 rows, batch 8, 8 steps
     _lockstep(stepq, "kda_rows", 8, 8, check=[0, 7], n_layers=2, n_pivots=16)
+
+
+def test_kda_scale16_lockstep(stepq):
+    _lockstep(stepq, "kda_rows", 8, 4, check=[0, 7], n_layers=2, n_pivots=16, fused=True, scale_bits=16)
 
 
 def test_kda_two_stream_equals_fused(stepq):

@@ -150,15 +150,21 @@ def test_calls_without_device_fail_cleanly():
     assert rc == stepq.ECUDA
 
 
+@pytest.mark.parametrize("sbits", [32, 16])
 @pytest.mark.parametrize("mode,quant", [(0, stepq.QUANT_ABSMAX), (0, stepq.QUANT_DUAL_AXIS), (1, stepq.QUANT_DUAL_AXIS)])
-def test_uniform_plan_file_matches_oracle(tmp_path, mode, quant):
+def test_uniform_plan_file_matches_oracle(tmp_path, mode, quant, sbits):
     L, H, D = 2, 3, 16
     wbar = np.linspace(0.5, 2.0, L * H * D).astype(np.float32)
     path = str(tmp_path / "u.plan")
-    p = stepq.Plan.build_uniform(mode, L, H, D, 6, quant, 4096, wbar, path=path)
-    ora = model.uniform_plan(mode, D, L, H, 6, quant, 4096, wbar)
+    p = stepq.Plan.build_uniform(mode, L, H, D, 6, quant, 4096, wbar, path=path, scale_bits=sbits)
+    ora = model.uniform_plan(mode, D, L, H, 6, quant, 4096, wbar, scale_bits=sbits)
     assert open(path, "rb").read() == plan_io.write_plan(None, ora)
-    assert p.info.quantizer == quant and p.info.n_pivots == 0
+    assert p.info.quantizer == quant and p.info.n_pivots == 0 and p.info.scale_bits == sbits
+    offs, slot = plan_io.pool_layout(ora)
+    assert p.slot_bytes == slot
+    for l in range(L):
+        for h in range(H):
+            assert p.record(l, h)[0] == offs[l * H + h]
     assert p.info.units_by_width[6] == p.info.n_units
 
 
@@ -166,7 +172,9 @@ def test_quantizer_field_validation():
     good = bytearray(plan_io.write_plan(None, model.uniform_plan(0, 16, 2, 2, 4, model.QUANT_ABSMAX, 4096)))
     assert stepq.Plan.from_bytes(bytes(good)).info.quantizer == stepq.QUANT_ABSMAX
     bad = bytearray(good); bad[56] = 2; _expect_format_error(_recrc(bad))                        # unknown quantizer
-    bad = bytearray(good); bad[60] = 1; _expect_format_error(_recrc(bad))                        # reserved word
+    bad = bytearray(good); bad[60] = 1; _expect_format_error(_recrc(bad))                        # scale word
+    ok16 = bytearray(good); ok16[60] = 16
+    assert stepq.Plan.from_bytes(_recrc(ok16)).info.scale_bits == 16
     kda = bytearray(plan_io.write_plan(None, model.uniform_plan(1, 16, 2, 2, 4, 0, 4096)))
     kda[56] = 1; _expect_format_error(_recrc(kda))                                               # absmax needs mode 0
     with pytest.raises(stepq.StepqError) as ei:
