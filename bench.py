@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--variant", default="fused", choices=["fused", "two_stream"])
     ap.add_argument("--batch", type=int, default=None, help="requests (default: 70 GDN pool, 128 KDA)")
     ap.add_argument("--plan", type=int, default=6, choices=[4, 6], help="nominal bits of the GDN pool plan")
+    ap.add_argument("--scale-bits", type=int, default=32, choices=[32, 16],
+                    help="storage of the r and c scales in the plan (16: bfloat16)")
     ap.add_argument("--workload", default="gdn", choices=["gdn", "kda"],
                     help="gdn: 2,304-head pool; kda: 81,920 key rows (20 x 32 x 128)")
     ap.add_argument("--sweep", action="store_true", help="also time batch 1/16/70/128/256")
@@ -208,7 +210,7 @@ def profiled_traffic(variant: str):
 # product path
 # ---------------------------------------------------------------------------
 
-def product_plan(stepq, synth, wl, device):
+def product_plan(stepq, synth, wl, device, scale_bits=32):
     """Calibrate on the GPU (FP32-state recurrence + omega / log-gate /
     distortion kernels) and build the plan with the library's planner."""
     import torch
@@ -252,7 +254,7 @@ def product_plan(stepq, synth, wl, device):
     else:
         lgate, dist = lmean.reshape(-1), d.reshape(-1, len(bits))
     plan = stepq.Plan.build(wl.mode, L, H, D, bits, wl.nominal_bits, wl.n_pivots, wl.horizon,
-                            lgate, dist, wbar.reshape(-1), path=path)
+                            lgate, dist, wbar.reshape(-1), path=path, scale_bits=scale_bits)
     data = open(path, "rb").read()
     os.unlink(path)
     return plan, data
@@ -366,7 +368,7 @@ def run_product(args):
     device = torch.device("cuda", local)
     wl = workload_of(args, synth)
     n = args.batch
-    plan, plan_bytes = product_plan(stepq, synth, wl, device)
+    plan, plan_bytes = product_plan(stepq, synth, wl, device, args.scale_bits)
     L, H, D = wl.n_layers, wl.n_heads, wl.d
     ctx = stepq.Context(plan, n)
     pool = torch.zeros(n * plan.slot_bytes, dtype=torch.uint8, device=device)
@@ -507,7 +509,7 @@ def run_product(args):
                 **workload_config(wl, n, ws),
                 "variant": args.variant,
                 "bits_per_value": plan.info.bits_per_value, "bits_per_value_s16": plan.info.bits_per_value_s16,
-                "pool_bytes": n * plan.slot_bytes,
+                "scale_bits": plan.info.scale_bits, "pool_bytes": n * plan.slot_bytes,
             },
             "hbm_gbs": gbs,
             "hbm_frac": gbs / peak,

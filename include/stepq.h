@@ -116,7 +116,7 @@ typedef struct stepq_plan_info {
     float nominal_bits;  /* average-bit budget of the non-pivot units */
     uint64_t horizon;    /* H of the lifetime weight */
     uint64_t slot_bytes; /* bytes of one request's packed state */
-    double bits_per_value;       /* codes + FP16 pivots + fp32 scales */
+    double bits_per_value;       /* codes + FP16 pivots + the plan's stored scales */
     double bits_per_value_s16;   /* the same with 16-bit scale accounting */
     int units_by_width[17];      /* histogram of unit widths (index = bits) */
     int quantizer;               /* STEPQ_QUANT_DUAL_AXIS or STEPQ_QUANT_ABSMAX */

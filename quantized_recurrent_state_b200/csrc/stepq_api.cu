@@ -220,7 +220,7 @@ static int plan_parse(const uint8_t *d, size_t n, stepq_plan *p) {
         if (nonpiv_rows) scale_heads += 1;
     }
     const double values = (double)heads * D * D;
-    p->bpv = (code_bits + 32.0 * (scale_rows + D * scale_heads)) / values;
+    p->bpv = (code_bits + (double)p->scale_bits * (scale_rows + D * scale_heads)) / values;
     p->bpv16 = (code_bits + 16.0 * (scale_rows + D * scale_heads)) / values;
     return STEPQ_OK;
 }

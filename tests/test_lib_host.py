@@ -160,6 +160,8 @@ def test_uniform_plan_file_matches_oracle(tmp_path, mode, quant, sbits):
     ora = model.uniform_plan(mode, D, L, H, 6, quant, 4096, wbar, scale_bits=sbits)
     assert open(path, "rb").read() == plan_io.write_plan(None, ora)
     assert p.info.quantizer == quant and p.info.n_pivots == 0 and p.info.scale_bits == sbits
+    assert p.info.bits_per_value == pytest.approx(
+        allocator.bits_per_value(mode, L, H, D, ora["widths"], scale_bits=sbits), rel=1e-15)
     offs, slot = plan_io.pool_layout(ora)
     assert p.slot_bytes == slot
     for l in range(L):
