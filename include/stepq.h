@@ -280,6 +280,14 @@ uint64_t stepq_launch_count(const stepq_ctx *ctx);
  * 2 fused, 3 pack/unpack/fp32/calibration), writes ms[4] and launches[4]
  * (host arrays) and forgets the recorded launches. */
 int stepq_ctx_set_timing(stepq_ctx *ctx, int enable);
+/* Bounded copy waits of the step kernels.  Every wait of a kernel on its
+ * shared-memory copies gives up after `polls` polls of the barrier (0: the
+ * default, 2^22), sets the device error word (stepq_sync then returns
+ * STEPQ_EDEVICE, "copy wait gave up") and ends its block without touching
+ * the pool.  phantom_bytes (< 65536, normally 0) adds bytes that never
+ * arrive to every stage's expected count, so every wait runs out: the test
+ * of that path.  Applies to later launches of the context. */
+int stepq_ctx_set_wait_limit(stepq_ctx *ctx, uint32_t polls, uint32_t phantom_bytes);
 int stepq_kernel_stats(stepq_ctx *ctx, double *ms, uint64_t *launches);
 
 const char *stepq_last_error(void);

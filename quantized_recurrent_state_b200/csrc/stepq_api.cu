@@ -572,6 +572,7 @@ struct stepq_ctx {
     std::vector<uint32_t> layer_max_rec;  // max non-pivot record bytes per layer
     uint64_t launches = 0;
     bool timing = false;
+    uint32_t wait_polls = 1u << 22, phantom_tx = 0;
     struct Timed { int kind; cudaEvent_t a, b; };
     std::vector<Timed> timed;
     std::vector<cudaEvent_t> ev_pool;
@@ -611,6 +612,8 @@ stepq::Args base_args(stepq_ctx *c, void *pool, const int32_t *slots, int n_req,
     a.H = c->plan->H;
     a.mode = c->plan->mode;
     a.quantizer = c->plan->quantizer;
+    a.wait_polls = c->wait_polls;
+    a.phantom_tx = c->phantom_tx;
     a.scale16 = c->plan->scale_bits == 16 ? 1 : 0;
     a.n_items = n_req * (le - lb) * c->plan->H;
     a.div_nreq = stepq::div_magic((uint32_t)n_req);
@@ -912,6 +915,14 @@ extern "C" int stepq_fp32_decode_step(stepq_ctx *c, float *S_pool, const int32_t
     const cudaError_t e = stepq::launch_fp32_step(c->plan->D, a, S_pool, c->plan->L, c->main);
     if (e != cudaSuccess) return cuda_fail(e, "fp32 step launch");
     lt.done();
+    return STEPQ_OK;
+}
+
+extern "C" int stepq_ctx_set_wait_limit(stepq_ctx *c, uint32_t polls, uint32_t phantom_bytes) {
+    if (!c) return fail(STEPQ_EINVAL, "set_wait_limit: null context");
+    if (phantom_bytes >= (1u << 16)) return fail(STEPQ_EINVAL, "set_wait_limit: phantom_bytes %u", phantom_bytes);
+    c->wait_polls = polls ? polls : (1u << 22);
+    c->phantom_tx = phantom_bytes;
     return STEPQ_OK;
 }
 

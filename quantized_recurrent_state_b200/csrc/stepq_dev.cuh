@@ -61,6 +61,8 @@ struct Args {
     int *err;
     float neg_zero;          // -0.0f (a run-time value the compiler cannot fold)
     uint32_t x_bits;         // 0x4B000000, the exponent word of the X encoding, held in a register
+    uint32_t wait_polls;     // polls before a copy wait gives up (error kErrWait)
+    uint32_t phantom_tx;     // extra expected bytes per stage that never arrive (0: none; timeout test)
     uint32_t stage_bytes;    // bytes of one pipeline stage
     uint32_t rec_stage_bytes;// bytes reserved for the record in a stage
 };

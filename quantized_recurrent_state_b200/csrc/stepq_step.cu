@@ -170,7 +170,7 @@ __device__ void issue_item(const Args &a, int it, uint4 dsc, int slot, uint8_t *
     uint32_t total = rec_bytes + (KIND != kFitPack ? 3 * RB : 2 * RB);
     if (KIND != kDecode) total += 2 * RB;
     if (MODE == 1) total += 2 * RB + D;
-    mbar_arrive_expect(bar, total);
+    mbar_arrive_expect(bar, total + a.phantom_tx);
     if (rec_bytes) bulk_g2s(stage, rec, rec_bytes, bar);
     const size_t off = (size_t)row * D;
     const size_t goff = (size_t)gl * D;
@@ -1219,13 +1219,13 @@ __global__ void __launch_bounds__(2 * D, 2) k_step(Args a) {
     int s = 0;
     uint32_t phase = 0;
     for (int it = blockIdx.x; it < a.n_items; it += G) {
-        const bool ok = mbar_wait_bounded(&bars[s], phase);
+        const bool ok = mbar_wait_bounded(&bars[s], phase, a.wait_polls);
         if (__syncthreads_or(!ok)) {
             if (tid == 0) {
                 flag_error(a.err, kErrWait);
                 // let every copy still in flight land before shared memory goes away
                 cp_async_wait_all();
-                for (int k = 0; k < kStages; ++k) mbar_wait_bounded(&bars[k], phase ^ (k < s ? 1u : 0u), 1u << 20);
+                for (int k = 0; k < kStages; ++k) mbar_wait_bounded(&bars[k], phase ^ (k < s ? 1u : 0u), a.wait_polls);
             }
             return;
         }

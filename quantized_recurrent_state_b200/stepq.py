@@ -25,7 +25,7 @@ EXPORTED = [
     "stepq_decode_step_fused", "stepq_sync", "stepq_unpack", "stepq_fp32_decode_step",
     "stepq_calib_accumulate", "stepq_calib_distortion", "stepq_copy_probe",
     "stepq_launch_count", "stepq_last_error", "stepq_ctx_set_timing", "stepq_kernel_stats",
-    "stepq_decode_step_noalloc", "stepq_plan_build_uniform",
+    "stepq_decode_step_noalloc", "stepq_plan_build_uniform", "stepq_ctx_set_wait_limit",
 ]
 QUANT_DUAL_AXIS = 0  # plan requantizer: STEPQuant row/column fit
 QUANT_ABSMAX = 1     # plan requantizer: per-row absmax baseline, c = 1
@@ -91,6 +91,7 @@ def lib():
         l.stepq_launch_count.argtypes = [P]
         l.stepq_launch_count.restype = ctypes.c_uint64
         l.stepq_ctx_set_timing.argtypes = [P, I]
+        l.stepq_ctx_set_wait_limit.argtypes = [P, ctypes.c_uint32, ctypes.c_uint32]
         l.stepq_kernel_stats.argtypes = [P, P, P]
         l.stepq_decode_step_noalloc.argtypes = [P, P, P, I, I, I, P, P, P, P, P, P]
         _lib = l
@@ -251,6 +252,11 @@ class Context:
 
     def set_timing(self, on: bool):
         return _check(lib().stepq_ctx_set_timing(self._h, 1 if on else 0))
+
+    def set_wait_limit(self, polls: int = 0, phantom_bytes: int = 0):
+        """Copy-wait poll limit of later launches (0: default); phantom_bytes > 0
+        makes every wait run out (tests of the timeout path)."""
+        return _check(lib().stepq_ctx_set_wait_limit(self._h, int(polls), int(phantom_bytes)))
 
     def kernel_stats(self):
         """{kind: (total ms, launches)} of the launches timed since the last call."""

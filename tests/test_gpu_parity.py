@@ -425,3 +425,67 @@ def test_kda_full_sampled_heads(stepq):
             zo, ho, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), new_rec)
             mism = (zg != zo) | (hg != ho)
             assert not (mism & (tie == 0)).any(), (r, l, h)
+
+
+# --------------------------------------------------------------------------
+# failure detection, checkpoint / resume, write set
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fused", [True, False])
+def test_copy_wait_timeout_reports_and_recovers(stepq, fused):
+    # every stage expects 16 bytes that never arrive: each block's bounded wait
+    # runs out, the error word is set, the pool is untouched, and the context
+    # keeps working once the limit is restored
+    a = Run(stepq, "qwen_layer", 5)
+    b = Run(stepq, "qwen_layer", 5)
+    a.pack_initial()
+    b.pack_initial()
+    a.step(0, fused=fused)
+    b.step(0, fused=fused)
+    before = a.pool.clone()
+    a.ctx.set_wait_limit(4096, 16)
+    with pytest.raises(stepq.StepqError) as ei:
+        a.step(1, fused=fused)
+    assert ei.value.code == stepq.EDEVICE and "copy wait gave up" in str(ei.value)
+    assert torch.equal(a.pool, before)
+    a.ctx.set_wait_limit(0, 0)
+    for t in range(1, 4):
+        _, oa = a.step(t, fused=fused)
+        _, ob = b.step(t, fused=fused)
+        assert np.array_equal(oa, ob)
+    assert torch.equal(a.pool, b.pool)
+
+
+def test_checkpoint_resume_bit_identical(stepq):
+    # snapshot the pool to the host mid-run, continue, restore, continue again
+    run = Run(stepq, "qwen_pool6", 7, n_layers=2, n_pivots=2)
+    run.pack_initial()
+    for t in range(3):
+        run.step(t, fused=True)
+    snap = run.pool.cpu().clone()
+    outs = [run.step(t, fused=True)[1] for t in range(3, 6)]
+    after = run.pool.clone()
+    run.pool.copy_(snap.cuda())
+    outs2 = [run.step(t, fused=True)[1] for t in range(3, 6)]
+    assert torch.equal(run.pool, after)
+    for x, y in zip(outs, outs2):
+        assert np.array_equal(x, y)
+
+
+@pytest.mark.parametrize("fused", [True, False])
+def test_write_set_canaries(stepq, fused):
+    # the pool sits between canary pages; slots outside the batch stay as they were
+    run = Run(stepq, "qwen_pool6", 4, n_layers=2, n_pivots=2, extra_slots=3)
+    G = 1 << 16
+    buf = torch.full((run.pool.numel() + 2 * G,), 0xA5, dtype=torch.uint8, device="cuda")
+    run.pool = buf[G:G + run.pool.numel()]
+    run.pool.zero_()
+    run.pack_initial()
+    idle = [s for s in range(run.n_slots) if s not in set(run.slots.tolist())]
+    sb = run.P.slot_bytes
+    idle_before = {s: run.pool[s * sb:(s + 1) * sb].clone() for s in idle}
+    for t in range(3):
+        run.step(t, fused=fused)
+    assert bool((buf[:G] == 0xA5).all()) and bool((buf[-G:] == 0xA5).all())
+    for s in idle:
+        assert torch.equal(run.pool[s * sb:(s + 1) * sb], idle_before[s])
