@@ -185,7 +185,7 @@ class Workload:
 
 
 def workloads():
-    """The five workload families (sizes as named; batch sizes are arguments)."""
+    """The workload families (sizes as named; batch sizes are arguments)."""
     return {
         "tiny_gdn": Workload("tiny_gdn", 0, 1, 4, 16, 1, 32, (2, 4, 6), 4.0, 1, (2.0, 500.0), 1001, 2001),
         "qwen_layer": Workload("qwen_layer", 0, 1, 48, 128, 64, 256, (4, 6, 8), 6.0, 1, (4.0, 20000.0),
@@ -198,6 +198,10 @@ def workloads():
                              1004, 2004, calib_req=1),
         "drift": Workload("drift", 0, 1, 8, 128, 4, 8192, (4, 6, 8), 6.0, 0, (1000.0, 20000.0),
                           1005, 2005, calib_req=2),
+        # head dimensions between the tiny and the Qwen-like cases (parity coverage of every
+        # compiled d): 2 layers x 8 heads, widths {2,4,6,8}, nominal 5, one pivot head
+        "gdn_d32": Workload("gdn_d32", 0, 2, 8, 32, 6, 16, (2, 4, 6, 8), 5.0, 1, (2.0, 2000.0), 1006, 2006),
+        "gdn_d64": Workload("gdn_d64", 0, 2, 8, 64, 6, 16, (2, 4, 6, 8), 5.0, 1, (2.0, 2000.0), 1007, 2007),
     }
 
 

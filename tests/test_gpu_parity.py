@@ -190,6 +190,18 @@ def test_scale16_absmax_lockstep(stepq):
               uniform=(6, model.QUANT_ABSMAX), scale_bits=16)
 
 
+@pytest.mark.parametrize("name", ["gdn_d32", "gdn_d64"])
+@pytest.mark.parametrize("fused", [False, True])
+def test_mid_head_dims_lockstep(stepq, name, fused):
+    # d = 32 and 64: every request checked, 8 steps, both step variants
+    _lockstep(stepq, name, 6, 8, check=list(range(6)), fused=fused)
+
+
+@pytest.mark.parametrize("name", ["gdn_d32", "gdn_d64"])
+def test_mid_head_dims_absmax_scale16(stepq, name):
+    _lockstep(stepq, name, 6, 4, check=[0, 5], fused=True, uniform=(4, model.QUANT_ABSMAX), scale_bits=16)
+
+
 def test_fused_bit_identical_to_two_stream(stepq):
     a = Run(stepq, "qwen_layer", 9)
     b = Run(stepq, "qwen_layer", 9)
