@@ -444,27 +444,49 @@ def run_product(args):
     # end to end through the C ABI with host buffers
     e2e = None
     if not args.no_e2e:
+        # Every step: its q, k, v, alpha, beta copied from pinned host memory, the step, and
+        # o copied back to pinned host memory.  Two input/output buffer sets and two copy
+        # streams let step i's upload and step i-1's download overlap step i-1's kernels.
+        NB = 2
         host = {k: v.cpu().pin_memory() for k, v in sets[0].items()}
-        dev_in = {k: torch.empty_like(v) for k, v in sets[0].items()}
-        o_host = torch.empty(o.shape, dtype=torch.float32).pin_memory()
+        dev_in = [{k: torch.empty_like(v) for k, v in sets[0].items()} for _ in range(NB)]
+        o_dev = [torch.empty_like(o) for _ in range(NB)]
+        o_host = [torch.empty(o.shape, dtype=torch.float32).pin_memory() for _ in range(NB)]
+        up, down = torch.cuda.Stream(), torch.cuda.Stream()
+        ev_in = [torch.cuda.Event() for _ in range(NB)]
+        ev_done = [torch.cuda.Event() for _ in range(NB)]
+        ev_out = [torch.cuda.Event() for _ in range(NB)]
         h2d = sum(v.numel() * 4 for v in host.values())
-        d2h = o_host.numel() * 4
+        d2h = o_host[0].numel() * 4
         k_e2e = min(args.steps, 16)
         torch.cuda.synchronize()
         barrier(ws)
         t0 = time.perf_counter()
-        with torch.cuda.stream(ctx.main):
-            for i in range(k_e2e):
+        for i in range(k_e2e):
+            bi = i % NB
+            with torch.cuda.stream(up):
+                if i >= NB:
+                    up.wait_event(ev_done[bi])  # step i-NB no longer reads these inputs
                 for kk in host:
-                    dev_in[kk].copy_(host[kk], non_blocking=True)
-                run_step(ctx, args.variant, pool, slots, n, L, dev_in, o, wsp)
+                    dev_in[bi][kk].copy_(host[kk], non_blocking=True)
+                ev_in[bi].record(up)
+            with torch.cuda.stream(ctx.main):
+                ctx.main.wait_event(ev_in[bi])
+                if i >= NB:
+                    ctx.main.wait_event(ev_out[bi])  # o of step i-NB is on the host
+                run_step(ctx, args.variant, pool, slots, n, L, dev_in[bi], o_dev[bi], wsp)
                 ctx.main.wait_stream(ctx.side)
-                o_host.copy_(o, non_blocking=True)
+                ev_done[bi].record(ctx.main)
+            with torch.cuda.stream(down):
+                down.wait_event(ev_done[bi])
+                o_host[bi].copy_(o_dev[bi], non_blocking=True)
+                ev_out[bi].record(down)
         ctx.sync()
         torch.cuda.synchronize()
         t_e2e = max_over_ranks(time.perf_counter() - t0, ws)
         e2e = {"value": sum_over_ranks(n * L * H * k_e2e, ws) / t_e2e, "unit": "head-steps/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e,
+               "overlap": "uploads and downloads on two copy streams, double-buffered, overlap the steps"}
 
     sweep = None
     if args.sweep and rank == 0:
