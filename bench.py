@@ -190,20 +190,28 @@ def kernel_hash():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(variant: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source (else None)."""
+def profiled_counts(variant: str):
+    """(DRAM bytes, warp-instructions) per full launch from the committed ncu
+    summary, each None unless it was taken on the current kernel source."""
     f = os.path.join(ROOT, "profiles", f"{variant}_kernel_traffic.txt")
     try:
         kv = dict(line.split(":", 1) for line in open(f) if ":" in line and not line.startswith("#"))
     except OSError:
-        return None
+        return None, None
     if kv.get("kernel_hash", "").strip() != kernel_hash():
-        return None
-    try:
-        return float(kv["dram_bytes_per_full_launch"])
-    except (KeyError, ValueError):
-        return None
+        return None, None
+
+    def num(key):
+        try:
+            return float(kv[key])
+        except (KeyError, ValueError):
+            return None
+    return num("dram_bytes_per_full_launch"), num("warp_instructions_per_full_launch")
+
+
+# SM issue peak: 4 schedulers per SM, one warp-instruction each per clock
+def issue_peak(n_sms: int, mhz: float) -> float:
+    return 4.0 * n_sms * mhz * 1e6
 
 
 # ---------------------------------------------------------------------------
@@ -357,6 +365,13 @@ def workload_config(wl, n, ws):
             "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"}
 
 
+def variant_is_full_launch(args) -> bool:
+    """The committed instruction count is for the default full launch (fused,
+    GDN pool, batch 70, nominal 6, fp32 scales)."""
+    return (args.variant == "fused" and args.workload == "gdn" and args.batch == 70 and args.plan == 6
+            and args.scale_bits == 32)
+
+
 def run_product(args):
     import torch
     from quantized_recurrent_state_b200 import build as qbuild
@@ -397,7 +412,7 @@ def run_product(args):
     # algorithmic bytes of one launch: the kernel's bytes per step over its launches per step
     k_bytes = kernel_bytes(plan, n, kind) / (k_n / args.steps) if k_n else None
     achieved = k_bytes / (k_ms / k_n / 1e3) / 1e9 if k_n else None
-    traffic = profiled_traffic(args.variant)
+    traffic, winst = profiled_counts(args.variant) if variant_is_full_launch(args) else (None, None)
 
     extra = {}
     # FP32-state reference kernel: same workload, fp32 state pool
@@ -514,6 +529,14 @@ def run_product(args):
 
     if rank == 0:
         csum = clocks.summary()
+        issue_view = None
+        if winst and k_n and variant_is_full_launch(args):
+            n_sms = torch.cuda.get_device_properties(device).multi_processor_count
+            ach = winst / (k_ms / k_n * 1e-3)
+            pk = issue_peak(n_sms, csum["sm_mhz"] or csum["sm_max_mhz"])
+            issue_view = {"achieved": ach, "peak": pk, "unit": "warp-inst/s", "frac": ach / pk,
+                          "instructions_per_launch": winst,
+                          "note": "what binds the kernel: instruction issue (4 per SM per clock at the sampled clock)"}
         out = {
             "metric": METRIC,
             "value": value,
@@ -539,7 +562,8 @@ def run_product(args):
             "roofline": {"bound": "hbm", "kernel": kind, "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak if achieved else None, "traffic": traffic,
                          "algorithmic_bytes_per_launch": k_bytes, "launch_ms": k_ms / k_n if k_n else None,
-                         "peak_source": peak_kind},
+                         "peak_source": peak_kind,
+                         "issue": issue_view},
             "kernel_ms": {k: v[0] for k, v in stats.items() if v[1]},
             "kernel_launches": {k: v[1] for k, v in stats.items() if v[1]},
             "gpu_launches": launches,
