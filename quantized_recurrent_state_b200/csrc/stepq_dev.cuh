@@ -187,9 +187,9 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 // ---------------------------------------------------------------------------
 // Packed fields.  A b-bit code z is stored as u = z + 2^(b-1).  The value
 //   X = 0x4B000000 | (u << 12)
-// is at once the fp32 number 2^23 + u 2^12 (so z 2^12 = X - (2^23 + off 2^12)
-// exactly) and, as the high word of an fp64 with a zero low word, the number
-// 2^177 + 2^169 u (so sum_i kap_i 2^-169 X_i = sum_i kap_i (256 + u_i)).
+// is the fp32 number 2^23 + u 2^12, so z 2^12 = X - (2^23 + off 2^12) exactly
+// (one subtraction); that fp32 value, widened to fp64, is the operand of the
+// fp64 projections (products with k_i a_i 2^-12 are exact).
 // ---------------------------------------------------------------------------
 
 template <int B>
@@ -206,7 +206,6 @@ __device__ __forceinline__ uint32_t field_x(const uint32_t *W, int p, uint32_t x
     return (x & (((1u << B) - 1u) << 12)) | xbits;
 }
 
-__device__ __forceinline__ double x_as_f64(uint32_t X) { return __hiloint2double((int)X, 0); }
 
 template <int B>
 __device__ __forceinline__ float x_as_zscaled(uint32_t X) {

@@ -26,7 +26,6 @@ enum Kind { kDecode = 0, kFitPack = 1, kFused = 2 };
 
 constexpr int kStages = 2;  // one item in flight while the other is worked on
 constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: fl(x + kMagic) - kMagic = rint(x), |x| < 2^22
-constexpr double kTwoM169 = 1.0 / 748288838313422294120286634350736906063837462003712.0;  // 2^-169
 
 template <int D>
 struct Geo {
@@ -62,8 +61,8 @@ struct __align__(16) Scratch {
     float pf1[8][D];
     float2 a2[D];     // (a_i, a_i), a_i = fl(alpha_i r_i)
     float2 k2[D];     // (k_i, k_i)
-    double kap[D];    // k_i a_i 2^-169   (pivot: k_i alpha_i)
-    double qt[D];     // q_i a_i 2^-169   (pivot: q_i alpha_i)
+    double kap[D];    // k_i a_i 2^-12   (FP16 rows and heads: k_i alpha_i)
+    double qt[D];     // q_i a_i 2^-12   (FP16 rows and heads: q_i alpha_i)
     float rho[D];     // (requant and calibration kernels; the step reads them from the stage)
     float wbar[D];
     float2 rinv2[D];  // (fl(1/r_i), fl(1/r_i)) of the refit
@@ -75,9 +74,7 @@ struct __align__(16) Scratch {
     float c0[D];
     float ic[D];
     float colmax[D];
-    double bandK[8];  // per band: sum_i k_i a_i (256 + off), sum_i q_i a_i (256 + off), sum_i q_i k_i
-    double bandQ[8];
-    double bandQK[8];
+    double bandQK[8];  // per band: sum_i q_i k_i
     uint4 dring[2];    // prefetched item descriptors (thread 0)
     int dslot[2];
     int meta[kStages][8];  // slot, width, valid, codes bytes, record address lo, hi
@@ -597,25 +594,16 @@ __device__ __forceinline__ void load_pivot(const uint8_t *rec, int tid, float2 (
     }
 }
 
-// Per-band fp64 sums of three per-row values.  Warp w holds rows
-// [16 w, 16 w + 16): lane L < 16 carries row 16 w + L (lanes 16..31 carry
-// zeros); a band is RT consecutive rows, so the butterfly over RT lanes
-// stays inside the warp.
+// Per-band fp64 sums of sum_i q_i k_i.  Warp w holds rows [16 w, 16 w + 16):
+// lane L < 16 carries row 16 w + L (lanes 16..31 carry zeros); a band is RT
+// consecutive rows, so the butterfly over RT lanes stays inside the warp.
 template <int D>
-__device__ __forceinline__ void band_sums(Scratch<D> &sc, int tid, double x0, double x1, double x2) {
+__device__ __forceinline__ void band_sums(Scratch<D> &sc, int tid, double x2) {
     constexpr int RT = D / 8;
 #pragma unroll
-    for (int m = 1; m < RT; m <<= 1) {
-        x0 += __shfl_xor_sync(0xffffffffu, x0, m);
-        x1 += __shfl_xor_sync(0xffffffffu, x1, m);
-        x2 += __shfl_xor_sync(0xffffffffu, x2, m);
-    }
+    for (int m = 1; m < RT; m <<= 1) x2 += __shfl_xor_sync(0xffffffffu, x2, m);
     const int lane = tid & 31, i = 16 * (tid >> 5) + lane;
-    if (lane < 16 && (lane % RT) == 0) {
-        sc.bandK[i / RT] = x0;
-        sc.bandQ[i / RT] = x1;
-        sc.bandQK[i / RT] = x2;
-    }
+    if (lane < 16 && (lane % RT) == 0) sc.bandQK[i / RT] = x2;
 }
 
 // Column phase of the decode: u, w, o of column j from the band partials
@@ -664,7 +652,7 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
     const float beta = ab[1];
 
     // per-row parameters of this warp's 16 rows (only this warp reads them)
-    double bk = 0.0, bq = 0.0, bqk = 0.0;
+    double bqk = 0.0;
     if ((tid & 31) < 16) {
         const int i = 16 * (tid >> 5) + (tid & 31);
         const float ai = __fmul_rn(alpha, scale_at(st_r, i, s16));
@@ -672,16 +660,13 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
         sc.a2[i] = make_float2(ai, ai);
         sc.k2[i] = make_float2(ki, ki);
         if (KIND != kFitPack) {
-            const double ka = (double)ks[i] * (double)ai;
-            const double qa = (double)qs[i] * (double)ai;
-            sc.kap[i] = ka * kTwoM169;
-            sc.qt[i] = qa * kTwoM169;
-            bk = ka * (double)(256 + OFF);
-            bq = qa * (double)(256 + OFF);
+            // k_i a_i and q_i a_i (exact in fp64) times 2^-12: the fp64 operand below is z 2^12
+            sc.kap[i] = (double)ks[i] * (double)ai * (1.0 / 4096.0);
+            sc.qt[i] = (double)qs[i] * (double)ai * (1.0 / 4096.0);
             bqk = (double)qs[i] * (double)ks[i];
         }
     }
-    if (KIND != kFitPack) band_sums<D>(sc, tid, bk, bq, bqk);
+    if (KIND != kFitPack) band_sums<D>(sc, tid, bqk);
     __syncwarp();
 
     uint32_t W[Stream<D, B>::NW];
@@ -723,19 +708,21 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
             uint32_t X[4];
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) X[jj] = field_x<B>(W, 4 * (r + rr) + jj, xb);
+            // z 2^12, exact in fp32
+            const float2 z01 = add2(make_float2(__uint_as_float(X[0]), __uint_as_float(X[1])), nzb);
+            const float2 z23 = add2(make_float2(__uint_as_float(X[2]), __uint_as_float(X[3])), nzb);
             if (KIND != kFitPack) {
+                // u and o partials: sums of the exact products (k_i a_i 2^-12) (z_ij 2^12) in fp64
                 const double kap = rr ? kap2.y : kap2.x, qt = rr ? qt2.y : qt2.x;
+                const double d[4] = {(double)z01.x, (double)z01.y, (double)z23.x, (double)z23.y};
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    const double d = x_as_f64(X[jj]);
-                    accU[jj] = fma(kap, d, accU[jj]);
-                    accO[jj] = fma(qt, d, accO[jj]);
+                    accU[jj] = fma(kap, d[jj], accU[jj]);
+                    accO[jj] = fma(qt, d[jj], accO[jj]);
                 }
             }
             if (KIND != kDecode) {
                 const float2 a2 = rr ? make_float2(a4.z, a4.w) : make_float2(a4.x, a4.y);
-                const float2 z01 = add2(make_float2(__uint_as_float(X[0]), __uint_as_float(X[1])), nzb);
-                const float2 z23 = add2(make_float2(__uint_as_float(X[2]), __uint_as_float(X[3])), nzb);
                 S[r + rr][0] = mul2(mul2(a2, cp01), z01);
                 S[r + rr][1] = mul2(mul2(a2, cp23), z23);
             }
@@ -743,12 +730,11 @@ __device__ void item_uniform(const Args &a, uint8_t *stage, uint8_t *rec_g, int 
     }
 
     if (KIND != kFitPack) {
-        // remove this band's offset-binary bias, then hand the partials over
-        const double bK = sc.bandK[g], bQ = sc.bandQ[g];
-        *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0]) = make_double2(accU[0] - bK, accU[1] - bK);
-        *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0 + 2]) = make_double2(accU[2] - bK, accU[3] - bK);
-        *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0]) = make_double2(accO[0] - bQ, accO[1] - bQ);
-        *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0 + 2]) = make_double2(accO[2] - bQ, accO[3] - bQ);
+        // hand this band's partials over
+        *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0]) = make_double2(accU[0], accU[1]);
+        *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0 + 2]) = make_double2(accU[2], accU[3]);
+        *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0]) = make_double2(accO[0], accO[1]);
+        *reinterpret_cast<double2 *>(&sc.u.col.pO[g][j0 + 2]) = make_double2(accO[2], accO[3]);
         __syncthreads();
         finish_columns<D, KIND, s16>(a, sc, tid, row, beta, vs, st_c);
         if (KIND == kFused) __syncthreads();
@@ -798,7 +784,7 @@ __device__ void item_pivot(const Args &a, uint8_t *stage, uint8_t *rec_g, int ro
             bqk = (double)qs[i] * (double)ks[i];
         }
     }
-    if (KIND != kFitPack) band_sums<D>(sc, tid, 0.0, 0.0, bqk);
+    if (KIND != kFitPack) band_sums<D>(sc, tid, bqk);
     __syncwarp();
     float2 S[RT][2];
     load_pivot<D>(rec_g, tid, S);
@@ -1069,7 +1055,7 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
     const uint8_t *rw = reinterpret_cast<const uint8_t *>(tf + kTailRw * D);
     const float beta = (tf + kTailRw * D + D / 4)[1];
 
-    double bk = 0.0, bq = 0.0, bqk = 0.0;
+    double bqk = 0.0;
     if ((tid & 31) < 16) {  // this warp's 16 rows
         const int i = 16 * (tid >> 5) + (tid & 31);
         const int b = rw[i];
@@ -1080,19 +1066,14 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
         if (KIND != kFitPack) {
             const double ka = (double)ks[i] * (double)ai;
             const double qa = (double)qs[i] * (double)ai;
-            if (b == kPivotBits) {
-                sc.kap[i] = ka;
-                sc.qt[i] = qa;
-            } else {
-                sc.kap[i] = ka * kTwoM169;
-                sc.qt[i] = qa * kTwoM169;
-                bk = ka * (double)(256 + (1 << (b - 1)));
-                bq = qa * (double)(256 + (1 << (b - 1)));
-            }
+            // quantized rows: times 2^-12, the fp64 operand below being z 2^12
+            const double sk = (b == kPivotBits) ? 1.0 : 1.0 / 4096.0;
+            sc.kap[i] = ka * sk;
+            sc.qt[i] = qa * sk;
             bqk = (double)qs[i] * (double)ks[i];
         }
     }
-    if (KIND != kFitPack) band_sums<D>(sc, tid, bk, bq, bqk);
+    if (KIND != kFitPack) band_sums<D>(sc, tid, bqk);
     __syncwarp();
 
     float2 S[RT][2];
@@ -1128,18 +1109,18 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
             uint32_t X[4];
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) X[jj] = (((f >> (b * jj)) & mask) << 12) | 0x4B000000u;
-            if (KIND != kFitPack) {
-                const double kap = sc.kap[i], qt = sc.qt[i];
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const double d = x_as_f64(X[jj]);
-                    accU[jj] = fma(kap, d, accU[jj]);
-                    accO[jj] = fma(qt, d, accO[jj]);
-                }
-            }
             const float2 nzb = make_float2(-zb, -zb);
             const float2 z01 = add2(make_float2(__uint_as_float(X[0]), __uint_as_float(X[1])), nzb);
             const float2 z23 = add2(make_float2(__uint_as_float(X[2]), __uint_as_float(X[3])), nzb);
+            if (KIND != kFitPack) {
+                const double kap = sc.kap[i], qt = sc.qt[i];
+                const double d[4] = {(double)z01.x, (double)z01.y, (double)z23.x, (double)z23.y};
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    accU[jj] = fma(kap, d[jj], accU[jj]);
+                    accO[jj] = fma(qt, d[jj], accO[jj]);
+                }
+            }
             S[r][0] = mul2(mul2(a2, cp01), z01);
             S[r][1] = mul2(mul2(a2, cp23), z23);
         }
@@ -1147,13 +1128,12 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
 
     if (KIND != kFitPack) {
         // quantized rows carry c_j; FP16 rows do not: scale the band partial here
-        const double bK = sc.bandK[g], bQ = sc.bandQ[g];
         double pu[4], po[4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
             const double cj = (double)scale_at(st_c, j0 + jj, s16);
-            pu[jj] = cj * (accU[jj] - bK) + accUp[jj];
-            po[jj] = cj * (accO[jj] - bQ) + accOp[jj];
+            pu[jj] = cj * accU[jj] + accUp[jj];
+            po[jj] = cj * accO[jj] + accOp[jj];
         }
         *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0]) = make_double2(pu[0], pu[1]);
         *reinterpret_cast<double2 *>(&sc.u.col.pU[g][j0 + 2]) = make_double2(pu[2], pu[3]);
