@@ -213,28 +213,10 @@ __device__ __forceinline__ float x_as_zscaled(uint32_t X) {
     return __fsub_rn(__uint_as_float(X), 8388608.0f + (float)(1 << (B - 1)) * 4096.0f);
 }
 
-// OR a B-bit field into stream position p of W (W zero-initialised).
-template <int B>
-__device__ __forceinline__ void field_put(uint32_t *W, int p, uint32_t u) {
-    const int bit = p * B;
-    const int w = bit >> 5;
-    const int s = bit & 31;
-    W[w] |= u << s;
-    if (s + B > 32) W[w + 1] |= u >> (32 - s);
-}
-
 // ---------------------------------------------------------------------------
-// Reductions: butterfly over `lanes` consecutive lanes.  Adding the partner's
-// value in xor order reproduces the balanced pairwise tree over lane order,
-// and a + b == b + a makes every lane hold the identical root.
+// Reduction: butterfly over LANES consecutive lanes (every lane ends with the
+// same fp64 sum).
 // ---------------------------------------------------------------------------
-
-template <int LANES>
-__device__ __forceinline__ float lane_pairwise_sum(float v) {
-#pragma unroll
-    for (int m = 1; m < LANES; m <<= 1) v = v + __shfl_xor_sync(0xffffffffu, v, m);
-    return v;
-}
 
 template <int LANES>
 __device__ __forceinline__ double lane_sum_f64(double v) {

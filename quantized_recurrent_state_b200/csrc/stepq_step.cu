@@ -73,7 +73,6 @@ struct __align__(16) Scratch {
     float ic0[D];
     float c0[D];
     float ic[D];
-    float colmax[D];
     double bandQK[8];  // per band: sum_i q_i k_i
     uint4 dring[2];    // prefetched item descriptors (thread 0)
     int dslot[2];
