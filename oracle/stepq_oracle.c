@@ -14,7 +14,7 @@
  * "方法-4 每个 decode step 的执行路径" (reconstruct -> retention + delta +
  * readout -> refit r, c -> pack).  The update formula, the quantizer formulas
  * and the numeric precision are not printed on the pages; the readings used
- * here are stated beside each function and listed in the design doc.
+ * here are stated beside each function.
  *
  * Build: gcc -O2 -ffp-contract=off -fno-fast-math -shared -fPIC
  * (no contraction: every fp32 operation below rounds exactly where written).
@@ -257,7 +257,8 @@ float sq_pairwise_sum(const float *x, int n)
 /*     which equal w r z0 S and w r^2 z0^2 up to the common factor 1/r;       */
 /*     rows of 16-bit (pivot) width contribute 0; a zero denominator keeps c0; */
 /*   - c_j is rounded to fp32 before the final codes are taken.               */
-/*   - 16-bit scale storage (scale_bits = 16, survey row f1): r_i is rounded  */
+/*   - 16-bit scale storage (scale_bits = 16, the pages' 16-bit scale        */
+/*     accounting, 局限): r_i is rounded                                      */
 /*     to bfloat16 (RNE) as soon as it is formed and that value is used      */
 /*     everywhere after (1/r, b_i, the record); c_j likewise after the        */
 /*     refinement, before the final codes.  sq_quantize = scale_bits 32.      */
