@@ -21,6 +21,8 @@
 #include <thread>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/stepq.h"
 #include "stepq_dev.cuh"
 
@@ -82,6 +84,14 @@ T rd(const uint8_t *p) {
 // ---------------------------------------------------------------------------
 // plan
 // ---------------------------------------------------------------------------
+
+// NVTX range around a public call (a no-op unless a profiler is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 struct stepq_plan {
     int mode = 0, L = 0, H = 0, D = 0, n_units = 0, n_pivots = 0;
@@ -802,6 +812,7 @@ extern "C" uint64_t stepq_launch_count(const stepq_ctx *c) { return c ? c->launc
 
 extern "C" int stepq_requant_pack(stepq_ctx *c, void *pool, const int32_t *slots, int n_req, int lb, int le,
                                   const float *S) {
+    NvtxRange nvtx_range("stepq_requant_pack");
     int rc = check_range(c, n_req, lb, le);
     if (rc) return rc;
     if ((rc = check_ptr(pool, 128, "pool")) || (rc = check_ptr(slots, 4, "slots")) || (rc = check_ptr(S, 16, "S"))) return rc;
@@ -818,6 +829,7 @@ extern "C" int stepq_requant_pack(stepq_ctx *c, void *pool, const int32_t *slots
 }
 
 extern "C" int stepq_unpack(stepq_ctx *c, const void *pool, const int32_t *slots, int n_req, int lb, int le, float *S) {
+    NvtxRange nvtx_range("stepq_unpack");
     int rc = check_range(c, n_req, lb, le);
     if (rc) return rc;
     if ((rc = check_ptr(pool, 128, "pool")) || (rc = check_ptr(slots, 4, "slots")) || (rc = check_ptr(S, 16, "S"))) return rc;
@@ -847,6 +859,7 @@ static int check_step_io(stepq_ctx *c, void *pool, const int32_t *slots, const f
 extern "C" int stepq_decode_step(stepq_ctx *c, void *pool, const int32_t *slots, int n_req, int lb, int le,
                                  const float *q, const float *k, const float *v, const float *alpha,
                                  const float *beta, float *o, void *workspace) {
+    NvtxRange nvtx_range("stepq_decode_step");
     int rc = check_range(c, n_req, lb, le);
     if (rc) return rc;
     if ((rc = check_step_io(c, pool, slots, q, k, v, alpha, beta, o))) return rc;
@@ -882,6 +895,7 @@ extern "C" int stepq_decode_step(stepq_ctx *c, void *pool, const int32_t *slots,
 extern "C" int stepq_decode_step_fused(stepq_ctx *c, void *pool, const int32_t *slots, int n_req, int lb, int le,
                                        const float *q, const float *k, const float *v, const float *alpha,
                                        const float *beta, float *o) {
+    NvtxRange nvtx_range("stepq_decode_step_fused");
     int rc = check_range(c, n_req, lb, le);
     if (rc) return rc;
     if ((rc = check_step_io(c, pool, slots, q, k, v, alpha, beta, o))) return rc;
@@ -901,6 +915,7 @@ extern "C" int stepq_decode_step_fused(stepq_ctx *c, void *pool, const int32_t *
 extern "C" int stepq_fp32_decode_step(stepq_ctx *c, float *S_pool, const int32_t *slots, int n_req, int lb, int le,
                                       const float *q, const float *k, const float *v, const float *alpha,
                                       const float *beta, float *o) {
+    NvtxRange nvtx_range("stepq_fp32_decode_step");
     int rc = check_range(c, n_req, lb, le);
     if (rc) return rc;
     if ((rc = check_ptr(S_pool, 16, "S_pool")) || (rc = check_ptr(slots, 4, "slots")) || (rc = check_ptr(q, 16, "q")) ||
@@ -1065,6 +1080,7 @@ int noalloc_scratch(int dev, float **out) {
 extern "C" int stepq_decode_step_noalloc(stepq_ctx *c, void *pool, const int32_t *slots, int n_req, int lb, int le,
                                          const float *q, const float *k, const float *v, const float *alpha,
                                          const float *beta, float *o) {
+    NvtxRange nvtx_range("stepq_decode_step_noalloc");
     int rc = check_range(c, n_req, lb, le);
     if (rc) return rc;
     if ((rc = check_step_io(c, pool, slots, q, k, v, alpha, beta, o))) return rc;
