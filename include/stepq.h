@@ -64,7 +64,10 @@
  *   - q, k, v, o, workspace: [n_req][n_layers_launched][n_heads][D] fp32.
  *     alpha: mode 0 [n_req][nL][n_heads], mode 1 [n_req][nL][n_heads][D].
  *     beta: [n_req][nL][n_heads].  S (fp32 states): [n_req][nL][n_heads][D][D].
- *     slots: device int32[n_req], each in [0, n_slots).
+ *     slots: device int32[n_req], each in [0, n_slots) (a slot outside it sets
+ *     the device error word and its records are skipped); the slots of one
+ *     call must be distinct: two requests on one slot would update the same
+ *     records concurrently (not checked, the array lives on the device).
  *   - Calls are asynchronous on the context's streams, except stepq_sync,
  *     the plan functions and stepq_last_error.
  *   - Return 0 (STEPQ_OK) or a negative STEPQ_E* code; stepq_last_error()
