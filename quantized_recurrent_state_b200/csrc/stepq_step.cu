@@ -1078,6 +1078,7 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
     float2 S[RT][2];
     double accU[4] = {0.0, 0.0, 0.0, 0.0}, accO[4] = {0.0, 0.0, 0.0, 0.0};
     double accUp[4] = {0.0, 0.0, 0.0, 0.0}, accOp[4] = {0.0, 0.0, 0.0, 0.0};
+    const uint32_t xb = a.x_bits;
     const float4 c4 = scale4_at(st_c, j0, s16);
     const float2 s12 = make_float2(1.0f / 4096.0f, 1.0f / 4096.0f);
     const float2 cp01 = mul2(make_float2(c4.x, c4.y), s12), cp23 = mul2(make_float2(c4.z, c4.w), s12);
@@ -1103,11 +1104,14 @@ __device__ void item_rows(const Args &a, uint8_t *stage, uint8_t *rec_g, int row
             S[r][1] = mul2(a2, h23);
         } else {
             const uint32_t f = row_field(stage + roff[i], b, l);
-            const uint32_t mask = (1u << b) - 1u;
-            const float zb = 8388608.0f + (float)(1 << (b - 1)) * 4096.0f;
+            // field jj of f moved to bits [12, 12 + b): a funnel shift of the 64-bit f << 12
+            const uint32_t flo = f << 12, fhi = f >> 20;
+            const uint32_t m12 = ((1u << b) - 1u) << 12;
+            const float zb = __uint_as_float(0x4B000000u | (1u << (b + 11)));  // 2^23 + 2^(b-1) 2^12
             uint32_t X[4];
+            X[0] = (flo & m12) | xb;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) X[jj] = (((f >> (b * jj)) & mask) << 12) | 0x4B000000u;
+            for (int jj = 1; jj < 4; ++jj) X[jj] = (__funnelshift_r(flo, fhi, b * jj) & m12) | xb;
             const float2 nzb = make_float2(-zb, -zb);
             const float2 z01 = add2(make_float2(__uint_as_float(X[0]), __uint_as_float(X[1])), nzb);
             const float2 z23 = add2(make_float2(__uint_as_float(X[2]), __uint_as_float(X[3])), nzb);
