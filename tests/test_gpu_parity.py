@@ -313,47 +313,74 @@ def test_calibration_kernels_match_oracle(stepq):
             assert np.allclose(dg[0, h, :, m], ref, rtol=1e-12, atol=0)
 
 
-def test_full_pool_sampled_heads(stepq):
-    """The 2,304-head pool at batch 70 (nominal 6 bits, 32 pivots), in the
-    launch configuration the benchmark times: one fused step, then sampled
-    (request, layer, head) records checked against the oracle."""
-    plan, data, wl, _ = oracle_plan("qwen_pool6")
+def _full_pool_sampled(stepq, name, n, steps, n_samples, seed, reverse_slots=False):
+    """The whole pool of a workload at batch n in the launch configuration the
+    benchmark times: S_0 and the step inputs drawn on the device by the same
+    generator, `steps` fused steps, then sampled (request, layer, head) records
+    (plus heads holding FP16 units) checked against the oracle from the records
+    the GPU held before the last step."""
+    plan, data, wl, _ = oracle_plan(name)
     pv = model.PlanView(plan)
     P = stepq.Plan.from_bytes(data)
-    n = 70
     ctx = stepq.Context(P, n)
     pool = torch.zeros(n * P.slot_bytes, dtype=torch.uint8, device="cuda")
     slots = torch.arange(n, dtype=torch.int32, device="cuda")
-    rng = np.random.default_rng(11)
-    for l in range(wl.n_layers):       # pack S_0 layer by layer to bound host memory
-        S0 = synth.initial_states(wl, wl.seed, n, layers=[l])
-        ctx.requant_pack(pool, slots, n, l, l + 1, torch.from_numpy(S0).cuda())
-    ctx.sync()
+    if reverse_slots:
+        slots = slots.flip(0).contiguous()
+    for l in range(wl.n_layers):
+        ctx.requant_pack(pool, slots, n, l, l + 1, synth.initial_states_torch(wl, wl.seed, n, l, "cuda"))
     alpha = synth.gates(wl, wl.seed)
-    inp = synth.step_inputs(wl, wl.seed, n, 0, alpha=alpha)
-    d = _inputs_to_dev(inp)
+    o = torch.zeros((n, wl.n_layers, wl.n_heads, wl.d), dtype=torch.float32, device="cuda")
     sb = P.slot_bytes
-    prev = pool.clone()
-    o = torch.zeros_like(d["q"])
-    ctx.decode_step_fused(pool, slots, n, 0, wl.n_layers, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)
+    for t in range(steps):
+        inp = synth.step_inputs_torch(wl, wl.seed, n, t, alpha, "cuda")
+        if t == steps - 1:
+            ctx.sync()
+            prev = pool.clone()
+        ctx.decode_step_fused(pool, slots, n, 0, wl.n_layers, inp["q"], inp["k"], inp["v"], inp["alpha"],
+                              inp["beta"], o)
     ctx.sync()
-    og = o.cpu().numpy()
-    widths = P.widths()
-    samples = [(int(rng.integers(n)), int(rng.integers(wl.n_layers)), int(rng.integers(wl.n_heads))) for _ in range(24)]
-    samples += [(5, int(u) // wl.n_heads, int(u) % wl.n_heads) for u in np.nonzero(widths == 16)[0][:3]]
+    rng = np.random.default_rng(seed)
+    units = P.widths().reshape(wl.n_layers * wl.n_heads, -1)
+    piv_heads = np.nonzero((units == 16).any(axis=1))[0]
+    samples = [(int(rng.integers(n)), int(rng.integers(wl.n_layers)), int(rng.integers(wl.n_heads)))
+               for _ in range(n_samples)]
+    samples += [(n - 1, int(u) // wl.n_heads, int(u) % wl.n_heads) for u in piv_heads[:3]]
+    slot_of = slots.cpu().numpy()
     for (r, l, h) in samples:
+        slot = int(slot_of[r])
         off, nb = P.record(l, h)
-        rec_prev = prev[r * sb + off:r * sb + off + nb].cpu().numpy()
-        rec_new = pool[r * sb + off:r * sb + off + nb].cpu().numpy()
+        rec_prev = prev[slot * sb + off:slot * sb + off + nb].cpu().numpy()
+        rec_new = pool[slot * sb + off:slot * sb + off + nb].cpu().numpy()
+        x = {k: inp[k][r, l, h].cpu().numpy() for k in ("q", "k", "v", "alpha", "beta")}
         new_rec, o_ref, tie, S, w = model.step_head(pv.mode, pv.D, pv.rw(l, h), pv.rho[l, h], pv.wbar[l, h],
-                                                    rec_prev, inp["q"][r, l, h], inp["k"][r, l, h],
-                                                    inp["v"][r, l, h], inp["alpha"][r, l, h], inp["beta"][r, l, h])
-        assert _close(og[r, l, h], o_ref).all(), (r, l, h)
+                                                    rec_prev, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+        assert _close(o[r, l, h].cpu().numpy(), o_ref).all(), (r, l, h)
         if not np.array_equal(rec_new, new_rec):
             zg, hg, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), rec_new)
             zo, ho, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), new_rec)
-            mism = (zg != zo) | (hg != ho)
-            assert not (mism & (tie == 0)).any(), (r, l, h)
+            assert not (((zg != zo) | (hg != ho)) & (tie == 0)).any(), (r, l, h)
+
+
+def test_full_pool_sampled_heads(stepq):
+    # the benchmark's workload: 2,304 heads, batch 70, nominal 6 bits, 32 FP16 heads; 2 steps
+    _full_pool_sampled(stepq, "qwen_pool6", 70, 2, 24, 11)
+
+
+def test_full_pool_sampled_heads_batch256(stepq):
+    # the largest batch the benchmark sweeps: 589,824 records in one launch, an 8 GB pool,
+    # slots in reverse request order
+    _full_pool_sampled(stepq, "qwen_pool6", 256, 2, 16, 12, reverse_slots=True)
+
+
+def test_kda_full_sampled_heads(stepq):
+    # 81,920 key rows (20 layers x 32 heads x 128), 512 FP16 rows, batch 128; 2 steps
+    _full_pool_sampled(stepq, "kda_rows", 128, 2, 16, 5)
+
+
+def test_kda_slice_lockstep_long(stepq):
+    # 64 steps of a 1-layer KDA slice, every request followed, fused
+    _lockstep(stepq, "kda_rows", 4, 64, check=[0, 1, 2, 3], n_layers=1, n_pivots=8, fused=True)
 
 
 # ---------------------------------------------------------------------------
@@ -394,49 +421,6 @@ def test_kda_unpack(stepq):
         g = run.slot_bytes_host(n)
         for (l, h) in [(0, 0), (1, 31), (0, 17)]:
             assert np.array_equal(Sh[n, l, h], pv.reconstruct(g, l, h))
-
-
-def test_kda_full_sampled_heads(stepq):
-    """81,920 key rows (20 layers x 32 heads x 128), 512 FP16 rows, batch 128:
-    one fused step, sampled heads checked against the oracle."""
-    plan, data, wl, _ = oracle_plan("kda_rows")
-    pv = model.PlanView(plan)
-    P = stepq.Plan.from_bytes(data)
-    n = 128
-    ctx = stepq.Context(P, n)
-    pool = torch.zeros(n * P.slot_bytes, dtype=torch.uint8, device="cuda")
-    slots = torch.arange(n, dtype=torch.int32, device="cuda")
-    for l in range(wl.n_layers):
-        S0 = synth.initial_states(wl, wl.seed, n, layers=[l])
-        ctx.requant_pack(pool, slots, n, l, l + 1, torch.from_numpy(S0).cuda())
-    ctx.sync()
-    alpha = synth.gates(wl, wl.seed)
-    inp = synth.step_inputs(wl, wl.seed, n, 0, alpha=alpha)
-    d = _inputs_to_dev(inp)
-    prev = pool.clone()
-    o = torch.zeros_like(d["q"])
-    ctx.decode_step_fused(pool, slots, n, 0, wl.n_layers, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)
-    ctx.sync()
-    og = o.cpu().numpy()
-    sb = P.slot_bytes
-    rng = np.random.default_rng(5)
-    widths = P.widths().reshape(wl.n_layers * wl.n_heads, wl.d)
-    piv_heads = np.nonzero((widths == 16).any(axis=1))[0]
-    samples = [(int(rng.integers(n)), int(rng.integers(wl.n_layers)), int(rng.integers(wl.n_heads))) for _ in range(16)]
-    samples += [(3, int(u) // wl.n_heads, int(u) % wl.n_heads) for u in piv_heads[:4]]
-    for (r, l, h) in samples:
-        off, nb = P.record(l, h)
-        rec_prev = prev[r * sb + off:r * sb + off + nb].cpu().numpy()
-        rec_new = pool[r * sb + off:r * sb + off + nb].cpu().numpy()
-        new_rec, o_ref, tie, S, w = model.step_head(pv.mode, pv.D, pv.rw(l, h), pv.rho[l, h], pv.wbar[l, h],
-                                                    rec_prev, inp["q"][r, l, h], inp["k"][r, l, h],
-                                                    inp["v"][r, l, h], inp["alpha"][r, l, h], inp["beta"][r, l, h])
-        assert _close(og[r, l, h], o_ref).all(), (r, l, h)
-        if not np.array_equal(rec_new, new_rec):
-            zg, hg, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), rec_new)
-            zo, ho, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), new_rec)
-            mism = (zg != zo) | (hg != ho)
-            assert not (mism & (tie == 0)).any(), (r, l, h)
 
 
 # --------------------------------------------------------------------------
