@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--variant", default="fused", choices=["fused", "two_stream"])
     ap.add_argument("--batch", type=int, default=None, help="requests (default: 70 GDN pool, 128 KDA)")
     ap.add_argument("--plan", type=int, default=6, choices=[4, 6], help="nominal bits of the GDN pool plan")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "layers"],
+                    help="replicas: one whole pool per rank (weak scaling); layers: one pool whose layers "
+                         "are split over the ranks, each rank holding its layers' records (strong scaling)")
     ap.add_argument("--scale-bits", type=int, default=32, choices=[32, 16],
                     help="storage of the r and c scales in the plan (16: bfloat16)")
     ap.add_argument("--workload", default="gdn", choices=["gdn", "kda"],
@@ -104,6 +107,16 @@ def sum_over_ranks(x: float, ws: int) -> float:
         return x
     import torch.distributed as dist
     return _reduce(x, ws, dist.ReduceOp.SUM)
+
+
+def layer_range(L: int, ws: int, rank: int):
+    """Layers [lb, le) of `rank` when a pool's L layers are split over ws ranks:
+    contiguous ranges whose sizes differ by at most one, covering [0, L)."""
+    if ws > L:
+        raise ValueError(f"cannot split {L} layers over {ws} ranks")
+    base, extra = divmod(L, ws)
+    lb = rank * base + min(rank, extra)
+    return lb, lb + base + (1 if rank < extra else 0)
 
 
 def replica_throughput(units_local: float, secs_local: float, ws: int):
@@ -369,7 +382,7 @@ def variant_is_full_launch(args) -> bool:
     """The committed instruction count is for the default full launch (fused,
     GDN pool, batch 70, nominal 6, fp32 scales)."""
     return (args.variant == "fused" and args.workload == "gdn" and args.batch == 70 and args.plan == 6
-            and args.scale_bits == 32)
+            and args.scale_bits == 32 and args.shard == "replicas")
 
 
 def run_product(args):
@@ -384,15 +397,20 @@ def run_product(args):
     wl = workload_of(args, synth)
     n = args.batch
     plan, plan_bytes = product_plan(stepq, synth, wl, device, args.scale_bits)
-    L, H, D = wl.n_layers, wl.n_heads, wl.d
+    H, D = wl.n_heads, wl.d
+    lb, le = (0, wl.n_layers) if args.shard == "replicas" else layer_range(wl.n_layers, ws, rank)
+    if args.shard == "layers":
+        plan = plan.slice(lb, le)   # this rank holds the records of its own layers only
+    L = le - lb
     ctx = stepq.Context(plan, n)
     pool = torch.zeros(n * plan.slot_bytes, dtype=torch.uint8, device=device)
     slots = torch.arange(n, dtype=torch.int32, device=device)
     for l in range(L):
-        ctx.requant_pack(pool, slots, n, l, l + 1, synth.initial_states_torch(wl, wl.seed, n, l, device))
+        ctx.requant_pack(pool, slots, n, l, l + 1, synth.initial_states_torch(wl, wl.seed, n, lb + l, device))
     ctx.sync()
     alpha = synth.gates(wl, wl.seed)
-    sets = [synth.step_inputs_torch(wl, wl.seed, n, t, alpha, device) for t in range(4)]
+    sets = [{k: v[:, lb:le].contiguous() for k, v in synth.step_inputs_torch(wl, wl.seed, n, t, alpha, device).items()}
+            for t in range(4)]
     o = torch.zeros((n, L, H, D), dtype=torch.float32, device=device)
     wsp = torch.empty(ctx.workspace_bytes(n, L) // 4, dtype=torch.float32, device=device)
     torch.cuda.synchronize()
@@ -419,7 +437,7 @@ def run_product(args):
     if rank == 0:
         S32 = torch.empty((n, L, H, D, D), dtype=torch.float32, device=device)
         for l in range(L):
-            S32[:, l:l + 1] = synth.initial_states_torch(wl, wl.seed, n, l, device)
+            S32[:, l:l + 1] = synth.initial_states_torch(wl, wl.seed, n, lb + l, device)
         for i in range(2):
             ctx.fp32_decode_step(S32, slots, n, 0, L, sets[i]["q"], sets[i]["k"], sets[i]["v"], sets[i]["alpha"],
                                  sets[i]["beta"], o)
@@ -511,8 +529,10 @@ def run_product(args):
             p2 = torch.zeros(bs * plan.slot_bytes, dtype=torch.uint8, device=device)
             s2 = torch.arange(bs, dtype=torch.int32, device=device)
             for l in range(L):
-                c2.requant_pack(p2, s2, bs, l, l + 1, synth.initial_states_torch(wl, wl.seed, bs, l, device))
-            st2 = [synth.step_inputs_torch(wl, wl.seed, bs, t, alpha, device) for t in range(2)]
+                c2.requant_pack(p2, s2, bs, l, l + 1, synth.initial_states_torch(wl, wl.seed, bs, lb + l, device))
+            st2 = [{k: v[:, lb:le].contiguous() for k, v in synth.step_inputs_torch(wl, wl.seed, bs, t, alpha,
+                                                                                     device).items()}
+                   for t in range(2)]
             o2 = torch.zeros((bs, L, H, D), dtype=torch.float32, device=device)
             w2 = torch.empty(c2.workspace_bytes(bs, L) // 4, dtype=torch.float32, device=device)
             sec2, _, _ = time_steps(torch, c2, args.variant, p2, s2, bs, L, st2, o2, w2, 3, 16, 1)
@@ -546,12 +566,13 @@ def run_product(args):
             "warmup": args.warmup,
             "ms_per_step": secs / args.steps * 1e3,
             "higher_is_better": True,
-            "scaling": "weak",
+            "scaling": "weak" if args.shard == "replicas" else "strong",
             "vs_baseline": None,
             "dtype": "f32",
             "data": "synthetic",
             "config": {
                 **workload_config(wl, n, ws),
+                **({"parallelism": f"layer shards x{ws} (rank 0: layers {lb}-{le - 1})"} if args.shard == "layers" else {}),
                 "variant": args.variant,
                 "bits_per_value": plan.info.bits_per_value, "bits_per_value_s16": plan.info.bits_per_value_s16,
                 "scale_bits": plan.info.scale_bits, "pool_bytes": n * plan.slot_bytes,

@@ -172,6 +172,15 @@ int stepq_plan_build_uniform(int mode, int n_layers, int n_heads, int d, int bit
                              uint64_t horizon, const float *wbar, int scale_bits, const char *path,
                              stepq_plan **out);
 
+/* The plan of layers [lb, le) of `plan` (a head- or layer-sharded pool: each
+ * GPU holds the records of its own layers).  Units, wbar, rho, l_u and L_u
+ * of those layers, the parent's mode, dims, bitset, horizon, requantizer and
+ * scale storage; n_pivots counts the slice's FP16 units; nominal bits become
+ * the slice's own average width (the parent's budget is global, not per
+ * layer), the smallest float whose floor(nominal * N) covers the widths.
+ * Errors: STEPQ_EINVAL. */
+int stepq_plan_slice(const stepq_plan *plan, int lb, int le, stepq_plan **out);
+
 /* ---- context ------------------------------------------------------------ */
 
 /* Bind a plan to the current CUDA device.  main/side are cudaStream_t (NULL

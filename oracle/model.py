@@ -261,5 +261,30 @@ def uniform_plan(mode: int, D: int, n_layers: int, n_heads: int, bits: int, quan
                 quantizer=int(quantizer), scale_bits=int(scale_bits))
 
 
+def slice_plan(plan: dict, lb: int, le: int) -> dict:
+    """The plan of layers [lb, le): their units and row weights, the parent's
+    other fields; n_pivots counts the slice's FP16 units; nominal bits are the
+    slice's own average width, the smallest float32 whose floor(nominal * N)
+    covers the widths (a global budget is not a per-layer constraint)."""
+    L, H, D = int(plan["n_layers"]), int(plan["n_heads"]), int(plan["d"])
+    per_units = H if int(plan["mode"]) == 0 else H * D
+    u = slice(lb * per_units, le * per_units)
+    rows = slice(lb * H * D, le * H * D)
+    widths = np.asarray(plan["widths"], np.uint8)[u].copy()
+    q = widths[widths != PIVOT_BITS].astype(np.int64)
+    nominal = np.float32(plan["nominal_bits"])
+    if q.size:
+        nominal = np.float32(int(q.sum()) / q.size)
+        while math.floor(float(nominal) * q.size) < int(q.sum()):
+            nominal = np.nextafter(nominal, np.float32(1e30))
+    out = dict(plan)
+    out.update(n_layers=le - lb, widths=widths, n_pivots=int((widths == PIVOT_BITS).sum()),
+               nominal_bits=float(nominal), wbar=np.asarray(plan["wbar"], np.float32).reshape(-1)[rows].copy(),
+               rho=np.asarray(plan["rho"], np.float32).reshape(-1)[rows].copy(),
+               lgate=np.asarray(plan["lgate"], np.float64)[u].copy(),
+               lifetime=np.asarray(plan["lifetime"], np.float64)[u].copy())
+    return out
+
+
 def lifetime_l_from_halflife(h: float) -> float:
     return -math.log(2.0) / h

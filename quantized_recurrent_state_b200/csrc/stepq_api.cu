@@ -565,6 +565,35 @@ extern "C" int stepq_plan_build_uniform(int mode, int n_layers, int n_heads, int
     return stepq_plan_load_mem(f.data(), f.size(), out);
 }
 
+extern "C" int stepq_plan_slice(const stepq_plan *p, int lb, int le, stepq_plan **out) {
+    if (!p || !out) return fail(STEPQ_EINVAL, "plan_slice: null argument");
+    if (lb < 0 || le > p->L || lb >= le) return fail(STEPQ_EINVAL, "plan_slice: layers [%d, %d) of %d", lb, le, p->L);
+    const size_t H = (size_t)p->H, D = (size_t)p->D;
+    const size_t per_layer_units = p->mode == 0 ? H : H * D, per_layer_rows = H * D;
+    const size_t u0 = (size_t)lb * per_layer_units, u1 = (size_t)le * per_layer_units;
+    const std::vector<uint8_t> width(p->width.begin() + u0, p->width.begin() + u1);
+    const std::vector<double> lgate(p->lgate.begin() + u0, p->lgate.begin() + u1);
+    const std::vector<double> life(p->life.begin() + u0, p->life.begin() + u1);
+    const std::vector<float> wbar(p->wbar.begin() + (size_t)lb * per_layer_rows, p->wbar.begin() + (size_t)le * per_layer_rows);
+    int piv = 0;
+    uint64_t bits = 0, n_q = 0;
+    for (uint8_t w : width) {
+        if (w == STEPQ_PIVOT_BITS) { ++piv; continue; }
+        bits += w;
+        ++n_q;
+    }
+    // the global budget is not a per-layer constraint: the slice carries its own average,
+    // the smallest float whose floor(nominal * N) still covers its widths
+    float nominal = p->nominal;
+    if (n_q) {
+        nominal = (float)((double)bits / (double)n_q);
+        while ((uint64_t)std::floor((double)nominal * (double)n_q) < bits) nominal = std::nextafter(nominal, 1e30f);
+    }
+    const std::vector<uint8_t> f = serialize_plan(p->mode, le - lb, p->H, p->D, piv, p->bitset, nominal, p->horizon,
+                                                  p->quantizer, p->scale_bits, width, wbar.data(), lgate.data(), life);
+    return stepq_plan_load_mem(f.data(), f.size(), out);
+}
+
 // ---------------------------------------------------------------------------
 // context
 // ---------------------------------------------------------------------------

@@ -25,7 +25,7 @@ EXPORTED = [
     "stepq_decode_step_fused", "stepq_sync", "stepq_unpack", "stepq_fp32_decode_step",
     "stepq_calib_accumulate", "stepq_calib_distortion", "stepq_copy_probe",
     "stepq_launch_count", "stepq_last_error", "stepq_ctx_set_timing", "stepq_kernel_stats",
-    "stepq_decode_step_noalloc", "stepq_plan_build_uniform", "stepq_ctx_set_wait_limit",
+    "stepq_decode_step_noalloc", "stepq_plan_build_uniform", "stepq_ctx_set_wait_limit", "stepq_plan_slice",
 ]
 QUANT_DUAL_AXIS = 0  # plan requantizer: STEPQuant row/column fit
 QUANT_ABSMAX = 1     # plan requantizer: per-row absmax baseline, c = 1
@@ -74,6 +74,7 @@ def lib():
                                        ctypes.c_char_p, ctypes.POINTER(P)]
         l.stepq_plan_build_uniform.argtypes = [I, I, I, I, I, I, ctypes.c_uint64, P, I, ctypes.c_char_p,
                                                ctypes.POINTER(P)]
+        l.stepq_plan_slice.argtypes = [P, I, I, ctypes.POINTER(P)]
         l.stepq_ctx_create.argtypes = [P, P, P, I, I, ctypes.POINTER(P)]
         l.stepq_ctx_free.argtypes = [P]
         l.stepq_ctx_free.restype = None
@@ -157,6 +158,12 @@ class Plan:
                                               None if wb is None else wb.ctypes.data, int(scale_bits),
                                               path.encode() if path else None, ctypes.byref(h)))
         return cls(h)
+
+    def slice(self, lb: int, le: int) -> "Plan":
+        """The plan of layers [lb, le) (its own pool layout)."""
+        h = P()
+        _check(lib().stepq_plan_slice(self._h, int(lb), int(le), ctypes.byref(h)))
+        return Plan(h)
 
     def widths(self) -> np.ndarray:
         out = np.zeros(self.info.n_units, dtype=np.uint8)

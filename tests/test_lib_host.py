@@ -182,3 +182,30 @@ def test_quantizer_field_validation():
     with pytest.raises(stepq.StepqError) as ei:
         stepq.Plan.build_uniform(1, 2, 2, 16, 4, stepq.QUANT_ABSMAX)
     assert ei.value.code == stepq.EINVAL
+
+
+@pytest.mark.parametrize("mode,sbits", [(0, 32), (0, 16), (1, 32)])
+def test_plan_slice_matches_oracle(mode, sbits):
+    L, H, D = 5, 4, 16
+    bits = (4, 6, 8)
+    st = _random_stats(mode, L, H, D, bits, 21)
+    pivots = 3 if mode == 0 else 12
+    ora = model.build_plan(mode, D, L, H, st, bits, 6.0, pivots, 4096, scale_bits=sbits)
+    p = stepq.Plan.from_bytes(plan_io.write_plan(None, ora))
+    for lb, le in ((0, 5), (1, 3), (4, 5), (0, 1)):
+        sp = p.slice(lb, le)
+        so = model.slice_plan(ora, lb, le)
+        assert (sp.n_layers, sp.info.n_pivots, sp.info.scale_bits) == (le - lb, so["n_pivots"], sbits)
+        assert np.array_equal(sp.widths(), so["widths"])
+        assert sp.info.nominal_bits == np.float32(so["nominal_bits"])
+        # the oracle's own file of the slice parses to the same plan
+        back = stepq.Plan.from_bytes(plan_io.write_plan(None, so))
+        assert back.slot_bytes == sp.slot_bytes
+        offs, slot = plan_io.pool_layout(so)
+        assert sp.slot_bytes == slot
+        for l in range(le - lb):
+            for h in range(H):
+                assert sp.record(l, h) == (int(offs[l * H + h]), plan_io.record_bytes(
+                    mode, D, plan_io.head_row_widths(so, l, h), sbits))
+    with pytest.raises(stepq.StepqError):
+        p.slice(3, 3)
