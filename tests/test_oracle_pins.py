@@ -630,3 +630,39 @@ def test_plan_roundtrip(tmp_path):
     offs, slot = plan_io.pool_layout(back)
     # records: b=2: 64+128 -> 256; b=6: 192+128 -> 384; pivot 512; b=4: 128+128 = 256
     assert list(offs) == [0, 256, 640, 1152] and slot == 1408
+
+
+# --------------------------------------------------------------------------
+# chunked prefill: the chunk formulas equal the sequential recurrence (fp64),
+# for ragged lengths and any chunk size; a one-token chunk is one step
+# --------------------------------------------------------------------------
+
+def _prompt(T, D, seed):
+    g = np.random.default_rng(seed)
+    Q = g.standard_normal((T, D))
+    K = g.standard_normal((T, D))
+    K /= np.linalg.norm(K, axis=1, keepdims=True)
+    V = g.standard_normal((T, D))
+    alpha = np.exp(-np.log(2) / np.exp(g.uniform(np.log(2), np.log(2000), T)))
+    beta = g.uniform(0, 1, T)
+    S0 = g.standard_normal((D, D))
+    return S0, Q, K, V, alpha, beta
+
+
+@pytest.mark.parametrize("T,C", [(1, 64), (63, 64), (64, 64), (65, 64), (200, 64), (130, 16), (37, 8)])
+def test_chunked_prefill_equals_sequential(T, C):
+    from oracle import prefill
+    S0, Q, K, V, alpha, beta = _prompt(T, 32, 700 + T + C)
+    O_seq, S_seq = prefill.sequential(S0, Q, K, V, alpha, beta)
+    O_chk, S_chk = prefill.chunked(S0, Q, K, V, alpha, beta, C)
+    assert np.max(np.abs(O_chk - O_seq)) <= 1e-11 * max(1.0, np.max(np.abs(O_seq)))
+    assert np.max(np.abs(S_chk - S_seq)) <= 1e-11 * max(1.0, np.max(np.abs(S_seq)))
+
+
+def test_chunk_of_one_token_is_one_step():
+    from oracle import prefill
+    S0, Q, K, V, alpha, beta = _prompt(1, 16, 9)
+    O, S = prefill.chunk(S0, Q, K, V, alpha, beta)
+    S_ref = alpha[0] * S0 + beta[0] * np.outer(K[0], V[0] - alpha[0] * S0.T @ K[0])
+    assert np.allclose(S, S_ref, rtol=1e-14, atol=1e-14)
+    assert np.allclose(O[0], S_ref.T @ Q[0], rtol=1e-13, atol=1e-13)
