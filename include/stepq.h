@@ -196,6 +196,37 @@ size_t stepq_workspace_bytes(const stepq_ctx *ctx, int n_req, int n_layers_launc
 
 /* ---- the decode step (方法-4) --------------------------------------------- */
 
+/* ---- prefill (the step before decode) ----------------------------------- */
+
+/* Chunked prefill of T tokens on fp32 states (per-head units, d = 128):
+ * for every (request, layer in [lb, le), head) the gated delta rule above,
+ * token by token in meaning, S_t = (I - beta_t k_t k_t^T) alpha_t S_{t-1} +
+ * beta_t k_t v_t^T and o_t = S_t^T q_t, evaluated in chunks of 64 tokens:
+ * with gamma_t the running gate product in the chunk, (I + M) U = V -
+ * diag(gamma) K S_0 with M_ts = gamma_t/gamma_s beta_s k_t.k_s (s < t),
+ * O = diag(gamma) Q S_0 + L_incl(Q K^T o gamma_t/gamma_s) diag(beta) U and
+ * S_C = gamma_C S_0 + K^T diag(beta gamma_C/gamma) U.  The dense products run
+ * on the tensor cores (TF32 with a TF32 remainder, near fp32), the
+ * triangular solve on the CUDA cores; results match the token-by-token fp64
+ * recurrence to the tolerance stated in the tests, not bit for bit.
+ *   S: [n_req][le-lb][n_heads][D][D] fp32, read (unless zero_init) and written.
+ *   q, k, v, o: [n_req][T][le-lb][n_heads][D];  alpha, beta: [n_req][T][le-lb][n_heads],
+ *   alpha in (0, 1] (its logarithm is taken).  Enqueued on main. */
+int stepq_prefill_fp32(stepq_ctx *ctx, float *S, int n_req, int lb, int le, int T, const float *q,
+                       const float *k, const float *v, const float *alpha, const float *beta, float *o,
+                       int zero_init);
+/* Bytes of the fp32 workspace stepq_prefill needs: one layer's states of the
+ * batch (n_req * n_heads * D * D * 4). */
+size_t stepq_prefill_workspace_bytes(const stepq_ctx *ctx, int n_req);
+/* Prefill into packed states: per layer, the pool records of the slots are
+ * unpacked into the workspace (from_zero: S_0 = 0 instead), prefilled as in
+ * stepq_prefill_fp32, and requantized into the pool (the plan's requantizer).
+ * Same input layouts; enqueued on main after the side stream's last work on
+ * those layers. */
+int stepq_prefill(stepq_ctx *ctx, void *pool, const int32_t *slots, int n_req, int lb, int le, int T,
+                  const float *q, const float *k, const float *v, const float *alpha, const float *beta,
+                  float *o, float *workspace, int from_zero);
+
 /* Pack fp32 states S into the pool records of (slots, layers [lb, le)):
  * the requantizer of the header comment (used for S_0).  Enqueued on main. */
 int stepq_requant_pack(stepq_ctx *ctx, void *pool, const int32_t *slots, int n_req, int lb, int le,

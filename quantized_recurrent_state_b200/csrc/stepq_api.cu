@@ -33,6 +33,7 @@ cudaError_t launch_fp32_step(int D, const Args &a, float *S_pool, int n_layers_t
 cudaError_t launch_copy(void *dst, const void *src, size_t bytes, int n_sms, cudaStream_t st);
 cudaError_t launch_calib_acc(int D, const Args &a, double *om, double *ls, cudaStream_t st);
 cudaError_t launch_calib_dist(int D, const Args &a, const int *bits, int n_bits, double *acc, cudaStream_t st);
+cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t st);
 }  // namespace stepq
 
 namespace {
@@ -995,6 +996,83 @@ extern "C" int stepq_sync(stepq_ctx *c, int timeout_ms) {
         cudaMemset(c->err, 0, sizeof(int));
         return fail(STEPQ_EDEVICE, "device error word 0x%x (%s%s%s)", word, (word & stepq::kErrBadSlot) ? "slot out of range " : "",
                     (word & stepq::kErrWait) ? "copy wait gave up " : "", (word & stepq::kErrArgs) ? "bad width " : "");
+    }
+    return STEPQ_OK;
+}
+
+extern "C" int stepq_prefill_fp32(stepq_ctx *c, float *S, int n_req, int lb, int le, int T, const float *q,
+                                  const float *k, const float *v, const float *alpha, const float *beta, float *o,
+                                  int zero_init) {
+    NvtxRange nvtx_range("stepq_prefill_fp32");
+    int rc = check_range(c, n_req, lb, le);
+    if (rc) return rc;
+    if (c->plan->mode != 0 || c->plan->D != 128)
+        return fail(STEPQ_EINVAL, "prefill: per-head units with d = 128 only (mode %d, d %d)", c->plan->mode, c->plan->D);
+    if (T < 0) return fail(STEPQ_EINVAL, "prefill: T = %d", T);
+    if ((rc = check_ptr(S, 16, "S")) || (rc = check_ptr(q, 16, "q")) || (rc = check_ptr(k, 16, "k")) ||
+        (rc = check_ptr(v, 16, "v")) || (rc = check_ptr(alpha, 4, "alpha")) || (rc = check_ptr(beta, 4, "beta")) ||
+        (rc = check_ptr(o, 16, "o")))
+        return rc;
+    if ((rc = set_device(c))) return rc;
+    if (n_req == 0 || T == 0) return STEPQ_OK;
+    stepq::PrefillArgs a{};
+    a.S = S; a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.o = o;
+    a.n_req = n_req; a.T = T; a.nL = le - lb; a.nL_in = le - lb; a.l_in0 = 0; a.H = c->plan->H;
+    a.zero_init = zero_init ? 1 : 0;
+    LaunchTimer lt(c, 3, c->main);
+    const cudaError_t e = stepq::launch_prefill(a, c->main);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+    lt.done();
+    return STEPQ_OK;
+}
+
+extern "C" size_t stepq_prefill_workspace_bytes(const stepq_ctx *c, int n_req) {
+    if (!c) return 0;
+    return (size_t)n_req * c->plan->H * c->plan->D * c->plan->D * sizeof(float);
+}
+
+extern "C" int stepq_prefill(stepq_ctx *c, void *pool, const int32_t *slots, int n_req, int lb, int le, int T,
+                             const float *q, const float *k, const float *v, const float *alpha, const float *beta,
+                             float *o, float *workspace, int from_zero) {
+    NvtxRange nvtx_range("stepq_prefill");
+    int rc = check_range(c, n_req, lb, le);
+    if (rc) return rc;
+    if (c->plan->mode != 0 || c->plan->D != 128)
+        return fail(STEPQ_EINVAL, "prefill: per-head units with d = 128 only (mode %d, d %d)", c->plan->mode, c->plan->D);
+    if (T < 0) return fail(STEPQ_EINVAL, "prefill: T = %d", T);
+    if ((rc = check_ptr(pool, 128, "pool")) || (rc = check_ptr(slots, 4, "slots")) || (rc = check_ptr(q, 16, "q")) ||
+        (rc = check_ptr(k, 16, "k")) || (rc = check_ptr(v, 16, "v")) || (rc = check_ptr(alpha, 4, "alpha")) ||
+        (rc = check_ptr(beta, 4, "beta")) || (rc = check_ptr(o, 16, "o")) || (rc = check_ptr(workspace, 16, "workspace")))
+        return rc;
+    if ((rc = set_device(c))) return rc;
+    if (n_req == 0 || T == 0) return STEPQ_OK;
+    if ((rc = wait_side(c, lb, le))) return rc;
+    // one layer at a time: state -> fp32 workspace, the chunked prefill, requantize into the pool
+    for (int l = lb; l < le; ++l) {
+        stepq::Args a = base_args(c, pool, slots, n_req, l, l + 1);
+        cudaError_t e = cudaSuccess;
+        if (!from_zero) {
+            a.S_out = workspace;
+            LaunchTimer lt(c, 3, c->main);
+            e = stepq::launch_pack(c->plan->D, a, true, c->main);
+            if (e != cudaSuccess) return cuda_fail(e, "prefill: unpack launch");
+            lt.done();
+        }
+        stepq::PrefillArgs p{};
+        p.S = workspace; p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta; p.o = o;
+        p.n_req = n_req; p.T = T; p.nL = 1; p.nL_in = le - lb; p.l_in0 = l - lb; p.H = c->plan->H;
+        p.zero_init = from_zero ? 1 : 0;
+        {
+            LaunchTimer lt(c, 3, c->main);
+            e = stepq::launch_prefill(p, c->main);
+            if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+            lt.done();
+        }
+        a.S_in = workspace;
+        LaunchTimer lt(c, 3, c->main);
+        e = stepq::launch_pack(c->plan->D, a, false, c->main);
+        if (e != cudaSuccess) return cuda_fail(e, "prefill: requant_pack launch");
+        lt.done();
     }
     return STEPQ_OK;
 }

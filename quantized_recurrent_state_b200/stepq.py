@@ -25,7 +25,8 @@ EXPORTED = [
     "stepq_decode_step_fused", "stepq_sync", "stepq_unpack", "stepq_fp32_decode_step",
     "stepq_calib_accumulate", "stepq_calib_distortion", "stepq_copy_probe",
     "stepq_launch_count", "stepq_last_error", "stepq_ctx_set_timing", "stepq_kernel_stats",
-    "stepq_decode_step_noalloc", "stepq_plan_build_uniform", "stepq_ctx_set_wait_limit", "stepq_plan_slice",
+    "stepq_decode_step_noalloc", "stepq_plan_build_uniform", "stepq_ctx_set_wait_limit", "stepq_plan_slice", "stepq_prefill_fp32", "stepq_prefill",
+    "stepq_prefill_workspace_bytes",
 ]
 QUANT_DUAL_AXIS = 0  # plan requantizer: STEPQuant row/column fit
 QUANT_ABSMAX = 1     # plan requantizer: per-row absmax baseline, c = 1
@@ -75,6 +76,10 @@ def lib():
         l.stepq_plan_build_uniform.argtypes = [I, I, I, I, I, I, ctypes.c_uint64, P, I, ctypes.c_char_p,
                                                ctypes.POINTER(P)]
         l.stepq_plan_slice.argtypes = [P, I, I, ctypes.POINTER(P)]
+        l.stepq_prefill_fp32.argtypes = [P, P, I, I, I, I, P, P, P, P, P, P, I]
+        l.stepq_prefill.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, P, P, I]
+        l.stepq_prefill_workspace_bytes.argtypes = [P, I]
+        l.stepq_prefill_workspace_bytes.restype = ctypes.c_size_t
         l.stepq_ctx_create.argtypes = [P, P, P, I, I, ctypes.POINTER(P)]
         l.stepq_ctx_free.argtypes = [P]
         l.stepq_ctx_free.restype = None
@@ -245,6 +250,20 @@ class Context:
         return _check(lib().stepq_fp32_decode_step(self._h, _ptr(S_pool), _ptr(slots), n_req, lb, le,
                                                    _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                                    _ptr(o)))
+
+    def prefill_fp32(self, S, n_req, lb, le, T, q, k, v, alpha, beta, o, zero_init=False):
+        self._after_caller()
+        return _check(lib().stepq_prefill_fp32(self._h, _ptr(S), n_req, lb, le, int(T), _ptr(q), _ptr(k), _ptr(v),
+                                               _ptr(alpha), _ptr(beta), _ptr(o), 1 if zero_init else 0))
+
+    def prefill_workspace_bytes(self, n_req: int) -> int:
+        return int(lib().stepq_prefill_workspace_bytes(self._h, n_req))
+
+    def prefill(self, pool, slots, n_req, lb, le, T, q, k, v, alpha, beta, o, workspace, from_zero=False):
+        self._after_caller()
+        return _check(lib().stepq_prefill(self._h, _ptr(pool), _ptr(slots), n_req, lb, le, int(T), _ptr(q), _ptr(k),
+                                          _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o), _ptr(workspace),
+                                          1 if from_zero else 0))
 
     def calib_accumulate(self, n_req, lb, le, q, k, alpha, beta, omega_acc, lsum_acc):
         self._after_caller()

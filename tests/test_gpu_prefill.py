@@ -1,0 +1,124 @@
+"""Chunked prefill on the GPU against the token-by-token fp64 recurrence.
+
+The prefill evaluates the gated delta rule in chunks of 64 tokens with the
+dense products on the tensor cores (TF32 plus a TF32 remainder) and an fp32
+triangular solve, so it matches the oracle to a tolerance, not bit for bit.
+Tolerance: each product has relative error about 2^-21 of its terms' sum
+(the dropped lo*lo term and the TF32 rounding of the remainders), the fp32
+solve about 64 * 2^-24, the gate ratios about |log gamma| 2^-24; over T/64
+chunks these add up, and 2e-4 of the largest magnitude (per head) covers
+T <= 256 with a wide margin.  Codes written by the packed prefill are
+checked bit for bit against the oracle's quantization of the GPU's own fp32
+final state.
+"""
+import numpy as np
+import pytest
+
+from oracle import model, prefill
+from quantized_recurrent_state_b200 import synth
+from tests._workloads import oracle_plan
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-4
+
+
+@pytest.fixture(scope="module")
+def stepq():
+    from quantized_recurrent_state_b200 import build as qbuild
+    qbuild.build()
+    from quantized_recurrent_state_b200 import stepq as s
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return s
+
+
+def _prompt(wl, n, T, seed):
+    """[n][T][L][H][D] q, k, v and [n][T][L][H] alpha, beta from the step generator."""
+    alpha = synth.gates(wl, seed)
+    steps = [synth.step_inputs(wl, seed, n, t, alpha=alpha) for t in range(T)]
+    return {key: np.ascontiguousarray(np.stack([s[key] for s in steps], axis=1)) for key in steps[0]}
+
+
+def _check_head(O_gpu, S_gpu, S0, inp, r, h):
+    O_ref, S_ref = prefill.sequential(S0, inp["q"][r, :, 0, h], inp["k"][r, :, 0, h], inp["v"][r, :, 0, h],
+                                      inp["alpha"][r, :, 0, h], inp["beta"][r, :, 0, h])
+    eo = np.max(np.abs(O_gpu - O_ref)) / max(1e-30, np.max(np.abs(O_ref)))
+    es = np.max(np.abs(S_gpu - S_ref)) / max(1e-30, np.max(np.abs(S_ref)))
+    assert eo <= TOL and es <= TOL, (r, h, eo, es)
+    return eo, es
+
+
+@pytest.mark.parametrize("T", [1, 64, 100, 256])
+def test_prefill_fp32_matches_sequential(stepq, T):
+    plan, data, wl, _ = oracle_plan("qwen_layer")
+    P = stepq.Plan.from_bytes(data)
+    n = 2
+    ctx = stepq.Context(P, n)
+    S0 = synth.initial_states(wl, wl.seed, n)                     # [n][1][H][D][D]
+    inp = _prompt(wl, n, T, 3000 + T)
+    d = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
+    S = torch.from_numpy(S0).cuda()
+    o = torch.zeros_like(d["q"])
+    ctx.prefill_fp32(S, n, 0, 1, T, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)
+    ctx.sync()
+    Sg, og = S.cpu().numpy(), o.cpu().numpy()
+    worst = (0.0, 0.0)
+    for (r, h) in [(0, 0), (1, 7), (0, 23), (1, 47)]:
+        e = _check_head(og[r, :, 0, h], Sg[r, 0, h], S0[r, 0, h].astype(np.float64), inp, r, h)
+        worst = (max(worst[0], e[0]), max(worst[1], e[1]))
+    print(f"T={T}: worst relative errors o {worst[0]:.2e}, S {worst[1]:.2e}")
+
+
+def test_prefill_fp32_zero_init_and_empty(stepq):
+    plan, data, wl, _ = oracle_plan("qwen_layer")
+    P = stepq.Plan.from_bytes(data)
+    ctx = stepq.Context(P, 1)
+    inp = _prompt(wl, 1, 70, 41)
+    d = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
+    S = torch.full((1, 1, wl.n_heads, wl.d, wl.d), float("nan"), dtype=torch.float32, device="cuda")
+    o = torch.zeros_like(d["q"])
+    ctx.prefill_fp32(S, 1, 0, 1, 70, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o, zero_init=True)
+    ctx.sync()
+    _check_head(o.cpu().numpy()[0, :, 0, 5], S.cpu().numpy()[0, 0, 5], np.zeros((wl.d, wl.d)), inp, 0, 5)
+    before = S.clone()
+    ctx.prefill_fp32(S, 1, 0, 1, 0, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)   # T = 0: nothing
+    ctx.sync()
+    assert torch.equal(S, before)
+
+
+@pytest.mark.parametrize("from_zero", [False, True])
+def test_prefill_into_packed_states(stepq, from_zero):
+    plan, data, wl, _ = oracle_plan("qwen_layer")
+    pv = model.PlanView(plan)
+    P = stepq.Plan.from_bytes(data)
+    n, T = 3, 130
+    ctx = stepq.Context(P, n + 2)
+    slots = torch.tensor([4, 0, 2], dtype=torch.int32, device="cuda")
+    pool = torch.zeros((n + 2) * P.slot_bytes, dtype=torch.uint8, device="cuda")
+    S0 = synth.initial_states(wl, wl.seed, n)
+    ctx.requant_pack(pool, slots, n, 0, 1, torch.from_numpy(S0).cuda())
+    ctx.sync()
+    sb = P.slot_bytes
+    before = pool.cpu().numpy().copy()
+    inp = _prompt(wl, n, T, 77)
+    d = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
+    o = torch.zeros_like(d["q"])
+    ws = torch.empty(ctx.prefill_workspace_bytes(n) // 4, dtype=torch.float32, device="cuda")
+    ctx.prefill(pool, slots, n, 0, 1, T, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o, ws, from_zero=from_zero)
+    ctx.sync()
+    after, og = pool.cpu().numpy(), o.cpu().numpy()
+    S_T = ws.view(n, 1, wl.n_heads, wl.d, wl.d).cpu().numpy()   # the last (only) layer's fp32 final states
+    slot_of = slots.cpu().numpy()
+    for r in range(n):
+        s = int(slot_of[r])
+        prev_slot = before[s * sb:(s + 1) * sb]
+        new_slot = after[s * sb:(s + 1) * sb]
+        for h in (0, 9, 30):
+            S_start = np.zeros((wl.d, wl.d)) if from_zero else pv.reconstruct(prev_slot, 0, h).astype(np.float64)
+            _check_head(og[r, :, 0, h], S_T[r, 0, h], S_start, inp, r, h)
+            expect = np.zeros_like(new_slot)
+            pv.quantize_into(expect, 0, h, S_T[r, 0, h])
+            assert np.array_equal(pv.record(new_slot, 0, h), pv.record(expect, 0, h)), (r, h)
+    for s in (1, 3):   # slots outside the batch are untouched
+        assert np.array_equal(after[s * sb:(s + 1) * sb], before[s * sb:(s + 1) * sb])
