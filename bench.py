@@ -34,7 +34,10 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "packed-state decode head-steps/s and HBM GB/s (% of peak), 2304 heads, bs=70"
+PREFILL_METRIC = "chunked prefill tokens/s into the packed 2304-head state pool"
+TF32_PER_BF16 = 1.1 / 2.25   # nominal dense TF32 / BF16 tensor throughput
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = ["stepq_step.cu", "stepq_dev.cuh"]
 
 
@@ -55,6 +58,9 @@ def parse():
     ap.add_argument("--workload", default="gdn", choices=["gdn", "kda"],
                     help="gdn: 2,304-head pool; kda: 81,920 key rows (20 x 32 x 128)")
     ap.add_argument("--sweep", action="store_true", help="also time batch 1/16/70/128/256")
+    ap.add_argument("--prefill", type=int, default=0, metavar="T",
+                    help="time chunked prefill of T-token prompt chunks into the packed pool (GDN) instead of "
+                         "the decode step; batch defaults to 1")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -194,6 +200,15 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_bf16_tflops():
+    """Dense bf16 tensor throughput measured by a cuBLAS GEMM burst (TFLOP/s)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        return float(json.load(open(p))["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def kernel_hash():
@@ -359,7 +374,7 @@ def workload_of(args, synth):
     else:
         wl = synth.workloads()["qwen_pool6" if args.plan == 6 else "qwen_pool4"]
     if args.batch is None:
-        args.batch = 128 if args.workload == "kda" else 70
+        args.batch = 1 if args.prefill else 128 if args.workload == "kda" else 70
     return wl
 
 
@@ -603,6 +618,194 @@ def run_product(args):
 
 
 # ---------------------------------------------------------------------------
+# chunked prefill
+# ---------------------------------------------------------------------------
+
+PREFILL_CHUNK = 64   # tokens per chunk of the prefill kernel
+PREFILL_CPU_TOKENS = 256   # tokens per head of the oracle's timed sample
+
+
+def prefill_flops(T: int, D: int, C: int = PREFILL_CHUNK) -> int:
+    """Algorithmic FLOPs of one head's T-token prefill in the chunk form: per
+    chunk of c tokens the six dense products (K K^T, Q K^T, A U: 2 c^2 D each;
+    K S_0, Q S_0, K^T U: 2 c D^2 each) and the triangular solve (c (c-1) D)."""
+    tot = 0
+    for c0 in range(0, T, C):
+        c = min(C, T - c0)
+        tot += 6 * c * c * D + 6 * c * D * D + c * (c - 1) * D
+    return tot
+
+
+def prefill_bytes(T: int, D: int) -> int:
+    """Algorithmic HBM bytes of one head in a prefill kernel launch: q, k, v
+    read and o written per token, alpha and beta read, the fp32 state read
+    and written once."""
+    return T * (4 * 4 * D + 8) + 2 * 4 * D * D
+
+
+def prefill_config(wl, n, T, ws):
+    L, H, D = wl.n_layers, wl.n_heads, wl.d
+    return {"workload": (f"chunked prefill of {T}-token prompt chunks into the GDN state pool, {L} layers x {H} "
+                         f"heads = {L * H} heads, d_k=d_v={D}, batch {n}, nominal {wl.nominal_bits:g}-bit plan "
+                         f"over {sorted(wl.bits)}, {wl.n_pivots} FP16 pivot heads; each step continues from the "
+                         f"packed states the previous one wrote"),
+            "batch": n, "prompt_chunk_tokens": T, "kernel_chunk_tokens": PREFILL_CHUNK, "heads": L * H, "d": D,
+            "l2": "inputs larger than L2 (one step's q, k, v far above 126 MB)",
+            "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"}
+
+
+def run_prefill(args):
+    """One step = the packed prefill of a T-token chunk for every (request,
+    layer, head): unpack the records, the chunked gated delta rule on the
+    tensor cores, requantize and pack (three launches)."""
+    import torch
+    from quantized_recurrent_state_b200 import build as qbuild
+    ws, rank, local = dist_init()
+    if rank == 0:
+        qbuild.build()
+    barrier(ws)
+    from quantized_recurrent_state_b200 import stepq, synth
+    device = torch.device("cuda", local)
+    wl = workload_of(args, synth)
+    n, T = args.batch, args.prefill
+    plan, plan_bytes = product_plan(stepq, synth, wl, device, args.scale_bits)
+    L, H, D = wl.n_layers, wl.n_heads, wl.d
+    ctx = stepq.Context(plan, n)
+    pool = torch.zeros(n * plan.slot_bytes, dtype=torch.uint8, device=device)
+    slots = torch.arange(n, dtype=torch.int32, device=device)
+    for l in range(L):
+        ctx.requant_pack(pool, slots, n, l, l + 1, synth.initial_states_torch(wl, wl.seed, n, l, device))
+    alpha = synth.gates(wl, wl.seed)
+    inp = synth.prompt_inputs_torch(wl, wl.seed, n, 0, T, alpha, device)
+    o = torch.zeros_like(inp["q"])
+    wsp = torch.empty(ctx.prefill_workspace_bytes(n, L) // 4, dtype=torch.float32, device=device)
+    torch.cuda.synchronize()
+
+    def step():
+        ctx.prefill(pool, slots, n, 0, L, T, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o, wsp)
+
+    for _ in range(args.warmup):
+        step()
+    ctx.sync()
+    ctx.kernel_stats()
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    ctx.set_timing(True)
+    launches0 = ctx.launches
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.__enter__()
+    e0.record(ctx.main)
+    for _ in range(args.steps):
+        step()
+    e1.record(ctx.main)
+    torch.cuda.synchronize()
+    clocks.__exit__(None, None, None)
+    ctx.sync()
+    barrier(ws)
+    torch.cuda.synchronize()
+    ctx.set_timing(False)
+    launches = ctx.launches - launches0
+    stats = ctx.kernel_stats()
+    value, secs = replica_throughput(n * T * args.steps, e0.elapsed_time(e1) / 1e3, ws)
+
+    k_ms, k_n = stats["prefill"]
+    launch_s = k_ms / k_n / 1e3
+    flops = n * L * H * prefill_flops(T, D)
+    bf16, peak_kind = measured_bf16_tflops()
+    peak = bf16 * TF32_PER_BF16
+    achieved = flops / launch_s / 1e12
+    hbm_peak, hbm_kind = measured_peaks()
+    k_bytes = n * L * H * prefill_bytes(T, D)
+
+    # the same tokens stepped one at a time by the fused decode step, for comparison
+    compare = None
+    if rank == 0:
+        sets = [synth.step_inputs_torch(wl, wl.seed, n, t, alpha, device) for t in range(4)]
+        o2 = torch.zeros((n, L, H, D), dtype=torch.float32, device=device)
+        w2 = torch.empty(ctx.workspace_bytes(n, L) // 4, dtype=torch.float32, device=device)
+        sec_dec, _, _ = time_steps(torch, ctx, "fused", pool, slots, n, L, sets, o2, w2, 3, 32, 1)
+        dec_tok = sec_dec / 32
+        pre_tok = e0.elapsed_time(e1) / 1e3 / (args.steps * T)
+        compare = {"fused_decode_ms_per_token": dec_tok * 1e3, "prefill_ms_per_token": pre_tok * 1e3,
+                   "speedup": dec_tok / pre_tok,
+                   "note": "per prompt token of the whole pool at this batch: the fused decode step run once "
+                           "per token against the chunked prefill"}
+        del sets, o2, w2
+
+    e2e = None
+    if not args.no_e2e:
+        # every step: the chunk's q, k, v, alpha, beta from pinned host memory, the prefill, o back
+        host = {k: v.cpu().pin_memory() for k, v in inp.items()}
+        o_host = torch.empty(o.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(v.numel() * 4 for v in host.values())
+        d2h = o_host.numel() * 4
+        k_e2e = min(args.steps, 3)
+        torch.cuda.synchronize()
+        barrier(ws)
+        t0 = time.perf_counter()
+        for _ in range(k_e2e):
+            with torch.cuda.stream(ctx.main):
+                for kk in host:
+                    inp[kk].copy_(host[kk], non_blocking=True)
+                step()
+                o_host.copy_(o, non_blocking=True)
+        torch.cuda.synchronize()
+        t_e2e = max_over_ranks(time.perf_counter() - t0, ws)
+        e2e = {"value": sum_over_ranks(n * T * k_e2e, ws) / t_e2e, "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e,
+               "overlap": "none: the copies and the launches of a step in order on one stream"}
+        del host, o_host
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu:
+        cpu = cpu_prefill_baseline(plan_bytes, wl, budget_s=12.0)
+
+    if rank == 0:
+        csum = clocks.summary()
+        out = {
+            "metric": PREFILL_METRIC,
+            "value": value,
+            "unit": "tokens/s",
+            "n_gpus": ws,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32 (tensor-core products in TF32 with a TF32 remainder)",
+            "data": "synthetic",
+            "config": {**prefill_config(wl, n, T, ws), "scale_bits": plan.info.scale_bits,
+                       "pool_bytes": n * plan.slot_bytes},
+            "head_tokens_per_s": value * L * H,
+            "roofline": {"bound": "tensor", "kernel": "prefill", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "algorithmic_flops_per_launch": flops, "launch_ms": launch_s * 1e3,
+                         "peak_source": f"{peak_kind} bf16 burst {bf16:g} TFLOP/s x nominal TF32/BF16 "
+                                        f"{TF32_PER_BF16:.4f}",
+                         "hbm": {"achieved": k_bytes / launch_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                                 "frac": k_bytes / launch_s / 1e9 / hbm_peak, "peak_source": hbm_kind,
+                                 "algorithmic_bytes_per_launch": k_bytes},
+                         "note": "each product runs as three TF32 MMAs (hi*hi + hi*lo + lo*hi), so the tensor "
+                                 "pipe caps frac at 1/3"},
+            "kernel_ms": {k: v[0] for k, v in stats.items() if v[1]},
+            "kernel_launches": {k: v[1] for k, v in stats.items() if v[1]},
+            "gpu_launches": launches,
+            "clocks": {"sm_mhz": csum["sm_mhz"], "sm_max_mhz": csum["sm_max_mhz"], "reasons": csum["reasons"]},
+            "vs_decode_loop": compare,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(out), flush=True)
+    ctx.close()
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle (cpu_baseline leg and --impl reference)
 # ---------------------------------------------------------------------------
 
@@ -634,6 +837,60 @@ def _oracle_sample(payload):
     return time.perf_counter() - t0
 
 
+def _oracle_prefill_sample(payload):
+    """The oracle's packed prefill of a T-token chunk for a set of (layer,
+    head) states of request 0: reconstruct the record, the chunk form of the
+    gated delta rule in fp64, requantize.  Packing S_0 and drawing inputs are
+    not timed; returns the seconds spent."""
+    import numpy as np
+    from oracle import model, plan_io, prefill
+    from quantized_recurrent_state_b200 import synth
+    plan_bytes, wname, heads, T = payload
+    pv = model.PlanView(plan_io.read_plan(plan_bytes))
+    wl = synth.workloads()[wname]
+    alpha = synth.gates(wl, wl.seed)
+    layers = sorted({l for l, _ in heads})
+    steps = [synth.step_inputs(wl, wl.seed, 1, t, alpha=alpha, layers=layers) for t in range(T)]
+    seq = {k: np.stack([st[k][0] for st in steps]) for k in steps[0]}   # [T, nL, H(, D)]
+    slot = np.zeros(pv.slot_bytes, np.uint8)
+    for l in layers:
+        S0 = synth.initial_states(wl, wl.seed, 1, layers=[l])
+        for (l2, h) in heads:
+            if l2 == l:
+                pv.quantize_into(slot, l, h, S0[0, 0, h])
+    t0 = time.perf_counter()
+    for (l, h) in heads:
+        li = layers.index(l)
+        S = pv.reconstruct(slot, l, h).astype(np.float64)
+        _, S_T = prefill.chunked(S, seq["q"][:, li, h], seq["k"][:, li, h], seq["v"][:, li, h],
+                                 seq["alpha"][:, li, h], seq["beta"][:, li, h])
+        pv.quantize_into(slot, l, h, S_T)
+    return time.perf_counter() - t0
+
+
+def cpu_prefill_rate(plan_bytes, wl, n_heads, T, pool, cores):
+    """Tokens/s (a token through all L*H heads) of the oracle's packed prefill
+    over a sample of n_heads heads, split across the worker processes; the
+    time is the slowest worker's."""
+    heads = [(l, h) for l in range(wl.n_layers) for h in range(wl.n_heads)][:n_heads]
+    chunks = [heads[i::cores] for i in range(cores)]
+    secs = max(pool.map(_oracle_prefill_sample, [(plan_bytes, wl.name, c, T) for c in chunks if c]))
+    return len(heads) * T / (wl.n_layers * wl.n_heads) / secs, len(heads), secs
+
+
+def cpu_prefill_baseline(plan_bytes, wl, budget_s=12.0):
+    cores = _n_cores()
+    T = PREFILL_CPU_TOKENS
+    per_head = _oracle_prefill_sample((plan_bytes, wl.name, [(0, 0)], T))
+    nh = int(min(wl.n_layers * wl.n_heads, max(cores, budget_s / max(per_head, 1e-4))))
+    with oracle_pool(cores) as pool:
+        rate, nh, _ = cpu_prefill_rate(plan_bytes, wl, nh, T, pool, cores)
+    return {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{nh} (layer, head) states of request 0, a {T}-token chunk each (reconstruct, fp64 chunk "
+                      f"form, requantize), split over {cores} spawned processes; tokens/s of a token through all "
+                      f"{wl.n_layers * wl.n_heads} heads, time = slowest process"}
+
+
 def _oracle_calib_layer(payload):
     """Oracle calibration statistics of one layer (all its heads)."""
     from oracle import model
@@ -651,6 +908,15 @@ def _n_cores():
     return max(1, min(os.cpu_count() or 1, 32))
 
 
+def oracle_pool(cores: int):
+    """`cores` spawned worker processes, each with one BLAS thread, so that
+    the oracle uses exactly `cores` threads."""
+    import multiprocessing as mp
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[var] = "1"   # read by the workers' numpy at import
+    return mp.get_context("spawn").Pool(cores)
+
+
 def cpu_sample_rate(plan_bytes, wl, heads_per_step, t, pool, cores):
     """Head-steps/s of the oracle over one sample: heads split across the
     worker processes; the step time is the slowest worker's stepping time."""
@@ -664,15 +930,61 @@ def cpu_baseline(plan_bytes, wl, budget_s=12.0):
     """The oracle, as it stands, on the host cores: a bounded sample of the
     same workload (request 0's heads in layer order, one decode step each)
     sized to about budget_s seconds of CPU work in total."""
-    import multiprocessing as mp
     cores = _n_cores()
     per_head = _oracle_sample((plan_bytes, wl.name, [(0, 0)], 0))
     heads = int(min(wl.n_layers * wl.n_heads, max(cores, budget_s / max(per_head, 1e-4))))
-    with mp.get_context("spawn").Pool(cores) as pool:
+    with oracle_pool(cores) as pool:
         nh, sec = cpu_sample_rate(plan_bytes, wl, heads, 0, pool, cores)
     return {"value": nh / sec, "unit": "head-steps/s", "cores": cores, "kind": "oracle",
             "sample": f"{nh} (layer, head) states of request 0, one decode step each, split over {cores} "
                       f"spawned processes; time = slowest process's stepping time"}
+
+
+def oracle_plan_bytes(wl, pool):
+    """The workload's plan from the oracle's calibration and allocator (one
+    worker per layer)."""
+    from oracle import model, plan_io
+    layer_stats = pool.map(_oracle_calib_layer, [(wl.name, l) for l in range(wl.n_layers)])
+    stats = {k: np.concatenate([np.asarray(s[k]).reshape((1,) + np.asarray(s[k]).shape[1:])
+                                if k in ("wbar", "rho") else np.asarray(s[k]) for s in layer_stats])
+             for k in ("wbar", "rho", "lgate", "dist")}
+    plan = model.build_plan(wl.mode, wl.d, wl.n_layers, wl.n_heads, stats, wl.bits, wl.nominal_bits,
+                            wl.n_pivots, wl.horizon)
+    return plan_io.write_plan(None, plan)
+
+
+def run_reference_prefill(args):
+    """The CPU oracle's packed prefill as the reference arm of --prefill:
+    each step a bounded sample of (layer, head) states of one request, a
+    PREFILL_CPU_TOKENS-token chunk each."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from quantized_recurrent_state_b200 import synth
+    wl = workload_of(args, synth)
+    cores = _n_cores()
+    T = PREFILL_CPU_TOKENS
+    with oracle_pool(cores) as pool:
+        plan_bytes = oracle_plan_bytes(wl, pool)
+        for _ in range(args.warmup):
+            cpu_prefill_rate(plan_bytes, wl, cores, T, pool, cores)
+        tot_tok, tot_s = 0.0, 0.0
+        for _ in range(args.steps):
+            rate, nh, sec = cpu_prefill_rate(plan_bytes, wl, cores, T, pool, cores)
+            tot_tok += rate * sec
+            tot_s += sec
+    value = tot_tok / tot_s
+    sample = (f"each step: {cores} (layer, head) states of one request, a {T}-token chunk each, split over "
+              f"{cores} spawned processes (time = slowest process); tokens/s of a token through all "
+              f"{wl.n_layers * wl.n_heads} heads")
+    out = {"impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic",
+           "config": {**prefill_config(wl, args.batch, args.prefill, args.gpus), "variant": "oracle (CPU)"},
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
 
 
 def run_reference(args):
@@ -681,19 +993,11 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    import multiprocessing as mp
-    from oracle import model, plan_io
     from quantized_recurrent_state_b200 import synth
     wl = workload_of(args, synth)
     cores = _n_cores()
-    with mp.get_context("spawn").Pool(cores) as pool:
-        layer_stats = pool.map(_oracle_calib_layer, [(wl.name, l) for l in range(wl.n_layers)])
-        stats = {k: np.concatenate([np.asarray(s[k]).reshape((1,) + np.asarray(s[k]).shape[1:])
-                                    if k in ("wbar", "rho") else np.asarray(s[k]) for s in layer_stats])
-                 for k in ("wbar", "rho", "lgate", "dist")}
-        plan = model.build_plan(wl.mode, wl.d, wl.n_layers, wl.n_heads, stats, wl.bits, wl.nominal_bits,
-                                wl.n_pivots, wl.horizon)
-        plan_bytes = plan_io.write_plan(None, plan)
+    with oracle_pool(cores) as pool:
+        plan_bytes = oracle_plan_bytes(wl, pool)
         heads_per_step = 4 * cores
         for i in range(args.warmup):
             cpu_sample_rate(plan_bytes, wl, heads_per_step, i, pool, cores)
@@ -718,7 +1022,11 @@ def run_reference(args):
 
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.prefill:
+        if args.workload != "gdn":
+            raise SystemExit("--prefill: per-head (GDN) units only")
+        (run_reference_prefill if args.impl == "reference" else run_prefill)(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_product(args)

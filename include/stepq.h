@@ -194,8 +194,6 @@ void stepq_ctx_free(stepq_ctx *ctx);
  * requests over nL layers (= n_req*nL*n_heads*d*4). */
 size_t stepq_workspace_bytes(const stepq_ctx *ctx, int n_req, int n_layers_launched);
 
-/* ---- the decode step (方法-4) --------------------------------------------- */
-
 /* ---- prefill (the step before decode) ----------------------------------- */
 
 /* Chunked prefill of T tokens on fp32 states (per-head units, d = 128):
@@ -215,14 +213,18 @@ size_t stepq_workspace_bytes(const stepq_ctx *ctx, int n_req, int n_layers_launc
 int stepq_prefill_fp32(stepq_ctx *ctx, float *S, int n_req, int lb, int le, int T, const float *q,
                        const float *k, const float *v, const float *alpha, const float *beta, float *o,
                        int zero_init);
-/* Bytes of the fp32 workspace stepq_prefill needs: one layer's states of the
- * batch (n_req * n_heads * D * D * 4). */
-size_t stepq_prefill_workspace_bytes(const stepq_ctx *ctx, int n_req);
-/* Prefill into packed states: per layer, the pool records of the slots are
- * unpacked into the workspace (from_zero: S_0 = 0 instead), prefilled as in
- * stepq_prefill_fp32, and requantized into the pool (the plan's requantizer).
- * Same input layouts; enqueued on main after the side stream's last work on
- * those layers. */
+/* Bytes of the fp32 workspace stepq_prefill needs for n_layers layers of the
+ * batch (n_req * n_layers * n_heads * D * D * 4); 0 for a null context or a
+ * negative count. */
+size_t stepq_prefill_workspace_bytes(const stepq_ctx *ctx, int n_req, int n_layers);
+/* Prefill into packed states: the pool records of (slots, layers [lb, le))
+ * are unpacked into the workspace (from_zero: S_0 = 0 instead), prefilled as
+ * in stepq_prefill_fp32, and requantized into the pool (the plan's
+ * requantizer): three launches over the whole range.  The workspace, of
+ * stepq_prefill_workspace_bytes(ctx, n_req, le - lb) bytes and owned by the
+ * caller, holds the final fp32 states [n_req][le-lb][n_heads][D][D] on
+ * return.  Same input layouts; enqueued on main after the side stream's last
+ * work on those layers. */
 int stepq_prefill(stepq_ctx *ctx, void *pool, const int32_t *slots, int n_req, int lb, int le, int T,
                   const float *q, const float *k, const float *v, const float *alpha, const float *beta,
                   float *o, float *workspace, int from_zero);
@@ -231,6 +233,8 @@ int stepq_prefill(stepq_ctx *ctx, void *pool, const int32_t *slots, int n_req, i
  * the requantizer of the header comment (used for S_0).  Enqueued on main. */
 int stepq_requant_pack(stepq_ctx *ctx, void *pool, const int32_t *slots, int n_req, int lb, int le,
                        const float *S);
+
+/* ---- the decode step (方法-4) --------------------------------------------- */
 
 /* One decode step over (slots, layers [lb, le), all heads), two streams:
  * per layer chunk, the decode kernel (reconstruct -> retention + delta ->
@@ -320,8 +324,8 @@ uint64_t stepq_launch_count(const stepq_ctx *ctx);
 /* Kernel timing.  While enabled, every launch of the context is bracketed by
  * two CUDA events on the stream it runs on.  stepq_kernel_stats waits for
  * them, adds up the device time per kernel kind (0 decode, 1 fit-pack,
- * 2 fused, 3 pack/unpack/fp32/calibration), writes ms[4] and launches[4]
- * (host arrays) and forgets the recorded launches. */
+ * 2 fused, 3 pack/unpack/fp32/calibration, 4 chunked prefill), writes
+ * ms[5] and launches[5] (host arrays) and forgets the recorded launches. */
 int stepq_ctx_set_timing(stepq_ctx *ctx, int enable);
 /* Bounded copy waits of the step kernels.  Every wait of a kernel on its
  * shared-memory copies gives up after `polls` polls of the barrier (0: the

@@ -25,6 +25,7 @@
 
 #include "../../include/stepq.h"
 #include "stepq_dev.cuh"
+#include "stepq_prefill.cuh"
 
 namespace stepq {
 cudaError_t launch_step(int kind, int D, const Args &a, int n_sms, cudaStream_t st, int *grid);
@@ -1019,16 +1020,16 @@ extern "C" int stepq_prefill_fp32(stepq_ctx *c, float *S, int n_req, int lb, int
     a.S = S; a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.o = o;
     a.n_req = n_req; a.T = T; a.nL = le - lb; a.nL_in = le - lb; a.l_in0 = 0; a.H = c->plan->H;
     a.zero_init = zero_init ? 1 : 0;
-    LaunchTimer lt(c, 3, c->main);
+    LaunchTimer lt(c, 4, c->main);
     const cudaError_t e = stepq::launch_prefill(a, c->main);
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
     lt.done();
     return STEPQ_OK;
 }
 
-extern "C" size_t stepq_prefill_workspace_bytes(const stepq_ctx *c, int n_req) {
-    if (!c) return 0;
-    return (size_t)n_req * c->plan->H * c->plan->D * c->plan->D * sizeof(float);
+extern "C" size_t stepq_prefill_workspace_bytes(const stepq_ctx *c, int n_req, int n_layers) {
+    if (!c || n_req < 0 || n_layers < 0) return 0;
+    return (size_t)n_req * n_layers * c->plan->H * c->plan->D * c->plan->D * sizeof(float);
 }
 
 extern "C" int stepq_prefill(stepq_ctx *c, void *pool, const int32_t *slots, int n_req, int lb, int le, int T,
@@ -1047,33 +1048,32 @@ extern "C" int stepq_prefill(stepq_ctx *c, void *pool, const int32_t *slots, int
     if ((rc = set_device(c))) return rc;
     if (n_req == 0 || T == 0) return STEPQ_OK;
     if ((rc = wait_side(c, lb, le))) return rc;
-    // one layer at a time: state -> fp32 workspace, the chunked prefill, requantize into the pool
-    for (int l = lb; l < le; ++l) {
-        stepq::Args a = base_args(c, pool, slots, n_req, l, l + 1);
-        cudaError_t e = cudaSuccess;
-        if (!from_zero) {
-            a.S_out = workspace;
-            LaunchTimer lt(c, 3, c->main);
-            e = stepq::launch_pack(c->plan->D, a, true, c->main);
-            if (e != cudaSuccess) return cuda_fail(e, "prefill: unpack launch");
-            lt.done();
-        }
-        stepq::PrefillArgs p{};
-        p.S = workspace; p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta; p.o = o;
-        p.n_req = n_req; p.T = T; p.nL = 1; p.nL_in = le - lb; p.l_in0 = l - lb; p.H = c->plan->H;
-        p.zero_init = from_zero ? 1 : 0;
-        {
-            LaunchTimer lt(c, 3, c->main);
-            e = stepq::launch_prefill(p, c->main);
-            if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
-            lt.done();
-        }
-        a.S_in = workspace;
+    // the whole layer range at once (n_req * layers * H CTAs per launch): states -> fp32
+    // workspace, the chunked prefill, requantize into the pool
+    stepq::Args a = base_args(c, pool, slots, n_req, lb, le);
+    cudaError_t e = cudaSuccess;
+    if (!from_zero) {
+        a.S_out = workspace;
         LaunchTimer lt(c, 3, c->main);
-        e = stepq::launch_pack(c->plan->D, a, false, c->main);
-        if (e != cudaSuccess) return cuda_fail(e, "prefill: requant_pack launch");
+        e = stepq::launch_pack(c->plan->D, a, true, c->main);
+        if (e != cudaSuccess) return cuda_fail(e, "prefill: unpack launch");
         lt.done();
     }
+    stepq::PrefillArgs p{};
+    p.S = workspace; p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta; p.o = o;
+    p.n_req = n_req; p.T = T; p.nL = le - lb; p.nL_in = le - lb; p.l_in0 = 0; p.H = c->plan->H;
+    p.zero_init = from_zero ? 1 : 0;
+    {
+        LaunchTimer lt(c, 4, c->main);
+        e = stepq::launch_prefill(p, c->main);
+        if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+        lt.done();
+    }
+    a.S_in = workspace;
+    LaunchTimer lt(c, 3, c->main);
+    e = stepq::launch_pack(c->plan->D, a, false, c->main);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill: requant_pack launch");
+    lt.done();
     return STEPQ_OK;
 }
 
@@ -1137,7 +1137,7 @@ extern "C" int stepq_kernel_stats(stepq_ctx *c, double *ms, uint64_t *launches) 
     if (!c || !ms || !launches) return fail(STEPQ_EINVAL, "kernel_stats: null argument");
     int rc = set_device(c);
     if (rc) return rc;
-    for (int k = 0; k < 4; ++k) { ms[k] = 0.0; launches[k] = 0; }
+    for (int k = 0; k < 5; ++k) { ms[k] = 0.0; launches[k] = 0; }
     for (auto &t : c->timed) {
         cudaError_t e = cudaEventSynchronize(t.b);
         if (e != cudaSuccess) return cuda_fail(e, "kernel_stats: cudaEventSynchronize");

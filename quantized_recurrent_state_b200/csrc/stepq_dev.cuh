@@ -67,16 +67,6 @@ struct Args {
     uint32_t rec_stage_bytes;// bytes reserved for the record in a stage
 };
 
-// Arguments of the chunked prefill (per-head units, d = 128).
-struct PrefillArgs {
-    float *S;                  // [n_req][nL][H][D][D] fp32 states, read (unless zero_init) and written
-    const float *q, *k, *v;    // [n_req][T][nL_in][H][D]
-    const float *alpha, *beta; // [n_req][T][nL_in][H]
-    float *o;                  // [n_req][T][nL_in][H][D]
-    int n_req, T, nL, nL_in, l_in0, H;
-    int zero_init;
-};
-
 // Tail of a pipeline stage (after the staged record), in 4-byte words of D:
 // q, k, v, x (the w workspace), rho, wbar, the per-row alpha (per-row
 // records), row byte offsets (per-row records), then D bytes of row widths

@@ -18,6 +18,7 @@
 // and the chunk's Q, K, V in shared memory (rows padded to avoid bank
 // conflicts).  Head dimension 128.
 #include "stepq_dev.cuh"
+#include "stepq_prefill.cuh"
 
 namespace stepq {
 

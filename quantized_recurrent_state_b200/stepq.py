@@ -78,7 +78,7 @@ def lib():
         l.stepq_plan_slice.argtypes = [P, I, I, ctypes.POINTER(P)]
         l.stepq_prefill_fp32.argtypes = [P, P, I, I, I, I, P, P, P, P, P, P, I]
         l.stepq_prefill.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, P, P, I]
-        l.stepq_prefill_workspace_bytes.argtypes = [P, I]
+        l.stepq_prefill_workspace_bytes.argtypes = [P, I, I]
         l.stepq_prefill_workspace_bytes.restype = ctypes.c_size_t
         l.stepq_ctx_create.argtypes = [P, P, P, I, I, ctypes.POINTER(P)]
         l.stepq_ctx_free.argtypes = [P]
@@ -256,8 +256,8 @@ class Context:
         return _check(lib().stepq_prefill_fp32(self._h, _ptr(S), n_req, lb, le, int(T), _ptr(q), _ptr(k), _ptr(v),
                                                _ptr(alpha), _ptr(beta), _ptr(o), 1 if zero_init else 0))
 
-    def prefill_workspace_bytes(self, n_req: int) -> int:
-        return int(lib().stepq_prefill_workspace_bytes(self._h, n_req))
+    def prefill_workspace_bytes(self, n_req: int, n_layers: int) -> int:
+        return int(lib().stepq_prefill_workspace_bytes(self._h, n_req, n_layers))
 
     def prefill(self, pool, slots, n_req, lb, le, T, q, k, v, alpha, beta, o, workspace, from_zero=False):
         self._after_caller()
@@ -286,11 +286,11 @@ class Context:
 
     def kernel_stats(self):
         """{kind: (total ms, launches)} of the launches timed since the last call."""
-        ms = (ctypes.c_double * 4)()
-        n = (ctypes.c_uint64 * 4)()
+        ms = (ctypes.c_double * 5)()
+        n = (ctypes.c_uint64 * 5)()
         _check(lib().stepq_kernel_stats(self._h, ms, n))
-        names = ("decode", "fitpack", "fused", "other")
-        return {names[i]: (float(ms[i]), int(n[i])) for i in range(4)}
+        names = ("decode", "fitpack", "fused", "other", "prefill")
+        return {names[i]: (float(ms[i]), int(n[i])) for i in range(5)}
 
     @property
     def launches(self) -> int:

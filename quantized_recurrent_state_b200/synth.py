@@ -58,16 +58,20 @@ def _bits_np(key: int, n: int, start: int = 0) -> np.ndarray:
     return z
 
 
-def uniform_np(key: int, shape) -> np.ndarray:
+def uniform_np(key: int, shape, start: int = 0) -> np.ndarray:
+    """Elements start .. start + size - 1 of the stream."""
     n = int(np.prod(shape))
-    z = _bits_np(key, n)
+    z = _bits_np(key, n, start)
     return ((z >> np.uint64(11)).astype(np.float64) * 2.0 ** -53).reshape(shape)
 
 
-def normal_np(key: int, shape) -> np.ndarray:
+def normal_np(key: int, shape, start: int = 0) -> np.ndarray:
+    """Elements start .. start + size - 1 of the stream (Box-Muller pairs, so
+    start must be even)."""
+    assert start % 2 == 0
     n = int(np.prod(shape))
     m = (n + 1) // 2
-    z = _bits_np(key, 2 * m)
+    z = _bits_np(key, 2 * m, start)
     u1 = ((z[0::2] >> np.uint64(11)).astype(np.float64) + 1.0) * 2.0 ** -53
     u2 = (z[1::2] >> np.uint64(11)).astype(np.float64) * 2.0 ** -53
     rad = np.sqrt(-2.0 * np.log(u1))
@@ -153,6 +157,23 @@ def step_inputs_torch(wl: "Workload", seed: int, n_req: int, t: int, alpha: np.n
     al = al.unsqueeze(0).expand((n_req,) + tuple(al.shape)).contiguous()
     return dict(q=q.float().contiguous(), k=k.float().contiguous(), v=v.float().contiguous(),
                 alpha=al.float().contiguous(), beta=beta.float().contiguous())
+
+
+def prompt_inputs_torch(wl: "Workload", seed: int, n_req: int, t0: int, T: int, alpha: np.ndarray, device,
+                        lb: int = 0, le: int = None) -> dict:
+    """Tokens t0 .. t0 + T - 1 of step_inputs_torch as one prompt for layers
+    [lb, le): q, k, v [n_req, T, le - lb, H, D], alpha, beta [n_req, T, le - lb, H]."""
+    import torch
+    le = wl.n_layers if le is None else le
+    out = None
+    for t in range(T):
+        s = step_inputs_torch(wl, seed, n_req, t0 + t, alpha, device)
+        if out is None:
+            out = {k: torch.empty((n_req, T) + tuple(v[:, lb:le].shape[1:]), dtype=v.dtype, device=device)
+                   for k, v in s.items()}
+        for k in out:
+            out[k][:, t] = s[k][:, lb:le]
+    return out
 
 
 # ---- workloads -------------------------------------------------------------
@@ -254,14 +275,19 @@ def step_inputs(wl: Workload, seed: int, n_req: int, t: int, alpha: np.ndarray =
                 layers=None) -> dict:
     """Inputs of decode step t: q, k, v [n_req, nL, H, D], alpha, beta."""
     layers = list(range(wl.n_layers) if layers is None else layers)
-    nL = len(layers)
-    shape = (n_req, wl.n_layers, wl.n_heads, wl.d)
-    q = normal_np(stream_key(seed, S_Q, t), shape)[:, layers]
-    n = normal_np(stream_key(seed, S_K, t), shape)[:, layers]
+    L, H, D = wl.n_layers, wl.n_heads, wl.d
+
+    def blocks(gen, key, blk):
+        # the (request, layer) blocks of the [n_req, L, ...] stream that are asked for
+        return np.stack([np.stack([gen(key, (blk,), start=(r * L + l) * blk) for l in layers])
+                         for r in range(n_req)])
+
+    q = blocks(normal_np, stream_key(seed, S_Q, t), H * D).reshape(n_req, len(layers), H, D)
+    n = blocks(normal_np, stream_key(seed, S_K, t), H * D).reshape(n_req, len(layers), H, D)
     k = n / np.sqrt((n * n).sum(axis=-1, keepdims=True))
     gam = column_scales(wl, seed)[layers]
-    v = normal_np(stream_key(seed, S_V, t), shape)[:, layers] * gam[None]
-    beta = uniform_np(stream_key(seed, S_BETA, t), (n_req, wl.n_layers, wl.n_heads))[:, layers]
+    v = blocks(normal_np, stream_key(seed, S_V, t), H * D).reshape(n_req, len(layers), H, D) * gam[None]
+    beta = blocks(uniform_np, stream_key(seed, S_BETA, t), H).reshape(n_req, len(layers), H)
     if alpha is None:
         alpha = gates(wl, seed)
     a = alpha[layers]

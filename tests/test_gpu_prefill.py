@@ -16,7 +16,7 @@ import pytest
 
 from oracle import model, prefill
 from quantized_recurrent_state_b200 import synth
-from tests._workloads import oracle_plan
+from tests._workloads import oracle_plan, uniform_plan
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -40,9 +40,9 @@ def _prompt(wl, n, T, seed):
     return {key: np.ascontiguousarray(np.stack([s[key] for s in steps], axis=1)) for key in steps[0]}
 
 
-def _check_head(O_gpu, S_gpu, S0, inp, r, h):
-    O_ref, S_ref = prefill.sequential(S0, inp["q"][r, :, 0, h], inp["k"][r, :, 0, h], inp["v"][r, :, 0, h],
-                                      inp["alpha"][r, :, 0, h], inp["beta"][r, :, 0, h])
+def _check_head(O_gpu, S_gpu, S0, inp, r, h, l=0):
+    O_ref, S_ref = prefill.sequential(S0, inp["q"][r, :, l, h], inp["k"][r, :, l, h], inp["v"][r, :, l, h],
+                                      inp["alpha"][r, :, l, h], inp["beta"][r, :, l, h])
     eo = np.max(np.abs(O_gpu - O_ref)) / max(1e-30, np.max(np.abs(O_ref)))
     es = np.max(np.abs(S_gpu - S_ref)) / max(1e-30, np.max(np.abs(S_ref)))
     assert eo <= TOL and es <= TOL, (r, h, eo, es)
@@ -104,7 +104,7 @@ def test_prefill_into_packed_states(stepq, from_zero):
     inp = _prompt(wl, n, T, 77)
     d = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
     o = torch.zeros_like(d["q"])
-    ws = torch.empty(ctx.prefill_workspace_bytes(n) // 4, dtype=torch.float32, device="cuda")
+    ws = torch.empty(ctx.prefill_workspace_bytes(n, 1) // 4, dtype=torch.float32, device="cuda")
     ctx.prefill(pool, slots, n, 0, 1, T, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o, ws, from_zero=from_zero)
     ctx.sync()
     after, og = pool.cpu().numpy(), o.cpu().numpy()
@@ -122,3 +122,41 @@ def test_prefill_into_packed_states(stepq, from_zero):
             assert np.array_equal(pv.record(new_slot, 0, h), pv.record(expect, 0, h)), (r, h)
     for s in (1, 3):   # slots outside the batch are untouched
         assert np.array_equal(after[s * sb:(s + 1) * sb], before[s * sb:(s + 1) * sb])
+
+
+def test_prefill_layer_range_uniform_plan(stepq):
+    """Layers [1, 3) of a three-layer uniform 6-bit plan (dual-axis), inputs
+    laid out for the range only; layer 0 and slots outside the batch stay put."""
+    plan, data, wl, _ = uniform_plan("qwen_pool6", 6, model.QUANT_DUAL_AXIS, n_layers=3)
+    pv = model.PlanView(plan)
+    P = stepq.Plan.from_bytes(data)
+    n, T, lb, le = 2, 70, 1, 3
+    ctx = stepq.Context(P, 3)
+    slots = torch.tensor([2, 0], dtype=torch.int32, device="cuda")
+    pool = torch.zeros(3 * P.slot_bytes, dtype=torch.uint8, device="cuda")
+    S0 = synth.initial_states(wl, wl.seed, n)
+    ctx.requant_pack(pool, slots, n, 0, 3, torch.from_numpy(S0).cuda())
+    ctx.sync()
+    before = pool.cpu().numpy().copy()
+    inp = {k: np.ascontiguousarray(v[:, :, lb:le]) for k, v in _prompt(wl, n, T, 5).items()}
+    d = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
+    o = torch.zeros_like(d["q"])
+    ws = torch.empty(ctx.prefill_workspace_bytes(n, le - lb) // 4, dtype=torch.float32, device="cuda")
+    assert ctx.prefill_workspace_bytes(n, le - lb) == n * (le - lb) * wl.n_heads * wl.d * wl.d * 4
+    ctx.prefill(pool, slots, n, lb, le, T, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o, ws)
+    ctx.sync()
+    after, og = pool.cpu().numpy(), o.cpu().numpy()
+    S_T = ws.view(n, le - lb, wl.n_heads, wl.d, wl.d).cpu().numpy()
+    sb = P.slot_bytes
+    for r, s in enumerate((2, 0)):
+        prev_slot, new_slot = before[s * sb:(s + 1) * sb], after[s * sb:(s + 1) * sb]
+        for h in range(wl.n_heads):
+            assert np.array_equal(pv.record(new_slot, 0, h), pv.record(prev_slot, 0, h))
+        for li, l in enumerate(range(lb, le)):
+            for h in (1, 20, 47):
+                S_start = pv.reconstruct(prev_slot, l, h).astype(np.float64)
+                _check_head(og[r, :, li, h], S_T[r, li, h], S_start, inp, r, h, li)
+                expect = np.zeros_like(new_slot)
+                pv.quantize_into(expect, l, h, S_T[r, li, h])
+                assert np.array_equal(pv.record(new_slot, l, h), pv.record(expect, l, h)), (r, l, h)
+    assert np.array_equal(after[sb:2 * sb], before[sb:2 * sb])
