@@ -27,15 +27,22 @@ namespace pf {
 constexpr int D = 128;         // d_k = d_v
 constexpr int C = 64;          // tokens per chunk
 constexpr int NT = 256;        // threads
-constexpr int SD = D + 4;      // padded row of a 128-wide tile
-constexpr int SC = C + 4;      // padded row of a 64-wide tile
+constexpr int SD = D + 4;      // row of K, Q: read as A (row, k) and as B (n, k) fragments
+constexpr int SV = D + 8;      // row of S, V: read as B (k, n) fragments
+constexpr int SC = C + 4;      // row of M
+
+// Row strides in 4-byte words, chosen so that a warp's fragment loads hit 32
+// distinct banks: an A fragment reads (g, t) at g * stride + t (stride = 4
+// mod 32), a B fragment from a row-major [k][n] tile reads (t, g) at
+// t * stride + g (stride = 8 mod 32); g < 8, t < 4.
+static_assert(SD % 32 == 4 && SC % 32 == 4 && SV % 32 == 8, "bank-conflict-free strides");
 
 struct Smem {
-    float S[D * SD];           // state, row i (key) x column j (value)
-    float K[C * SD];
+    float S[D * SV];           // state, row i (key) x column j (value)
+    float K[2][C * SD];        // this chunk's K and the next chunk's, fetched ahead
     float Q[C * SD];
-    float V[C * SD];           // V, then R = V - diag(gamma) K S, then U
-    float M[C * SC];           // M (strict lower), then A (lower incl.)
+    float V[C * SV];           // V, then R = V - diag(gamma) K S, then U
+    float M[C * SC];           // M (strict lower; diagonal 16 x 16 blocks then (I + M_bb)^-1), then A
     float lg[C];               // inclusive running sum of log alpha in the chunk
     float beta[C];
     float f[C];                // beta_s gamma_C / gamma_s
@@ -52,39 +59,57 @@ __device__ __forceinline__ void split(float x, uint32_t &hi, uint32_t &lo) {
     lo = tf32(x - __uint_as_float(hi));
 }
 
+// Not volatile: a pure function of its operands, so the compiler may
+// interleave independent tiles.
 __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// acc[nt] += A[m0 .. m0+16, 0 .. KK) B[0 .. KK, n0 + 8 nt .. + 8) for one warp.
-// A(r, c) = sA[r ars + c acs]; B(r, c) = sB[r brs + c bcs] (times bsc[r] when given).
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp16(float *dst, const float *src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+// acc[nt] += A[m0 .. m0+16, 0 .. kk) B[0 .. kk, n0 + 8 nt .. + 8) for one warp, kk a multiple of 8.
+// A(r, c) = sA[r ars + c acs] (times asc[c] when given); B(r, c) = sB[r brs + c bcs].
 // Fragment of acc[nt]: [0] (m0+g, n0+8nt+2t), [1] (.., +1), [2] (m0+g+8, ..), [3] (.., +1).
-template <int NTILE, int KK>
-__device__ __forceinline__ void warp_gemm(float (&acc)[NTILE][4], const float *sA, int ars, int acs, const float *sB,
-                                          int brs, int bcs, const float *bsc, int m0, int n0, int lane) {
+// Each product is hi*hi + hi*lo + lo*hi of the TF32 splits, issued as three
+// passes over the n-tiles so that consecutive MMAs never share an accumulator.
+template <int NTILE>
+__device__ __forceinline__ void warp_gemm(float (&acc)[NTILE][4], const float *sA, int ars, int acs, const float *asc,
+                                          const float *sB, int brs, int bcs, int m0, int n0, int kk, int lane) {
     const int g = lane >> 2, t = lane & 3;
-#pragma unroll 1
-    for (int k0 = 0; k0 < KK; k0 += 8) {
+#pragma unroll 2
+    for (int k0 = 0; k0 < kk; k0 += 8) {
+        float x[4];
+        x[0] = sA[(m0 + g) * ars + (k0 + t) * acs];
+        x[1] = sA[(m0 + g + 8) * ars + (k0 + t) * acs];
+        x[2] = sA[(m0 + g) * ars + (k0 + t + 4) * acs];
+        x[3] = sA[(m0 + g + 8) * ars + (k0 + t + 4) * acs];
+        if (asc) {
+            const float s0 = asc[k0 + t], s1 = asc[k0 + t + 4];
+            x[0] *= s0; x[1] *= s0; x[2] *= s1; x[3] *= s1;
+        }
         uint32_t ah[4], al[4];
-        split(sA[(m0 + g) * ars + (k0 + t) * acs], ah[0], al[0]);
-        split(sA[(m0 + g + 8) * ars + (k0 + t) * acs], ah[1], al[1]);
-        split(sA[(m0 + g) * ars + (k0 + t + 4) * acs], ah[2], al[2]);
-        split(sA[(m0 + g + 8) * ars + (k0 + t + 4) * acs], ah[3], al[3]);
-        const float s0 = bsc ? bsc[k0 + t] : 1.0f, s1 = bsc ? bsc[k0 + t + 4] : 1.0f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) split(x[u], ah[u], al[u]);
+        uint32_t bh[NTILE][2], bl[NTILE][2];
 #pragma unroll
         for (int nt = 0; nt < NTILE; ++nt) {
             const int n = n0 + 8 * nt + g;
-            uint32_t bh[2], bl[2];
-            split(sB[(k0 + t) * brs + n * bcs] * s0, bh[0], bl[0]);
-            split(sB[(k0 + t + 4) * brs + n * bcs] * s1, bh[1], bl[1]);
-            mma(acc[nt], ah, bh);
-            mma(acc[nt], ah, bl);
-            mma(acc[nt], al, bh);
+            split(sB[(k0 + t) * brs + n * bcs], bh[nt][0], bl[nt][0]);
+            split(sB[(k0 + t + 4) * brs + n * bcs], bh[nt][1], bl[nt][1]);
         }
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt) mma(acc[nt], ah, bh[nt]);
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt) mma(acc[nt], ah, bl[nt]);
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt) mma(acc[nt], al, bh[nt]);
     }
 }
 
@@ -106,32 +131,50 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
     const int per_req = a.nL * a.H;
     const int n = item / per_req, rem = item - n * per_req, ll = rem / a.H, h = rem - ll * a.H;
     float *Sg = a.S + (size_t)item * D * D;
+    // element offset of token tok's row of this (request, layer, head) in q, k, v, o
+    auto row_of = [&](int tok) { return (((size_t)(n * a.T + tok) * a.nL_in + a.l_in0 + ll) * a.H + h) * D; };
+    // the q, k, v rows of the chunk from token c0 into L2 ahead of their loads
+    auto prefetch_chunk = [&](int c0) {
+        const int cc = min(C, a.T - c0);
+        if (tid < 3 * cc) {
+            const int r = tid / 3, which = tid - 3 * r;
+            const float *base = which == 0 ? a.k : which == 1 ? a.q : a.v;
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + row_of(c0 + r)), "r"(D * 4)
+                         : "memory");
+        }
+    };
 
+    // asynchronous copy of the chunk from token c0 of one of q, k, v into rows of buf (zeros past T)
+    auto fetch_rows = [&](float *buf, int stride, const float *base, int c0) {
+        const int cc = min(C, a.T - c0);
+        for (int e = tid; e < C * D / 4; e += NT) {
+            const int r = e / (D / 4), j4 = e % (D / 4);
+            const bool ok = r < cc;
+            cp16(buf + r * stride + 4 * j4, ok ? base + row_of(c0 + r) + 4 * j4 : base, ok ? 16 : 0);
+        }
+    };
+
+    prefetch_chunk(0);
+    fetch_rows(sm.K[0], SD, a.k, 0);
+    fetch_rows(sm.Q, SD, a.q, 0);
+    cp_async_commit();
     // the state
     for (int e = tid; e < D * D / 4; e += NT) {
         const int i = e / (D / 4), j4 = e % (D / 4);
         const float4 x = a.zero_init ? make_float4(0.f, 0.f, 0.f, 0.f) : reinterpret_cast<const float4 *>(Sg)[e];
-        *reinterpret_cast<float4 *>(&sm.S[i * SD + 4 * j4]) = x;
+        *reinterpret_cast<float4 *>(&sm.S[i * SV + 4 * j4]) = x;
     }
 
-    for (int c0 = 0; c0 < a.T; c0 += C) {
+#pragma unroll 1
+    for (int c0 = 0, ci = 0; c0 < a.T; c0 += C, ++ci) {
         const int cc = min(C, a.T - c0);
-        __syncthreads();  // the previous chunk is done with K, Q, V, M
-        // 1. the chunk's rows (padded rows: zeros, alpha = 1, beta = 0)
-        for (int e = tid; e < C * D / 4; e += NT) {
-            const int r = e / (D / 4), j4 = e % (D / 4);
-            float4 kx = make_float4(0.f, 0.f, 0.f, 0.f), qx = kx, vx = kx;
-            if (r < cc) {
-                const size_t row = ((size_t)(n * a.T + c0 + r) * a.nL_in + a.l_in0 + ll) * a.H + h;
-                kx = reinterpret_cast<const float4 *>(a.k + row * D)[j4];
-                qx = reinterpret_cast<const float4 *>(a.q + row * D)[j4];
-                vx = reinterpret_cast<const float4 *>(a.v + row * D)[j4];
-            }
-            *reinterpret_cast<float4 *>(&sm.K[r * SD + 4 * j4]) = kx;
-            *reinterpret_cast<float4 *>(&sm.Q[r * SD + 4 * j4]) = qx;
-            *reinterpret_cast<float4 *>(&sm.V[r * SD + 4 * j4]) = vx;
-        }
-        if (w == 0) {  // gates: inclusive scan of log alpha over the 64 tokens, 2 per lane
+        const float *Kc = sm.K[ci & 1];
+        __syncthreads();  // the previous chunk is done with V, M and its K buffer
+        // 1. the chunk's rows: K and Q were fetched ahead, V now (rows past T: zeros,
+        //    alpha = 1, beta = 0); the gates' inclusive scan of log alpha meanwhile
+        fetch_rows(sm.V, SV, a.v, c0);
+        cp_async_commit();
+        if (w == 0) {
             float l2[2], b2[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
@@ -139,9 +182,9 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
                 l2[u] = 0.0f;
                 b2[u] = 0.0f;
                 if (r < cc) {
-                    const size_t row = ((size_t)(n * a.T + c0 + r) * a.nL_in + a.l_in0 + ll) * a.H + h;
-                    l2[u] = logf(a.alpha[row]);
-                    b2[u] = a.beta[row];
+                    const size_t gi = row_of(c0 + r) / D;
+                    l2[u] = logf(a.alpha[gi]);
+                    b2[u] = a.beta[gi];
                 }
             }
             float s = l2[0] + l2[1];
@@ -156,14 +199,20 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
             sm.beta[2 * lane] = b2[0];
             sm.beta[2 * lane + 1] = b2[1];
         }
+        cp_async_wait_all();
         __syncthreads();
+        if (c0 + C < a.T) {  // the next chunk: into L2, and its K into the other buffer
+            prefetch_chunk(c0 + C);
+            fetch_rows(sm.K[(ci + 1) & 1], SD, a.k, c0 + C);
+            cp_async_commit();
+        }
         if (tid < C) sm.f[tid] = sm.beta[tid] * expf(sm.lg[C - 1] - sm.lg[tid]);
         // 2. M = strict_lower(K K^T o Gamma) diag(beta)  and  R = V - diag(gamma) K S
         {
             float acc[4][4];
             zero(acc);
             const int m0 = 16 * (w >> 1), n0 = 32 * (w & 1);
-            warp_gemm<4, D>(acc, sm.K, SD, 1, sm.K, 1, SD, nullptr, m0, n0, lane);
+            warp_gemm<4>(acc, Kc, SD, 1, nullptr, Kc, 1, SD, m0, n0, D, lane);
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -176,25 +225,63 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
             float acc[8][4];
             zero(acc);
             const int m0 = 16 * (w >> 1), n0 = 64 * (w & 1);
-            warp_gemm<8, D>(acc, sm.K, SD, 1, sm.S, SD, 1, nullptr, m0, n0, lane);
+            warp_gemm<8>(acc, Kc, SD, 1, nullptr, sm.S, SV, 1, m0, n0, D, lane);
+            const float gm0 = expf(sm.lg[m0 + g]), gm1 = expf(sm.lg[m0 + g + 8]);
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int r = m0 + g + 8 * (e >> 1), j = n0 + 8 * nt + 2 * t4 + (e & 1);
-                    sm.V[r * SD + j] -= expf(sm.lg[r]) * acc[nt][e];
+                    sm.V[r * SV + j] -= ((e >> 1) ? gm1 : gm0) * acc[nt][e];
                 }
         }
         __syncthreads();
-        // 3. U = (I + M)^-1 R in place: warp w owns value columns [16 w, 16 w + 16),
-        //    two lanes per column (even / odd s), rows in order
+        // 3. U = (I + M)^-1 R in blocks of 16 rows.  (a) Warps 0-3 each invert one unit
+        //    lower triangular diagonal block, T_bb = (I + M_bb)^-1, by substitution down its
+        //    columns (lane c holds column c), and store it over M_bb.
+        if (w < 4) {
+            const int r0 = 16 * w, c = lane & 15;
+            float tc[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float acc = 0.0f;
+#pragma unroll
+                for (int s2 = 0; s2 < r; ++s2) acc = fmaf(sm.M[(r0 + r) * SC + r0 + s2], tc[s2], acc);
+                tc[r] = (r == c) ? 1.0f : (r < c ? 0.0f : -acc);
+            }
+            __syncwarp();
+            if (lane < 16) {
+#pragma unroll
+                for (int r = 0; r < 16; ++r) sm.M[(r0 + r) * SC + r0 + c] = tc[r];
+            }
+        }
+        __syncthreads();
+        //    (b) Warp w owns value columns [16 w, 16 w + 16); block by block,
+        //    U_b = T_bb (R_b - M[b, < b] U[< b]), both products on the tensor cores.
         {
-            const int j = 16 * w + (lane & 15), hs = lane >> 4;
-            for (int r = 1; r < C; ++r) {
-                float part = 0.0f;
-                for (int s = hs; s < r; s += 2) part += sm.M[r * SC + s] * sm.V[s * SD + j];
-                part += __shfl_xor_sync(0xffffffffu, part, 16);
-                if (hs == 0) sm.V[r * SD + j] -= part;
+            const int jw = 16 * w;
+#pragma unroll 1
+            for (int r0 = 0; r0 < C; r0 += 16) {
+                if (r0 > 0) {
+                    float acc[2][4];
+                    zero(acc);
+                    warp_gemm<2>(acc, sm.M, SC, 1, nullptr, sm.V, SV, 1, r0, jw, r0, lane);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            sm.V[(r0 + g + 8 * (e >> 1)) * SV + jw + 8 * nt + 2 * t4 + (e & 1)] -= acc[nt][e];
+                    __syncwarp();
+                }
+                float acc[2][4];
+                zero(acc);
+                warp_gemm<2>(acc, sm.M + r0, SC, 1, nullptr, sm.V + r0 * SV, SV, 1, r0, jw, 16, lane);
+                __syncwarp();  // every lane has read R_b
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        sm.V[(r0 + g + 8 * (e >> 1)) * SV + jw + 8 * nt + 2 * t4 + (e & 1)] = acc[nt][e];
                 __syncwarp();
             }
         }
@@ -204,7 +291,7 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
             float acc[4][4];
             zero(acc);
             const int m0 = 16 * (w >> 1), n0 = 32 * (w & 1);
-            warp_gemm<4, D>(acc, sm.Q, SD, 1, sm.K, 1, SD, nullptr, m0, n0, lane);
+            warp_gemm<4>(acc, sm.Q, SD, 1, nullptr, Kc, 1, SD, m0, n0, D, lane);
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -220,23 +307,29 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
             zero(acc);
             zero(acc2);
             const int m0 = 16 * (w >> 1), n0 = 64 * (w & 1);
-            warp_gemm<8, D>(acc, sm.Q, SD, 1, sm.S, SD, 1, nullptr, m0, n0, lane);
-            warp_gemm<8, C>(acc2, sm.M, SC, 1, sm.V, SD, 1, nullptr, m0, n0, lane);
+            warp_gemm<8>(acc, sm.Q, SD, 1, nullptr, sm.S, SV, 1, m0, n0, D, lane);
+            warp_gemm<8>(acc2, sm.M, SC, 1, nullptr, sm.V, SV, 1, m0, n0, C, lane);
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
+            for (int e2 = 0; e2 < 2; ++e2) {
+                const int r = m0 + g + 8 * e2;
+                if (r < cc) {
+                    const float gm = expf(sm.lg[r]);
+                    float *orow = a.o + row_of(c0 + r);
 #pragma unroll
-                for (int e2 = 0; e2 < 2; ++e2) {
-                    const int r = m0 + g + 8 * e2, j = n0 + 8 * nt + 2 * t4;
-                    if (r < cc) {
-                        const float gm = expf(sm.lg[r]);
-                        const size_t row = ((size_t)(n * a.T + c0 + r) * a.nL_in + a.l_in0 + ll) * a.H + h;
-                        *reinterpret_cast<float2 *>(a.o + row * D + j) =
-                            make_float2(gm * acc[nt][2 * e2] + acc2[nt][2 * e2], gm * acc[nt][2 * e2 + 1] + acc2[nt][2 * e2 + 1]);
+                    for (int nt = 0; nt < 8; ++nt) {
+                        const int j = n0 + 8 * nt + 2 * t4;
+                        *reinterpret_cast<float2 *>(orow + j) = make_float2(gm * acc[nt][2 * e2] + acc2[nt][2 * e2],
+                                                                            gm * acc[nt][2 * e2 + 1] + acc2[nt][2 * e2 + 1]);
                     }
                 }
+            }
         }
-        __syncthreads();  // every read of the old state is done
-        // 6. S = gamma_C S + K^T diag(f) U, warp w updates state rows [16 w, 16 w + 16)
+        __syncthreads();  // every read of the old state and of Q is done
+        if (c0 + C < a.T) {  // the next chunk's Q, during the state update
+            fetch_rows(sm.Q, SD, a.q, c0 + C);
+            cp_async_commit();
+        }
+        // 6. S = gamma_C S + (K^T diag(f)) U, warp w updates state rows [16 w, 16 w + 16)
         {
             const float gC = expf(sm.lg[C - 1]);
 #pragma unroll 1
@@ -244,21 +337,22 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
                 float acc[8][4];
                 zero(acc);
                 const int m0 = 16 * w, n0 = 64 * half;
-                warp_gemm<8, C>(acc, sm.K, 1, SD, sm.V, SD, 1, sm.f, m0, n0, lane);
+                warp_gemm<8>(acc, Kc, 1, SD, sm.f, sm.V, SV, 1, m0, n0, C, lane);
 #pragma unroll
                 for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int i = m0 + g + 8 * (e >> 1), j = n0 + 8 * nt + 2 * t4 + (e & 1);
-                        sm.S[i * SD + j] = gC * sm.S[i * SD + j] + acc[nt][e];
+                        sm.S[i * SV + j] = gC * sm.S[i * SV + j] + acc[nt][e];
                     }
             }
         }
     }
+    cp_async_wait_all();
     __syncthreads();
     for (int e = tid; e < D * D / 4; e += NT) {
         const int i = e / (D / 4), j4 = e % (D / 4);
-        reinterpret_cast<float4 *>(Sg)[e] = *reinterpret_cast<const float4 *>(&sm.S[i * SD + 4 * j4]);
+        reinterpret_cast<float4 *>(Sg)[e] = *reinterpret_cast<const float4 *>(&sm.S[i * SV + 4 * j4]);
     }
 }
 
