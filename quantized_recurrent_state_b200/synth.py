@@ -159,20 +159,72 @@ def step_inputs_torch(wl: "Workload", seed: int, n_req: int, t: int, alpha: np.n
                 alpha=al.float().contiguous(), beta=beta.float().contiguous())
 
 
+def _mixed_torch(keys, n: int, device):
+    """The integer streams of several keys at once: [len(keys), n] int64
+    (the rows of _bits_np for each key, as wrapped int64)."""
+    import torch
+
+    def srl(x, s):
+        return (x >> s) & ((1 << (64 - s)) - 1)
+
+    k = torch.tensor([_to_i64(int(x)) for x in keys], dtype=torch.int64, device=device)[:, None]
+    idx = torch.arange(1, n + 1, dtype=torch.int64, device=device)[None, :]
+    z = k + idx * _to_i64(GOLDEN)
+    z = (z ^ srl(z, 30)) * _to_i64(M1)
+    z = (z ^ srl(z, 27)) * _to_i64(M2)
+    return z ^ srl(z, 31)
+
+
+def _normal_rows_torch(keys, n: int, device):
+    """normal_torch(key, (n,)) for every key, stacked: [len(keys), n] float64."""
+    import torch
+    m = (n + 1) // 2
+    z = _mixed_torch(keys, 2 * m, device)
+    top = ((z >> 11) & ((1 << 53) - 1)).to(torch.float64)
+    u1 = (top[:, 0::2] + 1.0) * 2.0 ** -53
+    u2 = top[:, 1::2] * 2.0 ** -53
+    rad = torch.sqrt(-2.0 * torch.log(u1))
+    out = torch.empty((len(keys), 2 * m), dtype=torch.float64, device=device)
+    out[:, 0::2] = rad * torch.cos(2.0 * math.pi * u2)
+    out[:, 1::2] = rad * torch.sin(2.0 * math.pi * u2)
+    return out[:, :n]
+
+
 def prompt_inputs_torch(wl: "Workload", seed: int, n_req: int, t0: int, T: int, alpha: np.ndarray, device,
-                        lb: int = 0, le: int = None) -> dict:
+                        lb: int = 0, le: int = None, block: int = 256) -> dict:
     """Tokens t0 .. t0 + T - 1 of step_inputs_torch as one prompt for layers
-    [lb, le): q, k, v [n_req, T, le - lb, H, D], alpha, beta [n_req, T, le - lb, H]."""
+    [lb, le): q, k, v [n_req, T, le - lb, H, D], alpha, beta [n_req, T, le - lb, H].
+    Generated `block` tokens at a time (same values as one token at a time)."""
     import torch
     le = wl.n_layers if le is None else le
-    out = None
-    for t in range(T):
-        s = step_inputs_torch(wl, seed, n_req, t0 + t, alpha, device)
-        if out is None:
-            out = {k: torch.empty((n_req, T) + tuple(v[:, lb:le].shape[1:]), dtype=v.dtype, device=device)
-                   for k, v in s.items()}
-        for k in out:
-            out[k][:, t] = s[k][:, lb:le]
+    L, H, D, nL = wl.n_layers, wl.n_heads, wl.d, le - lb
+    shape = (n_req, L, H, D)
+    out = {k: torch.empty((n_req, T, nL, H, D), dtype=torch.float32, device=device) for k in ("q", "k", "v")}
+    out["alpha"] = torch.empty((n_req, T, nL, H), dtype=torch.float32, device=device)
+    out["beta"] = torch.empty((n_req, T, nL, H), dtype=torch.float32, device=device)
+    gam = torch.from_numpy(column_scales(wl, seed)).to(device).double()[lb:le]
+    al = torch.from_numpy(np.ascontiguousarray(alpha)).to(device).float()[lb:le]
+    n_el = int(np.prod(shape))
+    for b0 in range(0, T, block):
+        ts = list(range(t0 + b0, t0 + min(T, b0 + block)))
+        nb = len(ts)
+
+        def gen(stream):
+            x = _normal_rows_torch([stream_key(seed, stream, t) for t in ts], n_el, device)
+            return x.reshape((nb,) + shape)[:, :, lb:le].transpose(0, 1)   # [n_req, nb, nL, H, D]
+
+        q = gen(S_Q)
+        kn = gen(S_K)
+        k = kn / torch.sqrt((kn * kn).sum(dim=-1, keepdim=True))
+        v = gen(S_V) * gam[None, None]
+        zb = _mixed_torch([stream_key(seed, S_BETA, t) for t in ts], n_req * L * H, device)
+        beta = (((zb >> 11) & ((1 << 53) - 1)).to(torch.float64) * 2.0 ** -53).reshape(nb, n_req, L, H)
+        sl = slice(b0, b0 + nb)
+        out["q"][:, sl] = q.float()
+        out["k"][:, sl] = k.float()
+        out["v"][:, sl] = v.float()
+        out["beta"][:, sl] = beta[:, :, lb:le].transpose(0, 1).float()
+        out["alpha"][:, sl] = al[None, None].expand(n_req, nb, nL, H)
     return out
 
 
