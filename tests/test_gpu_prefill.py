@@ -160,3 +160,46 @@ def test_prefill_layer_range_uniform_plan(stepq):
                 pv.quantize_into(expect, l, h, S_T[r, li, h])
                 assert np.array_equal(pv.record(new_slot, l, h), pv.record(expect, l, h)), (r, l, h)
     assert np.array_equal(after[sb:2 * sb], before[sb:2 * sb])
+
+
+def test_prefill_full_pool_sampled(stepq):
+    """The launch the prefill benchmark times: a 2,048-token chunk for all
+    2,304 heads of the pool (nominal 6 bits, 32 FP16 heads) at batch 1, inputs
+    drawn on the device by the same generator.  Sampled heads (and FP16 heads)
+    are checked against the token-by-token fp64 recurrence from the records
+    the pool held before, and their new records against the oracle's
+    quantization of the kernel's final state."""
+    plan, data, wl, _ = oracle_plan("qwen_pool6")
+    pv = model.PlanView(plan)
+    P = stepq.Plan.from_bytes(data)
+    n, T, L = 1, 2048, wl.n_layers
+    ctx = stepq.Context(P, n)
+    pool = torch.zeros(n * P.slot_bytes, dtype=torch.uint8, device="cuda")
+    slots = torch.arange(n, dtype=torch.int32, device="cuda")
+    for l in range(L):
+        ctx.requant_pack(pool, slots, n, l, l + 1, synth.initial_states_torch(wl, wl.seed, n, l, "cuda"))
+    inp = synth.prompt_inputs_torch(wl, wl.seed, n, 0, T, synth.gates(wl, wl.seed), "cuda")
+    o = torch.zeros_like(inp["q"])
+    ws = torch.empty(ctx.prefill_workspace_bytes(n, L) // 4, dtype=torch.float32, device="cuda")
+    ctx.sync()
+    before = pool.cpu().numpy().copy()
+    ctx.prefill(pool, slots, n, 0, L, T, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o, ws)
+    ctx.sync()
+    after = pool.cpu().numpy()
+    S_T = ws.view(n, L, wl.n_heads, wl.d, wl.d)
+    rng = np.random.default_rng(21)
+    units = P.widths().reshape(L * wl.n_heads, -1)
+    piv = np.nonzero((units == 16).any(axis=1))[0]
+    samples = [(int(rng.integers(L)), int(rng.integers(wl.n_heads))) for _ in range(6)]
+    samples += [(int(u) // wl.n_heads, int(u) % wl.n_heads) for u in piv[:2]]
+    worst = (0.0, 0.0)
+    for (l, h) in samples:
+        x = {k: v[:, :, l:l + 1, h:h + 1].cpu().numpy() for k, v in inp.items()}
+        S_start = pv.reconstruct(before, l, h).astype(np.float64)
+        s_t = S_T[0, l, h].cpu().numpy()
+        e = _check_head(o[0, :, l, h].cpu().numpy(), s_t, S_start, x, 0, 0, 0)
+        worst = (max(worst[0], e[0]), max(worst[1], e[1]))
+        expect = np.zeros_like(after)
+        pv.quantize_into(expect, l, h, s_t)
+        assert np.array_equal(pv.record(after, l, h), pv.record(expect, l, h)), (l, h)
+    print(f"full pool, T={T}: worst relative errors o {worst[0]:.2e}, S {worst[1]:.2e}")
