@@ -21,6 +21,15 @@ with gamma_t = alpha_1 ... alpha_t and Gamma_ts = gamma_t / gamma_s:
 the same arithmetic in dense products, which is what lets a prefill run on
 matrix units; this module evaluates it in fp64 as written and is pinned
 against the sequential fp64 recurrence.
+
+Per-key-row units (KDA: a gate alpha_t in R^D per token, applied first as
+Diag(alpha_t), the order of the recurrence reading for per-row gates): with
+u_t = v_t - S_{t-1}^T Diag(alpha_t) k_t the step is S_t = Diag(alpha_t) S_{t-1}
++ beta_t k_t u_t^T, and with Gamma_t = alpha_1 o ... o alpha_t per key row,
+
+    (I + M) U = V - (K o Gamma) S_0,   M_ts = beta_s sum_i k_ti k_si Gamma_ti / Gamma_si  (s < t)
+    O   = (Q o Gamma) S_0 + L_incl(A) U,  A_ts = beta_s sum_i q_ti k_si Gamma_ti / Gamma_si
+    S_C = Diag(Gamma_C) S_0 + (K o (Gamma_C / Gamma) o beta)^T U
 """
 from __future__ import annotations
 
@@ -70,4 +79,39 @@ def chunked(S0, Q, K, V, alpha, beta, C=64):
     for c0 in range(0, T, C):
         c1 = min(T, c0 + C)
         O[c0:c1], S = chunk(S, Q[c0:c1], K[c0:c1], V[c0:c1], alpha[c0:c1], beta[c0:c1])
+    return O, S
+
+
+def chunk_rows(S0, Q, K, V, alpha, beta):
+    """One chunk of the per-key-row formulas above in fp64; alpha [C, D].
+    The ratios Gamma_ti / Gamma_si are formed per (t, s, i) as written.
+    Returns (O, S_C)."""
+    S0 = np.asarray(S0, np.float64)
+    Q, K, V = (np.asarray(x, np.float64) for x in (Q, K, V))
+    a = np.asarray(alpha, np.float64)
+    b = np.asarray(beta, np.float64)
+    C = len(b)
+    gamma = np.cumprod(a, axis=0)                            # [C, D]
+    ratio = gamma[:, None, :] / gamma[None, :, :]            # [t, s, i]
+    strict = np.tril(np.ones((C, C), dtype=bool), -1)
+    incl = np.tril(np.ones((C, C), dtype=bool), 0)
+    M = np.where(strict, np.einsum("ti,si,tsi->ts", K, K, ratio) * b[None, :], 0.0)
+    rhs = V - (K * gamma) @ S0
+    U = np.zeros_like(rhs)
+    for t in range(C):                                       # forward substitution, (I + M) unit lower
+        U[t] = rhs[t] - M[t, :t] @ U[:t]
+    A = np.where(incl, np.einsum("ti,si,tsi->ts", Q, K, ratio) * b[None, :], 0.0)
+    O = (Q * gamma) @ S0 + A @ U
+    S = gamma[-1][:, None] * S0 + (K * (gamma[-1][None, :] / gamma) * b[:, None]).T @ U
+    return O, S
+
+
+def chunked_rows(S0, Q, K, V, alpha, beta, C=64):
+    """A whole prompt with per-key-row gates (alpha [T, D]) in chunks of C tokens."""
+    T = len(beta)
+    S = np.asarray(S0, np.float64)
+    O = np.zeros((T, S.shape[1]))
+    for c0 in range(0, T, C):
+        c1 = min(T, c0 + C)
+        O[c0:c1], S = chunk_rows(S, Q[c0:c1], K[c0:c1], V[c0:c1], alpha[c0:c1], beta[c0:c1])
     return O, S

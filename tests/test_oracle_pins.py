@@ -666,3 +666,42 @@ def test_chunk_of_one_token_is_one_step():
     S_ref = alpha[0] * S0 + beta[0] * np.outer(K[0], V[0] - alpha[0] * S0.T @ K[0])
     assert np.allclose(S, S_ref, rtol=1e-14, atol=1e-14)
     assert np.allclose(O[0], S_ref.T @ Q[0], rtol=1e-13, atol=1e-13)
+
+
+def _prompt_rows(T, D, seed):
+    S0, Q, K, V, _, beta = _prompt(T, D, seed)
+    g = np.random.default_rng(seed + 1)
+    alpha = np.exp(-np.log(2) / np.exp(g.uniform(np.log(2), np.log(2000), (T, D))))
+    return S0, Q, K, V, alpha, beta
+
+
+@pytest.mark.parametrize("T,C", [(1, 64), (64, 64), (65, 64), (150, 64), (37, 8)])
+def test_chunked_prefill_rows_equals_sequential(T, C):
+    # per-key-row gates: the chunk form against the token-by-token recurrence
+    from oracle import prefill
+    S0, Q, K, V, alpha, beta = _prompt_rows(T, 32, 900 + T + C)
+    O_seq, S_seq = prefill.sequential(S0, Q, K, V, alpha, beta)
+    O_chk, S_chk = prefill.chunked_rows(S0, Q, K, V, alpha, beta, C)
+    assert np.max(np.abs(O_chk - O_seq)) <= 1e-11 * max(1.0, np.max(np.abs(O_seq)))
+    assert np.max(np.abs(S_chk - S_seq)) <= 1e-11 * max(1.0, np.max(np.abs(S_seq)))
+
+
+def test_chunked_prefill_rows_with_equal_gates_is_the_scalar_form():
+    # a gate that is the same for every key row reduces to the per-head chunk form
+    from oracle import prefill
+    S0, Q, K, V, alpha, beta = _prompt(70, 16, 31)
+    rows = np.repeat(alpha[:, None], 16, axis=1)
+    O1, S1 = prefill.chunked(S0, Q, K, V, alpha, beta)
+    O2, S2 = prefill.chunked_rows(S0, Q, K, V, rows, beta)
+    assert np.allclose(O1, O2, rtol=1e-12, atol=1e-12) and np.allclose(S1, S2, rtol=1e-12, atol=1e-12)
+
+
+def test_chunk_rows_of_one_token_is_the_gated_step():
+    # one token: S_1 = (I - beta k k^T) Diag(alpha) S_0 + beta k v^T written out
+    from oracle import prefill
+    S0, Q, K, V, alpha, beta = _prompt_rows(1, 12, 5)
+    O, S = prefill.chunk_rows(S0, Q, K, V, alpha, beta)
+    k = K[0]
+    S_ref = (np.eye(12) - beta[0] * np.outer(k, k)) @ (alpha[0][:, None] * S0) + beta[0] * np.outer(k, V[0])
+    assert np.allclose(S, S_ref, rtol=1e-13, atol=1e-13)
+    assert np.allclose(O[0], S_ref.T @ Q[0], rtol=1e-13, atol=1e-13)
