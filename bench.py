@@ -34,7 +34,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "packed-state decode head-steps/s and HBM GB/s (% of peak), 2304 heads, bs=70"
-PREFILL_METRIC = "chunked prefill tokens/s into the packed 2304-head state pool"
+PREFILL_METRIC = "chunked prefill tokens/s into the packed state pool"
 TF32_PER_BF16 = 1.1 / 2.25   # nominal dense TF32 / BF16 tensor throughput
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -636,18 +636,20 @@ def prefill_flops(T: int, D: int, C: int = PREFILL_CHUNK) -> int:
     return tot
 
 
-def prefill_bytes(T: int, D: int) -> int:
+def prefill_bytes(T: int, D: int, rows: bool = False) -> int:
     """Algorithmic HBM bytes of one head in a prefill kernel launch: q, k, v
-    read and o written per token, alpha and beta read, the fp32 state read
-    and written once."""
-    return T * (4 * 4 * D + 8) + 2 * 4 * D * D
+    read and o written per token, alpha (one per head, or one per key row)
+    and beta read, the fp32 state read and written once."""
+    return T * (4 * 4 * D + (4 * D if rows else 4) + 4) + 2 * 4 * D * D
 
 
 def prefill_config(wl, n, T, ws):
     L, H, D = wl.n_layers, wl.n_heads, wl.d
-    return {"workload": (f"chunked prefill of {T}-token prompt chunks into the GDN state pool, {L} layers x {H} "
-                         f"heads = {L * H} heads, d_k=d_v={D}, batch {n}, nominal {wl.nominal_bits:g}-bit plan "
-                         f"over {sorted(wl.bits)}, {wl.n_pivots} FP16 pivot heads; each step continues from the "
+    pool = (f"the GDN state pool, {L} layers x {H} heads = {L * H} heads, d_k=d_v={D}, batch {n}, nominal "
+            f"{wl.nominal_bits:g}-bit plan over {sorted(wl.bits)}, {wl.n_pivots} FP16 pivot heads" if wl.mode == 0 else
+            f"the KDA per-key-row pool, {L} layers x {H} heads x {D} rows, d_v={D}, batch {n}, Lagrangian nominal "
+            f"{wl.nominal_bits:g}-bit plan over {sorted(wl.bits)}, {wl.n_pivots} FP16 pivot rows, per-row gates")
+    return {"workload": (f"chunked prefill of {T}-token prompt chunks into {pool}; each step continues from the "
                          f"packed states the previous one wrote"),
             "batch": n, "prompt_chunk_tokens": T, "kernel_chunk_tokens": PREFILL_CHUNK, "heads": L * H, "d": D,
             "l2": "inputs larger than L2 (one step's q, k, v far above 126 MB)",
@@ -717,7 +719,7 @@ def run_prefill(args):
     peak = bf16 * TF32_PER_BF16
     achieved = flops / launch_s / 1e12
     hbm_peak, hbm_kind = measured_peaks()
-    k_bytes = n * L * H * prefill_bytes(T, D)
+    k_bytes = n * L * H * prefill_bytes(T, D, wl.mode == 1)
 
     # the same tokens stepped one at a time by the fused decode step, for comparison
     compare = None
@@ -846,6 +848,7 @@ def _oracle_prefill_sample(payload):
     from oracle import model, plan_io, prefill
     from quantized_recurrent_state_b200 import synth
     plan_bytes, wname, heads, T = payload
+    chunked = prefill.chunked_rows if synth.workloads()[wname].mode == 1 else prefill.chunked
     pv = model.PlanView(plan_io.read_plan(plan_bytes))
     wl = synth.workloads()[wname]
     alpha = synth.gates(wl, wl.seed)
@@ -862,8 +865,8 @@ def _oracle_prefill_sample(payload):
     for (l, h) in heads:
         li = layers.index(l)
         S = pv.reconstruct(slot, l, h).astype(np.float64)
-        _, S_T = prefill.chunked(S, seq["q"][:, li, h], seq["k"][:, li, h], seq["v"][:, li, h],
-                                 seq["alpha"][:, li, h], seq["beta"][:, li, h])
+        _, S_T = chunked(S, seq["q"][:, li, h], seq["k"][:, li, h], seq["v"][:, li, h],
+                         seq["alpha"][:, li, h], seq["beta"][:, li, h])
         pv.quantize_into(slot, l, h, S_T)
     return time.perf_counter() - t0
 
@@ -1023,8 +1026,6 @@ def run_reference(args):
 def main():
     args = parse()
     if args.prefill:
-        if args.workload != "gdn":
-            raise SystemExit("--prefill: per-head (GDN) units only")
         (run_reference_prefill if args.impl == "reference" else run_prefill)(args)
     elif args.impl == "reference":
         run_reference(args)

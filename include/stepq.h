@@ -196,20 +196,26 @@ size_t stepq_workspace_bytes(const stepq_ctx *ctx, int n_req, int n_layers_launc
 
 /* ---- prefill (the step before decode) ----------------------------------- */
 
-/* Chunked prefill of T tokens on fp32 states (per-head units, d = 128):
+/* Chunked prefill of T tokens on fp32 states (d = 128, either unit kind):
  * for every (request, layer in [lb, le), head) the gated delta rule above,
- * token by token in meaning, S_t = (I - beta_t k_t k_t^T) alpha_t S_{t-1} +
- * beta_t k_t v_t^T and o_t = S_t^T q_t, evaluated in chunks of 64 tokens:
- * with gamma_t the running gate product in the chunk, (I + M) U = V -
- * diag(gamma) K S_0 with M_ts = gamma_t/gamma_s beta_s k_t.k_s (s < t),
- * O = diag(gamma) Q S_0 + L_incl(Q K^T o gamma_t/gamma_s) diag(beta) U and
- * S_C = gamma_C S_0 + K^T diag(beta gamma_C/gamma) U.  The dense products run
- * on the tensor cores (TF32 with a TF32 remainder, near fp32), the
- * triangular solve on the CUDA cores; results match the token-by-token fp64
- * recurrence to the tolerance stated in the tests, not bit for bit.
+ * token by token in meaning, S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1}
+ * + beta_t k_t v_t^T and o_t = S_t^T q_t, evaluated in chunks of 64 tokens:
+ * with Gamma_t the running gate product in the chunk (per key row for
+ * per-row plans), (I + M) U = V - (K o Gamma) S_0 with M_ts = beta_s
+ * sum_i k_ti k_si Gamma_ti/Gamma_si (s < t), O = (Q o Gamma) S_0 + L_incl(A) U
+ * with A_ts = beta_s sum_i q_ti k_si Gamma_ti/Gamma_si, and S_C = Diag(Gamma_C)
+ * S_0 + (K o (Gamma_C/Gamma) o beta)^T U.  The dense products run on the
+ * tensor cores (TF32 with a TF32 remainder, near fp32), the triangular solve
+ * in fp32; results match the token-by-token fp64 recurrence to the
+ * tolerance stated in the tests, not bit for bit.
  *   S: [n_req][le-lb][n_heads][D][D] fp32, read (unless zero_init) and written.
- *   q, k, v, o: [n_req][T][le-lb][n_heads][D];  alpha, beta: [n_req][T][le-lb][n_heads],
- *   alpha in (0, 1] (its logarithm is taken).  Enqueued on main. */
+ *   q, k, v, o: [n_req][T][le-lb][n_heads][D];  beta: [n_req][T][le-lb][n_heads];
+ *   alpha: [n_req][T][le-lb][n_heads] for per-head plans, [..][n_heads][D]
+ *   (16-byte aligned) for per-row plans; alpha in (0, 1] (its logarithm is
+ *   taken).  Per-row gates are factored around the chunk's middle token, so
+ *   they need the sum of |ln alpha_i| over any 32 consecutive tokens of a row
+ *   below about 80 (any alpha >= 0.083 meets it); beyond that the fp32 gate
+ *   factors overflow.  Enqueued on main. */
 int stepq_prefill_fp32(stepq_ctx *ctx, float *S, int n_req, int lb, int le, int T, const float *q,
                        const float *k, const float *v, const float *alpha, const float *beta, float *o,
                        int zero_init);

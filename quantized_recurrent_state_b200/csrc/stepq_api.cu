@@ -1007,12 +1007,11 @@ extern "C" int stepq_prefill_fp32(stepq_ctx *c, float *S, int n_req, int lb, int
     NvtxRange nvtx_range("stepq_prefill_fp32");
     int rc = check_range(c, n_req, lb, le);
     if (rc) return rc;
-    if (c->plan->mode != 0 || c->plan->D != 128)
-        return fail(STEPQ_EINVAL, "prefill: per-head units with d = 128 only (mode %d, d %d)", c->plan->mode, c->plan->D);
+    if (c->plan->D != 128) return fail(STEPQ_EINVAL, "prefill: d = 128 only (d %d)", c->plan->D);
     if (T < 0) return fail(STEPQ_EINVAL, "prefill: T = %d", T);
     if ((rc = check_ptr(S, 16, "S")) || (rc = check_ptr(q, 16, "q")) || (rc = check_ptr(k, 16, "k")) ||
-        (rc = check_ptr(v, 16, "v")) || (rc = check_ptr(alpha, 4, "alpha")) || (rc = check_ptr(beta, 4, "beta")) ||
-        (rc = check_ptr(o, 16, "o")))
+        (rc = check_ptr(v, 16, "v")) || (rc = check_ptr(alpha, c->plan->mode ? 16 : 4, "alpha")) ||
+        (rc = check_ptr(beta, 4, "beta")) || (rc = check_ptr(o, 16, "o")))
         return rc;
     if ((rc = set_device(c))) return rc;
     if (n_req == 0 || T == 0) return STEPQ_OK;
@@ -1020,6 +1019,7 @@ extern "C" int stepq_prefill_fp32(stepq_ctx *c, float *S, int n_req, int lb, int
     a.S = S; a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.o = o;
     a.n_req = n_req; a.T = T; a.nL = le - lb; a.nL_in = le - lb; a.l_in0 = 0; a.H = c->plan->H;
     a.zero_init = zero_init ? 1 : 0;
+    a.rows = c->plan->mode == 1;
     LaunchTimer lt(c, 4, c->main);
     const cudaError_t e = stepq::launch_prefill(a, c->main);
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
@@ -1038,12 +1038,12 @@ extern "C" int stepq_prefill(stepq_ctx *c, void *pool, const int32_t *slots, int
     NvtxRange nvtx_range("stepq_prefill");
     int rc = check_range(c, n_req, lb, le);
     if (rc) return rc;
-    if (c->plan->mode != 0 || c->plan->D != 128)
-        return fail(STEPQ_EINVAL, "prefill: per-head units with d = 128 only (mode %d, d %d)", c->plan->mode, c->plan->D);
+    if (c->plan->D != 128) return fail(STEPQ_EINVAL, "prefill: d = 128 only (d %d)", c->plan->D);
     if (T < 0) return fail(STEPQ_EINVAL, "prefill: T = %d", T);
     if ((rc = check_ptr(pool, 128, "pool")) || (rc = check_ptr(slots, 4, "slots")) || (rc = check_ptr(q, 16, "q")) ||
-        (rc = check_ptr(k, 16, "k")) || (rc = check_ptr(v, 16, "v")) || (rc = check_ptr(alpha, 4, "alpha")) ||
-        (rc = check_ptr(beta, 4, "beta")) || (rc = check_ptr(o, 16, "o")) || (rc = check_ptr(workspace, 16, "workspace")))
+        (rc = check_ptr(k, 16, "k")) || (rc = check_ptr(v, 16, "v")) ||
+        (rc = check_ptr(alpha, c->plan->mode ? 16 : 4, "alpha")) || (rc = check_ptr(beta, 4, "beta")) ||
+        (rc = check_ptr(o, 16, "o")) || (rc = check_ptr(workspace, 16, "workspace")))
         return rc;
     if ((rc = set_device(c))) return rc;
     if (n_req == 0 || T == 0) return STEPQ_OK;
@@ -1063,6 +1063,7 @@ extern "C" int stepq_prefill(stepq_ctx *c, void *pool, const int32_t *slots, int
     p.S = workspace; p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta; p.o = o;
     p.n_req = n_req; p.T = T; p.nL = le - lb; p.nL_in = le - lb; p.l_in0 = 0; p.H = c->plan->H;
     p.zero_init = from_zero ? 1 : 0;
+    p.rows = c->plan->mode == 1;
     {
         LaunchTimer lt(c, 4, c->main);
         e = stepq::launch_prefill(p, c->main);

@@ -39,13 +39,18 @@ static_assert(SD % 32 == 4 && SC % 32 == 4 && SV % 32 == 8, "bank-conflict-free 
 
 struct Smem {
     float S[D * SV];           // state, row i (key) x column j (value)
-    float K[2][C * SD];        // this chunk's K and the next chunk's, fetched ahead
-    float Q[C * SD];
-    float V[C * SV];           // V, then R = V - diag(gamma) K S, then U
+    float K[2][C * SD];        // per-head gates: this chunk's K and the next chunk's, fetched ahead;
+                               // per-row gates: K o e^(g - g_ref) and K o e^(g_ref - g) (see k_prefill)
+    float Q[C * SD];           // Q (per-row gates: Q o e^(g - g_ref))
+    float V[C * SV];           // V, then R = V - (gated K) S, then U
     float M[C * SC];           // M (strict lower; diagonal 16 x 16 blocks then (I + M_bb)^-1), then A
-    float lg[C];               // inclusive running sum of log alpha in the chunk
+    float lg[C];               // per-head gates: inclusive running sum of log alpha in the chunk
     float beta[C];
-    float f[C];                // beta_s gamma_C / gamma_s
+    float f[C];                // per-head gates: beta_s gamma_C / gamma_s
+    float gref[D];             // per-row gates, per key row i: g_ref, e^(g_ref), e^(g_C), e^(g_C - g_ref)
+    float eref[D];
+    float egC[D];
+    float egCr[D];
 };
 
 __device__ __forceinline__ uint32_t tf32(float x) {
@@ -121,6 +126,18 @@ __device__ __forceinline__ void zero(float (&acc)[NTILE][4]) {
 
 }  // namespace pf
 
+// One CTA per (request, layer, head).  Per-row gates (ROWS): with g_ti the
+// running sum of log alpha_ti over the chunk's tokens and g_ref,i its value at
+// the chunk's middle token, the gate ratios factor per key row as
+// e^(g_ti - g_ref,i) e^(g_ref,i - g_si), so with Kt = K o e^(g - g_ref),
+// Kh = K o e^(g_ref - g) and Qt = Q o e^(g - g_ref):
+//   M = strict_lower(Kt Kh^T) diag(beta),  R = V - (Kt diag(e^g_ref)) S_0,
+//   A = L_incl(Qt Kh^T) diag(beta),        O = (Qt diag(e^g_ref)) S_0 + A U,
+//   S_C = Diag(e^g_C) S_0 + Diag(e^(g_C - g_ref)) (Kh^T diag(beta)) U.
+// The exponents stay within the gates of half a chunk (32 tokens) of the
+// reference, so fp32 holds them while the sum of |log alpha_i| over any 32
+// consecutive tokens stays below about 80.
+template <bool ROWS>
 __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
     using namespace pf;
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -155,7 +172,7 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
     };
 
     prefetch_chunk(0);
-    fetch_rows(sm.K[0], SD, a.k, 0);
+    if (!ROWS) fetch_rows(sm.K[0], SD, a.k, 0);   // per-row gates fetch K with the chunk's gates
     fetch_rows(sm.Q, SD, a.q, 0);
     cp_async_commit();
     // the state
@@ -168,13 +185,19 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
 #pragma unroll 1
     for (int c0 = 0, ci = 0; c0 < a.T; c0 += C, ++ci) {
         const int cc = min(C, a.T - c0);
-        const float *Kc = sm.K[ci & 1];
-        __syncthreads();  // the previous chunk is done with V, M and its K buffer
-        // 1. the chunk's rows: K and Q were fetched ahead, V now (rows past T: zeros,
-        //    alpha = 1, beta = 0); the gates' inclusive scan of log alpha meanwhile
+        // K as the row operand (A side) and as the column operand (B side) of K K^T and Q K^T
+        const float *Ka = ROWS ? sm.K[0] : sm.K[ci & 1];
+        const float *Kb = ROWS ? sm.K[1] : Ka;
+        __syncthreads();  // the previous chunk is done with V, M and its K buffers
+        // 1. the chunk's rows: Q (and per-head K) were fetched ahead, V now; per-row gates:
+        //    K and the gate rows now.  Rows past T: zeros, alpha = 1, beta = 0.
         fetch_rows(sm.V, SV, a.v, c0);
+        if (ROWS) {
+            fetch_rows(sm.K[1], SD, a.k, c0);
+            fetch_rows(sm.K[0], SD, a.alpha, c0);
+        }
         cp_async_commit();
-        if (w == 0) {
+        if (w == 0) {  // beta; per-head gates: inclusive scan of log alpha over the 64 tokens, 2 per lane
             float l2[2], b2[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
@@ -183,50 +206,88 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
                 b2[u] = 0.0f;
                 if (r < cc) {
                     const size_t gi = row_of(c0 + r) / D;
-                    l2[u] = logf(a.alpha[gi]);
+                    if (!ROWS) l2[u] = logf(a.alpha[gi]);
                     b2[u] = a.beta[gi];
                 }
             }
-            float s = l2[0] + l2[1];
+            if (!ROWS) {
+                float s = l2[0] + l2[1];
 #pragma unroll
-            for (int m = 1; m < 32; m <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, s, m);
-                if (lane >= m) s += y;
+                for (int m = 1; m < 32; m <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, s, m);
+                    if (lane >= m) s += y;
+                }
+                const float excl = s - (l2[0] + l2[1]);
+                sm.lg[2 * lane] = excl + l2[0];
+                sm.lg[2 * lane + 1] = s;
             }
-            const float excl = s - (l2[0] + l2[1]);
-            sm.lg[2 * lane] = excl + l2[0];
-            sm.lg[2 * lane + 1] = s;
             sm.beta[2 * lane] = b2[0];
             sm.beta[2 * lane + 1] = b2[1];
         }
         cp_async_wait_all();
         __syncthreads();
-        if (c0 + C < a.T) {  // the next chunk: into L2, and its K into the other buffer
+        if (c0 + C < a.T) {  // the next chunk into L2 (per-head gates: and its K into the other buffer)
             prefetch_chunk(c0 + C);
-            fetch_rows(sm.K[(ci + 1) & 1], SD, a.k, c0 + C);
-            cp_async_commit();
+            if (!ROWS) {
+                fetch_rows(sm.K[(ci + 1) & 1], SD, a.k, c0 + C);
+                cp_async_commit();
+            }
         }
-        if (tid < C) sm.f[tid] = sm.beta[tid] * expf(sm.lg[C - 1] - sm.lg[tid]);
-        // 2. M = strict_lower(K K^T o Gamma) diag(beta)  and  R = V - diag(gamma) K S
+        if (ROWS) {
+            // per key row i (thread i): g_ti = running sum of log alpha_ti in place of the gate
+            // rows, the reference g at the middle real token, and the row factors
+            if (tid < D) {
+                float *gcol = sm.K[0] + tid;
+                float gs = 0.0f;
+#pragma unroll 4
+                for (int t = 0; t < C; ++t) {
+                    if (t < cc) gs += logf(gcol[t * SD]);
+                    gcol[t * SD] = gs;
+                }
+                const float gr = gcol[((cc - 1) >> 1) * SD];
+                sm.gref[tid] = gr;
+                sm.eref[tid] = expf(gr);
+                sm.egC[tid] = expf(gs);
+                sm.egCr[tid] = expf(gs - gr);
+            }
+            __syncthreads();
+            {  // Kt = K o e^(g - g_ref) over the gates, Kh = K o e^(g_ref - g) over K, Qt = Q o e^(g - g_ref)
+                const int i = tid & (D - 1), tb = (tid / D) * (C / 2);
+                const float gr = sm.gref[i];
+#pragma unroll 4
+                for (int t = tb; t < tb + C / 2; ++t) {
+                    const float gt = sm.K[0][t * SD + i], kr = sm.K[1][t * SD + i];
+                    const float up = expf(gt - gr);
+                    sm.K[0][t * SD + i] = kr * up;
+                    sm.K[1][t * SD + i] = kr * expf(gr - gt);
+                    sm.Q[t * SD + i] *= up;
+                }
+            }
+            __syncthreads();
+        } else if (tid < C) {
+            sm.f[tid] = sm.beta[tid] * expf(sm.lg[C - 1] - sm.lg[tid]);
+        }
+        // 2. M = strict_lower(K K^T o Gamma) diag(beta)  and  R = V - (K o Gamma) S
         {
             float acc[4][4];
             zero(acc);
             const int m0 = 16 * (w >> 1), n0 = 32 * (w & 1);
-            warp_gemm<4>(acc, Kc, SD, 1, nullptr, Kc, 1, SD, m0, n0, D, lane);
+            warp_gemm<4>(acc, Ka, SD, 1, nullptr, Kb, 1, SD, m0, n0, D, lane);
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int r = m0 + g + 8 * (e >> 1), s = n0 + 8 * nt + 2 * t4 + (e & 1);
-                    sm.M[r * SC + s] = (s < r) ? acc[nt][e] * expf(sm.lg[r] - sm.lg[s]) * sm.beta[s] : 0.0f;
+                    const float x = ROWS ? acc[nt][e] : acc[nt][e] * expf(sm.lg[r] - sm.lg[s]);
+                    sm.M[r * SC + s] = (s < r) ? x * sm.beta[s] : 0.0f;
                 }
         }
         {
             float acc[8][4];
             zero(acc);
             const int m0 = 16 * (w >> 1), n0 = 64 * (w & 1);
-            warp_gemm<8>(acc, Kc, SD, 1, nullptr, sm.S, SV, 1, m0, n0, D, lane);
-            const float gm0 = expf(sm.lg[m0 + g]), gm1 = expf(sm.lg[m0 + g + 8]);
+            warp_gemm<8>(acc, Ka, SD, 1, ROWS ? sm.eref : nullptr, sm.S, SV, 1, m0, n0, D, lane);
+            const float gm0 = ROWS ? 1.0f : expf(sm.lg[m0 + g]), gm1 = ROWS ? 1.0f : expf(sm.lg[m0 + g + 8]);
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
@@ -291,29 +352,30 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
             float acc[4][4];
             zero(acc);
             const int m0 = 16 * (w >> 1), n0 = 32 * (w & 1);
-            warp_gemm<4>(acc, sm.Q, SD, 1, nullptr, Kc, 1, SD, m0, n0, D, lane);
+            warp_gemm<4>(acc, sm.Q, SD, 1, nullptr, Kb, 1, SD, m0, n0, D, lane);
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int r = m0 + g + 8 * (e >> 1), s = n0 + 8 * nt + 2 * t4 + (e & 1);
-                    sm.M[r * SC + s] = (s <= r) ? acc[nt][e] * expf(sm.lg[r] - sm.lg[s]) * sm.beta[s] : 0.0f;
+                    const float x = ROWS ? acc[nt][e] : acc[nt][e] * expf(sm.lg[r] - sm.lg[s]);
+                    sm.M[r * SC + s] = (s <= r) ? x * sm.beta[s] : 0.0f;
                 }
         }
         __syncthreads();
-        // 5. O = diag(gamma) Q S + A U, rows of this chunk to global
+        // 5. O = (Q o Gamma) S + A U, rows of this chunk to global
         {
             float acc[8][4], acc2[8][4];
             zero(acc);
             zero(acc2);
             const int m0 = 16 * (w >> 1), n0 = 64 * (w & 1);
-            warp_gemm<8>(acc, sm.Q, SD, 1, nullptr, sm.S, SV, 1, m0, n0, D, lane);
+            warp_gemm<8>(acc, sm.Q, SD, 1, ROWS ? sm.eref : nullptr, sm.S, SV, 1, m0, n0, D, lane);
             warp_gemm<8>(acc2, sm.M, SC, 1, nullptr, sm.V, SV, 1, m0, n0, C, lane);
 #pragma unroll
             for (int e2 = 0; e2 < 2; ++e2) {
                 const int r = m0 + g + 8 * e2;
                 if (r < cc) {
-                    const float gm = expf(sm.lg[r]);
+                    const float gm = ROWS ? 1.0f : expf(sm.lg[r]);
                     float *orow = a.o + row_of(c0 + r);
 #pragma unroll
                     for (int nt = 0; nt < 8; ++nt) {
@@ -329,22 +391,28 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
             fetch_rows(sm.Q, SD, a.q, c0 + C);
             cp_async_commit();
         }
-        // 6. S = gamma_C S + (K^T diag(f)) U, warp w updates state rows [16 w, 16 w + 16)
+        // 6. S = Gamma_C S + (K^T diag(beta Gamma_C / Gamma)) U, warp w updates state rows
+        //    [16 w, 16 w + 16); per-row gates: the row factors e^(g_C), e^(g_C - g_ref)
         {
-            const float gC = expf(sm.lg[C - 1]);
+            const float gC = ROWS ? 0.0f : expf(sm.lg[C - 1]);
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
                 float acc[8][4];
                 zero(acc);
                 const int m0 = 16 * w, n0 = 64 * half;
-                warp_gemm<8>(acc, Kc, 1, SD, sm.f, sm.V, SV, 1, m0, n0, C, lane);
+                warp_gemm<8>(acc, Kb, 1, SD, ROWS ? sm.beta : sm.f, sm.V, SV, 1, m0, n0, C, lane);
 #pragma unroll
-                for (int nt = 0; nt < 8; ++nt)
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    const int i = m0 + g + 8 * e2;
+                    const float dS = ROWS ? sm.egC[i] : gC, dU = ROWS ? sm.egCr[i] : 1.0f;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = m0 + g + 8 * (e >> 1), j = n0 + 8 * nt + 2 * t4 + (e & 1);
-                        sm.S[i * SV + j] = gC * sm.S[i * SV + j] + acc[nt][e];
-                    }
+                    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                        for (int e1 = 0; e1 < 2; ++e1) {
+                            const int j = n0 + 8 * nt + 2 * t4 + e1;
+                            sm.S[i * SV + j] = dS * sm.S[i * SV + j] + dU * acc[nt][2 * e2 + e1];
+                        }
+                }
             }
         }
     }
@@ -362,9 +430,10 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t st) {
     const int items = a.n_req * a.nL * a.H;
     if (items <= 0 || a.T <= 0) return cudaSuccess;
     const size_t smem = sizeof(pf::Smem);
-    cudaError_t e = cudaFuncSetAttribute(k_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = a.rows ? k_prefill<true> : k_prefill<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_prefill<<<items, pf::NT, smem, st>>>(a);
+    kern<<<items, pf::NT, smem, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -193,17 +193,18 @@ def _normal_rows_torch(keys, n: int, device):
 def prompt_inputs_torch(wl: "Workload", seed: int, n_req: int, t0: int, T: int, alpha: np.ndarray, device,
                         lb: int = 0, le: int = None, block: int = 256) -> dict:
     """Tokens t0 .. t0 + T - 1 of step_inputs_torch as one prompt for layers
-    [lb, le): q, k, v [n_req, T, le - lb, H, D], alpha, beta [n_req, T, le - lb, H].
+    [lb, le): q, k, v [n_req, T, le - lb, H, D], beta [n_req, T, le - lb, H],
+    alpha [n_req, T, le - lb, H] (per-head gates) or [.., H, D] (per-row gates).
     Generated `block` tokens at a time (same values as one token at a time)."""
     import torch
     le = wl.n_layers if le is None else le
     L, H, D, nL = wl.n_layers, wl.n_heads, wl.d, le - lb
     shape = (n_req, L, H, D)
     out = {k: torch.empty((n_req, T, nL, H, D), dtype=torch.float32, device=device) for k in ("q", "k", "v")}
-    out["alpha"] = torch.empty((n_req, T, nL, H), dtype=torch.float32, device=device)
+    al = torch.from_numpy(np.ascontiguousarray(alpha)).to(device).float()[lb:le]   # [nL, H] or [nL, H, D]
+    out["alpha"] = torch.empty((n_req, T) + tuple(al.shape), dtype=torch.float32, device=device)
     out["beta"] = torch.empty((n_req, T, nL, H), dtype=torch.float32, device=device)
     gam = torch.from_numpy(column_scales(wl, seed)).to(device).double()[lb:le]
-    al = torch.from_numpy(np.ascontiguousarray(alpha)).to(device).float()[lb:le]
     n_el = int(np.prod(shape))
     for b0 in range(0, T, block):
         ts = list(range(t0 + b0, t0 + min(T, b0 + block)))
@@ -224,7 +225,7 @@ def prompt_inputs_torch(wl: "Workload", seed: int, n_req: int, t0: int, T: int, 
         out["k"][:, sl] = k.float()
         out["v"][:, sl] = v.float()
         out["beta"][:, sl] = beta[:, :, lb:le].transpose(0, 1).float()
-        out["alpha"][:, sl] = al[None, None].expand(n_req, nb, nL, H)
+        out["alpha"][:, sl] = al[None, None].expand((n_req, nb) + tuple(al.shape))
     return out
 
 

@@ -203,3 +203,75 @@ def test_prefill_full_pool_sampled(stepq):
         pv.quantize_into(expect, l, h, s_t)
         assert np.array_equal(pv.record(after, l, h), pv.record(expect, l, h)), (l, h)
     print(f"full pool, T={T}: worst relative errors o {worst[0]:.2e}, S {worst[1]:.2e}")
+
+
+def _check_record(pv, new_slot, l, h, S):
+    """The record the GPU wrote for (l, h) against the oracle's quantization of
+    the kernel's fp32 state S: bit-exact except codes the oracle marks as ties."""
+    expect = np.zeros_like(new_slot)
+    tie = pv.quantize_into(expect, l, h, S)
+    rg, ro = pv.record(new_slot, l, h), pv.record(expect, l, h)
+    if np.array_equal(rg, ro):
+        return
+    zg, hg, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), rg)
+    zo, ho, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), ro)
+    assert not (((zg != zo) | (hg != ho)) & (tie == 0)).any(), (l, h)
+
+
+# ---- per-key-row gates (KDA units) -----------------------------------------
+
+@pytest.mark.parametrize("T", [1, 64, 100, 256])
+def test_prefill_rows_fp32_matches_sequential(stepq, T):
+    plan, data, wl, _ = oracle_plan("kda_rows", n_layers=1, n_pivots=8)
+    P = stepq.Plan.from_bytes(data)
+    n = 2
+    ctx = stepq.Context(P, n)
+    S0 = synth.initial_states(wl, wl.seed, n)
+    inp = _prompt(wl, n, T, 4000 + T)
+    assert inp["alpha"].shape == (n, T, 1, wl.n_heads, wl.d)
+    d = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
+    S = torch.from_numpy(S0).cuda()
+    o = torch.zeros_like(d["q"])
+    ctx.prefill_fp32(S, n, 0, 1, T, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)
+    ctx.sync()
+    Sg, og = S.cpu().numpy(), o.cpu().numpy()
+    worst = (0.0, 0.0)
+    for (r, h) in [(0, 0), (1, 7), (0, 19), (1, 31)]:
+        e = _check_head(og[r, :, 0, h], Sg[r, 0, h], S0[r, 0, h].astype(np.float64), inp, r, h)
+        worst = (max(worst[0], e[0]), max(worst[1], e[1]))
+    print(f"rows T={T}: worst relative errors o {worst[0]:.2e}, S {worst[1]:.2e}")
+
+
+@pytest.mark.parametrize("from_zero", [False, True])
+def test_prefill_rows_into_packed_states(stepq, from_zero):
+    """Layers [1, 3) of a three-layer per-row plan (pivot rows included)."""
+    plan, data, wl, _ = oracle_plan("kda_rows", n_layers=3, n_pivots=24)
+    pv = model.PlanView(plan)
+    P = stepq.Plan.from_bytes(data)
+    n, T, lb, le = 2, 130, 1, 3
+    ctx = stepq.Context(P, 3)
+    slots = torch.tensor([2, 0], dtype=torch.int32, device="cuda")
+    pool = torch.zeros(3 * P.slot_bytes, dtype=torch.uint8, device="cuda")
+    ctx.requant_pack(pool, slots, n, 0, 3, torch.from_numpy(synth.initial_states(wl, wl.seed, n)).cuda())
+    ctx.sync()
+    before = pool.cpu().numpy().copy()
+    inp = {k: np.ascontiguousarray(v[:, :, lb:le]) for k, v in _prompt(wl, n, T, 6).items()}
+    d = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
+    o = torch.zeros_like(d["q"])
+    ws = torch.empty(ctx.prefill_workspace_bytes(n, le - lb) // 4, dtype=torch.float32, device="cuda")
+    ctx.prefill(pool, slots, n, lb, le, T, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o, ws, from_zero=from_zero)
+    ctx.sync()
+    after, og = pool.cpu().numpy(), o.cpu().numpy()
+    S_T = ws.view(n, le - lb, wl.n_heads, wl.d, wl.d).cpu().numpy()
+    sb = P.slot_bytes
+    units = P.widths().reshape(3, wl.n_heads, -1)
+    for r, s in enumerate((2, 0)):
+        prev_slot, new_slot = before[s * sb:(s + 1) * sb], after[s * sb:(s + 1) * sb]
+        assert np.array_equal(new_slot[:int(pv.offsets[wl.n_heads])], prev_slot[:int(pv.offsets[wl.n_heads])])
+        for li, l in enumerate(range(lb, le)):
+            heads = [0, 13, 31] + [int(x) for x in np.nonzero((units[l] == 16).any(axis=1))[0][:2]]
+            for h in heads:
+                S_start = np.zeros((wl.d, wl.d)) if from_zero else pv.reconstruct(prev_slot, l, h).astype(np.float64)
+                _check_head(og[r, :, li, h], S_T[r, li, h], S_start, inp, r, h, li)
+                _check_record(pv, new_slot, l, h, S_T[r, li, h])
+    assert np.array_equal(after[sb:2 * sb], before[sb:2 * sb])
