@@ -486,6 +486,7 @@ def run_product(args):
             torch.cuda.synchronize()
             best = max(best, 2 * nb / (c0.elapsed_time(c1) / 1e3) / 1e9)
         extra["copy_probe_gbs"] = best
+        extra["kernel_frac_of_copy_probe"] = achieved / best if achieved else None
         del a, b
         torch.cuda.empty_cache()
 
@@ -934,13 +935,20 @@ def cpu_baseline(plan_bytes, wl, budget_s=12.0):
     same workload (request 0's heads in layer order, one decode step each)
     sized to about budget_s seconds of CPU work in total."""
     cores = _n_cores()
-    per_head = _oracle_sample((plan_bytes, wl.name, [(0, 0)], 0))
+    one = [(l, h) for l in range(2) for h in range(wl.n_heads)][:16]
+    with oracle_pool(1) as pool1:   # one process, one BLAS thread
+        sec1 = pool1.map(_oracle_sample, [(plan_bytes, wl.name, one, 0)])[0]
+    per_head = sec1 / len(one)
     heads = int(min(wl.n_layers * wl.n_heads, max(cores, budget_s / max(per_head, 1e-4))))
     with oracle_pool(cores) as pool:
         nh, sec = cpu_sample_rate(plan_bytes, wl, heads, 0, pool, cores)
-    return {"value": nh / sec, "unit": "head-steps/s", "cores": cores, "kind": "oracle",
+    return {"value": nh / sec, "unit": "head-steps/s", "cores": cores, "host_cores": os.cpu_count(),
+            "kind": "oracle",
             "sample": f"{nh} (layer, head) states of request 0, one decode step each, split over {cores} "
-                      f"spawned processes; time = slowest process's stepping time"}
+                      f"spawned processes; time = slowest process's stepping time",
+            "single_thread": {"value": len(one) / sec1, "unit": "head-steps/s", "cores": 1,
+                              "sample": f"{len(one)} (layer, head) states of request 0, one step each, "
+                                        f"one process with one BLAS thread"}}
 
 
 def oracle_plan_bytes(wl, pool):
