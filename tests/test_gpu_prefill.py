@@ -49,7 +49,7 @@ def _check_head(O_gpu, S_gpu, S0, inp, r, h, l=0):
     return eo, es
 
 
-@pytest.mark.parametrize("T", [1, 64, 100, 256])
+@pytest.mark.parametrize("T", [1, 64, 65, 100, 127, 256])
 def test_prefill_fp32_matches_sequential(stepq, T):
     plan, data, wl, _ = oracle_plan("qwen_layer")
     P = stepq.Plan.from_bytes(data)
@@ -275,3 +275,44 @@ def test_prefill_rows_into_packed_states(stepq, from_zero):
                 _check_head(og[r, :, li, h], S_T[r, li, h], S_start, inp, r, h, li)
                 _check_record(pv, new_slot, l, h, S_T[r, li, h])
     assert np.array_equal(after[sb:2 * sb], before[sb:2 * sb])
+
+
+def test_prefill_degenerate_gates_full_pool(stepq):
+    """alpha = 1, beta = 0 for every token of the whole pool (2,304 heads, batch
+    1, 300 tokens): M = 0 and the update adds exact zeros, so the fp32 state
+    comes back bit for bit, and o_t = S_0^T q_t."""
+    plan, data, wl, _ = uniform_plan("qwen_pool6", 6, model.QUANT_DUAL_AXIS)
+    P = stepq.Plan.from_bytes(data)
+    n, T, L = 1, 300, wl.n_layers
+    ctx = stepq.Context(P, n)
+    inp = synth.prompt_inputs_torch(wl, wl.seed, n, 0, T, synth.gates(wl, wl.seed), "cuda")
+    inp["alpha"].fill_(1.0)
+    inp["beta"].zero_()
+    S0 = torch.cat([synth.initial_states_torch(wl, wl.seed, n, l, "cuda") for l in range(L)], dim=1)
+    S = S0.clone()
+    o = torch.zeros_like(inp["q"])
+    ctx.prefill_fp32(S, n, 0, L, T, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o)
+    ctx.sync()
+    assert torch.equal(S, S0)
+    ref = torch.einsum("nlhij,ntlhi->ntlhj", S0.double(), inp["q"].double())
+    err = (o.double() - ref).abs().amax(dim=(1, 4)) / ref.abs().amax(dim=(1, 4))
+    assert float(err.max()) <= TOL, float(err.max())
+
+
+def test_packed_prefill_noop_calls(stepq):
+    """T = 0 and n_req = 0 leave the pool as it was."""
+    plan, data, wl, _ = oracle_plan("qwen_layer")
+    P = stepq.Plan.from_bytes(data)
+    ctx = stepq.Context(P, 2)
+    slots = torch.tensor([1, 0], dtype=torch.int32, device="cuda")
+    pool = torch.zeros(2 * P.slot_bytes, dtype=torch.uint8, device="cuda")
+    ctx.requant_pack(pool, slots, 2, 0, 1, torch.from_numpy(synth.initial_states(wl, wl.seed, 2)).cuda())
+    ctx.sync()
+    before = pool.clone()
+    inp = {k: torch.from_numpy(v).cuda() for k, v in _prompt(wl, 2, 3, 8).items()}
+    o = torch.zeros_like(inp["q"])
+    ws = torch.empty(ctx.prefill_workspace_bytes(2, 1) // 4, dtype=torch.float32, device="cuda")
+    ctx.prefill(pool, slots, 2, 0, 1, 0, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o, ws)
+    ctx.prefill(pool, slots, 0, 0, 1, 3, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o, ws)
+    ctx.sync()
+    assert torch.equal(pool, before)
