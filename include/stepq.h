@@ -215,7 +215,10 @@ size_t stepq_workspace_bytes(const stepq_ctx *ctx, int n_req, int n_layers_launc
  *   taken).  Per-row gates are factored around the chunk's middle token, so
  *   they need the sum of |ln alpha_i| over any 32 consecutive tokens of a row
  *   below about 80 (any alpha >= 0.083 meets it); beyond that the fp32 gate
- *   factors overflow.  Enqueued on main. */
+ *   factors overflow.  A gate outside (0, 1], or per-row gates beyond that
+ *   range, set the context's device error word: the next stepq_sync returns
+ *   STEPQ_EDEVICE ("prefill gate out of range") and the affected outputs are
+ *   not valid.  Enqueued on main. */
 int stepq_prefill_fp32(stepq_ctx *ctx, float *S, int n_req, int lb, int le, int T, const float *q,
                        const float *k, const float *v, const float *alpha, const float *beta, float *o,
                        int zero_init);

@@ -995,8 +995,9 @@ extern "C" int stepq_sync(stepq_ctx *c, int timeout_ms) {
     if (e != cudaSuccess) return cuda_fail(e, "sync: read error word");
     if (word) {
         cudaMemset(c->err, 0, sizeof(int));
-        return fail(STEPQ_EDEVICE, "device error word 0x%x (%s%s%s)", word, (word & stepq::kErrBadSlot) ? "slot out of range " : "",
-                    (word & stepq::kErrWait) ? "copy wait gave up " : "", (word & stepq::kErrArgs) ? "bad width " : "");
+        return fail(STEPQ_EDEVICE, "device error word 0x%x (%s%s%s%s)", word,
+                    (word & stepq::kErrBadSlot) ? "slot out of range " : "", (word & stepq::kErrWait) ? "copy wait gave up " : "",
+                    (word & stepq::kErrArgs) ? "bad width " : "", (word & stepq::kErrGateRange) ? "prefill gate out of range " : "");
     }
     return STEPQ_OK;
 }
@@ -1020,6 +1021,7 @@ extern "C" int stepq_prefill_fp32(stepq_ctx *c, float *S, int n_req, int lb, int
     a.n_req = n_req; a.T = T; a.nL = le - lb; a.nL_in = le - lb; a.l_in0 = 0; a.H = c->plan->H;
     a.zero_init = zero_init ? 1 : 0;
     a.rows = c->plan->mode == 1;
+    a.err = c->err;
     LaunchTimer lt(c, 4, c->main);
     const cudaError_t e = stepq::launch_prefill(a, c->main);
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
@@ -1064,6 +1066,7 @@ extern "C" int stepq_prefill(stepq_ctx *c, void *pool, const int32_t *slots, int
     p.n_req = n_req; p.T = T; p.nL = le - lb; p.nL_in = le - lb; p.l_in0 = 0; p.H = c->plan->H;
     p.zero_init = from_zero ? 1 : 0;
     p.rows = c->plan->mode == 1;
+    p.err = c->err;
     {
         LaunchTimer lt(c, 4, c->main);
         e = stepq::launch_prefill(p, c->main);

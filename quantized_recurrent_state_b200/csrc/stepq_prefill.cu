@@ -136,7 +136,9 @@ __device__ __forceinline__ void zero(float (&acc)[NTILE][4]) {
 //   S_C = Diag(e^g_C) S_0 + Diag(e^(g_C - g_ref)) (Kh^T diag(beta)) U.
 // The exponents stay within the gates of half a chunk (32 tokens) of the
 // reference, so fp32 holds them while the sum of |log alpha_i| over any 32
-// consecutive tokens stays below about 80.
+// consecutive tokens stays below about 80; a chunk where a row's gates leave
+// that range (or any gate is not in (0, 1]) sets kErrGateRange in the device
+// error word.
 template <bool ROWS>
 __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
     using namespace pf;
@@ -211,6 +213,7 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
                 }
             }
             if (!ROWS) {
+                if (!(isfinite(l2[0]) && isfinite(l2[1]))) atomicOr(a.err, kErrGateRange);
                 float s = l2[0] + l2[1];
 #pragma unroll
                 for (int m = 1; m < 32; m <<= 1) {
@@ -245,6 +248,8 @@ __global__ void __launch_bounds__(pf::NT, 1) k_prefill(PrefillArgs a) {
                     gcol[t * SD] = gs;
                 }
                 const float gr = gcol[((cc - 1) >> 1) * SD];
+                // the factors e^(g - g_ref), e^(g_ref - g) and e^(g_ref) must stay finite
+                if (!(gcol[0] - gr <= 80.0f && gr - gs <= 80.0f && -gr <= 80.0f)) atomicOr(a.err, kErrGateRange);
                 sm.gref[tid] = gr;
                 sm.eref[tid] = expf(gr);
                 sm.egC[tid] = expf(gs);

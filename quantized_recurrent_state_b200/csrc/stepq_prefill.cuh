@@ -4,6 +4,10 @@
 
 namespace stepq {
 
+// Device error word bit set by the prefill: a gate outside (0, 1], or per-row gates whose
+// running log-products leave the range the fp32 factors hold (see k_prefill).
+constexpr int kErrGateRange = 8;
+
 // d = 128; per-head gates (rows = 0) or one gate per key row (rows = 1).
 struct PrefillArgs {
     float *S;                  // [n_req][nL][H][D][D] fp32 states, read (unless zero_init) and written
@@ -14,6 +18,7 @@ struct PrefillArgs {
     int n_req, T, nL, nL_in, l_in0, H;
     int zero_init;
     int rows;
+    int *err;                  // device error word (kErrGateRange)
 };
 
 }  // namespace stepq

@@ -316,3 +316,36 @@ def test_packed_prefill_noop_calls(stepq):
     ctx.prefill(pool, slots, 0, 0, 1, 3, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o, ws)
     ctx.sync()
     assert torch.equal(pool, before)
+
+
+def test_prefill_gates_out_of_range_are_reported(stepq):
+    """Per-row gates whose 32-token log-products leave the fp32 range, and a
+    per-head gate of 0, set the device error word (stepq_sync fails with
+    "prefill gate out of range"); the next valid call runs clean."""
+    plan, data, wl, _ = oracle_plan("kda_rows", n_layers=1, n_pivots=8)
+    ctx = stepq.Context(stepq.Plan.from_bytes(data), 1)
+    inp = {k: torch.from_numpy(v).cuda() for k, v in _prompt(wl, 1, 64, 12).items()}
+    S = torch.zeros((1, 1, wl.n_heads, wl.d, wl.d), dtype=torch.float32, device="cuda")
+    o = torch.zeros_like(inp["q"])
+    bad = inp["alpha"].clone()
+    bad[0, :, 0, 3, 17] = 1e-3                      # one key row: 32 * ln(1e-3) = -221
+    ctx.prefill_fp32(S, 1, 0, 1, 64, inp["q"], inp["k"], inp["v"], bad, inp["beta"], o, zero_init=True)
+    with pytest.raises(stepq.StepqError, match="prefill gate out of range"):
+        ctx.sync()
+    ctx.prefill_fp32(S, 1, 0, 1, 64, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o, zero_init=True)
+    ctx.sync()
+    _check_head(o.cpu().numpy()[0, :, 0, 3], S.cpu().numpy()[0, 0, 3], np.zeros((wl.d, wl.d)),
+                {k: v.cpu().numpy() for k, v in inp.items()}, 0, 3)
+
+    plan, data, wl, _ = oracle_plan("qwen_layer")
+    ctx = stepq.Context(stepq.Plan.from_bytes(data), 1)
+    inp = {k: torch.from_numpy(v).cuda() for k, v in _prompt(wl, 1, 10, 13).items()}
+    S = torch.zeros((1, 1, wl.n_heads, wl.d, wl.d), dtype=torch.float32, device="cuda")
+    o = torch.zeros_like(inp["q"])
+    bad = inp["alpha"].clone()
+    bad[0, 4, 0, 7] = 0.0
+    ctx.prefill_fp32(S, 1, 0, 1, 10, inp["q"], inp["k"], inp["v"], bad, inp["beta"], o, zero_init=True)
+    with pytest.raises(stepq.StepqError, match="prefill gate out of range"):
+        ctx.sync()
+    ctx.prefill_fp32(S, 1, 0, 1, 10, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o, zero_init=True)
+    ctx.sync()
