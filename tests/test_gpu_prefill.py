@@ -349,3 +349,51 @@ def test_prefill_gates_out_of_range_are_reported(stepq):
         ctx.sync()
     ctx.prefill_fp32(S, 1, 0, 1, 10, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o, zero_init=True)
     ctx.sync()
+
+
+@pytest.mark.parametrize("name", ["qwen_layer", "kda_rows"])
+def test_prefill_then_decode(stepq, name):
+    """The serving order: a 100-token prompt prefilled into packed states,
+    then 3 fused decode steps from the records the prefill wrote, checked
+    against the oracle stepping the same records (codes bit-exact up to
+    rounding ties, o within rtol 1e-4 / atol 1e-5)."""
+    kw = {"n_layers": 1, "n_pivots": 8} if name == "kda_rows" else {}
+    plan, data, wl, _ = oracle_plan(name, **kw)
+    pv = model.PlanView(plan)
+    P = stepq.Plan.from_bytes(data)
+    n, T = 2, 100
+    ctx = stepq.Context(P, n)
+    slots = torch.tensor([1, 0], dtype=torch.int32, device="cuda")
+    pool = torch.zeros(n * P.slot_bytes, dtype=torch.uint8, device="cuda")
+    ctx.requant_pack(pool, slots, n, 0, 1, torch.from_numpy(synth.initial_states(wl, wl.seed, n)).cuda())
+    inp = {k: torch.from_numpy(v).cuda() for k, v in _prompt(wl, n, T, 31).items()}
+    o = torch.zeros_like(inp["q"])
+    ws = torch.empty(ctx.prefill_workspace_bytes(n, 1) // 4, dtype=torch.float32, device="cuda")
+    ctx.prefill(pool, slots, n, 0, 1, T, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o, ws)
+    ctx.sync()
+    ref = pool.cpu().numpy().copy()          # the oracle continues from the records the prefill wrote
+    sb = P.slot_bytes
+    alpha = synth.gates(wl, wl.seed)
+    slot_of = slots.cpu().numpy()
+    od = torch.zeros((n, 1, wl.n_heads, wl.d), dtype=torch.float32, device="cuda")
+    for t in range(3):
+        x = synth.step_inputs(wl, wl.seed + 1, n, T + t, alpha=alpha)
+        d = {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in x.items()}
+        ctx.decode_step_fused(pool, slots, n, 0, 1, d["q"], d["k"], d["v"], d["alpha"], d["beta"], od)
+        ctx.sync()
+        got, og = pool.cpu().numpy(), od.cpu().numpy()
+        for r in range(n):
+            s = int(slot_of[r])
+            slot = ref[s * sb:(s + 1) * sb]
+            for h in range(wl.n_heads):
+                o_ref, tie, S, w = pv.step(slot, 0, h, x["q"][r, 0, h], x["k"][r, 0, h], x["v"][r, 0, h],
+                                           x["alpha"][r, 0, h], x["beta"][r, 0, h])
+                assert (np.abs(og[r, 0, h] - o_ref) <= 1e-5 + 1e-4 * np.abs(o_ref)).all(), (t, r, h)
+                rg, ro = pv.record(got[s * sb:(s + 1) * sb], 0, h), pv.record(slot, 0, h)
+                if not np.array_equal(rg, ro):
+                    zg, hg, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(0, h), rg)
+                    zo, ho, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(0, h), ro)
+                    assert not (((zg != zo) | (hg != ho)) & (tie == 0)).any(), (t, r, h)
+            ref[s * sb:(s + 1) * sb] = slot
+        # continue both from the oracle's records, so a tie never compounds
+        pool.copy_(torch.from_numpy(ref).cuda())
