@@ -675,14 +675,18 @@ def run_prefill(args):
     wl = workload_of(args, synth)
     n, T = args.batch, args.prefill
     plan, plan_bytes = product_plan(stepq, synth, wl, device, args.scale_bits)
-    L, H, D = wl.n_layers, wl.n_heads, wl.d
+    H, D = wl.n_heads, wl.d
+    lb, le = (0, wl.n_layers) if args.shard == "replicas" else layer_range(wl.n_layers, ws, rank)
+    if args.shard == "layers":
+        plan = plan.slice(lb, le)   # this rank holds the records of its own layers only
+    L = le - lb
     ctx = stepq.Context(plan, n)
     pool = torch.zeros(n * plan.slot_bytes, dtype=torch.uint8, device=device)
     slots = torch.arange(n, dtype=torch.int32, device=device)
     for l in range(L):
-        ctx.requant_pack(pool, slots, n, l, l + 1, synth.initial_states_torch(wl, wl.seed, n, l, device))
+        ctx.requant_pack(pool, slots, n, l, l + 1, synth.initial_states_torch(wl, wl.seed, n, lb + l, device))
     alpha = synth.gates(wl, wl.seed)
-    inp = synth.prompt_inputs_torch(wl, wl.seed, n, 0, T, alpha, device)
+    inp = synth.prompt_inputs_torch(wl, wl.seed, n, 0, T, alpha, device, lb, le)
     o = torch.zeros_like(inp["q"])
     wsp = torch.empty(ctx.prefill_workspace_bytes(n, L) // 4, dtype=torch.float32, device=device)
     torch.cuda.synchronize()
@@ -714,7 +718,10 @@ def run_prefill(args):
     ctx.set_timing(False)
     launches = ctx.launches - launches0
     stats = ctx.kernel_stats()
-    value, secs = replica_throughput(n * T * args.steps, e0.elapsed_time(e1) / 1e3, ws)
+    # head-tokens summed over ranks, over the pool's heads: tokens through the whole pool
+    # (replicas: every replica's pool; layer shards: the one pool they split)
+    head_tokens, secs = replica_throughput(n * T * args.steps * L * H, e0.elapsed_time(e1) / 1e3, ws)
+    value = head_tokens / (wl.n_layers * H)
 
     k_ms, k_n = stats["prefill"]
     launch_s = k_ms / k_n / 1e3
@@ -728,7 +735,8 @@ def run_prefill(args):
     # the same tokens stepped one at a time by the fused decode step, for comparison
     compare = None
     if rank == 0:
-        sets = [synth.step_inputs_torch(wl, wl.seed, n, t, alpha, device) for t in range(4)]
+        sets = [{k: v[:, lb:le].contiguous() for k, v in synth.step_inputs_torch(wl, wl.seed, n, t, alpha, device).items()}
+                for t in range(4)]
         o2 = torch.zeros((n, L, H, D), dtype=torch.float32, device=device)
         w2 = torch.empty(ctx.workspace_bytes(n, L) // 4, dtype=torch.float32, device=device)
         sec_dec, _, _ = time_steps(torch, ctx, "fused", pool, slots, n, L, sets, o2, w2, 3, 32, 1)
@@ -759,7 +767,7 @@ def run_prefill(args):
                 o_host.copy_(o, non_blocking=True)
         torch.cuda.synchronize()
         t_e2e = max_over_ranks(time.perf_counter() - t0, ws)
-        e2e = {"value": sum_over_ranks(n * T * k_e2e, ws) / t_e2e, "unit": "tokens/s",
+        e2e = {"value": sum_over_ranks(n * T * k_e2e * L * H, ws) / (wl.n_layers * H) / t_e2e, "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e,
                "overlap": "none: the copies and the launches of a step in order on one stream"}
         del host, o_host
@@ -779,13 +787,15 @@ def run_prefill(args):
             "warmup": args.warmup,
             "ms_per_step": secs / args.steps * 1e3,
             "higher_is_better": True,
-            "scaling": "weak",
+            "scaling": "weak" if args.shard == "replicas" else "strong",
             "vs_baseline": None,
             "dtype": "f32 (tensor-core products in TF32 with a TF32 remainder)",
             "data": "synthetic",
             "config": {**prefill_config(wl, n, T, ws), "scale_bits": plan.info.scale_bits,
-                       "pool_bytes": n * plan.slot_bytes},
-            "head_tokens_per_s": value * L * H,
+                       "pool_bytes": n * plan.slot_bytes,
+                       **({"parallelism": f"layer shards x{ws} (rank 0: layers {lb}-{le - 1})"}
+                          if args.shard == "layers" else {})},
+            "head_tokens_per_s": head_tokens,
             "roofline": {"bound": "tensor", "kernel": "prefill", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
                          "algorithmic_flops_per_launch": flops, "launch_ms": launch_s * 1e3,

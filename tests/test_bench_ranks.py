@@ -83,3 +83,31 @@ def test_layer_shards_cover_the_pool_once():
     out = mgr.dict()
     mp.start_processes(_shard_worker, args=(2, port, out), nprocs=2, join=True, start_method="spawn")
     assert out[0] == out[1] == (70 * 48 * 48 * 10 / 1.25, 1.25)
+
+
+def _prefill_worker(rank, ws, port, shard, out):
+    import datetime
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws, timeout=datetime.timedelta(seconds=60))
+    import bench
+    L, H, n, T, steps = 48, 48, 1, 2048, 5
+    lb, le = (0, L) if shard == "replicas" else bench.layer_range(L, ws, rank)
+    secs = 2.0 + rank
+    head_tokens, smax = bench.replica_throughput(n * T * steps * (le - lb) * H, secs, ws)
+    bench.barrier(ws)
+    out[rank] = (head_tokens / (L * H), smax)
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("shard,expect", [("layers", 2048 * 5 / 3.0), ("replicas", 2 * 2048 * 5 / 3.0)])
+def test_prefill_tokens_per_second_two_ranks(shard, expect):
+    # prefill counts tokens through the whole pool: layer shards split one pool's tokens,
+    # replicas each prefill their own pool
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_prefill_worker, args=(2, port, shard, out), nprocs=2, join=True, start_method="spawn")
+    assert out[0] == out[1]
+    assert abs(out[0][0] - expect) < 1e-6 * expect and out[0][1] == 3.0
