@@ -348,6 +348,16 @@ int stepq_kernel_stats(stepq_ctx *ctx, double *ms, uint64_t *launches);
 
 const char *stepq_last_error(void);
 
+/* Self-test of the fifth-generation tensor-core path (tcgen05, kind::tf32) on this device:
+ * one CTA computes D1 = A B1^T with both operands K-major in shared memory and the
+ * accumulator in tensor memory, D2 = D1 B2^T with A read from tensor memory where the first
+ * product left it, and D3 = A B2^T with A written to tensor memory by tcgen05.st.
+ * A [128][32], B1 [32][32], B2 [64][32] (row-major fp32, device, 16-byte aligned);
+ * D1 [128][32], D2 and D3 [128][64] (device, written).  The tensor cores read the fp32
+ * operands truncated to TF32 (the low 13 mantissa bits are dropped).  Synchronous (default
+ * stream); every wait is bounded: STEPQ_EDEVICE if one gave up, tensor memory freed. */
+int stepq_selftest_tc(const float *A, const float *B1, const float *B2, float *D1, float *D2, float *D3);
+
 #ifdef __cplusplus
 }
 #endif

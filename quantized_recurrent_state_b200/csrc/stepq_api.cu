@@ -35,6 +35,8 @@ cudaError_t launch_copy(void *dst, const void *src, size_t bytes, int n_sms, cud
 cudaError_t launch_calib_acc(int D, const Args &a, double *om, double *ls, cudaStream_t st);
 cudaError_t launch_calib_dist(int D, const Args &a, const int *bits, int n_bits, double *acc, cudaStream_t st);
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t st);
+cudaError_t run_tc_selftest(const float *A, const float *B1, const float *B2, float *D1, float *D2, float *D3,
+                            int *word);
 }  // namespace stepq
 
 namespace {
@@ -1078,6 +1080,18 @@ extern "C" int stepq_prefill(stepq_ctx *c, void *pool, const int32_t *slots, int
     e = stepq::launch_pack(c->plan->D, a, false, c->main);
     if (e != cudaSuccess) return cuda_fail(e, "prefill: requant_pack launch");
     lt.done();
+    return STEPQ_OK;
+}
+
+extern "C" int stepq_selftest_tc(const float *A, const float *B1, const float *B2, float *D1, float *D2, float *D3) {
+    int rc;
+    if ((rc = check_ptr(A, 16, "A")) || (rc = check_ptr(B1, 16, "B1")) || (rc = check_ptr(B2, 16, "B2")) ||
+        (rc = check_ptr(D1, 16, "D1")) || (rc = check_ptr(D2, 16, "D2")) || (rc = check_ptr(D3, 16, "D3")))
+        return rc;
+    int word = 0;
+    const cudaError_t e = stepq::run_tc_selftest(A, B1, B2, D1, D2, D3, &word);
+    if (e != cudaSuccess) return cuda_fail(e, "selftest_tc");
+    if (word) return fail(STEPQ_EDEVICE, "selftest_tc: a tensor-core wait gave up");
     return STEPQ_OK;
 }
 

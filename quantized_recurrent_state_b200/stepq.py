@@ -26,7 +26,7 @@ EXPORTED = [
     "stepq_calib_accumulate", "stepq_calib_distortion", "stepq_copy_probe",
     "stepq_launch_count", "stepq_last_error", "stepq_ctx_set_timing", "stepq_kernel_stats",
     "stepq_decode_step_noalloc", "stepq_plan_build_uniform", "stepq_ctx_set_wait_limit", "stepq_plan_slice", "stepq_prefill_fp32", "stepq_prefill",
-    "stepq_prefill_workspace_bytes",
+    "stepq_prefill_workspace_bytes", "stepq_selftest_tc",
 ]
 QUANT_DUAL_AXIS = 0  # plan requantizer: STEPQuant row/column fit
 QUANT_ABSMAX = 1     # plan requantizer: per-row absmax baseline, c = 1
@@ -78,6 +78,7 @@ def lib():
         l.stepq_plan_slice.argtypes = [P, I, I, ctypes.POINTER(P)]
         l.stepq_prefill_fp32.argtypes = [P, P, I, I, I, I, P, P, P, P, P, P, I]
         l.stepq_prefill.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, P, P, I]
+        l.stepq_selftest_tc.argtypes = [P] * 6
         l.stepq_prefill_workspace_bytes.argtypes = [P, I, I]
         l.stepq_prefill_workspace_bytes.restype = ctypes.c_size_t
         l.stepq_ctx_create.argtypes = [P, P, P, I, I, ctypes.POINTER(P)]
@@ -306,6 +307,12 @@ class Context:
             self.close()
         except Exception:
             pass
+
+
+def selftest_tc(A, B1, B2, D1, D2, D3):
+    """stepq_selftest_tc: D1 = A B1^T, D2 = D1 B2^T, D3 = A B2^T on the tensor cores (device
+    tensors: A [128][32], B1 [32][32], B2 [64][32], D1 [128][32], D2 and D3 [128][64])."""
+    return _check(lib().stepq_selftest_tc(_ptr(A), _ptr(B1), _ptr(B2), _ptr(D1), _ptr(D2), _ptr(D3)))
 
 
 def copy_probe(dst, src, nbytes: int, stream):
