@@ -9,10 +9,15 @@ readout -> refit r, c -> pack -> write back.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
                     [--variant two_stream|fused] [--batch B] [--plan 6|4] [--sweep]
+                    [--workload gdn|kda] [--scale-bits 32|16] [--shard replicas|layers]
+                    [--prefill T]
+
+--prefill T times the chunked prefill of T-token prompt chunks into the
+packed pool instead (tokens/s through the whole pool, tensor roofline).
 
 Prints one JSON line (rank 0).  N > 1: launched by torch.distributed.run, one
 independent pool per GPU (no collective on the data path), barrier + max of
-the per-rank device times.
+the per-rank device times; --shard layers splits one pool's layers instead.
 """
 from __future__ import annotations
 

@@ -1,22 +1,30 @@
-// Chunked prefill of per-head states (the step before decode).
+// Chunked prefill of per-head and per-key-row states (the step before decode).
 //
 // A prompt of T tokens runs the same gated delta rule as the decode step
-// (STEPQuant paper digest page, 背景与动机), with a scalar gate alpha_t per
-// (token, head):  S_t = (I - beta_t k_t k_t^T) alpha_t S_{t-1} + beta_t k_t v_t^T,
-// o_t = S_t^T q_t.  In chunks of C = 64 tokens from S_0, with gamma_t the
-// running gate product inside the chunk and Gamma_ts = gamma_t / gamma_s:
-//   (I + M) U = V - diag(gamma) K S_0,   M_ts = Gamma_ts beta_s (k_t . k_s), s < t
-//   O   = diag(gamma) Q S_0 + (L_incl(Q K^T o Gamma) diag(beta)) U
-//   S_C = gamma_C S_0 + K^T diag(beta gamma_C / gamma) U
-// The seven dense products per chunk run on the tensor cores as
-// mma.m16n8k8 TF32 with each fp32 operand split into a TF32 high part and a
-// TF32 remainder (three products per tile: hi*hi + hi*lo + lo*hi), which keeps
-// them near fp32 accuracy; the unit-lower-triangular solve for U runs on the
-// CUDA cores, each warp owning 16 value columns.
+// (STEPQuant paper digest page, 背景与动机), gate first:
+// S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T and
+// o_t = S_t^T q_t, with alpha_t a scalar per (token, head) for per-head units
+// or a vector over the key rows for per-row units.  In chunks of C = 64
+// tokens from S_0, with Gamma_t the running gate product inside the chunk
+// (per key row for per-row gates):
+//   (I + M) U = V - (K o Gamma) S_0,  M_ts = beta_s sum_i k_ti k_si Gamma_ti / Gamma_si, s < t
+//   O   = (Q o Gamma) S_0 + L_incl(A) U,  A_ts = beta_s sum_i q_ti k_si Gamma_ti / Gamma_si
+//   S_C = Diag(Gamma_C) S_0 + (K o (Gamma_C / Gamma) o beta)^T U
+// For per-head gates the ratios are one factor per (t, s) pair; per-row gates
+// are factored per key row around the chunk's middle token (see k_prefill).
 //
-// One CTA of 256 threads per (request, layer, head) prompt, the fp32 state
-// and the chunk's Q, K, V in shared memory (rows padded to avoid bank
-// conflicts).  Head dimension 128.
+// The dense products run on the tensor cores as mma.m16n8k8 TF32 warp tiles
+// with each fp32 operand split into a TF32 high part and a TF32 remainder
+// (three products per tile: hi*hi + hi*lo + lo*hi), which keeps them near
+// fp32 accuracy.  The unit lower triangular solve for U goes in blocks of 16
+// rows: four warps invert the diagonal blocks by substitution in registers,
+// then each warp forms its 16 value columns of every block with two small
+// tensor-core products.
+//
+// One CTA of 256 threads per (request, layer, head) prompt holds the fp32
+// state and the chunk's K, Q, V, M in shared memory (row strides chosen for
+// conflict-free fragment loads); the next chunk's K (per-head gates) and Q
+// arrive by cp.async while the current chunk is computed.  Head dimension 128.
 #include "stepq_dev.cuh"
 #include "stepq_prefill.cuh"
 
