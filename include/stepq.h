@@ -222,6 +222,16 @@ size_t stepq_workspace_bytes(const stepq_ctx *ctx, int n_req, int n_layers_launc
 int stepq_prefill_fp32(stepq_ctx *ctx, float *S, int n_req, int lb, int le, int T, const float *q,
                        const float *k, const float *v, const float *alpha, const float *beta, float *o,
                        int zero_init);
+/* Which kernel the prefill of per-head plans runs (per-row plans always use the first):
+ * STEPQ_PREFILL_MMA_SYNC (default): the chunk's products as mma.sync TF32 warp tiles,
+ *   the state in shared memory;
+ * STEPQ_PREFILL_TCGEN05: the state in tensor memory as the A operand of K S and Q S
+ *   and the accumulator of the update, those three products on tcgen05 (kind::tf32,
+ *   operands from shared memory), the rest on mma.sync; same results within the
+ *   tolerance stated in the tests.  Applies to later calls. */
+#define STEPQ_PREFILL_MMA_SYNC 0
+#define STEPQ_PREFILL_TCGEN05 1
+int stepq_ctx_set_prefill_kernel(stepq_ctx *ctx, int kernel);
 /* Bytes of the fp32 workspace stepq_prefill needs for n_layers layers of the
  * batch (n_req * n_layers * n_heads * D * D * 4); 0 for a null context or a
  * negative count. */

@@ -35,6 +35,7 @@ cudaError_t launch_copy(void *dst, const void *src, size_t bytes, int n_sms, cud
 cudaError_t launch_calib_acc(int D, const Args &a, double *om, double *ls, cudaStream_t st);
 cudaError_t launch_calib_dist(int D, const Args &a, const int *bits, int n_bits, double *acc, cudaStream_t st);
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t st);
+cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st);
 cudaError_t run_tc_selftest(const float *A, const float *B1, const float *B2, float *D1, float *D2, float *D3,
                             int *word);
 }  // namespace stepq
@@ -616,6 +617,7 @@ struct stepq_ctx {
     uint64_t launches = 0;
     bool timing = false;
     uint32_t wait_polls = 1u << 22, phantom_tx = 0;
+    int prefill_kernel = STEPQ_PREFILL_MMA_SYNC;
     struct Timed { int kind; cudaEvent_t a, b; };
     std::vector<Timed> timed;
     std::vector<cudaEvent_t> ev_pool;
@@ -707,6 +709,9 @@ struct LaunchTimer {
         }
     }
 };
+
+// The tensor-memory prefill kernel serves per-head units; per-row plans keep the other one.
+bool use_tc_prefill(const stepq_ctx *c) { return c->prefill_kernel == STEPQ_PREFILL_TCGEN05 && c->plan->mode == 0; }
 
 int wait_side(stepq_ctx *c, int lb, int le) {
     for (int l = lb; l < le; ++l) {
@@ -974,6 +979,14 @@ extern "C" int stepq_ctx_set_wait_limit(stepq_ctx *c, uint32_t polls, uint32_t p
     return STEPQ_OK;
 }
 
+extern "C" int stepq_ctx_set_prefill_kernel(stepq_ctx *c, int kernel) {
+    if (!c) return fail(STEPQ_EINVAL, "set_prefill_kernel: null context");
+    if (kernel != STEPQ_PREFILL_MMA_SYNC && kernel != STEPQ_PREFILL_TCGEN05)
+        return fail(STEPQ_EINVAL, "set_prefill_kernel: kernel %d", kernel);
+    c->prefill_kernel = kernel;
+    return STEPQ_OK;
+}
+
 extern "C" int stepq_sync(stepq_ctx *c, int timeout_ms) {
     if (!c) return fail(STEPQ_EINVAL, "sync: null context");
     int rc = set_device(c);
@@ -1025,7 +1038,7 @@ extern "C" int stepq_prefill_fp32(stepq_ctx *c, float *S, int n_req, int lb, int
     a.rows = c->plan->mode == 1;
     a.err = c->err;
     LaunchTimer lt(c, 4, c->main);
-    const cudaError_t e = stepq::launch_prefill(a, c->main);
+    const cudaError_t e = use_tc_prefill(c) ? stepq::launch_prefill_tc(a, c->main) : stepq::launch_prefill(a, c->main);
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
     lt.done();
     return STEPQ_OK;
@@ -1071,7 +1084,7 @@ extern "C" int stepq_prefill(stepq_ctx *c, void *pool, const int32_t *slots, int
     p.err = c->err;
     {
         LaunchTimer lt(c, 4, c->main);
-        e = stepq::launch_prefill(p, c->main);
+        e = use_tc_prefill(c) ? stepq::launch_prefill_tc(p, c->main) : stepq::launch_prefill(p, c->main);
         if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
         lt.done();
     }

@@ -26,8 +26,10 @@ EXPORTED = [
     "stepq_calib_accumulate", "stepq_calib_distortion", "stepq_copy_probe",
     "stepq_launch_count", "stepq_last_error", "stepq_ctx_set_timing", "stepq_kernel_stats",
     "stepq_decode_step_noalloc", "stepq_plan_build_uniform", "stepq_ctx_set_wait_limit", "stepq_plan_slice", "stepq_prefill_fp32", "stepq_prefill",
-    "stepq_prefill_workspace_bytes", "stepq_selftest_tc",
+    "stepq_prefill_workspace_bytes", "stepq_selftest_tc", "stepq_ctx_set_prefill_kernel",
 ]
+PREFILL_MMA_SYNC = 0   # prefill kernel: mma.sync tiles, state in shared memory (default)
+PREFILL_TCGEN05 = 1    # prefill kernel: state in tensor memory, state products on tcgen05
 QUANT_DUAL_AXIS = 0  # plan requantizer: STEPQuant row/column fit
 QUANT_ABSMAX = 1     # plan requantizer: per-row absmax baseline, c = 1
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -79,6 +81,7 @@ def lib():
         l.stepq_prefill_fp32.argtypes = [P, P, I, I, I, I, P, P, P, P, P, P, I]
         l.stepq_prefill.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, P, P, I]
         l.stepq_selftest_tc.argtypes = [P] * 6
+        l.stepq_ctx_set_prefill_kernel.argtypes = [P, I]
         l.stepq_prefill_workspace_bytes.argtypes = [P, I, I]
         l.stepq_prefill_workspace_bytes.restype = ctypes.c_size_t
         l.stepq_ctx_create.argtypes = [P, P, P, I, I, ctypes.POINTER(P)]
@@ -256,6 +259,9 @@ class Context:
         self._after_caller()
         return _check(lib().stepq_prefill_fp32(self._h, _ptr(S), n_req, lb, le, int(T), _ptr(q), _ptr(k), _ptr(v),
                                                _ptr(alpha), _ptr(beta), _ptr(o), 1 if zero_init else 0))
+
+    def set_prefill_kernel(self, kernel: int):
+        return _check(lib().stepq_ctx_set_prefill_kernel(self._h, kernel))
 
     def prefill_workspace_bytes(self, n_req: int, n_layers: int) -> int:
         return int(lib().stepq_prefill_workspace_bytes(self._h, n_req, n_layers))

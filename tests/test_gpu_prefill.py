@@ -397,3 +397,73 @@ def test_prefill_then_decode(stepq, name):
             ref[s * sb:(s + 1) * sb] = slot
         # continue both from the oracle's records, so a tie never compounds
         pool.copy_(torch.from_numpy(ref).cuda())
+
+
+# ---- the tensor-memory (tcgen05) prefill kernel for per-head plans ------------------
+
+@pytest.mark.parametrize("T", [1, 65, 200])
+def test_prefill_tcgen05_matches_sequential(stepq, T):
+    plan, data, wl, _ = oracle_plan("qwen_layer")
+    ctx = stepq.Context(stepq.Plan.from_bytes(data), 2)
+    ctx.set_prefill_kernel(stepq.PREFILL_TCGEN05)
+    S0 = synth.initial_states(wl, wl.seed, 2)
+    inp = _prompt(wl, 2, T, 5000 + T)
+    d = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
+    S = torch.from_numpy(S0).cuda()
+    o = torch.zeros_like(d["q"])
+    ctx.prefill_fp32(S, 2, 0, 1, T, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)
+    ctx.sync()
+    Sg, og = S.cpu().numpy(), o.cpu().numpy()
+    for (r, h) in [(0, 0), (1, 11), (0, 30), (1, 47)]:
+        _check_head(og[r, :, 0, h], Sg[r, 0, h], S0[r, 0, h].astype(np.float64), inp, r, h)
+
+
+def test_prefill_tcgen05_packed_layer_range_and_gate_errors(stepq):
+    plan, data, wl, _ = uniform_plan("qwen_pool6", 6, model.QUANT_DUAL_AXIS, n_layers=3)
+    pv = model.PlanView(plan)
+    P = stepq.Plan.from_bytes(data)
+    n, T, lb, le = 2, 130, 1, 3
+    ctx = stepq.Context(P, 2)
+    ctx.set_prefill_kernel(stepq.PREFILL_TCGEN05)
+    slots = torch.tensor([1, 0], dtype=torch.int32, device="cuda")
+    pool = torch.zeros(2 * P.slot_bytes, dtype=torch.uint8, device="cuda")
+    ctx.requant_pack(pool, slots, n, 0, 3, torch.from_numpy(synth.initial_states(wl, wl.seed, n)).cuda())
+    ctx.sync()
+    before = pool.cpu().numpy().copy()
+    inp = {k: np.ascontiguousarray(v[:, :, lb:le]) for k, v in _prompt(wl, n, T, 9).items()}
+    d = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
+    o = torch.zeros_like(d["q"])
+    ws = torch.empty(ctx.prefill_workspace_bytes(n, le - lb) // 4, dtype=torch.float32, device="cuda")
+    ctx.prefill(pool, slots, n, lb, le, T, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o, ws)
+    ctx.sync()
+    after, og = pool.cpu().numpy(), o.cpu().numpy()
+    S_T = ws.view(n, le - lb, wl.n_heads, wl.d, wl.d).cpu().numpy()
+    sb = P.slot_bytes
+    for r, s in enumerate((1, 0)):
+        prev_slot, new_slot = before[s * sb:(s + 1) * sb], after[s * sb:(s + 1) * sb]
+        for li, l in enumerate(range(lb, le)):
+            for h in (0, 25, 47):
+                _check_head(og[r, :, li, h], S_T[r, li, h], pv.reconstruct(prev_slot, l, h).astype(np.float64),
+                            inp, r, h, li)
+                _check_record(pv, new_slot, l, h, S_T[r, li, h])
+    bad = d["alpha"].clone()
+    bad[0, 3, 0, 5] = 0.0
+    ctx.prefill(pool, slots, n, lb, le, T, d["q"], d["k"], d["v"], bad, d["beta"], o, ws)
+    with pytest.raises(stepq.StepqError, match="prefill gate out of range"):
+        ctx.sync()
+
+
+def test_prefill_tcgen05_setting_leaves_per_row_plans_on_mma_sync(stepq):
+    plan, data, wl, _ = oracle_plan("kda_rows", n_layers=1, n_pivots=8)
+    ctx = stepq.Context(stepq.Plan.from_bytes(data), 1)
+    ctx.set_prefill_kernel(stepq.PREFILL_TCGEN05)
+    with pytest.raises(stepq.StepqError):
+        ctx.set_prefill_kernel(7)
+    S0 = synth.initial_states(wl, wl.seed, 1)
+    inp = _prompt(wl, 1, 70, 4)
+    d = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
+    S = torch.from_numpy(S0).cuda()
+    o = torch.zeros_like(d["q"])
+    ctx.prefill_fp32(S, 1, 0, 1, 70, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)
+    ctx.sync()
+    _check_head(o.cpu().numpy()[0, :, 0, 9], S.cpu().numpy()[0, 0, 9], S0[0, 0, 9].astype(np.float64), inp, 0, 9)
