@@ -10,7 +10,7 @@ readout -> refit r, c -> pack -> write back.
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
                     [--variant two_stream|fused] [--batch B] [--plan 6|4] [--sweep]
                     [--workload gdn|kda] [--scale-bits 32|16] [--shard replicas|layers]
-                    [--prefill T]
+                    [--prefill T [--prefill-kernel mma_sync|tcgen05]]
 
 --prefill T times the chunked prefill of T-token prompt chunks into the
 packed pool instead (tokens/s through the whole pool, tensor roofline).
@@ -66,6 +66,9 @@ def parse():
     ap.add_argument("--prefill", type=int, default=0, metavar="T",
                     help="time chunked prefill of T-token prompt chunks into the packed pool (GDN) instead of "
                          "the decode step; batch defaults to 1")
+    ap.add_argument("--prefill-kernel", default="mma_sync", choices=["mma_sync", "tcgen05"],
+                    help="prefill kernel for per-head plans: mma.sync tiles (default) or the state in "
+                         "tensor memory with its products on tcgen05")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -686,6 +689,8 @@ def run_prefill(args):
         plan = plan.slice(lb, le)   # this rank holds the records of its own layers only
     L = le - lb
     ctx = stepq.Context(plan, n)
+    if args.prefill_kernel == "tcgen05":
+        ctx.set_prefill_kernel(stepq.PREFILL_TCGEN05)
     pool = torch.zeros(n * plan.slot_bytes, dtype=torch.uint8, device=device)
     slots = torch.arange(n, dtype=torch.int32, device=device)
     for l in range(L):
@@ -798,6 +803,7 @@ def run_prefill(args):
             "data": "synthetic",
             "config": {**prefill_config(wl, n, T, ws), "scale_bits": plan.info.scale_bits,
                        "pool_bytes": n * plan.slot_bytes,
+                       "prefill_kernel": args.prefill_kernel if wl.mode == 0 else "mma_sync",
                        **({"parallelism": f"layer shards x{ws} (rank 0: layers {lb}-{le - 1})"}
                           if args.shard == "layers" else {})},
             "head_tokens_per_s": head_tokens,
