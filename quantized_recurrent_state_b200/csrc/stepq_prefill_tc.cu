@@ -24,7 +24,6 @@ namespace stepq {
 
 namespace tcpf {
 
-
 constexpr int D = 128, C = 64, NT = 256;
 constexpr int SV = D + 8, SC = C + 4;
 constexpr uint32_t kPolls = 1u << 24;
@@ -133,10 +132,6 @@ __device__ __forceinline__ void warp_gemm_split(float (&acc)[NTILE][4], const fl
 
 __device__ __forceinline__ int xoff(int t, int i) { return (int)(tc::kmajor_off(t, i, D) >> 2); }   // X[t][i]
 __device__ __forceinline__ int ktoff(int i, int t) { return (int)(tc::kmajor_off(i, t, C) >> 2); }  // KT[i][t]
-
-}  // namespace tcpf
-
-namespace tcpf {
 
 __global__ void __launch_bounds__(NT, 1) k_prefill_tc(PrefillArgs a) {
     extern __shared__ __align__(1024) uint8_t smraw[];
