@@ -195,6 +195,10 @@ void stepq_ctx_free(stepq_ctx *ctx);
 size_t stepq_workspace_bytes(const stepq_ctx *ctx, int n_req, int n_layers_launched);
 
 /* ---- prefill (the step before decode) ----------------------------------- */
+/* Source: the STEPQuant project page, 快速上手 (the serving command prefills prompts in
+ * chunks of 2,048 tokens), with the recurrence of the paper digest page, 背景与动机; the
+ * chunk form below restates that recurrence over a block of tokens (no requantization
+ * between tokens; the packed entry point requantizes the final state once). */
 
 /* Chunked prefill of T tokens on fp32 states (d = 128, either unit kind):
  * for every (request, layer in [lb, le), head) the gated delta rule above,
