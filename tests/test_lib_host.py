@@ -209,3 +209,14 @@ def test_plan_slice_matches_oracle(mode, sbits):
                     mode, D, plan_io.head_row_widths(so, l, h), sbits))
     with pytest.raises(stepq.StepqError):
         p.slice(3, 3)
+
+
+def test_new_entry_points_reject_bad_arguments_without_a_device():
+    """Argument checks come before any CUDA call: a null context or pointer, or an
+    unknown prefill kernel, is STEPQ_EINVAL with a message."""
+    l = stepq.lib()
+    assert l.stepq_ctx_set_prefill_kernel(None, stepq.PREFILL_TCGEN05) == stepq.EINVAL
+    assert b"null context" in l.stepq_last_error()
+    assert l.stepq_selftest_tc(None, None, None, None, None, None) == stepq.EINVAL
+    assert b"A" in l.stepq_last_error()
+    assert l.stepq_prefill_workspace_bytes(None, 1, 1) == 0
