@@ -70,6 +70,8 @@ def _declare(l):
     l.sq_unpack_rows.argtypes = [I, P, P, P, P]
     l.sq_pairwise_sum.argtypes = [P, I]
     l.sq_pairwise_sum.restype = F
+    l.sq_band_dot.argtypes = [I, P, I, P, I]
+    l.sq_band_dot.restype = F
     l.sq_quantize.argtypes = [I, P, P, P, P, P, P, P, P, P, P]
     l.sq_quantize_absmax.argtypes = [I, P, P, P, P, P, P, P]
     l.sq_quantize_s.argtypes = [I, P, P, P, P, P, P, P, P, P, P, I]
@@ -165,6 +167,14 @@ def unpack_rows(D: int, widths, blk: np.ndarray):
 def pairwise_sum(x: np.ndarray) -> np.float32:
     x = _f32(x)
     return np.float32(lib().sq_pairwise_sum(_p(x), x.size))
+
+
+def band_dot(x: np.ndarray, y: np.ndarray) -> np.float32:
+    """sum_i x_i y_i over D = len(x) rows in band order (see sq_band_dot)."""
+    x = _f32(x)
+    y = _f32(y)
+    assert x.size == y.size and x.size % 16 == 0
+    return np.float32(lib().sq_band_dot(x.size, _p(x), 1, _p(y), 1))
 
 
 def f32_to_bf16(x: float) -> int:

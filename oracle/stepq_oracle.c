@@ -117,10 +117,18 @@ static float round_scale(float x, int scale_bits)
 /* u = z + 2^(b-1), in [1, 2^b - 1] for |z| <= qmax = 2^(b-1) - 1.            */
 /*                                                                          */
 /* Uniform-width unit (a head whose rows all share width b):                */
-/*   RT = D/8 rows per band, NT = 2D threads.  Element (i,j) belongs to     */
-/*   thread t = (i/RT)*(D/4) + j/4 at stream position p = (i%RT)*4 + j%4.    */
-/*   Its field occupies stream bits [p*b, p*b+b) (LSB-first bytes).  Stream  */
-/*   byte B of thread t lives at block byte ((B/RT)*NT + t)*RT + B%RT.        */
+/*   RT = D/8 rows per band, NT = 2D tiles.  Tile tau = (j/4)*8 + i/RT       */
+/*   holds the RT x 4 block of rows [RT*(i/RT), +RT) and columns             */
+/*   [4*(j/4), +4); inside it (i,j) is the tile code (r, c) = (i%RT, j%4).    */
+/*   Tile tau's codes form a bit stream; stream byte B lives at block byte   */
+/*   ((B/RT)*NT + tau)*RT + B%RT.  Inside the stream, code (r, c):           */
+/*     b = 2, 4, 8, and b = 6 with RT < 4: bits [(4r+c)*b, +b), LSB first;   */
+/*     b = 6 with RT >= 4: rows go in groups of four, r = 4g + s, over the    */
+/*       32-bit little-endian stream words 3g, 3g+1, 3g+2.  Rows s = 0, 1, 3 */
+/*       have their 24-bit row value V = sum_c u_c 2^(6c) in bits [0, 24) of */
+/*       words 3g, 3g+1, 3g+2; the 24-bit value of row s = 2 is stored byte  */
+/*       by byte in bits [24, 32) of the same three words (byte m in word     */
+/*       3g+m).                                                             */
 /* Row-major unit (rows of mixed width): row i starts at the sum of the     */
 /*   byte sizes D*b/8 of the rows before it; code j occupies row bits         */
 /*   [b*j, b*j+b).  A 16-bit row holds binary16 values, 2 bytes per column.  */
@@ -133,12 +141,26 @@ static void set_bit(uint8_t *blk, long bit, int v)
     else   blk[bit >> 3] &= (uint8_t)~(1u << (bit & 7));
 }
 
-/* Block bit address of stream bit s of thread t (uniform layout). */
-static long uniform_bit_addr(int D, int t, long s)
+/* Stream bit of bit k (0 = least significant) of tile code (r, c). */
+static long tile_stream_bit(int D, int b, int r, int c, int k)
+{
+    int RT = D / 8;
+    if (b != 6 || RT < 4) return (long)(4 * r + c) * b + k;
+    int g = r / 4, s = r % 4;
+    int v = 6 * c + k;                        /* bit of the 24-bit row value */
+    if (s == 2) return (long)(3 * g + v / 8) * 32 + 24 + v % 8;
+    int word = 3 * g + (s == 3 ? 2 : s);
+    return (long)word * 32 + v;
+}
+
+/* Block bit address of bit k of code (i, j) of a uniform-width unit. */
+static long uniform_bit_addr(int D, int b, int i, int j, int k)
 {
     int RT = D / 8, NT = 2 * D;
+    long tau = (long)(j / 4) * 8 + i / RT;
+    long s = tile_stream_bit(D, b, i % RT, j % 4, k);
     long B = s >> 3;
-    long byte = ((B / RT) * NT + t) * RT + (B % RT);
+    long byte = ((B / RT) * NT + tau) * RT + (B % RT);
     return byte * 8 + (s & 7);
 }
 
@@ -146,28 +168,22 @@ long sq_codes_bytes_uniform(int D, int b) { return (long)D * D * b / 8; }
 
 void sq_pack_uniform(int D, int b, const int32_t *z, uint8_t *blk)
 {
-    int RT = D / 8;
     memset(blk, 0, (size_t)sq_codes_bytes_uniform(D, b));
     for (int i = 0; i < D; i++)
         for (int j = 0; j < D; j++) {
-            int t = (i / RT) * (D / 4) + j / 4;
-            int p = (i % RT) * 4 + j % 4;
             unsigned u = (unsigned)(z[i * D + j] + (1 << (b - 1)));
             for (int k = 0; k < b; k++)
-                set_bit(blk, uniform_bit_addr(D, t, (long)p * b + k), (u >> k) & 1);
+                set_bit(blk, uniform_bit_addr(D, b, i, j, k), (u >> k) & 1);
         }
 }
 
 void sq_unpack_uniform(int D, int b, const uint8_t *blk, int32_t *z)
 {
-    int RT = D / 8;
     for (int i = 0; i < D; i++)
         for (int j = 0; j < D; j++) {
-            int t = (i / RT) * (D / 4) + j / 4;
-            int p = (i % RT) * 4 + j % 4;
             unsigned u = 0;
             for (int k = 0; k < b; k++)
-                u |= (unsigned)get_bit(blk, uniform_bit_addr(D, t, (long)p * b + k)) << k;
+                u |= (unsigned)get_bit(blk, uniform_bit_addr(D, b, i, j, k)) << k;
             z[i * D + j] = (int32_t)u - (1 << (b - 1));
         }
 }
@@ -230,13 +246,40 @@ void sq_unpack_rows(int D, const int *widths, const uint8_t *blk, int32_t *z, ui
 
 /* fp32 pairwise sum of n = 2^m terms: sum(x[0:n]) = sum(x[0:n/2]) +
  * sum(x[n/2:n]), each addition rounded to fp32.  This is the summation order
- * the quantizer's row and column sums are defined with. */
+ * of the quantizer's row sums (the row mean of r_i). */
 float sq_pairwise_sum(const float *x, int n)
 {
     if (n == 1) return x[0];
     float a = sq_pairwise_sum(x, n / 2);
     float b = sq_pairwise_sum(x + n / 2, n / 2);
     return a + b;
+}
+
+/* Band-order dot product over the D rows of a column: sum_i x_i y_i in fp32,
+ * the order in which u, o and the two refinement sums are defined.
+ *   - The rows form 8 bands of RT = D/8 consecutive rows.
+ *   - Inside band g the even rows (g*RT + 0, 2, ...) and the odd rows
+ *     (g*RT + 1, 3, ...) are each accumulated by a chain of fused
+ *     multiply-adds that starts at +0: acc = fma(x_i, y_i, acc), rows in
+ *     increasing order.  The band's value is fl(even chain + odd chain).
+ *   - The 8 band values are added in a balanced binary tree in band order:
+ *     ((b0 + b1) + (b2 + b3)) + ((b4 + b5) + (b6 + b7)).
+ * x and y are read with strides sx and sy (a column of a row-major D x D
+ * array has stride D). */
+float sq_band_dot(int D, const float *x, int sx, const float *y, int sy)
+{
+    int RT = D / 8;
+    float band[8];
+    for (int g = 0; g < 8; g++) {
+        float even = 0.0f, odd = 0.0f;
+        for (int m = 0; m < RT; m += 2) {
+            int i = g * RT + m;
+            even = fmaf(x[(long)i * sx], y[(long)i * sy], even);
+            odd = fmaf(x[(long)(i + 1) * sx], y[(long)(i + 1) * sy], odd);
+        }
+        band[g] = even + odd;
+    }
+    return sq_pairwise_sum(band, 8);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -251,11 +294,13 @@ float sq_pairwise_sum(const float *x, int n)
 /*   - the row mean is the fp32 pairwise sum of |S_ij| over j, times 1/D;     */
 /*   - S/(r c) is taken as y = fl(S * fl(1/r)) and then the exact product    */
 /*     y * fl(1/c) is rounded to the nearest integer, ties to even;          */
-/*   - c0_j = max_i fl(|y_ij| / qmax_i); an all-zero column gets c0 = 1;      */
-/*   - the refinement sums are fp32 pairwise sums over i of                   */
-/*     fl(b_i * fl(z0*y)) and fl(b_i * fl(z0*z0)), b_i = fl(wbar_i*fl(r_i r_i)),*/
-/*     which equal w r z0 S and w r^2 z0^2 up to the common factor 1/r;       */
-/*     rows of 16-bit (pivot) width contribute 0; a zero denominator keeps c0; */
+/*   - dividing by qmax is a product with fl(1/qmax):                        */
+/*     c0_j = max_i fl(|y_ij| * fl(1/qmax_i)); an all-zero column gets 1;     */
+/*   - with t_ij = fl(b_i * z0_ij), b_i = fl(wbar_i * fl(r_i * r_i)), the     */
+/*     refinement is c_j = fl(N_j / D_j) with N_j = sum_i t_ij y_ij and       */
+/*     D_j = sum_i t_ij z0_ij in band order (sq_band_dot); these equal        */
+/*     sum w r z0 S and sum w r^2 z0^2 up to the common factor 1/r;          */
+/*     rows of 16-bit (pivot) width have t = 0; a zero denominator keeps c0; */
 /*   - c_j is rounded to fp32 before the final codes are taken.               */
 /*   - 16-bit scale storage (scale_bits = 16, the pages' 16-bit scale        */
 /*     accounting, 局限): r_i is rounded                                      */
@@ -284,8 +329,9 @@ void sq_quantize_s(int D, const int *widths, const float *rho, const float *wbar
     float *absrow = (float *)malloc(sizeof(float) * D);
     float *y = (float *)malloc(sizeof(float) * D * D);
     float *bw = (float *)malloc(sizeof(float) * D);
-    float *tn = (float *)malloc(sizeof(float) * D);
-    float *td = (float *)malloc(sizeof(float) * D);
+    float *t = (float *)malloc(sizeof(float) * D);
+    float *z0f = (float *)malloc(sizeof(float) * D);
+    float *ycol = (float *)malloc(sizeof(float) * D);
     int32_t *z0 = (int32_t *)malloc(sizeof(int32_t) * D * D);
     uint8_t *coltie = (uint8_t *)calloc(D, 1);
 
@@ -319,25 +365,24 @@ void sq_quantize_s(int D, const int *widths, const float *rho, const float *wbar
         float c0 = 0.0f;
         for (int i = 0; i < D; i++) {
             if (widths[i] == SQ_PIVOT_BITS) continue;
-            float v = fabsf(y[i * D + j]) / (float)qmax_of(widths[i]);
+            float iq = 1.0f / (float)qmax_of(widths[i]);
+            float v = fabsf(y[i * D + j]) * iq;
             if (v > c0) c0 = v;
         }
         if (c0 == 0.0f) c0 = 1.0f;
         float inv_c0 = 1.0f / c0;
-        /* initial codes and weighted least-squares refinement */
+        /* initial codes and the weighted least-squares refinement */
         for (int i = 0; i < D; i++) {
-            if (widths[i] == SQ_PIVOT_BITS) { tn[i] = 0.0f; td[i] = 0.0f; continue; }
-            double x0 = (double)y[i * D + j] * (double)inv_c0;
+            ycol[i] = y[i * D + j];
+            if (widths[i] == SQ_PIVOT_BITS) { z0[i * D + j] = 0; z0f[i] = 0.0f; t[i] = 0.0f; continue; }
+            double x0 = (double)y[i * D + j] * (double)inv_c0; /* exact: 24 x 24 bits */
             z0[i * D + j] = (int32_t)rint(x0);
             if (near_half(x0)) coltie[j] = 1;
-            float zf = (float)z0[i * D + j];
-            float pn = zf * y[i * D + j];
-            float pd = zf * zf;
-            tn[i] = bw[i] * pn;
-            td[i] = bw[i] * pd;
+            z0f[i] = (float)z0[i * D + j];
+            t[i] = bw[i] * z0f[i];
         }
-        float num = sq_pairwise_sum(tn, D);
-        float den = sq_pairwise_sum(td, D);
+        float num = sq_band_dot(D, t, 1, ycol, 1);
+        float den = sq_band_dot(D, t, 1, z0f, 1);
         float cj = round_scale((den > 0.0f) ? num / den : c0, scale_bits);
         c[j] = cj;
         float inv_c = 1.0f / cj;
@@ -362,7 +407,7 @@ void sq_quantize_s(int D, const int *widths, const float *rho, const float *wbar
             for (int j = 0; j < D; j++)
                 z0_out[i * D + j] = (widths[i] == SQ_PIVOT_BITS) ? 0 : z0[i * D + j];
 
-    free(absrow); free(y); free(bw); free(tn); free(td); free(z0); free(coltie);
+    free(absrow); free(y); free(bw); free(t); free(z0f); free(ycol); free(z0); free(coltie);
 }
 
 void sq_quantize(int D, const int *widths, const float *rho, const float *wbar,
@@ -446,14 +491,13 @@ void sq_reconstruct(int D, const int *widths, const int32_t *z, const uint16_t *
 /*                                                                          */
 /* Recurrence (gated delta rule; KDA reading with Diag(alpha) applied first): */
 /*   S_t = (I - beta k k^T) Diag(alpha) S_{t-1} + beta k v^T,  o_t = S_t^T q  */
-/* Readings:                                                                 */
+/* Readings (the pages fix the update in fp32 and no summation order):        */
 /*   - retention is folded into the row factor: a_i = fl(alpha_i r_i) and      */
 /*     S'_ij = fl(fl(a_i c_j) z_ij); 16-bit rows: S'_ij = fl(alpha_i h_ij);   */
-/*   - u_j = sum_i k_i R_ij with R_ij = a_i c_j z_ij (or alpha_i h_ij) the    */
-/*     exact retained reconstruction, evaluated in fp64 and rounded once;     */
+/*   - u_j = sum_i k_i S'_ij in band order (sq_band_dot);                     */
 /*   - w_j = fl(beta * fl(v_j - u_j));  S_ij = fma(k_i, w_j, S'_ij);           */
-/*   - o_j = sum_i q_i (R_ij + k_i w_j) in fp64, rounded once: the readout of */
-/*     the updated state, taken before requantization.                        */
+/*   - o_j = sum_i q_i S_ij in band order over the updated fp32 state: the    */
+/*     readout of S_t, taken before requantization.                           */
 /* alpha has D entries (GDN: all equal).  S_out receives the fp32 S_t that    */
 /* the requantizer consumes.                                                 */
 /* ------------------------------------------------------------------------ */
@@ -464,43 +508,29 @@ void sq_step_from_codes(int D, const int *widths, const int32_t *z, const uint16
                         const float *alpha, float beta,
                         float *S_out, float *o_out, float *u_out, float *w_out)
 {
-    double *R = (double *)malloc(sizeof(double) * D * D);
     float *w = (float *)malloc(sizeof(float) * D);
     for (int i = 0; i < D; i++) {
         if (widths[i] == SQ_PIVOT_BITS) {
-            for (int j = 0; j < D; j++) {
-                float hv = sq_f16_to_f32(h[i * D + j]);
-                S_out[i * D + j] = alpha[i] * hv;
-                R[i * D + j] = (double)alpha[i] * (double)hv;
-            }
+            for (int j = 0; j < D; j++) S_out[i * D + j] = alpha[i] * sq_f16_to_f32(h[i * D + j]);
         } else {
             float a = alpha[i] * r[i];
             for (int j = 0; j < D; j++) {
                 float A = a * c[j];
                 S_out[i * D + j] = A * (float)z[i * D + j];
-                R[i * D + j] = (double)a * (double)c[j] * (double)z[i * D + j];
             }
         }
     }
     for (int j = 0; j < D; j++) {
-        double acc = 0.0;
-        for (int i = 0; i < D; i++) acc += (double)k[i] * R[i * D + j];
-        float u = (float)acc;
+        float u = sq_band_dot(D, k, 1, S_out + j, D);
         float d = v[j] - u;
         w[j] = beta * d;
         if (u_out) u_out[j] = u;
         if (w_out) w_out[j] = w[j];
     }
-    for (int j = 0; j < D; j++) {
-        double acc = 0.0;
-        for (int i = 0; i < D; i++)
-            acc += (double)q[i] * (R[i * D + j] + (double)k[i] * (double)w[j]);
-        o_out[j] = (float)acc;
-    }
     for (int i = 0; i < D; i++)
         for (int j = 0; j < D; j++)
             S_out[i * D + j] = fmaf(k[i], w[j], S_out[i * D + j]);
-    free(R);
+    for (int j = 0; j < D; j++) o_out[j] = sq_band_dot(D, q, 1, S_out + j, D);
     free(w);
 }
 

@@ -70,8 +70,9 @@ def test_rows_pack_roundtrip():
 
 
 def _golden_layout():
+    """Cases of tests/golden/layout_uniform.txt: name -> (D, b, sets, expect)."""
     cases = {}
-    with open(os.path.join(GOLDEN, "layout_d16.txt")) as f:
+    with open(os.path.join(GOLDEN, "layout_uniform.txt")) as f:
         for line in f:
             line = line.strip()
             if not line or line.startswith("#"):
@@ -81,30 +82,31 @@ def _golden_layout():
     return cases
 
 
-def test_uniform_layout_hand_bytes():
-    cases = _golden_layout()
-    # b = 4 case
-    z = np.zeros((16, 16), np.int32)
-    for item in cases["b4"]["set"]:
+@pytest.mark.parametrize("name", ["d16b4", "d16b6", "d16b8", "d16b2", "d32b6"])
+def test_uniform_layout_hand_bytes(name):
+    case = _golden_layout()[name]
+    D, b = int(name[1:name.index("b")]), int(name[name.index("b") + 1:])
+    z = np.zeros((D, D), np.int32)
+    for item in case["set"]:
         i, j, val = (int(x) for x in item.split(","))
         z[i, j] = val
-    blk = core.pack_uniform(16, 4, z)
-    exp = np.full(128, 0x88, np.uint8)
-    for item in cases["b4"]["expect"]:
-        if item.startswith("default="):
-            continue
-        k, val = item.split("=")
-        exp[int(k)] = int(val, 16)
+    blk = core.pack_uniform(D, b, z)
+    items = case["expect"]
+    exp = np.full(D * D * b // 8, int(items[0].split("=")[1], 16), np.uint8)
+    k = 1
+    while k < len(items):
+        if items[k] == "pattern":
+            rng_s, pat = items[k + 1].split("=")
+            a_, b_ = (int(x) for x in rng_s.split(":"))
+            p = np.array([int(x, 16) for x in pat.split(",")], np.uint8)
+            exp[a_:b_] = np.tile(p, (b_ - a_) // p.size)
+            k += 2
+        else:
+            off, val = items[k].split("=")
+            exp[int(off)] = int(val, 16)
+            k += 1
     assert np.array_equal(blk, exp)
-    # b = 6 case, all zero codes
-    blk = core.pack_uniform(16, 6, np.zeros((16, 16), np.int32))
-    exp = np.zeros(192, np.uint8)
-    for item in cases["b6"]["expect"][1:]:
-        rng_s, pat = item.split("=")
-        a, b_ = (int(x) for x in rng_s.split(":"))
-        p = [int(x, 16) for x in pat.split(",")]
-        exp[a:b_] = np.tile(np.array(p, np.uint8), (b_ - a) // 2)
-    assert np.array_equal(blk, exp)
+    assert np.array_equal(core.unpack_uniform(D, b, blk), z)
 
 
 def test_rows_layout_lsb_first():
@@ -131,6 +133,63 @@ def test_pairwise_sum_order_and_accuracy():
         s = float(core.pairwise_sum(x))
         exact = math.fsum(float(v) for v in x)
         assert abs(s - exact) <= math.log2(n) * 2.0 ** -24 * exact * 1.0001
+
+
+def _golden_band_dot():
+    cases = []
+    with open(os.path.join(GOLDEN, "band_dot.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            name, D = parts[0], int(parts[1])
+            x = np.full(D, float(parts[2].split("=")[1]), np.float64)
+            y = np.full(D, float(parts[3].split("=")[1]), np.float64)
+            cur, expect = None, None
+            for tok in parts[4:]:
+                if tok in ("x", "y", "expect"):
+                    cur = tok
+                    continue
+                if cur == "expect":
+                    expect = float.fromhex(tok)
+                else:
+                    i, val = tok.split("=")
+                    (x if cur == "x" else y)[int(i)] = float.fromhex(val)
+            cases.append((name, x.astype(np.float32), y.astype(np.float32), np.float32(expect)))
+    return cases
+
+
+@pytest.mark.parametrize("case", _golden_band_dot(), ids=lambda c: c[0])
+def test_band_dot_hand_values(case):
+    _, x, y, expect = case
+    assert core.band_dot(x, y) == expect
+
+
+@pytest.mark.parametrize("D", [16, 32, 64, 128])
+def test_band_dot_exact_when_partial_sums_are(D):
+    # small integers: every product and partial sum is exact, so any order gives the exact sum
+    x = rng.integers(-50, 51, D).astype(np.float32)
+    y = rng.integers(-50, 51, D).astype(np.float32)
+    assert float(core.band_dot(x, y)) == float(np.dot(x.astype(np.int64), y.astype(np.int64)))
+    # a single non-zero row picks exactly that product, wherever it sits
+    for i in (0, 1, D // 2 - 1, D - 1):
+        e = np.zeros(D, np.float32)
+        e[i] = 3.0
+        assert core.band_dot(e, y) == np.float32(3.0 * y[i])
+
+
+@pytest.mark.parametrize("D", [16, 128])
+def test_band_dot_error_bound(D):
+    # |fl-sum - exact| <= gamma_n sum |x_i y_i|, n = RT/2 + 2 + 3 roundings on any path
+    for _ in range(200):
+        x = rng.standard_normal(D).astype(np.float32)
+        y = (rng.standard_normal(D) * 10.0 ** rng.integers(-3, 4)).astype(np.float32)
+        s = float(core.band_dot(x, y))
+        exact = math.fsum(float(a) * float(b) for a, b in zip(x, y))
+        n = D // 16 + 5
+        bound = n * 2.0 ** -24 / (1 - n * 2.0 ** -24) * math.fsum(abs(float(a) * float(b)) for a, b in zip(x, y))
+        assert abs(s - exact) <= bound
 
 
 # --------------------------------------------------------------------------
@@ -224,6 +283,35 @@ def test_step_from_codes_matches_fp64_update(kda):
     scale = np.abs(ref).max()
     assert np.max(np.abs(St - ref)) < 4e-6 * scale
     assert np.allclose(o, o_ref, rtol=2e-5, atol=2e-5 * scale)
+
+
+@pytest.mark.parametrize("kda", [False, True])
+def test_step_u_and_o_are_column_dot_products(kda):
+    # u = S'^T k and o = S_t^T q column by column (not S k or S q): each within the
+    # fp32 bound of the exact column dot product of the oracle's own S' and S_t
+    D = 128
+    rw = np.where(rng.uniform(size=D) < 0.1, 16, 6).astype(np.int32) if kda else np.full(D, 6, np.int32)
+    S = (rng.standard_normal((D, D)) * rng.uniform(0.1, 10, (D, 1)) * rng.uniform(0.1, 10, (1, D))).astype(np.float32)
+    z, h, r, c, _ = core.quantize(D, rw, np.ones(D, np.float32), np.ones(D, np.float32), S)
+    q, k, v, alpha, beta = _rand_inputs(D, kda)
+    St, o, u, w = core.step_from_codes(D, rw, z, h, r, c, q, k, v, alpha, beta)
+    Shat = core.reconstruct(D, rw, z, h, r, c)
+    Sp = np.where(rw[:, None] == 16, alpha[:, None] * Shat, 0).astype(np.float32)
+    for i in range(D):  # S'_ij = fl(fl(alpha_i r_i) c_j) z_ij for quantized rows
+        if rw[i] != 16:
+            a = np.float32(alpha[i] * r[i])
+            Sp[i] = (a * c).astype(np.float32) * z[i].astype(np.float32)
+    k64, q64 = k.astype(np.float64), q.astype(np.float64)
+    gam = 13 * 2.0 ** -24
+    u_ex = Sp.astype(np.float64).T @ k64
+    assert np.all(np.abs(u - u_ex) <= gam * (np.abs(Sp).astype(np.float64).T @ np.abs(k64)) + 1e-30)
+    w_ex = (beta * (v - u)).astype(np.float32)
+    assert np.array_equal(w, w_ex)
+    assert np.array_equal(St, np.float32(Sp + k[:, None].astype(np.float64) * w[None, :].astype(np.float64)))
+    o_ex = St.astype(np.float64).T @ q64
+    assert np.all(np.abs(o - o_ex) <= gam * (np.abs(St).astype(np.float64).T @ np.abs(q64)) + 1e-30)
+    # transposed operands would not meet the bound (the state is far from symmetric)
+    assert not np.all(np.abs(o - St.astype(np.float64) @ q64) <= 1e-3 * np.abs(o_ex).max())
 
 
 def test_error_recursion_and_output_error_fp64():
