@@ -43,7 +43,7 @@ PREFILL_METRIC = "chunked prefill tokens/s into the packed state pool"
 TF32_PER_BF16 = 1.1 / 2.25   # nominal dense TF32 / BF16 tensor throughput
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-KERNEL_SOURCES = ["stepq_step.cu", "stepq_dev.cuh"]
+KERNEL_SOURCES = ["stepq_head.cu", "stepq_pipe.cuh", "stepq_dev.cuh"]
 
 
 def parse():
