@@ -535,8 +535,11 @@ void sq_step_from_codes(int D, const int *widths, const int32_t *z, const uint16
 }
 
 /* ------------------------------------------------------------------------ */
-/* Plain FP32-state recurrence (the unquantized reference the pages compare  */
-/* against, "FP32-state").  Same update; u and o summed in fp64, rounded once.*/
+/* Plain FP32-state recurrence (the unquantized state the pages compare      */
+/* against, "FP32-state").  Same update and the same band-order sums as the  */
+/* packed step: S'_ij = fl(alpha_i S_ij), u_j = band(k, S'_.j),              */
+/* w_j = fl(beta fl(v_j - u_j)), S_ij = fma(k_i, w_j, S'_ij),                */
+/* o_j = band(q, S_.j).                                                      */
 /* ------------------------------------------------------------------------ */
 
 void sq_step_fp32(int D, float *S, const float *q, const float *k, const float *v,
@@ -546,19 +549,13 @@ void sq_step_fp32(int D, float *S, const float *q, const float *k, const float *
     for (int i = 0; i < D; i++)
         for (int j = 0; j < D; j++) S[i * D + j] = alpha[i] * S[i * D + j];
     for (int j = 0; j < D; j++) {
-        double acc = 0.0;
-        for (int i = 0; i < D; i++) acc += (double)k[i] * (double)S[i * D + j];
-        float u = (float)acc;
+        float u = sq_band_dot(D, k, 1, S + j, D);
         float d = v[j] - u;
         w[j] = beta * d;
     }
     for (int i = 0; i < D; i++)
         for (int j = 0; j < D; j++) S[i * D + j] = fmaf(k[i], w[j], S[i * D + j]);
-    for (int j = 0; j < D; j++) {
-        double acc = 0.0;
-        for (int i = 0; i < D; i++) acc += (double)q[i] * (double)S[i * D + j];
-        o_out[j] = (float)acc;
-    }
+    for (int j = 0; j < D; j++) o_out[j] = sq_band_dot(D, q, 1, S + j, D);
     free(w);
 }
 
