@@ -8,12 +8,17 @@ pivot heads, synthetic seeded inputs.  A step is one decode step of every
 readout -> refit r, c -> pack -> write back.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
-                    [--variant two_stream|fused] [--batch B] [--plan 6|4] [--sweep]
+                    [--variant two_stream|fused] [--batch B] [--plan 6|4] [--no-sweep]
                     [--workload gdn|kda] [--scale-bits 32|16] [--shard replicas|layers]
                     [--prefill T [--prefill-kernel mma_sync|tcgen05]]
 
 --prefill T times the chunked prefill of T-token prompt chunks into the
 packed pool instead (tokens/s through the whole pool, tensor roofline).
+
+The default single-GPU line also carries the spec sweep (batch
+1/16/128/256 of the nominal-6 pool, the nominal-4 pool and bfloat16 scales at
+batch 70, KDA rows at batch 128, the FP32-state step beside each) under
+"north_star_sweep".
 
 Prints one JSON line (rank 0).  N > 1: launched by torch.distributed.run, one
 independent pool per GPU (no collective on the data path), barrier + max of
@@ -62,7 +67,9 @@ def parse():
                     help="storage of the r and c scales in the plan (16: bfloat16)")
     ap.add_argument("--workload", default="gdn", choices=["gdn", "kda"],
                     help="gdn: 2,304-head pool; kda: 81,920 key rows (20 x 32 x 128)")
-    ap.add_argument("--sweep", action="store_true", help="also time batch 1/16/70/128/256")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the north-star sweep that the default single-GPU line carries (batch 1/16/128/256, "
+                         "nominal-4 plan, KDA rows at batch 128, 16-bit scales, the FP32-state kernel for each)")
     ap.add_argument("--prefill", type=int, default=0, metavar="T",
                     help="time chunked prefill of T-token prompt chunks into the packed pool (GDN) instead of "
                          "the decode step; batch defaults to 1")
@@ -408,6 +415,96 @@ def variant_is_full_launch(args) -> bool:
             and args.scale_bits == 32 and args.shard == "replicas")
 
 
+def measure_packed(torch, stepq, synth, wl, plan, n, device, steps=12, warmup=3):
+    """Fused packed step of a whole pool at batch n: CUDA-event time of `steps`
+    steps on the context's main stream."""
+    L, H, D = wl.n_layers, wl.n_heads, wl.d
+    ctx = stepq.Context(plan, n)
+    pool = torch.zeros(n * plan.slot_bytes, dtype=torch.uint8, device=device)
+    slots = torch.arange(n, dtype=torch.int32, device=device)
+    for l in range(L):
+        ctx.requant_pack(pool, slots, n, l, l + 1, synth.initial_states_torch(wl, wl.seed, n, l, device))
+    alpha = synth.gates(wl, wl.seed)
+    sets = [synth.step_inputs_torch(wl, wl.seed, n, t, alpha, device) for t in range(2)]
+    o = torch.zeros((n, L, H, D), dtype=torch.float32, device=device)
+    ctx.sync()
+    secs, stats, _ = time_steps(torch, ctx, "fused", pool, slots, n, L, sets, o, None, warmup, steps, 1)
+    k_ms, k_n = stats["fused"]
+    ctx.close()
+    del pool, sets, o
+    torch.cuda.empty_cache()
+    return secs / steps, (k_ms / k_n / 1e3) if k_n else None
+
+
+def measure_fp32(torch, stepq, synth, wl, plan, n, device, steps=6, warmup=2):
+    """The FP32-state step on the same pool shape at batch n (seconds per step)."""
+    L, H, D = wl.n_layers, wl.n_heads, wl.d
+    ctx = stepq.Context(plan, n)
+    S32 = torch.empty((n, L, H, D, D), dtype=torch.float32, device=device)
+    for l in range(L):
+        S32[:, l:l + 1] = synth.initial_states_torch(wl, wl.seed, n, l, device)
+    slots = torch.arange(n, dtype=torch.int32, device=device)
+    alpha = synth.gates(wl, wl.seed)
+    sets = [synth.step_inputs_torch(wl, wl.seed, n, t, alpha, device) for t in range(2)]
+    o = torch.zeros((n, L, H, D), dtype=torch.float32, device=device)
+    for i in range(warmup):
+        x = sets[i % 2]
+        ctx.fp32_decode_step(S32, slots, n, 0, L, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(ctx.main)
+    for i in range(steps):
+        x = sets[i % 2]
+        ctx.fp32_decode_step(S32, slots, n, 0, L, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o)
+    e1.record(ctx.main)
+    torch.cuda.synchronize()
+    ctx.close()
+    del S32, sets, o
+    torch.cuda.empty_cache()
+    return e0.elapsed_time(e1) / 1e3 / steps
+
+
+def north_star_sweep(torch, stepq, synth, device, plan6, peak):
+    """The configurations the single-GPU line reports beside the headline: the
+    nominal-6 pool at batch 1/16/128/256, the nominal-4 pool over {2,4,6,8} and
+    16-bit scales at batch 70, KDA per-key-row units at batch 128, each with the
+    FP32-state step on the same pool shape.  Per entry: head-steps/s, tokens/s
+    (state updates of a request across the whole pool), algorithmic GB/s of the
+    single-pass step and its fraction of the measured peak."""
+    out = []
+
+    def entry(name, wl, plan, n, fp32=True):
+        t, t_k = measure_packed(torch, stepq, synth, wl, plan, n, device)
+        L, H, D = wl.n_layers, wl.n_heads, wl.d
+        b = step_bytes(plan, n)
+        e = {"config": name, "batch": n, "ms_per_step": t * 1e3, "head_steps_per_s": n * L * H / t,
+             "tokens_per_s": n / t, "gbs": b / t / 1e9, "frac": b / t / 1e9 / peak,
+             "kernel_ms": t_k * 1e3 if t_k else None, "bits_per_value": plan.info.bits_per_value,
+             "bits_per_value_s16": plan.info.bits_per_value_s16}
+        if n == 1:
+            e["l2"] = "the whole pool fits in the 126 MB L2 and stays there between steps"
+        if fp32:
+            t32 = measure_fp32(torch, stepq, synth, wl, plan, n, device)
+            b32 = n * L * H * (2 * 4 * D * D + 3 * 4 * D + gate_bytes(plan) + 4 * D)
+            e["fp32_state"] = {"ms_per_step": t32 * 1e3, "head_steps_per_s": n * L * H / t32,
+                               "gbs": b32 / t32 / 1e9, "frac": b32 / t32 / 1e9 / peak,
+                               "packed_speedup": t32 / t}
+        out.append(e)
+
+    wl6 = synth.workloads()["qwen_pool6"]
+    for n in (1, 16, 128, 256):
+        entry("GDN pool, nominal 6 over {4,6,8}, 32 pivots", wl6, plan6, n)
+    wl4 = synth.workloads()["qwen_pool4"]
+    plan4, _ = product_plan(stepq, synth, wl4, device)
+    entry("GDN pool, nominal 4 over {2,4,6,8}, 32 pivots", wl4, plan4, 70, fp32=False)
+    plan16, _ = product_plan(stepq, synth, wl6, device, scale_bits=16)
+    entry("GDN pool, nominal 6, bfloat16 r and c", wl6, plan16, 70, fp32=False)
+    wlk = synth.workloads()["kda_rows"]
+    plank, _ = product_plan(stepq, synth, wlk, device)
+    entry("KDA per-key-row units, 81,920 rows, nominal 6 over {4,6,8}, 512 pivot rows", wlk, plank, 128)
+    return out
+
+
 def run_product(args):
     import torch
     from quantized_recurrent_state_b200 import build as qbuild
@@ -549,26 +646,9 @@ def run_product(args):
                "overlap": "uploads (two streams) and downloads (one) double-buffered, overlapping the steps"}
 
     sweep = None
-    if args.sweep and rank == 0:
-        sweep = []
-        for bs in (1, 16, 70, 128, 256):
-            c2 = stepq.Context(plan, bs)
-            p2 = torch.zeros(bs * plan.slot_bytes, dtype=torch.uint8, device=device)
-            s2 = torch.arange(bs, dtype=torch.int32, device=device)
-            for l in range(L):
-                c2.requant_pack(p2, s2, bs, l, l + 1, synth.initial_states_torch(wl, wl.seed, bs, lb + l, device))
-            st2 = [{k: v[:, lb:le].contiguous() for k, v in synth.step_inputs_torch(wl, wl.seed, bs, t, alpha,
-                                                                                     device).items()}
-                   for t in range(2)]
-            o2 = torch.zeros((bs, L, H, D), dtype=torch.float32, device=device)
-            w2 = torch.empty(c2.workspace_bytes(bs, L) // 4, dtype=torch.float32, device=device)
-            sec2, _, _ = time_steps(torch, c2, args.variant, p2, s2, bs, L, st2, o2, w2, 3, 16, 1)
-            sweep.append({"batch": bs, "head_steps_per_s": bs * L * H * 16 / sec2,
-                          "tokens_per_s": bs * 16 / sec2, "gbs": step_bytes(plan, bs) * 16 / sec2 / 1e9,
-                          "ms_per_step": sec2 / 16 * 1e3})
-            c2.close()
-            del p2, st2, o2, w2
-            torch.cuda.empty_cache()
+    if (rank == 0 and ws == 1 and not args.no_sweep and args.workload == "gdn" and args.plan == 6
+            and args.scale_bits == 32 and args.variant == "fused" and args.batch == 70):
+        sweep = north_star_sweep(torch, stepq, synth, device, plan, peak)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -621,7 +701,7 @@ def run_product(args):
             **extra,
         }
         if sweep:
-            out["sweep"] = sweep
+            out["north_star_sweep"] = sweep
         print(json.dumps(out), flush=True)
     ctx.close()
     if ws > 1:

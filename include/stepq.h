@@ -23,23 +23,33 @@
  *               o_t = S_t^T q_t  (GDN: alpha scalar per head; KDA: per key row)
  *   decode      a_i = fl(alpha_i r_i);  S'_ij = fl(fl(a_i c_j) z_ij)
  *               (16-bit rows: S'_ij = fl(alpha_i h_ij))
- *               u_j = fl32(sum_i k_i a_i c_j z_ij)   exact sum, rounded once
+ *               u_j = band_i(k_i S'_ij)
  *               w_j = fl(beta fl(v_j - u_j));  S_t,ij = fma(k_i, w_j, S'_ij)
- *               o_j = fl32(sum_i q_i (a_i c_j z_ij + k_i w_j))  exact, rounded once
+ *               o_j = band_i(q_i S_t,ij)
  *   requantize  r_i = fl(max(pairwise_j |S_ij| / D, 1e-12) rho_i)
- *               y = fl(S fl(1/r));  c0_j = max_i fl(|y_ij| / qmax_i) (0 -> 1)
+ *               y = fl(S fl(1/r));  c0_j = max_i fl(|y_ij| fl(1/qmax_i)) (0 -> 1)
  *               z0 = rint(y * fl(1/c0))   (exact product, ties to even)
- *               c_j = fl(pairwise_i fl(b_i fl(z0 y)) / pairwise_i fl(b_i fl(z0 z0))),
- *                     b_i = fl(wbar_i fl(r_i r_i)); a zero denominator keeps c0
+ *               t_ij = fl(b_i z0_ij), b_i = fl(wbar_i fl(r_i r_i))
+ *               c_j = fl(band_i(t_ij y_ij) / band_i(t_ij z0_ij)); a zero
+ *                     denominator keeps c0
  *               z = clamp(rint(y * fl(1/c)), -qmax, qmax); 16-bit rows: fp16 RNE
  *   qmax(b) = 2^(b-1) - 1.  pairwise = fp32 sum in balanced binary-tree order.
+ *   band_i(x_i y_i) = fp32 sum over the D rows in band order: 8 bands of D/8
+ *     consecutive rows; in a band the even rows and the odd rows each form a
+ *     chain acc = fma(x_i, y_i, acc) from +0, the band's value is the sum of
+ *     the two chains, and the 8 band values are added in a balanced binary
+ *     tree in band order.
  *
  * Packed format (decided offline, 方法-4 "fixed packed layout").  Codes are
  * stored offset-binary, u = z + 2^(b-1).
- *   per-head units (mode 0), width b in {2,4,6,8}: thread-major layout with
- *     RT = D/8, NT = 2D: element (i,j) -> thread t = (i/RT)(D/4) + j/4,
- *     position p = (i%RT)*4 + j%4, stream bits [p b, p b + b) LSB first;
- *     stream byte B of thread t at block byte ((B/RT) NT + t) RT + B%RT.
+ *   per-head units (mode 0), width b in {2,4,6,8}: tile-major layout with
+ *     RT = D/8, NT = 2D tiles: element (i,j) -> tile t = (j/4)*8 + i/RT, tile
+ *     code (r, c) = (i%RT, j%4); tile stream bits [(4r + c) b, +b), LSB first,
+ *     except b = 6 with RT >= 4, where the rows of a tile go in groups of four
+ *     over three 32-bit words (rows 0, 1, 3 of a group in bits [0, 24) of
+ *     words 0, 1, 2 as 24-bit row values sum_c u_c 2^(6c); the 24-bit value of
+ *     row 2 byte by byte in bits [24, 32) of the same words); stream byte B
+ *     of tile t at block byte ((B/RT) NT + t) RT + B%RT.
  *   per-row units (mode 1): rows in order, row i = D*b_i/8 bytes, code j at
  *     row bits [b_i j, b_i j + b_i); a 16-bit row holds binary16 values.
  *   record = codes | r[D] | c[D], zero-padded to 128 bytes, r and c fp32, or
@@ -183,10 +193,13 @@ int stepq_plan_slice(const stepq_plan *plan, int lb, int le, stepq_plan **out);
 
 /* ---- context ------------------------------------------------------------ */
 
-/* Bind a plan to the current CUDA device.  main/side are cudaStream_t (NULL
- * for the legacy default stream is rejected: pass real streams).  n_slots is
- * the capacity of every pool used with this context.  chunk_layers groups
- * layers per launch pair in stepq_decode_step (<= 0: 4). */
+/* Bind a plan to the current CUDA device (paper digest page, 方法-4: the
+ * decode runs on one stream while scale fitting and packing run on a separate
+ * one; the context holds those two streams, the device copy of the plan's
+ * tables and the per-layer events that order them).  main/side are
+ * cudaStream_t (NULL for the legacy default stream is rejected: pass real
+ * streams).  n_slots is the capacity of every pool used with this context.
+ * chunk_layers groups layers per launch pair in stepq_decode_step (<= 0: 4). */
 int stepq_ctx_create(const stepq_plan *plan, void *main_stream, void *side_stream, int n_slots,
                      int chunk_layers, stepq_ctx **out);
 void stepq_ctx_free(stepq_ctx *ctx);
@@ -290,13 +303,19 @@ int stepq_decode_step_fused(stepq_ctx *ctx, void *pool, const int32_t *slots, in
  *     them, e.g. one layer range at a time).
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is looked up again when the
+ *     device's current context is no longer the one it was looked up in
+ *     (after a cudaDeviceReset, or a context made current through the driver
+ *     API); a device reset also invalidates every stepq_ctx of that device,
+ *     so create new contexts after one.
  *   - All calls on a device share the array and it keeps the last call's
  *     contents (nothing in it needs to start at zero: every value is written
  *     before it is read).  Before launching, the call makes `main` wait for
- *     all earlier side-stream work of this context; calls from different
- *     contexts, threads or processes' streams that overlap on the GPU race
- *     on the array.
+ *     all earlier side-stream (fit-and-pack) work of this context, on every
+ *     layer and not only on [lb, le): unlike stepq_decode_step, a call does
+ *     not overlap the previous call's fit-and-pack of other layers.  Calls
+ *     from different contexts, threads or processes' streams that overlap on
+ *     the GPU race on the array.
  * Results are bit-identical to stepq_decode_step. */
 #define STEPQ_NOALLOC_SCRATCH_BYTES (8u << 20)
 int stepq_decode_step_noalloc(stepq_ctx *ctx, void *pool, const int32_t *slots, int n_req, int lb, int le,
@@ -305,16 +324,22 @@ int stepq_decode_step_noalloc(stepq_ctx *ctx, void *pool, const int32_t *slots, 
 
 /* Wait for all work of the context (both streams) with a host-side timeout
  * (<= 0: wait without limit), then return the device error word:
- * STEPQ_OK, STEPQ_ETIMEDOUT, STEPQ_EDEVICE (the word is cleared) or ECUDA. */
+ * STEPQ_OK, STEPQ_ETIMEDOUT, STEPQ_EDEVICE (the word is cleared) or ECUDA.
+ * Paper digest page, 方法-4: the refitted, packed records are written back
+ * asynchronously and must be complete before the next read; this is the
+ * point where the host knows they are. */
 int stepq_sync(stepq_ctx *ctx, int timeout_ms);
 
-/* Reconstruct X_hat = r c z (16-bit rows: their value) into S. */
+/* Reconstruct X_hat_ij = fl(fl(r_i c_j) z_ij) (16-bit rows: their value) into S
+ * (paper digest page, 方法-3 Key-Row-Aware Dual-Axis Fitting: X_hat = r_i c_j z_ij). */
 int stepq_unpack(stepq_ctx *ctx, const void *pool, const int32_t *slots, int n_req, int lb, int le,
                  float *S);
 
-/* FP32-state reference step (the unquantized baseline) on an fp32 pool of
- * [n_slots][n_layers][n_heads][D][D]: S'_ij = fl(alpha_i S_ij), u and o
- * summed exactly and rounded once, S_ij = fma(k_i, w_j, S'_ij).  On main. */
+/* FP32-state reference step on an fp32 pool of [n_slots][n_layers][n_heads][D][D]:
+ * the unquantized recurrence the pages set the packed state against (paper
+ * digest page, 背景与动机 and 实验: the FP32 state pool), S'_ij =
+ * fl(alpha_i S_ij), u_j = band_i(k_i S'_ij), w_j = fl(beta fl(v_j - u_j)),
+ * S_ij = fma(k_i, w_j, S'_ij), o_j = band_i(q_i S_ij).  On main. */
 int stepq_fp32_decode_step(stepq_ctx *ctx, float *S_pool, const int32_t *slots, int n_req, int lb,
                            int le, const float *q, const float *k, const float *v,
                            const float *alpha, const float *beta, float *o);

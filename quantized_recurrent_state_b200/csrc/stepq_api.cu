@@ -30,7 +30,7 @@
 namespace stepq {
 cudaError_t launch_step(int kind, int D, const Args &a, int n_sms, cudaStream_t st, int *grid);
 cudaError_t launch_pack(int D, const Args &a, bool unpack, cudaStream_t st);
-cudaError_t launch_fp32_step(int D, const Args &a, float *S_pool, int n_layers_total, cudaStream_t st);
+cudaError_t launch_fp32_step(int D, const Args &a, float *S_pool, int n_layers_total, int n_sms, cudaStream_t st);
 cudaError_t launch_copy(void *dst, const void *src, size_t bytes, int n_sms, cudaStream_t st);
 cudaError_t launch_calib_acc(int D, const Args &a, double *om, double *ls, cudaStream_t st);
 cudaError_t launch_calib_dist(int D, const Args &a, const int *bits, int n_bits, double *acc, cudaStream_t st);
@@ -618,6 +618,7 @@ struct stepq_ctx {
     bool timing = false;
     uint32_t wait_polls = 1u << 22, phantom_tx = 0;
     int prefill_kernel = STEPQ_PREFILL_MMA_SYNC;
+    bool poisoned = false;  // a tensor-memory drain failure was reported: refuse further work
     struct Timed { int kind; cudaEvent_t a, b; };
     std::vector<Timed> timed;
     std::vector<cudaEvent_t> ev_pool;
@@ -633,6 +634,9 @@ int check_ptr(const void *p, size_t align, const char *name) {
 
 int check_range(const stepq_ctx *c, int n_req, int lb, int le) {
     if (!c) return fail(STEPQ_EINVAL, "null context");
+    if (c->poisoned)
+        return fail(STEPQ_EDEVICE, "context unusable: a tensor-memory kernel freed columns a product may still have "
+                                   "been writing (reported by an earlier stepq_sync); create a new context");
     if (n_req < 0) return fail(STEPQ_EINVAL, "n_req %d < 0", n_req);
     if (lb < 0 || le > c->plan->L || lb >= le) return fail(STEPQ_EINVAL, "layer range [%d, %d) outside [0, %d)", lb, le, c->plan->L);
     return STEPQ_OK;
@@ -965,7 +969,7 @@ extern "C" int stepq_fp32_decode_step(stepq_ctx *c, float *S_pool, const int32_t
     stepq::Args a = base_args(c, nullptr, slots, n_req, lb, le);
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.o = o;
     LaunchTimer lt(c, 3, c->main);
-    const cudaError_t e = stepq::launch_fp32_step(c->plan->D, a, S_pool, c->plan->L, c->main);
+    const cudaError_t e = stepq::launch_fp32_step(c->plan->D, a, S_pool, c->plan->L, c->n_sms, c->main);
     if (e != cudaSuccess) return cuda_fail(e, "fp32 step launch");
     lt.done();
     return STEPQ_OK;
@@ -1010,9 +1014,11 @@ extern "C" int stepq_sync(stepq_ctx *c, int timeout_ms) {
     if (e != cudaSuccess) return cuda_fail(e, "sync: read error word");
     if (word) {
         cudaMemset(c->err, 0, sizeof(int));
-        return fail(STEPQ_EDEVICE, "device error word 0x%x (%s%s%s%s)", word,
+        if (word & stepq::kErrTmemDrain) c->poisoned = true;
+        return fail(STEPQ_EDEVICE, "device error word 0x%x (%s%s%s%s%s)", word,
                     (word & stepq::kErrBadSlot) ? "slot out of range " : "", (word & stepq::kErrWait) ? "copy wait gave up " : "",
-                    (word & stepq::kErrArgs) ? "bad width " : "", (word & stepq::kErrGateRange) ? "prefill gate out of range " : "");
+                    (word & stepq::kErrArgs) ? "bad width " : "", (word & stepq::kErrGateRange) ? "prefill gate out of range " : "",
+                    (word & stepq::kErrTmemDrain) ? "tensor memory freed with a product in flight (context now unusable) " : "");
     }
     return STEPQ_OK;
 }
@@ -1197,20 +1203,47 @@ static __device__ __align__(256) float g_noalloc_w[STEPQ_NOALLOC_SCRATCH_BYTES /
 namespace {
 std::mutex g_noalloc_mu;
 constexpr int kMaxDevices = 128;
-float *g_noalloc_addr[kMaxDevices] = {};
+struct NoallocEntry {
+    void *ctx = nullptr;  // the CUDA context the address belongs to
+    float *addr = nullptr;
+};
+NoallocEntry g_noalloc[kMaxDevices];
 
-// Device address of g_noalloc_w on the current device `dev` (looked up once
-// per device; in host code the symbol itself is only a host-side stand-in).
+// The driver's current context, read through the runtime's driver entry
+// point (no link against the driver library).
+void *current_cu_context() {
+    using GetCurrent = int (*)(void **);
+    static GetCurrent fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<GetCurrent>(nullptr);
+        return reinterpret_cast<GetCurrent>(p);
+    }();
+    void *ctx = nullptr;
+    if (fn) fn(&ctx);
+    return ctx;
+}
+
+// Device address of g_noalloc_w on the current device `dev` and its current
+// context.  In host code the symbol is only a host-side stand-in; the address
+// is looked up on the first call per device and again whenever the current
+// context of that device is not the one it was looked up in (a device reset
+// or a context made current through the driver API).
 int noalloc_scratch(int dev, float **out) {
     if (dev < 0 || dev >= kMaxDevices) return fail(STEPQ_EINVAL, "decode_step_noalloc: device ordinal %d", dev);
+    void *ctx = current_cu_context();
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
+    NoallocEntry &e = g_noalloc[dev];
+    if (!e.addr || e.ctx != ctx) {
         void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_w);
-        if (e != cudaSuccess) return cuda_fail(e, "decode_step_noalloc: cudaGetSymbolAddress");
-        g_noalloc_addr[dev] = static_cast<float *>(p);
+        const cudaError_t err = cudaGetSymbolAddress(&p, g_noalloc_w);
+        if (err != cudaSuccess) return cuda_fail(err, "decode_step_noalloc: cudaGetSymbolAddress");
+        e.addr = static_cast<float *>(p);
+        e.ctx = ctx;
     }
-    *out = g_noalloc_addr[dev];
+    *out = e.addr;
     return STEPQ_OK;
 }
 }  // namespace

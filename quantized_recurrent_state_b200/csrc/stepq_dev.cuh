@@ -20,6 +20,10 @@ constexpr int kQuantAbsmax = 1;    // plan quantizer: per-row absmax, c = 1
 constexpr int kErrBadSlot = 1;
 constexpr int kErrWait = 2;
 constexpr int kErrArgs = 4;
+// A tensor-memory kernel freed its columns although a product it had issued
+// might still have been writing them (a bounded wait gave up): later results
+// of that memory cannot be trusted; the context refuses further work.
+constexpr int kErrTmemDrain = 16;
 
 // Device copy of the plan tables.
 struct Tables {

@@ -275,6 +275,44 @@ __device__ __forceinline__ float2 scale2_at(const uint8_t *base, int i, int s16)
     return *reinterpret_cast<const float2 *>(base + 4 * i);
 }
 
+// Row pairs (x_i, x_{i+1}), i = i0 + 2k, of NP pairs from a 16-byte aligned
+// row array (16-byte loads, two pairs each).
+template <int NP>
+__device__ __forceinline__ void load_pairs(const float *p, float2 (&out)[NP]) {
+    if constexpr (NP % 2 == 0) {
+#pragma unroll
+        for (int k = 0; k < NP; k += 2) {
+            const float4 v = *reinterpret_cast<const float4 *>(p + 2 * k);
+            out[k] = make_float2(v.x, v.y);
+            out[k + 1] = make_float2(v.z, v.w);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < NP; ++k) out[k] = *reinterpret_cast<const float2 *>(p + 2 * k);
+    }
+}
+
+// The same from a scale array (fp32 or bfloat16) at row i0.
+template <int NP>
+__device__ __forceinline__ void load_scale_pairs(const uint8_t *base, int i0, int s16, float2 (&out)[NP]) {
+    if (!s16) {
+        load_pairs<NP>(reinterpret_cast<const float *>(base) + i0, out);
+        return;
+    }
+    if constexpr (NP % 4 == 0) {
+#pragma unroll
+        for (int k = 0; k < NP; k += 4) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(base + 2 * (i0 + 2 * k));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) out[k + t] = make_float2(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xffff0000u));
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < NP; ++k) out[k] = scale2_at(base, i0 + 2 * k, 1);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Requantization of the fp32 tile S (registers) into codes, r and c.
 // ---------------------------------------------------------------------------
@@ -364,9 +402,11 @@ __device__ __forceinline__ void fit_codes(float2 (&S)[D / 16][4], ScratchH<D> &s
     const int g = tid & 7, lane = tid & 31, i0 = g * RT, j0 = 4 * (tid >> 3);
     // y and the column maxima of |y|
     float m[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float2 pr[NP];
+    load_pairs<NP>(&sc.rinv[i0], pr);
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
-        const float2 ir = *reinterpret_cast<const float2 *>(&sc.rinv[i0 + 2 * k]);
+        const float2 ir = pr[k];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             S[k][c] = mul2(S[k][c], ir);
@@ -387,9 +427,10 @@ __device__ __forceinline__ void fit_codes(float2 (&S)[D / 16][4], ScratchH<D> &s
     float2 na[4], da[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) na[c] = da[c] = make_float2(0.0f, 0.0f);
+    load_pairs<NP>(&sc.bw[i0], pr);
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
-        const float2 b2 = *reinterpret_cast<const float2 *>(&sc.bw[i0 + 2 * k]);
+        const float2 b2 = pr[k];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const float2 z0 = add2(fma2(S[k][c], ic0d[c], mg), nmg);
@@ -439,9 +480,11 @@ __device__ __forceinline__ void absmax_codes(const float2 (&S)[D / 16][4], const
     const int i0 = (tid & 7) * RT;
     const float2 mg2 = make_float2(kMagic + (float)OFF, kMagic + (float)OFF);
     uint32_t ha = 0u, hb = 0u;
+    float2 pr[NP];
+    load_pairs<NP>(&sc.rinv[i0], pr);
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
-        const float2 ir = *reinterpret_cast<const float2 *>(&sc.rinv[i0 + 2 * k]);
+        const float2 ir = pr[k];
         float2 T[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) T[c] = fma2(S[k][c], ir, mg2);
@@ -481,13 +524,15 @@ __device__ bool item_head(const Args &a, const uint8_t *stage, uint8_t *rec_g, i
     float2 acc[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[c] = make_float2(0.0f, 0.0f);
+    float2 rp[NP], kp[NP];
+    load_scale_pairs<NP>(st_r, i0, S16, rp);
+    load_pairs<NP>(ks + i0, kp);
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
-        const int i = i0 + 2 * k;
-        const float2 a2 = mul2(scale2_at(st_r, i, S16), al2);
+        const float2 a2 = mul2(rp[k], al2);
         float2 z[4];
         unpack_pair<D, B>(W, k, z);
-        const float2 k2 = *reinterpret_cast<const float2 *>(ks + i);
+        const float2 k2 = kp[k];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             S[k][c] = mul2(mul2(a2, cd[c]), z[c]);
@@ -516,18 +561,19 @@ __device__ bool item_head(const Args &a, const uint8_t *stage, uint8_t *rec_g, i
     // S = fma(k, w, S'); o chains
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[c] = make_float2(0.0f, 0.0f);
+    load_pairs<NP>(ks + i0, kp);
+    if (KIND != kFitPack) load_pairs<NP>(qs + i0, rp);
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
-        const int i = i0 + 2 * k;
-        const float2 k2 = *reinterpret_cast<const float2 *>(ks + i);
-        float2 q2;
-        if (KIND != kFitPack) q2 = *reinterpret_cast<const float2 *>(qs + i);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            S[k][c] = fma2(k2, wd[c], S[k][c]);
-            if (KIND != kFitPack) acc[c] = fma2(q2, S[k][c], acc[c]);
+            S[k][c] = fma2(kp[k], wd[c], S[k][c]);
+            if (KIND != kFitPack) acc[c] = fma2(rp[k], S[k][c], acc[c]);
         }
     }
+    // the row partials go out first: the readout's shuffles then overlap the
+    // stores and the wait at the block barrier
+    if (KIND != kDecode) row_partials<D, QUANT>(S, sc, g, cb);
     float o_mine = 0.0f;
     if (KIND != kFitPack)
         o_mine = band_sum4(acc[0].x + acc[0].y, acc[1].x + acc[1].y, acc[2].x + acc[2].y, acc[3].x + acc[3].y, g);
@@ -540,7 +586,6 @@ __device__ bool item_head(const Args &a, const uint8_t *stage, uint8_t *rec_g, i
         }
         return false;
     }
-    row_partials<D, QUANT>(S, sc, g, cb);
     if (__syncthreads_or(!ok)) return true;
     if (KIND == kFused && (g & 4) == 0) a.o[(size_t)row * D + j0 + cs] = o_mine;
     uint8_t *rec_r = rec_g + codes_bytes;

@@ -443,8 +443,12 @@ __global__ void __launch_bounds__(NT, 1) k_prefill_tc(PrefillArgs a) {
         }
     } else {
         if (tid == 0) atomicOr(a.err, kErrWait);
-        // let the products already issued finish (bounded) before the columns are freed
-        for (int b = 0; b < 3; ++b) tc::mbar_wait(&sm.bar[b], ci & 1, kPolls);
+        // let the products already issued finish (bounded) before the columns are freed;
+        // if one of these waits gives up too, the columns are freed with a product possibly
+        // still writing them, which the error word records as its own (fatal) condition
+        bool drained = true;
+        for (int b = 0; b < 3; ++b) drained = tc::mbar_wait(&sm.bar[b], ci & 1, kPolls) && drained;
+        if (!drained && tid == 0) atomicOr(a.err, kErrTmemDrain);
     }
     tc::fence_before();
     __syncthreads();

@@ -12,7 +12,7 @@ import pytest
 
 from oracle import core, model
 from quantized_recurrent_state_b200 import synth
-from tests._workloads import compare_records, oracle_plan, uniform_plan
+from tests._workloads import compare_records, oracle_plan, reconstruction_gap, uniform_plan
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -102,10 +102,11 @@ def _lockstep(stepq, name, n_req, steps, check, n_layers=None, n_pivots=None, fu
                 if heads is not None and h not in heads:
                     continue
                 ties[(l, h)] = pv.quantize_into(ora, l, h, S0[n, l, h])
-        c, e, b, _ = compare_records(pv, g, ora, ties)
+        c, e, b, sb = compare_records(pv, g, ora, ties)
         tot_codes += c; tot_exc += e; tot_bad += b
+        assert sb == 0, ("scales", n, sb)
     assert tot_bad == 0
-    worst_o = 0.0
+    worst_o = worst_s = 0.0
     for t in range(steps):
         prev = {n: run.slot_bytes_host(n) for n in check}
         inp, o = run.step(t, fused=fused)
@@ -123,10 +124,16 @@ def _lockstep(stepq, name, n_req, steps, check, n_layers=None, n_pivots=None, fu
                     ok = _close(o[n, l, h], o_ref)
                     assert ok.all(), (t, n, l, h, np.max(np.abs(o[n, l, h] - o_ref)))
                     worst_o = max(worst_o, float(np.max(np.abs(o[n, l, h] - o_ref) / (ATOL + RTOL * np.abs(o_ref)))))
-            c, e, b, _ = compare_records(pv, g, ora, ties)
+            c, e, b, sb = compare_records(pv, g, ora, ties)
             tot_codes += c; tot_exc += e; tot_bad += b
             assert b == 0, (t, n, b)
-    print(f"{name}: codes {tot_codes}, tie-excused {tot_exc}, bad {tot_bad}, worst o/tol {worst_o:.3g}")
+            assert sb == 0, ("scales", t, n, sb)
+            if t % 8 == 0 or t == steps - 1:  # reconstructed states (spec tolerance)
+                gap = reconstruction_gap(pv, g, ora, list(ties), ties)
+                assert gap <= 1.0, (t, n, gap)
+                worst_s = max(worst_s, gap)
+    print(f"{name}: codes {tot_codes}, tie-excused {tot_exc}, bad {tot_bad}, worst o/tol {worst_o:.3g}, "
+          f"worst S_hat/tol {worst_s:.3g}")
     assert tot_exc <= 1e-5 * tot_codes
     return run
 
@@ -153,10 +160,12 @@ def test_tiny_gdn_lockstep_32_steps(stepq, fused):
     _lockstep(stepq, "tiny_gdn", 1, 32, check=[0], fused=fused)
 
 
-def test_qwen_layer_lockstep_256_steps(stepq):
+@pytest.mark.parametrize("fused", [True, False])
+def test_qwen_layer_lockstep_256_steps(stepq, fused):
     # 64 requests x 48 heads, d = 128, nominal 6 bits over {4,6,8}, 1 pivot head;
-    # the oracle follows two of the requests (96 heads) at every step.
-    _lockstep(stepq, "qwen_layer", 64, 256, check=[0, 37])
+    # the oracle follows two of the requests (96 heads) at every step; both the
+    # fused step the benchmark times and the two-stream step.
+    _lockstep(stepq, "qwen_layer", 64, 256, check=[0, 37], fused=fused)
 
 
 @pytest.mark.parametrize("name", ["qwen_pool6", "qwen_pool4"])
@@ -253,32 +262,35 @@ def test_bad_slot_reports_device_error(stepq):
     assert ei.value.code == stepq.EINVAL
 
 
-def test_fp32_reference_kernel(stepq):
-    plan, data, wl, _ = oracle_plan("qwen_layer")
+@pytest.mark.parametrize("name,n,n_layers", [("qwen_layer", 3, None), ("kda_rows", 2, 1), ("tiny_gdn", 2, None),
+                                             ("gdn_d64", 3, None)])
+def test_fp32_reference_kernel(stepq, name, n, n_layers):
+    # the FP32-state step against the oracle's fp32 recurrence, bit for bit (same
+    # definition: band-order sums, one fma per element); per-head and per-row gates,
+    # d = 128, 64 and 16; 12 steps, every head
+    plan, data, wl, _ = oracle_plan(name, n_layers)
     P = stepq.Plan.from_bytes(data)
-    n = 3
     ctx = stepq.Context(P, n)
+    L = wl.n_layers
     S0 = synth.initial_states(wl, wl.seed, n)
     Sd = torch.from_numpy(S0).cuda().contiguous()
     slots = torch.arange(n, dtype=torch.int32, device="cuda")
     alpha = synth.gates(wl, wl.seed)
     S_ref = S0.copy()
-    for t in range(16):
+    for t in range(12):
         inp = synth.step_inputs(wl, wl.seed, n, t, alpha=alpha)
         d = _inputs_to_dev(inp)
         o = torch.zeros_like(d["q"])
-        ctx.fp32_decode_step(Sd, slots, n, 0, 1, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)
+        ctx.fp32_decode_step(Sd, slots, n, 0, L, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)
         ctx.sync()
         og = o.cpu().numpy()
         for r in range(n):
-            for h in range(0, wl.n_heads, 5):
-                o_ref = core.step_fp32(S_ref[r, 0, h], inp["q"][r, 0, h], inp["k"][r, 0, h], inp["v"][r, 0, h],
-                                       inp["alpha"][r, 0, h], inp["beta"][r, 0, h])
-                assert _close(og[r, 0, h], o_ref).all()
-    Sg = Sd.cpu().numpy()
-    for r in range(n):
-        for h in range(0, wl.n_heads, 5):
-            assert _close(Sg[r, 0, h], S_ref[r, 0, h]).all()
+            for l in range(L):
+                for h in range(wl.n_heads):
+                    o_ref = core.step_fp32(S_ref[r, l, h], inp["q"][r, l, h], inp["k"][r, l, h], inp["v"][r, l, h],
+                                           inp["alpha"][r, l, h], inp["beta"][r, l, h])
+                    assert np.array_equal(og[r, l, h], o_ref), (t, r, l, h)
+    assert np.array_equal(Sd.cpu().numpy(), S_ref)
 
 
 def test_calibration_kernels_match_oracle(stepq):
@@ -347,6 +359,7 @@ def _full_pool_sampled(stepq, name, n, steps, n_samples, seed, reverse_slots=Fal
                for _ in range(n_samples)]
     samples += [(n - 1, int(u) // wl.n_heads, int(u) % wl.n_heads) for u in piv_heads[:3]]
     slot_of = slots.cpu().numpy()
+    n_codes = n_exc = 0
     for (r, l, h) in samples:
         slot = int(slot_of[r])
         off, nb = P.record(l, h)
@@ -354,12 +367,67 @@ def _full_pool_sampled(stepq, name, n, steps, n_samples, seed, reverse_slots=Fal
         rec_new = pool[slot * sb + off:slot * sb + off + nb].cpu().numpy()
         x = {k: inp[k][r, l, h].cpu().numpy() for k in ("q", "k", "v", "alpha", "beta")}
         new_rec, o_ref, tie, S, w = model.step_head(pv.mode, pv.D, pv.rw(l, h), pv.rho[l, h], pv.wbar[l, h],
-                                                    rec_prev, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+                                                    rec_prev, x["q"], x["k"], x["v"], x["alpha"], x["beta"],
+                                                    pv.quantizer, pv.scale_bits)
         assert _close(o[r, l, h].cpu().numpy(), o_ref).all(), (r, l, h)
+        n_codes += pv.D * pv.D
         if not np.array_equal(rec_new, new_rec):
-            zg, hg, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), rec_new)
-            zo, ho, _, _ = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), new_rec)
-            assert not (((zg != zo) | (hg != ho)) & (tie == 0)).any(), (r, l, h)
+            zg, hg, rg, cg = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), rec_new, pv.scale_bits)
+            zo, ho, ro, co = model.unpack_head(pv.mode, pv.D, pv.rw(l, h), new_rec, pv.scale_bits)
+            mism = (zg != zo) | (hg != ho)
+            assert not (mism & (tie == 0)).any(), (r, l, h)
+            n_exc += int(mism.sum())
+            assert np.array_equal(rg.view(np.uint32), ro.view(np.uint32)), (r, l, h)
+            tie_cols = ((tie & 2) != 0).any(axis=0)
+            assert not ((cg.view(np.uint32) != co.view(np.uint32)) & ~tie_cols).any(), (r, l, h)
+    print(f"{name} batch {n}: sampled codes {n_codes}, tie-excused {n_exc}")
+    assert n_exc <= 1e-5 * n_codes
+
+
+def test_layer_shard_of_full_pool_lockstep(stepq):
+    # One GPU's share of a layer-sharded pool (the multi-GPU split, survey row f4):
+    # the library's slice of the 48-layer nominal-6 plan (stepq_plan_slice) with its own
+    # pool layout, stepped by the fused kernel, against the oracle's slice of the same
+    # plan (model.slice_plan) in lockstep for 4 steps, 3 layers x 48 heads x 2 requests.
+    plan, data, wl, _ = oracle_plan("qwen_pool6")
+    lb, le = 20, 23
+    Ps = stepq.Plan.from_bytes(data).slice(lb, le)
+    pv = model.PlanView(model.slice_plan(plan, lb, le))
+    assert Ps.slot_bytes == pv.slot_bytes
+    assert np.array_equal(Ps.widths(), np.asarray(pv.plan["widths"], np.uint8))
+    n, layers = 4, list(range(lb, le))
+    ctx = stepq.Context(Ps, n)
+    pool = torch.zeros(n * Ps.slot_bytes, dtype=torch.uint8, device="cuda")
+    slots = torch.arange(n, dtype=torch.int32, device="cuda")
+    S0 = synth.initial_states(wl, wl.seed, n, layers=layers)
+    ctx.requant_pack(pool, slots, n, 0, le - lb, torch.from_numpy(S0).cuda())
+    ctx.sync()
+    alpha = synth.gates(wl, wl.seed)
+    sb = Ps.slot_bytes
+    tot = exc = 0
+    for t in range(4):
+        prev = pool.cpu().numpy().reshape(n, sb)
+        inp = synth.step_inputs(wl, wl.seed, n, t, alpha=alpha, layers=layers)
+        d = _inputs_to_dev(inp)
+        o = torch.zeros_like(d["q"])
+        ctx.decode_step_fused(pool, slots, n, 0, le - lb, d["q"], d["k"], d["v"], d["alpha"], d["beta"], o)
+        ctx.sync()
+        got = pool.cpu().numpy().reshape(n, sb)
+        o = o.cpu().numpy()
+        for r in (0, n - 1):
+            ora = prev[r].copy()
+            ties = {}
+            for l in range(le - lb):
+                for h in range(pv.H):
+                    o_ref, tie, _, _ = pv.step(ora, l, h, inp["q"][r, l, h], inp["k"][r, l, h], inp["v"][r, l, h],
+                                               inp["alpha"][r, l, h], inp["beta"][r, l, h])
+                    ties[(l, h)] = tie
+                    assert _close(o[r, l, h], o_ref).all(), (t, r, l, h)
+            c, e, b, sbad = compare_records(pv, got[r], ora, ties)
+            tot += c
+            exc += e
+            assert b == 0 and sbad == 0, (t, r, b, sbad)
+    assert exc <= 1e-5 * tot
 
 
 def test_full_pool_sampled_heads(stepq):
