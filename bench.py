@@ -48,7 +48,7 @@ PREFILL_METRIC = "chunked prefill tokens/s into the packed state pool"
 TF32_PER_BF16 = 1.1 / 2.25   # nominal dense TF32 / BF16 tensor throughput
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-KERNEL_SOURCES = ["stepq_head.cu", "stepq_pipe.cuh", "stepq_dev.cuh"]
+KERNEL_SOURCES = ["stepq_head.cu", "stepq_head.cuh", "stepq_head_tm.cu", "stepq_pipe.cuh", "stepq_dev.cuh"]
 
 
 def parse():
@@ -76,6 +76,8 @@ def parse():
     ap.add_argument("--prefill-kernel", default="mma_sync", choices=["mma_sync", "tcgen05"],
                     help="prefill kernel for per-head plans: mma.sync tiles (default) or the state in "
                          "tensor memory with its products on tcgen05")
+    ap.add_argument("--step-kernel", default="registers", choices=["registers", "tmem"],
+                    help="fused step kernel for the per-head pool: state in registers (default) or in tensor memory")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -415,11 +417,12 @@ def variant_is_full_launch(args) -> bool:
             and args.scale_bits == 32 and args.shard == "replicas")
 
 
-def measure_packed(torch, stepq, synth, wl, plan, n, device, steps=12, warmup=3):
+def measure_packed(torch, stepq, synth, wl, plan, n, device, steps=12, warmup=3, step_kernel=0):
     """Fused packed step of a whole pool at batch n: CUDA-event time of `steps`
     steps on the context's main stream."""
     L, H, D = wl.n_layers, wl.n_heads, wl.d
     ctx = stepq.Context(plan, n)
+    ctx.set_step_kernel(step_kernel)
     pool = torch.zeros(n * plan.slot_bytes, dtype=torch.uint8, device=device)
     slots = torch.arange(n, dtype=torch.int32, device=device)
     for l in range(L):
@@ -464,7 +467,7 @@ def measure_fp32(torch, stepq, synth, wl, plan, n, device, steps=6, warmup=2):
     return e0.elapsed_time(e1) / 1e3 / steps
 
 
-def north_star_sweep(torch, stepq, synth, device, plan6, peak):
+def north_star_sweep(torch, stepq, synth, device, plan6, peak, step_kernel=0):
     """The configurations the single-GPU line reports beside the headline: the
     nominal-6 pool at batch 1/16/128/256, the nominal-4 pool over {2,4,6,8} and
     16-bit scales at batch 70, KDA per-key-row units at batch 128, each with the
@@ -474,7 +477,7 @@ def north_star_sweep(torch, stepq, synth, device, plan6, peak):
     out = []
 
     def entry(name, wl, plan, n, fp32=True):
-        t, t_k = measure_packed(torch, stepq, synth, wl, plan, n, device)
+        t, t_k = measure_packed(torch, stepq, synth, wl, plan, n, device, step_kernel=step_kernel)
         L, H, D = wl.n_layers, wl.n_heads, wl.d
         b = step_bytes(plan, n)
         e = {"config": name, "batch": n, "ms_per_step": t * 1e3, "head_steps_per_s": n * L * H / t,
@@ -522,7 +525,9 @@ def run_product(args):
     if args.shard == "layers":
         plan = plan.slice(lb, le)   # this rank holds the records of its own layers only
     L = le - lb
+    step_kernel = stepq.STEP_TMEM if args.step_kernel == "tmem" else stepq.STEP_REGISTERS
     ctx = stepq.Context(plan, n)
+    ctx.set_step_kernel(step_kernel)
     pool = torch.zeros(n * plan.slot_bytes, dtype=torch.uint8, device=device)
     slots = torch.arange(n, dtype=torch.int32, device=device)
     for l in range(L):
@@ -648,7 +653,7 @@ def run_product(args):
     sweep = None
     if (rank == 0 and ws == 1 and not args.no_sweep and args.workload == "gdn" and args.plan == 6
             and args.scale_bits == 32 and args.variant == "fused" and args.batch == 70):
-        sweep = north_star_sweep(torch, stepq, synth, device, plan, peak)
+        sweep = north_star_sweep(torch, stepq, synth, device, plan, peak, step_kernel)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -681,6 +686,7 @@ def run_product(args):
                 **workload_config(wl, n, ws),
                 **({"parallelism": f"layer shards x{ws} (rank 0: layers {lb}-{le - 1})"} if args.shard == "layers" else {}),
                 "variant": args.variant,
+                "step_kernel": args.step_kernel if (args.variant == "fused" and wl.mode == 0) else "registers",
                 "bits_per_value": plan.info.bits_per_value, "bits_per_value_s16": plan.info.bits_per_value_s16,
                 "scale_bits": plan.info.scale_bits, "pool_bytes": n * plan.slot_bytes,
             },

@@ -290,6 +290,17 @@ int stepq_decode_step_fused(stepq_ctx *ctx, void *pool, const int32_t *slots, in
                             int le, const float *q, const float *k, const float *v,
                             const float *alpha, const float *beta, float *o);
 
+/* Which kernel stepq_decode_step_fused runs for per-head plans at d = 128 (other plans
+ * always use the first; results are bit-identical):
+ * STEPQ_STEP_REGISTERS: each thread keeps its 64 state values in registers between the
+ *   passes over a record (two CTAs of 256 threads per SM);
+ * STEPQ_STEP_TMEM: each thread keeps them in its own tensor-memory lane (128 columns per
+ *   CTA, tcgen05.ld/st of 16 values at a time), which frees the registers for three CTAs
+ *   per SM.  Applies to later calls. */
+#define STEPQ_STEP_REGISTERS 0
+#define STEPQ_STEP_TMEM 1
+int stepq_ctx_set_step_kernel(stepq_ctx *ctx, int kernel);
+
 /* Allocation-free variant of stepq_decode_step (the paper has no
  * counterpart; it exists for callers that cannot allocate device memory,
  * such as plugins whose host framework owns every allocation, or latency-

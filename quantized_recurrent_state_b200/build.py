@@ -16,8 +16,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libstepq.so")
-SOURCES = ["stepq_api.cu", "stepq_step.cu", "stepq_head.cu", "stepq_aux.cu", "stepq_prefill.cu", "stepq_prefill_tc.cu", "stepq_tc_selftest.cu"]
-HEADERS = ["stepq_dev.cuh", "stepq_pipe.cuh", "stepq_prefill.cuh", "stepq_tc.cuh", os.path.join("..", "..", "include", "stepq.h")]
+SOURCES = ["stepq_api.cu", "stepq_step.cu", "stepq_head.cu", "stepq_head_tm.cu", "stepq_aux.cu", "stepq_prefill.cu", "stepq_prefill_tc.cu", "stepq_tc_selftest.cu"]
+HEADERS = ["stepq_dev.cuh", "stepq_pipe.cuh", "stepq_head.cuh", "stepq_prefill.cuh", "stepq_tc.cuh", os.path.join("..", "..", "include", "stepq.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 

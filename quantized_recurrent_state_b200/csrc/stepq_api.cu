@@ -36,6 +36,7 @@ cudaError_t launch_calib_acc(int D, const Args &a, double *om, double *ls, cudaS
 cudaError_t launch_calib_dist(int D, const Args &a, const int *bits, int n_bits, double *acc, cudaStream_t st);
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t st);
 cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t st);
+cudaError_t launch_step_tm(const Args &a, int n_sms, cudaStream_t st, int *grid);
 cudaError_t run_tc_selftest(const float *A, const float *B1, const float *B2, float *D1, float *D2, float *D3,
                             int *word);
 }  // namespace stepq
@@ -618,6 +619,7 @@ struct stepq_ctx {
     bool timing = false;
     uint32_t wait_polls = 1u << 22, phantom_tx = 0;
     int prefill_kernel = STEPQ_PREFILL_MMA_SYNC;
+    int step_kernel = STEPQ_STEP_REGISTERS;
     bool poisoned = false;  // a tensor-memory drain failure was reported: refuse further work
     struct Timed { int kind; cudaEvent_t a, b; };
     std::vector<Timed> timed;
@@ -948,7 +950,9 @@ extern "C" int stepq_decode_step_fused(stepq_ctx *c, void *pool, const int32_t *
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.o = o;
     set_stages(c, a, lb, le);
     LaunchTimer lt(c, 2, c->main);
-    const cudaError_t e = stepq::launch_step(2, c->plan->D, a, c->n_sms, c->main, nullptr);
+    const cudaError_t e = (c->step_kernel == STEPQ_STEP_TMEM && c->plan->mode == 0 && c->plan->D == 128)
+                              ? stepq::launch_step_tm(a, c->n_sms, c->main, nullptr)
+                              : stepq::launch_step(2, c->plan->D, a, c->n_sms, c->main, nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "fused launch");
     lt.done();
     return STEPQ_OK;
@@ -980,6 +984,14 @@ extern "C" int stepq_ctx_set_wait_limit(stepq_ctx *c, uint32_t polls, uint32_t p
     if (phantom_bytes >= (1u << 16)) return fail(STEPQ_EINVAL, "set_wait_limit: phantom_bytes %u", phantom_bytes);
     c->wait_polls = polls ? polls : (1u << 22);
     c->phantom_tx = phantom_bytes;
+    return STEPQ_OK;
+}
+
+extern "C" int stepq_ctx_set_step_kernel(stepq_ctx *c, int kernel) {
+    if (!c) return fail(STEPQ_EINVAL, "set_step_kernel: null context");
+    if (kernel != STEPQ_STEP_REGISTERS && kernel != STEPQ_STEP_TMEM)
+        return fail(STEPQ_EINVAL, "set_step_kernel: kernel %d", kernel);
+    c->step_kernel = kernel;
     return STEPQ_OK;
 }
 

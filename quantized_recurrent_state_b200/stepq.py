@@ -27,7 +27,10 @@ EXPORTED = [
     "stepq_launch_count", "stepq_last_error", "stepq_ctx_set_timing", "stepq_kernel_stats",
     "stepq_decode_step_noalloc", "stepq_plan_build_uniform", "stepq_ctx_set_wait_limit", "stepq_plan_slice", "stepq_prefill_fp32", "stepq_prefill",
     "stepq_prefill_workspace_bytes", "stepq_selftest_tc", "stepq_ctx_set_prefill_kernel",
+    "stepq_ctx_set_step_kernel",
 ]
+STEP_REGISTERS = 0    # fused step kernel: state in registers
+STEP_TMEM = 1         # fused step kernel: state in tensor memory (per-head plans, d = 128)
 PREFILL_MMA_SYNC = 0   # prefill kernel: mma.sync tiles, state in shared memory (default)
 PREFILL_TCGEN05 = 1    # prefill kernel: state in tensor memory, state products on tcgen05
 QUANT_DUAL_AXIS = 0  # plan requantizer: STEPQuant row/column fit
@@ -82,6 +85,7 @@ def lib():
         l.stepq_prefill.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, P, P, I]
         l.stepq_selftest_tc.argtypes = [P] * 6
         l.stepq_ctx_set_prefill_kernel.argtypes = [P, I]
+        l.stepq_ctx_set_step_kernel.argtypes = [P, I]
         l.stepq_prefill_workspace_bytes.argtypes = [P, I, I]
         l.stepq_prefill_workspace_bytes.restype = ctypes.c_size_t
         l.stepq_ctx_create.argtypes = [P, P, P, I, I, ctypes.POINTER(P)]
@@ -259,6 +263,9 @@ class Context:
         self._after_caller()
         return _check(lib().stepq_prefill_fp32(self._h, _ptr(S), n_req, lb, le, int(T), _ptr(q), _ptr(k), _ptr(v),
                                                _ptr(alpha), _ptr(beta), _ptr(o), 1 if zero_init else 0))
+
+    def set_step_kernel(self, kernel: int):
+        return _check(lib().stepq_ctx_set_step_kernel(self._h, kernel))
 
     def set_prefill_kernel(self, kernel: int):
         return _check(lib().stepq_ctx_set_prefill_kernel(self._h, kernel))

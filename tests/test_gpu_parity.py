@@ -41,7 +41,7 @@ class Run:
     """A GPU pool for a workload plus an oracle view of the same plan."""
 
     def __init__(self, stepq, name, n_req, n_layers=None, n_pivots=None, extra_slots=3, chunk=2, uniform=None,
-                 scale_bits=32):
+                 scale_bits=32, step_kernel=0):
         if uniform is None:
             self.plan, data, self.wl, _ = oracle_plan(name, n_layers, n_pivots, scale_bits=scale_bits)
         else:  # (bits, quantizer): a baseline plan over the workload's shape
@@ -54,6 +54,7 @@ class Run:
         self.slots = rng.permutation(self.n_slots)[:n_req].astype(np.int32)
         self.slots_t = torch.from_numpy(self.slots).cuda()
         self.ctx = stepq.Context(self.P, self.n_slots, chunk_layers=chunk)
+        self.ctx.set_step_kernel(step_kernel)
         self.pool = torch.zeros(self.n_slots * self.P.slot_bytes, dtype=torch.uint8, device="cuda")
         self.L = self.wl.n_layers
         self.alpha = synth.gates(self.wl, self.wl.seed)
@@ -87,8 +88,8 @@ class Run:
 
 
 def _lockstep(stepq, name, n_req, steps, check, n_layers=None, n_pivots=None, fused=False, heads=None,
-              uniform=None, scale_bits=32):
-    run = Run(stepq, name, n_req, n_layers, n_pivots, uniform=uniform, scale_bits=scale_bits)
+              uniform=None, scale_bits=32, step_kernel=0):
+    run = Run(stepq, name, n_req, n_layers, n_pivots, uniform=uniform, scale_bits=scale_bits, step_kernel=step_kernel)
     S0 = run.pack_initial()
     pv = run.pv
     tot_codes = tot_exc = tot_bad = 0
@@ -160,38 +161,43 @@ def test_tiny_gdn_lockstep_32_steps(stepq, fused):
     _lockstep(stepq, "tiny_gdn", 1, 32, check=[0], fused=fused)
 
 
-@pytest.mark.parametrize("fused", [True, False])
-def test_qwen_layer_lockstep_256_steps(stepq, fused):
+@pytest.mark.parametrize("fused,step_kernel", [(True, 1), (True, 0), (False, 0)])
+def test_qwen_layer_lockstep_256_steps(stepq, fused, step_kernel):
     # 64 requests x 48 heads, d = 128, nominal 6 bits over {4,6,8}, 1 pivot head;
-    # the oracle follows two of the requests (96 heads) at every step; both the
-    # fused step the benchmark times and the two-stream step.
-    _lockstep(stepq, "qwen_layer", 64, 256, check=[0, 37], fused=fused)
+    # the oracle follows two of the requests (96 heads) at every step; the fused
+    # step (state in tensor memory, and in registers) and the two-stream step.
+    _lockstep(stepq, "qwen_layer", 64, 256, check=[0, 37], fused=fused, step_kernel=step_kernel)
 
 
 @pytest.mark.parametrize("name", ["qwen_pool6", "qwen_pool4"])
-def test_pool_slice_lockstep(stepq, name):
+@pytest.mark.parametrize("fused,step_kernel", [(False, 0), (True, 1)])
+def test_pool_slice_lockstep(stepq, name, fused, step_kernel):
     # a 2-layer slice of the 2,304-head pool at batch 70 (2 pivot heads), 8 steps
-    _lockstep(stepq, name, 70, 8, check=[0, 69], n_layers=2, n_pivots=2)
+    _lockstep(stepq, name, 70, 8, check=[0, 69], n_layers=2, n_pivots=2, fused=fused, step_kernel=step_kernel)
 
 
-@pytest.mark.parametrize("bits", [4, 6, 8])
-@pytest.mark.parametrize("fused", [False, True])
-def test_absmax_baseline_lockstep(stepq, bits, fused):
+@pytest.mark.parametrize("bits", [2, 4, 6, 8])
+@pytest.mark.parametrize("fused,step_kernel", [(False, 0), (True, 0), (True, 1)])
+def test_absmax_baseline_lockstep(stepq, bits, fused, step_kernel):
     # uniform INT-b plans with the per-row absmax requantizer over a 2-layer
-    # slice of the pool, batch 70, 6 steps; both step variants
+    # slice of the pool, batch 70, 6 steps; every step variant
     _lockstep(stepq, "qwen_pool6", 70, 6, check=[0, 69], n_layers=2, fused=fused,
-              uniform=(bits, model.QUANT_ABSMAX))
+              uniform=(bits, model.QUANT_ABSMAX), step_kernel=step_kernel)
 
 
-def test_uniform_dual_axis_lockstep(stepq):
-    # uniform INT8 with the STEPQuant fit (no pivots), fused
-    _lockstep(stepq, "qwen_pool6", 70, 6, check=[0, 69], n_layers=2, fused=True, uniform=(8, model.QUANT_DUAL_AXIS))
+@pytest.mark.parametrize("bits", [2, 8])
+@pytest.mark.parametrize("step_kernel", [0, 1])
+def test_uniform_dual_axis_lockstep(stepq, bits, step_kernel):
+    # uniform INT-b with the STEPQuant fit (no pivots), fused
+    _lockstep(stepq, "qwen_pool6", 70, 6, check=[0, 69], n_layers=2, fused=True, uniform=(bits, model.QUANT_DUAL_AXIS),
+              step_kernel=step_kernel)
 
 
-@pytest.mark.parametrize("fused", [False, True])
-def test_scale16_lockstep(stepq, fused):
+@pytest.mark.parametrize("fused,step_kernel", [(False, 0), (True, 0), (True, 1)])
+def test_scale16_lockstep(stepq, fused, step_kernel):
     # calibrated nominal-6 plan with bfloat16 scale storage, 2-layer pool slice
-    _lockstep(stepq, "qwen_pool6", 70, 6, check=[0, 69], n_layers=2, n_pivots=2, fused=fused, scale_bits=16)
+    _lockstep(stepq, "qwen_pool6", 70, 6, check=[0, 69], n_layers=2, n_pivots=2, fused=fused, scale_bits=16,
+              step_kernel=step_kernel)
 
 
 def test_scale16_absmax_lockstep(stepq):
@@ -211,9 +217,10 @@ def test_mid_head_dims_absmax_scale16(stepq, name):
     _lockstep(stepq, name, 6, 4, check=[0, 5], fused=True, uniform=(4, model.QUANT_ABSMAX), scale_bits=16)
 
 
-def test_fused_bit_identical_to_two_stream(stepq):
+@pytest.mark.parametrize("step_kernel", [0, 1])
+def test_fused_bit_identical_to_two_stream(stepq, step_kernel):
     a = Run(stepq, "qwen_layer", 9)
-    b = Run(stepq, "qwen_layer", 9)
+    b = Run(stepq, "qwen_layer", 9, step_kernel=step_kernel)
     a.pack_initial()
     b.pack_initial()
     for t in range(6):
@@ -325,7 +332,7 @@ def test_calibration_kernels_match_oracle(stepq):
             assert np.allclose(dg[0, h, :, m], ref, rtol=1e-12, atol=0)
 
 
-def _full_pool_sampled(stepq, name, n, steps, n_samples, seed, reverse_slots=False):
+def _full_pool_sampled(stepq, name, n, steps, n_samples, seed, reverse_slots=False, step_kernel=0):
     """The whole pool of a workload at batch n in the launch configuration the
     benchmark times: S_0 and the step inputs drawn on the device by the same
     generator, `steps` fused steps, then sampled (request, layer, head) records
@@ -335,6 +342,7 @@ def _full_pool_sampled(stepq, name, n, steps, n_samples, seed, reverse_slots=Fal
     pv = model.PlanView(plan)
     P = stepq.Plan.from_bytes(data)
     ctx = stepq.Context(P, n)
+    ctx.set_step_kernel(step_kernel)
     pool = torch.zeros(n * P.slot_bytes, dtype=torch.uint8, device="cuda")
     slots = torch.arange(n, dtype=torch.int32, device="cuda")
     if reverse_slots:
@@ -430,15 +438,22 @@ def test_layer_shard_of_full_pool_lockstep(stepq):
     assert exc <= 1e-5 * tot
 
 
-def test_full_pool_sampled_heads(stepq):
+@pytest.mark.parametrize("step_kernel", [0, 1])
+def test_full_pool_sampled_heads(stepq, step_kernel):
     # the benchmark's workload: 2,304 heads, batch 70, nominal 6 bits, 32 FP16 heads; 2 steps
-    _full_pool_sampled(stepq, "qwen_pool6", 70, 2, 24, 11)
+    _full_pool_sampled(stepq, "qwen_pool6", 70, 2, 24, 11, step_kernel=step_kernel)
 
 
-def test_full_pool_sampled_heads_batch256(stepq):
+@pytest.mark.parametrize("step_kernel", [0, 1])
+def test_full_pool_sampled_heads_batch256(stepq, step_kernel):
     # the largest batch the benchmark sweeps: 589,824 records in one launch, an 8 GB pool,
     # slots in reverse request order
-    _full_pool_sampled(stepq, "qwen_pool6", 256, 2, 16, 12, reverse_slots=True)
+    _full_pool_sampled(stepq, "qwen_pool6", 256, 2, 16, 12, reverse_slots=True, step_kernel=step_kernel)
+
+
+def test_full_pool_nominal4_sampled_heads(stepq):
+    # the nominal-4 pool over {2,4,6,8} (every width in one launch), state in tensor memory
+    _full_pool_sampled(stepq, "qwen_pool4", 70, 2, 24, 13, step_kernel=1)
 
 
 def test_kda_full_sampled_heads(stepq):
