@@ -15,10 +15,10 @@ readout -> refit r, c -> pack -> write back.
 --prefill T times the chunked prefill of T-token prompt chunks into the
 packed pool instead (tokens/s through the whole pool, tensor roofline).
 
-The default single-GPU line also carries the spec sweep (batch
+The default single-GPU line also carries a sweep of workloads (batch
 1/16/128/256 of the nominal-6 pool, the nominal-4 pool and bfloat16 scales at
 batch 70, KDA rows at batch 128, the FP32-state step beside each) under
-"north_star_sweep".
+"sweep".
 
 Prints one JSON line (rank 0).  N > 1: launched by torch.distributed.run, one
 independent pool per GPU (no collective on the data path), barrier + max of
@@ -68,7 +68,7 @@ def parse():
     ap.add_argument("--workload", default="gdn", choices=["gdn", "kda"],
                     help="gdn: 2,304-head pool; kda: 81,920 key rows (20 x 32 x 128)")
     ap.add_argument("--no-sweep", action="store_true",
-                    help="skip the north-star sweep that the default single-GPU line carries (batch 1/16/128/256, "
+                    help="skip the workload sweep that the default single-GPU line carries (batch 1/16/128/256, "
                          "nominal-4 plan, KDA rows at batch 128, 16-bit scales, the FP32-state kernel for each)")
     ap.add_argument("--prefill", type=int, default=0, metavar="T",
                     help="time chunked prefill of T-token prompt chunks into the packed pool (GDN) instead of "
@@ -467,7 +467,7 @@ def measure_fp32(torch, stepq, synth, wl, plan, n, device, steps=6, warmup=2):
     return e0.elapsed_time(e1) / 1e3 / steps
 
 
-def north_star_sweep(torch, stepq, synth, device, plan6, peak, step_kernel=0):
+def workload_sweep(torch, stepq, synth, device, plan6, peak, step_kernel=0):
     """The configurations the single-GPU line reports beside the headline: the
     nominal-6 pool at batch 1/16/128/256, the nominal-4 pool over {2,4,6,8} and
     16-bit scales at batch 70, KDA per-key-row units at batch 128, each with the
@@ -653,7 +653,7 @@ def run_product(args):
     sweep = None
     if (rank == 0 and ws == 1 and not args.no_sweep and args.workload == "gdn" and args.plan == 6
             and args.scale_bits == 32 and args.variant == "fused" and args.batch == 70):
-        sweep = north_star_sweep(torch, stepq, synth, device, plan, peak, step_kernel)
+        sweep = workload_sweep(torch, stepq, synth, device, plan, peak, step_kernel)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -707,7 +707,7 @@ def run_product(args):
             **extra,
         }
         if sweep:
-            out["north_star_sweep"] = sweep
+            out["sweep"] = sweep
         print(json.dumps(out), flush=True)
     ctx.close()
     if ws > 1:

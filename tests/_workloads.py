@@ -80,7 +80,7 @@ def compare_records(pv: model.PlanView, gpu_slot: np.ndarray, ora_slot: np.ndarr
 
 def reconstruction_gap(pv: model.PlanView, gpu_slot: np.ndarray, ora_slot: np.ndarray, heads, excused=None):
     """Largest |S_hat_gpu - S_hat_oracle| / (1e-5 + 1e-4 |S_hat_oracle|) over the
-    reconstructed states of `heads` [(l, h)], the benchmark spec's tolerance on
+    reconstructed states of `heads` [(l, h)], the stated tolerance on
     reconstructed states (<= 1 passes); elements whose codes were excused as
     rounding ties are left out when `excused` maps (l, h) to the tie map."""
     worst = 0.0

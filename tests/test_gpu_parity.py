@@ -129,7 +129,7 @@ def _lockstep(stepq, name, n_req, steps, check, n_layers=None, n_pivots=None, fu
             tot_codes += c; tot_exc += e; tot_bad += b
             assert b == 0, (t, n, b)
             assert sb == 0, ("scales", t, n, sb)
-            if t % 8 == 0 or t == steps - 1:  # reconstructed states (spec tolerance)
+            if t % 8 == 0 or t == steps - 1:  # reconstructed states (1e-5 + 1e-4 relative)
                 gap = reconstruction_gap(pv, g, ora, list(ties), ties)
                 assert gap <= 1.0, (t, n, gap)
                 worst_s = max(worst_s, gap)
