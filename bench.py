@@ -73,9 +73,9 @@ def parse():
     ap.add_argument("--prefill", type=int, default=0, metavar="T",
                     help="time chunked prefill of T-token prompt chunks into the packed pool (GDN) instead of "
                          "the decode step; batch defaults to 1")
-    ap.add_argument("--prefill-kernel", default="mma_sync", choices=["mma_sync", "tcgen05"],
-                    help="prefill kernel for per-head plans: mma.sync tiles (default) or the state in "
-                         "tensor memory with its products on tcgen05")
+    ap.add_argument("--prefill-kernel", default="tcgen05", choices=["mma_sync", "tcgen05"],
+                    help="prefill kernel for per-head plans: the state in tensor memory with its products on "
+                         "tcgen05 (default) or mma.sync tiles")
     ap.add_argument("--step-kernel", default="registers", choices=["registers", "tmem"],
                     help="fused step kernel for the per-head pool: state in registers (default) or in tensor memory")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
@@ -775,8 +775,7 @@ def run_prefill(args):
         plan = plan.slice(lb, le)   # this rank holds the records of its own layers only
     L = le - lb
     ctx = stepq.Context(plan, n)
-    if args.prefill_kernel == "tcgen05":
-        ctx.set_prefill_kernel(stepq.PREFILL_TCGEN05)
+    ctx.set_prefill_kernel(stepq.PREFILL_TCGEN05 if args.prefill_kernel == "tcgen05" else stepq.PREFILL_MMA_SYNC)
     pool = torch.zeros(n * plan.slot_bytes, dtype=torch.uint8, device=device)
     slots = torch.arange(n, dtype=torch.int32, device=device)
     for l in range(L):

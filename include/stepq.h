@@ -43,8 +43,8 @@
  * Packed format (decided offline, 方法-4 "fixed packed layout").  Codes are
  * stored offset-binary, u = z + 2^(b-1).
  *   per-head units (mode 0), width b in {2,4,6,8}: tile-major layout with
- *     RT = D/8, NT = 2D tiles: element (i,j) -> tile t = (j/4)*8 + i/RT, tile
- *     code (r, c) = (i%RT, j%4); tile stream bits [(4r + c) b, +b), LSB first,
+ *     RT = D/8, NT = 2D tiles: element (i,j) -> tile
+ *     t = 32 (j/16) + 4 (i/RT) + (j/4)%4, tile code (r, c) = (i%RT, j%4); tile stream bits [(4r + c) b, +b), LSB first,
  *     except b = 6 with RT >= 4, where the rows of a tile go in groups of four
  *     over three 32-bit words (rows 0, 1, 3 of a group in bits [0, 24) of
  *     words 0, 1, 2 as 24-bit row values sum_c u_c 2^(6c); the 24-bit value of
@@ -240,12 +240,12 @@ int stepq_prefill_fp32(stepq_ctx *ctx, float *S, int n_req, int lb, int le, int 
                        const float *k, const float *v, const float *alpha, const float *beta, float *o,
                        int zero_init);
 /* Which kernel the prefill of per-head plans runs (per-row plans always use the first):
- * STEPQ_PREFILL_MMA_SYNC (default): the chunk's products as mma.sync TF32 warp tiles,
- *   the state in shared memory;
- * STEPQ_PREFILL_TCGEN05: the state in tensor memory as the A operand of K S and Q S
- *   and the accumulator of the update, those three products on tcgen05 (kind::tf32,
- *   operands from shared memory), the rest on mma.sync; same results within the
- *   tolerance stated in the tests.  Applies to later calls. */
+ * STEPQ_PREFILL_TCGEN05 (default): the state in tensor memory as the A operand of K S
+ *   and Q S and the accumulator of the update, those three products on tcgen05
+ *   (kind::tf32, operands from shared memory), the rest on mma.sync;
+ * STEPQ_PREFILL_MMA_SYNC: the chunk's products as mma.sync TF32 warp tiles, the state
+ *   in shared memory; same results within the tolerance stated in the tests.
+ * Applies to later calls. */
 #define STEPQ_PREFILL_MMA_SYNC 0
 #define STEPQ_PREFILL_TCGEN05 1
 int stepq_ctx_set_prefill_kernel(stepq_ctx *ctx, int kernel);

@@ -117,9 +117,10 @@ static float round_scale(float x, int scale_bits)
 /* u = z + 2^(b-1), in [1, 2^b - 1] for |z| <= qmax = 2^(b-1) - 1.            */
 /*                                                                          */
 /* Uniform-width unit (a head whose rows all share width b):                */
-/*   RT = D/8 rows per band, NT = 2D tiles.  Tile tau = (j/4)*8 + i/RT       */
-/*   holds the RT x 4 block of rows [RT*(i/RT), +RT) and columns             */
-/*   [4*(j/4), +4); inside it (i,j) is the tile code (r, c) = (i%RT, j%4).    */
+/*   RT = D/8 rows per band, NT = 2D tiles.  Tile                           */
+/*   tau = 32*(j/16) + 4*(i/RT) + (j/4)%4 holds the RT x 4 block of rows     */
+/*   [RT*(i/RT), +RT) and columns [4*(j/4), +4); inside it (i,j) is the     */
+/*   tile code (r, c) = (i%RT, j%4).                                        */
 /*   Tile tau's codes form a bit stream; stream byte B lives at block byte   */
 /*   ((B/RT)*NT + tau)*RT + B%RT.  Inside the stream, code (r, c):           */
 /*     b = 2, 4, 8, and b = 6 with RT < 4: bits [(4r+c)*b, +b), LSB first;   */
@@ -157,7 +158,7 @@ static long tile_stream_bit(int D, int b, int r, int c, int k)
 static long uniform_bit_addr(int D, int b, int i, int j, int k)
 {
     int RT = D / 8, NT = 2 * D;
-    long tau = (long)(j / 4) * 8 + i / RT;
+    long tau = (long)(j / 16) * 32 + (i / RT) * 4 + (j / 4) % 4;
     long s = tile_stream_bit(D, b, i % RT, j % 4, k);
     long B = s >> 3;
     long byte = ((B / RT) * NT + tau) * RT + (B % RT);

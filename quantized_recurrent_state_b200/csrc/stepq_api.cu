@@ -618,7 +618,7 @@ struct stepq_ctx {
     uint64_t launches = 0;
     bool timing = false;
     uint32_t wait_polls = 1u << 22, phantom_tx = 0;
-    int prefill_kernel = STEPQ_PREFILL_MMA_SYNC;
+    int prefill_kernel = STEPQ_PREFILL_TCGEN05;
     int step_kernel = STEPQ_STEP_REGISTERS;
     bool poisoned = false;  // a tensor-memory drain failure was reported: refuse further work
     struct Timed { int kind; cudaEvent_t a, b; };

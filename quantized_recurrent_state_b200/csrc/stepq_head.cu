@@ -10,11 +10,11 @@
 //
 // Mapping.  One CTA of NT = 2D threads works on one (request, layer, head)
 // record at a time.  Thread t owns tile t of the tile-major code layout:
-// rows [g RT, g RT + RT) (band g = t & 7, RT = D/8) of columns
-// [4 cb, 4 cb + 4) (cb = t >> 3).  A warp therefore holds 16 whole value
-// columns: every column reduction (u, o, the initial column factor and the
-// two least-squares sums) runs over the 8 bands of a column group inside one
-// warp (lanes xor 1, 2, 4), in the balanced tree of the band order; only the
+// rows [g RT, g RT + RT) (band g = (t / 4) % 8, RT = D/8) of columns
+// [4 cb, 4 cb + 4) (cb = 4 (t / 32) + t % 4).  A warp therefore holds 16 whole
+// value columns: every column reduction (u, o, the initial column factor and
+// the two least-squares sums) runs over the 8 bands of a column group inside
+// one warp (lanes xor 4, 8, 16), in the balanced tree of the band order; only the
 // row sums cross warps (one shared-memory exchange, two block barriers per
 // record).  The state lives in registers as row pairs: S[k][c] holds rows
 // g RT + 2k and g RT + 2k + 1 of column 4 cb + c, so the even/odd row chains
@@ -39,7 +39,7 @@ template <int D, int B, int KIND, int S16, int QUANT, class Rel>
 __device__ bool item_head(const Args &a, const uint8_t *stage, uint8_t *rec_g, int row, ScratchH<D> &sc, int tid,
                           bool ok, Rel &rel) {
     constexpr int NP = D / 16, RT = D / 8;
-    const int g = tid & 7, cb = tid >> 3, lane = tid & 31, i0 = g * RT, j0 = 4 * cb;
+    const int g = band_of(tid), cb = cblk_of(tid), lane = tid & 31, i0 = g * RT, j0 = 4 * cb;
     const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
     const uint8_t *st_r = stage + codes_bytes;
     const uint8_t *st_c = st_r + D * (S16 ? 2 : 4);
@@ -142,7 +142,7 @@ __device__ bool item_head(const Args &a, const uint8_t *stage, uint8_t *rec_g, i
 template <int D, int KIND, class Rel>
 __device__ bool item_pivot(const Args &a, const uint8_t *stage, uint8_t *rec_g, int row, int tid, bool ok, Rel &rel) {
     constexpr int NP = D / 16, RT = D / 8;
-    const int g = tid & 7, lane = tid & 31, i0 = g * RT, j0 = 4 * (tid >> 3);
+    const int g = band_of(tid), lane = tid & 31, i0 = g * RT, j0 = 4 * cblk_of(tid);
     const float *tf = stage_tail<D>(a, stage);
     const float *qs = tf + kTailQ * D, *ks = tf + kTailK * D, *vs = tf + kTailV * D, *xs = tf + kTailX * D;
     const float *ab = stage_ab<D>(a, stage);
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(2 * D, 2) k_step_head(Args a) {
 template <int D>
 __device__ __forceinline__ void load_tile(const float *Sg, int tid, float2 (&S)[D / 16][4]) {
     constexpr int NP = D / 16, RT = D / 8;
-    const int i0 = (tid & 7) * RT, j0 = 4 * (tid >> 3);
+    const int i0 = band_of(tid) * RT, j0 = 4 * cblk_of(tid);
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
         const float4 x = *reinterpret_cast<const float4 *>(Sg + (size_t)(i0 + 2 * k) * D + j0);
@@ -331,7 +331,7 @@ __device__ void requant_head(float2 (&S)[D / 16][4], uint8_t *rec, ScratchH<D> &
     const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
     uint8_t *rec_r = rec + codes_bytes;
     uint8_t *rec_c = rec_r + D * (S16 ? 2 : 4);
-    row_partials<D, QUANT>(S, sc, tid & 7, tid >> 3);
+    row_partials<D, QUANT>(S, sc, band_of(tid), cblk_of(tid));
     __syncthreads();
     row_phase<D, B, S16, QUANT>(sc, tid, sc.rho, sc.wbar, rec_r);
     uint32_t W[Stream<D, B>::NW];
@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(2 * D) k_requant_head(Args a) {
     load_tile<D>(a.S_in + (size_t)row * D * D, tid, S);
     const int width = a.t.width[gl];
     if (width == kPivotBits) {
-        const int i0 = (tid & 7) * RT, j0 = 4 * (tid >> 3);
+        const int i0 = band_of(tid) * RT, j0 = 4 * cblk_of(tid);
 #pragma unroll
         for (int k = 0; k < NP; ++k) {
             const int i = i0 + 2 * k;
@@ -403,7 +403,7 @@ __global__ void __launch_bounds__(2 * D) k_requant_head(Args a) {
 template <int D, int B>
 __device__ void unpack_head(const uint8_t *rec, float *out, int tid, int s16) {
     constexpr int NP = D / 16, RT = D / 8;
-    const int i0 = (tid & 7) * RT, j0 = 4 * (tid >> 3);
+    const int i0 = band_of(tid) * RT, j0 = 4 * cblk_of(tid);
     const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
     const uint8_t *rr = rec + codes_bytes;
     const uint8_t *cc = rr + D * (s16 ? 2 : 4);
@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(2 * D) k_unpack_head(Args a) {
         case 6: unpack_head<D, 6>(rec, out, tid, a.scale16); break;
         case 8: unpack_head<D, 8>(rec, out, tid, a.scale16); break;
         case kPivotBits: {
-            const int i0 = (tid & 7) * RT, j0 = 4 * (tid >> 3);
+            const int i0 = band_of(tid) * RT, j0 = 4 * cblk_of(tid);
 #pragma unroll
             for (int r = 0; r < RT; ++r) {
                 const int i = i0 + r;
@@ -473,10 +473,10 @@ struct BitList {
 template <int D, int B>
 __device__ void dist_head(const float *Sg, int gl, int m, int n_bits, double *dist_acc, ScratchH<D> &sc, int tid) {
     constexpr int NP = D / 16, RT = D / 8, Q = (1 << (B - 1)) - 1;
-    const int g = tid & 7, lane = tid & 31, i0 = g * RT, j0 = 4 * (tid >> 3);
+    const int g = band_of(tid), lane = tid & 31, i0 = g * RT, j0 = 4 * cblk_of(tid);
     float2 S[NP][4];
     load_tile<D>(Sg, tid, S);
-    row_partials<D, kQuantDualAxis>(S, sc, g, tid >> 3);
+    row_partials<D, kQuantDualAxis>(S, sc, g, cblk_of(tid));
     __syncthreads();
     row_phase<D, B, 0, kQuantDualAxis>(sc, tid, sc.rho, sc.wbar, nullptr);
     uint32_t W[Stream<D, B>::NW];
@@ -503,12 +503,12 @@ __device__ void dist_head(const float *Sg, int gl, int m, int n_bits, double *di
             ea = fma(da, da, ea);
             eb = fma(db, db, eb);
         }
-        // the row's other column blocks of this warp (lanes xor 8, 16)
-        ea += __shfl_xor_sync(kFull, ea, 8);
-        ea += __shfl_xor_sync(kFull, ea, 16);
-        eb += __shfl_xor_sync(kFull, eb, 8);
-        eb += __shfl_xor_sync(kFull, eb, 16);
-        if ((lane >> 3) == 0) {
+        // the row's other column blocks of this warp (lanes xor 1, 2)
+        ea += __shfl_xor_sync(kFull, ea, 1);
+        ea += __shfl_xor_sync(kFull, ea, 2);
+        eb += __shfl_xor_sync(kFull, eb, 1);
+        eb += __shfl_xor_sync(kFull, eb, 2);
+        if ((lane & 3) == 0) {
             atomicAdd(&dist_acc[((size_t)gl * D + i) * n_bits + m], ea);
             atomicAdd(&dist_acc[((size_t)gl * D + i + 1) * n_bits + m], eb);
         }

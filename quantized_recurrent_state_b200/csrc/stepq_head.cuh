@@ -47,48 +47,60 @@ __device__ __forceinline__ int pidx(int cb, int i) {
 
 constexpr unsigned kFull = 0xffffffffu;
 
+// Tile of thread t (tile t of the code layout): band g = lane bits [2, 5),
+// column block cb = 4 (t / 32) + (t % 4).  The 8 lanes of a quarter warp then
+// cover two bands and four column blocks, so the per-row operand loads (two
+// distinct 16-byte addresses per quarter) and the row-partial stores are free
+// of bank conflicts.
+__device__ __forceinline__ int band_of(int t) { return (t >> 2) & 7; }
+__device__ __forceinline__ int cblk_of(int t) { return ((t >> 5) << 2) | (t & 3); }
+// Lane xor masks that reach band g ^ 1, g ^ 2, g ^ 4 of the same column block.
+constexpr int kX1 = 4, kX2 = 8, kX4 = 16;
+// Lane of band gs in the column block of `lane`.
+__device__ __forceinline__ int band_lane(int lane, int gs) { return (lane & ~28) | (gs << 2); }
+
 // ---------------------------------------------------------------------------
-// Column reductions over the 8 bands of a column group (lanes xor 1, 2, 4).
-// Level 1 adds bands (g, g^1), level 2 pairs of those, level 3 the halves:
-// ((b0 + b1) + (b2 + b3)) + ((b4 + b5) + (b6 + b7)).  Each level keeps half
-// of the lane's columns and sends the other half to its partner, so after
-// the three levels the lane holds one finished column.
+// Column reductions over the 8 bands of a column group (bands g ^ 1, g ^ 2,
+// g ^ 4).  Level 1 adds bands (g, g^1), level 2 pairs of those, level 3 the
+// halves: ((b0 + b1) + (b2 + b3)) + ((b4 + b5) + (b6 + b7)).  Each level keeps
+// half of the lane's columns and sends the other half to its partner, so
+// after the three levels the lane holds one finished column.
 // ---------------------------------------------------------------------------
 
 // After band_sum4 / band_max4 the lane with band g holds column 2 (g & 1) + ((g >> 1) & 1).
 __device__ __forceinline__ int col4_of(int g) { return 2 * (g & 1) + ((g >> 1) & 1); }
-// Lane of the same column group that holds column c after band_sum4 / band_max4.
-__device__ __forceinline__ int col4_src(int lane, int c) { return (lane & ~7) | (c >> 1) | ((c & 1) << 1); }
+// Lane of the same column block that holds column c after band_sum4 / band_max4.
+__device__ __forceinline__ int col4_src(int lane, int c) { return band_lane(lane, (c >> 1) | ((c & 1) << 1)); }
 
 __device__ __forceinline__ float band_sum4(float v0, float v1, float v2, float v3, int g) {
     const bool h1 = g & 1, h2 = g & 2;
     float ka = h1 ? v2 : v0, kb = h1 ? v3 : v1;
     const float sa = h1 ? v0 : v2, sb = h1 ? v1 : v3;
-    ka = ka + __shfl_xor_sync(kFull, sa, 1);
-    kb = kb + __shfl_xor_sync(kFull, sb, 1);
+    ka = ka + __shfl_xor_sync(kFull, sa, kX1);
+    kb = kb + __shfl_xor_sync(kFull, sb, kX1);
     float k = h2 ? kb : ka;
     const float s = h2 ? ka : kb;
-    k = k + __shfl_xor_sync(kFull, s, 2);
-    return k + __shfl_xor_sync(kFull, k, 4);
+    k = k + __shfl_xor_sync(kFull, s, kX2);
+    return k + __shfl_xor_sync(kFull, k, kX4);
 }
 
 __device__ __forceinline__ float band_max4(float v0, float v1, float v2, float v3, int g) {
     const bool h1 = g & 1, h2 = g & 2;
     float ka = h1 ? v2 : v0, kb = h1 ? v3 : v1;
     const float sa = h1 ? v0 : v2, sb = h1 ? v1 : v3;
-    ka = fmaxf(ka, __shfl_xor_sync(kFull, sa, 1));
-    kb = fmaxf(kb, __shfl_xor_sync(kFull, sb, 1));
+    ka = fmaxf(ka, __shfl_xor_sync(kFull, sa, kX1));
+    kb = fmaxf(kb, __shfl_xor_sync(kFull, sb, kX1));
     float k = h2 ? kb : ka;
     const float s = h2 ? ka : kb;
-    k = fmaxf(k, __shfl_xor_sync(kFull, s, 2));
-    return fmaxf(k, __shfl_xor_sync(kFull, k, 4));
+    k = fmaxf(k, __shfl_xor_sync(kFull, s, kX2));
+    return fmaxf(k, __shfl_xor_sync(kFull, k, kX4));
 }
 
 // The two least-squares sums of four columns: the lane with band g ends with
 // N (g even) or D (g odd) of column 2 ((g >> 1) & 1) + ((g >> 2) & 1); its
 // partner lane g ^ 1 holds the other sum of the same column.
 __device__ __forceinline__ int col8_of(int g) { return 2 * ((g >> 1) & 1) + ((g >> 2) & 1); }
-__device__ __forceinline__ int col8_src(int lane, int c) { return (lane & ~7) | ((c >> 1) << 1) | ((c & 1) << 2); }
+__device__ __forceinline__ int col8_src(int lane, int c) { return band_lane(lane, ((c >> 1) << 1) | ((c & 1) << 2)); }
 
 __device__ __forceinline__ float band_sum8(const float (&N)[4], const float (&Dn)[4], int g) {
     const bool h1 = g & 1, h2 = g & 2, h4 = g & 4;
@@ -96,15 +108,15 @@ __device__ __forceinline__ float band_sum8(const float (&N)[4], const float (&Dn
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         const float keep = h1 ? Dn[c] : N[c], send = h1 ? N[c] : Dn[c];
-        k[c] = keep + __shfl_xor_sync(kFull, send, 1);
+        k[c] = keep + __shfl_xor_sync(kFull, send, kX1);
     }
     float ka = h2 ? k[2] : k[0], kb = h2 ? k[3] : k[1];
     const float sa = h2 ? k[0] : k[2], sb = h2 ? k[1] : k[3];
-    ka = ka + __shfl_xor_sync(kFull, sa, 2);
-    kb = kb + __shfl_xor_sync(kFull, sb, 2);
+    ka = ka + __shfl_xor_sync(kFull, sa, kX2);
+    kb = kb + __shfl_xor_sync(kFull, sb, kX2);
     float kk = h4 ? kb : ka;
     const float s = h4 ? ka : kb;
-    return kk + __shfl_xor_sync(kFull, s, 4);
+    return kk + __shfl_xor_sync(kFull, s, kX4);
 }
 
 // max(m, |x|, |y|)
@@ -385,7 +397,7 @@ __device__ __forceinline__ void fit_codes(float2 (&S)[D / 16][4], ScratchH<D> &s
     constexpr int NP = D / 16, RT = D / 8;
     constexpr int OFF = 1 << (B - 1), Q = OFF - 1;
     constexpr float IQ = 1.0f / (float)Q;
-    const int g = tid & 7, lane = tid & 31, i0 = g * RT, j0 = 4 * (tid >> 3);
+    const int g = band_of(tid), lane = tid & 31, i0 = g * RT, j0 = 4 * cblk_of(tid);
     // y and the column maxima of |y|
     float m[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     float2 pr[NP];
@@ -432,7 +444,7 @@ __device__ __forceinline__ void fit_codes(float2 (&S)[D / 16][4], ScratchH<D> &s
         Dn[c] = da[c].x + da[c].y;
     }
     const float mine = band_sum8(N, Dn, g);
-    const float other = __shfl_xor_sync(kFull, mine, 1);
+    const float other = __shfl_xor_sync(kFull, mine, kX1);
     const float num = (g & 1) ? other : mine, den = (g & 1) ? mine : other;
     const int c8 = col8_of(g);
     const float c0c = __shfl_sync(kFull, c0, col4_src(lane, c8));
@@ -463,7 +475,7 @@ template <int D, int B>
 __device__ __forceinline__ void absmax_codes(const float2 (&S)[D / 16][4], const ScratchH<D> &sc, int tid,
                                              uint32_t (&W)[Stream<D, B>::NW]) {
     constexpr int NP = D / 16, RT = D / 8, OFF = 1 << (B - 1);
-    const int i0 = (tid & 7) * RT;
+    const int i0 = band_of(tid) * RT;
     const float2 mg2 = make_float2(kMagic + (float)OFF, kMagic + (float)OFF);
     uint32_t ha = 0u, hb = 0u;
     float2 pr[NP];

@@ -7,8 +7,8 @@
 // Arithmetic definitions: include/stepq.h.
 //
 // Same mapping, arithmetic and order of operations as k_step_head (thread t
-// owns tile t: rows [16 g, 16 g + 16) x columns [4 cb, 4 cb + 4), g = t & 7,
-// cb = t >> 3; warps hold whole value columns), but the 64 state values of a
+// owns tile t: rows [16 g, 16 g + 16) x columns [4 cb, 4 cb + 4), g = band_of(t),
+// cb = cblk_of(t); warps hold whole value columns), but the 64 state values of a
 // thread live in its own tensor-memory lane between the passes, 16 at a time
 // in registers.  That frees the registers the state would hold, so three
 // CTAs (24 warps) share an SM instead of two and the column reductions and
@@ -204,7 +204,7 @@ __device__ bool item(const Args &a, const uint8_t *stage, uint8_t *rec_g, int ro
                      Rel &rel, uint32_t tb) {
     constexpr int OFF = 1 << (B - 1), Q = OFF - 1;
     constexpr float IQ = 1.0f / (float)Q;
-    const int g = tid & 7, cb = tid >> 3, lane = tid & 31, i0 = g * RT, j0 = 4 * cb;
+    const int g = band_of(tid), cb = cblk_of(tid), lane = tid & 31, i0 = g * RT, j0 = 4 * cb;
     const uint32_t codes_bytes = (uint32_t)D * D * B / 8;
     const uint8_t *st_r = stage + codes_bytes;
     const uint8_t *st_c = st_r + D * (S16 ? 2 : 4);
@@ -388,7 +388,7 @@ __device__ bool item(const Args &a, const uint8_t *stage, uint8_t *rec_g, int ro
             Dn[c] = da[c].x + da[c].y;
         }
         const float mine = band_sum8(N, Dn, g);
-        const float other = __shfl_xor_sync(kFull, mine, 1);
+        const float other = __shfl_xor_sync(kFull, mine, kX1);
         const float num = (g & 1) ? other : mine, den = (g & 1) ? mine : other;
         const int c8 = col8_of(g);
         const float c0c = __shfl_sync(kFull, c0, col4_src(lane, c8));
@@ -424,7 +424,7 @@ __device__ bool item(const Args &a, const uint8_t *stage, uint8_t *rec_g, int ro
 template <class Rel>
 __device__ bool item_pivot(const Args &a, const uint8_t *stage, uint8_t *rec_g, int row, int tid, bool ok, Rel &rel,
                            uint32_t tb) {
-    const int g = tid & 7, lane = tid & 31, i0 = g * RT, j0 = 4 * (tid >> 3);
+    const int g = band_of(tid), lane = tid & 31, i0 = g * RT, j0 = 4 * cblk_of(tid);
     const float *tf = stage_tail<D>(a, stage);
     const float *qs = tf + kTailQ * D, *ks = tf + kTailK * D, *vs = tf + kTailV * D;
     const float *ab = stage_ab<D>(a, stage);

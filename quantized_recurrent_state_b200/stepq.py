@@ -31,8 +31,8 @@ EXPORTED = [
 ]
 STEP_REGISTERS = 0    # fused step kernel: state in registers
 STEP_TMEM = 1         # fused step kernel: state in tensor memory (per-head plans, d = 128)
-PREFILL_MMA_SYNC = 0   # prefill kernel: mma.sync tiles, state in shared memory (default)
-PREFILL_TCGEN05 = 1    # prefill kernel: state in tensor memory, state products on tcgen05
+PREFILL_MMA_SYNC = 0   # prefill kernel: mma.sync tiles, state in shared memory
+PREFILL_TCGEN05 = 1    # prefill kernel: state in tensor memory, state products on tcgen05 (default)
 QUANT_DUAL_AXIS = 0  # plan requantizer: STEPQuant row/column fit
 QUANT_ABSMAX = 1     # plan requantizer: per-row absmax baseline, c = 1
 NOALLOC_SCRATCH_BYTES = 8 << 20

@@ -2,7 +2,8 @@
 
 The prefill evaluates the gated delta rule in chunks of 64 tokens with the
 dense products on the tensor cores (TF32 plus a TF32 remainder) and an fp32
-triangular solve, so it matches the oracle to a tolerance, not bit for bit.
+triangular solve (per-head plans: both prefill kernels, the tcgen05 default
+and the mma.sync one, run every per-head case), so it matches the oracle to a tolerance, not bit for bit.
 Tolerance: each product has relative error about 2^-21 of its terms' sum
 (the dropped lo*lo term and the TF32 rounding of the remainders), the fp32
 solve about 64 * 2^-24, the gate ratios about |log gamma| 2^-24; over T/64
@@ -22,6 +23,22 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-4
+
+
+# per-head plans run either prefill kernel; both are checked
+KERNELS = ["tcgen05", "mma_sync"]
+
+
+@pytest.fixture(params=KERNELS)
+def pk(request):
+    return request.param
+
+
+def _ctx(stepq, P, n, pk=None):
+    ctx = stepq.Context(P, n)
+    if pk is not None:
+        ctx.set_prefill_kernel(stepq.PREFILL_TCGEN05 if pk == "tcgen05" else stepq.PREFILL_MMA_SYNC)
+    return ctx
 
 
 @pytest.fixture(scope="module")
@@ -50,11 +67,11 @@ def _check_head(O_gpu, S_gpu, S0, inp, r, h, l=0):
 
 
 @pytest.mark.parametrize("T", [1, 64, 65, 100, 127, 256])
-def test_prefill_fp32_matches_sequential(stepq, T):
+def test_prefill_fp32_matches_sequential(stepq, pk, T):
     plan, data, wl, _ = oracle_plan("qwen_layer")
     P = stepq.Plan.from_bytes(data)
     n = 2
-    ctx = stepq.Context(P, n)
+    ctx = _ctx(stepq, P, n, pk)
     S0 = synth.initial_states(wl, wl.seed, n)                     # [n][1][H][D][D]
     inp = _prompt(wl, n, T, 3000 + T)
     d = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
@@ -70,10 +87,10 @@ def test_prefill_fp32_matches_sequential(stepq, T):
     print(f"T={T}: worst relative errors o {worst[0]:.2e}, S {worst[1]:.2e}")
 
 
-def test_prefill_fp32_zero_init_and_empty(stepq):
+def test_prefill_fp32_zero_init_and_empty(stepq, pk):
     plan, data, wl, _ = oracle_plan("qwen_layer")
     P = stepq.Plan.from_bytes(data)
-    ctx = stepq.Context(P, 1)
+    ctx = _ctx(stepq, P, 1, pk)
     inp = _prompt(wl, 1, 70, 41)
     d = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
     S = torch.full((1, 1, wl.n_heads, wl.d, wl.d), float("nan"), dtype=torch.float32, device="cuda")
@@ -88,12 +105,12 @@ def test_prefill_fp32_zero_init_and_empty(stepq):
 
 
 @pytest.mark.parametrize("from_zero", [False, True])
-def test_prefill_into_packed_states(stepq, from_zero):
+def test_prefill_into_packed_states(stepq, pk, from_zero):
     plan, data, wl, _ = oracle_plan("qwen_layer")
     pv = model.PlanView(plan)
     P = stepq.Plan.from_bytes(data)
     n, T = 3, 130
-    ctx = stepq.Context(P, n + 2)
+    ctx = _ctx(stepq, P, n + 2, pk)
     slots = torch.tensor([4, 0, 2], dtype=torch.int32, device="cuda")
     pool = torch.zeros((n + 2) * P.slot_bytes, dtype=torch.uint8, device="cuda")
     S0 = synth.initial_states(wl, wl.seed, n)
@@ -124,14 +141,14 @@ def test_prefill_into_packed_states(stepq, from_zero):
         assert np.array_equal(after[s * sb:(s + 1) * sb], before[s * sb:(s + 1) * sb])
 
 
-def test_prefill_layer_range_uniform_plan(stepq):
+def test_prefill_layer_range_uniform_plan(stepq, pk):
     """Layers [1, 3) of a three-layer uniform 6-bit plan (dual-axis), inputs
     laid out for the range only; layer 0 and slots outside the batch stay put."""
     plan, data, wl, _ = uniform_plan("qwen_pool6", 6, model.QUANT_DUAL_AXIS, n_layers=3)
     pv = model.PlanView(plan)
     P = stepq.Plan.from_bytes(data)
     n, T, lb, le = 2, 70, 1, 3
-    ctx = stepq.Context(P, 3)
+    ctx = _ctx(stepq, P, 3, pk)
     slots = torch.tensor([2, 0], dtype=torch.int32, device="cuda")
     pool = torch.zeros(3 * P.slot_bytes, dtype=torch.uint8, device="cuda")
     S0 = synth.initial_states(wl, wl.seed, n)
@@ -162,7 +179,7 @@ def test_prefill_layer_range_uniform_plan(stepq):
     assert np.array_equal(after[sb:2 * sb], before[sb:2 * sb])
 
 
-def test_prefill_full_pool_sampled(stepq):
+def test_prefill_full_pool_sampled(stepq, pk):
     """The launch the prefill benchmark times: a 2,048-token chunk for all
     2,304 heads of the pool (nominal 6 bits, 32 FP16 heads) at batch 1, inputs
     drawn on the device by the same generator.  Sampled heads (and FP16 heads)
@@ -173,7 +190,7 @@ def test_prefill_full_pool_sampled(stepq):
     pv = model.PlanView(plan)
     P = stepq.Plan.from_bytes(data)
     n, T, L = 1, 2048, wl.n_layers
-    ctx = stepq.Context(P, n)
+    ctx = _ctx(stepq, P, n, pk)
     pool = torch.zeros(n * P.slot_bytes, dtype=torch.uint8, device="cuda")
     slots = torch.arange(n, dtype=torch.int32, device="cuda")
     for l in range(L):
@@ -277,14 +294,14 @@ def test_prefill_rows_into_packed_states(stepq, from_zero):
     assert np.array_equal(after[sb:2 * sb], before[sb:2 * sb])
 
 
-def test_prefill_degenerate_gates_full_pool(stepq):
+def test_prefill_degenerate_gates_full_pool(stepq, pk):
     """alpha = 1, beta = 0 for every token of the whole pool (2,304 heads, batch
     1, 300 tokens): M = 0 and the update adds exact zeros, so the fp32 state
     comes back bit for bit, and o_t = S_0^T q_t."""
     plan, data, wl, _ = uniform_plan("qwen_pool6", 6, model.QUANT_DUAL_AXIS)
     P = stepq.Plan.from_bytes(data)
     n, T, L = 1, 300, wl.n_layers
-    ctx = stepq.Context(P, n)
+    ctx = _ctx(stepq, P, n, pk)
     inp = synth.prompt_inputs_torch(wl, wl.seed, n, 0, T, synth.gates(wl, wl.seed), "cuda")
     inp["alpha"].fill_(1.0)
     inp["beta"].zero_()
@@ -299,11 +316,11 @@ def test_prefill_degenerate_gates_full_pool(stepq):
     assert float(err.max()) <= TOL, float(err.max())
 
 
-def test_packed_prefill_noop_calls(stepq):
+def test_packed_prefill_noop_calls(stepq, pk):
     """T = 0 and n_req = 0 leave the pool as it was."""
     plan, data, wl, _ = oracle_plan("qwen_layer")
     P = stepq.Plan.from_bytes(data)
-    ctx = stepq.Context(P, 2)
+    ctx = _ctx(stepq, P, 2, pk)
     slots = torch.tensor([1, 0], dtype=torch.int32, device="cuda")
     pool = torch.zeros(2 * P.slot_bytes, dtype=torch.uint8, device="cuda")
     ctx.requant_pack(pool, slots, 2, 0, 1, torch.from_numpy(synth.initial_states(wl, wl.seed, 2)).cuda())
@@ -338,7 +355,7 @@ def test_prefill_gates_out_of_range_are_reported(stepq):
                 {k: v.cpu().numpy() for k, v in inp.items()}, 0, 3)
 
     plan, data, wl, _ = oracle_plan("qwen_layer")
-    ctx = stepq.Context(stepq.Plan.from_bytes(data), 1)
+    ctx = stepq.Context(stepq.Plan.from_bytes(data), 1)     # per-head plans: the default (tcgen05) kernel
     inp = {k: torch.from_numpy(v).cuda() for k, v in _prompt(wl, 1, 10, 13).items()}
     S = torch.zeros((1, 1, wl.n_heads, wl.d, wl.d), dtype=torch.float32, device="cuda")
     o = torch.zeros_like(inp["q"])
@@ -351,8 +368,8 @@ def test_prefill_gates_out_of_range_are_reported(stepq):
     ctx.sync()
 
 
-@pytest.mark.parametrize("name", ["qwen_layer", "kda_rows"])
-def test_prefill_then_decode(stepq, name):
+@pytest.mark.parametrize("name,kern", [("qwen_layer", "tcgen05"), ("qwen_layer", "mma_sync"), ("kda_rows", None)])
+def test_prefill_then_decode(stepq, name, kern):
     """The serving order: a 100-token prompt prefilled into packed states,
     then 3 fused decode steps from the records the prefill wrote, checked
     against the oracle stepping the same records (codes bit-exact up to
@@ -362,7 +379,7 @@ def test_prefill_then_decode(stepq, name):
     pv = model.PlanView(plan)
     P = stepq.Plan.from_bytes(data)
     n, T = 2, 100
-    ctx = stepq.Context(P, n)
+    ctx = _ctx(stepq, P, n, kern)
     slots = torch.tensor([1, 0], dtype=torch.int32, device="cuda")
     pool = torch.zeros(n * P.slot_bytes, dtype=torch.uint8, device="cuda")
     ctx.requant_pack(pool, slots, n, 0, 1, torch.from_numpy(synth.initial_states(wl, wl.seed, n)).cuda())
