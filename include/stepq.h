@@ -50,8 +50,14 @@
  *     words 0, 1, 2 as 24-bit row values sum_c u_c 2^(6c); the 24-bit value of
  *     row 2 byte by byte in bits [24, 32) of the same words); stream byte B
  *     of tile t at block byte ((B/RT) NT + t) RT + B%RT.
- *   per-row units (mode 1): rows in order, row i = D*b_i/8 bytes, code j at
- *     row bits [b_i j, b_i j + b_i); a 16-bit row holds binary16 values.
+ *   per-row units (mode 1): band-tile layout.  Band g = rows [g RT, g RT + RT),
+ *     RT = D/8; tile (g, cb) = the band's rows x columns [4 cb, 4 cb + 4), NCB = D/4
+ *     tiles per band.  A tile's stream holds, row after row, the row's four codes
+ *     of b_r bits each (LSB first; a 16-bit row holds binary16 values): row r at
+ *     stream bits [P_r, P_r + 4 b_r), P_r = 4 sum_{r'<r} b_r'.  Each tile takes
+ *     NW_g = ceil(P_RT / 32) 32-bit words; band g's block starts at word
+ *     W_g = NCB sum_{g'<g} NW_g', and stream word m of tile cb is word
+ *     W_g + m NCB + (cb + 4 g) mod NCB of the codes block, little endian.
  *   record = codes | r[D] | c[D], zero-padded to 128 bytes, r and c fp32, or
  *     bfloat16 in plans with 16-bit scales (header word at byte 60 = 16: r_i
  *     is rounded to bfloat16, RNE, as soon as it is formed and used rounded

@@ -68,6 +68,10 @@ def _declare(l):
     l.sq_codes_bytes_rows.restype = L
     l.sq_pack_rows.argtypes = [I, P, P, P, P]
     l.sq_unpack_rows.argtypes = [I, P, P, P, P]
+    l.sq_codes_bytes_bands.argtypes = [I, P]
+    l.sq_codes_bytes_bands.restype = L
+    l.sq_pack_bands.argtypes = [I, P, P, P, P]
+    l.sq_unpack_bands.argtypes = [I, P, P, P, P]
     l.sq_pairwise_sum.argtypes = [P, I]
     l.sq_pairwise_sum.restype = F
     l.sq_band_dot.argtypes = [I, P, I, P, I]
@@ -157,6 +161,29 @@ def unpack_rows(D: int, widths, blk: np.ndarray):
     z = np.zeros((D, D), dtype=np.int32)
     h = np.zeros((D, D), dtype=np.uint16)
     lib().sq_unpack_rows(D, _p(w), _p(blk), _p(z), _p(h))
+    return z, h
+
+
+def codes_bytes_bands(D: int, widths) -> int:
+    w = _i32(widths)
+    return int(lib().sq_codes_bytes_bands(D, _p(w)))
+
+
+def pack_bands(D: int, widths, z: np.ndarray, h: np.ndarray) -> np.ndarray:
+    w = _i32(widths)
+    z = _i32(z).reshape(D, D)
+    h = np.ascontiguousarray(h, dtype=np.uint16).reshape(D, D)
+    out = np.zeros(codes_bytes_bands(D, w), dtype=np.uint8)
+    lib().sq_pack_bands(D, _p(w), _p(z), _p(h), _p(out))
+    return out
+
+
+def unpack_bands(D: int, widths, blk: np.ndarray):
+    w = _i32(widths)
+    blk = np.ascontiguousarray(blk, dtype=np.uint8)
+    z = np.zeros((D, D), dtype=np.int32)
+    h = np.zeros((D, D), dtype=np.uint16)
+    lib().sq_unpack_bands(D, _p(w), _p(blk), _p(z), _p(h))
     return z, h
 
 

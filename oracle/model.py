@@ -45,7 +45,7 @@ def pack_head(mode: int, D: int, rw, z, h, r, c, scale_bits: int = 32) -> np.nda
     if mode == 0:
         blk = core.pack_uniform(D, int(rw[0]), z)
     else:
-        blk = core.pack_rows(D, rw, z, h)
+        blk = core.pack_bands(D, rw, z, h)
     rec[:blk.size] = blk
     e = scale_bits // 8
     rec[blk.size:blk.size + e * D] = _scales_to_bytes(r, scale_bits)
@@ -64,7 +64,7 @@ def unpack_head(mode: int, D: int, rw, rec: np.ndarray, scale_bits: int = 32):
         z = core.unpack_uniform(D, int(rw[0]), rec[:nb])
         h = np.zeros((D, D), np.uint16)
     else:
-        z, h = core.unpack_rows(D, rw, rec[:nb])
+        z, h = core.unpack_bands(D, rw, rec[:nb])
     e = scale_bits // 8
     r = _scales_from_bytes(rec[nb:nb + e * D], D, scale_bits)
     c = _scales_from_bytes(rec[nb + e * D:nb + 2 * e * D], D, scale_bits)

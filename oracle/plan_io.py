@@ -117,8 +117,7 @@ def record_bytes(mode: int, D: int, row_widths, scale_bits: int = 32) -> int:
         if b == PIVOT_BITS:
             return _align(D * D * 2, 128)
         return _align(D * D * b // 8 + sb, 128)
-    codes = int(sum(D * int(b) // 8 for b in rw))
-    return _align(codes + sb, 128)
+    return _align(codes_block_bytes(mode, D, rw) + sb, 128)
 
 
 def codes_block_bytes(mode: int, D: int, row_widths) -> int:
@@ -126,7 +125,10 @@ def codes_block_bytes(mode: int, D: int, row_widths) -> int:
     if mode == 0:
         b = int(rw[0])
         return D * D * 2 if b == PIVOT_BITS else D * D * b // 8
-    return int(sum(D * int(b) // 8 for b in rw))
+    # band-tile layout: per band of D/8 rows, D/4 tiles of ceil(4 * sum of the band's widths / 32) words
+    RT = D // 8
+    words = [-(-4 * int(sum(int(b) for b in rw[g * RT:(g + 1) * RT])) // 32) for g in range(8)]
+    return 4 * (D // 4) * int(sum(words))
 
 
 def pool_layout(plan: dict):

@@ -130,9 +130,19 @@ static float round_scale(float x, int scale_bits)
 /*       words 3g, 3g+1, 3g+2; the 24-bit value of row s = 2 is stored byte  */
 /*       by byte in bits [24, 32) of the same three words (byte m in word     */
 /*       3g+m).                                                             */
-/* Row-major unit (rows of mixed width): row i starts at the sum of the     */
-/*   byte sizes D*b/8 of the rows before it; code j occupies row bits         */
-/*   [b*j, b*j+b).  A 16-bit row holds binary16 values, 2 bytes per column.  */
+/* Row-major tile (a pivot head): row i starts at the sum of the byte sizes */
+/*   D*b/8 of the rows before it; code j occupies row bits [b*j, b*j+b).    */
+/*   A 16-bit row holds binary16 values, 2 bytes per column.                */
+/* Band-tile unit (per-row units, rows of mixed width): RT = D/8 rows per   */
+/*   band, NCB = D/4 tiles per band; tile (g, cb) holds rows [g*RT, +RT) x   */
+/*   columns [4*cb, +4).  Its stream: for r = 0 .. RT-1 the four codes of    */
+/*   row g*RT + r (columns 4cb .. 4cb+3), b_r bits each, LSB first, at       */
+/*   stream bits [P_r + c*b_r, +b_r), P_r = 4 * sum_{r' < r} b_r'; a 16-bit  */
+/*   row stores its binary16 patterns.  A tile stream takes                 */
+/*   NW_g = ceil(P_RT / 32) 32-bit words (the rest of the last word is 0).   */
+/*   Band g's block starts at word W_g = NCB * sum_{g' < g} NW_g'; stream    */
+/*   word m of tile cb is block word W_g + m*NCB + (cb + 4g) mod NCB, little */
+/*   endian.                                                                */
 /* ------------------------------------------------------------------------ */
 
 static int get_bit(const uint8_t *blk, long bit) { return (blk[bit >> 3] >> (bit & 7)) & 1; }
@@ -238,6 +248,68 @@ void sq_unpack_rows(int D, const int *widths, const uint8_t *blk, int32_t *z, ui
             }
         }
         off += sq_row_bytes(D, b);
+    }
+}
+
+/* Stream words of a tile of band g. */
+static long band_tile_words(int D, const int *widths, int g)
+{
+    int RT = D / 8;
+    long bits = 0;
+    for (int r = 0; r < RT; r++) bits += 4L * widths[g * RT + r];
+    return (bits + 31) / 32;
+}
+
+long sq_codes_bytes_bands(int D, const int *widths)
+{
+    long words = 0;
+    for (int g = 0; g < 8; g++) words += (long)(D / 4) * band_tile_words(D, widths, g);
+    return 4 * words;
+}
+
+/* Block bit address of bit k of the field of element (i, j). */
+static long band_bit_addr(int D, const int *widths, int i, int j, int k)
+{
+    int RT = D / 8, NCB = D / 4;
+    int g = i / RT, r = i % RT, cb = j / 4, c = j % 4;
+    long base = 0;
+    for (int gg = 0; gg < g; gg++) base += (long)NCB * band_tile_words(D, widths, gg);
+    long p = 0;
+    for (int rr = 0; rr < r; rr++) p += 4L * widths[g * RT + rr];
+    long s = p + (long)c * widths[i] + k;           /* stream bit */
+    long word = base + (s / 32) * NCB + (cb + 4 * g) % NCB;
+    return word * 32 + s % 32;
+}
+
+/* Band-tile pack.  z holds codes for quantized rows; h holds binary16
+ * patterns for 16-bit rows (entries of other rows are ignored). */
+void sq_pack_bands(int D, const int *widths, const int32_t *z, const uint16_t *h, uint8_t *blk)
+{
+    memset(blk, 0, (size_t)sq_codes_bytes_bands(D, widths));
+    for (int i = 0; i < D; i++) {
+        int b = widths[i];
+        for (int j = 0; j < D; j++) {
+            unsigned u = (b == SQ_PIVOT_BITS) ? (unsigned)h[i * D + j] : (unsigned)(z[i * D + j] + (1 << (b - 1)));
+            for (int k = 0; k < b; k++) set_bit(blk, band_bit_addr(D, widths, i, j, k), (u >> k) & 1);
+        }
+    }
+}
+
+void sq_unpack_bands(int D, const int *widths, const uint8_t *blk, int32_t *z, uint16_t *h)
+{
+    for (int i = 0; i < D; i++) {
+        int b = widths[i];
+        for (int j = 0; j < D; j++) {
+            unsigned u = 0;
+            for (int k = 0; k < b; k++) u |= (unsigned)get_bit(blk, band_bit_addr(D, widths, i, j, k)) << k;
+            if (b == SQ_PIVOT_BITS) {
+                h[i * D + j] = (uint16_t)u;
+                z[i * D + j] = 0;
+            } else {
+                z[i * D + j] = (int32_t)u - (1 << (b - 1));
+                h[i * D + j] = 0;
+            }
+        }
     }
 }
 

@@ -210,11 +210,19 @@ static int plan_parse(const uint8_t *d, size_t n, stepq_plan *p) {
             codes = (uint64_t)D * D * w / 8;
             rec = (w == STEPQ_PIVOT_BITS) ? align_up(codes, 128) : align_up(codes + 2ull * (p->scale_bits / 8) * D, 128);
         } else {
-            codes = 0;
-            for (int i = 0; i < D; ++i) {
-                p->row_off[hd * D + i] = (uint32_t)codes;
-                codes += (uint64_t)D * p->width[hd * D + i] / 8;
+            // band-tile layout: band g's tiles take NW_g = ceil(4 sum_r b_r / 32) words each;
+            // row_off = (first word of the band's block) << 11 | (stream bit of the row)
+            const int RT = D / 8, NCB = D / 4;
+            uint64_t words = 0;
+            for (int g = 0; g < 8; ++g) {
+                uint32_t bit = 0;
+                for (int r = 0; r < RT; ++r) {
+                    p->row_off[hd * D + g * RT + r] = (uint32_t)(words << 11) | bit;
+                    bit += 4u * p->width[hd * D + g * RT + r];
+                }
+                words += (uint64_t)NCB * ((bit + 31) / 32);
             }
+            codes = 4 * words;
             rec = align_up(codes + 2ull * (p->scale_bits / 8) * D, 128);
         }
         p->rec_off[hd] = off;

@@ -34,7 +34,7 @@ struct Tables {
     const uint32_t *codes_bytes; // [L*H] bytes of the codes block
     const uint8_t *width;        // [L*H] mode 0 unit width (16 = pivot head)
     const uint8_t *row_width;    // [L*H*D] mode 1 row widths (else null)
-    const uint32_t *row_off;     // [L*H*D] mode 1 row byte offsets (else null)
+    const uint32_t *row_off;     // [L*H*D] mode 1: (first word of the row's band block) << 11 | (stream bit of the row in its tile); else null
     const float *wbar;           // [L*H*D]
     const float *rho;            // [L*H*D]
 };

@@ -109,6 +109,72 @@ def test_uniform_layout_hand_bytes(name):
     assert np.array_equal(core.unpack_uniform(D, b, blk), z)
 
 
+def _golden_bands():
+    cases = {}
+    with open(os.path.join(GOLDEN, "layout_bands.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            cases.setdefault(parts[0], {})[parts[1]] = parts[2:]
+    return cases
+
+
+@pytest.mark.parametrize("name", ["d16mix", "d32w8"])
+def test_band_layout_hand_bytes(name):
+    case = _golden_bands()[name]
+    widths = np.array([int(x) for x in case["widths"][0].split(",")], np.int32)
+    D = widths.size
+    z = np.zeros((D, D), np.int32)
+    h = np.zeros((D, D), np.uint16)
+    for item in case.get("set", []):
+        i, j, val = (int(x) for x in item.split(","))
+        z[i, j] = val
+    for item in case.get("half", []):
+        i, j, val = item.split(",")
+        h[int(i), int(j)] = int(val, 16)
+    blk = core.pack_bands(D, widths, z, h)
+    exp = np.zeros(core.codes_bytes_bands(D, widths), np.uint8)
+    items = case["expect"]
+    k = 0
+    while k < len(items):
+        if items[k] == "pattern":
+            rng_s, pat = items[k + 1].split("=")
+            a_, b_ = (int(x) for x in rng_s.split(":"))
+            p = np.array([int(x, 16) for x in pat.split(",")], np.uint8)
+            exp[a_:b_] = np.tile(p, (b_ - a_) // p.size)
+            k += 2
+        else:
+            off, val = items[k].split("=")
+            exp[int(off)] = int(val, 16)
+            k += 1
+    assert blk.size == exp.size
+    assert np.array_equal(blk, exp)
+    z2, h2 = core.unpack_bands(D, widths, blk)
+    assert np.array_equal(z2, z) and np.array_equal(h2, h)
+
+
+def test_band_layout_roundtrip_and_size():
+    D = 128
+    widths = rng.choice([2, 4, 6, 8, 16], size=D).astype(np.int32)
+    z = np.zeros((D, D), np.int32)
+    h = np.zeros((D, D), np.uint16)
+    for i, b in enumerate(widths):
+        if b == 16:
+            h[i] = rng.integers(0, 1 << 16, size=D).astype(np.uint16)
+        else:
+            q = (1 << (b - 1)) - 1
+            z[i] = rng.integers(-q, q + 1, size=D)
+    blk = core.pack_bands(D, widths, z, h)
+    # each band pads its tiles to whole words: between the row-major size and 31 bits per tile more
+    raw = sum(D * int(b) // 8 for b in widths)
+    assert raw <= blk.size < raw + 8 * 32 * 4
+    assert blk.size == sum(128 * -(-int(widths[16 * g:16 * g + 16].sum()) // 8) for g in range(8))
+    z2, h2 = core.unpack_bands(D, widths, blk)
+    assert np.array_equal(z2, z) and np.array_equal(h2, h)
+
+
 def test_rows_layout_lsb_first():
     # row-major: code j of a b-bit row occupies row bits [b*j, b*j+b)
     D = 16
