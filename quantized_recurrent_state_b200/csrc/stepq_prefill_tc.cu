@@ -133,6 +133,23 @@ __device__ __forceinline__ void warp_gemm_split(float (&acc)[NTILE][4], const fl
 __device__ __forceinline__ int xoff(int t, int i) { return (int)(tc::kmajor_off(t, i, D) >> 2); }   // X[t][i]
 __device__ __forceinline__ int ktoff(int i, int t) { return (int)(tc::kmajor_off(i, t, C) >> 2); }  // KT[i][t]
 
+// TF32 hi/lo split of the chunk's rows of x (K or Q) into X (rows past cc are 0).  An
+// iteration covers one 8-row core group: thread -> row 8 it + (tid % 8), columns
+// 4 (tid / 8) .. + 3, so a quarter warp writes eight consecutive 16-byte core rows.
+template <class RowOf>
+__device__ __forceinline__ void split_rows(Smem &sm, const float *x, RowOf row_of, int c0, int cc, int tid) {
+#pragma unroll 4
+    for (int it = 0; it < C / 8; ++it) {
+        const int r = 8 * it + (tid & 7), i = 4 * (tid >> 3);
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < cc) v = *reinterpret_cast<const float4 *>(x + row_of(c0 + r) + i);
+        float4 hi, lo;
+        split(v.x, hi.x, lo.x); split(v.y, hi.y, lo.y); split(v.z, hi.z, lo.z); split(v.w, hi.w, lo.w);
+        *reinterpret_cast<float4 *>(&sm.Xhi[xoff(r, i)]) = hi;
+        *reinterpret_cast<float4 *>(&sm.Xlo[xoff(r, i)]) = lo;
+    }
+}
+
 __global__ void __launch_bounds__(NT, 1) k_prefill_tc(PrefillArgs a) {
     extern __shared__ __align__(1024) uint8_t smraw[];
     Smem &sm = *reinterpret_cast<Smem *>(smraw);
@@ -182,18 +199,15 @@ __global__ void __launch_bounds__(NT, 1) k_prefill_tc(PrefillArgs a) {
     for (int c0 = 0; c0 < a.T && ok; c0 += C, ++ci) {
         const int cc = min(C, a.T - c0);
         const uint32_t par = ci & 1;
-        // 1. K split into X, V, gates
+        // 1. K split into X, V, gates.  The split tiles are written 8 rows x 4 columns per
+        // quarter warp (row fastest): eight consecutive 16-byte core rows, free of bank
+        // conflicts; V keeps rows of consecutive columns per warp.
+        split_rows(sm, a.k, row_of, c0, cc, tid);
+#pragma unroll 4
         for (int e = tid; e < C * D / 4; e += NT) {
             const int r = e / (D / 4), i = 4 * (e % (D / 4));
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
-            if (r < cc) {
-                x = *reinterpret_cast<const float4 *>(a.k + row_of(c0 + r) + i);
-                y = *reinterpret_cast<const float4 *>(a.v + row_of(c0 + r) + i);
-            }
-            float4 hi, lo;
-            split(x.x, hi.x, lo.x); split(x.y, hi.y, lo.y); split(x.z, hi.z, lo.z); split(x.w, hi.w, lo.w);
-            *reinterpret_cast<float4 *>(&sm.Xhi[xoff(r, i)]) = hi;
-            *reinterpret_cast<float4 *>(&sm.Xlo[xoff(r, i)]) = lo;
+            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r < cc) y = *reinterpret_cast<const float4 *>(a.v + row_of(c0 + r) + i);
             *reinterpret_cast<float4 *>(&sm.V[r * SV + i]) = y;
         }
         if (w == 0) {
@@ -275,15 +289,7 @@ __global__ void __launch_bounds__(NT, 1) k_prefill_tc(PrefillArgs a) {
         }
         __syncthreads();
         // Q split into X
-        for (int e = tid; e < C * D / 4; e += NT) {
-            const int r = e / (D / 4), i = 4 * (e % (D / 4));
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (r < cc) x = *reinterpret_cast<const float4 *>(a.q + row_of(c0 + r) + i);
-            float4 hi, lo;
-            split(x.x, hi.x, lo.x); split(x.y, hi.y, lo.y); split(x.z, hi.z, lo.z); split(x.w, hi.w, lo.w);
-            *reinterpret_cast<float4 *>(&sm.Xhi[xoff(r, i)]) = hi;
-            *reinterpret_cast<float4 *>(&sm.Xlo[xoff(r, i)]) = lo;
-        }
+        split_rows(sm, a.q, row_of, c0, cc, tid);
         tc::fence_smem_to_async();
         tc::fence_before();
         __syncthreads();

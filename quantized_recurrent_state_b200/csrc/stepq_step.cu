@@ -85,16 +85,13 @@ struct StreamOut {
     uint8_t *tile0;
     uint32_t acc = 0, fill = 0, m = 0;
     __device__ __forceinline__ void put(uint32_t f, uint32_t nbits) {  // nbits <= 32
-        acc |= f << fill;
+        const uint32_t word = acc | (f << fill);
         const uint32_t nf = fill + nbits;
-        if (nf >= 32u) {
-            *reinterpret_cast<uint32_t *>(tile0 + m * (4u * NCB)) = acc;
-            ++m;
-            acc = __funnelshift_l(f, 0u, fill);  // the bits of f past the word end (0 when fill = 0)
-            fill = nf - 32u;
-        } else {
-            fill = nf;
-        }
+        const bool full = nf >= 32u;
+        if (full) *reinterpret_cast<uint32_t *>(tile0 + m * (4u * NCB)) = word;
+        acc = full ? __funnelshift_l(f, 0u, fill) : word;  // the bits of f past the word end (0 when fill = 0)
+        m += full ? 1u : 0u;
+        fill = full ? nf - 32u : nf;
     }
     __device__ __forceinline__ void flush() {
         if (fill) *reinterpret_cast<uint32_t *>(tile0 + m * (4u * NCB)) = acc;
@@ -232,7 +229,9 @@ __device__ __forceinline__ void fit_pack_rows(float2 (&S)[NP][4], const ScratchR
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
         const uint32_t ba = wid(wv, 2 * k), bb = wid(wv, 2 * k + 1);
-        const float2 mg2 = make_float2(kMagic + (float)(1u << (ba - 1u)), kMagic + (float)(1u << (bb - 1u)));
+        // 1.5 2^23 + 2^(b-1): the offset lands in the mantissa of 1.5 2^23 (0x4B400000)
+        const float2 mg2 = make_float2(__uint_as_float(0x4B400000u + (1u << (ba - 1u))),
+                                       __uint_as_float(0x4B400000u + (1u << (bb - 1u))));
         const uint32_t bound = ((2u << (ba - 1u)) - 2u) | (((2u << (bb - 1u)) - 2u) << 16);
         uint32_t e[4];
 #pragma unroll
