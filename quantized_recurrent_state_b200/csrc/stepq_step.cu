@@ -85,13 +85,16 @@ struct StreamOut {
     uint8_t *tile0;
     uint32_t acc = 0, fill = 0, m = 0;
     __device__ __forceinline__ void put(uint32_t f, uint32_t nbits) {  // nbits <= 32
-        const uint32_t word = acc | (f << fill);
+        acc |= f << fill;
         const uint32_t nf = fill + nbits;
-        const bool full = nf >= 32u;
-        if (full) *reinterpret_cast<uint32_t *>(tile0 + m * (4u * NCB)) = word;
-        acc = full ? __funnelshift_l(f, 0u, fill) : word;  // the bits of f past the word end (0 when fill = 0)
-        m += full ? 1u : 0u;
-        fill = full ? nf - 32u : nf;
+        if (nf >= 32u) {
+            *reinterpret_cast<uint32_t *>(tile0 + m * (4u * NCB)) = acc;
+            ++m;
+            acc = __funnelshift_l(f, 0u, fill);  // the bits of f past the word end (0 when fill = 0)
+            fill = nf - 32u;
+        } else {
+            fill = nf;
+        }
     }
     __device__ __forceinline__ void flush() {
         if (fill) *reinterpret_cast<uint32_t *>(tile0 + m * (4u * NCB)) = acc;
