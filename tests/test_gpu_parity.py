@@ -87,6 +87,50 @@ class Run:
         return inp, o.cpu().numpy()
 
 
+@pytest.mark.parametrize("name,n,steps,kw", [("qwen_layer", 3, 64, {}),
+                                              ("kda_rows", 2, 24, {"n_layers": 1, "n_pivots": 8})])
+def test_free_running_trajectory(stepq, name, n, steps, kw):
+    """The free-running comparison beside the lockstep one: the GPU (fused
+    step) and the oracle each step their own records from the same S_0, with
+    no resynchronisation.  Until the oracle meets a rounding tie (a non-zero
+    tie map) the two trajectories must stay identical bit for bit, records and
+    readouts; after a tie the run only reports the step of the first
+    difference and how far the readouts have drifted."""
+    run = Run(stepq, name, n, **kw)
+    S0 = run.pack_initial()
+    pv = run.pv
+    ora, tie_step = {}, None
+    for r in range(n):
+        slot = np.zeros(run.P.slot_bytes, np.uint8)
+        for l in range(pv.L):
+            for h in range(pv.H):
+                if pv.quantize_into(slot, l, h, S0[r, l, h]).any():
+                    tie_step = -1 if tie_step is None else tie_step
+        ora[r] = slot
+    first_diff, worst_o = None, 0.0
+    for t in range(-1, steps):
+        if t >= 0:
+            inp, o = run.step(t, fused=True)
+        for r in range(n):
+            if t >= 0:
+                for l in range(pv.L):
+                    for h in range(pv.H):
+                        o_ref, tie, _, _ = pv.step(ora[r], l, h, inp["q"][r, l, h], inp["k"][r, l, h], inp["v"][r, l, h],
+                                                   inp["alpha"][r, l, h], inp["beta"][r, l, h])
+                        if tie.any() and tie_step is None:
+                            tie_step = t
+                        if not np.array_equal(o[r, l, h], o_ref):
+                            first_diff = t if first_diff is None else first_diff
+                        scale = max(1e-30, float(np.max(np.abs(o_ref))))
+                        worst_o = max(worst_o, float(np.max(np.abs(o[r, l, h] - o_ref))) / scale)
+            if not np.array_equal(run.slot_bytes_host(r), ora[r]):
+                first_diff = t if first_diff is None else first_diff
+        if tie_step is None:
+            assert first_diff is None, (t, "trajectories differ before any rounding tie")
+    print(f"free-running {name}: {steps} steps, first tie {tie_step}, first difference {first_diff}, "
+          f"worst readout difference {worst_o:.3g} of the head's largest readout")
+
+
 def _lockstep(stepq, name, n_req, steps, check, n_layers=None, n_pivots=None, fused=False, heads=None,
               uniform=None, scale_bits=32, step_kernel=0):
     run = Run(stepq, name, n_req, n_layers, n_pivots, uniform=uniform, scale_bits=scale_bits, step_kernel=step_kernel)
