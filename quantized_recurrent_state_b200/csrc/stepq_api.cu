@@ -679,8 +679,6 @@ stepq::Args base_args(stepq_ctx *c, void *pool, const int32_t *slots, int n_req,
     a.div_h = stepq::div_magic((uint32_t)c->plan->H);
     a.t = c->t;
     a.err = c->err;
-    a.neg_zero = -0.0f;
-    a.x_bits = 0x4B000000u;
     return a;
 }
 

@@ -63,8 +63,6 @@ struct Args {
     float *S_out;            // unpack output
     Tables t;
     int *err;
-    float neg_zero;          // -0.0f (a run-time value the compiler cannot fold)
-    uint32_t x_bits;         // 0x4B000000, the exponent word of the X encoding, held in a register
     uint32_t wait_polls;     // polls before a copy wait gives up (error kErrWait)
     uint32_t phantom_tx;     // extra expected bytes per stage that never arrive (0: none; timeout test)
     uint32_t stage_bytes;    // bytes of one pipeline stage
@@ -186,47 +184,6 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
         : "=f"(d.x), "=f"(d.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
     return d;
-}
-
-// ---------------------------------------------------------------------------
-// Packed fields.  A b-bit code z is stored as u = z + 2^(b-1).  The value
-//   X = 0x4B000000 | (u << 12)
-// is the fp32 number 2^23 + u 2^12, so z 2^12 = X - (2^23 + off 2^12) exactly
-// (one subtraction); that fp32 value, widened to fp64, is the operand of the
-// fp64 projections (products with k_i a_i 2^-12 are exact).
-// ---------------------------------------------------------------------------
-
-template <int B>
-__device__ __forceinline__ uint32_t field_x(const uint32_t *W, int p, uint32_t xbits = 0x4B000000u) {
-    const int bit = p * B;
-    const int w = bit >> 5;
-    const int s = bit & 31;
-    uint32_t x;
-    if (s + B <= 32) {
-        x = (s >= 12) ? (W[w] >> (s - 12)) : (W[w] << (12 - s));
-    } else {
-        x = __funnelshift_r(W[w], W[w + 1], s - 12);
-    }
-    return (x & (((1u << B) - 1u) << 12)) | xbits;
-}
-
-
-template <int B>
-__device__ __forceinline__ float x_as_zscaled(uint32_t X) {
-    // z * 2^12, exact
-    return __fsub_rn(__uint_as_float(X), 8388608.0f + (float)(1 << (B - 1)) * 4096.0f);
-}
-
-// ---------------------------------------------------------------------------
-// Reduction: butterfly over LANES consecutive lanes (every lane ends with the
-// same fp64 sum).
-// ---------------------------------------------------------------------------
-
-template <int LANES>
-__device__ __forceinline__ double lane_sum_f64(double v) {
-#pragma unroll
-    for (int m = 1; m < LANES; m <<= 1) v = v + __shfl_xor_sync(0xffffffffu, v, m);
-    return v;
 }
 
 __device__ __forceinline__ void flag_error(int *err, int code) { atomicOr(err, code); }
