@@ -1,7 +1,7 @@
 // Pipeline pieces shared by the step kernels of both unit kinds: item
 // coordinates, the 16-byte step descriptors, the staging of one item (the
 // packed record, the input rows, the head's tables) into a shared-memory
-// stage by 1-D bulk copies, and the thread-major code streams.
+// stage by 1-D bulk copies, and the tile-major code streams.
 //
 // STEPQuant paper digest (vibe-research), 方法-4: every decode step reads the
 // packed record, updates, reads out and writes the record back before the
