@@ -119,6 +119,8 @@ __device__ __forceinline__ float band_sum8(const float (&N)[4], const float (&Dn
     return kk + __shfl_xor_sync(kFull, s, kX4);
 }
 
+__device__ __forceinline__ float2 abs2(float2 x) { return make_float2(fabsf(x.x), fabsf(x.y)); }
+
 // max(m, |x|, |y|)
 __device__ __forceinline__ float max3abs(float m, float x, float y) {
     float d;
@@ -326,9 +328,12 @@ __device__ __forceinline__ void row_partials(const float2 (&S)[D / 16][4], Scrat
         if (QUANT == kQuantAbsmax) {
             rs[2 * k] = fmaxf(fmaxf(fabsf(S[k][0].x), fabsf(S[k][1].x)), fmaxf(fabsf(S[k][2].x), fabsf(S[k][3].x)));
             rs[2 * k + 1] = fmaxf(fmaxf(fabsf(S[k][0].y), fabsf(S[k][1].y)), fmaxf(fabsf(S[k][2].y), fabsf(S[k][3].y)));
-        } else {  // pairwise over the four columns
-            rs[2 * k] = (fabsf(S[k][0].x) + fabsf(S[k][1].x)) + (fabsf(S[k][2].x) + fabsf(S[k][3].x));
-            rs[2 * k + 1] = (fabsf(S[k][0].y) + fabsf(S[k][1].y)) + (fabsf(S[k][2].y) + fabsf(S[k][3].y));
+        } else {  // pairwise over the four columns, both rows of the pair in one packed add
+            const float2 p01 = add2(abs2(S[k][0]), abs2(S[k][1]));
+            const float2 p23 = add2(abs2(S[k][2]), abs2(S[k][3]));
+            const float2 r = add2(p01, p23);
+            rs[2 * k] = r.x;
+            rs[2 * k + 1] = r.y;
         }
     }
     float *dst = &sc.part[pidx<D>(cb, g * (D / 8))];
