@@ -217,6 +217,8 @@ def test_new_entry_points_reject_bad_arguments_without_a_device():
     l = stepq.lib()
     assert l.stepq_ctx_set_prefill_kernel(None, stepq.PREFILL_TCGEN05) == stepq.EINVAL
     assert b"null context" in l.stepq_last_error()
+    assert l.stepq_ctx_set_step_kernel(None, stepq.STEP_TMEM) == stepq.EINVAL
+    assert b"null context" in l.stepq_last_error()
     assert l.stepq_selftest_tc(None, None, None, None, None, None) == stepq.EINVAL
     assert b"A" in l.stepq_last_error()
     assert l.stepq_prefill_workspace_bytes(None, 1, 1) == 0
