@@ -160,6 +160,16 @@ __global__ void __launch_bounds__(NT, 1) k_prefill_tc(PrefillArgs a) {
     const int n = item / per_req, rem = item - n * per_req, ll = rem / a.H, h = rem - ll * a.H;
     float *Sg = a.S + (size_t)item * D * D;
     auto row_of = [&](int tok) { return (((size_t)(n * a.T + tok) * a.nL_in + a.l_in0 + ll) * a.H + h) * D; };
+    // the k, q, v rows of the chunk from token c0 into L2 ahead of their (synchronous) loads
+    auto prefetch_chunk = [&](int c0) {
+        const int cc = min(C, a.T - c0);
+        if (tid < 3 * cc) {
+            const int r = tid / 3, which = tid - 3 * r;
+            const float *base = which == 0 ? a.k : which == 1 ? a.q : a.v;
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + row_of(c0 + r)), "r"(D * 4)
+                         : "memory");
+        }
+    };
     const int q4 = w & 3, hh = w >> 2;               // this warp's lane quadrant and half
     const int j = 32 * q4 + lane;                    // the lane (value column j) this thread reads in tensor memory
     const uint32_t quad = (uint32_t)(32 * q4) << 16;
@@ -167,6 +177,7 @@ __global__ void __launch_bounds__(NT, 1) k_prefill_tc(PrefillArgs a) {
     auto xo_t = [](int k, int nn) { return xoff(nn, k); };
     auto kto = [](int k, int nn) { return ktoff(k, nn); };
 
+    prefetch_chunk(0);
     if (tid == 0)
         for (int b = 0; b < 3; ++b) tc::mbar_init(&sm.bar[b]);
     if (w == 0) tc::alloc(&sm.taddr, NCOLS);
@@ -199,6 +210,7 @@ __global__ void __launch_bounds__(NT, 1) k_prefill_tc(PrefillArgs a) {
     for (int c0 = 0; c0 < a.T && ok; c0 += C, ++ci) {
         const int cc = min(C, a.T - c0);
         const uint32_t par = ci & 1;
+        if (c0 + C < a.T) prefetch_chunk(c0 + C);
         // 1. K split into X, V, gates.  The split tiles are written 8 rows x 4 columns per
         // quarter warp (row fastest): eight consecutive 16-byte core rows, free of bank
         // conflicts; V keeps rows of consecutive columns per warp.
