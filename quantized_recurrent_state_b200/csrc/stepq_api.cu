@@ -779,7 +779,8 @@ extern "C" int stepq_ctx_create(const stepq_plan *plan, void *main_stream, void 
     // heads in width order (per-head units; per-row units keep head order),
     // so concurrently running items mostly share one width's code path.
     // Entry: record offset low word, (offset bits 32..47) | head << 16,
-    // staged record bytes (0 for an FP16 head), width | codes bytes << 8.
+    // staged record bytes (0 for an FP16 head), width | codes bytes << 8
+    // (per-row units: 16 if the head has an FP16 row, else 0).
     if (p->slot_bytes >> 48) { cudaFree(c->tables_mem); delete c; return fail(STEPQ_EFORMAT, "ctx_create: slot above 2^48 bytes"); }
     std::vector<uint32_t> desc(4 * heads);
     for (int l = 0; l < p->L; ++l) {
@@ -795,7 +796,11 @@ extern "C" int stepq_ctx_create(const stepq_plan *plan, void *main_stream, void 
             desc[e] = (uint32_t)p->rec_off[hd];
             desc[e + 1] = (uint32_t)((p->rec_off[hd] >> 32) & 0xffffu) | ((uint32_t)order[k] << 16);
             desc[e + 2] = staged ? p->rec_bytes[hd] : 0u;
-            desc[e + 3] = (uint32_t)(p->mode == 0 ? p->head_width[hd] : 0) | (p->codes_bytes[hd] << 8);
+            uint32_t wbyte = p->mode == 0 ? p->head_width[hd] : 0u;
+            if (p->mode == 1)  // per-row units: 16 marks a head with FP16 rows (the step kernels' FP16 path)
+                for (int i = 0; i < p->D; ++i)
+                    if (p->row_width[hd * p->D + i] == STEPQ_PIVOT_BITS) wbyte = STEPQ_PIVOT_BITS;
+            desc[e + 3] = wbyte | (p->codes_bytes[hd] << 8);
         }
     }
     c->t.desc = (const uint4 *)put(desc.data(), sz_desc, sz_desc);

@@ -28,6 +28,9 @@ constexpr int D = 128, NT = 2 * D, RT = D / 8, NP = D / 16, NCB = D / 4;
 struct __align__(16) ScratchR {
     ScratchH<D> h;     // row partials, 1/r, b, r, rho, wbar, descriptors, stage metadata
     float iq[D];       // fl(1/qmax_i); 0 for FP16 rows
+    uint32_t mgb[D];   // bits of 1.5 2^23 + 2^(b_i - 1): the rounding constant of row i's final codes
+    uint32_t ones[D];  // sum_c 2^(c b_i): the offset 1 of each of the row's four fields
+    uint16_t bnd[D];   // 2 qmax_i: the clamp bound of e = z + qmax_i (0 for FP16 rows, like the two above)
     uint8_t rw[D];     // row widths (16 = FP16 row)
     uint32_t roff[D];  // (first word of the row's band block) << 11 | stream bit of the row
 };
@@ -80,30 +83,31 @@ __device__ __forceinline__ void unpack_pair_rows(const uint8_t *tile0, uint32_t 
 }
 
 // The codes of this tile, appended to its stream and written to the record
-// word by word (own words only: word m of the tile at tile0 + 4 NCB m).
+// word by word (own words only: word m of the tile at tile0 + 4 NCB m).  Every
+// put stores the word it reaches, complete or not (a partial word is stored
+// again once more bits have joined it), so the lanes of a warp, whose rows
+// have different widths, run it without a branch.
 struct StreamOut {
     uint8_t *tile0;
     uint32_t acc = 0, fill = 0, m = 0;
-    __device__ __forceinline__ void put(uint32_t f, uint32_t nbits) {  // nbits <= 32
+    __device__ __forceinline__ void put(uint32_t f, uint32_t nbits) {  // 0 < nbits <= 32
         acc |= f << fill;
+        *reinterpret_cast<uint32_t *>(tile0 + m * (4u * NCB)) = acc;
         const uint32_t nf = fill + nbits;
-        if (nf >= 32u) {
-            *reinterpret_cast<uint32_t *>(tile0 + m * (4u * NCB)) = acc;
-            ++m;
-            acc = __funnelshift_l(f, 0u, fill);  // the bits of f past the word end (0 when fill = 0)
-            fill = nf - 32u;
-        } else {
-            fill = nf;
-        }
+        const bool full = nf >= 32u;
+        const uint32_t spill = __funnelshift_l(f, 0u, fill);  // the bits of f past the word end (0 when fill = 0)
+        acc = full ? spill : acc;
+        m += full ? 1u : 0u;
+        fill = nf & 31u;
     }
     __device__ __forceinline__ void flush() {
         if (fill) *reinterpret_cast<uint32_t *>(tile0 + m * (4u * NCB)) = acc;
     }
 };
 
-// Field of a row of width b from the four clamped codes e_c in [0, 2 qmax]
-// held in the low (hi = false) or high 16 bits of e[c]: u_c = e_c + 1 at bits
-// [c b, c b + b).
+// sum_c e_c 2^(c b) of a row of width b from its four clamped codes e_c in
+// [0, 2 qmax], held in the low (hi = false) or high 16 bits of e[c]; adding
+// the row's `ones` gives the field, u_c = e_c + 1 at bits [c b, c b + b).
 __device__ __forceinline__ uint32_t field4(const uint32_t (&e)[4], bool hi, uint32_t b) {
     const uint32_t M = 1u << b;
     uint32_t f = hi ? (e[3] >> 16) : (e[3] & 0xffffu);
@@ -132,6 +136,7 @@ __device__ __forceinline__ void row_phase_rows(ScratchR &sc, int tid, const floa
     s = s + __shfl_xor_sync(kFull, s, 1);
     const uint32_t b = rw[i];
     float ri = 0.0f, inv = 0.0f, bw = 0.0f, iq = 0.0f;
+    uint32_t mgb = 0u, ones = 0u, bnd = 0u;
     if (b == (uint32_t)kPivotBits) {
         inv = 1.0f;  // y = S: an FP16 row's register holds its binary16 pattern as a tiny fp32 value
     } else {
@@ -140,15 +145,21 @@ __device__ __forceinline__ void row_phase_rows(ScratchR &sc, int tid, const floa
         inv = __frcp_rn(ri);
         bw = __fmul_rn(wbar[i], __fmul_rn(ri, ri));
         iq = __frcp_rn((float)((1u << (b - 1u)) - 1u));
+        mgb = 0x4B400000u + (1u << (b - 1u));
+        ones = 1u + (1u << b) + (1u << (2u * b)) + (1u << (3u * b));
+        bnd = (1u << b) - 2u;
     }
     if (h == 0) {
         sc.h.rinv[i] = inv;
         sc.h.rowr[i] = ri;
         sc.rw[i] = (uint8_t)b;
+        sc.mgb[i] = mgb;
+        sc.ones[i] = ones;
         if (rec_r) scale_put(rec_r, i, ri, S16);
     } else {
         sc.h.bw[i] = bw;
         sc.iq[i] = iq;
+        sc.bnd[i] = (uint16_t)bnd;
         sc.roff[i] = roff[i];
     }
     __syncthreads();
@@ -157,7 +168,7 @@ __device__ __forceinline__ void row_phase_rows(ScratchR &sc, int tid, const floa
 // After the row phase: y = fl(S fl(1/r)), c0_j = max_i fl(|y_ij| iq_i), the
 // initial codes, the least-squares refinement of c, then the final codes of
 // the tile written to the record (codes block at rec, c to rec_c).
-template <int S16>
+template <int S16, bool HAS16>
 __device__ __forceinline__ void fit_pack_rows(float2 (&S)[NP][4], const ScratchR &sc, int tid, uint8_t *rec,
                                               uint8_t *rec_c) {
     const int g = band_of(tid), cb = cblk_of(tid), lane = tid & 31, i0 = g * RT, j0 = 4 * cb;
@@ -224,28 +235,28 @@ __device__ __forceinline__ void fit_pack_rows(float2 (&S)[NP][4], const ScratchR
         const float t = __shfl_sync(kFull, icj, col8_src(lane, c));
         icd[c] = make_float2(t, t);
     }
-    // final codes: T = fma(y, 1/c, 1.5 2^23 + 2^(b-1)) per element; the low 16
-    // bits of a row pair's two results are joined and clamped to [0, 2 qmax]
+    // final codes: T = fma(y, 1/c, 1.5 2^23 + 2^(b-1)) per element (the offset
+    // lands in the mantissa of 1.5 2^23, 0x4B400000); the low 16 bits of a row
+    // pair's two results are joined and clamped to [0, 2 qmax]
     const uint4 wv = *reinterpret_cast<const uint4 *>(&sc.rw[i0]);
     StreamOut out;
     out.tile0 = rec + tile_byte0(sc.roff[i0], g, cb);
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
         const uint32_t ba = wid(wv, 2 * k), bb = wid(wv, 2 * k + 1);
-        // 1.5 2^23 + 2^(b-1): the offset lands in the mantissa of 1.5 2^23 (0x4B400000)
-        const float2 mg2 = make_float2(__uint_as_float(0x4B400000u + (1u << (ba - 1u))),
-                                       __uint_as_float(0x4B400000u + (1u << (bb - 1u))));
-        const uint32_t bound = ((2u << (ba - 1u)) - 2u) | (((2u << (bb - 1u)) - 2u) << 16);
+        const uint2 mgp = *reinterpret_cast<const uint2 *>(&sc.mgb[i0 + 2 * k]);
+        const uint2 onp = *reinterpret_cast<const uint2 *>(&sc.ones[i0 + 2 * k]);
+        const uint32_t bound = *reinterpret_cast<const uint32_t *>(&sc.bnd[i0 + 2 * k]);
+        const float2 mg2 = make_float2(__uint_as_float(mgp.x), __uint_as_float(mgp.y));
         uint32_t e[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const float2 T = fma2(S[k][c], icd[c], mg2);
-            e[c] = __viaddmin_s16x2_relu(__byte_perm(__float_as_uint(T.x), __float_as_uint(T.y), 0x5410u), 0xFFFFFFFFu, bound) +
-                   0x00010001u;
+            e[c] = __viaddmin_s16x2_relu(__byte_perm(__float_as_uint(T.x), __float_as_uint(T.y), 0x5410u), 0xFFFFFFFFu, bound);
         }
-        if (ba != (uint32_t)kPivotBits && bb != (uint32_t)kPivotBits) {
-            out.put(field4(e, false, ba), 4u * ba);
-            out.put(field4(e, true, bb), 4u * bb);
+        if (!HAS16 || (ba != (uint32_t)kPivotBits && bb != (uint32_t)kPivotBits)) {
+            out.put(field4(e, false, ba) + onp.x, 4u * ba);
+            out.put(field4(e, true, bb) + onp.y, 4u * bb);
         } else {  // FP16 rows carry their binary16 patterns in the low bits of S (see item_rows)
 #pragma unroll
             for (int hs = 0; hs < 2; ++hs) {
@@ -256,7 +267,7 @@ __device__ __forceinline__ void fit_pack_rows(float2 (&S)[NP][4], const ScratchR
                     out.put(__byte_perm(x0, x1, 0x5410u), 32u);
                     out.put(__byte_perm(x2, x3, 0x5410u), 32u);
                 } else {
-                    out.put(field4(e, hs != 0, b), 4u * b);
+                    out.put(field4(e, hs != 0, b) + (hs ? onp.y : onp.x), 4u * b);
                 }
             }
         }
@@ -271,7 +282,7 @@ __device__ __forceinline__ void fit_pack_rows(float2 (&S)[NP][4], const ScratchR
 // block barrier that follows the last read of the stage.  No global memory
 // is written before the vote.
 // ---------------------------------------------------------------------------
-template <int KIND, int S16, class Rel>
+template <int KIND, int S16, bool HAS16, class Rel>
 __device__ bool item_rows(const Args &a, const uint8_t *stage, uint8_t *rec_g, int row, uint32_t codes_bytes,
                           ScratchR &sc, int tid, bool ok, Rel &rel) {
     const int g = band_of(tid), cb = cblk_of(tid), lane = tid & 31, i0 = g * RT, j0 = 4 * cb;
@@ -310,7 +321,7 @@ __device__ bool item_rows(const Args &a, const uint8_t *stage, uint8_t *rec_g, i
             const float2 a2 = mul2(ap[k], rp[k]);
 #pragma unroll
             for (int c = 0; c < 4; ++c) S[k][c] = mul2(mul2(a2, cd[c]), z[c]);
-            if (ba == (uint32_t)kPivotBits || bb == (uint32_t)kPivotBits) {
+            if (HAS16 && (ba == (uint32_t)kPivotBits || bb == (uint32_t)kPivotBits)) {
                 float h[4];
                 if (ba == (uint32_t)kPivotBits) {
                     halves4(tile0, P, h);
@@ -364,7 +375,7 @@ __device__ bool item_rows(const Args &a, const uint8_t *stage, uint8_t *rec_g, i
                 S[k][c] = fma2(kp[k], wd[c], S[k][c]);
                 if (KIND != kFitPack) acc[c] = fma2(qp[k], S[k][c], acc[c]);
             }
-            if (KIND != kDecode) {
+            if (HAS16 && KIND != kDecode) {
                 const uint32_t ba = wid(wv, 2 * k), bb = wid(wv, 2 * k + 1);
                 if (ba == (uint32_t)kPivotBits || bb == (uint32_t)kPivotBits) {
 #pragma unroll
@@ -397,7 +408,7 @@ __device__ bool item_rows(const Args &a, const uint8_t *stage, uint8_t *rec_g, i
     uint8_t *rec_c = rec_r + D * (S16 ? 2 : 4);
     row_phase_rows<S16>(sc, tid, tf + kTailRho * D, tf + kTailWbar * D, rw, roff, rec_r);
     rel();
-    fit_pack_rows<S16>(S, sc, tid, rec_g, rec_c);
+    fit_pack_rows<S16, HAS16>(S, sc, tid, rec_g, rec_c);
     return false;
 }
 
@@ -453,7 +464,10 @@ __global__ void __launch_bounds__(NT, 2) k_step_rows(Args a) {
             abort = __syncthreads_or(!ok);
             if (!abort) rel();
         } else {
-            abort = item_rows<KIND, S16>(a, stage, rec_g, row, codes_bytes, sc, tid, ok, rel);
+            // the descriptor's width byte is 16 for a head with FP16 rows, else 0
+            abort = sc.h.meta[s][kMetaWidth] == kPivotBits
+                        ? item_rows<KIND, S16, true>(a, stage, rec_g, row, codes_bytes, sc, tid, ok, rel)
+                        : item_rows<KIND, S16, false>(a, stage, rec_g, row, codes_bytes, sc, tid, ok, rel);
         }
         if (abort) {
             if (tid == 0) {
@@ -512,7 +526,7 @@ __global__ void __launch_bounds__(NT) k_requant_rows(Args a) {
     const uint32_t codes_bytes = a.t.codes_bytes[gl];
     uint8_t *rec_r = rec + codes_bytes;
     row_phase_rows<S16>(sc, tid, sc.h.rho, sc.h.wbar, a.t.row_width + (size_t)gl * D, a.t.row_off + (size_t)gl * D, rec_r);
-    fit_pack_rows<S16>(S, sc, tid, rec, rec_r + D * (S16 ? 2 : 4));
+    fit_pack_rows<S16, true>(S, sc, tid, rec, rec_r + D * (S16 ? 2 : 4));
 }
 
 __global__ void __launch_bounds__(NT) k_unpack_rows(Args a) {
