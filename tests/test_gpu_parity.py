@@ -520,6 +520,18 @@ def test_kda_slice_lockstep(stepq):
     _lockstep(stepq, "kda_rows", 8, 8, check=[0, 7], n_layers=2, n_pivots=16)
 
 
+@pytest.mark.parametrize("n_pivots,fused", [(0, True), (0, False), (512, True), (512, False)])
+def test_kda_fp16_free_and_fp16_heavy_plans(stepq, n_pivots, fused):
+    # The per-row step kernels run one code path for heads without FP16 rows and
+    # another for heads with them (chosen per item from the step descriptor).  A
+    # 1-layer KDA slice with no FP16 row sends every head down the first; with 512
+    # FP16 rows over its 4,096 key rows every one of the 32 heads has some.
+    plan, _, wl, _ = oracle_plan("kda_rows", n_layers=1, n_pivots=n_pivots)
+    w = np.asarray(plan["widths"]).reshape(-1, wl.d)
+    assert int((w == 16).any(axis=1).sum()) == (0 if n_pivots == 0 else w.shape[0])
+    _lockstep(stepq, "kda_rows", 4, 6, check=[0, 3], n_layers=1, n_pivots=n_pivots, fused=fused)
+
+
 def test_kda_scale16_lockstep(stepq):
     _lockstep(stepq, "kda_rows", 8, 4, check=[0, 7], n_layers=2, n_pivots=16, fused=True, scale_bits=16)
 
