@@ -222,3 +222,37 @@ def test_new_entry_points_reject_bad_arguments_without_a_device():
     assert l.stepq_selftest_tc(None, None, None, None, None, None) == stepq.EINVAL
     assert b"A" in l.stepq_last_error()
     assert l.stepq_prefill_workspace_bytes(None, 1, 1) == 0
+
+
+@pytest.mark.parametrize("scale_bits", [32, 16])
+@pytest.mark.parametrize("bits", [2, 4, 6, 8])
+def test_benchmark_byte_model_per_head_step(bits, scale_bits):
+    """The roofline's algorithmic bytes, from the library's own record sizes,
+    against the closed form of one per-head-unit step at d = 128: the record
+    (D^2 b / 8 code bytes + r and c, 4 or 2 bytes each per row and column)
+    read and written once, q, k, v read, o written, alpha and beta read:
+    4096 b + 4104 bytes with fp32 scales (28,680 at b = 6), 4096 b + 3080 with
+    bfloat16 ones; the two-stream kernels' own counts beside it."""
+    import bench
+    L, H, D, n = 2, 3, 128, 5
+    p = stepq.Plan.build_uniform(0, L, H, D, bits, stepq.QUANT_DUAL_AXIS, 65536, scale_bits=scale_bits)
+    rec = D * D * bits // 8 + 2 * D * (scale_bits // 8)
+    assert all(p.record(l, h)[1] == rec for l in range(L) for h in range(H))
+    per = 4096 * bits + (4104 if scale_bits == 32 else 3080)
+    assert bench.step_bytes(p, n) == n * L * H * per
+    assert bench.kernel_bytes(p, n, "fused") == n * L * H * per
+    assert bench.kernel_bytes(p, n, "decode") == n * L * H * (rec + 3 * 4 * D + 8 + 2 * 4 * D)
+    assert bench.kernel_bytes(p, n, "fitpack") == n * L * H * (2 * rec + 2 * 4 * D + 8)
+    if bits == 6 and scale_bits == 32:
+        assert per == 28680
+
+
+def test_benchmark_byte_model_per_row_units():
+    """Per-row (KDA) units: the gate is one alpha per key row, so a head-step
+    reads 4 D + 4 gate bytes instead of 8."""
+    import bench
+    L, H, D, n = 1, 2, 128, 3
+    p = stepq.Plan.build_uniform(1, L, H, D, 6, stepq.QUANT_DUAL_AXIS, 65536)
+    rec = sum(p.record(0, h)[1] for h in range(H)) // H
+    assert bench.gate_bytes(p) == 4 * D + 4
+    assert bench.step_bytes(p, n) == n * L * H * (2 * rec + 3 * 4 * D + 4 * D + 4 + 4 * D)
